@@ -1,0 +1,123 @@
+"""Seeded synthetic inputs for the Mamba-3 SSM forward.
+
+This module only draws random tensors; it holds none of the method's
+arithmetic, so both the fp64 oracle (tests) and the CUDA library (tests,
+benchmark) can take their inputs from it without sharing any computation.
+
+Distributions (the 1.5B-scale workloads' synthetic recipe):
+  x ~ N(0, 1)                      [Bt, T, H, R, P]
+  B, C ~ N(0, 1/N)                 [Bt, T, H, R, N]
+  dt = softplus(N(-4, 1))          [Bt, T, H]
+  A = -exp(U(0, ln 16))            [H]        (fp32, never rounded)
+  lam = sigmoid(N(0, 1))           [Bt, T, H]
+  theta ~ U(-pi, pi)               [Bt, T, H, N/2]   (one angle rate per state pair)
+  D ~ N(0, 1)                      [H]        (fp32, never rounded)
+Draw order is fixed (x, B, C, dt, A, lam, theta, D) from one torch.Generator
+seeded with the workload's seed.  Tensors are drawn in fp32 and then rounded
+to the I/O dtype (round-to-nearest-even); consumers see only the rounded
+values.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import torch
+
+
+@dataclass(frozen=True)
+class Shape:
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int   # P
+    dstate: int    # N (even)
+    rank: int      # R (MIMO rank; 1 = SISO)
+    io: str        # "f32" or "bf16"
+    seed: int = 0
+
+    @property
+    def torch_io(self):
+        return torch.float32 if self.io == "f32" else torch.bfloat16
+
+    def with_(self, **kw) -> "Shape":
+        return replace(self, **kw)
+
+
+# The workloads the method is measured on (sizes of the pages' 1.5B-scale
+# models), named by what they are.
+WORKLOADS = {
+    # small fp32-I/O SISO scan (oracle-sized)
+    "siso_f32_b1_t256_h4_p64_n64": Shape(1, 256, 4, 64, 64, 1, "f32"),
+    # SISO prefill, bf16 I/O, fp32 state
+    "siso_bf16_b8_t4096_h32_p64_n128": Shape(8, 4096, 32, 64, 128, 1, "bf16"),
+    # MIMO rank-4 prefill, halved state
+    "mimo_bf16_b8_t4096_h32_p64_n64_r4": Shape(8, 4096, 32, 64, 64, 4, "bf16"),
+    # decode: state from a 1024-token prefill, then single-token steps
+    "decode_bf16_b256_h32_p64_n128_r1": Shape(256, 1024, 32, 64, 128, 1, "bf16"),
+    "decode_bf16_b256_h32_p64_n128_r4": Shape(256, 1024, 32, 64, 128, 4, "bf16"),
+    # long-context MIMO prefill
+    "long_mimo_bf16_b1_t65536_h64_p64_n128_r4": Shape(1, 65536, 64, 64, 128, 4, "bf16"),
+}
+DECODE_STEPS = 1000
+LONG_DECODE_STEPS = 256
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _draws(g, device, lead, H, R, P, N):
+    """Draw the per-token tensors with leading dims `lead` (e.g. (Bt, T))."""
+    f = dict(device=device, dtype=torch.float32, generator=g)
+    x = torch.randn(*lead, H, R, P, **f)
+    B = torch.randn(*lead, H, R, N, **f) / math.sqrt(N)
+    C = torch.randn(*lead, H, R, N, **f) / math.sqrt(N)
+    dt = torch.nn.functional.softplus(torch.randn(*lead, H, **f) - 4.0)
+    return x, B, C, dt
+
+
+def make_prefill(shape: Shape, device="cpu", seqlen: int | None = None):
+    """Inputs of one prefill call.  Returns a dict of tensors on `device`."""
+    T = shape.seqlen if seqlen is None else seqlen
+    Bt, H, R, P, N = shape.batch, shape.nheads, shape.rank, shape.headdim, shape.dstate
+    g = _gen(shape.seed, device)
+    f = dict(device=device, dtype=torch.float32, generator=g)
+    x, B, C, dt = _draws(g, device, (Bt, T), H, R, P, N)
+    A = -torch.exp(torch.rand(H, **f) * math.log(16.0))
+    lam = torch.sigmoid(torch.randn(Bt, T, H, **f))
+    theta = (torch.rand(Bt, T, H, N // 2, **f) * 2.0 - 1.0) * math.pi
+    D = torch.randn(H, **f)
+    io = shape.torch_io
+    return dict(x=x.to(io), B=B.to(io), C=C.to(io), dt=dt.to(io), lam=lam.to(io),
+                theta=theta.to(io), A=A.contiguous(), D=D.contiguous())
+
+
+def make_steps(shape: Shape, nsteps: int, device="cpu", seed_offset: int = 1):
+    """Per-step decode inputs, leading dim = step: x [S,Bt,H,R,P],
+    B/C [S,Bt,H,R,N], dt/lam [S,Bt,H], theta [S,Bt,H,N/2].  A and D are the
+    prefill's (same seed), so a prefill followed by these steps is one
+    continuous sequence with per-head parameters."""
+    Bt, H, R, P, N = shape.batch, shape.nheads, shape.rank, shape.headdim, shape.dstate
+    g = _gen(shape.seed + seed_offset, device)
+    f = dict(device=device, dtype=torch.float32, generator=g)
+    x, B, C, dt = _draws(g, device, (nsteps, Bt), H, R, P, N)
+    lam = torch.sigmoid(torch.randn(nsteps, Bt, H, **f))
+    theta = (torch.rand(nsteps, Bt, H, N // 2, **f) * 2.0 - 1.0) * math.pi
+    io = shape.torch_io
+    return dict(x=x.to(io), B=B.to(io), C=C.to(io), dt=dt.to(io), lam=lam.to(io),
+                theta=theta.to(io))
+
+
+def make_state(shape: Shape, device="cpu", seed_offset: int = 2, scale: float = 1.0):
+    """A random (h, b_prev, x_prev) state in fp32, for tests that start from a
+    nonzero state."""
+    Bt, H, R, P, N = shape.batch, shape.nheads, shape.rank, shape.headdim, shape.dstate
+    g = _gen(shape.seed + seed_offset, device)
+    f = dict(device=device, dtype=torch.float32, generator=g)
+    h = torch.randn(Bt, H, N, P, **f) * scale
+    bp = torch.randn(Bt, H, R, N, **f) / math.sqrt(N)
+    xp = torch.randn(Bt, H, R, P, **f)
+    return h, bp, xp

@@ -1,0 +1,401 @@
+"""Pins for the fp64 oracle: each test checks it against something other than
+itself -- a hand-derived worked example, a closed form, a special case that
+reduces to the Mamba-2 recurrence, an explicit complex-diagonal recurrence,
+the literal rotated-frame statement, the brute-force masked-attention dual,
+and a chunked restatement.  Everything here is fp64 and CPU-only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from m3_inputs import Shape, make_prefill, make_state
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+TOL = 1e-12
+
+
+def rand_case(Bt=1, T=37, H=2, P=5, N=8, R=3, seed=0, init=True):
+    s = Shape(Bt, T, H, P, N, R, "f32", seed)
+    d = {k: v.double().numpy() for k, v in make_prefill(s).items()}
+    st = None
+    if init:
+        h, bp, xp = (t.double().numpy() for t in make_state(s))
+        st = oracle.State(h, bp, xp)
+    return d, st
+
+
+def run(d, st=None):
+    return oracle.scan(d["x"], d["B"], d["C"], d["dt"], d["lam"], d["theta"], d["A"], d["D"], st)
+
+
+def rel(a, b):
+    return np.max(np.abs(a - b)) / max(1.0, np.max(np.abs(b)))
+
+
+# ---------------------------------------------------------------- worked examples
+@pytest.mark.parametrize("ex", json.load(open(GOLDEN))["examples"], ids=lambda e: e["name"])
+def test_hand_worked_examples(ex):
+    dm, inp, exp_ = ex["dims"], ex["inputs"], ex["expected"]
+    T, N, P = dm["seqlen"], dm["dstate"], dm["headdim"]
+    x = np.array(inp["x"]).reshape(1, T, 1, 1, P)
+    B = np.array(inp["B"]).reshape(1, T, 1, 1, N)
+    C = np.array(inp["C"]).reshape(1, T, 1, 1, N)
+    dt = np.array(inp["dt"]).reshape(1, T, 1)
+    lam = np.array(inp["lam"]).reshape(1, T, 1)
+    th = np.array(inp["theta"]).reshape(1, T, 1, N // 2)
+    A = np.array([inp["A"]])
+    D = np.array([inp["D"]])
+    st = None
+    if "h0" in inp:
+        st = oracle.State(np.array(inp["h0"]).reshape(1, 1, N, P),
+                          np.array(inp["b_prev0"]).reshape(1, 1, 1, N),
+                          np.array([inp["x_prev0"]]).reshape(1, 1, 1, P))
+    y, fs = oracle.scan(x, B, C, dt, lam, th, A, D, st)
+    np.testing.assert_allclose(y.reshape(-1), exp_["y"], atol=TOL, rtol=0)
+    np.testing.assert_allclose(fs.h.reshape(N, P), np.array(exp_["h"]), atol=TOL, rtol=0)
+    np.testing.assert_allclose(fs.b_prev.reshape(-1), exp_["b_prev"], atol=TOL, rtol=0)
+    np.testing.assert_allclose(fs.x_prev.reshape(-1), [exp_["x_prev"]], atol=TOL, rtol=0)
+
+
+# ---------------------------------------------------------------- closed forms
+def test_single_token_closed_form():
+    """T=1 from zero state: y_0 = lam_0 dt_0 (C_0^T B_0) x_0 + D x_0 (MIMO: the
+    R x R block C_0^T B_0 mixes ranks)."""
+    d, _ = rand_case(T=1, init=False)
+    y, fs = run(d)
+    gam = d["lam"] * d["dt"]                       # [1,1,H]
+    CB = np.einsum("bthrn,bthsn->bthrs", d["C"], d["B"])
+    ref = gam[..., None, None] * np.einsum("bthrs,bthsp->bthrp", CB, d["x"])
+    ref += d["D"][None, None, :, None, None] * d["x"]
+    assert rel(y, ref) < TOL
+    # state after one token: gamma_0 B_0 x_0^T (the pending term of token 0 is zero)
+    hs = gam[:, 0, :, None, None] * np.einsum("bhrn,bhrp->bhnp", d["B"][:, 0], d["x"][:, 0])
+    assert rel(fs.h, hs) < TOL
+
+
+def test_free_decay_closed_form():
+    """x = 0 and no pending input: the state only decays and rotates, so
+    h_t = exp(A sum dt) Rot(-sum dt*theta) h_0 in closed form."""
+    d, st = rand_case(T=29)
+    d["x"][:] = 0.0
+    st.x_prev[:] = 0.0
+    y, fs = run(d, st)
+    cumdt = np.cumsum(d["dt"], axis=1)                          # [Bt,T,H]
+    phi = np.cumsum(d["dt"][..., None] * d["theta"], axis=1)    # [Bt,T,H,N/2]
+    decay = np.exp(cumdt * d["A"][None, None, :])
+    h0 = st.h                                                   # [Bt,H,N,P]
+    u, v = h0[:, None, :, 0::2, :], h0[:, None, :, 1::2, :]
+    c, s = np.cos(phi)[..., None], np.sin(phi)[..., None]
+    hu = decay[..., None, None] * (u * c + v * s)
+    hv = decay[..., None, None] * (-u * s + v * c)
+    ht = np.empty(hu.shape[:3] + (hu.shape[3] * 2, hu.shape[4]))
+    ht[..., 0::2, :], ht[..., 1::2, :] = hu, hv
+    ref = np.einsum("bthnp,bthrn->bthrp", ht, d["C"])
+    assert rel(y, ref) < TOL
+    assert rel(fs.h, ht[:, -1]) < TOL
+
+
+def test_constant_input_fixed_point():
+    """theta = 0 and constant (dt, lam, B, x): the state converges to
+    (beta' a + gamma) B x^T / (1 - a) with a = exp(dt A)."""
+    T, N, P = 400, 4, 3
+    rng = np.random.default_rng(5)
+    Bv, xv = rng.normal(size=N), rng.normal(size=P)
+    dtv, lamv, A = 0.3, 0.3, np.array([-1.7])
+    x = np.broadcast_to(xv, (1, T, 1, 1, P)).copy()
+    B = np.broadcast_to(Bv, (1, T, 1, 1, N)).copy()
+    C = rng.normal(size=(1, T, 1, 1, N))
+    dt = np.full((1, T, 1), dtv)
+    lam = np.full((1, T, 1), lamv)
+    th = np.zeros((1, T, 1, N // 2))
+    y, fs = oracle.scan(x, B, C, dt, lam, th, A, np.zeros(1))
+    a = math.exp(dtv * A[0])
+    hstar = ((1 - lamv) * dtv * a + lamv * dtv) * np.outer(Bv, xv) / (1 - a)
+    assert rel(fs.h[0, 0], hstar) < 1e-10
+
+
+# ---------------------------------------------------------------- special cases
+def mamba2_reference(d):
+    """Independent Mamba-2 (exponential-Euler, real, scalar decay) recurrence in
+    the S in R^{P x N} orientation of the SSD chapter ('La dualità'):
+    S_t = e^{dt A} S_{t-1} + dt x_t B_t^T, y_t = S_t C_t + D x_t."""
+    x, B, C, dt, A, D = d["x"], d["B"], d["C"], d["dt"], d["A"], d["D"]
+    Bt, T, H, R, P = x.shape
+    N = B.shape[-1]
+    y = np.zeros_like(x)
+    for b in range(Bt):
+        for h in range(H):
+            S = np.zeros((P, N))
+            for t in range(T):
+                S = math.exp(dt[b, t, h] * A[h]) * S + dt[b, t, h] * x[b, t, h].T @ B[b, t, h]
+                y[b, t, h] = (S @ C[b, t, h].T).T + D[h] * x[b, t, h]
+    return y
+
+
+@pytest.mark.parametrize("R", [1, 3])
+def test_euler_real_reduces_to_mamba2(R):
+    """lam = 1 (Euler) and theta = 0 (real) reduce the method to Mamba-2."""
+    d, _ = rand_case(T=41, R=R, init=False)
+    d["lam"][:] = 1.0
+    d["theta"][:] = 0.0
+    y, _ = run(d)
+    assert rel(y, mamba2_reference(d)) < TOL
+
+
+def test_trapezoid_half_is_average_of_endpoints():
+    """lam = 1/2 is the classic trapezoid: the input integral is the average of
+    the two endpoint writes, the older one carried through one decay."""
+    d, _ = rand_case(T=23, R=1, init=False)
+    d["lam"][:] = 0.5
+    d["theta"][:] = 0.0
+    y, _ = run(d)
+    x, B, C, dt, A, D = d["x"], d["B"], d["C"], d["dt"], d["A"], d["D"]
+    Bt, T, H, R, P = x.shape
+    ref = np.zeros_like(y)
+    for b in range(Bt):
+        for h in range(H):
+            S = np.zeros((P, B.shape[-1]))
+            for t in range(T):
+                a = math.exp(dt[b, t, h] * A[h])
+                cur = np.outer(x[b, t, h, 0], B[b, t, h, 0])
+                prev = np.outer(x[b, t - 1, h, 0], B[b, t - 1, h, 0]) if t else 0.0
+                S = a * S + 0.5 * dt[b, t, h] * (a * prev + cur)
+                ref[b, t, h, 0] = S @ C[b, t, h, 0] + D[h] * x[b, t, h, 0]
+    assert rel(y, ref) < TOL
+
+
+# ---------------------------------------------------------------- equivalent forms
+def complex_diagonal_reference(d, st):
+    """Complex SSM of state N/2: z_k = h_{2k} + i h_{2k+1}, transition
+    exp(dt (A - i theta_k)), writes b_k x^T with b_k = B_{2k} + i B_{2k+1},
+    readout Re(conj(c_k) z_k) summed over k."""
+    x, B, C, dt, lam, th, A, D = (d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D"))
+    Bt, T, H, R, P = x.shape
+    y = np.zeros_like(x)
+    hT = np.zeros_like(st.h)
+    for b in range(Bt):
+        for h in range(H):
+            z = st.h[b, h, 0::2] + 1j * st.h[b, h, 1::2]             # [N/2, P]
+            bprev = st.b_prev[b, h, :, 0::2] + 1j * st.b_prev[b, h, :, 1::2]  # [R, N/2]
+            xprev = st.x_prev[b, h]                                  # [R, P]
+            for t in range(T):
+                lt = np.exp(dt[b, t, h] * (A[h] - 1j * th[b, t, h]))  # [N/2]
+                bt = B[b, t, h, :, 0::2] + 1j * B[b, t, h, :, 1::2]
+                ct = C[b, t, h, :, 0::2] + 1j * C[b, t, h, :, 1::2]
+                z = lt[:, None] * (z + (1 - lam[b, t, h]) * dt[b, t, h] * bprev.T @ xprev)
+                z = z + lam[b, t, h] * dt[b, t, h] * bt.T @ x[b, t, h]
+                y[b, t, h] = np.real(np.conj(ct) @ z) + D[h] * x[b, t, h]
+                bprev, xprev = bt, x[b, t, h]
+            hT[b, h, 0::2], hT[b, h, 1::2] = z.real, z.imag
+    return y, hT
+
+
+def test_equals_complex_diagonal_ssm():
+    d, st = rand_case()
+    y, fs = run(d, st)
+    yc, hc = complex_diagonal_reference(d, st)
+    assert rel(y, yc) < TOL and rel(fs.h, hc) < TOL
+
+
+def rot(v, ang):
+    """Rotate interleaved pairs (v[2k], v[2k+1]) of the last axis by +ang[k]."""
+    out = np.empty_like(v)
+    c, s = np.cos(ang), np.sin(ang)
+    out[..., 0::2] = v[..., 0::2] * c - v[..., 1::2] * s
+    out[..., 1::2] = v[..., 0::2] * s + v[..., 1::2] * c
+    return out
+
+
+def rotated_frame_reference(d, st):
+    """The literal statement: B_t, C_t rotated pair-wise by the cumulative angle
+    phi_t = sum_{s<=t} dt_s theta_s, and
+    g_t = a_t g_{t-1} + (1-lam_t) dt_t a_t B~_{t-1} x_{t-1}^T + lam_t dt_t B~_t x_t^T,
+    y_t = g_t^T C~_t + D x_t;  the plain-frame state is Rot(-phi_t) g_t."""
+    x, B, C, dt, lam, th, A, D = (d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D"))
+    Bt, T, H, R, P = x.shape
+    phi = np.cumsum(dt[..., None] * th, axis=1)
+    Bn = rot(B, phi[:, :, :, None, :])
+    Cn = rot(C, phi[:, :, :, None, :])
+    y = np.zeros_like(x)
+    hT = np.zeros_like(st.h)
+    for b in range(Bt):
+        for h in range(H):
+            g = st.h[b, h].copy()
+            bprev, xprev = st.b_prev[b, h], st.x_prev[b, h]
+            for t in range(T):
+                a = math.exp(dt[b, t, h] * A[h])
+                g = (a * g + (1 - lam[b, t, h]) * dt[b, t, h] * a * bprev.T @ xprev
+                     + lam[b, t, h] * dt[b, t, h] * Bn[b, t, h].T @ x[b, t, h])
+                y[b, t, h] = (g.T @ Cn[b, t, h].T).T + D[h] * x[b, t, h]
+                bprev, xprev = Bn[b, t, h], x[b, t, h]
+            hT[b, h] = rot(g.T, -phi[b, T - 1, h]).T
+    return y, hT
+
+
+def test_equals_rotated_frame_statement():
+    d, st = rand_case()
+    y, fs = run(d, st)
+    yr, hr = rotated_frame_reference(d, st)
+    assert rel(y, yr) < TOL and rel(fs.h, hr) < TOL
+
+
+def ssd_dual_reference(d, st):
+    """Brute-force masked-attention ('dual') form: materialise the full
+    (T R) x (T R) matrix M o (C~ B~^T) and multiply by X.  Weights:
+    w(t,t) = gamma_t; w(t,s<t) = exp(A sum_{k=s+1..t} dt_k) (gamma_s + beta'_{s+1}),
+    plus the initial state read out through the total decay since the start."""
+    x, B, C, dt, lam, th, A, D = (d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D"))
+    Bt, T, H, R, P = x.shape
+    phi = np.cumsum(dt[..., None] * th, axis=1)
+    Bn = rot(B, phi[:, :, :, None, :])
+    Cn = rot(C, phi[:, :, :, None, :])
+    y = np.zeros_like(x)
+    for b in range(Bt):
+        for h in range(H):
+            gam = lam[b, :, h] * dt[b, :, h]
+            betap = (1 - lam[b, :, h]) * dt[b, :, h]
+            cum = np.concatenate([[0.0], np.cumsum(dt[b, :, h] * A[h])])  # cum[t+1] = sum_{k<=t}
+            W = np.zeros((T, T))
+            for t in range(T):
+                W[t, t] = gam[t]
+                for s in range(t):
+                    W[t, s] = math.exp(cum[t + 1] - cum[s + 1]) * (gam[s] + betap[s + 1])
+            CB = np.einsum("trn,sqn->trsq", Cn[b, :, h], Bn[b, :, h])  # [T,R,T,R]
+            Mfull = W[:, None, :, None] * CB
+            Y = Mfull.reshape(T * R, T * R) @ x[b, :, h].reshape(T * R, P)
+            h0 = st.h[b, h] + betap[0] * st.b_prev[b, h].T @ st.x_prev[b, h]
+            for t in range(T):
+                Y[t * R:(t + 1) * R] += math.exp(cum[t + 1]) * (Cn[b, t, h] @ h0)
+            y[b, :, h] = Y.reshape(T, R, P) + D[h] * x[b, :, h]
+    return y
+
+
+@pytest.mark.parametrize("R", [1, 2])
+def test_equals_ssd_dual_bruteforce(R):
+    d, st = rand_case(T=24, R=R)
+    y, _ = run(d, st)
+    assert rel(y, ssd_dual_reference(d, st)) < TOL
+
+
+# ---------------------------------------------------------------- chunked restatement
+def chunked_reference(d, st, Q):
+    """Chunked form of the recurrence: chunk-local cumulative angles and
+    log-decays, a masked decay-weighted C~ B~^T block inside each chunk, a
+    decay-weighted chunk state G = (w o B~)^T X, and a plain-frame carried state
+    h*_c = Rot(-Phi_c)(exp(cA_end) h*_{c-1} + G_c) between chunks (the four
+    pieces of the chunked SSD algorithm, extended with the trapezoid's pending
+    term folded into gamma_hat_s = gamma_s + beta'_{s+1})."""
+    x, B, C, dt, lam, th, A, D = (d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D"))
+    Bt, T, H, R, P = x.shape
+    N = B.shape[-1]
+    y = np.zeros_like(x)
+    hT = np.zeros_like(st.h)
+    for b in range(Bt):
+        for h in range(H):
+            gam = lam[b, :, h] * dt[b, :, h]
+            betap = (1 - lam[b, :, h]) * dt[b, :, h]
+            ghat = gam.copy()
+            ghat[:-1] += betap[1:]
+            hs = st.h[b, h] + betap[0] * st.b_prev[b, h].T @ st.x_prev[b, h] if T else st.h[b, h]
+            for c0 in range(0, T, Q):
+                sl = slice(c0, min(T, c0 + Q))
+                L = sl.stop - sl.start
+                cA = np.cumsum(dt[b, sl, h] * A[h])
+                phi = np.cumsum(dt[b, sl, h][:, None] * th[b, sl, h], axis=0)   # [L, N/2]
+                Bn = rot(B[b, sl, h], phi[:, None, :])                            # [L,R,N]
+                Cn = rot(C[b, sl, h], phi[:, None, :])
+                Wm = np.zeros((L, L))
+                for i in range(L):
+                    for s in range(i + 1):
+                        coef = gam[c0 + i] if s == i else ghat[c0 + s]
+                        Wm[i, s] = math.exp(cA[i] - cA[s]) * coef
+                S = np.einsum("irn,sqn->irsq", Cn, Bn)
+                Xc = x[b, sl, h]
+                Yd = np.einsum("is,irsq,sqp->irp", Wm, S, Xc)
+                Yo = np.exp(cA)[:, None, None] * np.einsum("irn,np->irp", Cn, hs)
+                y[b, sl, h] = Yd + Yo + D[h] * Xc
+                w = np.exp(cA[-1] - cA) * ghat[sl]
+                if sl.stop == T:
+                    w[-1] = gam[T - 1]
+                G = np.einsum("s,sqn,sqp->np", w, Bn, Xc)
+                inner = math.exp(cA[-1]) * hs + G
+                hs = rot(inner.T, -phi[-1]).T
+            hT[b, h] = hs
+    return y, hT
+
+
+@pytest.mark.parametrize("Q", [1, 4, 16, 64])
+def test_chunked_form_matches(Q):
+    d, st = rand_case(T=53, R=2)
+    y, fs = run(d, st)
+    yc, hc = chunked_reference(d, st, Q)
+    assert rel(y, yc) < TOL and rel(fs.h, hc) < TOL
+
+
+# ---------------------------------------------------------------- structure
+def test_mimo_is_sum_of_rank_one_runs():
+    """The rank-R write is a sum of R outer products on one shared state, so the
+    MIMO output for output rank r equals the sum over input ranks q of SISO runs
+    driven by (B[:,q], x[:,q]) and read out with C[:,r]."""
+    d, _ = rand_case(T=31, R=3, init=False)
+    y, _ = run(d)
+    Bt, T, H, R, P = d["x"].shape
+    ref = np.zeros_like(y)
+    for r in range(R):
+        for q in range(R):
+            ys, _ = oracle.scan(d["x"][:, :, :, q:q + 1], d["B"][:, :, :, q:q + 1],
+                                d["C"][:, :, :, r:r + 1], d["dt"], d["lam"], d["theta"],
+                                d["A"], np.zeros_like(d["D"]))
+            ref[:, :, :, r] += ys[:, :, :, 0]
+        ref[:, :, :, r] += d["D"][None, None, :, None] * d["x"][:, :, :, r]
+    assert rel(y, ref) < TOL
+
+
+def test_prefill_then_decode_equals_full_scan():
+    d, st = rand_case(T=40, R=2)
+    yfull, sfull = run(d, st)
+    T1 = 25
+    part = {k: (v[:, :T1] if v.ndim >= 3 else v) for k, v in d.items()}
+    y1, s = run(part, st)
+    ys = [y1]
+    for t in range(T1, 40):
+        yt, s = oracle.step(d["x"][:, t], d["B"][:, t], d["C"][:, t], d["dt"][:, t],
+                            d["lam"][:, t], d["theta"][:, t], d["A"], d["D"], s)
+        ys.append(yt[:, None])
+    np.testing.assert_allclose(np.concatenate(ys, axis=1), yfull, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(s.h, sfull.h, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(s.b_prev, sfull.b_prev, atol=0, rtol=0)
+    np.testing.assert_allclose(s.x_prev, sfull.x_prev, atol=0, rtol=0)
+
+
+def test_split_scan_resumes_exactly():
+    """scan(T1) with its final state passed as the next call's initial state
+    equals one scan over T1+T2 (the pending term crosses the call boundary)."""
+    d, st = rand_case(T=30, R=1)
+    yfull, sfull = run(d, st)
+    a = {k: (v[:, :11] if v.ndim >= 3 else v) for k, v in d.items()}
+    b = {k: (v[:, 11:] if v.ndim >= 3 else v) for k, v in d.items()}
+    ya, sa = run(a, st)
+    yb, sb = run(b, sa)
+    np.testing.assert_allclose(np.concatenate([ya, yb], 1), yfull, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(sb.h, sfull.h, atol=1e-13, rtol=0)
+
+
+def test_empty_sequence_returns_initial_state():
+    d, st = rand_case(T=0)
+    y, fs = run(d, st)
+    assert y.shape[1] == 0
+    np.testing.assert_array_equal(fs.h, st.h)
+    np.testing.assert_array_equal(fs.b_prev, st.b_prev)
+    np.testing.assert_array_equal(fs.x_prev, st.x_prev)
+
+
+def test_threading_is_deterministic():
+    d, st = rand_case(Bt=3, H=3, T=17)
+    y1, s1 = oracle.scan(*(d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D")), st, nthreads=1)
+    y4, s4 = oracle.scan(*(d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D")), st, nthreads=4)
+    np.testing.assert_array_equal(y1, y4)
+    np.testing.assert_array_equal(s1.h, s4.h)
