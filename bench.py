@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-3 SSM forward on B200: prefill scan tokens/s (the
+headline line) plus the decode step, each with its roofline fraction.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one m3_scan_fwd over the whole batch of the SISO bf16 prefill
+workload (batch 8, T=4096, 32 heads, P=64, N=128, R=1), inputs resident in
+HBM (943 MB per step, larger than the 126 MB L2, so no flush is needed).
+With N > 1 (torchrun) every rank runs its own batch (weak scaling, replicas:
+the (batch, head) slices are independent, there is no collective on the data
+path); time is the max over ranks of CUDA-event time.  Rank 0 prints one JSON
+line.  `--impl reference` times the fp64 CPU oracle on bounded samples of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Mamba-3 SSM tokens/s (prefill scan, decode step) and % of roofline, 1 B200"
+PREFILL_WORKLOAD = "siso_bf16_b8_t4096_h32_p64_n128"
+DECODE_WORKLOADS = ["decode_bf16_b256_h32_p64_n128_r1", "decode_bf16_b256_h32_p64_n128_r4"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=PREFILL_WORKLOAD)
+    ap.add_argument("--algo", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier measurement on this pool)"
+
+
+def file_hash(paths):
+    h = hashlib.sha256()
+    for p in sorted(paths):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def kernel_sources(kernel):
+    csrc = os.path.join(ROOT, "state_space_sequence_ssm_b200", "csrc")
+    files = {"prefill_simt_kernel": ["prefill_simt.cu"], "step_kernel": ["decode.cu"],
+             "prefill_tc_kernel": ["prefill_tc.cu", "tc_primitives.cuh"]}[kernel]
+    return [os.path.join(csrc, f) for f in files if os.path.exists(os.path.join(csrc, f))]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, valid only while the
+    kernel's source is unchanged since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{kernel}:{workload}")
+    if not d or d.get("source_hash") != file_hash(kernel_sources(kernel)):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 10]
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        pw = [float(r[4]) for r in rows if r[4].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        load = [s for s, p in zip(sm, pw) if p >= 0.5 * max(pw)] if pw else sm
+        return {"sm_mhz": statistics.median(load or sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(pw) if pw else None}
+
+
+def prefill_bytes(s, with_final=True, with_init=False):
+    """Algorithmic HBM bytes of one prefill call: each input read once, y
+    written once, the final state written once (init read once if given)."""
+    io = 2 if s.io == "bf16" else 4
+    th = s.batch * s.seqlen * s.nheads
+    per_tok = io * (2 * s.rank * s.headdim + 2 * s.rank * s.dstate + 2 + s.dstate // 2)
+    state = 4 * s.batch * s.nheads * (s.dstate * s.headdim + s.rank * (s.dstate + s.headdim))
+    return th * per_tok + state * (int(with_final) + int(with_init)) + 8 * s.nheads
+
+
+def step_bytes(s):
+    """Algorithmic HBM bytes of one decode step (state read + written once,
+    pending inputs read + written once, the token's io inputs, y)."""
+    io = 2 if s.io == "bf16" else 4
+    bh = s.batch * s.nheads
+    state = 4 * (s.dstate * s.headdim + s.rank * (s.dstate + s.headdim))
+    inp = io * (s.rank * s.headdim + 2 * s.rank * s.dstate + 2 + s.dstate // 2)
+    return bh * (2 * state + inp + io * s.rank * s.headdim) + 8 * s.nheads
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args):
+    import numpy as np
+    import torch
+
+    import oracle
+    from m3_inputs import WORKLOADS, make_prefill
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    s = WORKLOADS[args.workload]
+    cores = oracle.num_cores()
+    nslices = max(1, cores)
+    sub = s.with_(batch=1, nheads=nslices)  # bounded sample: `cores` full-length slices
+    inp = {k: v.double().numpy() for k, v in make_prefill(sub).items()}
+    keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
+    for _ in range(args.warmup):
+        oracle.scan(*(inp[k] for k in keys))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.scan(*(inp[k] for k in keys))
+    el = time.perf_counter() - t0
+    # tokens of the workload's model (all heads) per second
+    value = args.steps * nslices * s.seqlen / s.nheads / el
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "batch": s.batch, "seq_len": s.seqlen,
+                                            "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
+                                            "rank": s.rank, "io": s.io},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{nslices} (batch, head) slices x {s.seqlen} tokens per step, "
+                                       f"scaled to tokens of all {s.nheads} heads"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import state_space_sequence_ssm_b200 as m3
+    from m3_inputs import WORKLOADS, make_prefill, make_steps
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    hbm_peak, peak_src = peaks()
+    keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
+    algo = {"auto": m3.ALGO_AUTO, "simt": m3.ALGO_SIMT, "tc": m3.ALGO_TC}[args.algo]
+    s = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    inp = make_prefill(s, device=dev)
+    dims = m3.make_dims(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.rank, s.torch_io)
+    use_tc = algo != m3.ALGO_SIMT and m3.workspace_size(dims) >= 0 and _tc_supported(m3, inp, keys, algo)
+    kernel = "prefill_tc_kernel" if use_tc else "prefill_simt_kernel"
+    y = torch.empty_like(inp["x"])
+    fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device=dev)
+    wsn = m3.workspace_size(dims) if use_tc else 0
+    ws = torch.empty(max(wsn, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, workspace=ws, algo=algo, stream=stream)
+
+    for _ in range(args.warmup):
+        prefill()
+    torch.cuda.synchronize()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    clocks = ClockSampler(uuid)
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        ev[2 * i].record(stream)
+        prefill()
+        ev[2 * i + 1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    launch = statistics.mean(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)) / 1e3
+    tokens = world * K * s.batch * s.seqlen
+    value = tokens / elapsed
+    abytes = prefill_bytes(s)
+    achieved = abytes / launch / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if use_tc else "f32",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "batch": s.batch, "seq_len": s.seqlen, "nheads": s.nheads,
+                       "headdim": s.headdim, "dstate": s.dstate, "rank": s.rank, "io": s.io,
+                       "global_batch": world * s.batch, "parallelism": f"replicas x{world} (no collective)",
+                       "l2": f"inputs larger than L2 ({abytes / 1e6:.0f} MB per step), no flush"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": recorded_traffic(kernel, args.workload),
+                         "kernel": kernel, "algorithmic_bytes_per_launch": abytes,
+                         "launch_ms": launch * 1e3, "peak_source": peak_src},
+            "gpu_launches": K, "clocks": clk}
+
+    # ---- end to end through the public API: pinned host inputs, H2D, call, D2H of y and state
+    if not args.no_e2e:
+        host = {k: v.to("cpu").pin_memory() for k, v in inp.items()}
+        yh = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        hh = torch.empty(fin.h.shape, dtype=torch.float32, pin_memory=True)
+        dbuf = {k: torch.empty_like(v) for k, v in inp.items()}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = yh.numel() * yh.element_size() + hh.numel() * 4
+
+        def e2e_step():
+            for k in keys:
+                dbuf[k].copy_(host[k], non_blocking=True)
+            m3.scan_fwd(*(dbuf[k] for k in keys), None, y=y, final=fin, workspace=ws, algo=algo, stream=stream)
+            yh.copy_(y, non_blocking=True)
+            hh.copy_(fin.h, non_blocking=True)
+
+        for _ in range(min(2, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        el2 = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+        line["e2e"] = {"value": tokens / el2, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h}
+        del host, dbuf, yh, hh
+
+    # ---- decode step: state from a 1024-token prefill, then single-token steps in one CUDA graph
+    if not args.no_decode:
+        del inp, y, fin
+        torch.cuda.empty_cache()
+        line["decode"] = [run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
+                                     peak_src, keys) for name in DECODE_WORKLOADS]
+
+    # ---- CPU baseline: the oracle as it stands on this machine's host cores (rank 0, N = 1)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(s, keys)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _tc_supported(m3, inp, keys, algo):
+    if algo == m3.ALGO_SIMT:
+        return False
+    try:
+        import torch
+        sub = {k: (v[:1, :1].contiguous() if v.dim() >= 3 else v) for k, v in inp.items()}
+        m3.scan_fwd(*(sub[k] for k in keys), None, algo=m3.ALGO_TC)
+        torch.cuda.synchronize()
+        return True
+    except m3.M3Error as e:
+        if e.status == m3.M3_ERR_UNSUPPORTED:
+            return False
+        raise
+
+
+def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys):
+    import torch
+    from m3_inputs import WORKLOADS, make_prefill, make_steps
+
+    s = WORKLOADS[name].with_(seed=WORKLOADS[name].seed + rank)
+    pre = make_prefill(s, device=dev)
+    _, st = m3.scan_fwd(*(pre[k] for k in keys), None)
+    A, D = pre["A"], pre["D"]
+    del pre
+    torch.cuda.empty_cache()
+    S = args.decode_steps
+    steps = make_steps(s, S, device=dev)
+    y = torch.empty(s.batch, s.nheads, s.rank, s.headdim, dtype=s.torch_io, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sk = ("x", "B", "C", "dt", "lam", "theta")
+    # warm-up launches (they advance the state, as real decode would)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            m3.step(*(steps[k][i] for k in sk), A, D, st, y=y, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(S):
+            m3.step(*(steps[k][i] for k in sk), A, D, st, y=y, stream=stream)
+    g.replay()  # warm replay
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    el = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    per = el / S
+    ab = step_bytes(s)
+    ach = ab / per / 1e9
+    del g, steps
+    torch.cuda.empty_cache()
+    return {"workload": name, "value": world * s.batch / per, "unit": "tokens/s", "steps": S,
+            "us_per_step": per * 1e6, "gpu_launches": S,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": ach / hbm_peak, "traffic": recorded_traffic("step_kernel", name),
+                         "kernel": "step_kernel", "algorithmic_bytes_per_launch": ab,
+                         "note": "per-step time includes graph launch gaps", "peak_source": peak_src}}
+
+
+def cpu_baseline(s, keys):
+    import numpy as np
+
+    import oracle
+    from m3_inputs import make_prefill
+
+    cores = oracle.num_cores()
+    nslices = max(1, cores)
+    sub = s.with_(batch=1, nheads=nslices, seed=s.seed)
+    inp = {k: v.double().numpy() for k, v in make_prefill(sub).items()}
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.scan(*(inp[k] for k in keys))
+        reps += 1
+        if time.perf_counter() - t0 > 10.0:
+            break
+    el = time.perf_counter() - t0
+    value = reps * nslices * s.seqlen / s.nheads / el
+    return {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} x {nslices} (batch, head) slices x {s.seqlen} tokens of the same workload, "
+                      f"{el:.1f} s, scaled to tokens of all {s.nheads} heads"}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

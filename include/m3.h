@@ -1,0 +1,149 @@
+/*
+ * m3.h -- C ABI of the B200 (sm_100a) Mamba-3 SSM sequence-mixer forward.
+ *
+ * The method (per batch b, head h, token t; state H_t in R^{N x P}):
+ *
+ *   h_t = a_t h_{t-1} + (1 - lam_t) dt_t a_t B~_{t-1} x_{t-1}^T + lam_t dt_t B~_t x_t^T,
+ *   a_t = exp(dt_t A_h),      y_t = h_t^T C~_t + D_h x_t,
+ *
+ * the three-term exponential-trapezoidal recurrence displayed in
+ * "Знакомство с Mamba-3" (chernovdev.ru), section 1; with B~, C~ the inputs
+ * rotated pair-wise by the cumulative data-dependent angle
+ * phi_t[k] = sum_{s<=t} dt_s theta_s[k] (the complex-state "RoPE trick":
+ * same page, section 2, and "La dualità: Mamba-2 e Mamba-3", section
+ * "Mamba-3"); and MIMO rank R: x_t in R^{P x R}, B_t, C_t in R^{N x R}, the
+ * write a sum of R outer products (same chapter, MIMO paragraph).
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - state pairs are interleaved: pair k = rows (2k, 2k+1); theta has N/2
+ *     angle rates per token-head;
+ *   - rotation sign: B and C are rotated by +phi (standard RoPE), i.e. the
+ *     state transition on pair k is the complex eigenvalue
+ *     exp(dt (A - i theta[k])) acting on z = h[2k] + i h[2k+1];
+ *   - the state handed between calls is the plain-frame h_{T-1} together with
+ *     the raw last inputs (b_prev = B_{T-1}, x_prev = x_{T-1}), so that the
+ *     next call's t-1 trapezoid term is exact; a zero / absent initial state
+ *     means h = 0, b_prev = 0, x_prev = 0;
+ *   - B and C are per head; A and D are per head (fp32).
+ *
+ * Memory: every pointer is a DEVICE pointer owned by the caller; the library
+ * never allocates on these paths.  Tensors are dense, row-major (last index
+ * fastest), base addresses 16-byte aligned.  "io" tensors are fp32 or bf16
+ * according to m3_dims.io; A, D and all state buffers are fp32.
+ *
+ *   x, y      [batch, seqlen, nheads, rank, headdim]   io
+ *   B, C      [batch, seqlen, nheads, rank, dstate]    io
+ *   dt, lam   [batch, seqlen, nheads]                  io
+ *   theta     [batch, seqlen, nheads, dstate/2]        io
+ *   A, D      [nheads]                                 fp32
+ *   h         [batch, nheads, dstate, headdim]         fp32
+ *   b_prev    [batch, nheads, rank, dstate]            fp32
+ *   x_prev    [batch, nheads, rank, headdim]           fp32
+ *
+ * Execution: every call is asynchronous on the given CUDA stream (a
+ * cudaStream_t passed as void*, NULL = legacy default stream) and never
+ * synchronises the device.  Errors are returned as m3_status; the message of
+ * the calling thread's last failure is available from m3_last_error().  No
+ * C++ exception crosses this boundary and no kernel traps.
+ */
+#ifndef M3_H
+#define M3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define M3_API __attribute__((visibility("default")))
+#else
+#define M3_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum m3_status {
+    M3_OK = 0,
+    M3_ERR_INVALID_ARG = 1,  /* null/misaligned/overlapping pointer, bad size */
+    M3_ERR_UNSUPPORTED = 2,  /* valid sizes outside what the kernels support   */
+    M3_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed          */
+    M3_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up            */
+} m3_status;
+
+typedef enum m3_dtype { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
+
+typedef struct m3_dims {
+    int64_t batch;    /* Bt >= 0                                   */
+    int64_t seqlen;   /* T >= 0 (ignored by m3_step)               */
+    int64_t nheads;   /* H >= 1                                    */
+    int64_t headdim;  /* P >= 1                                    */
+    int64_t dstate;   /* N >= 2, even                              */
+    int64_t rank;     /* R >= 1 (MIMO rank; 1 = SISO)              */
+    int32_t io;       /* m3_dtype of x, B, C, dt, lam, theta, y    */
+    int32_t reserved; /* must be 0                                 */
+} m3_dims;
+
+typedef struct m3_state {
+    float *h;       /* [batch, nheads, dstate, headdim] */
+    float *b_prev;  /* [batch, nheads, rank, dstate]    */
+    float *x_prev;  /* [batch, nheads, rank, headdim]   */
+} m3_state;
+
+/* Prefill kernel selection for m3_scan_fwd_algo. */
+typedef enum m3_algo {
+    M3_ALGO_AUTO = 0,   /* tensor-core path for bf16 where supported, else SIMT */
+    M3_ALGO_SIMT = 1,   /* fp32 CUDA-core chunked scan (any supported size)      */
+    M3_ALGO_TC = 2      /* tcgen05/TMEM/TMA chunked scan (bf16 only)             */
+} m3_algo;
+
+/* Bytes of device workspace m3_scan_fwd needs for these dims (0 = none; the
+ * workspace pointer may then be NULL).  Pure host function. */
+M3_API m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes);
+
+/* Prefill: the chunked scan over a whole sequence (the four-piece chunked
+ * algorithm of "La dualità: Mamba-2 e Mamba-3", section "Perché conviene: i
+ * tensor core", extended with the trapezoid's previous-token term and the
+ * pair rotations).  Reads x, B, C, dt, lam, theta, A, D and the optional
+ * initial state `init` (NULL = zero state; its three buffers all required
+ * when given); writes y and, when `final_state` is non-NULL, the state after
+ * the last token.  `init` and `final_state` may be the same buffers only if
+ * they are identical (in-place resume); partial overlaps are rejected, as is
+ * any overlap of y with an input.  seqlen = 0 copies init to final_state. */
+M3_API m3_status m3_scan_fwd(const m3_dims *d,
+                      const void *x, const void *B, const void *C,
+                      const void *dt, const void *lam, const void *theta,
+                      const float *A, const float *D,
+                      const m3_state *init, void *y, const m3_state *final_state,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same as m3_scan_fwd with an explicit kernel choice (for cross-checks).
+ * M3_ALGO_TC returns M3_ERR_UNSUPPORTED for sizes that path does not cover. */
+M3_API m3_status m3_scan_fwd_algo(int algo, const m3_dims *d,
+                           const void *x, const void *B, const void *C,
+                           const void *dt, const void *lam, const void *theta,
+                           const float *A, const float *D,
+                           const m3_state *init, void *y, const m3_state *final_state,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Decode: one token per (batch, head) against a resident state, updated in
+ * place (the recurrent form of the same method, one token at a time).
+ * x [batch,nheads,rank,headdim], B/C [batch,nheads,rank,dstate],
+ * dt/lam [batch,nheads], theta [batch,nheads,dstate/2] (io dtype);
+ * y [batch,nheads,rank,headdim] (io).  `state` buffers are read and written
+ * once each; y must not overlap anything else. */
+M3_API m3_status m3_step(const m3_dims *d,
+                  const void *x, const void *B, const void *C,
+                  const void *dt, const void *lam, const void *theta,
+                  const float *A, const float *D,
+                  const m3_state *state, void *y, void *stream);
+
+/* Message describing the calling thread's most recent failure ("" if none). */
+M3_API const char *m3_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+M3_API int m3_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* M3_H */

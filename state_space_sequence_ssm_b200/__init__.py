@@ -1,0 +1,168 @@
+"""Thin Python binding of the m3 C ABI (include/m3.h).
+
+Argument marshalling only: every step of the method runs in the CUDA
+library ``libm3.so`` built from ``csrc/``.  PyTorch supplies device memory and
+streams.  There is no fallback: if the library is missing, the first call
+raises ImportError, and every call checks that its tensors live on a CUDA
+device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libm3.so")
+
+M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
+M3_F32, M3_BF16 = 0, 1
+ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
+_STATUS = {0: "M3_OK", 1: "M3_ERR_INVALID_ARG", 2: "M3_ERR_UNSUPPORTED", 3: "M3_ERR_CUDA", 4: "M3_ERR_TIMEOUT"}
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("rank", ctypes.c_int64),
+                ("io", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class CState(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_void_p), ("b_prev", ctypes.c_void_p), ("x_prev", ctypes.c_void_p)]
+
+
+class M3Error(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class State(NamedTuple):
+    h: torch.Tensor       # [Bt, H, N, P] fp32
+    b_prev: torch.Tensor  # [Bt, H, R, N] fp32
+    x_prev: torch.Tensor  # [Bt, H, R, P] fp32
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"m3 CUDA library not built ({LIB_PATH} missing); "
+                          "run `python -m state_space_sequence_ssm_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, dp = ctypes.c_void_p, ctypes.POINTER(Dims)
+    sp = ctypes.POINTER(CState)
+    lib.m3_scan_workspace_size.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.m3_scan_fwd.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_scan_fwd_algo.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
+    for f in (lib.m3_scan_workspace_size, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
+        f.restype = ctypes.c_int
+    lib.m3_last_error.argtypes = []
+    lib.m3_last_error.restype = ctypes.c_char_p
+    lib.m3_version.restype = ctypes.c_int
+    return lib
+
+
+_lib = None
+
+
+def get_lib():
+    """The loaded libm3.so (raises ImportError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def __getattr__(name):
+    if name == "lib":
+        return get_lib()
+    raise AttributeError(name)
+
+
+def _check(status: int):
+    if status != M3_OK:
+        raise M3Error(status, get_lib().m3_last_error().decode(errors="replace"))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("m3: tensors must be on a CUDA device (no CPU path)")
+            if not t.is_contiguous():
+                raise ValueError("m3: tensors must be contiguous")
+
+
+def make_dims(Bt, T, H, P, N, R, dtype) -> Dims:
+    io = M3_BF16 if dtype == torch.bfloat16 else M3_F32
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("io dtype must be float32 or bfloat16")
+    return Dims(Bt, T, H, P, N, R, io, 0)
+
+
+def _cstate(s: State | None):
+    if s is None:
+        return None
+    _require_cuda(*s)
+    return ctypes.pointer(CState(s.h.data_ptr(), s.b_prev.data_ptr(), s.x_prev.data_ptr()))
+
+
+def empty_state(Bt, H, N, P, R, device="cuda") -> State:
+    f = dict(device=device, dtype=torch.float32)
+    return State(torch.zeros(Bt, H, N, P, **f), torch.zeros(Bt, H, R, N, **f), torch.zeros(Bt, H, R, P, **f))
+
+
+def workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(get_lib().m3_scan_workspace_size(ctypes.byref(dims), ctypes.byref(n)))
+    return n.value
+
+
+def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
+             y=None, final: State | None = None, workspace=None, algo: int = ALGO_AUTO, stream=None):
+    """Prefill scan.  x [Bt,T,H,R,P], B/C [Bt,T,H,R,N], dt/lam [Bt,T,H],
+    theta [Bt,T,H,N/2] in one io dtype (fp32 or bf16); A/D [H] fp32.
+    Returns (y, final State or None)."""
+    _require_cuda(x, B, C, dt, lam, theta, A, D, y, workspace)
+    Bt, T, H, R, P = x.shape
+    N = B.shape[-1]
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype)
+    if y is None:
+        y = torch.empty_like(x)
+    if final is None and want_state:
+        final = State(torch.empty(Bt, H, N, P, device=x.device), torch.empty(Bt, H, R, N, device=x.device),
+                      torch.empty(Bt, H, R, P, device=x.device))
+    ws_need = workspace_size(dims) if algo != ALGO_SIMT else 0
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(get_lib().m3_scan_fwd_algo(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
+                                _cstate(init), _ptr(y), _cstate(final), _ptr(workspace), ws_bytes,
+                                _stream(stream)))
+    return y, final
+
+
+def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None):
+    """One decode step in place on `state`.  x [Bt,H,R,P], B/C [Bt,H,R,N],
+    dt/lam [Bt,H], theta [Bt,H,N/2].  Returns y [Bt,H,R,P]."""
+    _require_cuda(x, B, C, dt, lam, theta, A, D, y)
+    Bt, H, R, P = x.shape
+    N = B.shape[-1]
+    dims = make_dims(Bt, 1, H, P, N, R, x.dtype)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(get_lib().m3_step(ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state),
+                       _ptr(y), _stream(stream)))
+    return y

@@ -1,0 +1,267 @@
+// api.cpp -- the C ABI of include/m3.h: argument validation, dispatch to the
+// kernels, and thread-local error reporting.  No exception crosses the
+// boundary; nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <exception>
+#include <string>
+
+#include "m3_internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+m3_status fail(m3_status s, const char *fmt, const char *a = nullptr) {
+    char buf[512];
+    std::snprintf(buf, sizeof buf, fmt, a ? a : "");
+    g_err = buf;
+    return s;
+}
+
+m3_status cuda_fail(cudaError_t e, const char *where) {
+    char buf[512];
+    std::snprintf(buf, sizeof buf, "%s: %s (%s)", where, cudaGetErrorString(e), cudaGetErrorName(e));
+    g_err = buf;
+    return M3_ERR_CUDA;
+}
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+    bool empty() const { return hi <= lo; }
+};
+Range range(const void *p, size_t bytes) {
+    uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    return {lo, lo + (p ? bytes : 0)};
+}
+bool overlap(Range a, Range b) { return !a.empty() && !b.empty() && a.lo < b.hi && b.lo < a.hi; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+m3_status check_dims(const m3_dims *d, bool decode) {
+    if (!d) return fail(M3_ERR_INVALID_ARG, "dims is NULL");
+    if (d->batch < 0 || (!decode && d->seqlen < 0))
+        return fail(M3_ERR_INVALID_ARG, "batch and seqlen must be >= 0");
+    if (d->nheads < 1 || d->headdim < 1 || d->rank < 1)
+        return fail(M3_ERR_INVALID_ARG, "nheads, headdim and rank must be >= 1");
+    if (d->dstate < 2 || (d->dstate & 1))
+        return fail(M3_ERR_INVALID_ARG, "dstate must be even and >= 2 (state pairs)");
+    if (d->io != M3_F32 && d->io != M3_BF16) return fail(M3_ERR_INVALID_ARG, "io must be M3_F32 or M3_BF16");
+    if (d->reserved != 0) return fail(M3_ERR_INVALID_ARG, "reserved field must be 0");
+    if (d->dstate > 256 || d->headdim > 256 || d->rank > 8)
+        return fail(M3_ERR_UNSUPPORTED, "supported sizes: dstate <= 256, headdim <= 256, rank <= 8");
+    if (d->headdim % 4 != 0 && d->headdim != 1 && d->headdim != 2)
+        return fail(M3_ERR_UNSUPPORTED, "headdim must be a multiple of 4 (or 1, 2)");
+    // every flat index must fit comfortably in int64
+    const double elems = double(d->batch) * double(decode ? 1 : d->seqlen) * double(d->nheads) *
+                         double(d->rank) * double(d->dstate > d->headdim ? d->dstate : d->headdim);
+    if (elems > 4.0e18) return fail(M3_ERR_INVALID_ARG, "problem too large");
+    return M3_OK;
+}
+
+// Shared validation of tensor pointers.  `tok` = number of token-heads.
+m3_status check_tensors(const m3_dims *d, int64_t tok, const void *x, const void *B, const void *C,
+                        const void *dt, const void *lam, const void *theta, const float *A,
+                        const float *D, const void *y, Range *ins, int *nin, Range *yr) {
+    const size_t es = d->io == M3_BF16 ? 2 : 4;
+    const int64_t R = d->rank, P = d->headdim, N = d->dstate;
+    if (tok > 0) {
+        if (!x || !B || !C || !dt || !lam || !theta || !y)
+            return fail(M3_ERR_INVALID_ARG, "x, B, C, dt, lam, theta and y are required");
+        const void *ptrs[] = {x, B, C, theta, y};
+        for (const void *p : ptrs)
+            if (!aligned16(p)) return fail(M3_ERR_INVALID_ARG, "x, B, C, theta and y must be 16-byte aligned");
+        if ((reinterpret_cast<uintptr_t>(dt) | reinterpret_cast<uintptr_t>(lam)) % es)
+            return fail(M3_ERR_INVALID_ARG, "dt and lam must be aligned to their element size");
+    }
+    if (!A || !D) return fail(M3_ERR_INVALID_ARG, "A and D are required");
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(D)) % 4)
+        return fail(M3_ERR_INVALID_ARG, "A and D must be 4-byte aligned");
+    int n = 0;
+    ins[n++] = range(x, tok * R * P * es);
+    ins[n++] = range(B, tok * R * N * es);
+    ins[n++] = range(C, tok * R * N * es);
+    ins[n++] = range(dt, tok * es);
+    ins[n++] = range(lam, tok * es);
+    ins[n++] = range(theta, tok * (N / 2) * es);
+    ins[n++] = range(A, d->nheads * 4);
+    ins[n++] = range(D, d->nheads * 4);
+    *nin = n;
+    *yr = range(y, tok * R * P * es);
+    for (int i = 0; i < n; ++i)
+        if (overlap(*yr, ins[i])) return fail(M3_ERR_INVALID_ARG, "y overlaps an input tensor");
+    return M3_OK;
+}
+
+m3_status check_state(const m3_dims *d, const m3_state *s, const char *what, Range out[3]) {
+    const int64_t BH = d->batch * d->nheads;
+    const int64_t N = d->dstate, P = d->headdim, R = d->rank;
+    if (!s->h || !s->b_prev || !s->x_prev) {
+        g_err = std::string(what) + ": h, b_prev and x_prev are all required";
+        return M3_ERR_INVALID_ARG;
+    }
+    if (!aligned16(s->h) || !aligned16(s->b_prev) || !aligned16(s->x_prev)) {
+        g_err = std::string(what) + ": state buffers must be 16-byte aligned";
+        return M3_ERR_INVALID_ARG;
+    }
+    out[0] = range(s->h, BH * N * P * 4);
+    out[1] = range(s->b_prev, BH * R * N * 4);
+    out[2] = range(s->x_prev, BH * R * P * 4);
+    for (int i = 0; i < 3; ++i)
+        for (int j = i + 1; j < 3; ++j)
+            if (overlap(out[i], out[j])) {
+                g_err = std::string(what) + ": state buffers overlap each other";
+                return M3_ERR_INVALID_ARG;
+            }
+    return M3_OK;
+}
+
+m3::Problem make_problem(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
+                         const void *lam, const void *theta, const float *A, const float *D, void *y,
+                         void *stream) {
+    m3::Problem p{};
+    p.Bt = d->batch; p.T = d->seqlen; p.H = d->nheads; p.P = d->headdim; p.N = d->dstate; p.R = d->rank;
+    p.bf16 = d->io == M3_BF16;
+    p.x = x; p.B = B; p.C = C; p.dt = dt; p.lam = lam; p.theta = theta; p.A = A; p.D = D; p.y = y;
+    p.stream = static_cast<cudaStream_t>(stream);
+    return p;
+}
+
+m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
+                    const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
+                    void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream) {
+    m3_status s = check_dims(d, false);
+    if (s != M3_OK) return s;
+    if (algo != M3_ALGO_AUTO && algo != M3_ALGO_SIMT && algo != M3_ALGO_TC)
+        return fail(M3_ERR_INVALID_ARG, "unknown algo");
+    const int64_t tok = d->batch * d->seqlen * d->nheads;
+    Range ins[8], yr;
+    int nin = 0;
+    s = check_tensors(d, tok, x, B, C, dt, lam, theta, A, D, y, ins, &nin, &yr);
+    if (s != M3_OK) return s;
+    Range ir[3] = {}, fr[3] = {};
+    if (init && (s = check_state(d, init, "init", ir)) != M3_OK) return s;
+    if (fin && (s = check_state(d, fin, "final_state", fr)) != M3_OK) return s;
+    for (int i = 0; i < 3; ++i) {
+        if (overlap(fr[i], yr)) return fail(M3_ERR_INVALID_ARG, "final_state overlaps y");
+        for (int j = 0; j < nin; ++j)
+            if (overlap(fr[i], ins[j]) || overlap(ir[i], yr))
+                return fail(M3_ERR_INVALID_ARG, "state buffers overlap the sequence tensors");
+        for (int j = 0; j < 3; ++j) {
+            // in-place resume (identical buffers) is allowed; partial overlap is not
+            const bool same = i == j && fr[i].lo == ir[j].lo && fr[i].hi == ir[j].hi;
+            if (!same && overlap(fr[i], ir[j]))
+                return fail(M3_ERR_INVALID_ARG, "final_state partially overlaps init");
+        }
+    }
+    m3::Problem p = make_problem(d, x, B, C, dt, lam, theta, A, D, y, stream);
+    if (init) { p.h0 = init->h; p.bp0 = init->b_prev; p.xp0 = init->x_prev; }
+    if (fin) { p.hT = fin->h; p.bpT = fin->b_prev; p.xpT = fin->x_prev; }
+    p.ws = ws;
+    p.ws_bytes = ws_bytes;
+
+    const char *why = nullptr;
+    const char *tc_why = nullptr;
+    const bool tc_ok = m3::prefill_tc_supported(p, &tc_why);
+    bool use_tc = false;
+    if (algo == M3_ALGO_TC) {
+        if (!tc_ok) return fail(M3_ERR_UNSUPPORTED, "%s", tc_why ? tc_why : "tensor-core path unsupported");
+        use_tc = true;
+    } else if (algo == M3_ALGO_AUTO) {
+        use_tc = tc_ok;
+    }
+    if (use_tc) {
+        const size_t need = m3::prefill_tc_workspace(p);
+        if (need > ws_bytes || (need && !ws))
+            return fail(M3_ERR_INVALID_ARG, "workspace too small (query m3_scan_workspace_size)");
+    }
+    cudaError_t e = use_tc ? m3::launch_prefill_tc(p, &why) : m3::launch_prefill_simt(p, &why);
+    if (e == cudaErrorNotSupported && why) return fail(M3_ERR_UNSUPPORTED, "%s", why);
+    if (e != cudaSuccess) return cuda_fail(e, use_tc ? "m3_scan_fwd (tensor-core kernel)" : "m3_scan_fwd (SIMT kernel)");
+    return M3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int m3_version(void) { return 100; }
+
+const char *m3_last_error(void) { return g_err.c_str(); }
+
+m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes) {
+    try {
+        m3_status s = check_dims(d, false);
+        if (s != M3_OK) return s;
+        if (!bytes) return fail(M3_ERR_INVALID_ARG, "bytes is NULL");
+        m3::Problem p{};
+        p.Bt = d->batch; p.T = d->seqlen; p.H = d->nheads; p.P = d->headdim; p.N = d->dstate; p.R = d->rank;
+        p.bf16 = d->io == M3_BF16;
+        const char *why = nullptr;
+        *bytes = m3::prefill_tc_supported(p, &why) ? m3::prefill_tc_workspace(p) : 0;
+        return M3_OK;
+    } catch (const std::exception &ex) {
+        return fail(M3_ERR_INVALID_ARG, "internal error: %s", ex.what());
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
+m3_status m3_scan_fwd(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
+                      const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
+                      void *y, const m3_state *final_state, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+    try {
+        return scan_impl(M3_ALGO_AUTO, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace,
+                         workspace_bytes, stream);
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
+m3_status m3_scan_fwd_algo(int algo, const m3_dims *d, const void *x, const void *B, const void *C,
+                           const void *dt, const void *lam, const void *theta, const float *A, const float *D,
+                           const m3_state *init, void *y, const m3_state *final_state, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    try {
+        return scan_impl(algo, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace,
+                         workspace_bytes, stream);
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
+m3_status m3_step(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
+                  const void *lam, const void *theta, const float *A, const float *D, const m3_state *state,
+                  void *y, void *stream) {
+    try {
+        m3_status s = check_dims(d, true);
+        if (s != M3_OK) return s;
+        const int64_t tok = d->batch * d->nheads;
+        Range ins[8], yr;
+        int nin = 0;
+        s = check_tensors(d, tok, x, B, C, dt, lam, theta, A, D, y, ins, &nin, &yr);
+        if (s != M3_OK) return s;
+        if (!state) return fail(M3_ERR_INVALID_ARG, "state is required");
+        Range sr[3];
+        if ((s = check_state(d, state, "state", sr)) != M3_OK) return s;
+        for (int i = 0; i < 3; ++i) {
+            if (overlap(sr[i], yr)) return fail(M3_ERR_INVALID_ARG, "state overlaps y");
+            for (int j = 0; j < nin; ++j)
+                if (overlap(sr[i], ins[j])) return fail(M3_ERR_INVALID_ARG, "state overlaps an input tensor");
+        }
+        m3::Problem p = make_problem(d, x, B, C, dt, lam, theta, A, D, y, stream);
+        p.T = 1;
+        p.hT = state->h; p.bpT = state->b_prev; p.xpT = state->x_prev;
+        const char *why = nullptr;
+        cudaError_t e = m3::launch_step(p, &why);
+        if (e == cudaErrorNotSupported && why) return fail(M3_ERR_UNSUPPORTED, "%s", why);
+        if (e != cudaSuccess) return cuda_fail(e, "m3_step");
+        return M3_OK;
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,34 @@
+// Internal interface between the C ABI layer (api.cpp) and the kernel
+// translation units.  Not installed, not part of the public ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/m3.h"
+
+namespace m3 {
+
+// Validated problem description handed to the launchers.
+struct Problem {
+    int64_t Bt, T, H, P, N, R;
+    bool bf16;
+    const void *x, *B, *C, *dt, *lam, *theta;
+    const float *A, *D;
+    const float *h0, *bp0, *xp0;  // nullable (zero initial state)
+    void *y;
+    float *hT, *bpT, *xpT;        // nullable (no final state wanted)
+    void *ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+// Each launcher returns cudaSuccess or the launch error; `why` receives a
+// static message for M3_ERR_UNSUPPORTED-style refusals (returned as
+// cudaErrorNotSupported).
+cudaError_t launch_prefill_simt(const Problem &p, const char **why);
+bool prefill_tc_supported(const Problem &p, const char **why);
+size_t prefill_tc_workspace(const Problem &p);
+cudaError_t launch_prefill_tc(const Problem &p, const char **why);
+cudaError_t launch_step(const Problem &p, const char **why);
+
+}  // namespace m3

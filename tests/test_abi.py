@@ -1,0 +1,133 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+include/m3.h declares, and rejects bad arguments with a status (never a
+crash) before touching any device memory.  CPU-only."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "m3.h")
+
+
+@pytest.fixture(scope="module")
+def m3():
+    from state_space_sequence_ssm_b200 import build
+    build.build()
+    import state_space_sequence_ssm_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(m3_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(m3):
+    names = declared_functions()
+    assert {"m3_scan_fwd", "m3_step", "m3_scan_workspace_size", "m3_last_error"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", m3.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (m3_[a-z0-9_]+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in names:
+        getattr(m3.lib, n)  # resolvable through ctypes
+
+
+def test_only_abi_symbols_exported(m3):
+    out = subprocess.run(["nm", "-D", "--defined-only", m3.LIB_PATH], capture_output=True, text=True).stdout
+    ours = set(re.findall(r"\bT (m3\w*)", out))
+    assert ours == set(declared_functions())
+
+
+def dims(m3, Bt=2, T=8, H=2, P=8, N=8, R=1, io=0, reserved=0):
+    return m3.Dims(Bt, T, H, P, N, R, io, reserved)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def call_scan(m3, d, ptrs=None, init=None, fin=None, y=None, algo=0):
+    p = ptrs or [FAKE + i * 0x100000 for i in range(8)]
+    vp = [ctypes.c_void_p(v) if v is not None else None for v in p]
+    yv = ctypes.c_void_p(y if y is not None else FAKE + 9 * 0x100000)
+    return m3.lib.m3_scan_fwd_algo(algo, ctypes.byref(d) if d is not None else None, *vp, init, yv, fin,
+                                   None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=7), 1), (dict(N=0), 1), (dict(H=0), 1), (dict(P=0), 1), (dict(R=0), 1),
+    (dict(Bt=-1), 1), (dict(T=-2), 1), (dict(io=5), 1), (dict(reserved=1), 1),
+    (dict(N=512), 2), (dict(R=16), 2), (dict(P=6), 2),
+])
+def test_bad_dims_rejected(m3, kw, status):
+    assert call_scan(m3, dims(m3, **kw)) == status
+    assert m3.lib.m3_last_error().decode()
+
+
+def test_null_dims(m3):
+    assert call_scan(m3, None) == 1
+    n = ctypes.c_size_t(7)
+    assert m3.lib.m3_scan_workspace_size(None, ctypes.byref(n)) == 1
+
+
+def test_missing_tensor_rejected(m3):
+    p = [FAKE + i * 0x100000 for i in range(8)]
+    p[1] = None
+    assert call_scan(m3, dims(m3), ptrs=p) == 1
+    assert "required" in m3.lib.m3_last_error().decode()
+
+
+def test_misaligned_rejected(m3):
+    p = [FAKE + i * 0x100000 for i in range(8)]
+    p[0] += 4
+    assert call_scan(m3, dims(m3), ptrs=p) == 1
+    assert "aligned" in m3.lib.m3_last_error().decode()
+
+
+def test_y_overlapping_input_rejected(m3):
+    p = [FAKE + i * 0x100000 for i in range(8)]
+    assert call_scan(m3, dims(m3), ptrs=p, y=p[2] + 16) == 1
+    assert "overlap" in m3.lib.m3_last_error().decode()
+
+
+def test_partial_state_overlap_rejected(m3):
+    base = 0x4000000
+    init = m3.CState(base, base + 0x10000, base + 0x20000)
+    fin = m3.CState(base + 0x100, base + 0x30000, base + 0x40000)   # h overlaps init.h partially
+    assert call_scan(m3, dims(m3), init=ctypes.pointer(init), fin=ctypes.pointer(fin)) == 1
+    assert "overlap" in m3.lib.m3_last_error().decode()
+
+
+def test_incomplete_state_rejected(m3):
+    init = m3.CState(0x4000000, None, 0x4020000)
+    assert call_scan(m3, dims(m3), init=ctypes.pointer(init)) == 1
+
+
+def test_tc_algo_refuses_fp32_io(m3):
+    assert call_scan(m3, dims(m3, io=0), algo=2) == 2
+
+
+def test_unknown_algo(m3):
+    assert call_scan(m3, dims(m3), algo=9) == 1
+
+
+def test_step_validation(m3):
+    d = dims(m3)
+    vp = [ctypes.c_void_p(FAKE + i * 0x100000) for i in range(8)]
+    assert m3.lib.m3_step(ctypes.byref(d), *vp, None, ctypes.c_void_p(FAKE + 9 * 0x100000), None) == 1
+    st = m3.CState(FAKE + 3 * 0x100000, 0x7000000, 0x7100000)  # h overlaps C
+    assert m3.lib.m3_step(ctypes.byref(d), *vp, ctypes.pointer(st), ctypes.c_void_p(0x7200000), None) == 1
+
+
+def test_workspace_query_is_host_only(m3):
+    n = ctypes.c_size_t(123)
+    assert m3.lib.m3_scan_workspace_size(ctypes.byref(dims(m3, io=0)), ctypes.byref(n)) == 0
+    assert n.value == 0  # fp32 I/O runs the SIMT path, which needs none
+
+
+def test_version(m3):
+    assert m3.lib.m3_version() == 100
