@@ -108,7 +108,8 @@ M3_API m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes);
  * when given); writes y and, when `final_state` is non-NULL, the state after
  * the last token.  `init` and `final_state` may be the same buffers only if
  * they are identical (in-place resume); partial overlaps are rejected, as is
- * any overlap of y with an input.  seqlen = 0 copies init to final_state. */
+ * any overlap of y with an input.  seqlen = 0 copies init to final_state.
+ * With batch = 0 nothing is read or written and every pointer may be NULL. */
 M3_API m3_status m3_scan_fwd(const m3_dims *d,
                       const void *x, const void *B, const void *C,
                       const void *dt, const void *lam, const void *theta,
@@ -136,6 +137,16 @@ M3_API m3_status m3_step(const m3_dims *d,
                   const void *dt, const void *lam, const void *theta,
                   const float *A, const float *D,
                   const m3_state *state, void *y, void *stream);
+
+/* Wait for all work queued on `stream` (blocking the calling host thread),
+ * then report any device-side failure recorded since the previous call:
+ * M3_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel
+ * drained its own copies and returned without trapping; its outputs are then
+ * incomplete), M3_ERR_CUDA if the stream itself reported an error.  The
+ * recorded failure is cleared.  A device-side wait gives up only on a
+ * library bug; this call exists so that such a bug surfaces as a status
+ * instead of a hang. */
+M3_API m3_status m3_stream_status(void *stream);
 
 /* Message describing the calling thread's most recent failure ("" if none). */
 M3_API const char *m3_last_error(void);

@@ -58,6 +58,8 @@ def _load():
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
     for f in (lib.m3_scan_workspace_size, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
         f.restype = ctypes.c_int
+    lib.m3_stream_status.argtypes = [vp]
+    lib.m3_stream_status.restype = ctypes.c_int
     lib.m3_last_error.argtypes = []
     lib.m3_last_error.restype = ctypes.c_char_p
     lib.m3_version.restype = ctypes.c_int
@@ -152,6 +154,11 @@ def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_s
                                 _cstate(init), _ptr(y), _cstate(final), _ptr(workspace), ws_bytes,
                                 _stream(stream)))
     return y, final
+
+
+def stream_status(stream=None):
+    """Synchronise the stream and raise if a kernel's bounded wait gave up."""
+    _check(get_lib().m3_stream_status(_stream(stream)))
 
 
 def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None):

@@ -97,6 +97,10 @@ m3_status check_tensors(const m3_dims *d, int64_t tok, const void *x, const void
 m3_status check_state(const m3_dims *d, const m3_state *s, const char *what, Range out[3]) {
     const int64_t BH = d->batch * d->nheads;
     const int64_t N = d->dstate, P = d->headdim, R = d->rank;
+    if (BH == 0) {  // zero-sized state: nothing is read or written, pointers may be NULL
+        out[0] = out[1] = out[2] = Range{0, 0};
+        return M3_OK;
+    }
     if (!s->h || !s->b_prev || !s->x_prev) {
         g_err = std::string(what) + ": h, b_prev and x_prev are all required";
         return M3_ERR_INVALID_ARG;
@@ -227,6 +231,23 @@ m3_status m3_scan_fwd_algo(int algo, const m3_dims *d, const void *x, const void
     try {
         return scan_impl(algo, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace,
                          workspace_bytes, stream);
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
+m3_status m3_stream_status(void *stream) {
+    try {
+        unsigned code = 0;
+        cudaError_t e = m3::read_device_error(&code, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "m3_stream_status");
+        if (code) {
+            char buf[128];
+            std::snprintf(buf, sizeof buf, "a bounded device-side wait gave up (code 0x%x)", code);
+            g_err = buf;
+            return M3_ERR_TIMEOUT;
+        }
+        return M3_OK;
     } catch (...) {
         return fail(M3_ERR_INVALID_ARG, "internal error");
     }

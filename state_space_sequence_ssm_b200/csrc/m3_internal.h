@@ -30,5 +30,8 @@ bool prefill_tc_supported(const Problem &p, const char **why);
 size_t prefill_tc_workspace(const Problem &p);
 cudaError_t launch_prefill_tc(const Problem &p, const char **why);
 cudaError_t launch_step(const Problem &p, const char **why);
+// Synchronise `stream`, then read and clear the device error word that the
+// tensor-core kernel's bounded waits set when they give up.
+cudaError_t read_device_error(unsigned *code, cudaStream_t stream);
 
 }  // namespace m3
