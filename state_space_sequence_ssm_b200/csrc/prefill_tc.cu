@@ -9,21 +9,30 @@
 // of B and C by the chunk-local cumulative angle, and rank-R MIMO rows.
 //
 // One CTA per (batch, head) walks its sequence in chunks of 128 rows
-// (Q = 128 / R tokens x R ranks), which is the M = 128 shape of one tcgen05
-// MMA.  Roles (192 threads):
-//   warps 0-3  compute warpgroup: per-token scalars, angles, in-place
-//              rotation of the B/C tiles, the decay mask S -> P, the fp32
-//              carried state (in registers), and the output epilogue;
-//   warp 4     TMA producer: x, B, C tiles (128B-swizzled) into a 2-stage ring;
-//   warp 5     TMEM owner and single-thread MMA issuer.
-// Per chunk c (tensor cores, bf16 operands from shared memory, fp32 in TMEM):
-//   S  = C~ B~^T               (128 x 128, K = N)      -> masked into P (bf16)
-//   G  = B~^T (w o X)          (N x 64,  K = 128 rows) chunk state
-//   Yo = C~ h*_{c-1}           (128 x 64, K = N)       carried-state readout
-//   Yd = P X                   (128 x 64, K = 128 rows) diagonal block
-// and on CUDA cores: y = Yd + exp(cA_t) Yo + D x;
-// h*_c = Rot(-Phi_c)(exp(cA_end) h*_{c-1} + G) kept in fp32 registers (the
-// plain frame, so no angle ever exceeds one chunk's sum).
+// (Q = 128 / R tokens x R ranks), the M = 128 shape of one tcgen05 MMA.
+// Per chunk c the tensor cores compute (bf16 operands in shared memory,
+// fp32 accumulators in TMEM)
+//   S  = C~ B~^T          (128 x 128, K = N)        masked into P (bf16)
+//   G  = B~^T (w o X)     (N x 64,  K = 128 rows)   chunk state
+//   Yo = C~ h*_{c-1}      (128 x 64, K = N)         carried-state readout
+//   Yd = P X              (128 x 64, K = 128 rows)  diagonal block
+// and the CUDA cores y = Yd + exp(cA_t) Yo + D x and
+// h*_c = Rot(-Phi_c)(exp(cA_end) h*_{c-1} + G), the carried state kept in
+// fp32 registers in the plain frame (no angle exceeds one chunk's sum).
+//
+// Warp roles (320 threads), pipelined across chunks:
+//   warps 0-3  prologue warpgroup: per-token scalars, cumulative angles, the
+//              in-place rotation of the B and C tiles, and w o X;
+//   warps 4-7  state warpgroup: the carried state update, the decay mask
+//              S -> P (written to TMEM, the A operand of Yd) and the
+//              epilogue (about one chunk behind warps 0-3);
+//   warp 8     TMA producers: lane 0 fills a 2-stage ring of B and C tiles
+//              (freed as soon as S, G and Yo have read them), lane 1 a
+//              3-stage ring of x tiles (freed after the epilogue), both
+//              128B-swizzled, with L2 prefetches of the chunks ahead;
+//   warp 9     TMEM owner and single-thread MMA issuer.
+// Every wait is bounded; a wait that gives up records a code that the host
+// reads back with m3_stream_status() and the CTA drains and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -43,38 +52,47 @@ using namespace tc;
 
 constexpr int kP = 64;           // head dim this kernel is built for
 constexpr int kRows = 128;       // rows per chunk = MMA M
-constexpr int kCompute = 128;    // compute warpgroup threads (warps 0-3)
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
-constexpr int kThreads = 192;
+constexpr int kWG = 128;         // threads per warpgroup
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColG = 128, kColYo = 192, kColYd = 256;
+// TMEM columns: S [0,128), G [128,192), Yo double-buffered [192,320), Yd [320,384),
+// P (bf16 pairs) [384,448)
+constexpr uint32_t kColS = 0, kColG = 128, kColYo = 192, kColYd = 320, kColP = 384;
+constexpr int kNX = 3;   // x tile stages (also the number of per-chunk scalar buffers)
+constexpr uint32_t kBarPro = 1, kBarState = 2;  // named barriers of the two warpgroups
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPrefetchAhead = 3;  // chunks of tiles prefetched into L2 ahead of their load
 
 template <int N, int R>
 struct Cfg {
     static constexpr int Q = kRows / R;      // tokens per chunk
     static constexpr int K2 = N / 2;         // state pairs
     static constexpr int KB = N / 64;        // 64-wide blocks of the state dim
-    static constexpr int TPP = kCompute / K2;  // threads per pair (angle pass)
-    static constexpr int TPT = Q / TPP;      // tokens per thread (angle pass)
+    static constexpr int G4 = K2 / 4;        // groups of 4 pairs = one 16-byte chunk of a row
+    static constexpr int NPART = kWG / G4;   // token parts of the angle pass
+    static constexpr int TPT = Q / NPART;    // tokens per thread in the angle pass
+    static constexpr int TB = (4 / R) < TPT ? (4 / R) : TPT;  // tokens per rotation batch
     static constexpr uint32_t X_BYTES = kRows * 128;         // 16 KB
     static constexpr uint32_t BC_BYTES = KB * kRows * 128;   // one B or C tile
-    static constexpr uint32_t STAGE_BYTES = X_BYTES + 2 * BC_BYTES;
-    static constexpr bool P_IN_C = (N >= 128);  // P reuses the chunk's C~ tile
-    static constexpr uint32_t OFF_XW = 2 * STAGE_BYTES;
+    static constexpr uint32_t BCS_BYTES = 2 * BC_BYTES;      // one stage of the B/C ring
+    static constexpr uint32_t OFF_BC = 0;                    // 2 stages of {B, C}
+    static constexpr uint32_t OFF_X = OFF_BC + 2 * BCS_BYTES;  // kNX stages of x
+    static constexpr uint32_t OFF_XW = OFF_X + kNX * X_BYTES;
     static constexpr uint32_t OFF_HB = OFF_XW + X_BYTES;
     static constexpr uint32_t HB_BYTES = N * 128;
-    static constexpr uint32_t OFF_P = OFF_HB + HB_BYTES;
-    static constexpr uint32_t P_BYTES = P_IN_C ? 0u : 2u * kRows * 128u;
-    static constexpr uint32_t OFF_SCAL = OFF_P + P_BYTES;
-    static constexpr uint32_t SCAL_FLOATS = 5 * Q + 2 * K2 + TPP * K2 + 8;
+    static constexpr uint32_t OFF_SCAL = OFF_HB + HB_BYTES;
+    // kNX buffers of {cAl2, gam, ghat, colf}[Q] + {cos, sin}[K2] (read by the
+    // state warpgroup a chunk later) + {wst, dts}[Q] + phis[NPART][K2] + wtot[8]
+    static constexpr uint32_t SB = 4 * Q + 2 * K2;
+    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 8;
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
-    static constexpr uint32_t NBARS = 9;
+    static constexpr uint32_t NBARS = 19;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024 alignment
-    static_assert(K2 <= kCompute && kCompute % K2 == 0, "pairs must tile the warpgroup");
-    static_assert(Q % TPP == 0, "tokens must split across a pair's threads");
+    static_assert(K2 % 4 == 0 && kWG % G4 == 0, "pair groups must tile the warpgroup");
+    static_assert(Q % NPART == 0 && TPT % TB == 0, "tokens must split across the angle-pass parts");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -88,22 +106,23 @@ struct TcArgs {
 };
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ float bf16_bits(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
 
-// OR-reduction over the compute warpgroup that doubles as its barrier: every
-// thread gets the same answer, so control flow stays uniform on failure.
+// OR-reduction over one warpgroup that doubles as its barrier: every thread
+// gets the same answer, so control flow stays uniform on failure.
+template <uint32_t ID>
 __device__ __forceinline__ bool bar_any(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, 1, 128, q;\n\t"
+        "bar.red.or.pred p, %2, 128, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred)
+        : "r"((uint32_t)pred), "n"(ID)
         : "memory");
     return r != 0;
 }
-__device__ __forceinline__ void cbar() { named_bar(1, kCompute); }
 
 // bf16 copy of the 64 fp32 values of state row n into the 128B-swizzled
 // MN-major operand tile (row n = K index of the readout MMA).
@@ -119,26 +138,130 @@ __device__ __forceinline__ void store_state_row(uint8_t *hb, int n, const float 
     }
 }
 
+// Rotate the pair (u, v) packed in `uv` (u in the low half) by the angle whose
+// cosine is packed twice in `cc` and whose sine is packed as (-s, s) in `nss`:
+// (u c - v s, u s + v c), in packed bf16x2 arithmetic.
+__device__ __forceinline__ uint32_t rot_pair(uint32_t uv, uint32_t cc, uint32_t nss) {
+    const uint32_t vu = __byte_perm(uv, 0u, 0x1032u);  // (v, u)
+    __nv_bfloat162 t = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&vu),
+                               *reinterpret_cast<const __nv_bfloat162 *>(&nss));
+    __nv_bfloat162 o = __hfma2(*reinterpret_cast<const __nv_bfloat162 *>(&uv),
+                               *reinterpret_cast<const __nv_bfloat162 *>(&cc), t);
+    return *reinterpret_cast<uint32_t *>(&o);
+}
+
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 o = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&a),
+                               *reinterpret_cast<const __nv_bfloat162 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&o);
+}
+
+// Decay mask of S (from TMEM) into P (bf16 pairs, written back to TMEM as the
+// A operand of Yd = P X): P(t,s) = S(t,s) exp(cA_t - cA_s) (s < t ? ghat_s :
+// gam_t) for s <= t, else 0.  `row` is the thread's row (its TMEM lane), `wq`
+// its lane quarter; 32-column blocks strictly right of the quarter's diagonal
+// are all zero (warp-uniform), blocks strictly left need no causal test.
+// When the chunk's whole decay stays within 2^-100 the exponential factorises
+// into a row factor exp(cA_t - cA_0) and a column factor
+// colf_s = exp(cA_0 - cA_s) ghat_s (both in fp32 range), so each element
+// costs two multiplies; otherwise every element takes its own exp.
+template <int R, int Q>
+__device__ __forceinline__ void mask_to_tmem(int wq, int row, uint32_t tl, const float *cAl2, const float *gam,
+                                             const float *ghat, const float *colf) {
+    constexpr int NT = 16 / R;  // tokens per 16-column half block
+    const int ti = row / R;
+    const float cai = cAl2[ti], gi = gam[ti];
+    const float ca0 = cAl2[0];
+    const bool fact = (ca0 - cAl2[Q - 1]) < 100.f;  // uniform across the CTA
+    const float rowf = ex2(cai - ca0);
+#pragma unroll 1
+    for (int cb = 0; cb < 4; ++cb) {
+        uint32_t pk[16];
+        if (cb <= wq) {
+            float v[32];
+            tmem_ld32(tl + kColS + 32 * cb, v);
+            const int tb0 = (32 * cb) / R;
+            tmem_wait_ld();
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int tb = tb0 + hf * NT;
+                if (fact) {
+                    float cf[NT];
+#pragma unroll
+                    for (int k = 0; k < NT; ++k) cf[k] = colf[tb + k];
+                    if (cb < wq) {
+#pragma unroll
+                        for (int k = 0; k < 16; k += 2)
+                            pk[8 * hf + (k >> 1)] = pack_bf16(v[16 * hf + k] * cf[k / R] * rowf,
+                                                              v[16 * hf + k + 1] * cf[(k + 1) / R] * rowf);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; k += 2) {
+                            float pv[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int tj = tb + (k + u) / R;
+                                const float f = tj < ti ? cf[(k + u) / R] * rowf : (tj == ti ? gi : 0.f);
+                                pv[u] = v[16 * hf + k + u] * f;
+                            }
+                            pk[8 * hf + (k >> 1)] = pack_bf16(pv[0], pv[1]);
+                        }
+                    }
+                } else {
+                    float ca[NT], gh[NT];
+#pragma unroll
+                    for (int k = 0; k < NT; ++k) {
+                        ca[k] = cAl2[tb + k];
+                        gh[k] = ghat[tb + k];
+                    }
+#pragma unroll
+                    for (int k = 0; k < 16; k += 2) {
+                        float pv[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int tj = tb + (k + u) / R;
+                            const float coef = tj < ti ? gh[(k + u) / R] : (tj == ti ? gi : 0.f);
+                            pv[u] = v[16 * hf + k + u] * ex2(fminf(cai - ca[(k + u) / R], 0.f)) * coef;
+                        }
+                        pk[8 * hf + (k >> 1)] = pack_bf16(pv[0], pv[1]);
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        }
+        tmem_st16(tl + kColP + 16 * cb, pk);
+    }
+    tmem_wait_st();
+}
+
+struct Bars {
+    uint64_t *full_bc, *empty_bc, *full_x, *empty_x, *ops, *sg, *hrdy, *p, *yd, *drain, *sc;
+};
+
 template <int N, int R>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmC, const TcArgs a) {
+                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmT,
+                  const TcArgs a) {
     using C = Cfg<N, R>;
-    constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, TPP = C::TPP, TPT = C::TPT;
+    constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, G4 = C::G4, NPART = C::NPART, TPT = C::TPT, TB = C::TB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *cAl2 = reinterpret_cast<float *>(smem + C::OFF_SCAL);  // chunk-local cumsum of dt*A, log2 units
-    float *gam = cAl2 + Q;      // lam dt           (diagonal weight)
-    float *ghat = gam + Q;      // lam dt + (1-lam') dt'  (off-diagonal weight)
-    float *wst = ghat + Q;      // exp(cA_end - cA_s) * ghat_s  (chunk-state weight)
-    float *dts = wst + Q;       // dt
-    float *cosE = dts + Q;      // cos/sin of the chunk's total angle per pair
-    float *sinE = cosE + K2;
-    float *phis = sinE + K2;    // partial angle sums [TPP][K2]
-    float *wtot = phis + TPP * K2;  // per-warp totals of the dt*A scan
+    float *scal = reinterpret_cast<float *>(smem + C::OFF_SCAL);
+    // kNX per-chunk buffers (index c % kNX) of cAl2 (chunk-local cumsum of
+    // dt*A, log2 units), gam = lam dt (diagonal weight), ghat = lam dt +
+    // (1-lam') dt' (off-diagonal weight), colf (column factor of the mask) and
+    // cos/sin of each pair's total angle over the chunk
+    float *sbuf = scal;
+    float *wst = scal + kNX * C::SB;  // exp(cA_end - cA_s) ghat_s (chunk-state weight)
+    float *dts = wst + Q;             // dt
+    float *phis = dts + Q;            // partial angle sums [NPART][K2]
+    float *wtot = phis + NPART * K2;  // per-warp totals of the dt*A scan; [4] = cA of token 0
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *full = bars, *empty = bars + 2, *ops_ready = bars + 4, *sgo_done = bars + 5, *p_ready = bars + 6,
-             *yd_done = bars + 7, *drain = bars + 8;
+    Bars bb{bars, bars + 2, bars + 4, bars + 7, bars + 10, bars + 11, bars + 12, bars + 13, bars + 14, bars + 15,
+            bars + 16};
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     unsigned *err = &g_device_error;
@@ -150,15 +273,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     auto tok = [&](int64_t t) { return (b * T + t) * H + h; };
 
     if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init(&empty[0], 1);
-        mbar_init(&empty[1], 1);
-        mbar_init(ops_ready, 1);
-        mbar_init(sgo_done, 1);
-        mbar_init(p_ready, 1);
-        mbar_init(yd_done, 1);
-        mbar_init(drain, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bb.full_bc[i], 1);
+            mbar_init(&bb.empty_bc[i], 1);
+        }
+        for (int i = 0; i < kNX; ++i) {
+            mbar_init(&bb.full_x[i], 1);
+            mbar_init(&bb.empty_x[i], 1);
+            mbar_init(&bb.sc[i], 1);  // per-chunk scalars published to the state warpgroup
+        }
+        mbar_init(bb.ops, 1);
+        mbar_init(bb.sg, 1);
+        mbar_init(bb.hrdy, 1);
+        mbar_init(bb.p, 1);
+        mbar_init(bb.yd, 1);
+        mbar_init(bb.drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -170,6 +299,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmC);
+        prefetch_tmap(&tmT);
     }
     tc_fence_before();
     __syncthreads();
@@ -178,95 +308,337 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int nchunks = a.nchunks;
 
     if (warp == kWarpTma) {
-        // ------------------------------------------------------------ TMA producer
+        // ============================================================ TMA producers
         if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !mbar_wait(&empty[s], ((c >> 1) - 1) & 1, abort_flag, err, kErrWaitCompute)) break;
-                uint8_t *st = smem + s * C::STAGE_BYTES;
+            // B/C ring (2 stages), plus L2 prefetches of everything a chunk needs
+            auto prefetch_chunk = [&](int c) {
                 const int t0 = c * Q;
-                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                tma_load_5d(st, &tmX, &full[s], 0, 0, (int)h, t0, (int)b);
+                tma_prefetch_5d(&tmX, 0, 0, (int)h, t0, (int)b);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_5d(st + C::X_BYTES + kb * 16384, &tmB, &full[s], kb * 64, 0, (int)h, t0, (int)b);
-                    tma_load_5d(st + C::X_BYTES + C::BC_BYTES + kb * 16384, &tmC, &full[s], kb * 64, 0, (int)h, t0,
-                                (int)b);
+                    tma_prefetch_5d(&tmB, kb * 64, 0, (int)h, t0, (int)b);
+                    tma_prefetch_5d(&tmC, kb * 64, 0, (int)h, t0, (int)b);
+                }
+                tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // theta is read straight into registers
+            };
+            int issued = 0;
+            for (int c = 0; c < kPrefetchAhead && c < nchunks; ++c) prefetch_chunk(c);
+            for (int c = 0; c < nchunks; ++c) {
+                if (c + kPrefetchAhead < nchunks) prefetch_chunk(c + kPrefetchAhead);
+                const int s = c & 1;
+                if (c >= 2 && !mbar_wait(&bb.empty_bc[s], ((c >> 1) - 1) & 1, abort_flag, err, kErrWaitMma)) break;
+                uint8_t *st = smem + C::OFF_BC + s * C::BCS_BYTES;
+                const int t0 = c * Q;
+                mbar_arrive_expect_tx(&bb.full_bc[s], C::BCS_BYTES);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_5d(st + kb * 16384, &tmB, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
+                    tma_load_5d(st + C::BC_BYTES + kb * 16384, &tmC, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
                 }
                 issued = c + 1;
             }
             if (*abort_flag) {  // let the copies already in flight land before the CTA exits
                 for (int c = issued - 2 > 0 ? issued - 2 : 0; c < issued; ++c)
-                    mbar_wait(&full[c & 1], (c >> 1) & 1, nullptr, err, 0, 400000000LL);
+                    mbar_wait(&bb.full_bc[c & 1], (c >> 1) & 1, nullptr, err, 0, 400000000LL);
+            }
+        } else if (lane == 1) {
+            // x ring (kNX stages), freed by the epilogue
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % kNX;
+                if (c >= kNX && !mbar_wait(&bb.empty_x[s], ((c / kNX) - 1) & 1, abort_flag, err, kErrWaitCompute))
+                    break;
+                mbar_arrive_expect_tx(&bb.full_x[s], C::X_BYTES);
+                tma_load_5d(smem + C::OFF_X + s * C::X_BYTES, &tmX, &bb.full_x[s], 0, 0, (int)h, c * Q, (int)b);
+                issued = c + 1;
+            }
+            if (*abort_flag) {
+                for (int c = issued - kNX > 0 ? issued - kNX : 0; c < issued; ++c)
+                    mbar_wait(&bb.full_x[c % kNX], (c / kNX) & 1, nullptr, err, 0, 400000000LL);
             }
         }
     } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
+        // ============================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idG = idesc_bf16(N, 64, 1, 1);
             constexpr uint32_t idY = idesc_bf16(128, 64, 0, 1);
-            const uint32_t xw = smem_u32(smem + C::OFF_XW);
-            const uint32_t hb = smem_u32(smem + C::OFF_HB);
+            // Operand descriptors per tile; an offset inside a tile is added to the
+            // 14-bit start-address field (address >> 4), which cannot carry because
+            // shared-memory addresses stay below 256 KB.
+            const uint64_t dXw = sdesc_sw128(smem_u32(smem + C::OFF_XW), 16384, 1024);
+            const uint64_t dHb = sdesc_sw128(smem_u32(smem + C::OFF_HB), 16384, 1024);
+            const uint32_t bc0 = smem_u32(smem + C::OFF_BC);
+            const uint32_t x0 = smem_u32(smem + C::OFF_X);
             bool any = false;
             for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1;
-                const uint32_t xs = smem_u32(smem + s * C::STAGE_BYTES);
-                const uint32_t bs = xs + C::X_BYTES;
+                const int s = c & 1, sx = c % kNX;
+                const uint32_t bs = bc0 + (uint32_t)s * C::BCS_BYTES;
                 const uint32_t cs = bs + C::BC_BYTES;
-                const uint32_t pb = C::P_IN_C ? cs : smem_u32(smem + C::OFF_P);
-                if (!mbar_wait(ops_ready, c & 1, abort_flag, err, kErrWaitCompute)) break;
+                const uint64_t dX = sdesc_sw128(x0 + (uint32_t)sx * C::X_BYTES, 16384, 1024);  // X, MN-major
+                const uint64_t dBk = sdesc_sw128(bs, 16, 1024);     // B~, K-major
+                const uint64_t dBm = sdesc_sw128(bs, 16384, 1024);  // B~^T, MN-major
+                const uint64_t dCk = sdesc_sw128(cs, 16, 1024);     // C~, K-major
+                // S(c) as soon as the rotated tiles and w o X are in place
+                if (!mbar_wait(bb.ops, c & 1, abort_flag, err, kErrWaitCompute)) break;
                 tc_fence_after();
                 any = true;
-                // S = C~ B~^T  (both K-major over the state dim)
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tbase + kColS, sdesc_sw128(cs + kb * 16384 + kk * 32, 16, 1024),
-                                 sdesc_sw128(bs + kb * 16384 + kk * 32, 16, 1024), idS, (kb | kk) != 0);
-                // G = B~^T (w o X)  (both MN-major, K = the chunk's 128 rows)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(tbase + kColG, sdesc_sw128(bs + ks * 2048, 16384, 1024),
-                             sdesc_sw128(xw + ks * 2048, 16384, 1024), idG, ks != 0);
-                // Yo = C~ h*  (C~ K-major; h* MN-major, K = state rows)
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tbase + kColYo, sdesc_sw128(cs + kb * 16384 + kk * 32, 16, 1024),
-                                 sdesc_sw128(hb + (kb * 4 + kk) * 2048, 16384, 1024), idY, (kb | kk) != 0);
-                mma_commit(sgo_done);
-                if (!mbar_wait(p_ready, c & 1, abort_flag, err, kErrWaitCompute)) break;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t o = (uint64_t)((kb * 16384 + kk * 32) >> 4);
+                        mma_bf16(tbase + kColS, dCk + o, dBk + o, idS, (kb | kk) != 0);
+                    }
+                // G(c) and Yo(c) once the state warpgroup has consumed G(c-1) and
+                // published h*_{c-1} (completion c of hrdy; the first is the initial state)
+                if (!mbar_wait(bb.hrdy, c & 1, abort_flag, err, kErrWaitCompute)) break;
                 tc_fence_after();
-                // Yd = P X  (P K-major over the chunk's rows; X MN-major)
 #pragma unroll
-                for (int kb = 0; kb < 2; ++kb)
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t o = (uint64_t)((ks * 2048) >> 4);
+                    mma_bf16(tbase + kColG, dBm + o, dXw + o, idG, ks != 0);
+                }
+                const uint32_t yo = tbase + kColYo + (uint32_t)(c & 1) * 64u;
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tbase + kColYd, sdesc_sw128(pb + kb * 16384 + kk * 32, 16, 1024),
-                                 sdesc_sw128(xs + (kb * 4 + kk) * 2048, 16384, 1024), idY, (kb | kk) != 0);
-                mma_commit(yd_done);
+                        mma_bf16(yo, dCk + (uint64_t)((kb * 16384 + kk * 32) >> 4),
+                                 dHb + (uint64_t)(((kb * 4 + kk) * 2048) >> 4), idY, (kb | kk) != 0);
+                mma_commit(bb.sg);
+                mma_commit(&bb.empty_bc[s]);  // the B/C stage is free once these MMAs are done
+                // Yd(c) = P X once P is in TMEM and the epilogue of c-1 has read Yd
+                if (!mbar_wait(bb.p, c & 1, abort_flag, err, kErrWaitCompute)) break;
+                if (c >= 1 && !mbar_wait(&bb.empty_x[(c - 1) % kNX], ((c - 1) / kNX) & 1, abort_flag, err,
+                                         kErrWaitCompute))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tbase + kColYd, tbase + kColP + (uint32_t)kk * 8u,
+                                dX + (uint64_t)((kk * 2048) >> 4), idY, kk != 0);
+                mma_commit(bb.yd);
             }
             if (*abort_flag && any) {  // no MMA may still run when TMEM is released
-                mma_commit(drain);
-                mbar_wait(drain, 0, nullptr, err, 0, 400000000LL);
+                mma_commit(bb.drain);
+                mbar_wait(bb.drain, 0, nullptr, err, 0, 400000000LL);
+            }
+        }
+    } else if (warp < 4) {
+        // ============================================================ prologue warpgroup
+        const float Ah2 = a.A[h] * kLog2e;
+        uint8_t *xw = smem + C::OFF_XW;
+        const unsigned short *dtr = reinterpret_cast<const unsigned short *>(a.dt);
+        const unsigned short *lmr = reinterpret_cast<const unsigned short *>(a.lam);
+        const int g = tid % G4, part = tid / G4;  // angle pass: 4 pairs x TPT tokens per thread
+        // raw bf16 bits of dt, lam for this thread's token and the one after it,
+        // loaded one chunk ahead and converted only when used
+        unsigned short pd = 0, pl = 0, pd1 = 0, pl1 = 0;
+        auto prefetch_scalars = [&](int64_t t0s) {
+            const int64_t t = t0s + tid;
+            pd = pl = pd1 = pl1 = 0;
+            if (tid < Q && t < T) {
+                pd = __ldg(dtr + tok(t));
+                pl = __ldg(lmr + tok(t));
+                if (t + 1 < T) {
+                    pd1 = __ldg(dtr + tok(t + 1));
+                    pl1 = __ldg(lmr + tok(t + 1));
+                }
+            }
+        };
+        // theta of this thread's 4 pairs for its TPT tokens, read straight from
+        // global memory into registers one chunk ahead of use
+        uint2 thr[TPT];
+        auto prefetch_theta = [&](int64_t t0s) {
+#pragma unroll
+            for (int j = 0; j < TPT; ++j) {
+                const int64_t t = t0s + part * TPT + j;
+                thr[j] = t < T ? __ldg(reinterpret_cast<const uint2 *>(a.theta + tok(t) * K2 + 4 * g))
+                               : make_uint2(0u, 0u);
+            }
+        };
+        prefetch_scalars(0);
+        prefetch_theta(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1, sx = c % kNX;
+            float *cAl2 = sbuf + sx * C::SB;
+            float *gam = cAl2 + Q;
+            float *ghat = gam + Q;
+            float *colf = ghat + Q;
+            float *cosE = colf + Q;
+            float *sinE = cosE + K2;
+            uint8_t *bst = smem + C::OFF_BC + s * C::BCS_BYTES;
+            uint8_t *cst = bst + C::BC_BYTES;
+            uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
+            // the scalar buffer c % kNX is free once the epilogue of c - kNX is done
+            if (c >= kNX && bar_any<kBarPro>(!mbar_wait(&bb.empty_x[sx], ((c / kNX) - 1) & 1, abort_flag, err,
+                                                        kErrWaitCompute)))
+                break;
+
+            // ---- A. per-token scalars and the chunk-local scan of dt*A
+            float acc = 0.f;
+            {
+                const float d = bf16_bits(pd), l = bf16_bits(pl);
+                const float nx = (1.f - bf16_bits(pl1)) * bf16_bits(pd1);  // 0 past the sequence end
+                if (c + 1 < nchunks) prefetch_scalars((int64_t)(c + 1) * Q);
+                if (tid < Q) {
+                    dts[tid] = d;
+                    gam[tid] = l * d;
+                    ghat[tid] = l * d + nx;
+                    acc = d * Ah2;
+                    if (tid == 0) wtot[4] = acc;  // cA of the chunk's first token
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float v = __shfl_up_sync(0xffffffffu, acc, off);
+                        if (lane >= off) acc += v;
+                    }
+                    if (lane == 31) wtot[warp] = acc;
+                }
+            }
+            named_bar(kBarPro, kWG);
+            if (tid < Q) {
+                float off = 0.f, tot = 0.f;
+#pragma unroll
+                for (int w = 0; w < Q / 32; ++w) {
+                    const float v = wtot[w];
+                    if (w < warp) off += v;
+                    tot += v;
+                }
+                const float ca = acc + off;
+                cAl2[tid] = ca;
+                wst[tid] = ex2(tot - ca) * ghat[tid];
+                // column factor of the decay mask, relative to the chunk's first token
+                colf[tid] = ex2(wtot[4] - ca) * ghat[tid];
+            }
+
+            // ---- B. cumulative angles of 4 pairs per thread, in-place rotation
+            //      of B and C
+            {
+                float loc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < TPT; ++j) {
+                    const float di = dts[part * TPT + j];
+                    const float2 t01 = unpack_bf16(thr[j].x), t23 = unpack_bf16(thr[j].y);
+                    loc[0] = fmaf(di, t01.x, loc[0]);
+                    loc[1] = fmaf(di, t01.y, loc[1]);
+                    loc[2] = fmaf(di, t23.x, loc[2]);
+                    loc[3] = fmaf(di, t23.y, loc[3]);
+                }
+                *reinterpret_cast<float4 *>(phis + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
+                // the B/C tiles of this chunk
+                if (bar_any<kBarPro>(!mbar_wait(&bb.full_bc[s], (c >> 1) & 1, abort_flag, err, kErrWaitTma))) break;
+                float phi[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int q = 0; q < part; ++q) {
+                    const float4 v = *reinterpret_cast<const float4 *>(phis + q * K2 + 4 * g);
+                    phi[0] += v.x;
+                    phi[1] += v.y;
+                    phi[2] += v.z;
+                    phi[3] += v.w;
+                }
+                const uint32_t kbo = (uint32_t)(g >> 3) * 16384u;
+                const uint32_t jchunk = (uint32_t)(g & 7);
+#pragma unroll
+                for (int j0 = 0; j0 < TPT; j0 += TB) {
+                    // all loads of the batch first (the stores below go to the same
+                    // tiles, so the compiler could not hoist them itself)
+                    uint4 vb[TB][R], vc[TB][R];
+#pragma unroll
+                    for (int jj = 0; jj < TB; ++jj) {
+                        const int i = part * TPT + j0 + jj;
+#pragma unroll
+                        for (int r = 0; r < R; ++r) {
+                            const uint32_t off = kbo + sw128((uint32_t)(i * R + r), jchunk);
+                            vb[jj][r] = *reinterpret_cast<const uint4 *>(bst + off);
+                            vc[jj][r] = *reinterpret_cast<const uint4 *>(cst + off);
+                        }
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < TB; ++jj) {
+                        const int i = part * TPT + j0 + jj;
+                        const float di = dts[i];
+                        const float2 t01 = unpack_bf16(thr[j0 + jj].x), t23 = unpack_bf16(thr[j0 + jj].y);
+                        phi[0] = fmaf(di, t01.x, phi[0]);
+                        phi[1] = fmaf(di, t01.y, phi[1]);
+                        phi[2] = fmaf(di, t23.x, phi[2]);
+                        phi[3] = fmaf(di, t23.y, phi[3]);
+                        uint32_t cc[4], nss[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float sn, cs;
+                            __sincosf(phi[e], &sn, &cs);
+                            cc[e] = pack_bf16(cs, cs);
+                            nss[e] = pack_bf16(-sn, sn);
+                        }
+#pragma unroll
+                        for (int r = 0; r < R; ++r) {
+                            const uint32_t off = kbo + sw128((uint32_t)(i * R + r), jchunk);
+                            uint4 b4 = vb[jj][r], c4 = vc[jj][r];
+                            b4.x = rot_pair(b4.x, cc[0], nss[0]);
+                            b4.y = rot_pair(b4.y, cc[1], nss[1]);
+                            b4.z = rot_pair(b4.z, cc[2], nss[2]);
+                            b4.w = rot_pair(b4.w, cc[3], nss[3]);
+                            c4.x = rot_pair(c4.x, cc[0], nss[0]);
+                            c4.y = rot_pair(c4.y, cc[1], nss[1]);
+                            c4.z = rot_pair(c4.z, cc[2], nss[2]);
+                            c4.w = rot_pair(c4.w, cc[3], nss[3]);
+                            *reinterpret_cast<uint4 *>(bst + off) = b4;
+                            *reinterpret_cast<uint4 *>(cst + off) = c4;
+                        }
+                    }
+                }
+                if (part == NPART - 1) {  // phi now holds each pair's total angle over the chunk
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float sn, cs;
+                        __sincosf(phi[e], &sn, &cs);
+                        cosE[4 * g + e] = cs;
+                        sinE[4 * g + e] = sn;
+                    }
+                }
+                if (c + 1 < nchunks) prefetch_theta((int64_t)(c + 1) * Q);
+            }
+            // ---- C. w o X (chunk-state weights on the value rows), once G(c-1)
+            //      has finished reading the previous w o X and x of chunk c is in
+            if (bar_any<kBarPro>((c >= 1 && !mbar_wait(bb.sg, (c - 1) & 1, abort_flag, err, kErrWaitMma)) ||
+                                 !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma)))
+                break;
+            {
+                const int row = tid;
+                const float wv = wst[row / R];
+                const uint32_t ww = pack_bf16(wv, wv);
+                uint4 v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4 *>(xst + sw128(row, j));
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    v[j].x = mul_bf16x2(v[j].x, ww);
+                    v[j].y = mul_bf16x2(v[j].y, ww);
+                    v[j].z = mul_bf16x2(v[j].z, ww);
+                    v[j].w = mul_bf16x2(v[j].w, ww);
+                    *reinterpret_cast<uint4 *>(xw + sw128(row, j)) = v[j];
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar(kBarPro, kWG);
+            if (tid == 0) {
+                mbar_arrive(bb.ops);
+                mbar_arrive(&bb.sc[sx]);
             }
         }
     } else {
-        // ------------------------------------------------------------ compute warpgroup
+        // ============================================================ state warpgroup
+        const int lt = tid - kWG;          // 0..127
+        const int wq = warp & 3;           // TMEM lane quarter
         const bool own_state = (N == 128) || (lane < 16);
-        const int srow = (N == 128) ? tid : (warp * 16 + lane);  // TMEM lane layout of G
+        const int srow = (N == 128) ? lt : (wq * 16 + lane);  // TMEM lane layout of G (M = N)
         uint8_t *hbuf = smem + C::OFF_HB;
-        const float Ah2 = a.A[h] * kLog2e;
         const float Dh = a.D[h];
+        const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
         float hreg[64];
         // initial state h0 + beta'_0 b_prev x_prev^T (pending write of token -1)
         {
-            float betap0 = 0.f;
-            if (T > 0) betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
+            const float betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
 #pragma unroll
             for (int p = 0; p < 64; ++p) hreg[p] = 0.f;
             if (own_state) {
@@ -284,215 +656,72 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 store_state_row(hbuf, srow, hreg);
             }
         }
+        fence_proxy_async_smem();
+        named_bar(kBarState, kWG);
+        if (lt == 0) mbar_arrive(bb.hrdy);
         bool ok = true;
-        for (int c = 0; c < nchunks && ok; ++c) {
-            const int s = c & 1;
-            const int64_t t0 = (int64_t)c * Q;
-            uint8_t *st = smem + s * C::STAGE_BYTES;
-            uint8_t *xst = st;
-            uint8_t *bst = st + C::X_BYTES;
-            uint8_t *cst = bst + C::BC_BYTES;
-            uint8_t *pbuf = C::P_IN_C ? cst : smem + C::OFF_P;
-
-            // ---- A. per-token scalars and the chunk-local scan of dt*A
-            float acc = 0.f;
-            if (tid < Q) {
-                const int64_t t = t0 + tid;
-                float d = 0.f, l = 0.f, nx = 0.f;
-                if (t < T) {
-                    d = bf(a.dt, tok(t));
-                    l = bf(a.lam, tok(t));
-                }
-                if (t + 1 < T) nx = (1.f - bf(a.lam, tok(t + 1))) * bf(a.dt, tok(t + 1));
-                dts[tid] = d;
-                gam[tid] = l * d;
-                ghat[tid] = l * d + nx;
-                acc = d * Ah2;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, acc, off);
-                    if (lane >= off) acc += v;
-                }
-                if (lane == 31 || tid == Q - 1) wtot[warp] = acc;
+        for (int c = 0; c < nchunks; ++c) {
+            const int sx = c % kNX;
+            const float *cAl2 = sbuf + sx * C::SB;
+            const float *gam = cAl2 + Q;
+            const float *ghat = gam + Q;
+            const float *colf = ghat + Q;
+            const float *cosE = colf + Q;
+            const float *sinE = cosE + K2;
+            const uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
+            // scalars of chunk c (release/acquire through sc), its x tile, and G(c)
+            if (bar_any<kBarState>(!mbar_wait(&bb.sc[sx], (c / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
+                                   !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma) ||
+                                   !mbar_wait(bb.sg, c & 1, abort_flag, err, kErrWaitMma))) {
+                ok = false;
+                break;
             }
-            cbar();
-            if (tid < Q) {
-                float off = 0.f, tot = 0.f;
-#pragma unroll
-                for (int w = 0; w < (Q + 31) / 32; ++w) {
-                    const float v = wtot[w];
-                    if (w < warp) off += v;
-                    tot += v;
-                }
-                const float ca = acc + off;
-                cAl2[tid] = ca;
-                wst[tid] = ex2(tot - ca) * ghat[tid];
-            }
-            // ---- wait for this chunk's tiles
-            ok = !bar_any(!mbar_wait(&full[s], (c >> 1) & 1, abort_flag, err, kErrWaitTma));
-            if (!ok) break;
-
-            // ---- B. cumulative angles per pair and in-place rotation of B and C
-            {
-                const int k = tid % K2, part = tid / K2;
-                const int64_t thb = (int64_t)k;
-                float loc = 0.f;
-#pragma unroll 4
-                for (int j = 0; j < TPT; ++j) {
-                    const int i = part * TPT + j;
-                    const int64_t t = t0 + i;
-                    const float th = t < T ? bf(a.theta, tok(t) * K2 + thb) : 0.f;
-                    loc = fmaf(dts[i], th, loc);
-                }
-                phis[part * K2 + k] = loc;
-                cbar();
-                float phi = 0.f;
-                for (int q = 0; q < part; ++q) phi += phis[q * K2 + k];
-                const uint32_t cofs = (uint32_t)(k >> 5) * 16384u;       // 64-wide K block
-                const uint32_t chunkj = (uint32_t)((k & 31) >> 2);        // 16-byte chunk in the row
-                const uint32_t within = (uint32_t)(k & 3) * 4u;           // byte offset of the pair
-#pragma unroll 2
-                for (int j = 0; j < TPT; ++j) {
-                    const int i = part * TPT + j;
-                    const int64_t t = t0 + i;
-                    const float th = t < T ? bf(a.theta, tok(t) * K2 + thb) : 0.f;
-                    phi = fmaf(dts[i], th, phi);
-                    float sn, cs;
-                    sincos_reduced(phi, &sn, &cs);
-#pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        const uint32_t row = (uint32_t)(i * R + r);
-                        const uint32_t off = cofs + sw128(row, chunkj) + within;
-                        uint32_t *pb = reinterpret_cast<uint32_t *>(bst + off);
-                        uint32_t *pc = reinterpret_cast<uint32_t *>(cst + off);
-                        const float2 vb = unpack_bf16(*pb);
-                        const float2 vc = unpack_bf16(*pc);
-                        *pb = pack_bf16(vb.x * cs - vb.y * sn, vb.x * sn + vb.y * cs);
-                        *pc = pack_bf16(vc.x * cs - vc.y * sn, vc.x * sn + vc.y * cs);
-                    }
-                }
-                if (part == TPP - 1) {
-                    float sn, cs;
-                    sincos_reduced(phi, &sn, &cs);
-                    cosE[k] = cs;
-                    sinE[k] = sn;
-                }
-            }
-            // ---- C. w o X (chunk-state weights on the value rows)
-            {
-                const int row = tid;
-                const float wv = wst[row / R];
-                uint8_t *xw = smem + C::OFF_XW;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t off = sw128(row, j);
-                    uint4 v = *reinterpret_cast<const uint4 *>(xst + off);
-                    float2 f;
-                    f = unpack_bf16(v.x); v.x = pack_bf16(f.x * wv, f.y * wv);
-                    f = unpack_bf16(v.y); v.y = pack_bf16(f.x * wv, f.y * wv);
-                    f = unpack_bf16(v.z); v.z = pack_bf16(f.x * wv, f.y * wv);
-                    f = unpack_bf16(v.w); v.w = pack_bf16(f.x * wv, f.y * wv);
-                    *reinterpret_cast<uint4 *>(xw + off) = v;
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            cbar();
-            if (tid == 0) mbar_arrive(ops_ready);
-
-            // ---- D. decay mask: P = S o L, L(t,s) = exp(cA_t - cA_s) * (s < t ? ghat_s : gam_t), s <= t
-            ok = !bar_any(!mbar_wait(sgo_done, c & 1, abort_flag, err, kErrWaitMma));
-            if (!ok) break;
             tc_fence_after();
-            {
-                const int row = tid;
-                const int ti = row / R;
-                const float cai = cAl2[ti], gi = gam[ti];
-                const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
-                    uint8_t *dst = pbuf + (cb >> 1) * 16384;
-                    if (cb <= warp) {  // warp-uniform: blocks right of the diagonal are all zero
-                        float v[32];
-                        tmem_ld32(tl + kColS + 32 * cb, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                float pv[2];
-#pragma unroll
-                                for (int u = 0; u < 2; ++u) {
-                                    const int jcol = 32 * cb + 8 * q + e + u;
-                                    const int tj = jcol / R;
-                                    float val = 0.f;
-                                    if (tj < ti) val = v[8 * q + e + u] * ex2(cai - cAl2[tj]) * ghat[tj];
-                                    else if (tj == ti) val = v[8 * q + e + u] * gi;
-                                    pv[u] = val;
-                                }
-                                pk[e >> 1] = pack_bf16(pv[0], pv[1]);
-                            }
-                            const uint32_t jj = (uint32_t)((cb & 1) * 4 + q);
-                            *reinterpret_cast<uint4 *>(dst + sw128(row, jj)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t jj = (uint32_t)((cb & 1) * 4 + q);
-                            *reinterpret_cast<uint4 *>(dst + sw128(row, jj)) = make_uint4(0u, 0u, 0u, 0u);
-                        }
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            cbar();
-            if (tid == 0) mbar_arrive(p_ready);
-
             // ---- E. carried state: h* <- Rot(-Phi)(exp(cA_end) h* + G), fp32 in registers
             {
-                const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
-                float g[64];
-                {
-                    float g0[32], g1[32];
-                    tmem_ld32(tl + kColG, g0);
-                    tmem_ld32(tl + kColG + 32, g1);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int p = 0; p < 32; ++p) {
-                        g[p] = g0[p];
-                        g[32 + p] = g1[p];
-                    }
-                }
                 const float eA = ex2(cAl2[Q - 1]);
                 const int kp = (own_state ? srow : 0) >> 1;
                 const float cs = cosE[kp], sn = sinE[kp];
                 const float sgn = (srow & 1) ? -sn : sn;
 #pragma unroll
-                for (int p = 0; p < 64; ++p) {
-                    const float u = fmaf(eA, hreg[p], g[p]);
-                    const float o = __shfl_xor_sync(0xffffffffu, u, 1);
-                    hreg[p] = fmaf(u, cs, o * sgn);
+                for (int half = 0; half < 2; ++half) {
+                    float gv[32];
+                    tmem_ld32(tl + kColG + 32 * half, gv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int p = 0; p < 32; ++p) {
+                        const float u = fmaf(eA, hreg[32 * half + p], gv[p]);
+                        const float o = __shfl_xor_sync(0xffffffffu, u, 1);
+                        hreg[32 * half + p] = fmaf(u, cs, o * sgn);
+                    }
                 }
                 if (own_state) store_state_row(hbuf, srow, hreg);
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(kBarState, kWG);
+            if (lt == 0) mbar_arrive(bb.hrdy);
+
+            // ---- D. decay mask S -> P (TMEM)
+            mask_to_tmem<R, Q>(wq, lt, tl, cAl2, gam, ghat, colf);
+            tc_fence_before();
+            named_bar(kBarState, kWG);
+            if (lt == 0) mbar_arrive(bb.p);
 
             // ---- F. epilogue: y = Yd + exp(cA_t) Yo + D x
-            ok = !bar_any(!mbar_wait(yd_done, c & 1, abort_flag, err, kErrWaitMma));
-            if (!ok) break;
+            if (bar_any<kBarState>(!mbar_wait(bb.yd, c & 1, abort_flag, err, kErrWaitMma))) { ok = false; break; }
             tc_fence_after();
             {
-                const int row = tid;
+                const int row = lt;
                 const int ti = row / R, r = row % R;
-                const int64_t t = t0 + ti;
+                const int64_t t = (int64_t)c * Q + ti;
                 const float sc = ex2(cAl2[ti]);
-                const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
-#pragma unroll
+                const uint32_t yo = kColYo + (uint32_t)(c & 1) * 64u;
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
-                    float yd[32], yo[32];
+                    float yd[32], yv[32];
                     tmem_ld32(tl + kColYd + 32 * half, yd);
-                    tmem_ld32(tl + kColYo + 32 * half, yo);
+                    tmem_ld32(tl + yo + 32 * half, yv);
                     tmem_wait_ld();
                     if (t < T) {
                         __nv_bfloat16 *yrow = a.y + (tok(t) * R + r) * kP + 32 * half;
@@ -505,8 +734,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                             for (int e = 0; e < 4; ++e) {
                                 const float2 xf = unpack_bf16(xs[e]);
                                 const int p = 8 * q + 2 * e;
-                                const float y0 = fmaf(Dh, xf.x, fmaf(sc, yo[p], yd[p]));
-                                const float y1 = fmaf(Dh, xf.y, fmaf(sc, yo[p + 1], yd[p + 1]));
+                                const float y0 = fmaf(Dh, xf.x, fmaf(sc, yv[p], yd[p]));
+                                const float y1 = fmaf(Dh, xf.y, fmaf(sc, yv[p + 1], yd[p + 1]));
                                 o[e] = pack_bf16(y0, y1);
                             }
                             *reinterpret_cast<uint4 *>(yrow + 8 * q) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -515,8 +744,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
             }
             tc_fence_before();
-            cbar();
-            if (tid == 0) mbar_arrive(&empty[s]);
+            named_bar(kBarState, kWG);
+            if (lt == 0) mbar_arrive(&bb.empty_x[sx]);
         }
         // ---- final state: plain-frame h_{T-1}, raw last token as the pending term
         if (ok) {
@@ -527,11 +756,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
             }
             if (a.bpT)
-                for (int i = tid; i < R * N; i += kCompute)
-                    a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
+                for (int i = lt; i < R * N; i += kWG) a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
             if (a.xpT)
-                for (int i = tid; i < R * kP; i += kCompute)
-                    a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
+                for (int i = lt; i < R * kP; i += kWG) a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
         }
     }
 
@@ -577,12 +804,25 @@ bool make_map(CUtensorMap *m, const void *base, int64_t inner, int64_t R, int64_
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// theta [Bt, T, H, N/2] bf16, box = {N/2, 1 head, Q tokens, 1 batch}, no swizzle.
+bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int64_t T, int64_t Bt, int Q) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)K2, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)Bt};
+    const cuuint64_t strides[3] = {(cuuint64_t)(K2 * 2), (cuuint64_t)(H * K2 * 2), (cuuint64_t)(T * H * K2 * 2)};
+    const cuuint32_t box[4] = {(cuuint32_t)K2, 1, (cuuint32_t)Q, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int N, int R>
 cudaError_t launch_nr(const Problem &p, const char **why) {
     using C = Cfg<N, R>;
-    CUtensorMap mx, mb, mc;
+    CUtensorMap mx, mb, mc, mt;
     if (!make_map(&mx, p.x, kP, R, p.H, p.T, p.Bt, C::Q) || !make_map(&mb, p.B, N, R, p.H, p.T, p.Bt, C::Q) ||
-        !make_map(&mc, p.C, N, R, p.H, p.T, p.Bt, C::Q)) {
+        !make_map(&mc, p.C, N, R, p.H, p.T, p.Bt, C::Q) || !make_theta_map(&mt, p.theta, N / 2, p.H, p.T, p.Bt, C::Q)) {
         *why = "tensor-core prefill: TMA descriptor encoding failed";
         return cudaErrorNotSupported;
     }
@@ -607,7 +847,7 @@ cudaError_t launch_nr(const Problem &p, const char **why) {
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<N, R><<<(unsigned)(p.Bt * p.H), kThreads, C::SMEM_BYTES, p.stream>>>(mx, mb, mc, a);
+    prefill_tc_kernel<N, R><<<(unsigned)(p.Bt * p.H), kThreads, C::SMEM_BYTES, p.stream>>>(mx, mb, mc, mt, a);
     return cudaGetLastError();
 }
 
