@@ -48,7 +48,41 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--case", choices=["prefill", "decode"], default=None,
+                    help="profiling case: only run --case-launches launches of one kernel at --case-batch "
+                         "(for ncu captures; prints no bench line)")
+    ap.add_argument("--case-batch", type=int, default=None)
+    ap.add_argument("--case-launches", type=int, default=3)
     return ap.parse_args()
+
+
+def run_case(args):
+    """Small fixed case for ncu captures: the workload's shape at a reduced
+    batch, a few launches of the one kernel, no timing."""
+    import torch
+
+    import state_space_sequence_ssm_b200 as m3
+    from m3_inputs import WORKLOADS, make_prefill, make_state, make_steps
+
+    keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
+    if args.case == "prefill":
+        s = WORKLOADS[args.workload]
+        s = s.with_(batch=args.case_batch or s.batch)
+        inp = make_prefill(s, device="cuda")
+        for _ in range(args.case_launches):
+            m3.scan_fwd(*(inp[k] for k in keys), None)
+    else:
+        name = args.workload if args.workload.startswith("decode") else DECODE_WORKLOADS[0]
+        s = WORKLOADS[name]
+        s = s.with_(batch=args.case_batch or s.batch)
+        st = m3.State(*(t.cuda() for t in make_state(s)))
+        steps = make_steps(s, args.case_launches, device="cuda")
+        pre = make_prefill(s.with_(seqlen=1), device="cuda")
+        for i in range(args.case_launches):
+            m3.step(*(steps[k][i] for k in keys[:6]), pre["A"], pre["D"], st)
+    m3.stream_status()
+    torch.cuda.synchronize()
+    print(f"case {args.case} {s} x{args.case_launches} done")
 
 
 # ---------------------------------------------------------------- helpers
@@ -418,7 +452,9 @@ def cpu_baseline(s, keys):
 
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -241,6 +241,10 @@ m3_status m3_stream_status(void *stream) {
         unsigned code = 0;
         cudaError_t e = m3::read_device_error(&code, static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_fail(e, "m3_stream_status");
+        unsigned dcode = 0;
+        e = m3::read_decode_error(&dcode);
+        if (e != cudaSuccess) return cuda_fail(e, "m3_stream_status");
+        code |= dcode << 8;
         if (code) {
             char buf[128];
             std::snprintf(buf, sizeof buf, "a bounded device-side wait gave up (code 0x%x)", code);

@@ -18,8 +18,13 @@
 #include <cuda_bf16.h>
 
 #include "m3_internal.h"
+#include "tc_primitives.cuh"
 
 namespace m3 {
+
+// Device-side failure word of the decode kernels (bounded waits that gave up).
+__device__ unsigned g_decode_error;
+
 namespace {
 
 template <typename T>
@@ -76,13 +81,17 @@ struct StepArgs {
     IO *y;
 };
 
-// Register-tiled kernel for the common sizes.  PT pairs per thread.
+// Register-tiled kernel for the common sizes.  Each thread owns PT pairs x 4
+// columns of the state (both rows of each pair, so the rotation is local);
+// the slice's small per-token vectors (b_prev, x_prev, B, C, x and the
+// decay-scaled cos/sin of each pair's angle) are staged once in shared memory
+// with coalesced loads while the state loads are in flight.
 template <int N, int P, int R, typename IO>
 struct StepCfg {
     static constexpr int K2 = N / 2;
-    static constexpr int CG = P / 4;                      // column groups (float4)
-    static constexpr int PT = (K2 * CG >= 1024) ? 8 : 4;  // pairs per thread
-    static constexpr int KK = K2 / PT;                    // pair groups
+    static constexpr int CG = P / 4;        // column groups (float4)
+    static constexpr int PT = 4;            // pairs per thread
+    static constexpr int KK = K2 / PT;      // pair groups
     static constexpr int THREADS = KK * CG;
     static constexpr int WARPS = THREADS / 32;
     static_assert(K2 % PT == 0, "pairs must split evenly");
@@ -94,7 +103,10 @@ template <int N, int P, int R, typename IO>
 __global__ void __launch_bounds__(StepCfg<N, P, R, IO>::THREADS)
 step_kernel(const StepArgs<IO> a) {
     using Cfg = StepCfg<N, P, R, IO>;
-    constexpr int K2 = Cfg::K2, CG = Cfg::CG, PT = Cfg::PT, KK = Cfg::KK;
+    constexpr int K2 = Cfg::K2, CG = Cfg::CG, PT = Cfg::PT, KK = Cfg::KK, NT = Cfg::THREADS;
+    __shared__ __align__(16) float sBp[R][N], sB[R][N], sC[R][N];
+    __shared__ __align__(16) float sXp[R][P], sX[R][P];
+    __shared__ __align__(16) float sAc[K2], sAs[K2];  // alpha cos, alpha sin of each pair's angle
     __shared__ float ypart[Cfg::WARPS][R][P];
 
     const int tid = threadIdx.x;
@@ -115,16 +127,27 @@ step_kernel(const StepArgs<IO> a) {
     const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
     const float alpha = __expf(dtv * a.A[h]);
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
-    float4 xpv[R], xv[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        xpv[r] = __ldg(reinterpret_cast<const float4 *>(a.xp + (bh * R + r) * P + p0));
-        xv[r] = ld4(a.x, (bh * R + r) * P + p0);
+    // ---- stage the slice's small vectors
+    for (int i = tid; i < R * N; i += NT) {
+        (&sBp[0][0])[i] = a.bp[bh * R * N + i];
+        (&sB[0][0])[i] = ldv(a.B, bh * R * N + i);
+        (&sC[0][0])[i] = ldv(a.C, bh * R * N + i);
     }
+    for (int i = tid; i < R * P; i += NT) {
+        (&sXp[0][0])[i] = a.xp[bh * R * P + i];
+        (&sX[0][0])[i] = ldv(a.x, bh * R * P + i);
+    }
+    for (int k = tid; k < K2; k += NT) {
+        float sn, cs;
+        sincosf(dtv * ldv(a.theta, bh * K2 + k), &sn, &cs);
+        sAc[k] = alpha * cs;
+        sAs[k] = alpha * sn;
+    }
+    __syncthreads();
+
     float4 yacc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) yacc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-
 #pragma unroll
     for (int j = 0; j < PT; ++j) {
         const int k = kk + j * KK;
@@ -132,15 +155,14 @@ step_kernel(const StepArgs<IO> a) {
         // previous-token trapezoid write
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const float2 bpk = __ldg(reinterpret_cast<const float2 *>(a.bp + (bh * R + r) * N + 2 * k));
+            const float2 bpk = *reinterpret_cast<const float2 *>(&sBp[r][2 * k]);
+            const float4 xp = *reinterpret_cast<const float4 *>(&sXp[r][p0]);
             const float cu = betap * bpk.x, cv = betap * bpk.y;
-            u.x += cu * xpv[r].x; u.y += cu * xpv[r].y; u.z += cu * xpv[r].z; u.w += cu * xpv[r].w;
-            v.x += cv * xpv[r].x; v.y += cv * xpv[r].y; v.z += cv * xpv[r].z; v.w += cv * xpv[r].w;
+            u.x = fmaf(cu, xp.x, u.x); u.y = fmaf(cu, xp.y, u.y); u.z = fmaf(cu, xp.z, u.z); u.w = fmaf(cu, xp.w, u.w);
+            v.x = fmaf(cv, xp.x, v.x); v.y = fmaf(cv, xp.y, v.y); v.z = fmaf(cv, xp.z, v.z); v.w = fmaf(cv, xp.w, v.w);
         }
         // decay + rotation by -dt*theta_k
-        float sn, cs;
-        sincosf(dtv * ldv(a.theta, bh * K2 + k), &sn, &cs);
-        const float ac = alpha * cs, as = alpha * sn;
+        const float ac = sAc[k], as = sAs[k];
         float4 nu, nv;
         nu.x = ac * u.x + as * v.x; nv.x = ac * v.x - as * u.x;
         nu.y = ac * u.y + as * v.y; nv.y = ac * v.y - as * u.y;
@@ -149,21 +171,22 @@ step_kernel(const StepArgs<IO> a) {
         // current-token write and readout
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const float2 bk = ld2(a.B, (bh * R + r) * N + 2 * k);
+            const float2 bk = *reinterpret_cast<const float2 *>(&sB[r][2 * k]);
+            const float4 xv = *reinterpret_cast<const float4 *>(&sX[r][p0]);
             const float cu = gam * bk.x, cv = gam * bk.y;
-            nu.x += cu * xv[r].x; nu.y += cu * xv[r].y; nu.z += cu * xv[r].z; nu.w += cu * xv[r].w;
-            nv.x += cv * xv[r].x; nv.y += cv * xv[r].y; nv.z += cv * xv[r].z; nv.w += cv * xv[r].w;
+            nu.x = fmaf(cu, xv.x, nu.x); nu.y = fmaf(cu, xv.y, nu.y); nu.z = fmaf(cu, xv.z, nu.z); nu.w = fmaf(cu, xv.w, nu.w);
+            nv.x = fmaf(cv, xv.x, nv.x); nv.y = fmaf(cv, xv.y, nv.y); nv.z = fmaf(cv, xv.z, nv.z); nv.w = fmaf(cv, xv.w, nv.w);
         }
+        __stcs(hst + ((2 * k) * P + p0) / 4, nu);
+        __stcs(hst + ((2 * k + 1) * P + p0) / 4, nv);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const float2 ck = ld2(a.C, (bh * R + r) * N + 2 * k);
+            const float2 ck = *reinterpret_cast<const float2 *>(&sC[r][2 * k]);
             yacc[r].x += nu.x * ck.x + nv.x * ck.y;
             yacc[r].y += nu.y * ck.x + nv.y * ck.y;
             yacc[r].z += nu.z * ck.x + nv.z * ck.y;
             yacc[r].w += nu.w * ck.x + nv.w * ck.y;
         }
-        __stcs(hst + ((2 * k) * P + p0) / 4, nu);
-        __stcs(hst + ((2 * k + 1) * P + p0) / 4, nv);
     }
     // ---- readout: sum over pair groups (same cg) -- shuffle within the warp
 #pragma unroll
@@ -179,26 +202,20 @@ step_kernel(const StepArgs<IO> a) {
     const int warp = tid / 32, lane = tid % 32;
     if (lane < CG || CG >= 32) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            ypart[warp][r][p0 + 0] = yacc[r].x;
-            ypart[warp][r][p0 + 1] = yacc[r].y;
-            ypart[warp][r][p0 + 2] = yacc[r].z;
-            ypart[warp][r][p0 + 3] = yacc[r].w;
-        }
+        for (int r = 0; r < R; ++r) *reinterpret_cast<float4 *>(&ypart[warp][r][p0]) = yacc[r];
     }
-    __syncthreads();  // also orders every read of b_prev/x_prev before the writes below
+    __syncthreads();
     const float Dh = a.D[h];
-    for (int idx = tid; idx < R * P; idx += Cfg::THREADS) {
+    for (int idx = tid; idx < R * P; idx += NT) {
         const int r = idx / P, p = idx % P;
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < Cfg::WARPS; ++w) s += ypart[w][r][p];
-        const float xval = ldv(a.x, (bh * R + r) * P + p);
+        const float xval = sX[r][p];
         stv(a.y, (bh * R + r) * P + p, s + Dh * xval);
         a.xp[(bh * R + r) * P + p] = xval;
     }
-    for (int idx = tid; idx < R * N; idx += Cfg::THREADS)
-        a.bp[bh * R * N + idx] = ldv(a.B, bh * R * N + idx);
+    for (int i = tid; i < R * N; i += NT) a.bp[bh * R * N + i] = (&sB[0][0])[i];
 }
 
 // Generic kernel for any even N and any P: one thread per (pair, column),
@@ -248,6 +265,225 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a)
         a.bp[bh * R * N + idx] = ldv(a.B, bh * R * N + idx);
 }
 
+// Persistent streaming variant: each CTA walks slices bh = blockIdx.x,
+// blockIdx.x + gridDim.x, ...; a bulk asynchronous copy brings the next-but-one
+// slice's state and small vectors into a 2-stage shared-memory ring while the
+// current slice is computed, so every SM keeps state bytes in flight all the
+// time instead of alternating load, compute and store per CTA.
+template <int N, int P, int R, typename IO>
+struct StreamCfg {
+    static constexpr int K2 = N / 2;
+    static constexpr int CG = P / 4;
+    static constexpr int PT = 4;
+    static constexpr int KK = K2 / PT;
+    static constexpr int THREADS = KK * CG;
+    static constexpr int WARPS = THREADS / 32;
+    // one stage: state, b_prev, x_prev (fp32); B, C, x, theta (io)
+    static constexpr uint32_t B_H = N * P * 4;
+    static constexpr uint32_t B_BP = R * N * 4, B_XP = R * P * 4;
+    static constexpr uint32_t B_B = R * N * sizeof(IO), B_X = R * P * sizeof(IO), B_TH = K2 * sizeof(IO);
+    static constexpr uint32_t O_BP = B_H, O_XP = O_BP + B_BP, O_B = O_XP + B_XP, O_C = O_B + B_B,
+                              O_X = O_C + B_B, O_TH = O_X + B_X;
+    static constexpr uint32_t STAGE = ((O_TH + B_TH + 127) / 128) * 128;
+    static constexpr uint32_t TX = B_H + B_BP + B_XP + 2 * B_B + B_X + B_TH;
+    static constexpr uint32_t O_YP = 2 * STAGE;                       // ypart [WARPS][R][P]
+    static constexpr uint32_t O_AC = O_YP + WARPS * R * P * 4;        // alpha cos [K2], alpha sin [K2]
+    static constexpr uint32_t O_BAR = O_AC + 2 * K2 * 4;
+    static constexpr uint32_t SMEM = O_BAR + 16;
+    static constexpr int CTAS_PER_SM = (3 * (SMEM + 1024) <= 232448) ? 3 : 2;  // as many as shared memory allows
+    static_assert(B_BP % 16 == 0 && B_XP % 16 == 0 && B_B % 16 == 0 && B_X % 16 == 0 && B_TH % 16 == 0,
+                  "bulk copies move multiples of 16 bytes");
+    static_assert(THREADS % 32 == 0 && THREADS <= 1024, "bad block size");
+};
+
+template <typename T>
+__device__ __forceinline__ float sv(const T *p, int i);
+template <>
+__device__ __forceinline__ float sv<float>(const float *p, int i) { return p[i]; }
+template <>
+__device__ __forceinline__ float sv<__nv_bfloat16>(const __nv_bfloat16 *p, int i) { return __bfloat162float(p[i]); }
+template <typename T>
+__device__ __forceinline__ float2 sv2(const T *p, int i);
+template <>
+__device__ __forceinline__ float2 sv2<float>(const float *p, int i) { return *reinterpret_cast<const float2 *>(p + i); }
+template <>
+__device__ __forceinline__ float2 sv2<__nv_bfloat16>(const __nv_bfloat16 *p, int i) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p + i));
+}
+template <typename T>
+__device__ __forceinline__ float4 sv4(const T *p, int i);
+template <>
+__device__ __forceinline__ float4 sv4<float>(const float *p, int i) { return *reinterpret_cast<const float4 *>(p + i); }
+template <>
+__device__ __forceinline__ float4 sv4<__nv_bfloat16>(const __nv_bfloat16 *p, int i) {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p + i);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+template <int N, int P, int R, typename IO>
+__global__ void __launch_bounds__(StreamCfg<N, P, R, IO>::THREADS, StreamCfg<N, P, R, IO>::CTAS_PER_SM)
+step_stream_kernel(const StepArgs<IO> a) {
+    using Cfg = StreamCfg<N, P, R, IO>;
+    constexpr int K2 = Cfg::K2, CG = Cfg::CG, PT = Cfg::PT, KK = Cfg::KK, NT = Cfg::THREADS;
+    extern __shared__ __align__(128) uint8_t sm[];
+    float *ypart = reinterpret_cast<float *>(sm + Cfg::O_YP);
+    float *sAc = reinterpret_cast<float *>(sm + Cfg::O_AC);
+    float *sAs = sAc + K2;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + Cfg::O_BAR);
+    __shared__ int abort_flag;
+    const int tid = threadIdx.x;
+    const int cg = tid % CG, kk = tid / CG, p0 = cg * 4;
+    const int warp = tid / 32, lane = tid % 32;
+    const int64_t BH = a.BH, step = gridDim.x;
+
+    auto issue = [&](int64_t bh, int st) {
+        uint8_t *s = sm + st * Cfg::STAGE;
+        tc::mbar_arrive_expect_tx(&full[st], Cfg::TX);
+        tc::bulk_g2s(s, a.h + bh * N * P, Cfg::B_H, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_BP, a.bp + bh * R * N, Cfg::B_BP, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_XP, a.xp + bh * R * P, Cfg::B_XP, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_B, a.B + bh * R * N, Cfg::B_B, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_C, a.C + bh * R * N, Cfg::B_B, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_X, a.x + bh * R * P, Cfg::B_X, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_TH, a.theta + bh * K2, Cfg::B_TH, &full[st]);
+    };
+    if (tid == 0) {
+        tc::mbar_init(&full[0], 1);
+        tc::mbar_init(&full[1], 1);
+        abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        if ((int64_t)blockIdx.x < BH) issue(blockIdx.x, 0);
+        if ((int64_t)blockIdx.x + step < BH) issue(blockIdx.x + step, 1);
+    }
+    int it = 0;
+    for (int64_t bh = blockIdx.x; bh < BH; bh += step, ++it) {
+        const int st = it & 1;
+        const uint8_t *s = sm + st * Cfg::STAGE;
+        const float *sh = reinterpret_cast<const float *>(s);
+        const float *sBp = reinterpret_cast<const float *>(s + Cfg::O_BP);
+        const float *sXp = reinterpret_cast<const float *>(s + Cfg::O_XP);
+        const IO *sB = reinterpret_cast<const IO *>(s + Cfg::O_B);
+        const IO *sC = reinterpret_cast<const IO *>(s + Cfg::O_C);
+        const IO *sX = reinterpret_cast<const IO *>(s + Cfg::O_X);
+        const IO *sTh = reinterpret_cast<const IO *>(s + Cfg::O_TH);
+        const int h = (int)(bh % a.H);
+        const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
+        const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
+        const bool ok = tc::mbar_wait(&full[st], (it >> 1) & 1, &abort_flag, &g_decode_error, tc::kErrWaitTma);
+        if (__syncthreads_or(!ok)) break;
+        if (tid < K2) {
+            const float alpha = __expf(dtv * a.A[h]);
+            float sn, cs;
+            sincosf(dtv * sv(sTh, tid), &sn, &cs);
+            sAc[tid] = alpha * cs;
+            sAs[tid] = alpha * sn;
+        }
+        __syncthreads();
+        float4 xp[R], xv[R], yacc[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            xp[r] = *reinterpret_cast<const float4 *>(sXp + r * P + p0);
+            xv[r] = sv4(sX, r * P + p0);
+            yacc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float4 *hg = reinterpret_cast<float4 *>(a.h + bh * N * P);
+#pragma unroll
+        for (int j = 0; j < PT; ++j) {
+            const int k = kk + j * KK;
+            float4 u = *reinterpret_cast<const float4 *>(sh + (2 * k) * P + p0);
+            float4 v = *reinterpret_cast<const float4 *>(sh + (2 * k + 1) * P + p0);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float2 bpk = *reinterpret_cast<const float2 *>(sBp + r * N + 2 * k);
+                const float cu = betap * bpk.x, cv = betap * bpk.y;
+                u.x = fmaf(cu, xp[r].x, u.x); u.y = fmaf(cu, xp[r].y, u.y);
+                u.z = fmaf(cu, xp[r].z, u.z); u.w = fmaf(cu, xp[r].w, u.w);
+                v.x = fmaf(cv, xp[r].x, v.x); v.y = fmaf(cv, xp[r].y, v.y);
+                v.z = fmaf(cv, xp[r].z, v.z); v.w = fmaf(cv, xp[r].w, v.w);
+            }
+            const float ac = sAc[k], as = sAs[k];
+            float4 nu, nv;
+            nu.x = ac * u.x + as * v.x; nv.x = ac * v.x - as * u.x;
+            nu.y = ac * u.y + as * v.y; nv.y = ac * v.y - as * u.y;
+            nu.z = ac * u.z + as * v.z; nv.z = ac * v.z - as * u.z;
+            nu.w = ac * u.w + as * v.w; nv.w = ac * v.w - as * u.w;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float2 bk = sv2(sB, r * N + 2 * k);
+                const float cu = gam * bk.x, cv = gam * bk.y;
+                nu.x = fmaf(cu, xv[r].x, nu.x); nu.y = fmaf(cu, xv[r].y, nu.y);
+                nu.z = fmaf(cu, xv[r].z, nu.z); nu.w = fmaf(cu, xv[r].w, nu.w);
+                nv.x = fmaf(cv, xv[r].x, nv.x); nv.y = fmaf(cv, xv[r].y, nv.y);
+                nv.z = fmaf(cv, xv[r].z, nv.z); nv.w = fmaf(cv, xv[r].w, nv.w);
+            }
+            __stcs(hg + ((2 * k) * P + p0) / 4, nu);
+            __stcs(hg + ((2 * k + 1) * P + p0) / 4, nv);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float2 ck = sv2(sC, r * N + 2 * k);
+                yacc[r].x += nu.x * ck.x + nv.x * ck.y;
+                yacc[r].y += nu.y * ck.x + nv.y * ck.y;
+                yacc[r].z += nu.z * ck.x + nv.z * ck.y;
+                yacc[r].w += nu.w * ck.x + nv.w * ck.y;
+            }
+        }
+#pragma unroll
+        for (int off = CG; off < 32; off *= 2) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                yacc[r].x += __shfl_xor_sync(0xffffffffu, yacc[r].x, off);
+                yacc[r].y += __shfl_xor_sync(0xffffffffu, yacc[r].y, off);
+                yacc[r].z += __shfl_xor_sync(0xffffffffu, yacc[r].z, off);
+                yacc[r].w += __shfl_xor_sync(0xffffffffu, yacc[r].w, off);
+            }
+        }
+        if (lane < CG || CG >= 32) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                *reinterpret_cast<float4 *>(ypart + (warp * R + r) * P + p0) = yacc[r];
+        }
+        __syncthreads();
+        const float Dh = a.D[h];
+        for (int idx = tid; idx < R * P; idx += NT) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < Cfg::WARPS; ++w) sum += ypart[w * R * P + idx];
+            const float xval = sv(sX, idx);
+            stv(a.y, bh * R * P + idx, sum + Dh * xval);
+            a.xp[bh * R * P + idx] = xval;
+        }
+        for (int i = tid; i < R * N; i += NT) a.bp[bh * R * N + i] = sv(sB, i);
+        __syncthreads();  // every read of this stage is done: refill it
+        if (tid == 0 && bh + 2 * step < BH) issue(bh + 2 * step, st);
+    }
+    // let any copy still in flight land before the CTA exits (only after an abort)
+    if (tid == 0 && abort_flag) {
+        for (int q = 0; q < 2; ++q) tc::mbar_wait(&full[q], 0, nullptr, &g_decode_error, 0, 400000000LL);
+    }
+}
+
+template <int N, int P, int R, typename IO>
+cudaError_t launch_stream(const StepArgs<IO> &a, cudaStream_t s) {
+    using Cfg = StreamCfg<N, P, R, IO>;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(step_stream_kernel<N, P, R, IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    int64_t grid = (int64_t)sms * Cfg::CTAS_PER_SM;
+    if (grid > a.BH) grid = a.BH;
+    step_stream_kernel<N, P, R, IO><<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <int N, int P, int R, typename IO>
 cudaError_t launch_tiled(const StepArgs<IO> &a, cudaStream_t s) {
     step_kernel<N, P, R, IO><<<(unsigned)a.BH, StepCfg<N, P, R, IO>::THREADS, 0, s>>>(a);
@@ -257,8 +493,10 @@ cudaError_t launch_tiled(const StepArgs<IO> &a, cudaStream_t s) {
 template <typename IO, int R>
 cudaError_t dispatch_np(const StepArgs<IO> &a, cudaStream_t s, bool *done) {
     *done = true;
-    if (a.N == 128 && a.P == 64) return launch_tiled<128, 64, R, IO>(a, s);
-    if (a.N == 64 && a.P == 64) return launch_tiled<64, 64, R, IO>(a, s);
+    // rank 1: one CTA per slice (measured faster); rank >= 2: the persistent
+    // streaming kernel (its heavier per-element work overlaps the next slice's load)
+    if (a.N == 128 && a.P == 64) return R == 1 ? launch_tiled<128, 64, R, IO>(a, s) : launch_stream<128, 64, R, IO>(a, s);
+    if (a.N == 64 && a.P == 64) return R == 1 ? launch_tiled<64, 64, R, IO>(a, s) : launch_stream<64, 64, R, IO>(a, s);
     if (a.N == 128 && a.P == 128) return launch_tiled<128, 128, R, IO>(a, s);
     if (a.N == 64 && a.P == 128) return launch_tiled<64, 128, R, IO>(a, s);
     if (a.N == 256 && a.P == 64) return launch_tiled<256, 64, R, IO>(a, s);
@@ -292,6 +530,18 @@ cudaError_t launch_typed(const Problem &p) {
 
 cudaError_t launch_step(const Problem &p, const char **) {
     return p.bf16 ? launch_typed<__nv_bfloat16>(p) : launch_typed<float>(p);
+}
+
+cudaError_t read_decode_error(unsigned *code) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_decode_error, sizeof v);
+    if (e != cudaSuccess) return e;
+    if (v) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_decode_error, &zero, sizeof zero);
+    }
+    *code = v;
+    return e;
 }
 
 }  // namespace m3

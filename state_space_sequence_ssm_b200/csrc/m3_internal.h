@@ -33,5 +33,7 @@ cudaError_t launch_step(const Problem &p, const char **why);
 // Synchronise `stream`, then read and clear the device error word that the
 // tensor-core kernel's bounded waits set when they give up.
 cudaError_t read_device_error(unsigned *code, cudaStream_t stream);
+// Read and clear the decode kernels' device error word (after a sync).
+cudaError_t read_decode_error(unsigned *code);
 
 }  // namespace m3
