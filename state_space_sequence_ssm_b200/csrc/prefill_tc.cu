@@ -52,10 +52,11 @@ using namespace tc;
 
 constexpr int kP = 64;           // head dim this kernel is built for
 constexpr int kRows = 128;       // rows per chunk = MMA M
-constexpr int kWG = 128;         // threads per warpgroup
-constexpr int kWarpTma = 8;
-constexpr int kWarpMma = 9;
-constexpr int kThreads = 320;
+constexpr int kPro = 256;        // prologue threads (warps 0-7)
+constexpr int kSt = 256;         // state / epilogue threads (warps 8-15)
+constexpr int kWarpTma = 16;
+constexpr int kWarpMma = 17;
+constexpr int kThreads = 576;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S [0,128), G [128,192), Yo double-buffered [192,320), Yd [320,384),
 // P (bf16 pairs) [384,448)
@@ -71,9 +72,9 @@ struct Cfg {
     static constexpr int K2 = N / 2;         // state pairs
     static constexpr int KB = N / 64;        // 64-wide blocks of the state dim
     static constexpr int G4 = K2 / 4;        // groups of 4 pairs = one 16-byte chunk of a row
-    static constexpr int NPART = kWG / G4;   // token parts of the angle pass
+    static constexpr int NPART = kPro / G4;  // token parts of the angle pass
     static constexpr int TPT = Q / NPART;    // tokens per thread in the angle pass
-    static constexpr int TB = (4 / R) < TPT ? (4 / R) : TPT;  // tokens per rotation batch
+    static constexpr int TB = (2 / R) < 1 ? 1 : ((2 / R) < TPT ? (2 / R) : TPT);  // tokens per rotation batch
     static constexpr uint32_t X_BYTES = kRows * 128;         // 16 KB
     static constexpr uint32_t BC_BYTES = KB * kRows * 128;   // one B or C tile
     static constexpr uint32_t BCS_BYTES = 2 * BC_BYTES;      // one stage of the B/C ring
@@ -91,7 +92,7 @@ struct Cfg {
     static constexpr uint32_t NBARS = 19;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024 alignment
-    static_assert(K2 % 4 == 0 && kWG % G4 == 0, "pair groups must tile the warpgroup");
+    static_assert(K2 % 4 == 0 && kPro % G4 == 0, "pair groups must tile the prologue threads");
     static_assert(Q % NPART == 0 && TPT % TB == 0, "tokens must split across the angle-pass parts");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -108,18 +109,18 @@ struct TcArgs {
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
 __device__ __forceinline__ float bf16_bits(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
 
-// OR-reduction over one warpgroup that doubles as its barrier: every thread
-// gets the same answer, so control flow stays uniform on failure.
-template <uint32_t ID>
+// OR-reduction over one role's threads that doubles as its barrier: every
+// thread gets the same answer, so control flow stays uniform on failure.
+template <uint32_t ID, uint32_t COUNT>
 __device__ __forceinline__ bool bar_any(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, %2, 128, q;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "n"(ID)
+        : "r"((uint32_t)pred), "n"(ID), "n"(COUNT)
         : "memory");
     return r != 0;
 }
@@ -135,6 +136,20 @@ __device__ __forceinline__ void store_state_row(uint8_t *hb, int n, const float 
         v.z = pack_bf16(h[8 * j + 4], h[8 * j + 5]);
         v.w = pack_bf16(h[8 * j + 6], h[8 * j + 7]);
         *reinterpret_cast<uint4 *>(hb + sw128(n, j)) = v;
+    }
+}
+
+// bf16 copy of 32 fp32 values (columns 32*half ..) of state row n into the
+// 128B-swizzled MN-major operand tile (row n = K index of the readout MMA).
+__device__ __forceinline__ void store_state_half(uint8_t *hb, int n, int half, const float (&h)[32]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint4 v;
+        v.x = pack_bf16(h[8 * j + 0], h[8 * j + 1]);
+        v.y = pack_bf16(h[8 * j + 2], h[8 * j + 3]);
+        v.z = pack_bf16(h[8 * j + 4], h[8 * j + 5]);
+        v.w = pack_bf16(h[8 * j + 6], h[8 * j + 7]);
+        *reinterpret_cast<uint4 *>(hb + sw128(n, 4 * half + j)) = v;
     }
 }
 
@@ -166,8 +181,8 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 // colf_s = exp(cA_0 - cA_s) ghat_s (both in fp32 range), so each element
 // costs two multiplies; otherwise every element takes its own exp.
 template <int R, int Q>
-__device__ __forceinline__ void mask_to_tmem(int wq, int row, uint32_t tl, const float *cAl2, const float *gam,
-                                             const float *ghat, const float *colf) {
+__device__ __forceinline__ void mask_to_tmem(int cbA, int cbB, int wq, int row, uint32_t tl, const float *cAl2,
+                                             const float *gam, const float *ghat, const float *colf) {
     constexpr int NT = 16 / R;  // tokens per 16-column half block
     const int ti = row / R;
     const float cai = cAl2[ti], gi = gam[ti];
@@ -175,25 +190,24 @@ __device__ __forceinline__ void mask_to_tmem(int wq, int row, uint32_t tl, const
     const bool fact = (ca0 - cAl2[Q - 1]) < 100.f;  // uniform across the CTA
     const float rowf = ex2(cai - ca0);
 #pragma unroll 1
-    for (int cb = 0; cb < 4; ++cb) {
-        uint32_t pk[16];
-        if (cb <= wq) {
-            float v[32];
-            tmem_ld32(tl + kColS + 32 * cb, v);
-            const int tb0 = (32 * cb) / R;
-            tmem_wait_ld();
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int tb = tb0 + hf * NT;
+    for (int bi = 0; bi < 2; ++bi) {
+        const int cb = bi == 0 ? cbA : cbB;  // this thread's two 32-column blocks
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+            uint32_t pk[8];
+            if (cb <= wq) {
+                float v[16];
+                tmem_ld16(tl + kColS + 32 * cb + 16 * hf, v);
+                const int tb = (32 * cb + 16 * hf) / R;
                 if (fact) {
                     float cf[NT];
 #pragma unroll
                     for (int k = 0; k < NT; ++k) cf[k] = colf[tb + k];
+                    tmem_wait_ld();
                     if (cb < wq) {
 #pragma unroll
                         for (int k = 0; k < 16; k += 2)
-                            pk[8 * hf + (k >> 1)] = pack_bf16(v[16 * hf + k] * cf[k / R] * rowf,
-                                                              v[16 * hf + k + 1] * cf[(k + 1) / R] * rowf);
+                            pk[k >> 1] = pack_bf16(v[k] * cf[k / R] * rowf, v[k + 1] * cf[(k + 1) / R] * rowf);
                     } else {
 #pragma unroll
                         for (int k = 0; k < 16; k += 2) {
@@ -202,9 +216,9 @@ __device__ __forceinline__ void mask_to_tmem(int wq, int row, uint32_t tl, const
                             for (int u = 0; u < 2; ++u) {
                                 const int tj = tb + (k + u) / R;
                                 const float f = tj < ti ? cf[(k + u) / R] * rowf : (tj == ti ? gi : 0.f);
-                                pv[u] = v[16 * hf + k + u] * f;
+                                pv[u] = v[k + u] * f;
                             }
-                            pk[8 * hf + (k >> 1)] = pack_bf16(pv[0], pv[1]);
+                            pk[k >> 1] = pack_bf16(pv[0], pv[1]);
                         }
                     }
                 } else {
@@ -214,6 +228,7 @@ __device__ __forceinline__ void mask_to_tmem(int wq, int row, uint32_t tl, const
                         ca[k] = cAl2[tb + k];
                         gh[k] = ghat[tb + k];
                     }
+                    tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < 16; k += 2) {
                         float pv[2];
@@ -221,17 +236,17 @@ __device__ __forceinline__ void mask_to_tmem(int wq, int row, uint32_t tl, const
                         for (int u = 0; u < 2; ++u) {
                             const int tj = tb + (k + u) / R;
                             const float coef = tj < ti ? gh[(k + u) / R] : (tj == ti ? gi : 0.f);
-                            pv[u] = v[16 * hf + k + u] * ex2(fminf(cai - ca[(k + u) / R], 0.f)) * coef;
+                            pv[u] = v[k + u] * ex2(fminf(cai - ca[(k + u) / R], 0.f)) * coef;
                         }
-                        pk[8 * hf + (k >> 1)] = pack_bf16(pv[0], pv[1]);
+                        pk[k >> 1] = pack_bf16(pv[0], pv[1]);
                     }
                 }
-            }
-        } else {
+            } else {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                for (int k = 0; k < 8; ++k) pk[k] = 0u;
+            }
+            tmem_st8(tl + kColP + 16 * cb + 8 * hf, pk);
         }
-        tmem_st16(tl + kColP + 16 * cb, pk);
     }
     tmem_wait_st();
 }
@@ -425,8 +440,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 mbar_wait(bb.drain, 0, nullptr, err, 0, 400000000LL);
             }
         }
-    } else if (warp < 4) {
-        // ============================================================ prologue warpgroup
+    } else if (warp < 8) {
+        // ============================================================ prologue warps (0-7)
         const float Ah2 = a.A[h] * kLog2e;
         uint8_t *xw = smem + C::OFF_XW;
         const unsigned short *dtr = reinterpret_cast<const unsigned short *>(a.dt);
@@ -472,8 +487,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             uint8_t *cst = bst + C::BC_BYTES;
             uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
             // the scalar buffer c % kNX is free once the epilogue of c - kNX is done
-            if (c >= kNX && bar_any<kBarPro>(!mbar_wait(&bb.empty_x[sx], ((c / kNX) - 1) & 1, abort_flag, err,
-                                                        kErrWaitCompute)))
+            if (c >= kNX && bar_any<kBarPro, kPro>(!mbar_wait(&bb.empty_x[sx], ((c / kNX) - 1) & 1, abort_flag,
+                                                              err, kErrWaitCompute)))
                 break;
 
             // ---- A. per-token scalars and the chunk-local scan of dt*A
@@ -496,7 +511,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     if (lane == 31) wtot[warp] = acc;
                 }
             }
-            named_bar(kBarPro, kWG);
+            named_bar(kBarPro, kPro);
             if (tid < Q) {
                 float off = 0.f, tot = 0.f;
 #pragma unroll
@@ -527,7 +542,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
                 *reinterpret_cast<float4 *>(phis + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
                 // the B/C tiles of this chunk
-                if (bar_any<kBarPro>(!mbar_wait(&bb.full_bc[s], (c >> 1) & 1, abort_flag, err, kErrWaitTma))) break;
+                if (bar_any<kBarPro, kPro>(!mbar_wait(&bb.full_bc[s], (c >> 1) & 1, abort_flag, err, kErrWaitTma)))
+                    break;
                 float phi[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int q = 0; q < part; ++q) {
                     const float4 v = *reinterpret_cast<const float4 *>(phis + q * K2 + 4 * g);
@@ -600,64 +616,70 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
             // ---- C. w o X (chunk-state weights on the value rows), once G(c-1)
             //      has finished reading the previous w o X and x of chunk c is in
-            if (bar_any<kBarPro>((c >= 1 && !mbar_wait(bb.sg, (c - 1) & 1, abort_flag, err, kErrWaitMma)) ||
-                                 !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma)))
+            if (bar_any<kBarPro, kPro>((c >= 1 && !mbar_wait(bb.sg, (c - 1) & 1, abort_flag, err, kErrWaitMma)) ||
+                                       !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma)))
                 break;
             {
-                const int row = tid;
+                const int row = tid >> 1, j0 = (tid & 1) * 4;  // half a row per thread
                 const float wv = wst[row / R];
                 const uint32_t ww = pack_bf16(wv, wv);
-                uint4 v[8];
+                uint4 v[4];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4 *>(xst + sw128(row, j));
+                for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4 *>(xst + sw128(row, j0 + j));
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     v[j].x = mul_bf16x2(v[j].x, ww);
                     v[j].y = mul_bf16x2(v[j].y, ww);
                     v[j].z = mul_bf16x2(v[j].z, ww);
                     v[j].w = mul_bf16x2(v[j].w, ww);
-                    *reinterpret_cast<uint4 *>(xw + sw128(row, j)) = v[j];
+                    *reinterpret_cast<uint4 *>(xw + sw128(row, j0 + j)) = v[j];
                 }
             }
             fence_proxy_async_smem();
-            named_bar(kBarPro, kWG);
+            named_bar(kBarPro, kPro);
             if (tid == 0) {
                 mbar_arrive(bb.ops);
                 mbar_arrive(&bb.sc[sx]);
             }
         }
     } else {
-        // ============================================================ state warpgroup
-        const int lt = tid - kWG;          // 0..127
+        // ============================================================ state warps (8-15)
+        // Thread (wq, lane, hf): TMEM lane quarter wq, state row / output row of
+        // that lane, and half hf of the 64 columns.
+        const int lt = tid - kPro;         // 0..255
+        const int hf = lt >> 7;            // column half
+        const int lq = lt & 127;           // TMEM lane = row
         const int wq = warp & 3;           // TMEM lane quarter
         const bool own_state = (N == 128) || (lane < 16);
-        const int srow = (N == 128) ? lt : (wq * 16 + lane);  // TMEM lane layout of G (M = N)
+        const int srow = (N == 128) ? lq : (wq * 16 + lane);  // TMEM lane layout of G (M = N)
         uint8_t *hbuf = smem + C::OFF_HB;
         const float Dh = a.D[h];
         const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
-        float hreg[64];
+        const int c0 = 32 * hf;            // first column of this thread's half
+        float hreg[32];
         // initial state h0 + beta'_0 b_prev x_prev^T (pending write of token -1)
         {
             const float betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
 #pragma unroll
-            for (int p = 0; p < 64; ++p) hreg[p] = 0.f;
+            for (int p = 0; p < 32; ++p) hreg[p] = 0.f;
             if (own_state) {
                 if (a.h0) {
 #pragma unroll
-                    for (int p = 0; p < 64; ++p) hreg[p] = a.h0[(bh * N + srow) * kP + p];
+                    for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * N + srow) * kP + c0 + p];
                 }
                 if (a.bp0 && a.xp0) {
                     for (int r = 0; r < R; ++r) {
                         const float cb = betap0 * a.bp0[(bh * R + r) * N + srow];
 #pragma unroll
-                        for (int p = 0; p < 64; ++p) hreg[p] = fmaf(cb, a.xp0[(bh * R + r) * kP + p], hreg[p]);
+                        for (int p = 0; p < 32; ++p)
+                            hreg[p] = fmaf(cb, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
                     }
                 }
-                store_state_row(hbuf, srow, hreg);
+                store_state_half(hbuf, srow, hf, hreg);
             }
         }
         fence_proxy_async_smem();
-        named_bar(kBarState, kWG);
+        named_bar(kBarState, kSt);
         if (lt == 0) mbar_arrive(bb.hrdy);
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
@@ -670,9 +692,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const float *sinE = cosE + K2;
             const uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
             // scalars of chunk c (release/acquire through sc), its x tile, and G(c)
-            if (bar_any<kBarState>(!mbar_wait(&bb.sc[sx], (c / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
-                                   !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma) ||
-                                   !mbar_wait(bb.sg, c & 1, abort_flag, err, kErrWaitMma))) {
+            if (bar_any<kBarState, kSt>(!mbar_wait(&bb.sc[sx], (c / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
+                                        !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma) ||
+                                        !mbar_wait(bb.sg, c & 1, abort_flag, err, kErrWaitMma))) {
                 ok = false;
                 break;
             }
@@ -683,51 +705,53 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const int kp = (own_state ? srow : 0) >> 1;
                 const float cs = cosE[kp], sn = sinE[kp];
                 const float sgn = (srow & 1) ? -sn : sn;
+                float gv[32];
+                tmem_ld32(tl + kColG + c0, gv);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float gv[32];
-                    tmem_ld32(tl + kColG + 32 * half, gv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int p = 0; p < 32; ++p) {
-                        const float u = fmaf(eA, hreg[32 * half + p], gv[p]);
-                        const float o = __shfl_xor_sync(0xffffffffu, u, 1);
-                        hreg[32 * half + p] = fmaf(u, cs, o * sgn);
-                    }
+                for (int p = 0; p < 32; ++p) {
+                    const float u = fmaf(eA, hreg[p], gv[p]);
+                    const float o = __shfl_xor_sync(0xffffffffu, u, 1);
+                    hreg[p] = fmaf(u, cs, o * sgn);
                 }
-                if (own_state) store_state_row(hbuf, srow, hreg);
+                if (own_state) store_state_half(hbuf, srow, hf, hreg);
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(kBarState, kWG);
+            named_bar(kBarState, kSt);
             if (lt == 0) mbar_arrive(bb.hrdy);
 
-            // ---- D. decay mask S -> P (TMEM)
-            mask_to_tmem<R, Q>(wq, lt, tl, cAl2, gam, ghat, colf);
+            // ---- D. decay mask S -> P (TMEM): half 0 takes column blocks 0 and 3,
+            //      half 1 blocks 1 and 2 (balances the lower triangle)
+            mask_to_tmem<R, Q>(hf == 0 ? 0 : 1, hf == 0 ? 3 : 2, wq, lq, tl, cAl2, gam, ghat, colf);
             tc_fence_before();
-            named_bar(kBarState, kWG);
+            named_bar(kBarState, kSt);
             if (lt == 0) mbar_arrive(bb.p);
 
-            // ---- F. epilogue: y = Yd + exp(cA_t) Yo + D x
-            if (bar_any<kBarState>(!mbar_wait(bb.yd, c & 1, abort_flag, err, kErrWaitMma))) { ok = false; break; }
+            // ---- F. epilogue: y = Yd + exp(cA_t) Yo + D x, this thread's 32 columns
+            if (bar_any<kBarState, kSt>(!mbar_wait(bb.yd, c & 1, abort_flag, err, kErrWaitMma))) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
             {
-                const int row = lt;
+                const int row = lq;
                 const int ti = row / R, r = row % R;
                 const int64_t t = (int64_t)c * Q + ti;
                 const float sc = ex2(cAl2[ti]);
                 const uint32_t yo = kColYo + (uint32_t)(c & 1) * 64u;
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float yd[32], yv[32];
-                    tmem_ld32(tl + kColYd + 32 * half, yd);
-                    tmem_ld32(tl + yo + 32 * half, yv);
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    float yd[16], yv[16];
+                    tmem_ld16(tl + kColYd + c0 + 16 * qq, yd);
+                    tmem_ld16(tl + yo + c0 + 16 * qq, yv);
                     tmem_wait_ld();
                     if (t < T) {
-                        __nv_bfloat16 *yrow = a.y + (tok(t) * R + r) * kP + 32 * half;
+                        __nv_bfloat16 *yrow = a.y + (tok(t) * R + r) * kP + c0 + 16 * qq;
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 xv = *reinterpret_cast<const uint4 *>(xst + sw128(row, 4 * half + q));
+                        for (int q = 0; q < 2; ++q) {
+                            const uint4 xv =
+                                *reinterpret_cast<const uint4 *>(xst + sw128(row, (c0 >> 3) + 2 * qq + q));
                             const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
                             uint32_t o[4];
 #pragma unroll
@@ -744,24 +768,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
             }
             tc_fence_before();
-            named_bar(kBarState, kWG);
+            named_bar(kBarState, kSt);
             if (lt == 0) mbar_arrive(&bb.empty_x[sx]);
         }
         // ---- final state: plain-frame h_{T-1}, raw last token as the pending term
         if (ok) {
             if (a.hT && own_state) {
-                float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * N + srow) * kP);
+                float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * N + srow) * kP + c0);
 #pragma unroll
-                for (int p = 0; p < 16; ++p)
+                for (int p = 0; p < 8; ++p)
                     dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
             }
             if (a.bpT)
-                for (int i = lt; i < R * N; i += kWG) a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
+                for (int i = lt; i < R * N; i += kSt) a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
             if (a.xpT)
-                for (int i = lt; i < R * kP; i += kWG) a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
+                for (int i = lt; i < R * kP; i += kSt) a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
         }
     }
-
     __syncwarp();  // reconverge the single-lane roles before the block barrier
     tc_fence_before();
     __syncthreads();
