@@ -104,6 +104,7 @@ def file_hash(paths):
 def kernel_sources(kernel):
     csrc = os.path.join(ROOT, "state_space_sequence_ssm_b200", "csrc")
     files = {"prefill_simt_kernel": ["prefill_simt.cu"], "step_kernel": ["decode.cu"],
+             "step_stream_kernel": ["decode.cu"],
              "prefill_tc_kernel": ["prefill_tc.cu", "tc_primitives.cuh"]}[kernel]
     return [os.path.join(csrc, f) for f in files if os.path.exists(os.path.join(csrc, f))]
 
@@ -415,14 +416,17 @@ def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_pe
     el = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     per = el / S
     ab = step_bytes(s)
+    # the library runs rank 1 (and P = 128 or N = 256) on the one-CTA-per-slice
+    # kernel and rank >= 2 with P = 64, N in {64, 128} on the persistent one
+    kernel = "step_stream_kernel" if (s.rank >= 2 and s.headdim == 64 and s.dstate in (64, 128)) else "step_kernel"
     ach = ab / per / 1e9
     del g, steps
     torch.cuda.empty_cache()
     return {"workload": name, "value": world * s.batch / per, "unit": "tokens/s", "steps": S,
             "us_per_step": per * 1e6, "gpu_launches": S,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": ach / hbm_peak, "traffic": recorded_traffic("step_kernel", name),
-                         "kernel": "step_kernel", "algorithmic_bytes_per_launch": ab,
+                         "frac": ach / hbm_peak, "traffic": recorded_traffic(kernel, name),
+                         "kernel": kernel, "algorithmic_bytes_per_launch": ab,
                          "note": "per-step time includes graph launch gaps", "peak_source": peak_src}}
 
 
