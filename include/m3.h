@@ -96,9 +96,33 @@ typedef enum m3_algo {
     M3_ALGO_TC = 2      /* tcgen05/TMEM/TMA chunked scan (bf16 only)             */
 } m3_algo;
 
+/* The tensor-core path forced to split every sequence into s >= 1 segments
+ * (fewer if the sequence has fewer chunks); M3_ALGO_TC and M3_ALGO_AUTO
+ * choose the number themselves.  A split sequence runs as three launches:
+ * a summary pass (each segment's local end state from a zero state and its
+ * transition exp(sum dt A) Rot(-sum dt theta)), a scan of those summaries
+ * across the segments -- the chunk-state recurrence of "La dualità: Mamba-2
+ * e Mamba-3", section "Perché conviene: i tensor core", applied one level up
+ * -- and the full pass of every segment from its scanned initial state, so
+ * that a few long sequences still fill every SM. */
+#define M3_ALGO_TC_SEGMENTS(s) (M3_ALGO_TC | ((int)(s) << 8))
+
 /* Bytes of device workspace m3_scan_fwd needs for these dims (0 = none; the
- * workspace pointer may then be NULL).  Pure host function. */
+ * workspace pointer may then be NULL).  Host function; the answer depends on
+ * the current CUDA device's SM count (it sets how sequences are split).  The
+ * workspace holds fp32 per-segment states of split sequences,
+ * [segments][batch*nheads][dstate][headdim + 1]; it needs no initialisation,
+ * its contents are meaningless after the call, and calls that may run at the
+ * same time (other streams) must not share one. */
 M3_API m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes);
+
+/* How m3_scan_fwd_algo(algo, d, ...) will run on the current device:
+ * workspace bytes, segments per sequence (1 = not split) and the number of
+ * kernel launches of one call.  Any output pointer may be NULL.
+ * M3_ERR_UNSUPPORTED if `algo` names the tensor-core path for sizes it does
+ * not cover. */
+M3_API m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_bytes, int *segments,
+                              int *launches);
 
 /* Prefill: the chunked scan over a whole sequence (the four-piece chunked
  * algorithm of "La dualità: Mamba-2 e Mamba-3", section "Perché conviene: i
@@ -117,8 +141,10 @@ M3_API m3_status m3_scan_fwd(const m3_dims *d,
                       const m3_state *init, void *y, const m3_state *final_state,
                       void *workspace, size_t workspace_bytes, void *stream);
 
-/* Same as m3_scan_fwd with an explicit kernel choice (for cross-checks).
- * M3_ALGO_TC returns M3_ERR_UNSUPPORTED for sizes that path does not cover. */
+/* Same as m3_scan_fwd with an explicit kernel choice (for cross-checks):
+ * an m3_algo value or M3_ALGO_TC_SEGMENTS(s); the workspace must be at
+ * least m3_scan_plan's answer for the same `algo`.  The tensor-core choices
+ * return M3_ERR_UNSUPPORTED for sizes that path does not cover. */
 M3_API m3_status m3_scan_fwd_algo(int algo, const m3_dims *d,
                            const void *x, const void *B, const void *C,
                            const void *dt, const void *lam, const void *theta,

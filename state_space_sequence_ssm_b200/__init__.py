@@ -20,6 +20,12 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
 M3_F32, M3_BF16 = 0, 1
 ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
+
+
+def ALGO_TC_SEGMENTS(s: int) -> int:
+    """The tensor-core path with every sequence split into `s` segments."""
+    return ALGO_TC | (int(s) << 8)
+
 _STATUS = {0: "M3_OK", 1: "M3_ERR_INVALID_ARG", 2: "M3_ERR_UNSUPPORTED", 3: "M3_ERR_CUDA", 4: "M3_ERR_TIMEOUT"}
 
 
@@ -53,10 +59,12 @@ def _load():
     vp, dp = ctypes.c_void_p, ctypes.POINTER(Dims)
     sp = ctypes.POINTER(CState)
     lib.m3_scan_workspace_size.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.m3_scan_plan.argtypes = [ctypes.c_int, dp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_int),
+                                 ctypes.POINTER(ctypes.c_int)]
     lib.m3_scan_fwd.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     lib.m3_scan_fwd_algo.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
-    for f in (lib.m3_scan_workspace_size, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
+    for f in (lib.m3_scan_workspace_size, lib.m3_scan_plan, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
         f.restype = ctypes.c_int
     lib.m3_stream_status.argtypes = [vp]
     lib.m3_stream_status.restype = ctypes.c_int
@@ -126,10 +134,22 @@ def empty_state(Bt, H, N, P, R, device="cuda") -> State:
     return State(torch.zeros(Bt, H, N, P, **f), torch.zeros(Bt, H, R, N, **f), torch.zeros(Bt, H, R, P, **f))
 
 
-def workspace_size(dims: Dims) -> int:
-    n = ctypes.c_size_t(0)
-    _check(get_lib().m3_scan_workspace_size(ctypes.byref(dims), ctypes.byref(n)))
-    return n.value
+def workspace_size(dims: Dims, algo: int = ALGO_AUTO) -> int:
+    """Workspace bytes m3_scan_fwd_algo(algo, dims, ...) needs."""
+    return scan_plan(dims, algo)[0]
+
+
+class Plan(NamedTuple):
+    workspace_bytes: int
+    segments: int   # per sequence (1 = not split)
+    launches: int   # kernel launches of one call
+
+
+def scan_plan(dims: Dims, algo: int = ALGO_AUTO) -> Plan:
+    """How one prefill call with this `algo` runs on the current device."""
+    n, sg, ln = ctypes.c_size_t(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(get_lib().m3_scan_plan(algo, ctypes.byref(dims), ctypes.byref(n), ctypes.byref(sg), ctypes.byref(ln)))
+    return Plan(n.value, sg.value, ln.value)
 
 
 def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
@@ -146,7 +166,7 @@ def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_s
     if final is None and want_state:
         final = State(torch.empty(Bt, H, N, P, device=x.device), torch.empty(Bt, H, R, N, device=x.device),
                       torch.empty(Bt, H, R, P, device=x.device))
-    ws_need = workspace_size(dims) if algo != ALGO_SIMT else 0
+    ws_need = workspace_size(dims, algo) if algo != ALGO_SIMT else 0
     if workspace is None and ws_need:
         workspace = torch.empty(ws_need, dtype=torch.uint8, device=x.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0

@@ -14,6 +14,8 @@ namespace {
 
 thread_local std::string g_err;
 
+constexpr int kMaxForcedSegments = 4096;  // upper bound of M3_ALGO_TC_SEGMENTS(s)
+
 m3_status fail(m3_status s, const char *fmt, const char *a = nullptr) {
     char buf[512];
     std::snprintf(buf, sizeof buf, fmt, a ? a : "");
@@ -137,8 +139,12 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
                     void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream) {
     m3_status s = check_dims(d, false);
     if (s != M3_OK) return s;
+    const int segments = algo >> 8;
+    algo &= 0xff;
     if (algo != M3_ALGO_AUTO && algo != M3_ALGO_SIMT && algo != M3_ALGO_TC)
         return fail(M3_ERR_INVALID_ARG, "unknown algo");
+    if (segments < 0 || segments > kMaxForcedSegments || (segments && algo != M3_ALGO_TC))
+        return fail(M3_ERR_INVALID_ARG, "bad segment count in algo");
     const int64_t tok = d->batch * d->seqlen * d->nheads;
     Range ins[8], yr;
     int nin = 0;
@@ -164,6 +170,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
     if (fin) { p.hT = fin->h; p.bpT = fin->b_prev; p.xpT = fin->x_prev; }
     p.ws = ws;
     p.ws_bytes = ws_bytes;
+    p.segments = segments;
 
     const char *why = nullptr;
     const char *tc_why = nullptr;
@@ -194,22 +201,40 @@ int m3_version(void) { return 100; }
 
 const char *m3_last_error(void) { return g_err.c_str(); }
 
-m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes) {
+m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_bytes, int *segments, int *launches) {
     try {
         m3_status s = check_dims(d, false);
         if (s != M3_OK) return s;
-        if (!bytes) return fail(M3_ERR_INVALID_ARG, "bytes is NULL");
+        const int forced = algo >> 8;
+        const int base = algo & 0xff;
+        if (base != M3_ALGO_AUTO && base != M3_ALGO_SIMT && base != M3_ALGO_TC)
+            return fail(M3_ERR_INVALID_ARG, "unknown algo");
+        if (forced < 0 || forced > kMaxForcedSegments || (forced && base != M3_ALGO_TC))
+            return fail(M3_ERR_INVALID_ARG, "bad segment count in algo");
         m3::Problem p{};
         p.Bt = d->batch; p.T = d->seqlen; p.H = d->nheads; p.P = d->headdim; p.N = d->dstate; p.R = d->rank;
         p.bf16 = d->io == M3_BF16;
+        p.segments = forced;
         const char *why = nullptr;
-        *bytes = m3::prefill_tc_supported(p, &why) ? m3::prefill_tc_workspace(p) : 0;
+        const bool tc = base != M3_ALGO_SIMT && m3::prefill_tc_supported(p, &why);
+        if (base == M3_ALGO_TC && !tc)
+            return fail(M3_ERR_UNSUPPORTED, "%s", why ? why : "tensor-core path unsupported");
+        m3::TcPlan plan{};
+        if (tc) plan = m3::prefill_tc_plan(p);
+        if (workspace_bytes) *workspace_bytes = tc ? plan.ws_bytes : 0;
+        if (segments) *segments = tc ? plan.nseg : 1;
+        if (launches) *launches = (d->batch == 0 || d->nheads == 0) ? 0 : (tc ? plan.launches : 1);
         return M3_OK;
     } catch (const std::exception &ex) {
         return fail(M3_ERR_INVALID_ARG, "internal error: %s", ex.what());
     } catch (...) {
         return fail(M3_ERR_INVALID_ARG, "internal error");
     }
+}
+
+m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes) {
+    if (!bytes) return fail(M3_ERR_INVALID_ARG, "bytes is NULL");
+    return m3_scan_plan(M3_ALGO_AUTO, d, bytes, nullptr, nullptr);
 }
 
 m3_status m3_scan_fwd(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,

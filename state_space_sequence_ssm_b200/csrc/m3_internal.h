@@ -19,7 +19,17 @@ struct Problem {
     float *hT, *bpT, *xpT;        // nullable (no final state wanted)
     void *ws;
     size_t ws_bytes;
+    int segments;                 // tensor-core prefill: segments per sequence (0 = chosen by the library)
     cudaStream_t stream;
+};
+
+// How the tensor-core prefill runs one problem: every sequence in `nseg`
+// segments of `cpseg` chunks (nseg = 1: one CTA per sequence, one launch;
+// nseg > 1: summary pass, segment scan, main pass = three launches and a
+// workspace of ws_bytes).
+struct TcPlan {
+    int nchunks, cpseg, nseg, launches;
+    size_t ws_bytes;
 };
 
 // Each launcher returns cudaSuccess or the launch error; `why` receives a
@@ -27,6 +37,7 @@ struct Problem {
 // cudaErrorNotSupported).
 cudaError_t launch_prefill_simt(const Problem &p, const char **why);
 bool prefill_tc_supported(const Problem &p, const char **why);
+TcPlan prefill_tc_plan(const Problem &p);
 size_t prefill_tc_workspace(const Problem &p);
 cudaError_t launch_prefill_tc(const Problem &p, const char **why);
 cudaError_t launch_step(const Problem &p, const char **why);

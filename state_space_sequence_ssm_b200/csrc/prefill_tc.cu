@@ -65,6 +65,11 @@ constexpr int kNX = 3;   // x tile stages (also the number of per-chunk scalar b
 constexpr uint32_t kBarPro = 1, kBarState = 2;  // named barriers of the two warpgroups
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kPrefetchAhead = 3;  // chunks of tiles prefetched into L2 ahead of their load
+// Sequence splitting (host policy): at most kMaxSegments segments of at least
+// kMinSegChunks chunks; the summary pass costs about kSumCost of the full pass
+// per chunk and the segment scan about kScanCost chunk-times.
+constexpr int64_t kMaxSegments = 64, kMinSegChunks = 8;
+constexpr double kSumCost = 0.55, kScanCost = 2.0;
 
 template <int N, int R>
 struct Cfg {
@@ -98,12 +103,19 @@ struct Cfg {
 };
 
 struct TcArgs {
-    int64_t T, H;
+    int64_t T, H, BH;  // BH = batch * heads
     int nchunks;
+    int cpseg;         // chunks per segment (nchunks when the sequence is not split)
+    int nseg;          // segments per sequence
     const __nv_bfloat16 *x, *B, *dt, *lam, *theta;
     const float *A, *D, *h0, *bp0, *xp0;
     __nv_bfloat16 *y;
     float *hT, *bpT, *xpT;
+    // Split sequences: ws_h [nseg][BH][N][P] fp32 holds, per segment j, the
+    // summary pass's local end state (slot j + 1) and after the segment scan the
+    // pending-inclusive state entering segment j (slot j); ws_m [nseg][BH][N]
+    // holds segment j's transition exp(cA) Rot(-Phi) as (e cos, e sin) per pair.
+    float *ws_h, *ws_m;
 };
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
@@ -255,13 +267,22 @@ struct Bars {
     uint64_t *full_bc, *empty_bc, *full_x, *empty_x, *ops, *sg, *hrdy, *p, *yd, *drain, *sc;
 };
 
-template <int N, int R>
+// Pass kinds.  kWhole: the full forward pass, one CTA per sequence.
+// kSummary: the summary pass of a split sequence -- only the chunk states and
+// the carried-state chain over one segment, from a zero state (segment 0: the
+// caller's initial state), ending in the segment's local end state and its
+// transition, for the segment scan.  kSegment: the full forward pass over one
+// segment, from the scanned state.
+constexpr int kWhole = 0, kSummary = 1, kSegment = 2;
+
+template <int N, int R, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmT,
                   const TcArgs a) {
     using C = Cfg<N, R>;
     constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, G4 = C::G4, NPART = C::NPART, TPT = C::TPT, TB = C::TB;
+    constexpr bool SUM = MODE == kSummary, SEGD = MODE != kWhole;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *scal = reinterpret_cast<float *>(smem + C::OFF_SCAL);
@@ -279,10 +300,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             bars + 16};
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    // first chunk of this CTA's segment, re-read where needed (a register
+    // held across the prologue warps' loop would spill)
+    volatile int *chunk0 = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
     unsigned *err = &g_device_error;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t bh = blockIdx.x;
+    // segment-major CTA order: CTAs of neighbouring heads share dt/lam sectors
+    const uint32_t BH = SEGD ? (uint32_t)a.BH : gridDim.x;
+    const int seg = SEGD ? (int)(blockIdx.x / BH) : 0;
+    const int64_t bh = SEGD ? blockIdx.x % BH : blockIdx.x;
     const int64_t T = a.T, H = a.H;
     const int64_t b = bh / H, h = bh % H;
     auto tok = [&](int64_t t) { return (b * T + t) * H + h; };
@@ -304,6 +331,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         mbar_init(bb.yd, 1);
         mbar_init(bb.drain, 1);
         *abort_flag = 0;
+        *chunk0 = SEGD ? (int)(blockIdx.x / (uint32_t)a.BH) * a.cpseg : 0;
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -320,7 +348,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const int nchunks = a.nchunks;
+    // this CTA's chunks [cb, cb + nloc); ring stages and mbarrier phases
+    // count from the segment's first chunk (local index i)
+    const int cb = SEGD ? seg * a.cpseg : 0;
+    const int nloc = SEGD ? ((a.nchunks - cb < a.cpseg) ? a.nchunks - cb : a.cpseg) : a.nchunks;
+    auto first_chunk = [&]() { return SEGD ? *chunk0 : 0; };
 
     if (warp == kWarpTma) {
         // ============================================================ TMA producers
@@ -332,44 +364,48 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
                     tma_prefetch_5d(&tmB, kb * 64, 0, (int)h, t0, (int)b);
-                    tma_prefetch_5d(&tmC, kb * 64, 0, (int)h, t0, (int)b);
+                    if (!SUM) tma_prefetch_5d(&tmC, kb * 64, 0, (int)h, t0, (int)b);
                 }
                 tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // theta is read straight into registers
             };
             int issued = 0;
-            for (int c = 0; c < kPrefetchAhead && c < nchunks; ++c) prefetch_chunk(c);
-            for (int c = 0; c < nchunks; ++c) {
-                if (c + kPrefetchAhead < nchunks) prefetch_chunk(c + kPrefetchAhead);
-                const int s = c & 1;
-                if (c >= 2 && !mbar_wait(&bb.empty_bc[s], ((c >> 1) - 1) & 1, abort_flag, err, kErrWaitMma)) break;
+            for (int i = 0; i < kPrefetchAhead && i < nloc; ++i) prefetch_chunk(cb + i);
+            for (int i = 0; i < nloc; ++i) {
+                if (i + kPrefetchAhead < nloc) prefetch_chunk(cb + i + kPrefetchAhead);
+                const int s = i & 1;
+                if (i >= 2 && !mbar_wait(&bb.empty_bc[s], ((i >> 1) - 1) & 1, abort_flag, err, kErrWaitMma)) break;
                 uint8_t *st = smem + C::OFF_BC + s * C::BCS_BYTES;
-                const int t0 = c * Q;
-                mbar_arrive_expect_tx(&bb.full_bc[s], C::BCS_BYTES);
+                const int t0 = (cb + i) * Q;
+                mbar_arrive_expect_tx(&bb.full_bc[s], SUM ? C::BC_BYTES : C::BCS_BYTES);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
                     tma_load_5d(st + kb * 16384, &tmB, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
-                    tma_load_5d(st + C::BC_BYTES + kb * 16384, &tmC, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
+                    if (!SUM)
+                        tma_load_5d(st + C::BC_BYTES + kb * 16384, &tmC, &bb.full_bc[s], kb * 64, 0, (int)h, t0,
+                                    (int)b);
                 }
-                issued = c + 1;
+                issued = i + 1;
             }
             if (*abort_flag) {  // let the copies already in flight land before the CTA exits
-                for (int c = issued - 2 > 0 ? issued - 2 : 0; c < issued; ++c)
-                    mbar_wait(&bb.full_bc[c & 1], (c >> 1) & 1, nullptr, err, 0, 400000000LL);
+                for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
+                    mbar_wait(&bb.full_bc[i & 1], (i >> 1) & 1, nullptr, err, 0, 400000000LL);
             }
         } else if (lane == 1) {
-            // x ring (kNX stages), freed by the epilogue
+            // x ring (kNX stages), freed by the epilogue (the summary pass: by the
+            // state update, once w o X has been formed from it)
             int issued = 0;
-            for (int c = 0; c < nchunks; ++c) {
-                const int s = c % kNX;
-                if (c >= kNX && !mbar_wait(&bb.empty_x[s], ((c / kNX) - 1) & 1, abort_flag, err, kErrWaitCompute))
+            for (int i = 0; i < nloc; ++i) {
+                const int s = i % kNX;
+                if (i >= kNX && !mbar_wait(&bb.empty_x[s], ((i / kNX) - 1) & 1, abort_flag, err, kErrWaitCompute))
                     break;
                 mbar_arrive_expect_tx(&bb.full_x[s], C::X_BYTES);
-                tma_load_5d(smem + C::OFF_X + s * C::X_BYTES, &tmX, &bb.full_x[s], 0, 0, (int)h, c * Q, (int)b);
-                issued = c + 1;
+                tma_load_5d(smem + C::OFF_X + s * C::X_BYTES, &tmX, &bb.full_x[s], 0, 0, (int)h, (cb + i) * Q,
+                            (int)b);
+                issued = i + 1;
             }
             if (*abort_flag) {
-                for (int c = issued - kNX > 0 ? issued - kNX : 0; c < issued; ++c)
-                    mbar_wait(&bb.full_x[c % kNX], (c / kNX) & 1, nullptr, err, 0, 400000000LL);
+                for (int i = issued - kNX > 0 ? issued - kNX : 0; i < issued; ++i)
+                    mbar_wait(&bb.full_x[i % kNX], (i / kNX) & 1, nullptr, err, 0, 400000000LL);
             }
         }
     } else if (warp == kWarpMma) {
@@ -386,46 +422,51 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const uint32_t bc0 = smem_u32(smem + C::OFF_BC);
             const uint32_t x0 = smem_u32(smem + C::OFF_X);
             bool any = false;
-            for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1, sx = c % kNX;
+            for (int i = 0; i < nloc; ++i) {
+                const int s = i & 1, sx = i % kNX;
                 const uint32_t bs = bc0 + (uint32_t)s * C::BCS_BYTES;
                 const uint32_t cs = bs + C::BC_BYTES;
                 const uint64_t dX = sdesc_sw128(x0 + (uint32_t)sx * C::X_BYTES, 16384, 1024);  // X, MN-major
                 const uint64_t dBk = sdesc_sw128(bs, 16, 1024);     // B~, K-major
                 const uint64_t dBm = sdesc_sw128(bs, 16384, 1024);  // B~^T, MN-major
                 const uint64_t dCk = sdesc_sw128(cs, 16, 1024);     // C~, K-major
-                // S(c) as soon as the rotated tiles and w o X are in place
-                if (!mbar_wait(bb.ops, c & 1, abort_flag, err, kErrWaitCompute)) break;
+                // S(i) as soon as the rotated tiles and w o X are in place
+                if (!mbar_wait(bb.ops, i & 1, abort_flag, err, kErrWaitCompute)) break;
                 tc_fence_after();
                 any = true;
+                if (!SUM) {
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
+                    for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t o = (uint64_t)((kb * 16384 + kk * 32) >> 4);
-                        mma_bf16(tbase + kColS, dCk + o, dBk + o, idS, (kb | kk) != 0);
-                    }
-                // G(c) and Yo(c) once the state warpgroup has consumed G(c-1) and
-                // published h*_{c-1} (completion c of hrdy; the first is the initial state)
-                if (!mbar_wait(bb.hrdy, c & 1, abort_flag, err, kErrWaitCompute)) break;
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t o = (uint64_t)((kb * 16384 + kk * 32) >> 4);
+                            mma_bf16(tbase + kColS, dCk + o, dBk + o, idS, (kb | kk) != 0);
+                        }
+                }
+                // G(i) and Yo(i) once the state warpgroup has consumed G(i-1) and
+                // published h*_{i-1} (completion i of hrdy; the first is the initial state)
+                if (!mbar_wait(bb.hrdy, i & 1, abort_flag, err, kErrWaitCompute)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t o = (uint64_t)((ks * 2048) >> 4);
                     mma_bf16(tbase + kColG, dBm + o, dXw + o, idG, ks != 0);
                 }
-                const uint32_t yo = tbase + kColYo + (uint32_t)(c & 1) * 64u;
+                if (!SUM) {
+                    const uint32_t yo = tbase + kColYo + (uint32_t)(i & 1) * 64u;
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
+                    for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(yo, dCk + (uint64_t)((kb * 16384 + kk * 32) >> 4),
-                                 dHb + (uint64_t)(((kb * 4 + kk) * 2048) >> 4), idY, (kb | kk) != 0);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16(yo, dCk + (uint64_t)((kb * 16384 + kk * 32) >> 4),
+                                     dHb + (uint64_t)(((kb * 4 + kk) * 2048) >> 4), idY, (kb | kk) != 0);
+                }
                 mma_commit(bb.sg);
                 mma_commit(&bb.empty_bc[s]);  // the B/C stage is free once these MMAs are done
-                // Yd(c) = P X once P is in TMEM and the epilogue of c-1 has read Yd
-                if (!mbar_wait(bb.p, c & 1, abort_flag, err, kErrWaitCompute)) break;
-                if (c >= 1 && !mbar_wait(&bb.empty_x[(c - 1) % kNX], ((c - 1) / kNX) & 1, abort_flag, err,
+                if (SUM) continue;
+                // Yd(i) = P X once P is in TMEM and the epilogue of i-1 has read Yd
+                if (!mbar_wait(bb.p, i & 1, abort_flag, err, kErrWaitCompute)) break;
+                if (i >= 1 && !mbar_wait(&bb.empty_x[(i - 1) % kNX], ((i - 1) / kNX) & 1, abort_flag, err,
                                          kErrWaitCompute))
                     break;
                 tc_fence_after();
@@ -473,10 +514,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                                : make_uint2(0u, 0u);
             }
         };
-        prefetch_scalars(0);
-        prefetch_theta(0);
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1, sx = c % kNX;
+        prefetch_scalars((int64_t)cb * Q);
+        prefetch_theta((int64_t)cb * Q);
+        for (int lc = 0; lc < nloc; ++lc) {
+            const int s = lc & 1, sx = lc % kNX;
             float *cAl2 = sbuf + sx * C::SB;
             float *gam = cAl2 + Q;
             float *ghat = gam + Q;
@@ -486,8 +527,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             uint8_t *bst = smem + C::OFF_BC + s * C::BCS_BYTES;
             uint8_t *cst = bst + C::BC_BYTES;
             uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
-            // the scalar buffer c % kNX is free once the epilogue of c - kNX is done
-            if (c >= kNX && bar_any<kBarPro, kPro>(!mbar_wait(&bb.empty_x[sx], ((c / kNX) - 1) & 1, abort_flag,
+            // the scalar buffer lc % kNX is free once the epilogue of lc - kNX is done
+            if (lc >= kNX && bar_any<kBarPro, kPro>(!mbar_wait(&bb.empty_x[sx], ((lc / kNX) - 1) & 1, abort_flag,
                                                               err, kErrWaitCompute)))
                 break;
 
@@ -496,7 +537,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             {
                 const float d = bf16_bits(pd), l = bf16_bits(pl);
                 const float nx = (1.f - bf16_bits(pl1)) * bf16_bits(pd1);  // 0 past the sequence end
-                if (c + 1 < nchunks) prefetch_scalars((int64_t)(c + 1) * Q);
+                if (lc + 1 < nloc) prefetch_scalars((int64_t)(first_chunk() + lc + 1) * Q);
                 if (tid < Q) {
                     dts[tid] = d;
                     gam[tid] = l * d;
@@ -542,7 +583,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
                 *reinterpret_cast<float4 *>(phis + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
                 // the B/C tiles of this chunk
-                if (bar_any<kBarPro, kPro>(!mbar_wait(&bb.full_bc[s], (c >> 1) & 1, abort_flag, err, kErrWaitTma)))
+                if (bar_any<kBarPro, kPro>(!mbar_wait(&bb.full_bc[s], (lc >> 1) & 1, abort_flag, err, kErrWaitTma)))
                     break;
                 float phi[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int q = 0; q < part; ++q) {
@@ -566,7 +607,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         for (int r = 0; r < R; ++r) {
                             const uint32_t off = kbo + sw128((uint32_t)(i * R + r), jchunk);
                             vb[jj][r] = *reinterpret_cast<const uint4 *>(bst + off);
-                            vc[jj][r] = *reinterpret_cast<const uint4 *>(cst + off);
+                            if (!SUM) vc[jj][r] = *reinterpret_cast<const uint4 *>(cst + off);
                         }
                     }
 #pragma unroll
@@ -589,17 +630,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
                         for (int r = 0; r < R; ++r) {
                             const uint32_t off = kbo + sw128((uint32_t)(i * R + r), jchunk);
-                            uint4 b4 = vb[jj][r], c4 = vc[jj][r];
+                            uint4 b4 = vb[jj][r];
                             b4.x = rot_pair(b4.x, cc[0], nss[0]);
                             b4.y = rot_pair(b4.y, cc[1], nss[1]);
                             b4.z = rot_pair(b4.z, cc[2], nss[2]);
                             b4.w = rot_pair(b4.w, cc[3], nss[3]);
-                            c4.x = rot_pair(c4.x, cc[0], nss[0]);
-                            c4.y = rot_pair(c4.y, cc[1], nss[1]);
-                            c4.z = rot_pair(c4.z, cc[2], nss[2]);
-                            c4.w = rot_pair(c4.w, cc[3], nss[3]);
                             *reinterpret_cast<uint4 *>(bst + off) = b4;
-                            *reinterpret_cast<uint4 *>(cst + off) = c4;
+                            if (!SUM) {
+                                uint4 c4 = vc[jj][r];
+                                c4.x = rot_pair(c4.x, cc[0], nss[0]);
+                                c4.y = rot_pair(c4.y, cc[1], nss[1]);
+                                c4.z = rot_pair(c4.z, cc[2], nss[2]);
+                                c4.w = rot_pair(c4.w, cc[3], nss[3]);
+                                *reinterpret_cast<uint4 *>(cst + off) = c4;
+                            }
                         }
                     }
                 }
@@ -612,12 +656,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         sinE[4 * g + e] = sn;
                     }
                 }
-                if (c + 1 < nchunks) prefetch_theta((int64_t)(c + 1) * Q);
+                if (lc + 1 < nloc) prefetch_theta((int64_t)(first_chunk() + lc + 1) * Q);
             }
             // ---- C. w o X (chunk-state weights on the value rows), once G(c-1)
             //      has finished reading the previous w o X and x of chunk c is in
-            if (bar_any<kBarPro, kPro>((c >= 1 && !mbar_wait(bb.sg, (c - 1) & 1, abort_flag, err, kErrWaitMma)) ||
-                                       !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma)))
+            if (bar_any<kBarPro, kPro>((lc >= 1 && !mbar_wait(bb.sg, (lc - 1) & 1, abort_flag, err, kErrWaitMma)) ||
+                                       !mbar_wait(&bb.full_x[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitTma)))
                 break;
             {
                 const int row = tid >> 1, j0 = (tid & 1) * 4;  // half a row per thread
@@ -657,33 +701,46 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
         const int c0 = 32 * hf;            // first column of this thread's half
         float hreg[32];
-        // initial state h0 + beta'_0 b_prev x_prev^T (pending write of token -1)
+        // Pending-inclusive state entering the segment.  The whole sequence and
+        // segment 0 of the summary pass: the caller's h0 + beta'_0 b_prev
+        // x_prev^T (pending write of token -1); later summary segments: zero
+        // (their local state); segments of the main pass: the scanned state.
         {
-            const float betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
 #pragma unroll
             for (int p = 0; p < 32; ++p) hreg[p] = 0.f;
-            if (own_state) {
-                if (a.h0) {
+            if (MODE == kSegment) {
+                if (own_state) {
+                    const float *hin = a.ws_h + ((int64_t)seg * BH + bh) * N * kP;
 #pragma unroll
-                    for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * N + srow) * kP + c0 + p];
+                    for (int p = 0; p < 32; ++p) hreg[p] = hin[srow * kP + c0 + p];
                 }
-                if (a.bp0 && a.xp0) {
-                    for (int r = 0; r < R; ++r) {
-                        const float cb = betap0 * a.bp0[(bh * R + r) * N + srow];
+            } else if (seg == 0) {
+                const float betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
+                if (own_state) {
+                    if (a.h0) {
 #pragma unroll
-                        for (int p = 0; p < 32; ++p)
-                            hreg[p] = fmaf(cb, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
+                        for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * N + srow) * kP + c0 + p];
+                    }
+                    if (a.bp0 && a.xp0) {
+                        for (int r = 0; r < R; ++r) {
+                            const float cw = betap0 * a.bp0[(bh * R + r) * N + srow];
+#pragma unroll
+                            for (int p = 0; p < 32; ++p)
+                                hreg[p] = fmaf(cw, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
+                        }
                     }
                 }
-                store_state_half(hbuf, srow, hf, hreg);
             }
+            if (!SUM && own_state) store_state_half(hbuf, srow, hf, hreg);
         }
+        // summary pass: the segment's transition exp(cA) Rot(-Phi) on this row's pair
+        float m_l2 = 0.f, m_cs = 1.f, m_sn = 0.f;
         fence_proxy_async_smem();
         named_bar(kBarState, kSt);
         if (lt == 0) mbar_arrive(bb.hrdy);
         bool ok = true;
-        for (int c = 0; c < nchunks; ++c) {
-            const int sx = c % kNX;
+        for (int lc = 0; lc < nloc; ++lc) {
+            const int sx = lc % kNX;
             const float *cAl2 = sbuf + sx * C::SB;
             const float *gam = cAl2 + Q;
             const float *ghat = gam + Q;
@@ -692,9 +749,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const float *sinE = cosE + K2;
             const uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
             // scalars of chunk c (release/acquire through sc), its x tile, and G(c)
-            if (bar_any<kBarState, kSt>(!mbar_wait(&bb.sc[sx], (c / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
-                                        !mbar_wait(&bb.full_x[sx], (c / kNX) & 1, abort_flag, err, kErrWaitTma) ||
-                                        !mbar_wait(bb.sg, c & 1, abort_flag, err, kErrWaitMma))) {
+            if (bar_any<kBarState, kSt>(!mbar_wait(&bb.sc[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
+                                        !mbar_wait(&bb.full_x[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitTma) ||
+                                        !mbar_wait(bb.sg, lc & 1, abort_flag, err, kErrWaitMma))) {
                 ok = false;
                 break;
             }
@@ -714,12 +771,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const float o = __shfl_xor_sync(0xffffffffu, u, 1);
                     hreg[p] = fmaf(u, cs, o * sgn);
                 }
-                if (own_state) store_state_half(hbuf, srow, hf, hreg);
+                if (SUM) {
+                    m_l2 += cAl2[Q - 1];
+                    const float ncs = m_cs * cs - m_sn * sn;
+                    m_sn = fmaf(m_sn, cs, m_cs * sn);
+                    m_cs = ncs;
+                } else if (own_state) {
+                    store_state_half(hbuf, srow, hf, hreg);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarState, kSt);
-            if (lt == 0) mbar_arrive(bb.hrdy);
+            if (lt == 0) {
+                mbar_arrive(bb.hrdy);
+                if (SUM) mbar_arrive(&bb.empty_x[sx]);  // x tile and scalars consumed
+            }
+            if (SUM) continue;
 
             // ---- D. decay mask S -> P (TMEM): half 0 takes column blocks 0 and 3,
             //      half 1 blocks 1 and 2 (balances the lower triangle)
@@ -729,7 +797,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (lt == 0) mbar_arrive(bb.p);
 
             // ---- F. epilogue: y = Yd + exp(cA_t) Yo + D x, this thread's 32 columns
-            if (bar_any<kBarState, kSt>(!mbar_wait(bb.yd, c & 1, abort_flag, err, kErrWaitMma))) {
+            if (bar_any<kBarState, kSt>(!mbar_wait(bb.yd, lc & 1, abort_flag, err, kErrWaitMma))) {
                 ok = false;
                 break;
             }
@@ -737,9 +805,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             {
                 const int row = lq;
                 const int ti = row / R, r = row % R;
-                const int64_t t = (int64_t)c * Q + ti;
+                const int64_t t = (int64_t)(first_chunk() + lc) * Q + ti;
                 const float sc = ex2(cAl2[ti]);
-                const uint32_t yo = kColYo + (uint32_t)(c & 1) * 64u;
+                const uint32_t yo = kColYo + (uint32_t)(lc & 1) * 64u;
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
                     float yd[16], yv[16];
@@ -771,8 +839,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             named_bar(kBarState, kSt);
             if (lt == 0) mbar_arrive(&bb.empty_x[sx]);
         }
-        // ---- final state: plain-frame h_{T-1}, raw last token as the pending term
-        if (ok) {
+        if (SUM) {
+            // ---- summary: the segment's local end state (pending-inclusive) into
+            //      slot seg + 1, its transition exp(cA) Rot(-Phi) per pair
+            if (ok && own_state) {
+                float4 *dst = reinterpret_cast<float4 *>(a.ws_h + (((int64_t)seg + 1) * BH + bh) * N * kP +
+                                                         srow * kP + c0);
+#pragma unroll
+                for (int p = 0; p < 8; ++p)
+                    dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
+                if (hf == 0 && (srow & 1) == 0) {
+                    const float e = ex2(m_l2);
+                    *reinterpret_cast<float2 *>(a.ws_m + ((int64_t)seg * BH + bh) * N + srow) =
+                        make_float2(e * m_cs, e * m_sn);
+                }
+            }
+        } else if (ok && (!SEGD || seg == a.nseg - 1)) {
+            // ---- final state: plain-frame h_{T-1}, raw last token as the pending term
             if (a.hT && own_state) {
                 float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * N + srow) * kP + c0);
 #pragma unroll
@@ -791,6 +874,70 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- segment scan
+// Exclusive scan over the segments of each split sequence, element-wise on the
+// N x P state: slot 0 <- h0 + beta'_0 b_prev x_prev^T (the pending-inclusive
+// state before token 0); slot 1 already holds segment 0's end state (its
+// summary pass started from the caller's state); slot j >= 2 <- M_{j-1}
+// slot(j-1) + slot j, M_{j-1} = exp(cA) Rot(-Phi) of segment j-1.  The same
+// linear recurrence as the carried state between chunks, one level up.
+struct ScanArgs {
+    int64_t BH, H, T;
+    int nseg;
+    const __nv_bfloat16 *dt, *lam;
+    const float *h0, *bp0, *xp0;
+    float *ws_h;
+    const float *ws_m;
+};
+
+template <int N, int R>
+__global__ void __launch_bounds__(256) segment_scan_kernel(const ScanArgs a) {
+    constexpr int QD = kP / 4;  // column quads of a state row
+    const int64_t bh = blockIdx.x;
+    const int64_t b = bh / a.H, h = bh % a.H;
+    const bool pend = a.bp0 && a.xp0;
+    const int64_t t0 = (b * a.T) * a.H + h;  // token 0 of this sequence
+    const float betap0 = pend ? (1.f - bf(a.lam, t0)) * bf(a.dt, t0) : 0.f;
+    const int64_t slot = a.BH * N * kP;
+    float *base = a.ws_h + bh * N * kP;
+    for (int it = threadIdx.x; it < (N / 2) * QD; it += blockDim.x) {
+        const int k = it / QD, col = 4 * (it % QD);
+        const int ru = 2 * k, rv = 2 * k + 1;
+        float4 u = make_float4(0.f, 0.f, 0.f, 0.f), v = u;
+        if (a.h0) {
+            u = *reinterpret_cast<const float4 *>(a.h0 + (bh * N + ru) * kP + col);
+            v = *reinterpret_cast<const float4 *>(a.h0 + (bh * N + rv) * kP + col);
+        }
+        if (pend) {
+            for (int r = 0; r < R; ++r) {
+                const float wu = betap0 * a.bp0[(bh * R + r) * N + ru];
+                const float wv = betap0 * a.bp0[(bh * R + r) * N + rv];
+                const float4 xq = *reinterpret_cast<const float4 *>(a.xp0 + (bh * R + r) * kP + col);
+                u = make_float4(fmaf(wu, xq.x, u.x), fmaf(wu, xq.y, u.y), fmaf(wu, xq.z, u.z), fmaf(wu, xq.w, u.w));
+                v = make_float4(fmaf(wv, xq.x, v.x), fmaf(wv, xq.y, v.y), fmaf(wv, xq.z, v.z), fmaf(wv, xq.w, v.w));
+            }
+        }
+        *reinterpret_cast<float4 *>(base + ru * kP + col) = u;
+        *reinterpret_cast<float4 *>(base + rv * kP + col) = v;
+        if (a.nseg < 2) continue;
+        u = *reinterpret_cast<const float4 *>(base + slot + ru * kP + col);
+        v = *reinterpret_cast<const float4 *>(base + slot + rv * kP + col);
+        for (int j = 2; j < a.nseg; ++j) {
+            const float2 m = *reinterpret_cast<const float2 *>(a.ws_m + ((int64_t)(j - 1) * a.BH + bh) * N + ru);
+            float *pu = base + j * slot + ru * kP + col, *pv = base + j * slot + rv * kP + col;
+            const float4 cu = *reinterpret_cast<const float4 *>(pu), cv = *reinterpret_cast<const float4 *>(pv);
+            const float4 nu = make_float4(fmaf(m.x, u.x, fmaf(m.y, v.x, cu.x)), fmaf(m.x, u.y, fmaf(m.y, v.y, cu.y)),
+                                          fmaf(m.x, u.z, fmaf(m.y, v.z, cu.z)), fmaf(m.x, u.w, fmaf(m.y, v.w, cu.w)));
+            const float4 nv = make_float4(fmaf(m.x, v.x, fmaf(-m.y, u.x, cv.x)), fmaf(m.x, v.y, fmaf(-m.y, u.y, cv.y)),
+                                          fmaf(m.x, v.z, fmaf(-m.y, u.z, cv.z)), fmaf(m.x, v.w, fmaf(-m.y, u.w, cv.w)));
+            *reinterpret_cast<float4 *>(pu) = nu;
+            *reinterpret_cast<float4 *>(pv) = nv;
+            u = nu;
+            v = nv;
+        }
     }
 }
 
@@ -840,8 +987,19 @@ bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int N, int R, int MODE>
+cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc, const CUtensorMap &mt,
+                        const TcArgs &a, int64_t ctas, cudaStream_t stream) {
+    using C = Cfg<N, R>;
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    prefill_tc_kernel<N, R, MODE><<<(unsigned)ctas, kThreads, C::SMEM_BYTES, stream>>>(mx, mb, mc, mt, a);
+    return cudaGetLastError();
+}
+
 template <int N, int R>
-cudaError_t launch_nr(const Problem &p, const char **why) {
+cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     using C = Cfg<N, R>;
     CUtensorMap mx, mb, mc, mt;
     if (!make_map(&mx, p.x, kP, R, p.H, p.T, p.Bt, C::Q) || !make_map(&mb, p.B, N, R, p.H, p.T, p.Bt, C::Q) ||
@@ -849,10 +1007,14 @@ cudaError_t launch_nr(const Problem &p, const char **why) {
         *why = "tensor-core prefill: TMA descriptor encoding failed";
         return cudaErrorNotSupported;
     }
-    TcArgs a;
+    const int64_t BH = p.Bt * p.H;
+    TcArgs a{};
     a.T = p.T;
     a.H = p.H;
-    a.nchunks = (int)((p.T + C::Q - 1) / C::Q);
+    a.BH = BH;
+    a.nchunks = plan.nchunks;
+    a.cpseg = plan.cpseg;
+    a.nseg = plan.nseg;
     a.x = (const __nv_bfloat16 *)p.x;
     a.B = (const __nv_bfloat16 *)p.B;
     a.dt = (const __nv_bfloat16 *)p.dt;
@@ -863,15 +1025,39 @@ cudaError_t launch_nr(const Problem &p, const char **why) {
     a.h0 = p.h0;
     a.bp0 = p.bp0;
     a.xp0 = p.xp0;
+    if (plan.nseg == 1) {
+        a.y = (__nv_bfloat16 *)p.y;
+        a.hT = p.hT;
+        a.bpT = p.bpT;
+        a.xpT = p.xpT;
+        return launch_pass<N, R, kWhole>(mx, mb, mc, mt, a, BH, p.stream);
+    }
+    // split sequences: summary pass over segments 0 .. nseg-2, segment scan,
+    // then the main pass over all segments from the scanned states
+    a.ws_h = static_cast<float *>(p.ws);
+    a.ws_m = a.ws_h + (size_t)plan.nseg * BH * N * kP;
+    cudaError_t e = launch_pass<N, R, kSummary>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
+    if (e != cudaSuccess) return e;
+    ScanArgs sa{};
+    sa.BH = BH;
+    sa.H = p.H;
+    sa.T = p.T;
+    sa.nseg = plan.nseg;
+    sa.dt = a.dt;
+    sa.lam = a.lam;
+    sa.h0 = p.h0;
+    sa.bp0 = p.bp0;
+    sa.xp0 = p.xp0;
+    sa.ws_h = a.ws_h;
+    sa.ws_m = a.ws_m;
+    segment_scan_kernel<N, R><<<(unsigned)BH, 256, 0, p.stream>>>(sa);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    a.h0 = a.bp0 = a.xp0 = nullptr;  // the main pass reads only the scanned states
     a.y = (__nv_bfloat16 *)p.y;
     a.hT = p.hT;
     a.bpT = p.bpT;
     a.xpT = p.xpT;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    prefill_tc_kernel<N, R><<<(unsigned)(p.Bt * p.H), kThreads, C::SMEM_BYTES, p.stream>>>(mx, mb, mc, mt, a);
-    return cudaGetLastError();
+    return launch_pass<N, R, kSegment>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream);
 }
 
 bool device_is_sm100() {
@@ -895,17 +1081,61 @@ bool prefill_tc_supported(const Problem &p, const char **why) {
     return true;
 }
 
-size_t prefill_tc_workspace(const Problem &) { return 0; }
+TcPlan prefill_tc_plan(const Problem &p) {
+    TcPlan plan{};
+    const int64_t Q = kRows / p.R;
+    const int64_t nch = (p.T + Q - 1) / Q;
+    const int64_t BH = p.Bt * p.H;
+    int64_t S = 1;
+    if (p.segments > 0) {
+        S = p.segments;
+    } else {
+        // Split a sequence only when it shortens the estimated critical path:
+        // waves of one CTA per SM, a summary chunk costing kSumCost of a full
+        // one, segments of at least kMinSegChunks chunks.
+        int dev = 0, nsm = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (nsm < 1) nsm = 1;
+        auto waves = [&](int64_t ctas) { return (double)((ctas + nsm - 1) / nsm); };
+        double best = waves(BH) * (double)nch;
+        for (int64_t s = 2; s <= kMaxSegments && s * kMinSegChunks <= nch; ++s) {
+            const int64_t L = (nch + s - 1) / s, Se = (nch + L - 1) / L;
+            if (Se != s) continue;
+            const double cost = waves(BH * Se) * L + waves(BH * (Se - 1)) * L * kSumCost + kScanCost;
+            if (cost < best * 0.97) {
+                best = cost;
+                S = s;
+            }
+        }
+    }
+    if (S > nch) S = nch;
+    if (S < 1) S = 1;
+    const int64_t L = (nch + S - 1) / S;
+    S = (nch + L - 1) / L;  // no empty segment
+    plan.nchunks = (int)nch;
+    plan.cpseg = (int)L;
+    plan.nseg = (int)S;
+    plan.launches = S > 1 ? 3 : 1;
+    plan.ws_bytes = S > 1 ? (size_t)S * BH * p.N * (p.P + 1) * sizeof(float) : 0;
+    return plan;
+}
+
+size_t prefill_tc_workspace(const Problem &p) { return prefill_tc_plan(p).ws_bytes; }
 
 cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
-    if (p.N == 128) {
-        if (p.R == 1) return launch_nr<128, 1>(p, why);
-        if (p.R == 2) return launch_nr<128, 2>(p, why);
-        return launch_nr<128, 4>(p, why);
+    const TcPlan plan = prefill_tc_plan(p);
+    if (plan.nseg > 1 && (!p.ws || p.ws_bytes < plan.ws_bytes)) {
+        *why = "tensor-core prefill: workspace too small for the split sequence";
+        return cudaErrorNotSupported;
     }
-    if (p.R == 1) return launch_nr<64, 1>(p, why);
-    if (p.R == 2) return launch_nr<64, 2>(p, why);
-    return launch_nr<64, 4>(p, why);
+    if (p.N == 128) {
+        if (p.R == 1) return launch_nr<128, 1>(p, plan, why);
+        if (p.R == 2) return launch_nr<128, 2>(p, plan, why);
+        return launch_nr<128, 4>(p, plan, why);
+    }
+    if (p.R == 1) return launch_nr<64, 1>(p, plan, why);
+    if (p.R == 2) return launch_nr<64, 2>(p, plan, why);
+    return launch_nr<64, 4>(p, plan, why);
 }
 
 cudaError_t read_device_error(unsigned *code, cudaStream_t stream) {

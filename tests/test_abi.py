@@ -131,3 +131,25 @@ def test_workspace_query_is_host_only(m3):
 
 def test_version(m3):
     assert m3.lib.m3_version() == 100
+
+
+def test_segment_count_only_with_tc(m3):
+    # a segment count belongs to the tensor-core choice only; out-of-range counts are refused
+    assert call_scan(m3, dims(m3, io=1), algo=m3.ALGO_SIMT | (3 << 8)) == 1
+    assert call_scan(m3, dims(m3, io=1), algo=m3.ALGO_AUTO | (3 << 8)) == 1
+    assert call_scan(m3, dims(m3, io=1), algo=m3.ALGO_TC_SEGMENTS(5000)) == 1
+    assert "segment" in m3.lib.m3_last_error().decode()
+
+
+def test_scan_plan_host_side(m3):
+    size, segs, launches = ctypes.c_size_t(7), ctypes.c_int(7), ctypes.c_int(7)
+    d = dims(m3, io=0)
+    assert m3.lib.m3_scan_plan(m3.ALGO_AUTO, ctypes.byref(d), ctypes.byref(size), ctypes.byref(segs),
+                               ctypes.byref(launches)) == 0
+    assert (size.value, segs.value, launches.value) == (0, 1, 1)  # fp32 I/O: one SIMT launch, no workspace
+    z = dims(m3, Bt=0, io=0)
+    assert m3.lib.m3_scan_plan(m3.ALGO_SIMT, ctypes.byref(z), None, None, ctypes.byref(launches)) == 0
+    assert launches.value == 0
+    assert m3.lib.m3_scan_plan(m3.ALGO_TC, ctypes.byref(d), None, None, None) == 2  # TC refuses fp32 I/O
+    assert m3.lib.m3_scan_plan(9, ctypes.byref(d), None, None, None) == 1
+    assert m3.lib.m3_scan_plan(m3.ALGO_AUTO, None, None, None, None) == 1
