@@ -20,17 +20,22 @@
 // h*_c = Rot(-Phi_c)(exp(cA_end) h*_{c-1} + G), the carried state kept in
 // fp32 registers in the plain frame (no angle exceeds one chunk's sum).
 //
-// Warp roles (320 threads), pipelined across chunks:
-//   warps 0-3  prologue warpgroup: per-token scalars, cumulative angles, the
-//              in-place rotation of the B and C tiles, and w o X;
-//   warps 4-7  state warpgroup: the carried state update, the decay mask
-//              S -> P (written to TMEM, the A operand of Yd) and the
-//              epilogue (about one chunk behind warps 0-3);
-//   warp 8     TMA producers: lane 0 fills a 2-stage ring of B and C tiles
-//              (freed as soon as S, G and Yo have read them), lane 1 a
-//              3-stage ring of x tiles (freed after the epilogue), both
-//              128B-swizzled, with L2 prefetches of the chunks ahead;
-//   warp 9     TMEM owner and single-thread MMA issuer.
+// Warp roles (576 threads: 18 warps of 96 registers), pipelined across chunks:
+//   warps 0-7   prologue: per-token scalars and the chunk-local scan of dt*A,
+//               cumulative angles, the in-place rotation of the B and C
+//               tiles, and w o X;
+//   warps 8-15  state: the carried state update, the decay mask S -> P
+//               (written to TMEM, the A operand of Yd) and the epilogue
+//               (about one chunk behind the prologue); each thread owns one
+//               TMEM lane (row) and one 32-column half;
+//   warp 16     TMA producers: lane 0 fills a 2-stage ring of B and C tiles
+//               (freed as soon as S, G and Yo have read them), lane 1 a
+//               3-stage ring of x tiles (freed after the epilogue), both
+//               128B-swizzled, with L2 prefetches of the chunks ahead;
+//   warp 17     TMEM owner and single-thread MMA issuer.
+// A sequence too long for the grid to fill the GPU is split into segments
+// (a summary pass, a scan over the segments, then this pass per segment:
+// the MODE template argument).
 // Every wait is bounded; a wait that gives up records a code that the host
 // reads back with m3_stream_status() and the CTA drains and returns.
 #include <cuda.h>
