@@ -152,6 +152,28 @@ M3_API m3_status m3_scan_fwd_algo(int algo, const m3_dims *d,
                            const m3_state *init, void *y, const m3_state *final_state,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* m3_scan_fwd_algo without a workspace argument: the per-segment states of
+ * split sequences go to a scratch area the library itself holds in device
+ * memory (a static 24 MiB array, reserved on each device when the library's
+ * code is loaded there).  The pages have no counterpart to this entry point;
+ * it exists for callers that cannot hand over device memory.
+ *   - Size limit: the library's own segment choice is capped so that it fits
+ *     the 24 MiB; a forced M3_ALGO_TC_SEGMENTS(s) whose states would not fit
+ *     returns M3_ERR_UNSUPPORTED.
+ *   - Nothing in the scratch needs to start at zero: every value a call reads
+ *     there was written earlier in the same call.
+ *   - Calls that may overlap in time on one device (other streams, other host
+ *     threads) race on the single scratch area: serialise them.
+ *   - The first call on each device looks the scratch address up
+ *     (cudaGetSymbolAddress): make one call outside CUDA-graph stream capture
+ *     before capturing calls to this entry point. */
+M3_API m3_status m3_scan_fwd_static(int algo, const m3_dims *d,
+                             const void *x, const void *B, const void *C,
+                             const void *dt, const void *lam, const void *theta,
+                             const float *A, const float *D,
+                             const m3_state *init, void *y, const m3_state *final_state,
+                             void *stream);
+
 /* Decode: one token per (batch, head) against a resident state, updated in
  * place (the recurrent form of the same method, one token at a time).
  * x [batch,nheads,rank,headdim], B/C [batch,nheads,rank,dstate],

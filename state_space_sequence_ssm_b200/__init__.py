@@ -63,6 +63,8 @@ def _load():
                                  ctypes.POINTER(ctypes.c_int)]
     lib.m3_scan_fwd.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     lib.m3_scan_fwd_algo.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_scan_fwd_static.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp]
+    lib.m3_scan_fwd_static.restype = ctypes.c_int
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
     for f in (lib.m3_scan_workspace_size, lib.m3_scan_plan, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
         f.restype = ctypes.c_int
@@ -173,6 +175,24 @@ def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_s
     _check(get_lib().m3_scan_fwd_algo(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
                                 _cstate(init), _ptr(y), _cstate(final), _ptr(workspace), ws_bytes,
                                 _stream(stream)))
+    return y, final
+
+
+def scan_fwd_static(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
+                    y=None, final: State | None = None, algo: int = ALGO_AUTO, stream=None):
+    """scan_fwd without a workspace: split sequences use the library's own
+    device scratch (see m3_scan_fwd_static in include/m3.h for its limits)."""
+    _require_cuda(x, B, C, dt, lam, theta, A, D, y)
+    Bt, T, H, R, P = x.shape
+    N = B.shape[-1]
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype)
+    if y is None:
+        y = torch.empty_like(x)
+    if final is None and want_state:
+        final = State(torch.empty(Bt, H, N, P, device=x.device), torch.empty(Bt, H, R, N, device=x.device),
+                      torch.empty(Bt, H, R, P, device=x.device))
+    _check(get_lib().m3_scan_fwd_static(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
+                                        _cstate(init), _ptr(y), _cstate(final), _stream(stream)))
     return y, final
 
 

@@ -136,7 +136,8 @@ m3::Problem make_problem(const m3_dims *d, const void *x, const void *B, const v
 
 m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
                     const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
-                    void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream) {
+                    void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream,
+                    bool static_ws = false) {
     m3_status s = check_dims(d, false);
     if (s != M3_OK) return s;
     const int segments = algo >> 8;
@@ -183,9 +184,22 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
         use_tc = tc_ok;
     }
     if (use_tc) {
-        const size_t need = m3::prefill_tc_workspace(p);
-        if (need > ws_bytes || (need && !ws))
-            return fail(M3_ERR_INVALID_ARG, "workspace too small (query m3_scan_workspace_size)");
+        if (static_ws) {
+            p.ws_cap = m3::static_scratch_bytes();
+            const size_t need = m3::prefill_tc_workspace(p);
+            if (need > p.ws_cap)
+                return fail(M3_ERR_UNSUPPORTED,
+                            "m3_scan_fwd_static: this segment count needs more than the library's 24 MiB scratch "
+                            "(use m3_scan_fwd_algo with a workspace)");
+            if (need) {
+                const cudaError_t e = m3::static_scratch(&p.ws, &p.ws_bytes);
+                if (e != cudaSuccess) return cuda_fail(e, "m3_scan_fwd_static (scratch address)");
+            }
+        } else {
+            const size_t need = m3::prefill_tc_workspace(p);
+            if (need > ws_bytes || (need && !ws))
+                return fail(M3_ERR_INVALID_ARG, "workspace too small (query m3_scan_workspace_size)");
+        }
     }
     cudaError_t e = use_tc ? m3::launch_prefill_tc(p, &why) : m3::launch_prefill_simt(p, &why);
     if (e == cudaErrorNotSupported && why) return fail(M3_ERR_UNSUPPORTED, "%s", why);
@@ -256,6 +270,16 @@ m3_status m3_scan_fwd_algo(int algo, const m3_dims *d, const void *x, const void
     try {
         return scan_impl(algo, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace,
                          workspace_bytes, stream);
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
+m3_status m3_scan_fwd_static(int algo, const m3_dims *d, const void *x, const void *B, const void *C,
+                             const void *dt, const void *lam, const void *theta, const float *A, const float *D,
+                             const m3_state *init, void *y, const m3_state *final_state, void *stream) {
+    try {
+        return scan_impl(algo, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, nullptr, 0, stream, true);
     } catch (...) {
         return fail(M3_ERR_INVALID_ARG, "internal error");
     }

@@ -20,6 +20,7 @@ struct Problem {
     void *ws;
     size_t ws_bytes;
     int segments;                 // tensor-core prefill: segments per sequence (0 = chosen by the library)
+    size_t ws_cap;                // > 0: the library's choice of segments must fit this workspace
     cudaStream_t stream;
 };
 
@@ -41,6 +42,10 @@ TcPlan prefill_tc_plan(const Problem &p);
 size_t prefill_tc_workspace(const Problem &p);
 cudaError_t launch_prefill_tc(const Problem &p, const char **why);
 cudaError_t launch_step(const Problem &p, const char **why);
+// The library's own device scratch for m3_scan_fwd_static: its address on the
+// current device (looked up once per device) and its size.
+cudaError_t static_scratch(void **ptr, size_t *bytes);
+size_t static_scratch_bytes();
 // Synchronise `stream`, then read and clear the device error word that the
 // tensor-core kernel's bounded waits set when they give up.
 cudaError_t read_device_error(unsigned *code, cudaStream_t stream);

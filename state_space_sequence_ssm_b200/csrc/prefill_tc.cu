@@ -52,6 +52,12 @@ namespace m3 {
 // read_device_error() on the host.
 __device__ unsigned g_device_error;
 
+// Scratch of m3_scan_fwd_static (per-segment states of split sequences), so
+// that entry point needs no caller workspace.  24 MiB covers the split of a
+// 64-sequence, 65,536-token, N = 128 problem (about 19 MiB).
+constexpr size_t kStaticScratchBytes = size_t(24) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
 namespace {
 using namespace tc;
 
@@ -1106,6 +1112,7 @@ TcPlan prefill_tc_plan(const Problem &p) {
         for (int64_t s = 2; s <= kMaxSegments && s * kMinSegChunks <= nch; ++s) {
             const int64_t L = (nch + s - 1) / s, Se = (nch + L - 1) / L;
             if (Se != s) continue;
+            if (p.ws_cap && (size_t)Se * BH * p.N * (p.P + 1) * sizeof(float) > p.ws_cap) break;
             const double cost = waves(BH * Se) * L + waves(BH * (Se - 1)) * L * kSumCost + kScanCost;
             if (cost < best * 0.97) {
                 best = cost;
@@ -1141,6 +1148,27 @@ cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
     if (p.R == 1) return launch_nr<64, 1>(p, plan, why);
     if (p.R == 2) return launch_nr<64, 2>(p, plan, why);
     return launch_nr<64, 4>(p, plan, why);
+}
+
+size_t static_scratch_bytes() { return kStaticScratchBytes; }
+
+cudaError_t static_scratch(void **ptr, size_t *bytes) {
+    static std::mutex mu;
+    static void *addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    *bytes = kStaticScratchBytes;
+    return cudaSuccess;
 }
 
 cudaError_t read_device_error(unsigned *code, cudaStream_t stream) {
