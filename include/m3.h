@@ -196,6 +196,14 @@ M3_API m3_status m3_step(const m3_dims *d,
  * instead of a hang. */
 M3_API m3_status m3_stream_status(void *stream);
 
+/* Failure-path self-test: queues on `stream` one kernel whose bounded
+ * device-side wait is made to give up (about 1 ms; nothing ever completes the
+ * awaited phase).  The next m3_stream_status on that stream then returns
+ * M3_ERR_TIMEOUT, and the device stays usable: the same path a stuck wait in
+ * the prefill or decode kernels takes, without a fault, trap or hang.  The
+ * pages have no counterpart to this call. */
+M3_API m3_status m3_selftest_wait_timeout(void *stream);
+
 /* Message describing the calling thread's most recent failure ("" if none). */
 M3_API const char *m3_last_error(void);
 

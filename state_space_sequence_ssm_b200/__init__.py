@@ -68,6 +68,8 @@ def _load():
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
     for f in (lib.m3_scan_workspace_size, lib.m3_scan_plan, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
         f.restype = ctypes.c_int
+    lib.m3_selftest_wait_timeout.argtypes = [vp]
+    lib.m3_selftest_wait_timeout.restype = ctypes.c_int
     lib.m3_stream_status.argtypes = [vp]
     lib.m3_stream_status.restype = ctypes.c_int
     lib.m3_last_error.argtypes = []
@@ -194,6 +196,12 @@ def scan_fwd_static(x, B, C, dt, lam, theta, A, D, init: State | None = None, *,
     _check(get_lib().m3_scan_fwd_static(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
                                         _cstate(init), _ptr(y), _cstate(final), _stream(stream)))
     return y, final
+
+
+def selftest_wait_timeout(stream=None):
+    """Queue a kernel whose bounded device wait gives up; the next
+    stream_status() on that stream raises M3Error(M3_ERR_TIMEOUT)."""
+    _check(get_lib().m3_selftest_wait_timeout(_stream(stream)))
 
 
 def stream_status(stream=None):

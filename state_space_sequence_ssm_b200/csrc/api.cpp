@@ -285,6 +285,16 @@ m3_status m3_scan_fwd_static(int algo, const m3_dims *d, const void *x, const vo
     }
 }
 
+m3_status m3_selftest_wait_timeout(void *stream) {
+    try {
+        const cudaError_t e = m3::launch_wait_selftest(static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "m3_selftest_wait_timeout");
+        return M3_OK;
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
 m3_status m3_stream_status(void *stream) {
     try {
         unsigned code = 0;

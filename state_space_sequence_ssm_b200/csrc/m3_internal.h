@@ -46,6 +46,8 @@ cudaError_t launch_step(const Problem &p, const char **why);
 // current device (looked up once per device) and its size.
 cudaError_t static_scratch(void **ptr, size_t *bytes);
 size_t static_scratch_bytes();
+// One bounded device wait that is made to give up (failure-path self-test).
+cudaError_t launch_wait_selftest(cudaStream_t stream);
 // Synchronise `stream`, then read and clear the device error word that the
 // tensor-core kernel's bounded waits set when they give up.
 cudaError_t read_device_error(unsigned *code, cudaStream_t stream);

@@ -1150,6 +1150,24 @@ cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
     return launch_nr<64, 4>(p, plan, why);
 }
 
+// Failure-path self-test: one thread waits, with a bounded wait, on an
+// mbarrier phase that nothing ever completes; the wait gives up after
+// `budget` cycles and records kErrWaitSelftest, exactly as a stuck wait in the
+// prefill kernel would.  No trap, no fault: the context stays usable.
+__global__ void __launch_bounds__(32) wait_selftest_kernel(long long budget) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::fence_mbar_init();
+        tc::mbar_wait(&bar, 0, nullptr, &g_device_error, tc::kErrWaitSelftest, budget);
+    }
+}
+
+cudaError_t launch_wait_selftest(cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(2000000LL);  // about 1 ms
+    return cudaGetLastError();
+}
+
 size_t static_scratch_bytes() { return kStaticScratchBytes; }
 
 cudaError_t static_scratch(void **ptr, size_t *bytes) {

@@ -18,6 +18,7 @@ enum : unsigned {
     kErrWaitMma = 1u << 1,
     kErrWaitCompute = 1u << 2,
     kErrWaitProducer = 1u << 3,
+    kErrWaitSelftest = 1u << 4,  // the self-test wait of m3_selftest_wait_timeout
     kErrTmemAlloc = 1u << 4,
 };
 
