@@ -8,7 +8,8 @@ Distributions (the 1.5B-scale workloads' synthetic recipe):
   x ~ N(0, 1)                      [Bt, T, H, R, P]
   B, C ~ N(0, 1/N)                 [Bt, T, H, R, N]
   dt = softplus(N(-4, 1))          [Bt, T, H]
-  A = -exp(U(0, ln 16))            [H]        (fp32, never rounded)
+  A = -exp(U(0, ln 16))            [H]        (fp32, never rounded; or, with
+                                               a_per_token, [Bt, T, H])
   lam = sigmoid(N(0, 1))           [Bt, T, H]
   theta ~ U(-pi, pi)               [Bt, T, H, N/2]   (one angle rate per state pair)
   D ~ N(0, 1)                      [H]        (fp32, never rounded)
@@ -79,14 +80,16 @@ def _draws(g, device, lead, H, R, P, N):
     return x, B, C, dt
 
 
-def make_prefill(shape: Shape, device="cpu", seqlen: int | None = None):
-    """Inputs of one prefill call.  Returns a dict of tensors on `device`."""
+def make_prefill(shape: Shape, device="cpu", seqlen: int | None = None, a_per_token: bool = False):
+    """Inputs of one prefill call.  Returns a dict of tensors on `device`.
+    With a_per_token, A is drawn per token-head ([Bt, T, H], fp32) in A's
+    place in the draw order."""
     T = shape.seqlen if seqlen is None else seqlen
     Bt, H, R, P, N = shape.batch, shape.nheads, shape.rank, shape.headdim, shape.dstate
     g = _gen(shape.seed, device)
     f = dict(device=device, dtype=torch.float32, generator=g)
     x, B, C, dt = _draws(g, device, (Bt, T), H, R, P, N)
-    A = -torch.exp(torch.rand(H, **f) * math.log(16.0))
+    A = -torch.exp(torch.rand(*((Bt, T, H) if a_per_token else (H,)), **f) * math.log(16.0))
     lam = torch.sigmoid(torch.randn(Bt, T, H, **f))
     theta = (torch.rand(Bt, T, H, N // 2, **f) * 2.0 - 1.0) * math.pi
     D = torch.randn(H, **f)
@@ -95,11 +98,12 @@ def make_prefill(shape: Shape, device="cpu", seqlen: int | None = None):
                 theta=theta.to(io), A=A.contiguous(), D=D.contiguous())
 
 
-def make_steps(shape: Shape, nsteps: int, device="cpu", seed_offset: int = 1):
+def make_steps(shape: Shape, nsteps: int, device="cpu", seed_offset: int = 1, a_per_token: bool = False):
     """Per-step decode inputs, leading dim = step: x [S,Bt,H,R,P],
     B/C [S,Bt,H,R,N], dt/lam [S,Bt,H], theta [S,Bt,H,N/2].  A and D are the
     prefill's (same seed), so a prefill followed by these steps is one
-    continuous sequence with per-head parameters."""
+    continuous sequence with per-head parameters; with a_per_token the steps
+    also carry their own A [S,Bt,H] (fp32, drawn last)."""
     Bt, H, R, P, N = shape.batch, shape.nheads, shape.rank, shape.headdim, shape.dstate
     g = _gen(shape.seed + seed_offset, device)
     f = dict(device=device, dtype=torch.float32, generator=g)
@@ -107,8 +111,10 @@ def make_steps(shape: Shape, nsteps: int, device="cpu", seed_offset: int = 1):
     lam = torch.sigmoid(torch.randn(nsteps, Bt, H, **f))
     theta = (torch.rand(nsteps, Bt, H, N // 2, **f) * 2.0 - 1.0) * math.pi
     io = shape.torch_io
-    return dict(x=x.to(io), B=B.to(io), C=C.to(io), dt=dt.to(io), lam=lam.to(io),
-                theta=theta.to(io))
+    out = dict(x=x.to(io), B=B.to(io), C=C.to(io), dt=dt.to(io), lam=lam.to(io), theta=theta.to(io))
+    if a_per_token:
+        out["A"] = -torch.exp(torch.rand(nsteps, Bt, H, **f) * math.log(16.0))
+    return out
 
 
 def make_state(shape: Shape, device="cpu", seed_offset: int = 2, scale: float = 1.0):

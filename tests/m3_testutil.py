@@ -52,7 +52,11 @@ def oracle_scan_slices(inp: dict, bh_list, init=None):
     hi = [h for _, h in bh_list]
     sl = {k: np.ascontiguousarray(np.stack([host64(inp[k][b, :, h]) for b, h in bh_list], axis=1)[None])
           for k in KEYS if k not in ("A", "D")}
-    sl["A"] = host64(inp["A"])[hi]
+    A = host64(inp["A"])
+    if A.ndim == 3:  # per-token A [Bt, T, H]: sliced like dt
+        sl["A"] = np.ascontiguousarray(np.stack([A[b, :, h] for b, h in bh_list], axis=1)[None])
+    else:
+        sl["A"] = A[hi]
     sl["D"] = host64(inp["D"])[hi]
     st = None
     if init is not None:

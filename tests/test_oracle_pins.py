@@ -399,3 +399,84 @@ def test_threading_is_deterministic():
     y4, s4 = oracle.scan(*(d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D")), st, nthreads=4)
     np.testing.assert_array_equal(y1, y4)
     np.testing.assert_array_equal(s1.h, s4.h)
+
+
+# ---------------------------------------------------------------- per-token A
+def per_token_case(T=31, R=2, seed=11):
+    s = Shape(2, T, 2, 5, 8, R, "f32", seed)
+    d = {k: v.double().numpy() for k, v in make_prefill(s, a_per_token=True).items()}
+    h, bp, xp = (t.double().numpy() for t in make_state(s))
+    return d, oracle.State(h, bp, xp)
+
+
+def test_per_token_A_constant_in_time_equals_per_head():
+    """A_t held fixed per head is the per-head method: same arithmetic, so the
+    results agree to the last bit."""
+    d, st = rand_case(T=29)
+    Bt, T, H = d["dt"].shape
+    y1, f1 = run(d, st)
+    d2 = dict(d, A=np.ascontiguousarray(np.broadcast_to(d["A"], (Bt, T, H))))
+    y2, f2 = run(d2, st)
+    np.testing.assert_array_equal(y1, y2)
+    np.testing.assert_array_equal(f1.h, f2.h)
+
+
+def test_per_token_A_free_decay_closed_form():
+    """x = 0, no pending input, A varying per token: the state decays by
+    exp(sum_t dt_t A_t) and rotates by sum_t dt_t theta_t."""
+    d, st = per_token_case(T=27)
+    d["x"][:] = 0.0
+    st.x_prev[:] = 0.0
+    y, fs = run(d, st)
+    ldec = np.cumsum(d["dt"] * d["A"], axis=1)                    # [Bt,T,H]
+    phi = np.cumsum(d["dt"][..., None] * d["theta"], axis=1)
+    u, v = st.h[:, None, :, 0::2, :], st.h[:, None, :, 1::2, :]
+    c, s = np.cos(phi)[..., None], np.sin(phi)[..., None]
+    e = np.exp(ldec)[..., None, None]
+    ht = np.empty(u.shape[:1] + (phi.shape[1],) + u.shape[2:3] + (u.shape[3] * 2, u.shape[4]))
+    ht[..., 0::2, :], ht[..., 1::2, :] = e * (u * c + v * s), e * (-u * s + v * c)
+    ref = np.einsum("bthnp,bthrn->bthrp", ht, d["C"])
+    assert rel(y, ref) < TOL
+    assert rel(fs.h, ht[:, -1]) < TOL
+
+
+def test_per_token_A_ssd_dual_bruteforce():
+    """The masked-attention dual with the decay between s and t taken as
+    exp(sum_{k=s+1..t} dt_k A_k)."""
+    d, st = per_token_case(T=19, R=2)
+    y, _ = run(d, st)
+    x, B, C, dt, lam, th, A, D = (d[k] for k in ("x", "B", "C", "dt", "lam", "theta", "A", "D"))
+    Bt, T, H, R, P = x.shape
+    phi = np.cumsum(dt[..., None] * th, axis=1)
+    Bn, Cn = rot(B, phi[:, :, :, None, :]), rot(C, phi[:, :, :, None, :])
+    ref = np.zeros_like(x)
+    for b in range(Bt):
+        for h in range(H):
+            gam, betap = lam[b, :, h] * dt[b, :, h], (1 - lam[b, :, h]) * dt[b, :, h]
+            cum = np.concatenate([[0.0], np.cumsum(dt[b, :, h] * A[b, :, h])])
+            Y = np.zeros((T, R, P))
+            h0 = st.h[b, h] + betap[0] * st.b_prev[b, h].T @ st.x_prev[b, h]
+            for t in range(T):
+                acc = math.exp(cum[t + 1]) * (Cn[b, t, h] @ h0)
+                for s_ in range(t + 1):
+                    w = gam[t] if s_ == t else math.exp(cum[t + 1] - cum[s_ + 1]) * (gam[s_] + betap[s_ + 1])
+                    acc = acc + w * (Cn[b, t, h] @ Bn[b, s_, h].T) @ x[b, s_, h]
+                Y[t] = acc + D[h] * x[b, t, h]
+            ref[b, :, h] = Y
+    assert rel(y, ref) < TOL
+
+
+def test_per_token_A_decode_continues_the_scan():
+    """Decode steps with their own A_t continue the per-token-A scan exactly."""
+    d, st = per_token_case(T=20)
+    y_full, f_full = run(d, st)
+    k = 13
+    part = {key: (v[:, :k] if v.ndim >= 3 and key not in ("D",) else v) for key, v in d.items()}
+    _, fs = run(part, st)
+    ys = []
+    for t in range(k, d["x"].shape[1]):
+        args = [d[key][:, t] for key in ("x", "B", "C", "dt", "lam", "theta")]
+        yt, fs = oracle.step(*args, d["A"][:, t], d["D"], fs)
+        ys.append(yt)
+    assert rel(np.stack(ys, 1), y_full[:, k:]) < TOL
+    assert rel(fs.h, f_full.h) < TOL
