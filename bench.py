@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the data-dependent-A variant of the prefill workload")
     ap.add_argument("--case", choices=["prefill", "decode"], default=None,
                     help="profiling case: only run --case-launches launches of one kernel at --case-batch "
                          "(for ncu captures; prints no bench line)")
@@ -169,14 +171,16 @@ class ClockSampler:
                 "power_w_max": max(pw) if pw else None}
 
 
-def prefill_bytes(s, with_final=True, with_init=False):
+def prefill_bytes(s, with_final=True, with_init=False, a_per_token=False):
     """Algorithmic HBM bytes of one prefill call: each input read once, y
-    written once, the final state written once (init read once if given)."""
+    written once, the final state written once (init read once if given);
+    a data-dependent A adds one fp32 per token-head."""
     io = 2 if s.io == "bf16" else 4
     th = s.batch * s.seqlen * s.nheads
-    per_tok = io * (2 * s.rank * s.headdim + 2 * s.rank * s.dstate + 2 + s.dstate // 2)
+    per_tok = io * (2 * s.rank * s.headdim + 2 * s.rank * s.dstate + 2 + s.dstate // 2) + 4 * int(a_per_token)
     state = 4 * s.batch * s.nheads * (s.dstate * s.headdim + s.rank * (s.dstate + s.headdim))
-    return th * per_tok + state * (int(with_final) + int(with_init)) + 8 * s.nheads
+    a_bytes = 0 if a_per_token else 4 * s.nheads
+    return th * per_tok + state * (int(with_final) + int(with_init)) + 4 * s.nheads + a_bytes
 
 
 def step_bytes(s):
@@ -351,6 +355,9 @@ def run_ours(args):
         del host, dbuf, yh, hh
 
     # ---- decode step: state from a 1024-token prefill, then single-token steps in one CUDA graph
+    if not args.no_variants and use_tc:
+        line["variants"] = [run_a_per_token(m3, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
+                                            peak_src, keys, stream)]
     if not args.no_decode:
         del inp, y, fin
         torch.cuda.empty_cache()
@@ -380,6 +387,42 @@ def _tc_supported(m3, inp, keys, algo):
         if e.status == m3.M3_ERR_UNSUPPORTED:
             return False
         raise
+
+
+def run_a_per_token(m3, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys, stream):
+    """The prefill workload with a data-dependent A_t ([Bt, T, H] fp32), timed
+    like the headline (CUDA events on the launching stream, K launches)."""
+    import torch
+    from m3_inputs import WORKLOADS, make_prefill
+
+    s = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    inp = make_prefill(s, device=dev, a_per_token=True)
+    y = torch.empty_like(inp["x"])
+    fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device=dev)
+    for _ in range(args.warmup):
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream)
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    m3.stream_status(stream)
+    el = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    ab = prefill_bytes(s, a_per_token=True)
+    ach = ab / (el / K) / 1e9
+    del inp, y, fin
+    torch.cuda.empty_cache()
+    return {"variant": "data-dependent A_t (M3_FLAG_A_PER_TOKEN)", "workload": args.workload,
+            "value": world * K * s.batch * s.seqlen / el, "unit": "tokens/s", "steps": K,
+            "ms_per_step": 1e3 * el / K, "gpu_launches": K,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                         "traffic": None, "kernel": "prefill_tc_kernel", "algorithmic_bytes_per_launch": ab,
+                         "peak_source": peak_src}}
 
 
 def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys):

@@ -36,6 +36,7 @@
  *   dt, lam   [batch, seqlen, nheads]                  io
  *   theta     [batch, seqlen, nheads, dstate/2]        io
  *   A, D      [nheads]                                 fp32
+ *             (A: [batch, seqlen, nheads] with M3_FLAG_A_PER_TOKEN)
  *   h         [batch, nheads, dstate, headdim]         fp32
  *   b_prev    [batch, nheads, rank, dstate]            fp32
  *   x_prev    [batch, nheads, rank, headdim]           fp32
@@ -80,8 +81,16 @@ typedef struct m3_dims {
     int64_t dstate;   /* N >= 2, even                              */
     int64_t rank;     /* R >= 1 (MIMO rank; 1 = SISO)              */
     int32_t io;       /* m3_dtype of x, B, C, dt, lam, theta, y    */
-    int32_t reserved; /* must be 0                                 */
+    int32_t flags;    /* 0 or M3_FLAG_A_PER_TOKEN                  */
 } m3_dims;
+
+/* A is data-dependent: one fp32 value per token-head, [batch, seqlen, nheads]
+ * for m3_scan_fwd and [batch, nheads] for m3_step, instead of one per head.
+ * Mamba-3 produces the transition scalar A_t from the input at every token
+ * ("La dualità: Mamba-2 e Mamba-3", section "Mamba-3", paragraph on the
+ * exponential-trapezoidal rule; Mamba-2 held it fixed per head); the decay
+ * of token t is exp(dt_t A_t) and everything else is unchanged. */
+#define M3_FLAG_A_PER_TOKEN 1
 
 typedef struct m3_state {
     float *h;       /* [batch, nheads, dstate, headdim] */

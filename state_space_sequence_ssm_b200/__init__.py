@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 
 M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
 M3_F32, M3_BF16 = 0, 1
+M3_FLAG_A_PER_TOKEN = 1
 ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
 
 
@@ -32,7 +33,7 @@ _STATUS = {0: "M3_OK", 1: "M3_ERR_INVALID_ARG", 2: "M3_ERR_UNSUPPORTED", 3: "M3_
 class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
                 ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("rank", ctypes.c_int64),
-                ("io", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("io", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 class CState(ctypes.Structure):
@@ -119,11 +120,11 @@ def _require_cuda(*ts):
                 raise ValueError("m3: tensors must be contiguous")
 
 
-def make_dims(Bt, T, H, P, N, R, dtype) -> Dims:
+def make_dims(Bt, T, H, P, N, R, dtype, a_per_token: bool = False) -> Dims:
     io = M3_BF16 if dtype == torch.bfloat16 else M3_F32
     if dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("io dtype must be float32 or bfloat16")
-    return Dims(Bt, T, H, P, N, R, io, 0)
+    return Dims(Bt, T, H, P, N, R, io, M3_FLAG_A_PER_TOKEN if a_per_token else 0)
 
 
 def _cstate(s: State | None):
@@ -159,12 +160,12 @@ def scan_plan(dims: Dims, algo: int = ALGO_AUTO) -> Plan:
 def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
              y=None, final: State | None = None, workspace=None, algo: int = ALGO_AUTO, stream=None):
     """Prefill scan.  x [Bt,T,H,R,P], B/C [Bt,T,H,R,N], dt/lam [Bt,T,H],
-    theta [Bt,T,H,N/2] in one io dtype (fp32 or bf16); A/D [H] fp32.
-    Returns (y, final State or None)."""
+    theta [Bt,T,H,N/2] in one io dtype (fp32 or bf16); D [H] fp32; A [H] fp32,
+    or [Bt,T,H] fp32 for a data-dependent A_t.  Returns (y, final State or None)."""
     _require_cuda(x, B, C, dt, lam, theta, A, D, y, workspace)
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
-    dims = make_dims(Bt, T, H, P, N, R, x.dtype)
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3)
     if y is None:
         y = torch.empty_like(x)
     if final is None and want_state:
@@ -187,7 +188,7 @@ def scan_fwd_static(x, B, C, dt, lam, theta, A, D, init: State | None = None, *,
     _require_cuda(x, B, C, dt, lam, theta, A, D, y)
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
-    dims = make_dims(Bt, T, H, P, N, R, x.dtype)
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3)
     if y is None:
         y = torch.empty_like(x)
     if final is None and want_state:
@@ -211,11 +212,12 @@ def stream_status(stream=None):
 
 def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None):
     """One decode step in place on `state`.  x [Bt,H,R,P], B/C [Bt,H,R,N],
-    dt/lam [Bt,H], theta [Bt,H,N/2].  Returns y [Bt,H,R,P]."""
+    dt/lam [Bt,H], theta [Bt,H,N/2]; A [H] fp32, or [Bt,H] fp32 for a
+    data-dependent A_t.  Returns y [Bt,H,R,P]."""
     _require_cuda(x, B, C, dt, lam, theta, A, D, y)
     Bt, H, R, P = x.shape
     N = B.shape[-1]
-    dims = make_dims(Bt, 1, H, P, N, R, x.dtype)
+    dims = make_dims(Bt, 1, H, P, N, R, x.dtype, a_per_token=A.dim() == 2)
     if y is None:
         y = torch.empty_like(x)
     _check(get_lib().m3_step(ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state),

@@ -77,6 +77,7 @@ struct StepArgs {
     int P, N, R;
     const IO *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
+    int a_tok;  // A is [Bt, H] (per token-head) instead of [H]
     float *h, *bp, *xp;
     IO *y;
 };
@@ -125,7 +126,7 @@ step_kernel(const StepArgs<IO> a) {
         hv[j] = __ldcs(hst + ((2 * k + 1) * P + p0) / 4);
     }
     const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
-    const float alpha = __expf(dtv * a.A[h]);
+    const float alpha = __expf(dtv * a.A[a.a_tok ? bh : h]);
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
     // ---- stage the slice's small vectors
     for (int i = tid; i < R * N; i += NT) {
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a)
     for (int i = threadIdx.x; i < R * P; i += blockDim.x) ysum[i] = 0.f;
     __syncthreads();
     const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
-    const float alpha = expf(dtv * a.A[h]);
+    const float alpha = expf(dtv * a.A[a.a_tok ? bh : h]);
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
     float *hs = a.h + bh * N * P;
     for (int idx = threadIdx.x; idx < K2 * P; idx += blockDim.x) {
@@ -377,7 +378,7 @@ step_stream_kernel(const StepArgs<IO> a) {
         const bool ok = tc::mbar_wait(&full[st], (it >> 1) & 1, &abort_flag, &g_decode_error, tc::kErrWaitTma);
         if (__syncthreads_or(!ok)) break;
         if (tid < K2) {
-            const float alpha = __expf(dtv * a.A[h]);
+            const float alpha = __expf(dtv * a.A[a.a_tok ? bh : h]);
             float sn, cs;
             sincosf(dtv * sv(sTh, tid), &sn, &cs);
             sAc[tid] = alpha * cs;
@@ -512,6 +513,7 @@ cudaError_t launch_typed(const Problem &p) {
     a.x = (const IO *)p.x; a.B = (const IO *)p.B; a.C = (const IO *)p.C;
     a.dt = (const IO *)p.dt; a.lam = (const IO *)p.lam; a.theta = (const IO *)p.theta;
     a.A = p.A; a.D = p.D;
+    a.a_tok = p.a_tok;
     a.h = p.hT; a.bp = p.bpT; a.xp = p.xpT;
     a.y = (IO *)p.y;
     if (a.BH == 0) return cudaSuccess;

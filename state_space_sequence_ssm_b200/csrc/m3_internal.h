@@ -12,6 +12,7 @@ namespace m3 {
 struct Problem {
     int64_t Bt, T, H, P, N, R;
     bool bf16;
+    bool a_tok;                   // A per token-head ([Bt,T,H]; decode [Bt,H]) instead of per head
     const void *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
     const float *h0, *bp0, *xp0;  // nullable (zero initial state)

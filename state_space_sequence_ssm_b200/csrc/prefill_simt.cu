@@ -46,6 +46,7 @@ struct SimtArgs {
     int P, N, R, Q;  // Q tokens per chunk, rows = Q * R
     const IO *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
+    int a_tok;  // A is [Bt, T, H] (per token-head)
     const float *h0, *bp0, *xp0;
     IO *y;
     float *hT, *bpT, *xpT;
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
     const int64_t bh = blockIdx.x;
     const int64_t b = bh / a.H, h = bh % a.H;
     const int64_t T = a.T, H = a.H;
-    const float Ah = a.A[h], Dh = a.D[h];
+    const float Ah = a.a_tok ? 0.f : a.A[h], Dh = a.D[h];
     auto tok = [&](int64_t t) { return (b * T + t) * H + h; };  // token-head index
 
     // ---- initial state: h0 + beta'_0 * b_prev x_prev^T (pending write of token -1)
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             const int64_t t = t0 + s;
             const float d = ldv(a.dt, tok(t)), l = ldv(a.lam, tok(t));
             dts[s] = d;
-            cA[s] = d * Ah;
+            cA[s] = d * (a.a_tok ? a.A[tok(t)] : Ah);
             gam[s] = l * d;
             float nxt = 0.f;  // (1 - lam_{t+1}) dt_{t+1}; absent after the last token
             if (t + 1 < T) {
@@ -241,6 +242,7 @@ cudaError_t launch_typed(const Problem &p, const char **why) {
     a.x = (const IO *)p.x; a.B = (const IO *)p.B; a.C = (const IO *)p.C;
     a.dt = (const IO *)p.dt; a.lam = (const IO *)p.lam; a.theta = (const IO *)p.theta;
     a.A = p.A; a.D = p.D; a.h0 = p.h0; a.bp0 = p.bp0; a.xp0 = p.xp0;
+    a.a_tok = p.a_tok;
     a.y = (IO *)p.y; a.hT = p.hT; a.bpT = p.bpT; a.xpT = p.xpT;
     // largest chunk (<= 64 rows) whose working set fits in shared memory
     int dev = 0;

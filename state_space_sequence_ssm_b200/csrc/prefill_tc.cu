@@ -120,6 +120,7 @@ struct TcArgs {
     int nseg;          // segments per sequence
     const __nv_bfloat16 *x, *B, *dt, *lam, *theta;
     const float *A, *D, *h0, *bp0, *xp0;
+    const float *A_tok;  // non-null: A per token-head [Bt, T, H] (A unused)
     __nv_bfloat16 *y;
     float *hT, *bpT, *xpT;
     // Split sequences: ws_h [nseg][BH][N][P] fp32 holds, per segment j, the
@@ -494,7 +495,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
     } else if (warp < 8) {
         // ============================================================ prologue warps (0-7)
-        const float Ah2 = a.A[h] * kLog2e;
+        const float Ah2 = a.A_tok ? 0.f : a.A[h] * kLog2e;
         uint8_t *xw = smem + C::OFF_XW;
         const unsigned short *dtr = reinterpret_cast<const unsigned short *>(a.dt);
         const unsigned short *lmr = reinterpret_cast<const unsigned short *>(a.lam);
@@ -502,12 +503,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         // raw bf16 bits of dt, lam for this thread's token and the one after it,
         // loaded one chunk ahead and converted only when used
         unsigned short pd = 0, pl = 0, pd1 = 0, pl1 = 0;
+        float pa = 0.f;  // A of this thread's token (per-token A only)
         auto prefetch_scalars = [&](int64_t t0s) {
             const int64_t t = t0s + tid;
             pd = pl = pd1 = pl1 = 0;
             if (tid < Q && t < T) {
                 pd = __ldg(dtr + tok(t));
                 pl = __ldg(lmr + tok(t));
+                if (a.A_tok) pa = __ldg(a.A_tok + tok(t));
                 if (t + 1 < T) {
                     pd1 = __ldg(dtr + tok(t + 1));
                     pl1 = __ldg(lmr + tok(t + 1));
@@ -548,12 +551,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             {
                 const float d = bf16_bits(pd), l = bf16_bits(pl);
                 const float nx = (1.f - bf16_bits(pl1)) * bf16_bits(pd1);  // 0 past the sequence end
+                const float a2 = a.A_tok ? pa * kLog2e : Ah2;                // A_t in log2 units
                 if (lc + 1 < nloc) prefetch_scalars((int64_t)(first_chunk() + lc + 1) * Q);
                 if (tid < Q) {
                     dts[tid] = d;
                     gam[tid] = l * d;
                     ghat[tid] = l * d + nx;
-                    acc = d * Ah2;
+                    acc = d * a2;
                     if (tid == 0) wtot[4] = acc;  // cA of the chunk's first token
 #pragma unroll
                     for (int off = 1; off < 32; off <<= 1) {
@@ -1032,6 +1036,7 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     a.lam = (const __nv_bfloat16 *)p.lam;
     a.theta = (const __nv_bfloat16 *)p.theta;
     a.A = p.A;
+    a.A_tok = p.a_tok ? p.A : nullptr;
     a.D = p.D;
     a.h0 = p.h0;
     a.bp0 = p.bp0;

@@ -43,8 +43,8 @@ def test_only_abi_symbols_exported(m3):
     assert ours == set(declared_functions())
 
 
-def dims(m3, Bt=2, T=8, H=2, P=8, N=8, R=1, io=0, reserved=0):
-    return m3.Dims(Bt, T, H, P, N, R, io, reserved)
+def dims(m3, Bt=2, T=8, H=2, P=8, N=8, R=1, io=0, flags=0):
+    return m3.Dims(Bt, T, H, P, N, R, io, flags)
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
@@ -60,7 +60,7 @@ def call_scan(m3, d, ptrs=None, init=None, fin=None, y=None, algo=0):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(N=7), 1), (dict(N=0), 1), (dict(H=0), 1), (dict(P=0), 1), (dict(R=0), 1),
-    (dict(Bt=-1), 1), (dict(T=-2), 1), (dict(io=5), 1), (dict(reserved=1), 1),
+    (dict(Bt=-1), 1), (dict(T=-2), 1), (dict(io=5), 1), (dict(flags=2), 1), (dict(flags=-1), 1),
     (dict(N=512), 2), (dict(R=16), 2), (dict(P=6), 2),
 ])
 def test_bad_dims_rejected(m3, kw, status):
