@@ -11,7 +11,8 @@ Distributions (the 1.5B-scale workloads' synthetic recipe):
   A = -exp(U(0, ln 16))            [H]        (fp32, never rounded; or, with
                                                a_per_token, [Bt, T, H])
   lam = sigmoid(N(0, 1))           [Bt, T, H]
-  theta ~ U(-pi, pi)               [Bt, T, H, N/2]   (one angle rate per state pair)
+  theta ~ U(-pi, pi)               [Bt, T, H, N/2]   (one angle rate per state pair;
+                                                      or, with theta_per_head, [H, N/2])
   D ~ N(0, 1)                      [H]        (fp32, never rounded)
 Draw order is fixed (x, B, C, dt, A, lam, theta, D) from one torch.Generator
 seeded with the workload's seed.  Tensors are drawn in fp32 and then rounded
@@ -80,10 +81,12 @@ def _draws(g, device, lead, H, R, P, N):
     return x, B, C, dt
 
 
-def make_prefill(shape: Shape, device="cpu", seqlen: int | None = None, a_per_token: bool = False):
+def make_prefill(shape: Shape, device="cpu", seqlen: int | None = None, a_per_token: bool = False,
+                 theta_per_head: bool = False):
     """Inputs of one prefill call.  Returns a dict of tensors on `device`.
     With a_per_token, A is drawn per token-head ([Bt, T, H], fp32) in A's
-    place in the draw order."""
+    place in the draw order; with theta_per_head, theta is drawn per head
+    ([H, N/2], same distribution) in theta's place."""
     T = shape.seqlen if seqlen is None else seqlen
     Bt, H, R, P, N = shape.batch, shape.nheads, shape.rank, shape.headdim, shape.dstate
     g = _gen(shape.seed, device)
@@ -91,7 +94,7 @@ def make_prefill(shape: Shape, device="cpu", seqlen: int | None = None, a_per_to
     x, B, C, dt = _draws(g, device, (Bt, T), H, R, P, N)
     A = -torch.exp(torch.rand(*((Bt, T, H) if a_per_token else (H,)), **f) * math.log(16.0))
     lam = torch.sigmoid(torch.randn(Bt, T, H, **f))
-    theta = (torch.rand(Bt, T, H, N // 2, **f) * 2.0 - 1.0) * math.pi
+    theta = (torch.rand(*((H,) if theta_per_head else (Bt, T, H)), N // 2, **f) * 2.0 - 1.0) * math.pi
     D = torch.randn(H, **f)
     io = shape.torch_io
     return dict(x=x.to(io), B=B.to(io), C=C.to(io), dt=dt.to(io), lam=lam.to(io),

@@ -50,9 +50,9 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         i64 = ctypes.c_int64
         dp = ctypes.c_void_p
-        lib.m3o_scan.argtypes = [i64] * 6 + [dp] * 8 + [dp] * 3 + [dp] * 4 + [ctypes.c_int, ctypes.c_int]
+        lib.m3o_scan.argtypes = [i64] * 6 + [dp] * 8 + [dp] * 3 + [dp] * 4 + [ctypes.c_int] * 3
         lib.m3o_scan.restype = ctypes.c_int
-        lib.m3o_step.argtypes = [i64] * 5 + [dp] * 8 + [dp] * 4 + [ctypes.c_int]
+        lib.m3o_step.argtypes = [i64] * 5 + [dp] * 8 + [dp] * 4 + [ctypes.c_int] * 2
         lib.m3o_step.restype = ctypes.c_int
         lib.m3o_num_cores.argtypes = []
         lib.m3o_num_cores.restype = ctypes.c_int
@@ -85,14 +85,15 @@ class State:
 
 def scan(x, B, C, dt, lam, theta, A, D, init: State | None = None, nthreads: int = 0):
     """Full-sequence scan.  Shapes: x [Bt,T,H,R,P], B/C [Bt,T,H,R,N],
-    dt/lam [Bt,T,H], theta [Bt,T,H,N/2], D [H], A [H] (per head) or [Bt,T,H]
-    (per token).  Returns (y, State)."""
+    dt/lam [Bt,T,H], theta [Bt,T,H,N/2] (or [H,N/2]: fixed per head), D [H],
+    A [H] (per head) or [Bt,T,H] (per token).  Returns (y, State)."""
     x, B, C, dt, lam, theta, A, D = map(_f64, (x, B, C, dt, lam, theta, A, D))
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
     assert B.shape == (Bt, T, H, R, N) and C.shape == B.shape
     assert dt.shape == (Bt, T, H) and lam.shape == dt.shape
-    assert theta.shape == (Bt, T, H, N // 2) and D.shape == (H,)
+    assert theta.shape in ((Bt, T, H, N // 2), (H, N // 2)) and D.shape == (H,)
+    th_head = int(theta.ndim == 2)
     assert A.shape in ((H,), (Bt, T, H))
     a_tok = int(A.shape == (Bt, T, H) and A.ndim == 3)
     h0 = bp0 = xp0 = None
@@ -105,7 +106,7 @@ def scan(x, B, C, dt, lam, theta, A, D, init: State | None = None, nthreads: int
     xpT = np.zeros((Bt, H, R, P))
     rc = _load().m3o_scan(Bt, T, H, P, N, R, *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
                           _ptr(h0), _ptr(bp0), _ptr(xp0),
-                          _ptr(y), _ptr(hT), _ptr(bpT), _ptr(xpT), int(nthreads), a_tok)
+                          _ptr(y), _ptr(hT), _ptr(bpT), _ptr(xpT), int(nthreads), a_tok, th_head)
     if rc != 0:
         raise ValueError("oracle scan rejected its arguments")
     return y, State(hT, bpT, xpT)
@@ -123,9 +124,11 @@ def step(x, B, C, dt, lam, theta, A, D, state: State):
     xp = _f64(state.x_prev).copy()
     y = np.zeros((Bt, H, R, P))
     assert A.shape in ((H,), (Bt, H))
+    assert theta.shape in ((Bt, H, N // 2), (H, N // 2))
     a_tok = int(A.ndim == 2)
+    th_head = int(theta.ndim == 2)
     rc = _load().m3o_step(Bt, H, P, N, R, *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
-                          _ptr(h), _ptr(bp), _ptr(xp), _ptr(y), a_tok)
+                          _ptr(h), _ptr(bp), _ptr(xp), _ptr(y), a_tok, th_head)
     if rc != 0:
         raise ValueError("oracle step rejected its arguments")
     return y, State(h, bp, xp)

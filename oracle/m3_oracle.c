@@ -44,6 +44,11 @@
  * token-head; [Bt, H] for a decode step); the token update is the same with
  * A read at the token.
  *
+ * theta per token or per head.  The angle rates may also be fixed per head,
+ * theta [H, N/2] (a time-constant rotation, as in the complex-diagonal SSMs
+ * where the eigenvalue's phase is a learned constant): the token's angle is
+ * then D_t * theta[h][k], everything else unchanged.
+ *
  * Layouts (row-major, last index fastest), all fp64 here:
  *   x, y  [Bt, T, H, R, P]     B, C [Bt, T, H, R, N]
  *   dt, lam [Bt, T, H]         theta [Bt, T, H, N/2]      D [H]
@@ -63,6 +68,7 @@ typedef struct {
     const double *h0, *bp0, *xp0; /* nullable: zero initial state */
     double *y, *hT, *bpT, *xpT;   /* y required; final-state outputs nullable */
     int a_per_token;              /* A is [Bt, T, H] instead of [H] */
+    int theta_per_head;           /* theta is [H, N/2] instead of [Bt, T, H, N/2] */
     int64_t next;                 /* next (b,h) slice to claim */
     pthread_mutex_t lock;
 } job_t;
@@ -133,7 +139,7 @@ static void run_slice(job_t *j, int64_t bh)
         const int64_t th_ = (b * T + t) * H + hd; /* token-head index */
         token_update(N, P, R, h, bp, xp, j->x + th_ * R * P, j->B + th_ * R * N,
                      j->C + th_ * R * N, j->dt[th_], j->lam[th_],
-                     j->theta + th_ * (N / 2), j->A[j->a_per_token ? th_ : hd], j->D[hd],
+                     j->theta + (j->theta_per_head ? hd : th_) * (N / 2), j->A[j->a_per_token ? th_ : hd], j->D[hd],
                      j->y + th_ * R * P);
     }
     if (j->hT) memcpy(j->hT + bh * N * P, h, sizeof(double) * (size_t)(N * P));
@@ -165,13 +171,14 @@ int m3o_num_cores(void)
 
 /* Full sequence scan.  Returns 0 on success, -1 on bad arguments.
  * nthreads <= 0 means one thread per online core; a_per_token != 0 means A is
- * [Bt, T, H] (else [H]). */
+ * [Bt, T, H] (else [H]); theta_per_head != 0 means theta is [H, N/2]. */
 int m3o_scan(int64_t Bt, int64_t T, int64_t H, int64_t P, int64_t N, int64_t R,
              const double *x, const double *B, const double *C,
              const double *dt, const double *lam, const double *theta,
              const double *A, const double *D,
              const double *h0, const double *bp0, const double *xp0,
-             double *y, double *hT, double *bpT, double *xpT, int nthreads, int a_per_token)
+             double *y, double *hT, double *bpT, double *xpT, int nthreads, int a_per_token,
+             int theta_per_head)
 {
     if (Bt < 0 || T < 0 || H <= 0 || P <= 0 || N <= 0 || (N & 1) || R <= 0) return -1;
     if (!y && T > 0) return -1;
@@ -182,6 +189,7 @@ int m3o_scan(int64_t Bt, int64_t T, int64_t H, int64_t P, int64_t N, int64_t R,
     j.A = A; j.D = D; j.h0 = h0; j.bp0 = bp0; j.xp0 = xp0;
     j.y = y; j.hT = hT; j.bpT = bpT; j.xpT = xpT;
     j.a_per_token = a_per_token;
+    j.theta_per_head = theta_per_head;
     pthread_mutex_init(&j.lock, NULL);
     int nt = nthreads > 0 ? nthreads : m3o_num_cores();
     if (nt > Bt * H) nt = (int)(Bt * H);
@@ -199,20 +207,22 @@ int m3o_scan(int64_t Bt, int64_t T, int64_t H, int64_t P, int64_t N, int64_t R,
 
 /* One decode step for every (b,h) slice, in place on (h, b_prev, x_prev).
  * Inputs are one token per slice: x [Bt,H,R,P], B/C [Bt,H,R,N], dt/lam [Bt,H],
- * theta [Bt,H,N/2], A [H] or (a_per_token) [Bt,H]; y [Bt,H,R,P].  It is the
+ * theta [Bt,H,N/2] or (theta_per_head) [H,N/2], A [H] or (a_per_token)
+ * [Bt,H]; y [Bt,H,R,P].  It is the
  * same token update as the scan. */
 int m3o_step(int64_t Bt, int64_t H, int64_t P, int64_t N, int64_t R,
              const double *x, const double *B, const double *C,
              const double *dt, const double *lam, const double *theta,
              const double *A, const double *D,
-             double *h, double *bp, double *xp, double *y, int a_per_token)
+             double *h, double *bp, double *xp, double *y, int a_per_token, int theta_per_head)
 {
     if (Bt < 0 || H <= 0 || P <= 0 || N <= 0 || (N & 1) || R <= 0) return -1;
     for (int64_t bh = 0; bh < Bt * H; ++bh) {
         const int64_t hd = bh % H;
         token_update(N, P, R, h + bh * N * P, bp + bh * R * N, xp + bh * R * P,
                      x + bh * R * P, B + bh * R * N, C + bh * R * N, dt[bh], lam[bh],
-                     theta + bh * (N / 2), A[a_per_token ? bh : hd], D[hd], y + bh * R * P);
+                     theta + (theta_per_head ? hd : bh) * (N / 2), A[a_per_token ? bh : hd], D[hd],
+                     y + bh * R * P);
     }
     return 0;
 }

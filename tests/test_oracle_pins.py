@@ -480,3 +480,39 @@ def test_per_token_A_decode_continues_the_scan():
         ys.append(yt)
     assert rel(np.stack(ys, 1), y_full[:, k:]) < TOL
     assert rel(fs.h, f_full.h) < TOL
+
+
+# ---------------------------------------------------------------- theta fixed per head
+def test_theta_per_head_equals_broadcast_per_token():
+    """theta [H, N/2] is the per-token method with theta repeated over tokens:
+    same arithmetic, bit for bit (scan and decode step)."""
+    s = Shape(2, 23, 2, 5, 8, 2, "f32", 12)
+    d = {k: v.double().numpy() for k, v in make_prefill(s, theta_per_head=True).items()}
+    assert d["theta"].shape == (2, 4)
+    h, bp, xp = (t.double().numpy() for t in make_state(s))
+    st = oracle.State(h, bp, xp)
+    y1, f1 = run(d, st)
+    d2 = dict(d, theta=np.ascontiguousarray(np.broadcast_to(d["theta"][None, None], (2, 23, 2, 4))))
+    y2, f2 = run(d2, st)
+    np.testing.assert_array_equal(y1, y2)
+    np.testing.assert_array_equal(f1.h, f2.h)
+    args = [d[k][:, 0] for k in ("x", "B", "C", "dt", "lam")]
+    ya, sa = oracle.step(*args, d["theta"], d["A"], d["D"], st)
+    yb, sb = oracle.step(*args, d2["theta"][:, 0], d["A"], d["D"], st)
+    np.testing.assert_array_equal(ya, yb)
+    np.testing.assert_array_equal(sa.h, sb.h)
+
+
+def test_theta_per_head_free_rotation_closed_form():
+    """x = 0, no pending input, theta fixed per head: pair k turns by
+    theta_k * sum_t dt_t, so z_t = exp(sum dt (A - i theta_k)) z_0."""
+    s = Shape(1, 33, 2, 3, 6, 1, "f32", 13)
+    d = {k: v.double().numpy() for k, v in make_prefill(s, theta_per_head=True).items()}
+    d["x"][:] = 0.0
+    h, bp, xp = (t.double().numpy() for t in make_state(s))
+    xp[:] = 0.0
+    y, fs = run(d, oracle.State(h, bp, xp))
+    cd = np.sum(d["dt"][0], axis=0)                                  # [H]
+    z0 = h[0, :, 0::2, :] + 1j * h[0, :, 1::2, :]                   # [H, N/2, P]
+    z = np.exp((cd * d["A"])[:, None, None] - 1j * (cd[:, None] * d["theta"])[:, :, None]) * z0
+    assert rel(fs.h[0, :, 0::2, :], z.real) < TOL and rel(fs.h[0, :, 1::2, :], z.imag) < TOL
