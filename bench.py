@@ -171,16 +171,19 @@ class ClockSampler:
                 "power_w_max": max(pw) if pw else None}
 
 
-def prefill_bytes(s, with_final=True, with_init=False, a_per_token=False):
+def prefill_bytes(s, with_final=True, with_init=False, a_per_token=False, theta_per_head=False):
     """Algorithmic HBM bytes of one prefill call: each input read once, y
     written once, the final state written once (init read once if given);
-    a data-dependent A adds one fp32 per token-head."""
+    a data-dependent A adds one fp32 per token-head, angle rates fixed per head
+    are read once per head instead of once per token-head."""
     io = 2 if s.io == "bf16" else 4
     th = s.batch * s.seqlen * s.nheads
-    per_tok = io * (2 * s.rank * s.headdim + 2 * s.rank * s.dstate + 2 + s.dstate // 2) + 4 * int(a_per_token)
+    theta_tok = 0 if theta_per_head else s.dstate // 2
+    per_tok = io * (2 * s.rank * s.headdim + 2 * s.rank * s.dstate + 2 + theta_tok) + 4 * int(a_per_token)
     state = 4 * s.batch * s.nheads * (s.dstate * s.headdim + s.rank * (s.dstate + s.headdim))
     a_bytes = 0 if a_per_token else 4 * s.nheads
-    return th * per_tok + state * (int(with_final) + int(with_init)) + 4 * s.nheads + a_bytes
+    theta_bytes = io * s.nheads * (s.dstate // 2) if theta_per_head else 0
+    return th * per_tok + state * (int(with_final) + int(with_init)) + 4 * s.nheads + a_bytes + theta_bytes
 
 
 def step_bytes(s):
@@ -356,8 +359,8 @@ def run_ours(args):
 
     # ---- decode step: state from a 1024-token prefill, then single-token steps in one CUDA graph
     if not args.no_variants and use_tc:
-        line["variants"] = [run_a_per_token(m3, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
-                                            peak_src, keys, stream)]
+        line["variants"] = [run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
+                                        peak_src, keys, stream) for kind in ("a_per_token", "theta_per_head")]
     if not args.no_decode:
         del inp, y, fin
         torch.cuda.empty_cache()
@@ -389,14 +392,19 @@ def _tc_supported(m3, inp, keys, algo):
         raise
 
 
-def run_a_per_token(m3, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys, stream):
-    """The prefill workload with a data-dependent A_t ([Bt, T, H] fp32), timed
-    like the headline (CUDA events on the launching stream, K launches)."""
+VARIANTS = {"a_per_token": "data-dependent A_t (M3_FLAG_A_PER_TOKEN)",
+            "theta_per_head": "angle rates fixed per head (M3_FLAG_THETA_PER_HEAD)"}
+
+
+def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys, stream):
+    """The prefill workload with a data-dependent A_t ([Bt, T, H] fp32) or
+    with theta fixed per head ([H, N/2]), timed like the headline (CUDA events
+    on the launching stream, K launches)."""
     import torch
     from m3_inputs import WORKLOADS, make_prefill
 
     s = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
-    inp = make_prefill(s, device=dev, a_per_token=True)
+    inp = make_prefill(s, device=dev, **{kind: True})
     y = torch.empty_like(inp["x"])
     fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device=dev)
     for _ in range(args.warmup):
@@ -413,11 +421,11 @@ def run_a_per_token(m3, args, dev, rank, world, barrier, max_over_ranks, hbm_pea
     barrier()
     m3.stream_status(stream)
     el = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-    ab = prefill_bytes(s, a_per_token=True)
+    ab = prefill_bytes(s, **{kind: True})
     ach = ab / (el / K) / 1e9
     del inp, y, fin
     torch.cuda.empty_cache()
-    return {"variant": "data-dependent A_t (M3_FLAG_A_PER_TOKEN)", "workload": args.workload,
+    return {"variant": VARIANTS[kind], "workload": args.workload,
             "value": world * K * s.batch * s.seqlen / el, "unit": "tokens/s", "steps": K,
             "ms_per_step": 1e3 * el / K, "gpu_launches": K,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,

@@ -37,6 +37,7 @@
  *   theta     [batch, seqlen, nheads, dstate/2]        io
  *   A, D      [nheads]                                 fp32
  *             (A: [batch, seqlen, nheads] with M3_FLAG_A_PER_TOKEN)
+ *   theta with M3_FLAG_THETA_PER_HEAD: [nheads, dstate/2]      io
  *   h         [batch, nheads, dstate, headdim]         fp32
  *   b_prev    [batch, nheads, rank, dstate]            fp32
  *   x_prev    [batch, nheads, rank, headdim]           fp32
@@ -81,7 +82,7 @@ typedef struct m3_dims {
     int64_t dstate;   /* N >= 2, even                              */
     int64_t rank;     /* R >= 1 (MIMO rank; 1 = SISO)              */
     int32_t io;       /* m3_dtype of x, B, C, dt, lam, theta, y    */
-    int32_t flags;    /* 0 or M3_FLAG_A_PER_TOKEN                  */
+    int32_t flags;    /* 0 or M3_FLAG_* bits                       */
 } m3_dims;
 
 /* A is data-dependent: one fp32 value per token-head, [batch, seqlen, nheads]
@@ -91,6 +92,14 @@ typedef struct m3_dims {
  * exponential-trapezoidal rule; Mamba-2 held it fixed per head); the decay
  * of token t is exp(dt_t A_t) and everything else is unchanged. */
 #define M3_FLAG_A_PER_TOKEN 1
+
+/* theta fixed per head: [nheads, dstate/2] (io dtype) for m3_scan_fwd and
+ * m3_step alike, instead of one set of angle rates per token-head.  The
+ * angle of pair k at token t is then dt_t theta[h][k] -- the time-constant
+ * rotation of a complex-diagonal SSM, the form the complex-state equivalence
+ * starts from ("La dualità: Mamba-2 e Mamba-3", section "Mamba-3", paragraph
+ * on complex transitions).  It saves reading theta per token. */
+#define M3_FLAG_THETA_PER_HEAD 2
 
 typedef struct m3_state {
     float *h;       /* [batch, nheads, dstate, headdim] */

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_A_PER_TOKEN = 1
+M3_FLAG_THETA_PER_HEAD = 2
 ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
 
 
@@ -120,11 +121,12 @@ def _require_cuda(*ts):
                 raise ValueError("m3: tensors must be contiguous")
 
 
-def make_dims(Bt, T, H, P, N, R, dtype, a_per_token: bool = False) -> Dims:
+def make_dims(Bt, T, H, P, N, R, dtype, a_per_token: bool = False, theta_per_head: bool = False) -> Dims:
     io = M3_BF16 if dtype == torch.bfloat16 else M3_F32
     if dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("io dtype must be float32 or bfloat16")
-    return Dims(Bt, T, H, P, N, R, io, M3_FLAG_A_PER_TOKEN if a_per_token else 0)
+    flags = (M3_FLAG_A_PER_TOKEN if a_per_token else 0) | (M3_FLAG_THETA_PER_HEAD if theta_per_head else 0)
+    return Dims(Bt, T, H, P, N, R, io, flags)
 
 
 def _cstate(s: State | None):
@@ -160,12 +162,13 @@ def scan_plan(dims: Dims, algo: int = ALGO_AUTO) -> Plan:
 def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
              y=None, final: State | None = None, workspace=None, algo: int = ALGO_AUTO, stream=None):
     """Prefill scan.  x [Bt,T,H,R,P], B/C [Bt,T,H,R,N], dt/lam [Bt,T,H],
-    theta [Bt,T,H,N/2] in one io dtype (fp32 or bf16); D [H] fp32; A [H] fp32,
-    or [Bt,T,H] fp32 for a data-dependent A_t.  Returns (y, final State or None)."""
+    theta [Bt,T,H,N/2] (or [H,N/2]: fixed per head) in one io dtype (fp32 or
+    bf16); D [H] fp32; A [H] fp32, or [Bt,T,H] fp32 for a data-dependent A_t.
+    Returns (y, final State or None)."""
     _require_cuda(x, B, C, dt, lam, theta, A, D, y, workspace)
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
-    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3)
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
     if y is None:
         y = torch.empty_like(x)
     if final is None and want_state:
@@ -188,7 +191,7 @@ def scan_fwd_static(x, B, C, dt, lam, theta, A, D, init: State | None = None, *,
     _require_cuda(x, B, C, dt, lam, theta, A, D, y)
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
-    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3)
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
     if y is None:
         y = torch.empty_like(x)
     if final is None and want_state:
@@ -212,12 +215,12 @@ def stream_status(stream=None):
 
 def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None):
     """One decode step in place on `state`.  x [Bt,H,R,P], B/C [Bt,H,R,N],
-    dt/lam [Bt,H], theta [Bt,H,N/2]; A [H] fp32, or [Bt,H] fp32 for a
-    data-dependent A_t.  Returns y [Bt,H,R,P]."""
+    dt/lam [Bt,H], theta [Bt,H,N/2] (or [H,N/2]: fixed per head); A [H] fp32,
+    or [Bt,H] fp32 for a data-dependent A_t.  Returns y [Bt,H,R,P]."""
     _require_cuda(x, B, C, dt, lam, theta, A, D, y)
     Bt, H, R, P = x.shape
     N = B.shape[-1]
-    dims = make_dims(Bt, 1, H, P, N, R, x.dtype, a_per_token=A.dim() == 2)
+    dims = make_dims(Bt, 1, H, P, N, R, x.dtype, a_per_token=A.dim() == 2, theta_per_head=theta.dim() == 2)
     if y is None:
         y = torch.empty_like(x)
     _check(get_lib().m3_step(ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state),

@@ -50,7 +50,8 @@ m3_status check_dims(const m3_dims *d, bool decode) {
     if (d->dstate < 2 || (d->dstate & 1))
         return fail(M3_ERR_INVALID_ARG, "dstate must be even and >= 2 (state pairs)");
     if (d->io != M3_F32 && d->io != M3_BF16) return fail(M3_ERR_INVALID_ARG, "io must be M3_F32 or M3_BF16");
-    if (d->flags & ~M3_FLAG_A_PER_TOKEN) return fail(M3_ERR_INVALID_ARG, "unknown bits in flags");
+    if (d->flags & ~(M3_FLAG_A_PER_TOKEN | M3_FLAG_THETA_PER_HEAD))
+        return fail(M3_ERR_INVALID_ARG, "unknown bits in flags");
     if (d->dstate > 256 || d->headdim > 256 || d->rank > 8)
         return fail(M3_ERR_UNSUPPORTED, "supported sizes: dstate <= 256, headdim <= 256, rank <= 8");
     if (d->headdim % 4 != 0 && d->headdim != 1 && d->headdim != 2)
@@ -86,7 +87,7 @@ m3_status check_tensors(const m3_dims *d, int64_t tok, const void *x, const void
     ins[n++] = range(C, tok * R * N * es);
     ins[n++] = range(dt, tok * es);
     ins[n++] = range(lam, tok * es);
-    ins[n++] = range(theta, tok * (N / 2) * es);
+    ins[n++] = range(theta, ((d->flags & M3_FLAG_THETA_PER_HEAD) ? d->nheads : tok) * (N / 2) * es);
     ins[n++] = range(A, ((d->flags & M3_FLAG_A_PER_TOKEN) ? tok : d->nheads) * 4);
     ins[n++] = range(D, d->nheads * 4);
     *nin = n;
@@ -130,6 +131,7 @@ m3::Problem make_problem(const m3_dims *d, const void *x, const void *B, const v
     p.Bt = d->batch; p.T = d->seqlen; p.H = d->nheads; p.P = d->headdim; p.N = d->dstate; p.R = d->rank;
     p.bf16 = d->io == M3_BF16;
     p.a_tok = (d->flags & M3_FLAG_A_PER_TOKEN) != 0;
+    p.th_head = (d->flags & M3_FLAG_THETA_PER_HEAD) != 0;
     p.x = x; p.B = B; p.C = C; p.dt = dt; p.lam = lam; p.theta = theta; p.A = A; p.D = D; p.y = y;
     p.stream = static_cast<cudaStream_t>(stream);
     return p;

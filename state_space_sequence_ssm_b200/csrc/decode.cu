@@ -77,7 +77,8 @@ struct StepArgs {
     int P, N, R;
     const IO *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
-    int a_tok;  // A is [Bt, H] (per token-head) instead of [H]
+    int a_tok;    // A is [Bt, H] (per token-head) instead of [H]
+    int th_head;  // theta is [H, N/2] (fixed per head)
     float *h, *bp, *xp;
     IO *y;
 };
@@ -140,7 +141,7 @@ step_kernel(const StepArgs<IO> a) {
     }
     for (int k = tid; k < K2; k += NT) {
         float sn, cs;
-        sincosf(dtv * ldv(a.theta, bh * K2 + k), &sn, &cs);
+        sincosf(dtv * ldv(a.theta, (a.th_head ? (int64_t)h : bh) * K2 + k), &sn, &cs);
         sAc[k] = alpha * cs;
         sAs[k] = alpha * sn;
     }
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a)
             v += betap * a.bp[(bh * R + r) * N + 2 * k + 1] * xpp;
         }
         float sn, cs;
-        sincosf(dtv * ldv(a.theta, bh * K2 + k), &sn, &cs);
+        sincosf(dtv * ldv(a.theta, (a.th_head ? (int64_t)h : bh) * K2 + k), &sn, &cs);
         float nu = alpha * (u * cs + v * sn), nv = alpha * (-u * sn + v * cs);
         for (int r = 0; r < R; ++r) {
             const float xx = ldv(a.x, (bh * R + r) * P + p);
@@ -348,7 +349,7 @@ step_stream_kernel(const StepArgs<IO> a) {
         tc::bulk_g2s(s + Cfg::O_B, a.B + bh * R * N, Cfg::B_B, &full[st]);
         tc::bulk_g2s(s + Cfg::O_C, a.C + bh * R * N, Cfg::B_B, &full[st]);
         tc::bulk_g2s(s + Cfg::O_X, a.x + bh * R * P, Cfg::B_X, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_TH, a.theta + bh * K2, Cfg::B_TH, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_TH, a.theta + (a.th_head ? bh % a.H : bh) * K2, Cfg::B_TH, &full[st]);
     };
     if (tid == 0) {
         tc::mbar_init(&full[0], 1);
@@ -514,6 +515,7 @@ cudaError_t launch_typed(const Problem &p) {
     a.dt = (const IO *)p.dt; a.lam = (const IO *)p.lam; a.theta = (const IO *)p.theta;
     a.A = p.A; a.D = p.D;
     a.a_tok = p.a_tok;
+    a.th_head = p.th_head;
     a.h = p.hT; a.bp = p.bpT; a.xp = p.xpT;
     a.y = (IO *)p.y;
     if (a.BH == 0) return cudaSuccess;

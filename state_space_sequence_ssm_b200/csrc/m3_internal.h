@@ -13,6 +13,7 @@ struct Problem {
     int64_t Bt, T, H, P, N, R;
     bool bf16;
     bool a_tok;                   // A per token-head ([Bt,T,H]; decode [Bt,H]) instead of per head
+    bool th_head;                 // theta fixed per head ([H,N/2]) instead of per token-head
     const void *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
     const float *h0, *bp0, *xp0;  // nullable (zero initial state)

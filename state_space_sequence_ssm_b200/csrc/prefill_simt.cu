@@ -46,7 +46,8 @@ struct SimtArgs {
     int P, N, R, Q;  // Q tokens per chunk, rows = Q * R
     const IO *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
-    int a_tok;  // A is [Bt, T, H] (per token-head)
+    int a_tok;    // A is [Bt, T, H] (per token-head)
+    int th_head;  // theta is [H, N/2] (fixed per head)
     const float *h0, *bp0, *xp0;
     IO *y;
     float *hT, *bpT, *xpT;
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
         for (int k = tid; k < K2; k += kThreads) {
             float phi = 0.f;
             for (int s = 0; s < L; ++s) {
-                phi += dts[s] * ldv(a.theta, tok(t0 + s) * K2 + k);
+                phi += dts[s] * ldv(a.theta, (a.th_head ? (int64_t)h : tok(t0 + s)) * K2 + k);
                 float sn, cs;
                 sincosf(phi, &sn, &cs);
                 for (int r = 0; r < R; ++r) {
@@ -243,6 +244,7 @@ cudaError_t launch_typed(const Problem &p, const char **why) {
     a.dt = (const IO *)p.dt; a.lam = (const IO *)p.lam; a.theta = (const IO *)p.theta;
     a.A = p.A; a.D = p.D; a.h0 = p.h0; a.bp0 = p.bp0; a.xp0 = p.xp0;
     a.a_tok = p.a_tok;
+    a.th_head = p.th_head;
     a.y = (IO *)p.y; a.hT = p.hT; a.bpT = p.bpT; a.xpT = p.xpT;
     // largest chunk (<= 64 rows) whose working set fits in shared memory
     int dev = 0;

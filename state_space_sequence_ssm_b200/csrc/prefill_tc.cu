@@ -101,9 +101,9 @@ struct Cfg {
     static constexpr uint32_t HB_BYTES = N * 128;
     static constexpr uint32_t OFF_SCAL = OFF_HB + HB_BYTES;
     // kNX buffers of {cAl2, gam, ghat, colf}[Q] + {cos, sin}[K2] (read by the
-    // state warpgroup a chunk later) + {wst, dts}[Q] + phis[NPART][K2] + wtot[8]
+    // state warpgroup a chunk later) + {wst, dts}[Q] + phis[NPART][K2] + wtot[16]
     static constexpr uint32_t SB = 4 * Q + 2 * K2;
-    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 8;
+    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16;
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
     static constexpr uint32_t NBARS = 19;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
@@ -121,6 +121,7 @@ struct TcArgs {
     const __nv_bfloat16 *x, *B, *dt, *lam, *theta;
     const float *A, *D, *h0, *bp0, *xp0;
     const float *A_tok;  // non-null: A per token-head [Bt, T, H] (A unused)
+    int th_head;         // theta fixed per head, [H, N/2]
     __nv_bfloat16 *y;
     float *hT, *bpT, *xpT;
     // Split sequences: ws_h [nseg][BH][N][P] fp32 holds, per segment j, the
@@ -306,7 +307,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     float *wst = scal + kNX * C::SB;  // exp(cA_end - cA_s) ghat_s (chunk-state weight)
     float *dts = wst + Q;             // dt
     float *phis = dts + Q;            // partial angle sums [NPART][K2]
-    float *wtot = phis + NPART * K2;  // per-warp totals of the dt*A scan; [4] = cA of token 0
+    // per-warp totals of the dt*A scan ([0, 4)); [4] = cA of token 0; [8, 12):
+    // per-warp totals of the dt scan (angle rates fixed per head)
+    float *wtot = phis + NPART * K2;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     Bars bb{bars, bars + 2, bars + 4, bars + 7, bars + 10, bars + 11, bars + 12, bars + 13, bars + 14, bars + 15,
             bars + 16};
@@ -378,7 +381,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     tma_prefetch_5d(&tmB, kb * 64, 0, (int)h, t0, (int)b);
                     if (!SUM) tma_prefetch_5d(&tmC, kb * 64, 0, (int)h, t0, (int)b);
                 }
-                tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // theta is read straight into registers
+                if (!a.th_head) tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // read straight into registers
             };
             int issued = 0;
             for (int i = 0; i < kPrefetchAhead && i < nloc; ++i) prefetch_chunk(cb + i);
@@ -520,7 +523,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         // theta of this thread's 4 pairs for its TPT tokens, read straight from
         // global memory into registers one chunk ahead of use
         uint2 thr[TPT];
+        // angle rates fixed per head: the thread's 4 pairs, for the whole sequence
+        float thh[4] = {0.f, 0.f, 0.f, 0.f};
+        if (a.th_head) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) thh[e] = bf(a.theta, h * K2 + 4 * g + e);
+        }
         auto prefetch_theta = [&](int64_t t0s) {
+            if (a.th_head) return;
 #pragma unroll
             for (int j = 0; j < TPT; ++j) {
                 const int64_t t = t0s + part * TPT + j;
@@ -547,7 +557,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 break;
 
             // ---- A. per-token scalars and the chunk-local scan of dt*A
-            float acc = 0.f;
+            float acc = 0.f, acd = 0.f;
             {
                 const float d = bf16_bits(pd), l = bf16_bits(pl);
                 const float nx = (1.f - bf16_bits(pl1)) * bf16_bits(pd1);  // 0 past the sequence end
@@ -565,6 +575,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         if (lane >= off) acc += v;
                     }
                     if (lane == 31) wtot[warp] = acc;
+                    if (a.th_head) {  // chunk-local cumulative dt: the angle is theta_k times it
+                        acd = d;
+#pragma unroll
+                        for (int off = 1; off < 32; off <<= 1) {
+                            const float v = __shfl_up_sync(0xffffffffu, acd, off);
+                            if (lane >= off) acd += v;
+                        }
+                        if (lane == 31) wtot[8 + warp] = acd;
+                    }
                 }
             }
             named_bar(kBarPro, kPro);
@@ -581,6 +600,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 wst[tid] = ex2(tot - ca) * ghat[tid];
                 // column factor of the decay mask, relative to the chunk's first token
                 colf[tid] = ex2(wtot[4] - ca) * ghat[tid];
+                if (a.th_head) {  // dts becomes the cumulative dt (read after the next barrier)
+                    float offd = 0.f;
+#pragma unroll
+                    for (int w = 0; w < Q / 32; ++w)
+                        if (w < warp) offd += wtot[8 + w];
+                    dts[tid] = acd + offd;
+                }
             }
 
             // ---- B. cumulative angles of 4 pairs per thread, in-place rotation
@@ -589,6 +615,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 float loc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < TPT; ++j) {
+                    if (a.th_head) break;
                     const float di = dts[part * TPT + j];
                     const float2 t01 = unpack_bf16(thr[j].x), t23 = unpack_bf16(thr[j].y);
                     loc[0] = fmaf(di, t01.x, loc[0]);
@@ -601,7 +628,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (bar_any<kBarPro, kPro>(!mbar_wait(&bb.full_bc[s], (lc >> 1) & 1, abort_flag, err, kErrWaitTma)))
                     break;
                 float phi[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int q = 0; q < part; ++q) {
+                for (int q = 0; q < (a.th_head ? 0 : part); ++q) {
                     const float4 v = *reinterpret_cast<const float4 *>(phis + q * K2 + 4 * g);
                     phi[0] += v.x;
                     phi[1] += v.y;
@@ -629,11 +656,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     for (int jj = 0; jj < TB; ++jj) {
                         const int i = part * TPT + j0 + jj;
                         const float di = dts[i];
-                        const float2 t01 = unpack_bf16(thr[j0 + jj].x), t23 = unpack_bf16(thr[j0 + jj].y);
-                        phi[0] = fmaf(di, t01.x, phi[0]);
-                        phi[1] = fmaf(di, t01.y, phi[1]);
-                        phi[2] = fmaf(di, t23.x, phi[2]);
-                        phi[3] = fmaf(di, t23.y, phi[3]);
+                        if (a.th_head) {  // di is the cumulative dt of token i
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) phi[e] = di * thh[e];
+                        } else {
+                            const float2 t01 = unpack_bf16(thr[j0 + jj].x), t23 = unpack_bf16(thr[j0 + jj].y);
+                            phi[0] = fmaf(di, t01.x, phi[0]);
+                            phi[1] = fmaf(di, t01.y, phi[1]);
+                            phi[2] = fmaf(di, t23.x, phi[2]);
+                            phi[3] = fmaf(di, t23.y, phi[3]);
+                        }
                         uint32_t cc[4], nss[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -1017,8 +1049,10 @@ template <int N, int R>
 cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     using C = Cfg<N, R>;
     CUtensorMap mx, mb, mc, mt;
+    // (theta fixed per head: a valid map over [H, N/2] that the kernel never loads from)
     if (!make_map(&mx, p.x, kP, R, p.H, p.T, p.Bt, C::Q) || !make_map(&mb, p.B, N, R, p.H, p.T, p.Bt, C::Q) ||
-        !make_map(&mc, p.C, N, R, p.H, p.T, p.Bt, C::Q) || !make_theta_map(&mt, p.theta, N / 2, p.H, p.T, p.Bt, C::Q)) {
+        !make_map(&mc, p.C, N, R, p.H, p.T, p.Bt, C::Q) ||
+        !make_theta_map(&mt, p.theta, N / 2, p.H, p.th_head ? 1 : p.T, p.th_head ? 1 : p.Bt, p.th_head ? 1 : C::Q)) {
         *why = "tensor-core prefill: TMA descriptor encoding failed";
         return cudaErrorNotSupported;
     }
@@ -1037,6 +1071,7 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     a.theta = (const __nv_bfloat16 *)p.theta;
     a.A = p.A;
     a.A_tok = p.a_tok ? p.A : nullptr;
+    a.th_head = p.th_head;
     a.D = p.D;
     a.h0 = p.h0;
     a.bp0 = p.bp0;

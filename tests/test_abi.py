@@ -60,7 +60,7 @@ def call_scan(m3, d, ptrs=None, init=None, fin=None, y=None, algo=0):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(N=7), 1), (dict(N=0), 1), (dict(H=0), 1), (dict(P=0), 1), (dict(R=0), 1),
-    (dict(Bt=-1), 1), (dict(T=-2), 1), (dict(io=5), 1), (dict(flags=2), 1), (dict(flags=-1), 1),
+    (dict(Bt=-1), 1), (dict(T=-2), 1), (dict(io=5), 1), (dict(flags=4), 1), (dict(flags=-1), 1),
     (dict(N=512), 2), (dict(R=16), 2), (dict(P=6), 2),
 ])
 def test_bad_dims_rejected(m3, kw, status):
