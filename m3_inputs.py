@@ -120,6 +120,21 @@ def make_steps(shape: Shape, nsteps: int, device="cpu", seed_offset: int = 1, a_
     return out
 
 
+def make_bcnorm(shape: Shape, device="cpu", seed_offset: int = 3):
+    """Synthetic BC-norm parameters (fp32): RMS-norm weights wB, wC [N] ~
+    (1 + 0.1 N(0,1)) / sqrt(N) and head-specific biases bB, bC [H, R, N] ~
+    0.1 N(0,1) / sqrt(N), so the normalised rows keep the scale of the raw
+    B, C draws (RMS about 1/sqrt(N))."""
+    H, R, N = shape.nheads, shape.rank, shape.dstate
+    g = _gen(shape.seed + seed_offset, device)
+    f = dict(device=device, dtype=torch.float32, generator=g)
+    wB = (1.0 + 0.1 * torch.randn(N, **f)) / math.sqrt(N)
+    wC = (1.0 + 0.1 * torch.randn(N, **f)) / math.sqrt(N)
+    bB = 0.1 * torch.randn(H, R, N, **f) / math.sqrt(N)
+    bC = 0.1 * torch.randn(H, R, N, **f) / math.sqrt(N)
+    return dict(wB=wB, wC=wC, bB=bB, bC=bC, eps=1e-6)
+
+
 def make_state(shape: Shape, device="cpu", seed_offset: int = 2, scale: float = 1.0):
     """A random (h, b_prev, x_prev) state in fp32, for tests that start from a
     nonzero state."""

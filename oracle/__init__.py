@@ -50,9 +50,10 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         i64 = ctypes.c_int64
         dp = ctypes.c_void_p
-        lib.m3o_scan.argtypes = [i64] * 6 + [dp] * 8 + [dp] * 3 + [dp] * 4 + [ctypes.c_int] * 3
+        lib.m3o_scan.argtypes = ([i64] * 6 + [dp] * 8 + [dp] * 3 + [dp] * 4 + [ctypes.c_int] * 3 + [dp] * 4
+                                 + [ctypes.c_double])
         lib.m3o_scan.restype = ctypes.c_int
-        lib.m3o_step.argtypes = [i64] * 5 + [dp] * 8 + [dp] * 4 + [ctypes.c_int] * 2
+        lib.m3o_step.argtypes = [i64] * 5 + [dp] * 8 + [dp] * 4 + [ctypes.c_int] * 2 + [dp] * 4 + [ctypes.c_double]
         lib.m3o_step.restype = ctypes.c_int
         lib.m3o_num_cores.argtypes = []
         lib.m3o_num_cores.restype = ctypes.c_int
@@ -77,16 +78,35 @@ def _ptr(a):
 
 
 @dataclass
+class BCNorm:
+    """BC-norm prologue: RMS norm of every (token, head, rank) row of B and C
+    over N, times w [N], plus the head-specific bias b [H, R, N]."""
+    wB: np.ndarray
+    wC: np.ndarray
+    bB: np.ndarray
+    bC: np.ndarray
+    eps: float
+
+
+def _bcn_args(bcn):
+    if bcn is None:
+        return [None] * 4 + [0.0]
+    return [_f64(bcn.wB), _f64(bcn.wC), _f64(bcn.bB), _f64(bcn.bC), float(bcn.eps)]
+
+
+@dataclass
 class State:
     h: np.ndarray       # [Bt, H, N, P]
     b_prev: np.ndarray  # [Bt, H, R, N]
     x_prev: np.ndarray  # [Bt, H, R, P]
 
 
-def scan(x, B, C, dt, lam, theta, A, D, init: State | None = None, nthreads: int = 0):
+def scan(x, B, C, dt, lam, theta, A, D, init: State | None = None, nthreads: int = 0,
+         bcnorm: BCNorm | None = None):
     """Full-sequence scan.  Shapes: x [Bt,T,H,R,P], B/C [Bt,T,H,R,N],
     dt/lam [Bt,T,H], theta [Bt,T,H,N/2] (or [H,N/2]: fixed per head), D [H],
-    A [H] (per head) or [Bt,T,H] (per token).  Returns (y, State)."""
+    A [H] (per head) or [Bt,T,H] (per token); optional BC-norm prologue.
+    Returns (y, State)."""
     x, B, C, dt, lam, theta, A, D = map(_f64, (x, B, C, dt, lam, theta, A, D))
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
@@ -104,15 +124,17 @@ def scan(x, B, C, dt, lam, theta, A, D, init: State | None = None, nthreads: int
     hT = np.zeros((Bt, H, N, P))
     bpT = np.zeros((Bt, H, R, N))
     xpT = np.zeros((Bt, H, R, P))
+    bn = _bcn_args(bcnorm)
     rc = _load().m3o_scan(Bt, T, H, P, N, R, *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
                           _ptr(h0), _ptr(bp0), _ptr(xp0),
-                          _ptr(y), _ptr(hT), _ptr(bpT), _ptr(xpT), int(nthreads), a_tok, th_head)
+                          _ptr(y), _ptr(hT), _ptr(bpT), _ptr(xpT), int(nthreads), a_tok, th_head,
+                          *map(_ptr, bn[:4]), bn[4])
     if rc != 0:
         raise ValueError("oracle scan rejected its arguments")
     return y, State(hT, bpT, xpT)
 
 
-def step(x, B, C, dt, lam, theta, A, D, state: State):
+def step(x, B, C, dt, lam, theta, A, D, state: State, bcnorm: BCNorm | None = None):
     """One decode step for every (b,h).  x [Bt,H,R,P], B/C [Bt,H,R,N],
     dt/lam [Bt,H], theta [Bt,H,N/2], D [H], A [H] or [Bt,H] (per token).
     Returns (y, new State); the input state is not modified."""
@@ -127,8 +149,9 @@ def step(x, B, C, dt, lam, theta, A, D, state: State):
     assert theta.shape in ((Bt, H, N // 2), (H, N // 2))
     a_tok = int(A.ndim == 2)
     th_head = int(theta.ndim == 2)
+    bn = _bcn_args(bcnorm)
     rc = _load().m3o_step(Bt, H, P, N, R, *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
-                          _ptr(h), _ptr(bp), _ptr(xp), _ptr(y), a_tok, th_head)
+                          _ptr(h), _ptr(bp), _ptr(xp), _ptr(y), a_tok, th_head, *map(_ptr, bn[:4]), bn[4])
     if rc != 0:
         raise ValueError("oracle step rejected its arguments")
     return y, State(h, bp, xp)

@@ -49,6 +49,17 @@
  * where the eigenvalue's phase is a learned constant): the token's angle is
  * then D_t * theta[h][k], everything else unchanged.
  *
+ * BC-norm prologue (optional).  Mamba-3 normalises the B and C projections
+ * with an RMS norm, as QKNorm does for queries and keys, and adds learnable
+ * head-specific biases after the norm ("Знакомство с Mamba-3", section
+ * "Архитектура и нормализация"; "Mamba-3, parte 1", paragraphs on the
+ * normalisations and on dropping the short convolution).  Reading taken here:
+ * every (token, head, rank) row of B (and of C) over its N entries becomes
+ *   B^ = B / sqrt(mean_n B^2 + eps) * w_B + b_B[h, r],
+ * w_B [N] shared by heads and ranks, b_B [H, R, N]; the recurrence then uses
+ * B^ and C^ wherever it used B and C (rotation included), and b_prev holds
+ * the last token's B^.
+ *
  * Layouts (row-major, last index fastest), all fp64 here:
  *   x, y  [Bt, T, H, R, P]     B, C [Bt, T, H, R, N]
  *   dt, lam [Bt, T, H]         theta [Bt, T, H, N/2]      D [H]
@@ -69,6 +80,8 @@ typedef struct {
     double *y, *hT, *bpT, *xpT;   /* y required; final-state outputs nullable */
     int a_per_token;              /* A is [Bt, T, H] instead of [H] */
     int theta_per_head;           /* theta is [H, N/2] instead of [Bt, T, H, N/2] */
+    const double *wB, *wC, *bB, *bC; /* BC-norm (all or none) */
+    double eps;
     int64_t next;                 /* next (b,h) slice to claim */
     pthread_mutex_t lock;
 } job_t;
@@ -125,6 +138,18 @@ static void token_update(int64_t N, int64_t P, int64_t R,
     memcpy(xp, xt, sizeof(double) * (size_t)(R * P));
 }
 
+/* The BC-norm of one token's R rows of N entries, out of place. */
+static void bc_norm(int64_t N, int64_t R, const double *in, const double *w, const double *bias,
+                    double eps, double *out)
+{
+    for (int64_t r = 0; r < R; ++r) {
+        double ss = 0.0;
+        for (int64_t n = 0; n < N; ++n) ss += in[r * N + n] * in[r * N + n];
+        const double inv = 1.0 / sqrt(ss / (double)N + eps);
+        for (int64_t n = 0; n < N; ++n) out[r * N + n] = in[r * N + n] * inv * w[n] + bias[r * N + n];
+    }
+}
+
 static void run_slice(job_t *j, int64_t bh)
 {
     const int64_t H = j->H, T = j->T, N = j->N, P = j->P, R = j->R;
@@ -135,16 +160,27 @@ static void run_slice(job_t *j, int64_t bh)
     if (j->h0) memcpy(h, j->h0 + bh * N * P, sizeof(double) * (size_t)(N * P));
     if (j->bp0) memcpy(bp, j->bp0 + bh * R * N, sizeof(double) * (size_t)(R * N));
     if (j->xp0) memcpy(xp, j->xp0 + bh * R * P, sizeof(double) * (size_t)(R * P));
+    double *Bn = (double *)malloc(sizeof(double) * (size_t)(R * N));
+    double *Cn = (double *)malloc(sizeof(double) * (size_t)(R * N));
     for (int64_t t = 0; t < T; ++t) {
         const int64_t th_ = (b * T + t) * H + hd; /* token-head index */
-        token_update(N, P, R, h, bp, xp, j->x + th_ * R * P, j->B + th_ * R * N,
-                     j->C + th_ * R * N, j->dt[th_], j->lam[th_],
+        const double *Bt = j->B + th_ * R * N, *Ct = j->C + th_ * R * N;
+        if (j->wB) {
+            bc_norm(N, R, Bt, j->wB, j->bB + hd * R * N, j->eps, Bn);
+            bc_norm(N, R, Ct, j->wC, j->bC + hd * R * N, j->eps, Cn);
+            Bt = Bn;
+            Ct = Cn;
+        }
+        token_update(N, P, R, h, bp, xp, j->x + th_ * R * P, Bt,
+                     Ct, j->dt[th_], j->lam[th_],
                      j->theta + (j->theta_per_head ? hd : th_) * (N / 2), j->A[j->a_per_token ? th_ : hd], j->D[hd],
                      j->y + th_ * R * P);
     }
     if (j->hT) memcpy(j->hT + bh * N * P, h, sizeof(double) * (size_t)(N * P));
     if (j->bpT) memcpy(j->bpT + bh * R * N, bp, sizeof(double) * (size_t)(R * N));
     if (j->xpT) memcpy(j->xpT + bh * R * P, xp, sizeof(double) * (size_t)(R * P));
+    free(Bn);
+    free(Cn);
     free(h);
     free(bp);
     free(xp);
@@ -178,7 +214,8 @@ int m3o_scan(int64_t Bt, int64_t T, int64_t H, int64_t P, int64_t N, int64_t R,
              const double *A, const double *D,
              const double *h0, const double *bp0, const double *xp0,
              double *y, double *hT, double *bpT, double *xpT, int nthreads, int a_per_token,
-             int theta_per_head)
+             int theta_per_head, const double *wB, const double *wC, const double *bB,
+             const double *bC, double eps)
 {
     if (Bt < 0 || T < 0 || H <= 0 || P <= 0 || N <= 0 || (N & 1) || R <= 0) return -1;
     if (!y && T > 0) return -1;
@@ -190,6 +227,8 @@ int m3o_scan(int64_t Bt, int64_t T, int64_t H, int64_t P, int64_t N, int64_t R,
     j.y = y; j.hT = hT; j.bpT = bpT; j.xpT = xpT;
     j.a_per_token = a_per_token;
     j.theta_per_head = theta_per_head;
+    if ((wB != NULL) != (wC != NULL) || (wB != NULL) != (bB != NULL) || (wB != NULL) != (bC != NULL)) return -1;
+    j.wB = wB; j.wC = wC; j.bB = bB; j.bC = bC; j.eps = eps;
     pthread_mutex_init(&j.lock, NULL);
     int nt = nthreads > 0 ? nthreads : m3o_num_cores();
     if (nt > Bt * H) nt = (int)(Bt * H);
@@ -214,15 +253,28 @@ int m3o_step(int64_t Bt, int64_t H, int64_t P, int64_t N, int64_t R,
              const double *x, const double *B, const double *C,
              const double *dt, const double *lam, const double *theta,
              const double *A, const double *D,
-             double *h, double *bp, double *xp, double *y, int a_per_token, int theta_per_head)
+             double *h, double *bp, double *xp, double *y, int a_per_token, int theta_per_head,
+             const double *wB, const double *wC, const double *bB, const double *bC, double eps)
 {
+    if ((wB != NULL) != (wC != NULL) || (wB != NULL) != (bB != NULL) || (wB != NULL) != (bC != NULL)) return -1;
     if (Bt < 0 || H <= 0 || P <= 0 || N <= 0 || (N & 1) || R <= 0) return -1;
+    double *Bn = (double *)malloc(sizeof(double) * (size_t)(R * N));
+    double *Cn = (double *)malloc(sizeof(double) * (size_t)(R * N));
     for (int64_t bh = 0; bh < Bt * H; ++bh) {
         const int64_t hd = bh % H;
+        const double *Bt_ = B + bh * R * N, *Ct_ = C + bh * R * N;
+        if (wB) {
+            bc_norm(N, R, Bt_, wB, bB + hd * R * N, eps, Bn);
+            bc_norm(N, R, Ct_, wC, bC + hd * R * N, eps, Cn);
+            Bt_ = Bn;
+            Ct_ = Cn;
+        }
         token_update(N, P, R, h + bh * N * P, bp + bh * R * N, xp + bh * R * P,
-                     x + bh * R * P, B + bh * R * N, C + bh * R * N, dt[bh], lam[bh],
+                     x + bh * R * P, Bt_, Ct_, dt[bh], lam[bh],
                      theta + (theta_per_head ? hd : bh) * (N / 2), A[a_per_token ? bh : hd], D[hd],
                      y + bh * R * P);
     }
+    free(Bn);
+    free(Cn);
     return 0;
 }

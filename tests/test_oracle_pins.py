@@ -516,3 +516,73 @@ def test_theta_per_head_free_rotation_closed_form():
     z0 = h[0, :, 0::2, :] + 1j * h[0, :, 1::2, :]                   # [H, N/2, P]
     z = np.exp((cd * d["A"])[:, None, None] - 1j * (cd[:, None] * d["theta"])[:, :, None]) * z0
     assert rel(fs.h[0, :, 0::2, :], z.real) < TOL and rel(fs.h[0, :, 1::2, :], z.imag) < TOL
+
+
+# ---------------------------------------------------------------- BC-norm prologue
+def bcn_case(T=21, R=2, seed=14, eps=1e-6):
+    from m3_inputs import make_bcnorm
+    s = Shape(1, T, 2, 5, 8, R, "f32", seed)
+    d = {k: v.double().numpy() for k, v in make_prefill(s).items()}
+    bn = {k: (v.double().numpy() if hasattr(v, "double") else v) for k, v in make_bcnorm(s).items()}
+    h, bp, xp = (t.double().numpy() for t in make_state(s))
+    return d, oracle.BCNorm(bn["wB"], bn["wC"], bn["bB"], bn["bC"], eps), oracle.State(h, bp, xp)
+
+
+def run_bcn(d, bcn, st=None):
+    return oracle.scan(d["x"], d["B"], d["C"], d["dt"], d["lam"], d["theta"], d["A"], d["D"], st, bcnorm=bcn)
+
+
+def test_bcnorm_row_scale_invariance():
+    """The RMS norm divides out any positive scale of a (token, head, rank)
+    row: rescaling every row of B and C by its own factor leaves y and the
+    state unchanged (eps negligible)."""
+    d, bcn, st = bcn_case(eps=1e-300)
+    y1, f1 = run_bcn(d, bcn, st)
+    rng = np.random.default_rng(3)
+    d2 = dict(d)
+    d2["B"] = d["B"] * rng.uniform(0.1, 10.0, size=d["B"].shape[:-1] + (1,))
+    d2["C"] = d["C"] * rng.uniform(0.1, 10.0, size=d["C"].shape[:-1] + (1,))
+    y2, f2 = run_bcn(d2, bcn, st)
+    assert rel(y2, y1) < 1e-12 and rel(f2.h, f1.h) < 1e-12 and rel(f2.b_prev, f1.b_prev) < 1e-12
+
+
+def unit_rms(a):
+    return a / np.sqrt(np.mean(a * a, axis=-1, keepdims=True))
+
+
+def test_bcnorm_identity_on_unit_rms_rows():
+    """Rows already at unit RMS, w = 1, no bias: the prologue is the identity."""
+    d, bcn, st = bcn_case(eps=1e-300)
+    d["B"], d["C"] = unit_rms(d["B"]), unit_rms(d["C"])
+    N = d["B"].shape[-1]
+    ident = oracle.BCNorm(np.ones(N), np.ones(N), np.zeros_like(bcn.bB), np.zeros_like(bcn.bC), 1e-300)
+    y1, f1 = run_bcn(d, ident, st)
+    y2, f2 = run(d, st)
+    assert rel(y1, y2) < 1e-12 and rel(f1.h, f2.h) < 1e-12
+
+
+def test_bcnorm_weight_and_bias_placement():
+    """Unit-RMS rows: the prologue reduces to B w + b[h, r] (w over the state
+    index, b per head and rank), i.e. the plain method on those inputs."""
+    d, bcn, st = bcn_case(eps=1e-300)
+    d["B"], d["C"] = unit_rms(d["B"]), unit_rms(d["C"])
+    y1, f1 = run_bcn(d, bcn, st)
+    d2 = dict(d)
+    d2["B"] = d["B"] * bcn.wB + bcn.bB[None, None]
+    d2["C"] = d["C"] * bcn.wC + bcn.bC[None, None]
+    y2, f2 = run(d2, st)
+    assert rel(y1, y2) < 1e-12 and rel(f1.h, f2.h) < 1e-12 and rel(f1.b_prev, f2.b_prev) < 1e-12
+
+
+def test_bcnorm_decode_continues_the_scan():
+    d, bcn, st = bcn_case(T=16)
+    y_full, f_full = run_bcn(d, bcn, st)
+    k = 9
+    part = {key: (v[:, :k] if v.ndim >= 3 else v) for key, v in d.items()}
+    _, fs = run_bcn(part, bcn, st)
+    ys = []
+    for t in range(k, 16):
+        args = [d[key][:, t] for key in ("x", "B", "C", "dt", "lam", "theta")]
+        yt, fs = oracle.step(*args, d["A"], d["D"], fs, bcnorm=bcn)
+        ys.append(yt)
+    assert rel(np.stack(ys, 1), y_full[:, k:]) < TOL and rel(fs.h, f_full.h) < TOL
