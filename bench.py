@@ -360,7 +360,7 @@ def run_ours(args):
     # ---- decode step: state from a 1024-token prefill, then single-token steps in one CUDA graph
     if not args.no_variants and use_tc:
         line["variants"] = [run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
-                                        peak_src, keys, stream) for kind in ("a_per_token", "theta_per_head")]
+                                        peak_src, keys, stream) for kind in VARIANTS]
     if not args.no_decode:
         del inp, y, fin
         torch.cuda.empty_cache()
@@ -393,7 +393,8 @@ def _tc_supported(m3, inp, keys, algo):
 
 
 VARIANTS = {"a_per_token": "data-dependent A_t (M3_FLAG_A_PER_TOKEN)",
-            "theta_per_head": "angle rates fixed per head (M3_FLAG_THETA_PER_HEAD)"}
+            "theta_per_head": "angle rates fixed per head (M3_FLAG_THETA_PER_HEAD)",
+            "bcnorm": "fused BC-norm prologue (m3_scan_fwd_bcnorm)"}
 
 
 def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys, stream):
@@ -403,25 +404,33 @@ def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_p
     import torch
     from m3_inputs import WORKLOADS, make_prefill
 
+    from m3_inputs import make_bcnorm
+
     s = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
-    inp = make_prefill(s, device=dev, **{kind: True})
+    inp = make_prefill(s, device=dev, **({} if kind == "bcnorm" else {kind: True}))
+    bcn = None
+    if kind == "bcnorm":
+        p = make_bcnorm(s, device=dev)
+        bcn = m3.BCNorm(p["wB"], p["wC"], p["bB"], p["bC"], p["eps"])
     y = torch.empty_like(inp["x"])
     fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device=dev)
     for _ in range(args.warmup):
-        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream)
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream, bcnorm=bcn)
     K = args.steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(K):
-        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream)
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream, bcnorm=bcn)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     m3.stream_status(stream)
     el = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-    ab = prefill_bytes(s, **{kind: True})
+    ab = prefill_bytes(s, **({} if kind == "bcnorm" else {kind: True}))
+    if kind == "bcnorm":  # the norm weights and the biases, read once
+        ab += 4 * (2 * s.dstate + 2 * s.nheads * s.rank * s.dstate)
     ach = ab / (el / K) / 1e9
     del inp, y, fin
     torch.cuda.empty_cache()

@@ -107,6 +107,25 @@ typedef struct m3_state {
     float *x_prev;  /* [batch, nheads, rank, headdim]   */
 } m3_state;
 
+/* BC-norm prologue (optional).  Mamba-3 normalises the B and C projections
+ * with an RMS norm, as QKNorm does for queries and keys, and adds learnable
+ * head-specific biases after the norm ("Знакомство с Mamba-3", section
+ * "Архитектура и нормализация"; "Mamba-3, parte 1", paragraphs on the
+ * normalisations and on dropping the short convolution).  With it, every
+ * (token, head, rank) row of B -- and of C -- over its dstate entries becomes
+ *     B^ = B / sqrt(mean_n B^2 + eps) * wB + bB[head][rank]
+ * before anything else uses it (the rotation included), and the state's
+ * b_prev holds the last token's B^.  All device pointers, fp32, caller-owned:
+ *     wB, wC  [dstate]                      (shared by heads and ranks)
+ *     bB, bC  [nheads, rank, dstate]        (head-specific biases)
+ * eps > 0.  The pages give the norm and the biases, not their shapes or eps;
+ * these are this library's reading. */
+typedef struct m3_bcnorm {
+    const float *wB, *wC;
+    const float *bB, *bC;
+    float eps;
+} m3_bcnorm;
+
 /* Prefill kernel selection for m3_scan_fwd_algo. */
 typedef enum m3_algo {
     M3_ALGO_AUTO = 0,   /* tensor-core path for bf16 where supported, else SIMT */
@@ -170,6 +189,14 @@ M3_API m3_status m3_scan_fwd_algo(int algo, const m3_dims *d,
                            const m3_state *init, void *y, const m3_state *final_state,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* m3_scan_fwd_algo with the BC-norm prologue fused in (`bcn` required). */
+M3_API m3_status m3_scan_fwd_bcnorm(int algo, const m3_dims *d, const m3_bcnorm *bcn,
+                             const void *x, const void *B, const void *C,
+                             const void *dt, const void *lam, const void *theta,
+                             const float *A, const float *D,
+                             const m3_state *init, void *y, const m3_state *final_state,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* m3_scan_fwd_algo without a workspace argument: the per-segment states of
  * split sequences go to a scratch area the library itself holds in device
  * memory (a static 24 MiB array, reserved on each device when the library's
@@ -203,6 +230,14 @@ M3_API m3_status m3_step(const m3_dims *d,
                   const void *dt, const void *lam, const void *theta,
                   const float *A, const float *D,
                   const m3_state *state, void *y, void *stream);
+
+/* m3_step with the BC-norm prologue fused in (`bcn` required); the state's
+ * b_prev must hold normalised B (as m3_scan_fwd_bcnorm leaves it). */
+M3_API m3_status m3_step_bcnorm(const m3_dims *d, const m3_bcnorm *bcn,
+                         const void *x, const void *B, const void *C,
+                         const void *dt, const void *lam, const void *theta,
+                         const float *A, const float *D,
+                         const m3_state *state, void *y, void *stream);
 
 /* Wait for all work queued on `stream` (blocking the calling host thread),
  * then report any device-side failure recorded since the previous call:

@@ -37,6 +37,26 @@ class Dims(ctypes.Structure):
                 ("io", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
+class CBCNorm(ctypes.Structure):
+    _fields_ = [("wB", ctypes.c_void_p), ("wC", ctypes.c_void_p), ("bB", ctypes.c_void_p),
+                ("bC", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
+class BCNorm(NamedTuple):
+    """BC-norm prologue parameters (device fp32 tensors): RMS-norm weights
+    wB, wC [N] and head-specific biases bB, bC [H, R, N]; eps > 0."""
+    wB: torch.Tensor
+    wC: torch.Tensor
+    bB: torch.Tensor
+    bC: torch.Tensor
+    eps: float = 1e-6
+
+
+def _cbcn(b: BCNorm):
+    _require_cuda(b.wB, b.wC, b.bB, b.bC)
+    return ctypes.byref(CBCNorm(b.wB.data_ptr(), b.wC.data_ptr(), b.bB.data_ptr(), b.bC.data_ptr(), float(b.eps)))
+
+
 class CState(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("b_prev", ctypes.c_void_p), ("x_prev", ctypes.c_void_p)]
 
@@ -65,6 +85,11 @@ def _load():
                                  ctypes.POINTER(ctypes.c_int)]
     lib.m3_scan_fwd.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     lib.m3_scan_fwd_algo.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    bp_ = ctypes.POINTER(CBCNorm)
+    lib.m3_scan_fwd_bcnorm.argtypes = [ctypes.c_int, dp, bp_] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_scan_fwd_bcnorm.restype = ctypes.c_int
+    lib.m3_step_bcnorm.argtypes = [dp, bp_] + [vp] * 8 + [sp, vp, vp]
+    lib.m3_step_bcnorm.restype = ctypes.c_int
     lib.m3_scan_fwd_static.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp]
     lib.m3_scan_fwd_static.restype = ctypes.c_int
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
@@ -160,8 +185,9 @@ def scan_plan(dims: Dims, algo: int = ALGO_AUTO) -> Plan:
 
 
 def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
-             y=None, final: State | None = None, workspace=None, algo: int = ALGO_AUTO, stream=None):
-    """Prefill scan.  x [Bt,T,H,R,P], B/C [Bt,T,H,R,N], dt/lam [Bt,T,H],
+             y=None, final: State | None = None, workspace=None, algo: int = ALGO_AUTO, stream=None,
+             bcnorm: BCNorm | None = None):
+    """Prefill scan (with the BC-norm prologue when `bcnorm` is given).  x [Bt,T,H,R,P], B/C [Bt,T,H,R,N], dt/lam [Bt,T,H],
     theta [Bt,T,H,N/2] (or [H,N/2]: fixed per head) in one io dtype (fp32 or
     bf16); D [H] fp32; A [H] fp32, or [Bt,T,H] fp32 for a data-dependent A_t.
     Returns (y, final State or None)."""
@@ -178,9 +204,12 @@ def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_s
     if workspace is None and ws_need:
         workspace = torch.empty(ws_need, dtype=torch.uint8, device=x.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(get_lib().m3_scan_fwd_algo(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
-                                _cstate(init), _ptr(y), _cstate(final), _ptr(workspace), ws_bytes,
-                                _stream(stream)))
+    args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(init), _ptr(y), _cstate(final), _ptr(workspace),
+            ws_bytes, _stream(stream))
+    if bcnorm is None:
+        _check(get_lib().m3_scan_fwd_algo(algo, ctypes.byref(dims), *args))
+    else:
+        _check(get_lib().m3_scan_fwd_bcnorm(algo, ctypes.byref(dims), _cbcn(bcnorm), *args))
     return y, final
 
 
@@ -213,7 +242,7 @@ def stream_status(stream=None):
     _check(get_lib().m3_stream_status(_stream(stream)))
 
 
-def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None):
+def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None, bcnorm: BCNorm | None = None):
     """One decode step in place on `state`.  x [Bt,H,R,P], B/C [Bt,H,R,N],
     dt/lam [Bt,H], theta [Bt,H,N/2] (or [H,N/2]: fixed per head); A [H] fp32,
     or [Bt,H] fp32 for a data-dependent A_t.  Returns y [Bt,H,R,P]."""
@@ -223,6 +252,9 @@ def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None):
     dims = make_dims(Bt, 1, H, P, N, R, x.dtype, a_per_token=A.dim() == 2, theta_per_head=theta.dim() == 2)
     if y is None:
         y = torch.empty_like(x)
-    _check(get_lib().m3_step(ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state),
-                       _ptr(y), _stream(stream)))
+    args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state), _ptr(y), _stream(stream))
+    if bcnorm is None:
+        _check(get_lib().m3_step(ctypes.byref(dims), *args))
+    else:
+        _check(get_lib().m3_step_bcnorm(ctypes.byref(dims), _cbcn(bcnorm), *args))
     return y

@@ -137,10 +137,27 @@ m3::Problem make_problem(const m3_dims *d, const void *x, const void *B, const v
     return p;
 }
 
+// BC-norm parameters: all four arrays, 4-byte aligned, eps > 0, no overlap with y.
+m3_status check_bcnorm(const m3_dims *d, const m3_bcnorm *bcn, Range yr) {
+    if (!bcn) return fail(M3_ERR_INVALID_ARG, "bcn is NULL");
+    if (!bcn->wB || !bcn->wC || !bcn->bB || !bcn->bC)
+        return fail(M3_ERR_INVALID_ARG, "bcn: wB, wC, bB and bC are all required");
+    if ((reinterpret_cast<uintptr_t>(bcn->wB) | reinterpret_cast<uintptr_t>(bcn->wC) |
+         reinterpret_cast<uintptr_t>(bcn->bB) | reinterpret_cast<uintptr_t>(bcn->bC)) % 4)
+        return fail(M3_ERR_INVALID_ARG, "bcn arrays must be 4-byte aligned");
+    if (!(bcn->eps > 0.f)) return fail(M3_ERR_INVALID_ARG, "bcn eps must be > 0");
+    const Range rs[4] = {range(bcn->wB, d->dstate * 4), range(bcn->wC, d->dstate * 4),
+                         range(bcn->bB, d->nheads * d->rank * d->dstate * 4),
+                         range(bcn->bC, d->nheads * d->rank * d->dstate * 4)};
+    for (const Range &r : rs)
+        if (overlap(r, yr)) return fail(M3_ERR_INVALID_ARG, "y overlaps a bcn array");
+    return M3_OK;
+}
+
 m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
                     const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
                     void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream,
-                    bool static_ws = false) {
+                    bool static_ws = false, const m3_bcnorm *bcn = nullptr) {
     m3_status s = check_dims(d, false);
     if (s != M3_OK) return s;
     const int segments = algo >> 8;
@@ -169,7 +186,9 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
                 return fail(M3_ERR_INVALID_ARG, "final_state partially overlaps init");
         }
     }
+    if (bcn && (s = check_bcnorm(d, bcn, yr)) != M3_OK) return s;
     m3::Problem p = make_problem(d, x, B, C, dt, lam, theta, A, D, y, stream);
+    if (bcn) { p.wB = bcn->wB; p.wC = bcn->wC; p.bB = bcn->bB; p.bC = bcn->bC; p.eps = bcn->eps; }
     if (init) { p.h0 = init->h; p.bp0 = init->b_prev; p.xp0 = init->x_prev; }
     if (fin) { p.hT = fin->h; p.bpT = fin->b_prev; p.xpT = fin->x_prev; }
     p.ws = ws;
@@ -278,6 +297,19 @@ m3_status m3_scan_fwd_algo(int algo, const m3_dims *d, const void *x, const void
     }
 }
 
+m3_status m3_scan_fwd_bcnorm(int algo, const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B,
+                             const void *C, const void *dt, const void *lam, const void *theta, const float *A,
+                             const float *D, const m3_state *init, void *y, const m3_state *final_state,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    try {
+        if (!bcn) return fail(M3_ERR_INVALID_ARG, "bcn is NULL");
+        return scan_impl(algo, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace,
+                         workspace_bytes, stream, false, bcn);
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
 m3_status m3_scan_fwd_static(int algo, const m3_dims *d, const void *x, const void *B, const void *C,
                              const void *dt, const void *lam, const void *theta, const float *A, const float *D,
                              const m3_state *init, void *y, const m3_state *final_state, void *stream) {
@@ -319,9 +351,26 @@ m3_status m3_stream_status(void *stream) {
     }
 }
 
+m3_status step_impl(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B, const void *C,
+                    const void *dt, const void *lam, const void *theta, const float *A, const float *D,
+                    const m3_state *state, void *y, void *stream);
+
 m3_status m3_step(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
                   const void *lam, const void *theta, const float *A, const float *D, const m3_state *state,
                   void *y, void *stream) {
+    return step_impl(d, nullptr, x, B, C, dt, lam, theta, A, D, state, y, stream);
+}
+
+m3_status m3_step_bcnorm(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B, const void *C,
+                         const void *dt, const void *lam, const void *theta, const float *A, const float *D,
+                         const m3_state *state, void *y, void *stream) {
+    if (!bcn) return fail(M3_ERR_INVALID_ARG, "bcn is NULL");
+    return step_impl(d, bcn, x, B, C, dt, lam, theta, A, D, state, y, stream);
+}
+
+m3_status step_impl(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B, const void *C,
+                    const void *dt, const void *lam, const void *theta, const float *A, const float *D,
+                    const m3_state *state, void *y, void *stream) {
     try {
         m3_status s = check_dims(d, true);
         if (s != M3_OK) return s;
@@ -338,7 +387,9 @@ m3_status m3_step(const m3_dims *d, const void *x, const void *B, const void *C,
             for (int j = 0; j < nin; ++j)
                 if (overlap(sr[i], ins[j])) return fail(M3_ERR_INVALID_ARG, "state overlaps an input tensor");
         }
+        if (bcn && (s = check_bcnorm(d, bcn, yr)) != M3_OK) return s;
         m3::Problem p = make_problem(d, x, B, C, dt, lam, theta, A, D, y, stream);
+        if (bcn) { p.wB = bcn->wB; p.wC = bcn->wC; p.bB = bcn->bB; p.bC = bcn->bC; p.eps = bcn->eps; }
         p.T = 1;
         p.hT = state->h; p.bpT = state->b_prev; p.xpT = state->x_prev;
         const char *why = nullptr;

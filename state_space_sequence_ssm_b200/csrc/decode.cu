@@ -17,6 +17,7 @@
 // N is a warp shuffle plus one shared-memory pass.
 #include <cuda_bf16.h>
 
+#include "bcnorm.cuh"
 #include "m3_internal.h"
 #include "tc_primitives.cuh"
 
@@ -79,6 +80,8 @@ struct StepArgs {
     const float *A, *D;
     int a_tok;    // A is [Bt, H] (per token-head) instead of [H]
     int th_head;  // theta is [H, N/2] (fixed per head)
+    const float *wB, *wC, *bB, *bC;  // BC-norm prologue (wB == nullptr: off)
+    float eps;
     float *h, *bp, *xp;
     IO *y;
 };
@@ -146,6 +149,19 @@ step_kernel(const StepArgs<IO> a) {
         sAs[k] = alpha * sn;
     }
     __syncthreads();
+    if (a.wB) {  // BC-norm prologue on the staged rows: one warp per row of B, then of C
+        const int warp = tid / 32, lane = tid % 32;
+        for (int row = warp; row < 2 * R; row += Cfg::WARPS) {
+            const bool isB = row < R;
+            const int r = isB ? row : row - R;
+            float *v = isB ? sB[r] : sC[r];
+            const float *w = isB ? a.wB : a.wC;
+            const float *bias = (isB ? a.bB : a.bC) + (h * R + r) * N;
+            const float sc = bcn_row_scale_warp([&](int n) { return v[n]; }, N, a.eps);
+            for (int n = lane; n < N; n += 32) v[n] = fmaf(v[n] * sc, w[n], bias[n]);
+        }
+        __syncthreads();
+    }
 
     float4 yacc[R];
 #pragma unroll
@@ -224,12 +240,28 @@ step_kernel(const StepArgs<IO> a) {
 // shared-memory atomics for the readout.  Same arithmetic, no tiling.
 template <typename IO>
 __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a) {
-    extern __shared__ float ysum[];  // [R][P]
+    extern __shared__ float ysum[];  // [R][P], then (BC-norm) normalised B and C [R][N] each
     const int N = a.N, P = a.P, R = a.R, K2 = N / 2;
     const int64_t bh = blockIdx.x;
     const int h = (int)(bh % a.H);
+    float *nB = ysum + R * P, *nC = nB + R * N;
     for (int i = threadIdx.x; i < R * P; i += blockDim.x) ysum[i] = 0.f;
+    if (a.wB) {  // BC-norm prologue: one warp per row of B, then of C
+        const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+        for (int row = warp; row < 2 * R; row += blockDim.x / 32) {
+            const bool isB = row < R;
+            const int r = isB ? row : row - R;
+            const IO *src = (isB ? a.B : a.C) + (bh * R + r) * N;
+            const float *w = isB ? a.wB : a.wC;
+            const float *bias = (isB ? a.bB : a.bC) + (h * R + r) * N;
+            float *dst = (isB ? nB : nC) + r * N;
+            const float sc = bcn_row_scale_warp([&](int n) { return ldv(src, n); }, N, a.eps);
+            for (int n = lane; n < N; n += 32) dst[n] = fmaf(ldv(src, n) * sc, w[n], bias[n]);
+        }
+    }
     __syncthreads();
+    auto Bv = [&](int i) { return a.wB ? nB[i] : ldv(a.B, bh * R * N + i); };  // i = r * N + n
+    auto Cv = [&](int i) { return a.wB ? nC[i] : ldv(a.C, bh * R * N + i); };
     const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
     const float alpha = expf(dtv * a.A[a.a_tok ? bh : h]);
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
@@ -247,14 +279,13 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a)
         float nu = alpha * (u * cs + v * sn), nv = alpha * (-u * sn + v * cs);
         for (int r = 0; r < R; ++r) {
             const float xx = ldv(a.x, (bh * R + r) * P + p);
-            nu += gam * ldv(a.B, (bh * R + r) * N + 2 * k) * xx;
-            nv += gam * ldv(a.B, (bh * R + r) * N + 2 * k + 1) * xx;
+            nu += gam * Bv(r * N + 2 * k) * xx;
+            nv += gam * Bv(r * N + 2 * k + 1) * xx;
         }
         hs[(2 * k) * P + p] = nu;
         hs[(2 * k + 1) * P + p] = nv;
         for (int r = 0; r < R; ++r)
-            atomicAdd(&ysum[r * P + p], nu * ldv(a.C, (bh * R + r) * N + 2 * k) +
-                                            nv * ldv(a.C, (bh * R + r) * N + 2 * k + 1));
+            atomicAdd(&ysum[r * P + p], nu * Cv(r * N + 2 * k) + nv * Cv(r * N + 2 * k + 1));
     }
     __syncthreads();
     const float Dh = a.D[h];
@@ -263,8 +294,7 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a)
         stv(a.y, bh * R * P + idx, ysum[idx] + Dh * xval);
         a.xp[bh * R * P + idx] = xval;
     }
-    for (int idx = threadIdx.x; idx < R * N; idx += blockDim.x)
-        a.bp[bh * R * N + idx] = ldv(a.B, bh * R * N + idx);
+    for (int idx = threadIdx.x; idx < R * N; idx += blockDim.x) a.bp[bh * R * N + idx] = Bv(idx);
 }
 
 // Persistent streaming variant: each CTA walks slices bh = blockIdx.x,
@@ -497,8 +527,10 @@ cudaError_t dispatch_np(const StepArgs<IO> &a, cudaStream_t s, bool *done) {
     *done = true;
     // rank 1: one CTA per slice (measured faster); rank >= 2: the persistent
     // streaming kernel (its heavier per-element work overlaps the next slice's load)
-    if (a.N == 128 && a.P == 64) return R == 1 ? launch_tiled<128, 64, R, IO>(a, s) : launch_stream<128, 64, R, IO>(a, s);
-    if (a.N == 64 && a.P == 64) return R == 1 ? launch_tiled<64, 64, R, IO>(a, s) : launch_stream<64, 64, R, IO>(a, s);
+    // (BC-norm: the tiled kernel, which normalises its staged rows in place)
+    const bool tiled = R == 1 || a.wB;
+    if (a.N == 128 && a.P == 64) return tiled ? launch_tiled<128, 64, R, IO>(a, s) : launch_stream<128, 64, R, IO>(a, s);
+    if (a.N == 64 && a.P == 64) return tiled ? launch_tiled<64, 64, R, IO>(a, s) : launch_stream<64, 64, R, IO>(a, s);
     if (a.N == 128 && a.P == 128) return launch_tiled<128, 128, R, IO>(a, s);
     if (a.N == 64 && a.P == 128) return launch_tiled<64, 128, R, IO>(a, s);
     if (a.N == 256 && a.P == 64) return launch_tiled<256, 64, R, IO>(a, s);
@@ -516,6 +548,7 @@ cudaError_t launch_typed(const Problem &p) {
     a.A = p.A; a.D = p.D;
     a.a_tok = p.a_tok;
     a.th_head = p.th_head;
+    a.wB = p.wB; a.wC = p.wC; a.bB = p.bB; a.bC = p.bC; a.eps = p.eps;
     a.h = p.hT; a.bp = p.bpT; a.xp = p.xpT;
     a.y = (IO *)p.y;
     if (a.BH == 0) return cudaSuccess;
@@ -525,7 +558,7 @@ cudaError_t launch_typed(const Problem &p) {
     else if (a.R == 2) e = dispatch_np<IO, 2>(a, p.stream, &done);
     else if (a.R == 4) e = dispatch_np<IO, 4>(a, p.stream, &done);
     if (done) return e;
-    const size_t smem = sizeof(float) * (size_t)a.R * a.P;
+    const size_t smem = sizeof(float) * ((size_t)a.R * a.P + (a.wB ? 2 * (size_t)a.R * a.N : 0));
     step_generic_kernel<IO><<<(unsigned)a.BH, 256, smem, p.stream>>>(a);
     return cudaGetLastError();
 }

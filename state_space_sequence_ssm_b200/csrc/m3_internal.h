@@ -14,6 +14,8 @@ struct Problem {
     bool bf16;
     bool a_tok;                   // A per token-head ([Bt,T,H]; decode [Bt,H]) instead of per head
     bool th_head;                 // theta fixed per head ([H,N/2]) instead of per token-head
+    const float *wB, *wC, *bB, *bC;  // BC-norm prologue (wB == nullptr: off)
+    float eps;
     const void *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
     const float *h0, *bp0, *xp0;  // nullable (zero initial state)

@@ -18,6 +18,7 @@
 // fp32 I/O and the in-repo cross-check of the tensor-core kernel.
 #include <cuda_bf16.h>
 
+#include "bcnorm.cuh"
 #include "m3_internal.h"
 
 namespace m3 {
@@ -48,6 +49,8 @@ struct SimtArgs {
     const float *A, *D;
     int a_tok;    // A is [Bt, T, H] (per token-head)
     int th_head;  // theta is [H, N/2] (fixed per head)
+    const float *wB, *wC, *bB, *bC;  // BC-norm prologue (wB == nullptr: off)
+    float eps;
     const float *h0, *bp0, *xp0;
     IO *y;
     float *hT, *bpT, *xpT;
@@ -135,6 +138,19 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             ghat[s] = l * d + nxt;
         }
         __syncthreads();
+        if (a.wB) {  // BC-norm prologue: one warp per (token, rank) row of B, then of C
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int row = warp; row < 2 * rows; row += kThreads / 32) {
+                const bool isB = row < rows;
+                float *v = isB ? Bs + row * N : Cs + (row - rows) * N;
+                const int r = (isB ? row : row - rows) % R;
+                const float *w = isB ? a.wB : a.wC;
+                const float *bias = (isB ? a.bB : a.bC) + (h * R + r) * N;
+                const float sc = bcn_row_scale_warp([&](int n) { return v[n]; }, N, a.eps);
+                for (int n = lane; n < N; n += 32) v[n] = fmaf(v[n] * sc, w[n], bias[n]);
+            }
+            __syncthreads();
+        }
         if (tid == 0) {  // chunk-local inclusive prefix of dt*A
             float run = 0.f;
             for (int s = 0; s < L; ++s) { run += cA[s]; cA[s] = run; }
@@ -223,7 +239,15 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             a.hT[bh * N * P + idx] = v;
         }
     }
-    if (a.bpT) {
+    if (a.bpT && a.wB && T > 0) {  // the last token's normalised B, one warp per rank row
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int r = warp; r < R; r += kThreads / 32) {
+            const int64_t src = tok(T - 1) * R * N + r * N;
+            const float sc = bcn_row_scale_warp([&](int n) { return ldv(a.B, src + n); }, N, a.eps);
+            for (int n = lane; n < N; n += 32)
+                a.bpT[(bh * R + r) * N + n] = fmaf(ldv(a.B, src + n) * sc, a.wB[n], a.bB[(h * R + r) * N + n]);
+        }
+    } else if (a.bpT) {
         for (int idx = tid; idx < R * N; idx += kThreads)
             a.bpT[bh * R * N + idx] = T > 0 ? ldv(a.B, tok(T - 1) * R * N + idx)
                                             : (a.bp0 ? a.bp0[bh * R * N + idx] : 0.f);
@@ -245,6 +269,7 @@ cudaError_t launch_typed(const Problem &p, const char **why) {
     a.A = p.A; a.D = p.D; a.h0 = p.h0; a.bp0 = p.bp0; a.xp0 = p.xp0;
     a.a_tok = p.a_tok;
     a.th_head = p.th_head;
+    a.wB = p.wB; a.wC = p.wC; a.bB = p.bB; a.bC = p.bC; a.eps = p.eps;
     a.y = (IO *)p.y; a.hT = p.hT; a.bpT = p.bpT; a.xpT = p.xpT;
     // largest chunk (<= 64 rows) whose working set fits in shared memory
     int dev = 0;

@@ -103,7 +103,8 @@ struct Cfg {
     // kNX buffers of {cAl2, gam, ghat, colf}[Q] + {cos, sin}[K2] (read by the
     // state warpgroup a chunk later) + {wst, dts}[Q] + phis[NPART][K2] + wtot[16]
     static constexpr uint32_t SB = 4 * Q + 2 * K2;
-    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16;
+    // + the BC-norm biases of this head as bf16 pairs [2][R][K2]
+    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16 + 2 * R * K2;
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
     static constexpr uint32_t NBARS = 19;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
@@ -122,6 +123,8 @@ struct TcArgs {
     const float *A, *D, *h0, *bp0, *xp0;
     const float *A_tok;  // non-null: A per token-head [Bt, T, H] (A unused)
     int th_head;         // theta fixed per head, [H, N/2]
+    const float *wB, *wC, *bB, *bC;  // BC-norm prologue (BCN instantiations)
+    float eps;
     __nv_bfloat16 *y;
     float *hT, *bpT, *xpT;
     // Split sequences: ws_h [nseg][BH][N][P] fp32 holds, per segment j, the
@@ -194,6 +197,37 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
     __nv_bfloat162 o = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&a),
                                *reinterpret_cast<const __nv_bfloat162 *>(&b));
     return *reinterpret_cast<uint32_t *>(&o);
+}
+
+// BC-norm of one (token, rank) row held by G4 consecutive lanes, 4 pairs each:
+// the row's sum of squares (fp32) is reduced over those lanes, then every entry
+// becomes b * scale * w + bias in packed bf16x2 arithmetic (w: this thread's
+// four weight pairs; bias: its four bias pairs of this head and rank).
+template <int G4>
+__device__ __forceinline__ uint4 bc_norm_row(uint4 v, const uint32_t (&w2)[4], uint4 b2, float inv_n, float eps) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack_bf16(u[e]);
+        ss = fmaf(f.x, f.x, ss);
+        ss = fmaf(f.y, f.y, ss);
+    }
+#pragma unroll
+    for (int off = 1; off < G4; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float sc = rsqrtf(fmaf(ss, inv_n, eps));
+    const uint32_t s2 = pack_bf16(sc, sc);
+    const uint32_t bb[4] = {b2.x, b2.y, b2.z, b2.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const uint32_t sw = mul_bf16x2(s2, w2[e]);
+        __nv_bfloat162 r = __hfma2(*reinterpret_cast<const __nv_bfloat162 *>(&u[e]),
+                                   *reinterpret_cast<const __nv_bfloat162 *>(&sw),
+                                   *reinterpret_cast<const __nv_bfloat162 *>(&bb[e]));
+        o[e] = *reinterpret_cast<uint32_t *>(&r);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // Decay mask of S (from TMEM) into P (bf16 pairs, written back to TMEM as the
@@ -288,7 +322,7 @@ struct Bars {
 // segment, from the scanned state.
 constexpr int kWhole = 0, kSummary = 1, kSegment = 2;
 
-template <int N, int R, int MODE>
+template <int N, int R, int MODE, bool BCN>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmT,
@@ -310,6 +344,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     // per-warp totals of the dt*A scan ([0, 4)); [4] = cA of token 0; [8, 12):
     // per-warp totals of the dt scan (angle rates fixed per head)
     float *wtot = phis + NPART * K2;
+    uint32_t *sbias = reinterpret_cast<uint32_t *>(wtot + 16);  // BC-norm biases [B, C][R][K2] (bf16 pairs)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     Bars bb{bars, bars + 2, bars + 4, bars + 7, bars + 10, bars + 11, bars + 12, bars + 13, bars + 14, bars + 15,
             bars + 16};
@@ -523,6 +558,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         // theta of this thread's 4 pairs for its TPT tokens, read straight from
         // global memory into registers one chunk ahead of use
         uint2 thr[TPT];
+        // BC-norm: this thread's 4 weight pairs of B and C; the head's biases in
+        // shared memory (visible after the first barrier of the chunk loop)
+        uint32_t wB2[4] = {0u, 0u, 0u, 0u}, wC2[4] = {0u, 0u, 0u, 0u};
+        if (BCN) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int n = 8 * g + 2 * e;
+                wB2[e] = pack_bf16(a.wB[n], a.wB[n + 1]);
+                wC2[e] = pack_bf16(a.wC[n], a.wC[n + 1]);
+            }
+            for (int i = tid; i < 2 * R * K2; i += kPro) {
+                const int which = i / (R * K2), rk = i % (R * K2);
+                const float *src = (which ? a.bC : a.bB) + (h * R + rk / K2) * N + 2 * (rk % K2);
+                sbias[i] = pack_bf16(src[0], src[1]);
+            }
+        }
         // angle rates fixed per head: the thread's 4 pairs, for the whole sequence
         float thh[4] = {0.f, 0.f, 0.f, 0.f};
         if (a.th_head) {
@@ -651,6 +702,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                             vb[jj][r] = *reinterpret_cast<const uint4 *>(bst + off);
                             if (!SUM) vc[jj][r] = *reinterpret_cast<const uint4 *>(cst + off);
                         }
+                    }
+                    if (BCN) {
+#pragma unroll
+                        for (int jj = 0; jj < TB; ++jj)
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                vb[jj][r] = bc_norm_row<G4>(vb[jj][r], wB2,
+                                                            *reinterpret_cast<const uint4 *>(sbias + r * K2 + 4 * g),
+                                                            1.f / N, a.eps);
+                                if (!SUM)
+                                    vc[jj][r] = bc_norm_row<G4>(
+                                        vc[jj][r], wC2, *reinterpret_cast<const uint4 *>(sbias + (R + r) * K2 + 4 * g),
+                                        1.f / N, a.eps);
+                            }
                     }
 #pragma unroll
                     for (int jj = 0; jj < TB; ++jj) {
@@ -909,8 +974,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 for (int p = 0; p < 8; ++p)
                     dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
             }
-            if (a.bpT)
+            if (a.bpT && BCN) {  // the last token's normalised B, one state warp per rank row
+                const int wl = lt >> 5;
+                if (wl < R) {
+                    const int64_t src = tok(T - 1) * R * N + wl * N;
+                    float ss = 0.f;
+                    for (int n = lane; n < N; n += 32) ss = fmaf(bf(a.B, src + n), bf(a.B, src + n), ss);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    const float sc = rsqrtf(ss / N + a.eps);
+                    for (int n = lane; n < N; n += 32)
+                        a.bpT[(bh * R + wl) * N + n] = fmaf(bf(a.B, src + n) * sc, a.wB[n], a.bB[(h * R + wl) * N + n]);
+                }
+            } else if (a.bpT) {
                 for (int i = lt; i < R * N; i += kSt) a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
+            }
             if (a.xpT)
                 for (int i = lt; i < R * kP; i += kSt) a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
         }
@@ -1034,18 +1112,18 @@ bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, int R, int MODE>
+template <int N, int R, int MODE, bool BCN>
 cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc, const CUtensorMap &mt,
                         const TcArgs &a, int64_t ctas, cudaStream_t stream) {
     using C = Cfg<N, R>;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, BCN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<N, R, MODE><<<(unsigned)ctas, kThreads, C::SMEM_BYTES, stream>>>(mx, mb, mc, mt, a);
+    prefill_tc_kernel<N, R, MODE, BCN><<<(unsigned)ctas, kThreads, C::SMEM_BYTES, stream>>>(mx, mb, mc, mt, a);
     return cudaGetLastError();
 }
 
-template <int N, int R>
+template <int N, int R, bool BCN>
 cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     using C = Cfg<N, R>;
     CUtensorMap mx, mb, mc, mt;
@@ -1072,6 +1150,11 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     a.A = p.A;
     a.A_tok = p.a_tok ? p.A : nullptr;
     a.th_head = p.th_head;
+    a.wB = p.wB;
+    a.wC = p.wC;
+    a.bB = p.bB;
+    a.bC = p.bC;
+    a.eps = p.eps;
     a.D = p.D;
     a.h0 = p.h0;
     a.bp0 = p.bp0;
@@ -1081,13 +1164,13 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
         a.hT = p.hT;
         a.bpT = p.bpT;
         a.xpT = p.xpT;
-        return launch_pass<N, R, kWhole>(mx, mb, mc, mt, a, BH, p.stream);
+        return launch_pass<N, R, kWhole, BCN>(mx, mb, mc, mt, a, BH, p.stream);
     }
     // split sequences: summary pass over segments 0 .. nseg-2, segment scan,
     // then the main pass over all segments from the scanned states
     a.ws_h = static_cast<float *>(p.ws);
     a.ws_m = a.ws_h + (size_t)plan.nseg * BH * N * kP;
-    cudaError_t e = launch_pass<N, R, kSummary>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
+    cudaError_t e = launch_pass<N, R, kSummary, BCN>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
     if (e != cudaSuccess) return e;
     ScanArgs sa{};
     sa.BH = BH;
@@ -1108,7 +1191,7 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     a.hT = p.hT;
     a.bpT = p.bpT;
     a.xpT = p.xpT;
-    return launch_pass<N, R, kSegment>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream);
+    return launch_pass<N, R, kSegment, BCN>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream);
 }
 
 bool device_is_sm100() {
@@ -1180,14 +1263,24 @@ cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
         *why = "tensor-core prefill: workspace too small for the split sequence";
         return cudaErrorNotSupported;
     }
-    if (p.N == 128) {
-        if (p.R == 1) return launch_nr<128, 1>(p, plan, why);
-        if (p.R == 2) return launch_nr<128, 2>(p, plan, why);
-        return launch_nr<128, 4>(p, plan, why);
+    if (p.wB) {
+        if (p.N == 128) {
+            if (p.R == 1) return launch_nr<128, 1, true>(p, plan, why);
+            if (p.R == 2) return launch_nr<128, 2, true>(p, plan, why);
+            return launch_nr<128, 4, true>(p, plan, why);
+        }
+        if (p.R == 1) return launch_nr<64, 1, true>(p, plan, why);
+        if (p.R == 2) return launch_nr<64, 2, true>(p, plan, why);
+        return launch_nr<64, 4, true>(p, plan, why);
     }
-    if (p.R == 1) return launch_nr<64, 1>(p, plan, why);
-    if (p.R == 2) return launch_nr<64, 2>(p, plan, why);
-    return launch_nr<64, 4>(p, plan, why);
+    if (p.N == 128) {
+        if (p.R == 1) return launch_nr<128, 1, false>(p, plan, why);
+        if (p.R == 2) return launch_nr<128, 2, false>(p, plan, why);
+        return launch_nr<128, 4, false>(p, plan, why);
+    }
+    if (p.R == 1) return launch_nr<64, 1, false>(p, plan, why);
+    if (p.R == 2) return launch_nr<64, 2, false>(p, plan, why);
+    return launch_nr<64, 4, false>(p, plan, why);
 }
 
 // Failure-path self-test: one thread waits, with a bounded wait, on an
