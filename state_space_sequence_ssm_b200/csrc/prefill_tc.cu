@@ -103,8 +103,9 @@ struct Cfg {
     // kNX buffers of {cAl2, gam, ghat, colf}[Q] + {cos, sin}[K2] (read by the
     // state warpgroup a chunk later) + {wst, dts}[Q] + phis[NPART][K2] + wtot[16]
     static constexpr uint32_t SB = 4 * Q + 2 * K2;
-    // + the BC-norm biases of this head as bf16 pairs [2][R][K2]
-    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16 + 2 * R * K2;
+    // + the BC-norm biases of this head as bf16 pairs [2][R][K2] and the row
+    // scales of the chunk's B and C tiles [2][128]
+    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16 + 2 * R * K2 + 2 * kRows;
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
     static constexpr uint32_t NBARS = 19;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
@@ -199,23 +200,32 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
     return *reinterpret_cast<uint32_t *>(&o);
 }
 
-// BC-norm of one (token, rank) row held by G4 consecutive lanes, 4 pairs each:
-// the row's sum of squares (fp32) is reduced over those lanes, then every entry
-// becomes b * scale * w + bias in packed bf16x2 arithmetic (w: this thread's
-// four weight pairs; bias: its four bias pairs of this head and rank).
-template <int G4>
-__device__ __forceinline__ uint4 bc_norm_row(uint4 v, const uint32_t (&w2)[4], uint4 b2, float inv_n, float eps) {
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+// BC-norm row scale 1 / sqrt(mean_n v^2 + eps) of row `row` of a 128B-swizzled
+// K-major tile of KB 64-column blocks (one thread per row).
+template <int KB>
+__device__ __forceinline__ float bc_row_scale(const uint8_t *tile, uint32_t row, float inv_n, float eps) {
     float ss = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 f = unpack_bf16(u[e]);
-        ss = fmaf(f.x, f.x, ss);
-        ss = fmaf(f.y, f.y, ss);
-    }
+    for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-    for (int off = 1; off < G4; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float sc = rsqrtf(fmaf(ss, inv_n, eps));
+        for (uint32_t j = 0; j < 8; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(tile + kb * 16384 + sw128(row, j));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = unpack_bf16(u[e]);
+                ss = fmaf(f.x, f.x, ss);
+                ss = fmaf(f.y, f.y, ss);
+            }
+        }
+    return rsqrtf(fmaf(ss, inv_n, eps));
+}
+
+// The BC-norm affine map of this thread's 4 pairs of one row: b * sc * w + bias
+// in packed bf16x2 arithmetic (w: the thread's four weight pairs; bias: its
+// four bias pairs of this head and rank; sc: the row's scale).
+__device__ __forceinline__ uint4 bc_norm_row(uint4 v, const uint32_t (&w2)[4], uint4 b2, float sc) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
     const uint32_t s2 = pack_bf16(sc, sc);
     const uint32_t bb[4] = {b2.x, b2.y, b2.z, b2.w};
     uint32_t o[4];
@@ -345,6 +355,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     // per-warp totals of the dt scan (angle rates fixed per head)
     float *wtot = phis + NPART * K2;
     uint32_t *sbias = reinterpret_cast<uint32_t *>(wtot + 16);  // BC-norm biases [B, C][R][K2] (bf16 pairs)
+    float *rsc = reinterpret_cast<float *>(sbias + 2 * R * C::K2);  // BC-norm row scales [B, C][128]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     Bars bb{bars, bars + 2, bars + 4, bars + 7, bars + 10, bars + 11, bars + 12, bars + 13, bars + 14, bars + 15,
             bars + 16};
@@ -678,6 +689,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 // the B/C tiles of this chunk
                 if (bar_any<kBarPro, kPro>(!mbar_wait(&bb.full_bc[s], (lc >> 1) & 1, abort_flag, err, kErrWaitTma)))
                     break;
+                if (BCN) {  // one row scale per thread: B rows (tid < 128), then C rows
+                    if (!SUM || tid < kRows)
+                        rsc[tid] = bc_row_scale<KB>(tid < kRows ? bst : cst, (uint32_t)(tid % kRows), 1.f / N, a.eps);
+                    named_bar(kBarPro, kPro);
+                }
                 float phi[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int q = 0; q < (a.th_head ? 0 : part); ++q) {
                     const float4 v = *reinterpret_cast<const float4 *>(phis + q * K2 + 4 * g);
@@ -708,13 +724,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         for (int jj = 0; jj < TB; ++jj)
 #pragma unroll
                             for (int r = 0; r < R; ++r) {
-                                vb[jj][r] = bc_norm_row<G4>(vb[jj][r], wB2,
-                                                            *reinterpret_cast<const uint4 *>(sbias + r * K2 + 4 * g),
-                                                            1.f / N, a.eps);
+                                const int row = (part * TPT + j0 + jj) * R + r;
+                                vb[jj][r] = bc_norm_row(vb[jj][r], wB2,
+                                                        *reinterpret_cast<const uint4 *>(sbias + r * K2 + 4 * g),
+                                                        rsc[row]);
                                 if (!SUM)
-                                    vc[jj][r] = bc_norm_row<G4>(
+                                    vc[jj][r] = bc_norm_row(
                                         vc[jj][r], wC2, *reinterpret_cast<const uint4 *>(sbias + (R + r) * K2 + 4 * g),
-                                        1.f / N, a.eps);
+                                        rsc[kRows + row]);
                             }
                     }
 #pragma unroll
