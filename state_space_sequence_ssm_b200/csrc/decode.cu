@@ -78,12 +78,18 @@ struct StepArgs {
     int P, N, R;
     const IO *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
+    float *h, *bp, *xp;
+    IO *y;
+};
+
+// The optional features, a kernel argument of their own: growing StepArgs
+// changed the plain kernel's code generation (and cost it 7 % of its
+// bandwidth), a second argument does not.
+struct StepFeat {
     int a_tok;    // A is [Bt, H] (per token-head) instead of [H]
     int th_head;  // theta is [H, N/2] (fixed per head)
     const float *wB, *wC, *bB, *bC;  // BC-norm prologue (wB == nullptr: off)
     float eps;
-    float *h, *bp, *xp;
-    IO *y;
 };
 
 // Register-tiled kernel for the common sizes.  Each thread owns PT pairs x 4
@@ -104,9 +110,12 @@ struct StepCfg {
     static_assert(32 % CG == 0 || CG % 32 == 0, "column groups must tile a warp");
 };
 
-template <int N, int P, int R, typename IO>
+// GEN = false: the plain method (A per head, theta per token, no BC-norm),
+// compiled without the optional features' branches; GEN = true reads them
+// from the arguments.
+template <int N, int P, int R, typename IO, bool GEN>
 __global__ void __launch_bounds__(StepCfg<N, P, R, IO>::THREADS)
-step_kernel(const StepArgs<IO> a) {
+step_kernel(const StepArgs<IO> a, const StepFeat f) {
     using Cfg = StepCfg<N, P, R, IO>;
     constexpr int K2 = Cfg::K2, CG = Cfg::CG, PT = Cfg::PT, KK = Cfg::KK, NT = Cfg::THREADS;
     __shared__ __align__(16) float sBp[R][N], sB[R][N], sC[R][N];
@@ -130,7 +139,7 @@ step_kernel(const StepArgs<IO> a) {
         hv[j] = __ldcs(hst + ((2 * k + 1) * P + p0) / 4);
     }
     const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
-    const float alpha = __expf(dtv * a.A[a.a_tok ? bh : h]);
+    const float alpha = __expf(dtv * a.A[(GEN && f.a_tok) ? bh : h]);
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
     // ---- stage the slice's small vectors
     for (int i = tid; i < R * N; i += NT) {
@@ -144,20 +153,20 @@ step_kernel(const StepArgs<IO> a) {
     }
     for (int k = tid; k < K2; k += NT) {
         float sn, cs;
-        sincosf(dtv * ldv(a.theta, (a.th_head ? (int64_t)h : bh) * K2 + k), &sn, &cs);
+        sincosf(dtv * ldv(a.theta, ((GEN && f.th_head) ? (int64_t)h : bh) * K2 + k), &sn, &cs);
         sAc[k] = alpha * cs;
         sAs[k] = alpha * sn;
     }
     __syncthreads();
-    if (a.wB) {  // BC-norm prologue on the staged rows: one warp per row of B, then of C
+    if (GEN && f.wB) {  // BC-norm prologue on the staged rows: one warp per row of B, then of C
         const int warp = tid / 32, lane = tid % 32;
         for (int row = warp; row < 2 * R; row += Cfg::WARPS) {
             const bool isB = row < R;
             const int r = isB ? row : row - R;
             float *v = isB ? sB[r] : sC[r];
-            const float *w = isB ? a.wB : a.wC;
-            const float *bias = (isB ? a.bB : a.bC) + (h * R + r) * N;
-            const float sc = bcn_row_scale_warp([&](int n) { return v[n]; }, N, a.eps);
+            const float *w = isB ? f.wB : f.wC;
+            const float *bias = (isB ? f.bB : f.bC) + (h * R + r) * N;
+            const float sc = bcn_row_scale_warp([&](int n) { return v[n]; }, N, f.eps);
             for (int n = lane; n < N; n += 32) v[n] = fmaf(v[n] * sc, w[n], bias[n]);
         }
         __syncthreads();
@@ -239,31 +248,31 @@ step_kernel(const StepArgs<IO> a) {
 // Generic kernel for any even N and any P: one thread per (pair, column),
 // shared-memory atomics for the readout.  Same arithmetic, no tiling.
 template <typename IO>
-__global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a) {
+__global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a, const StepFeat f) {
     extern __shared__ float ysum[];  // [R][P], then (BC-norm) normalised B and C [R][N] each
     const int N = a.N, P = a.P, R = a.R, K2 = N / 2;
     const int64_t bh = blockIdx.x;
     const int h = (int)(bh % a.H);
     float *nB = ysum + R * P, *nC = nB + R * N;
     for (int i = threadIdx.x; i < R * P; i += blockDim.x) ysum[i] = 0.f;
-    if (a.wB) {  // BC-norm prologue: one warp per row of B, then of C
+    if (f.wB) {  // BC-norm prologue: one warp per row of B, then of C
         const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
         for (int row = warp; row < 2 * R; row += blockDim.x / 32) {
             const bool isB = row < R;
             const int r = isB ? row : row - R;
             const IO *src = (isB ? a.B : a.C) + (bh * R + r) * N;
-            const float *w = isB ? a.wB : a.wC;
-            const float *bias = (isB ? a.bB : a.bC) + (h * R + r) * N;
+            const float *w = isB ? f.wB : f.wC;
+            const float *bias = (isB ? f.bB : f.bC) + (h * R + r) * N;
             float *dst = (isB ? nB : nC) + r * N;
-            const float sc = bcn_row_scale_warp([&](int n) { return ldv(src, n); }, N, a.eps);
+            const float sc = bcn_row_scale_warp([&](int n) { return ldv(src, n); }, N, f.eps);
             for (int n = lane; n < N; n += 32) dst[n] = fmaf(ldv(src, n) * sc, w[n], bias[n]);
         }
     }
     __syncthreads();
-    auto Bv = [&](int i) { return a.wB ? nB[i] : ldv(a.B, bh * R * N + i); };  // i = r * N + n
-    auto Cv = [&](int i) { return a.wB ? nC[i] : ldv(a.C, bh * R * N + i); };
+    auto Bv = [&](int i) { return f.wB ? nB[i] : ldv(a.B, bh * R * N + i); };  // i = r * N + n
+    auto Cv = [&](int i) { return f.wB ? nC[i] : ldv(a.C, bh * R * N + i); };
     const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
-    const float alpha = expf(dtv * a.A[a.a_tok ? bh : h]);
+    const float alpha = expf(dtv * a.A[f.a_tok ? bh : h]);
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
     float *hs = a.h + bh * N * P;
     for (int idx = threadIdx.x; idx < K2 * P; idx += blockDim.x) {
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a)
             v += betap * a.bp[(bh * R + r) * N + 2 * k + 1] * xpp;
         }
         float sn, cs;
-        sincosf(dtv * ldv(a.theta, (a.th_head ? (int64_t)h : bh) * K2 + k), &sn, &cs);
+        sincosf(dtv * ldv(a.theta, (f.th_head ? (int64_t)h : bh) * K2 + k), &sn, &cs);
         float nu = alpha * (u * cs + v * sn), nv = alpha * (-u * sn + v * cs);
         for (int r = 0; r < R; ++r) {
             const float xx = ldv(a.x, (bh * R + r) * P + p);
@@ -354,9 +363,9 @@ __device__ __forceinline__ float4 sv4<__nv_bfloat16>(const __nv_bfloat16 *p, int
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
-template <int N, int P, int R, typename IO>
+template <int N, int P, int R, typename IO, bool GEN>
 __global__ void __launch_bounds__(StreamCfg<N, P, R, IO>::THREADS, StreamCfg<N, P, R, IO>::CTAS_PER_SM)
-step_stream_kernel(const StepArgs<IO> a) {
+step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
     using Cfg = StreamCfg<N, P, R, IO>;
     constexpr int K2 = Cfg::K2, CG = Cfg::CG, PT = Cfg::PT, KK = Cfg::KK, NT = Cfg::THREADS;
     extern __shared__ __align__(128) uint8_t sm[];
@@ -379,7 +388,7 @@ step_stream_kernel(const StepArgs<IO> a) {
         tc::bulk_g2s(s + Cfg::O_B, a.B + bh * R * N, Cfg::B_B, &full[st]);
         tc::bulk_g2s(s + Cfg::O_C, a.C + bh * R * N, Cfg::B_B, &full[st]);
         tc::bulk_g2s(s + Cfg::O_X, a.x + bh * R * P, Cfg::B_X, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_TH, a.theta + (a.th_head ? bh % a.H : bh) * K2, Cfg::B_TH, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_TH, a.theta + ((GEN && f.th_head) ? bh % a.H : bh) * K2, Cfg::B_TH, &full[st]);
     };
     if (tid == 0) {
         tc::mbar_init(&full[0], 1);
@@ -409,7 +418,7 @@ step_stream_kernel(const StepArgs<IO> a) {
         const bool ok = tc::mbar_wait(&full[st], (it >> 1) & 1, &abort_flag, &g_decode_error, tc::kErrWaitTma);
         if (__syncthreads_or(!ok)) break;
         if (tid < K2) {
-            const float alpha = __expf(dtv * a.A[a.a_tok ? bh : h]);
+            const float alpha = __expf(dtv * a.A[(GEN && f.a_tok) ? bh : h]);
             float sn, cs;
             sincosf(dtv * sv(sTh, tid), &sn, &cs);
             sAc[tid] = alpha * cs;
@@ -499,41 +508,43 @@ step_stream_kernel(const StepArgs<IO> a) {
     }
 }
 
-template <int N, int P, int R, typename IO>
-cudaError_t launch_stream(const StepArgs<IO> &a, cudaStream_t s) {
+template <int N, int P, int R, typename IO, bool GEN>
+cudaError_t launch_stream(const StepArgs<IO> &a, const StepFeat &f, cudaStream_t s) {
     using Cfg = StreamCfg<N, P, R, IO>;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(step_stream_kernel<N, P, R, IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(step_stream_kernel<N, P, R, IO, GEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Cfg::SMEM);
     if (e != cudaSuccess) return e;
     int64_t grid = (int64_t)sms * Cfg::CTAS_PER_SM;
     if (grid > a.BH) grid = a.BH;
-    step_stream_kernel<N, P, R, IO><<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, s>>>(a);
+    step_stream_kernel<N, P, R, IO, GEN><<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, s>>>(a, f);
     return cudaGetLastError();
 }
 
-template <int N, int P, int R, typename IO>
-cudaError_t launch_tiled(const StepArgs<IO> &a, cudaStream_t s) {
-    step_kernel<N, P, R, IO><<<(unsigned)a.BH, StepCfg<N, P, R, IO>::THREADS, 0, s>>>(a);
+template <int N, int P, int R, typename IO, bool GEN>
+cudaError_t launch_tiled(const StepArgs<IO> &a, const StepFeat &f, cudaStream_t s) {
+    step_kernel<N, P, R, IO, GEN><<<(unsigned)a.BH, StepCfg<N, P, R, IO>::THREADS, 0, s>>>(a, f);
     return cudaGetLastError();
 }
 
-template <typename IO, int R>
-cudaError_t dispatch_np(const StepArgs<IO> &a, cudaStream_t s, bool *done) {
+template <typename IO, int R, bool GEN>
+cudaError_t dispatch_np(const StepArgs<IO> &a, const StepFeat &f, cudaStream_t s, bool *done) {
     *done = true;
     // rank 1: one CTA per slice (measured faster); rank >= 2: the persistent
     // streaming kernel (its heavier per-element work overlaps the next slice's load)
     // (BC-norm: the tiled kernel, which normalises its staged rows in place)
-    const bool tiled = R == 1 || a.wB;
-    if (a.N == 128 && a.P == 64) return tiled ? launch_tiled<128, 64, R, IO>(a, s) : launch_stream<128, 64, R, IO>(a, s);
-    if (a.N == 64 && a.P == 64) return tiled ? launch_tiled<64, 64, R, IO>(a, s) : launch_stream<64, 64, R, IO>(a, s);
-    if (a.N == 128 && a.P == 128) return launch_tiled<128, 128, R, IO>(a, s);
-    if (a.N == 64 && a.P == 128) return launch_tiled<64, 128, R, IO>(a, s);
-    if (a.N == 256 && a.P == 64) return launch_tiled<256, 64, R, IO>(a, s);
+    const bool tiled = R == 1 || f.wB;
+    if (a.N == 128 && a.P == 64)
+        return tiled ? launch_tiled<128, 64, R, IO, GEN>(a, f, s) : launch_stream<128, 64, R, IO, GEN>(a, f, s);
+    if (a.N == 64 && a.P == 64)
+        return tiled ? launch_tiled<64, 64, R, IO, GEN>(a, f, s) : launch_stream<64, 64, R, IO, GEN>(a, f, s);
+    if (a.N == 128 && a.P == 128) return launch_tiled<128, 128, R, IO, GEN>(a, f, s);
+    if (a.N == 64 && a.P == 128) return launch_tiled<64, 128, R, IO, GEN>(a, f, s);
+    if (a.N == 256 && a.P == 64) return launch_tiled<256, 64, R, IO, GEN>(a, f, s);
     *done = false;
     return cudaSuccess;
 }
@@ -546,20 +557,22 @@ cudaError_t launch_typed(const Problem &p) {
     a.x = (const IO *)p.x; a.B = (const IO *)p.B; a.C = (const IO *)p.C;
     a.dt = (const IO *)p.dt; a.lam = (const IO *)p.lam; a.theta = (const IO *)p.theta;
     a.A = p.A; a.D = p.D;
-    a.a_tok = p.a_tok;
-    a.th_head = p.th_head;
-    a.wB = p.wB; a.wC = p.wC; a.bB = p.bB; a.bC = p.bC; a.eps = p.eps;
+    StepFeat f{};
+    f.a_tok = p.a_tok;
+    f.th_head = p.th_head;
+    f.wB = p.wB; f.wC = p.wC; f.bB = p.bB; f.bC = p.bC; f.eps = p.eps;
     a.h = p.hT; a.bp = p.bpT; a.xp = p.xpT;
     a.y = (IO *)p.y;
     if (a.BH == 0) return cudaSuccess;
     bool done = false;
     cudaError_t e = cudaSuccess;
-    if (a.R == 1) e = dispatch_np<IO, 1>(a, p.stream, &done);
-    else if (a.R == 2) e = dispatch_np<IO, 2>(a, p.stream, &done);
-    else if (a.R == 4) e = dispatch_np<IO, 4>(a, p.stream, &done);
+    const bool gen = f.a_tok || f.th_head || f.wB;  // any optional feature on
+    if (a.R == 1) e = gen ? dispatch_np<IO, 1, true>(a, f, p.stream, &done) : dispatch_np<IO, 1, false>(a, f, p.stream, &done);
+    else if (a.R == 2) e = gen ? dispatch_np<IO, 2, true>(a, f, p.stream, &done) : dispatch_np<IO, 2, false>(a, f, p.stream, &done);
+    else if (a.R == 4) e = gen ? dispatch_np<IO, 4, true>(a, f, p.stream, &done) : dispatch_np<IO, 4, false>(a, f, p.stream, &done);
     if (done) return e;
-    const size_t smem = sizeof(float) * ((size_t)a.R * a.P + (a.wB ? 2 * (size_t)a.R * a.N : 0));
-    step_generic_kernel<IO><<<(unsigned)a.BH, 256, smem, p.stream>>>(a);
+    const size_t smem = sizeof(float) * ((size_t)a.R * a.P + (f.wB ? 2 * (size_t)a.R * a.N : 0));
+    step_generic_kernel<IO><<<(unsigned)a.BH, 256, smem, p.stream>>>(a, f);
     return cudaGetLastError();
 }
 

@@ -332,7 +332,10 @@ struct Bars {
 // segment, from the scanned state.
 constexpr int kWhole = 0, kSummary = 1, kSegment = 2;
 
-template <int N, int R, int MODE, bool BCN>
+// GEN = false: the plain method (A per head, theta per token), compiled
+// without the optional features' branches; GEN = true reads A_tok and th_head
+// from the arguments.  BCN: the BC-norm prologue (only with GEN).
+template <int N, int R, int MODE, bool GEN, bool BCN>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmT,
@@ -340,6 +343,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     using C = Cfg<N, R>;
     constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, G4 = C::G4, NPART = C::NPART, TPT = C::TPT, TB = C::TB;
     constexpr bool SUM = MODE == kSummary, SEGD = MODE != kWhole;
+    const float *const A_tok = GEN ? a.A_tok : nullptr;  // A per token-head, or none
+    const bool th_head = GEN && a.th_head;               // theta fixed per head
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *scal = reinterpret_cast<float *>(smem + C::OFF_SCAL);
@@ -427,7 +432,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     tma_prefetch_5d(&tmB, kb * 64, 0, (int)h, t0, (int)b);
                     if (!SUM) tma_prefetch_5d(&tmC, kb * 64, 0, (int)h, t0, (int)b);
                 }
-                if (!a.th_head) tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // read straight into registers
+                if (!th_head) tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // read straight into registers
             };
             int issued = 0;
             for (int i = 0; i < kPrefetchAhead && i < nloc; ++i) prefetch_chunk(cb + i);
@@ -544,7 +549,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
     } else if (warp < 8) {
         // ============================================================ prologue warps (0-7)
-        const float Ah2 = a.A_tok ? 0.f : a.A[h] * kLog2e;
+        const float Ah2 = A_tok ? 0.f : a.A[h] * kLog2e;
         uint8_t *xw = smem + C::OFF_XW;
         const unsigned short *dtr = reinterpret_cast<const unsigned short *>(a.dt);
         const unsigned short *lmr = reinterpret_cast<const unsigned short *>(a.lam);
@@ -559,7 +564,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (tid < Q && t < T) {
                 pd = __ldg(dtr + tok(t));
                 pl = __ldg(lmr + tok(t));
-                if (a.A_tok) pa = __ldg(a.A_tok + tok(t));
+                if (A_tok) pa = __ldg(A_tok + tok(t));
                 if (t + 1 < T) {
                     pd1 = __ldg(dtr + tok(t + 1));
                     pl1 = __ldg(lmr + tok(t + 1));
@@ -587,12 +592,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         // angle rates fixed per head: the thread's 4 pairs, for the whole sequence
         float thh[4] = {0.f, 0.f, 0.f, 0.f};
-        if (a.th_head) {
+        if (th_head) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) thh[e] = bf(a.theta, h * K2 + 4 * g + e);
         }
         auto prefetch_theta = [&](int64_t t0s) {
-            if (a.th_head) return;
+            if (th_head) return;
 #pragma unroll
             for (int j = 0; j < TPT; ++j) {
                 const int64_t t = t0s + part * TPT + j;
@@ -623,7 +628,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             {
                 const float d = bf16_bits(pd), l = bf16_bits(pl);
                 const float nx = (1.f - bf16_bits(pl1)) * bf16_bits(pd1);  // 0 past the sequence end
-                const float a2 = a.A_tok ? pa * kLog2e : Ah2;                // A_t in log2 units
+                const float a2 = A_tok ? pa * kLog2e : Ah2;                // A_t in log2 units
                 if (lc + 1 < nloc) prefetch_scalars((int64_t)(first_chunk() + lc + 1) * Q);
                 if (tid < Q) {
                     dts[tid] = d;
@@ -637,7 +642,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         if (lane >= off) acc += v;
                     }
                     if (lane == 31) wtot[warp] = acc;
-                    if (a.th_head) {  // chunk-local cumulative dt: the angle is theta_k times it
+                    if (th_head) {  // chunk-local cumulative dt: the angle is theta_k times it
                         acd = d;
 #pragma unroll
                         for (int off = 1; off < 32; off <<= 1) {
@@ -662,7 +667,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 wst[tid] = ex2(tot - ca) * ghat[tid];
                 // column factor of the decay mask, relative to the chunk's first token
                 colf[tid] = ex2(wtot[4] - ca) * ghat[tid];
-                if (a.th_head) {  // dts becomes the cumulative dt (read after the next barrier)
+                if (th_head) {  // dts becomes the cumulative dt (read after the next barrier)
                     float offd = 0.f;
 #pragma unroll
                     for (int w = 0; w < Q / 32; ++w)
@@ -677,7 +682,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 float loc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < TPT; ++j) {
-                    if (a.th_head) break;
+                    if (th_head) break;
                     const float di = dts[part * TPT + j];
                     const float2 t01 = unpack_bf16(thr[j].x), t23 = unpack_bf16(thr[j].y);
                     loc[0] = fmaf(di, t01.x, loc[0]);
@@ -695,7 +700,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     named_bar(kBarPro, kPro);
                 }
                 float phi[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int q = 0; q < (a.th_head ? 0 : part); ++q) {
+                for (int q = 0; q < (th_head ? 0 : part); ++q) {
                     const float4 v = *reinterpret_cast<const float4 *>(phis + q * K2 + 4 * g);
                     phi[0] += v.x;
                     phi[1] += v.y;
@@ -738,7 +743,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     for (int jj = 0; jj < TB; ++jj) {
                         const int i = part * TPT + j0 + jj;
                         const float di = dts[i];
-                        if (a.th_head) {  // di is the cumulative dt of token i
+                        if (th_head) {  // di is the cumulative dt of token i
 #pragma unroll
                             for (int e = 0; e < 4; ++e) phi[e] = di * thh[e];
                         } else {
@@ -1129,18 +1134,18 @@ bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, int R, int MODE, bool BCN>
+template <int N, int R, int MODE, bool GEN, bool BCN>
 cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc, const CUtensorMap &mt,
                         const TcArgs &a, int64_t ctas, cudaStream_t stream) {
     using C = Cfg<N, R>;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, BCN>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, GEN, BCN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<N, R, MODE, BCN><<<(unsigned)ctas, kThreads, C::SMEM_BYTES, stream>>>(mx, mb, mc, mt, a);
+    prefill_tc_kernel<N, R, MODE, GEN, BCN><<<(unsigned)ctas, kThreads, C::SMEM_BYTES, stream>>>(mx, mb, mc, mt, a);
     return cudaGetLastError();
 }
 
-template <int N, int R, bool BCN>
+template <int N, int R, bool GEN, bool BCN>
 cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     using C = Cfg<N, R>;
     CUtensorMap mx, mb, mc, mt;
@@ -1181,13 +1186,13 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
         a.hT = p.hT;
         a.bpT = p.bpT;
         a.xpT = p.xpT;
-        return launch_pass<N, R, kWhole, BCN>(mx, mb, mc, mt, a, BH, p.stream);
+        return launch_pass<N, R, kWhole, GEN, BCN>(mx, mb, mc, mt, a, BH, p.stream);
     }
     // split sequences: summary pass over segments 0 .. nseg-2, segment scan,
     // then the main pass over all segments from the scanned states
     a.ws_h = static_cast<float *>(p.ws);
     a.ws_m = a.ws_h + (size_t)plan.nseg * BH * N * kP;
-    cudaError_t e = launch_pass<N, R, kSummary, BCN>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
+    cudaError_t e = launch_pass<N, R, kSummary, GEN, BCN>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
     if (e != cudaSuccess) return e;
     ScanArgs sa{};
     sa.BH = BH;
@@ -1208,7 +1213,7 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     a.hT = p.hT;
     a.bpT = p.bpT;
     a.xpT = p.xpT;
-    return launch_pass<N, R, kSegment, BCN>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream);
+    return launch_pass<N, R, kSegment, GEN, BCN>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream);
 }
 
 bool device_is_sm100() {
@@ -1280,24 +1285,36 @@ cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
         *why = "tensor-core prefill: workspace too small for the split sequence";
         return cudaErrorNotSupported;
     }
+    // plain instantiations unless an optional feature is on
+    const bool gen = p.a_tok || p.th_head || p.wB;
     if (p.wB) {
         if (p.N == 128) {
-            if (p.R == 1) return launch_nr<128, 1, true>(p, plan, why);
-            if (p.R == 2) return launch_nr<128, 2, true>(p, plan, why);
-            return launch_nr<128, 4, true>(p, plan, why);
+            if (p.R == 1) return launch_nr<128, 1, true, true>(p, plan, why);
+            if (p.R == 2) return launch_nr<128, 2, true, true>(p, plan, why);
+            return launch_nr<128, 4, true, true>(p, plan, why);
         }
-        if (p.R == 1) return launch_nr<64, 1, true>(p, plan, why);
-        if (p.R == 2) return launch_nr<64, 2, true>(p, plan, why);
-        return launch_nr<64, 4, true>(p, plan, why);
+        if (p.R == 1) return launch_nr<64, 1, true, true>(p, plan, why);
+        if (p.R == 2) return launch_nr<64, 2, true, true>(p, plan, why);
+        return launch_nr<64, 4, true, true>(p, plan, why);
+    }
+    if (gen) {
+        if (p.N == 128) {
+            if (p.R == 1) return launch_nr<128, 1, true, false>(p, plan, why);
+            if (p.R == 2) return launch_nr<128, 2, true, false>(p, plan, why);
+            return launch_nr<128, 4, true, false>(p, plan, why);
+        }
+        if (p.R == 1) return launch_nr<64, 1, true, false>(p, plan, why);
+        if (p.R == 2) return launch_nr<64, 2, true, false>(p, plan, why);
+        return launch_nr<64, 4, true, false>(p, plan, why);
     }
     if (p.N == 128) {
-        if (p.R == 1) return launch_nr<128, 1, false>(p, plan, why);
-        if (p.R == 2) return launch_nr<128, 2, false>(p, plan, why);
-        return launch_nr<128, 4, false>(p, plan, why);
+        if (p.R == 1) return launch_nr<128, 1, false, false>(p, plan, why);
+        if (p.R == 2) return launch_nr<128, 2, false, false>(p, plan, why);
+        return launch_nr<128, 4, false, false>(p, plan, why);
     }
-    if (p.R == 1) return launch_nr<64, 1, false>(p, plan, why);
-    if (p.R == 2) return launch_nr<64, 2, false>(p, plan, why);
-    return launch_nr<64, 4, false>(p, plan, why);
+    if (p.R == 1) return launch_nr<64, 1, false, false>(p, plan, why);
+    if (p.R == 2) return launch_nr<64, 2, false, false>(p, plan, why);
+    return launch_nr<64, 4, false, false>(p, plan, why);
 }
 
 // Failure-path self-test: one thread waits, with a bounded wait, on an

@@ -153,3 +153,12 @@ def test_scan_plan_host_side(m3):
     assert m3.lib.m3_scan_plan(m3.ALGO_TC, ctypes.byref(d), None, None, None) == 2  # TC refuses fp32 I/O
     assert m3.lib.m3_scan_plan(9, ctypes.byref(d), None, None, None) == 1
     assert m3.lib.m3_scan_plan(m3.ALGO_AUTO, None, None, None, None) == 1
+
+
+def test_library_has_no_unresolved_internal_symbols(m3):
+    """Every internal (namespace m3) function the library calls is defined in
+    it: a missing definition would only surface when the GPU loads it."""
+    out = subprocess.run(["nm", "-D", "--undefined-only", m3.LIB_PATH], capture_output=True, text=True).stdout
+    missing = [l.split()[-1] for l in out.splitlines() if "_ZN2m3" in l]
+    assert not missing, f"undefined library-internal symbols: {missing}"
+    ctypes.CDLL(m3.LIB_PATH, mode=os.RTLD_NOW)  # resolves every symbol now
