@@ -187,6 +187,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
         }
     }
     if (bcn && (s = check_bcnorm(d, bcn, yr)) != M3_OK) return s;
+    if (d->batch == 0) return M3_OK;  // nothing to read or write, whichever kernel was asked for
     m3::Problem p = make_problem(d, x, B, C, dt, lam, theta, A, D, y, stream);
     if (bcn) { p.wB = bcn->wB; p.wC = bcn->wC; p.bB = bcn->bB; p.bC = bcn->bC; p.eps = bcn->eps; }
     if (init) { p.h0 = init->h; p.bp0 = init->b_prev; p.xp0 = init->x_prev; }
@@ -247,6 +248,12 @@ m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_bytes, int 
             return fail(M3_ERR_INVALID_ARG, "unknown algo");
         if (forced < 0 || forced > kMaxForcedSegments || (forced && base != M3_ALGO_TC))
             return fail(M3_ERR_INVALID_ARG, "bad segment count in algo");
+        if (d->batch == 0) {  // nothing to run, whichever kernel was asked for
+            if (workspace_bytes) *workspace_bytes = 0;
+            if (segments) *segments = 1;
+            if (launches) *launches = 0;
+            return M3_OK;
+        }
         m3::Problem p{};
         p.Bt = d->batch; p.T = d->seqlen; p.H = d->nheads; p.P = d->headdim; p.N = d->dstate; p.R = d->rank;
         p.bf16 = d->io == M3_BF16;

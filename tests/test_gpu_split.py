@@ -91,3 +91,28 @@ def test_auto_plan_splits_only_the_few_long_sequences():
     assert long_plan.segments > 1 and long_plan.launches == 3
     assert plan("siso_bf16_b8_t4096_h32_p64_n128") == (0, 1, 1)
     assert plan("mimo_bf16_b8_t4096_h32_p64_n64_r4").segments == 1
+
+
+@pytest.mark.parametrize("shape,segs", [
+    (Shape(1, 1, 2, 64, 128, 1, "bf16", 151), 4),      # one token: the plan falls back to one segment
+    (Shape(1, 256, 1, 64, 128, 1, "bf16", 152), 2),    # segment boundary at the last chunk boundary
+    (Shape(1, 129, 1, 64, 128, 1, "bf16", 153), 2),    # second segment holds a single token
+    (Shape(3, 520, 1, 64, 64, 2, "bf16", 154), 7),     # several sequences, many short segments
+], ids=lambda v: f"t{v.seqlen}b{v.batch}r{v.rank}" if isinstance(v, Shape) else f"s{v}")
+def test_split_edge_cases(shape, segs):
+    dims = m3.make_dims(shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.rank,
+                        shape.torch_io)
+    plan = m3.scan_plan(dims, m3.ALGO_TC_SEGMENTS(segs))
+    nch = -(-shape.seqlen // (128 // shape.rank))
+    assert 1 <= plan.segments <= min(segs, nch)
+    assert plan.launches == (3 if plan.segments > 1 else 1)
+    check_scan(shape, m3.ALGO_TC_SEGMENTS(segs), with_init=True)
+    m3.stream_status()
+
+
+def test_split_zero_batch_is_noop():
+    s = Shape(0, 1000, 2, 64, 128, 1, "bf16", 155)
+    inp = to_dev(make_prefill(s))
+    y, fs = m3.scan_fwd(*(inp[k] for k in KEYS), None, algo=m3.ALGO_TC_SEGMENTS(3))
+    m3.stream_status()
+    assert y.numel() == 0 and fs.h.numel() == 0
