@@ -329,7 +329,10 @@ struct StreamCfg {
     static constexpr uint32_t TX = B_H + B_BP + B_XP + 2 * B_B + B_X + B_TH;
     static constexpr uint32_t O_YP = 2 * STAGE;                       // ypart [WARPS][R][P]
     static constexpr uint32_t O_AC = O_YP + WARPS * R * P * 4;        // alpha cos [K2], alpha sin [K2]
-    static constexpr uint32_t O_BAR = O_AC + 2 * K2 * 4;
+    // the slice's vectors, scaled and in fp32 once per slice: beta' b_prev,
+    // gamma B and C, each [R][N]
+    static constexpr uint32_t O_VEC = O_AC + 2 * K2 * 4;
+    static constexpr uint32_t O_BAR = O_VEC + 3 * R * N * 4;
     static constexpr uint32_t SMEM = O_BAR + 16;
     static constexpr int CTAS_PER_SM = (3 * (SMEM + 1024) <= 232448) ? 3 : 2;  // as many as shared memory allows
     static_assert(B_BP % 16 == 0 && B_XP % 16 == 0 && B_B % 16 == 0 && B_X % 16 == 0 && B_TH % 16 == 0,
@@ -372,6 +375,7 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
     float *ypart = reinterpret_cast<float *>(sm + Cfg::O_YP);
     float *sAc = reinterpret_cast<float *>(sm + Cfg::O_AC);
     float *sAs = sAc + K2;
+    float *vBp = reinterpret_cast<float *>(sm + Cfg::O_VEC), *vB = vBp + R * N, *vC = vB + R * N;
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + Cfg::O_BAR);
     __shared__ int abort_flag;
     const int tid = threadIdx.x;
@@ -424,6 +428,11 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
             sAc[tid] = alpha * cs;
             sAs[tid] = alpha * sn;
         }
+        for (int i = tid; i < R * N; i += NT) {
+            vBp[i] = betap * sBp[i];
+            vB[i] = gam * sv(sB, i);
+            vC[i] = sv(sC, i);
+        }
         __syncthreads();
         float4 xp[R], xv[R], yacc[R];
 #pragma unroll
@@ -440,8 +449,8 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
             float4 v = *reinterpret_cast<const float4 *>(sh + (2 * k + 1) * P + p0);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float2 bpk = *reinterpret_cast<const float2 *>(sBp + r * N + 2 * k);
-                const float cu = betap * bpk.x, cv = betap * bpk.y;
+                const float2 bpk = *reinterpret_cast<const float2 *>(vBp + r * N + 2 * k);
+                const float cu = bpk.x, cv = bpk.y;
                 u.x = fmaf(cu, xp[r].x, u.x); u.y = fmaf(cu, xp[r].y, u.y);
                 u.z = fmaf(cu, xp[r].z, u.z); u.w = fmaf(cu, xp[r].w, u.w);
                 v.x = fmaf(cv, xp[r].x, v.x); v.y = fmaf(cv, xp[r].y, v.y);
@@ -455,8 +464,8 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
             nu.w = ac * u.w + as * v.w; nv.w = ac * v.w - as * u.w;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float2 bk = sv2(sB, r * N + 2 * k);
-                const float cu = gam * bk.x, cv = gam * bk.y;
+                const float2 bk = *reinterpret_cast<const float2 *>(vB + r * N + 2 * k);
+                const float cu = bk.x, cv = bk.y;
                 nu.x = fmaf(cu, xv[r].x, nu.x); nu.y = fmaf(cu, xv[r].y, nu.y);
                 nu.z = fmaf(cu, xv[r].z, nu.z); nu.w = fmaf(cu, xv[r].w, nu.w);
                 nv.x = fmaf(cv, xv[r].x, nv.x); nv.y = fmaf(cv, xv[r].y, nv.y);
@@ -466,7 +475,7 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
             __stcs(hg + ((2 * k + 1) * P + p0) / 4, nv);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float2 ck = sv2(sC, r * N + 2 * k);
+                const float2 ck = *reinterpret_cast<const float2 *>(vC + r * N + 2 * k);
                 yacc[r].x += nu.x * ck.x + nv.x * ck.y;
                 yacc[r].y += nu.y * ck.x + nv.y * ck.y;
                 yacc[r].z += nu.z * ck.x + nv.z * ck.y;
