@@ -196,6 +196,39 @@ def step_bytes(s):
     return bh * (2 * state + inp + io * s.rank * s.headdim) + 8 * s.nheads
 
 
+# ---------------------------------------------------------------- ranks (replicas, no data-path collective)
+def dist_helpers(world, device=None):
+    """barrier() and max_over_ranks(v) over the default process group of
+    `world` ranks (both plain no-ops for one rank).  Timing is taken as the
+    maximum over ranks of each rank's device-timed interval."""
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def replica_shape(name, rank):
+    """Weak scaling: every rank runs the whole workload on its own seeded batch."""
+    from m3_inputs import WORKLOADS
+    return WORKLOADS[name].with_(seed=WORKLOADS[name].seed + rank)
+
+
+def job_tokens_per_s(world, steps, shape, elapsed_s):
+    """Whole-job throughput: tokens of all ranks over the max-over-ranks time."""
+    return world * steps * shape.batch * shape.seqlen / elapsed_s
+
+
 # ---------------------------------------------------------------- reference arm (the oracle)
 def run_reference(args):
     import numpy as np
@@ -251,21 +284,12 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = dist_helpers(world, dev)
 
     hbm_peak, peak_src = peaks()
     keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
     algo = {"auto": m3.ALGO_AUTO, "simt": m3.ALGO_SIMT, "tc": m3.ALGO_TC}[args.algo]
-    s = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    s = replica_shape(args.workload, rank)
     inp = make_prefill(s, device=dev)
     dims = m3.make_dims(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.rank, s.torch_io)
     use_tc = algo != m3.ALGO_SIMT and m3.workspace_size(dims) >= 0 and _tc_supported(m3, inp, keys, algo)
@@ -304,8 +328,7 @@ def run_ours(args):
     clk = clocks.stop()
     elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     launch = statistics.mean(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)) / 1e3
-    tokens = world * K * s.batch * s.seqlen
-    value = tokens / elapsed
+    value = job_tokens_per_s(world, K, s, elapsed)
     abytes = prefill_bytes(s)
     achieved = abytes / launch / 1e9
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -406,7 +429,7 @@ def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_p
 
     from m3_inputs import make_bcnorm
 
-    s = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    s = replica_shape(args.workload, rank)
     inp = make_prefill(s, device=dev, **({} if kind == "bcnorm" else {kind: True}))
     bcn = None
     if kind == "bcnorm":
@@ -446,7 +469,7 @@ def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_pe
     import torch
     from m3_inputs import WORKLOADS, make_prefill, make_steps
 
-    s = WORKLOADS[name].with_(seed=WORKLOADS[name].seed + rank)
+    s = replica_shape(name, rank)
     pre = make_prefill(s, device=dev)
     _, st = m3.scan_fwd(*(pre[k] for k in keys), None)
     A, D = pre["A"], pre["D"]
