@@ -376,7 +376,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
         el2 = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-        line["e2e"] = {"value": tokens / el2, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        line["e2e"] = {"value": job_tokens_per_s(world, K, s, el2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h}
         del host, dbuf, yh, hh
 

@@ -75,7 +75,6 @@ constexpr uint32_t kColS = 0, kColG = 128, kColYo = 192, kColYd = 320, kColP = 3
 constexpr int kNX = 3;   // x tile stages (also the number of per-chunk scalar buffers)
 constexpr uint32_t kBarPro = 1, kBarState = 2;  // named barriers of the two warpgroups
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kPrefetchAhead = 3;  // chunks of tiles prefetched into L2 ahead of their load
 // Sequence splitting (host policy): at most kMaxSegments segments of at least
 // kMinSegChunks chunks; the summary pass costs about kSumCost of the full pass
 // per chunk and the segment scan about kScanCost chunk-times.
@@ -91,6 +90,9 @@ struct Cfg {
     static constexpr int NPART = kPro / G4;  // token parts of the angle pass
     static constexpr int TPT = Q / NPART;    // tokens per thread in the angle pass
     static constexpr int TB = (2 / R) < 1 ? 1 : ((2 / R) < TPT ? (2 / R) : TPT);  // tokens per rotation batch
+    // chunks of tiles prefetched into L2 ahead of their load (measured: 2 for
+    // the 128-token chunks of rank 1, 3 for the shorter chunks of MIMO)
+    static constexpr int PREFETCH = R == 1 ? 2 : 3;
     static constexpr uint32_t X_BYTES = kRows * 128;         // 16 KB
     static constexpr uint32_t BC_BYTES = KB * kRows * 128;   // one B or C tile
     static constexpr uint32_t BCS_BYTES = 2 * BC_BYTES;      // one stage of the B/C ring
@@ -435,9 +437,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (!th_head) tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // read straight into registers
             };
             int issued = 0;
-            for (int i = 0; i < kPrefetchAhead && i < nloc; ++i) prefetch_chunk(cb + i);
+            for (int i = 0; i < C::PREFETCH && i < nloc; ++i) prefetch_chunk(cb + i);
             for (int i = 0; i < nloc; ++i) {
-                if (i + kPrefetchAhead < nloc) prefetch_chunk(cb + i + kPrefetchAhead);
+                if (i + C::PREFETCH < nloc) prefetch_chunk(cb + i + C::PREFETCH);
                 const int s = i & 1;
                 if (i >= 2 && !mbar_wait(&bb.empty_bc[s], ((i >> 1) - 1) & 1, abort_flag, err, kErrWaitMma)) break;
                 uint8_t *st = smem + C::OFF_BC + s * C::BCS_BYTES;

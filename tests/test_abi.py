@@ -162,3 +162,49 @@ def test_library_has_no_unresolved_internal_symbols(m3):
     missing = [l.split()[-1] for l in out.splitlines() if "_ZN2m3" in l]
     assert not missing, f"undefined library-internal symbols: {missing}"
     ctypes.CDLL(m3.LIB_PATH, mode=os.RTLD_NOW)  # resolves every symbol now
+
+
+def _undefined_names(path):
+    """Names a function of `path` loads but that are bound nowhere: not in the
+    function (or an enclosing one), not at module level, not a builtin."""
+    import ast
+    import builtins
+    tree = ast.parse(open(path).read())
+    module_names = set(dir(builtins))
+    for node in ast.walk(tree):
+        if isinstance(node, (ast.FunctionDef, ast.ClassDef)):
+            module_names.add(node.name)
+        elif isinstance(node, (ast.Import, ast.ImportFrom)):
+            module_names.update((a.asname or a.name).split(".")[0] for a in node.names)
+    for node in tree.body:
+        for t in ast.walk(node) if isinstance(node, (ast.Assign, ast.AnnAssign)) else []:
+            if isinstance(t, ast.Name):
+                module_names.add(t.id)
+    missing = set()
+
+    def visit(fn, bound):
+        local = set(bound)
+        for n in ast.walk(fn):
+            if isinstance(n, ast.Name) and isinstance(n.ctx, (ast.Store, ast.Del)):
+                local.add(n.id)
+            elif isinstance(n, ast.arg):
+                local.add(n.arg)
+            elif isinstance(n, (ast.FunctionDef, ast.Lambda)) and n is not fn and isinstance(n, ast.FunctionDef):
+                local.add(n.name)
+            elif isinstance(n, (ast.Import, ast.ImportFrom)):
+                local.update((a.asname or a.name).split(".")[0] for a in n.names)
+            elif isinstance(n, ast.ExceptHandler) and n.name:
+                local.add(n.name)
+        for n in ast.walk(fn):
+            if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load) and n.id not in local | module_names:
+                missing.add(n.id)
+
+    for node in tree.body:
+        if isinstance(node, ast.FunctionDef):
+            visit(node, set())
+    return missing
+
+
+def test_bench_has_no_undefined_names():
+    """bench.py's GPU legs cannot run here; at least every name they load is bound."""
+    assert _undefined_names(os.path.join(ROOT, "bench.py")) == set()
