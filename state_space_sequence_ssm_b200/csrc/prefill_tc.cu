@@ -90,9 +90,11 @@ struct Cfg {
     static constexpr int NPART = kPro / G4;  // token parts of the angle pass
     static constexpr int TPT = Q / NPART;    // tokens per thread in the angle pass
     static constexpr int TB = (2 / R) < 1 ? 1 : ((2 / R) < TPT ? (2 / R) : TPT);  // tokens per rotation batch
-    // chunks of tiles prefetched into L2 ahead of their load (measured: 2 for
-    // the 128-token chunks of rank 1, 3 for the shorter chunks of MIMO)
-    static constexpr int PREFETCH = R == 1 ? 2 : 3;
+    // chunks of tiles prefetched into L2 ahead of their load.  Measured: for
+    // N = 128 any prefetch distance over-fetches (lines evicted before their
+    // load) and costs time, so none; for N = 64 (half the bytes per chunk)
+    // three chunks are as good as or better than fewer.
+    static constexpr int PREFETCH = N == 128 ? 0 : 3;
     static constexpr uint32_t X_BYTES = kRows * 128;         // 16 KB
     static constexpr uint32_t BC_BYTES = KB * kRows * 128;   // one B or C tile
     static constexpr uint32_t BCS_BYTES = 2 * BC_BYTES;      // one stage of the B/C ring
