@@ -219,6 +219,47 @@ M3_API m3_status m3_scan_fwd_static(int algo, const m3_dims *d,
                              const m3_state *init, void *y, const m3_state *final_state,
                              void *stream);
 
+/* How m3_scan_fwd_host will run `d` on the current device: the device
+ * workspace it needs (bytes), the tokens per time slice, the sequences per
+ * group and the number of (group, slice) units.  Any output pointer may be
+ * NULL.  Slices are multiples of 128 tokens (one slice when seqlen <= 128);
+ * the plan aims for 8 units, cutting time first and batch after. */
+M3_API m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *slice_tokens,
+                                   int64_t *group_batch, int64_t *units);
+
+/* m3_scan_fwd for sequences held in HOST memory: x, B, C, dt, lam, theta, A,
+ * D, y and the optional init / final_state buffers are host pointers (same
+ * shapes, dtypes and m3_dims flags as m3_scan_fwd); `workspace` is DEVICE
+ * memory of at least m3_scan_host_plan's size, 16-byte aligned.  The result
+ * is the scan of the whole sequence, as m3_scan_fwd computes it.
+ *   - Pipelining: the call cuts the problem into (group of sequences) x
+ *     (time slice) units and chains the slices of a group through the
+ *     recurrent state (each slice resumes from the state the previous one
+ *     left, exactly as a caller resumes one m3_scan_fwd with the previous
+ *     call's final_state).  Copies in, kernels and copies out of successive
+ *     units overlap on two copy streams of the library's own (created once
+ *     per device on first use) and the caller's `stream`.
+ *   - Asynchronous on `stream`: all of the call's work, copies included, is
+ *     ordered after the work queued on `stream` before the call, and work
+ *     queued on `stream` afterwards runs after all of it (y and final_state
+ *     are complete once `stream` has reached that point).  Host buffers must
+ *     stay valid and unmodified until then.  Pinned (page-locked) host memory
+ *     lets the copies overlap; pageable memory works but serialises them.
+ *   - Calls on one device are serialised while they enqueue; two calls must
+ *     not share a workspace unless `stream` orders them.
+ *   - Host buffers: y must not overlap an input; final_state must not overlap
+ *     the inputs or y; init and final_state may be identical (in-place
+ *     resume), not partially overlapping.
+ *   - No BC-norm prologue and no explicit kernel choice (m3_scan_fwd's
+ *     automatic choice runs every unit).  On an error returned after some
+ *     units were queued, y and final_state are undefined. */
+M3_API m3_status m3_scan_fwd_host(const m3_dims *d,
+                           const void *x, const void *B, const void *C,
+                           const void *dt, const void *lam, const void *theta,
+                           const float *A, const float *D,
+                           const m3_state *init, void *y, const m3_state *final_state,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
 /* Decode: one token per (batch, head) against a resident state, updated in
  * place (the recurrent form of the same method, one token at a time).
  * x [batch,nheads,rank,headdim], B/C [batch,nheads,rank,dstate],

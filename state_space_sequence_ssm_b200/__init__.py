@@ -93,6 +93,11 @@ def _load():
     lib.m3_scan_fwd_static.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp]
     lib.m3_scan_fwd_static.restype = ctypes.c_int
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    lib.m3_scan_host_plan.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t), i64p, i64p, i64p]
+    lib.m3_scan_host_plan.restype = ctypes.c_int
+    lib.m3_scan_fwd_host.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_scan_fwd_host.restype = ctypes.c_int
     for f in (lib.m3_scan_workspace_size, lib.m3_scan_plan, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
         f.restype = ctypes.c_int
     lib.m3_selftest_wait_timeout.argtypes = [vp]
@@ -228,6 +233,66 @@ def scan_fwd_static(x, B, C, dt, lam, theta, A, D, init: State | None = None, *,
                       torch.empty(Bt, H, R, P, device=x.device))
     _check(get_lib().m3_scan_fwd_static(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
                                         _cstate(init), _ptr(y), _cstate(final), _stream(stream)))
+    return y, final
+
+
+class HostPlan(NamedTuple):
+    workspace_bytes: int  # device staging memory scan_fwd_host needs
+    slice_tokens: int     # tokens per time slice
+    group_batch: int      # sequences per group
+    units: int            # (group, slice) units of one call
+
+
+def scan_host_plan(dims: Dims) -> HostPlan:
+    """How scan_fwd_host cuts a problem of these dims into pipelined units."""
+    n, ts, gb, u = ctypes.c_size_t(0), ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(get_lib().m3_scan_host_plan(ctypes.byref(dims), ctypes.byref(n), ctypes.byref(ts), ctypes.byref(gb),
+                                       ctypes.byref(u)))
+    return HostPlan(n.value, ts.value, gb.value, u.value)
+
+
+def _require_host(*ts):
+    for t in ts:
+        if t is not None:
+            if t.is_cuda:
+                raise ValueError("m3: scan_fwd_host takes host tensors (pinned for overlapped copies)")
+            if not t.is_contiguous():
+                raise ValueError("m3: tensors must be contiguous")
+
+
+def _hstate(s: State | None):
+    if s is None:
+        return None
+    _require_host(*s)
+    return ctypes.pointer(CState(s.h.data_ptr(), s.b_prev.data_ptr(), s.x_prev.data_ptr()))
+
+
+def scan_fwd_host(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
+                  y=None, final: State | None = None, workspace=None, stream=None):
+    """scan_fwd over host tensors (same shapes as scan_fwd; pinned memory lets
+    the copies overlap): the library copies the inputs in, runs the scan and
+    copies y (and the final state) back, pipelined over time slices, all
+    ordered on `stream`.  `workspace` is a CUDA uint8 tensor of at least
+    scan_host_plan(dims).workspace_bytes (allocated when None).  Returns
+    (y, final State or None) as host tensors, complete once `stream` has
+    reached the end of the call."""
+    _require_host(x, B, C, dt, lam, theta, A, D, y)
+    Bt, T, H, R, P = x.shape
+    N = B.shape[-1]
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    if final is None and want_state:
+        f = dict(dtype=torch.float32, pin_memory=True)
+        final = State(torch.empty(Bt, H, N, P, **f), torch.empty(Bt, H, R, N, **f), torch.empty(Bt, H, R, P, **f))
+    if workspace is None:
+        need = scan_host_plan(dims).workspace_bytes
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    _require_cuda(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(get_lib().m3_scan_fwd_host(ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
+                                      _hstate(init), _ptr(y), _hstate(final), _ptr(workspace), ws_bytes,
+                                      _stream(stream)))
     return y, final
 
 

@@ -232,6 +232,11 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
 
 }  // namespace
 
+namespace m3 {
+m3_status set_error(m3_status s, const char *msg) { return fail(s, "%s", msg); }
+m3_status set_cuda_error(cudaError_t e, const char *where) { return cuda_fail(e, where); }
+}  // namespace m3
+
 extern "C" {
 
 int m3_version(void) { return 100; }

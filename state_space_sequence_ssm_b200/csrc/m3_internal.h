@@ -57,5 +57,8 @@ cudaError_t launch_wait_selftest(cudaStream_t stream);
 cudaError_t read_device_error(unsigned *code, cudaStream_t stream);
 // Read and clear the decode kernels' device error word (after a sync).
 cudaError_t read_decode_error(unsigned *code);
+// Record the calling thread's failure message (m3_last_error) and return `s`.
+m3_status set_error(m3_status s, const char *msg);
+m3_status set_cuda_error(cudaError_t e, const char *where);
 
 }  // namespace m3
