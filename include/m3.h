@@ -26,8 +26,9 @@
  *     means h = 0, b_prev = 0, x_prev = 0;
  *   - B and C are per head; A and D are per head (fp32).
  *
- * Memory: every pointer is a DEVICE pointer owned by the caller; the library
- * never allocates on these paths.  Tensors are dense, row-major (last index
+ * Memory: every pointer is a DEVICE pointer owned by the caller (except the
+ * sequence and state pointers of m3_scan_fwd_host, which are host memory);
+ * the library never allocates memory on these paths.  Tensors are dense, row-major (last index
  * fastest), base addresses 16-byte aligned.  "io" tensors are fp32 or bf16
  * according to m3_dims.io; A, D and all state buffers are fp32.
  *
@@ -223,7 +224,8 @@ M3_API m3_status m3_scan_fwd_static(int algo, const m3_dims *d,
  * workspace it needs (bytes), the tokens per time slice, the sequences per
  * group and the number of (group, slice) units.  Any output pointer may be
  * NULL.  Slices are multiples of 128 tokens (one slice when seqlen <= 128);
- * the plan aims for 8 units, cutting time first and batch after. */
+ * the plan aims for 8 units: groups of whole sequences first, then time
+ * slices when there are fewer than 8 groups. */
 M3_API m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *slice_tokens,
                                    int64_t *group_batch, int64_t *units);
 

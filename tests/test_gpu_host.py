@@ -57,12 +57,13 @@ def by_units(inp, init, plan, shape):
 
 CASES = [
     # (shape, per-token A, theta per head, with init)
-    (Shape(2, 1000, 2, 64, 128, 1, "bf16", 301), False, False, True),    # 8 time slices, ragged last
+    (Shape(2, 1000, 2, 64, 128, 1, "bf16", 301), False, False, True),    # 2 sequences x 4 slices, ragged last
     (Shape(2, 1000, 2, 64, 128, 1, "bf16", 302), False, False, False),
-    (Shape(5, 300, 2, 64, 128, 2, "bf16", 303), False, False, True),     # 3 groups x 3 slices
+    (Shape(5, 300, 2, 64, 128, 2, "bf16", 303), False, False, True),     # 5 x 2 slices (256 + 44 tokens)
     (Shape(3, 300, 2, 64, 64, 4, "bf16", 304), True, True, True),        # MIMO, both optional features
-    (Shape(16, 100, 2, 64, 64, 1, "f32", 305), False, False, True),      # 8 groups, one slice each
-    (Shape(1, 2600, 1, 64, 128, 1, "bf16", 306), True, False, False),    # long slices (384 tokens)
+    (Shape(16, 100, 2, 64, 64, 1, "f32", 305), False, False, True),      # 8 groups of 2, one slice each
+    (Shape(12, 300, 1, 64, 64, 1, "bf16", 307), False, False, True),     # groups of 2 x 2 slices: strided copies
+    (Shape(1, 2600, 1, 64, 128, 1, "bf16", 306), True, False, False),    # 7 slices of 384 tokens
 ]
 
 
