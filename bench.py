@@ -393,10 +393,35 @@ def run_ours(args):
             ref[name] = 3 * n / (c0.elapsed_time(c1) / 1e3) / 1e9
             del hbuf, dbuf
         bound = max(h2d / ref["h2d"], d2h / ref["d2h"]) / 1e9  # seconds per step if the copies alone set the pace
+        # both directions at once (two streams), the step's bytes scaled to at most 1 GiB in total
+        f = min(1.0, (1 << 30) / (h2d + d2h))
+        nin, nout = max(16, int(h2d * f)), max(16, int(d2h * f))
+        hin = torch.empty(nin, dtype=torch.uint8, pin_memory=True)
+        din = torch.empty(nin, dtype=torch.uint8, device=dev)
+        hout = torch.empty(nout, dtype=torch.uint8, pin_memory=True)
+        dout = torch.empty(nout, dtype=torch.uint8, device=dev)
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for rep in range(2):
+            torch.cuda.synchronize()
+            c0.record(stream)
+            s_in.wait_stream(stream)
+            s_out.wait_stream(stream)
+            with torch.cuda.stream(s_in):
+                din.copy_(hin, non_blocking=True)
+            with torch.cuda.stream(s_out):
+                hout.copy_(dout, non_blocking=True)
+            stream.wait_stream(s_in)
+            stream.wait_stream(s_out)
+            c1.record(stream)
+            torch.cuda.synchronize()
+        duplex = c0.elapsed_time(c1) / 1e3 / f
+        del hin, din, hout, dout
         line["e2e"] = {"value": job_tokens_per_s(world, K, s, el2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "api": "m3_scan_fwd_host", "ms_per_step": el2 / K * 1e3,
                        "copy_reference": {"h2d_gbs": ref["h2d"], "d2h_gbs": ref["d2h"], "bound_ms": bound * 1e3,
-                                          "frac": bound / (el2 / K)},
+                                          "frac": bound / (el2 / K), "duplex_ms": duplex * 1e3,
+                                          "frac_of_duplex": duplex / (el2 / K)},
                        "pipeline": {"units": hplan.units, "slice_tokens": hplan.slice_tokens,
                                     "group_batch": hplan.group_batch}}
         del host, yh, fh, hws
