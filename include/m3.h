@@ -221,13 +221,15 @@ M3_API m3_status m3_scan_fwd_static(int algo, const m3_dims *d,
                              void *stream);
 
 /* How m3_scan_fwd_host will run `d` on the current device: the device
- * workspace it needs (bytes), the tokens per time slice, the sequences per
- * group and the number of (group, slice) units.  Any output pointer may be
- * NULL.  Slices are multiples of 128 tokens (one slice when seqlen <= 128);
- * the plan aims for 8 units: groups of whole sequences first, then time
- * slices when there are fewer than 8 groups. */
+ * workspace it needs (bytes), the tokens per time slice (of every group but
+ * the last, and of the last), the sequences per group and the number of
+ * (group, slice) units.  Any output pointer may be NULL.  Slices are
+ * multiples of 128 tokens (one slice when seqlen <= 128); the plan aims for 8
+ * units: groups of whole sequences first, then time slices when there are
+ * fewer than 8 groups; the last group is cut into at least 4 slices (when
+ * seqlen allows), so that little work is left once the last copy-in ends. */
 M3_API m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *slice_tokens,
-                                   int64_t *group_batch, int64_t *units);
+                                   int64_t *last_slice_tokens, int64_t *group_batch, int64_t *units);
 
 /* m3_scan_fwd for sequences held in HOST memory: x, B, C, dt, lam, theta, A,
  * D, y and the optional init / final_state buffers are host pointers (same

@@ -94,7 +94,7 @@ def _load():
     lib.m3_scan_fwd_static.restype = ctypes.c_int
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
     i64p = ctypes.POINTER(ctypes.c_int64)
-    lib.m3_scan_host_plan.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t), i64p, i64p, i64p]
+    lib.m3_scan_host_plan.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t), i64p, i64p, i64p, i64p]
     lib.m3_scan_host_plan.restype = ctypes.c_int
     lib.m3_scan_fwd_host.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     lib.m3_scan_fwd_host.restype = ctypes.c_int
@@ -237,18 +237,20 @@ def scan_fwd_static(x, B, C, dt, lam, theta, A, D, init: State | None = None, *,
 
 
 class HostPlan(NamedTuple):
-    workspace_bytes: int  # device staging memory scan_fwd_host needs
-    slice_tokens: int     # tokens per time slice
-    group_batch: int      # sequences per group
-    units: int            # (group, slice) units of one call
+    workspace_bytes: int    # device staging memory scan_fwd_host needs
+    slice_tokens: int       # tokens per time slice (every group but the last)
+    last_slice_tokens: int  # tokens per time slice of the last group
+    group_batch: int        # sequences per group
+    units: int              # (group, slice) units of one call
 
 
 def scan_host_plan(dims: Dims) -> HostPlan:
     """How scan_fwd_host cuts a problem of these dims into pipelined units."""
-    n, ts, gb, u = ctypes.c_size_t(0), ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
-    _check(get_lib().m3_scan_host_plan(ctypes.byref(dims), ctypes.byref(n), ctypes.byref(ts), ctypes.byref(gb),
-                                       ctypes.byref(u)))
-    return HostPlan(n.value, ts.value, gb.value, u.value)
+    n = ctypes.c_size_t(0)
+    ts, tl, gb, u = (ctypes.c_int64(0) for _ in range(4))
+    _check(get_lib().m3_scan_host_plan(ctypes.byref(dims), ctypes.byref(n), ctypes.byref(ts), ctypes.byref(tl),
+                                       ctypes.byref(gb), ctypes.byref(u)))
+    return HostPlan(n.value, ts.value, tl.value, gb.value, u.value)
 
 
 def _require_host(*ts):

@@ -36,6 +36,7 @@ namespace {
 
 constexpr int64_t kSliceAlign = 128;   // tokens; a multiple of every chunk length
 constexpr int64_t kUnitsTarget = 8;    // units per call the plan aims for
+constexpr int64_t kTailSlices = 4;     // the last group is cut into at least this many slices
 constexpr size_t kAlign = 256;         // byte alignment of every staging buffer
 constexpr int kMaxDevices = 64;
 
@@ -74,6 +75,7 @@ cudaError_t streams_for(int dev, Streams **out) {
 // workspace (byte offsets from its start).
 struct Layout {
     int64_t slice, group, nslice, ngroup;
+    int64_t slice_last, nslice_last;    // the last group's slicing (finer: a short pipeline tail)
     size_t A, D, theta;                 // per-head constants (theta only when fixed per head)
     size_t st[3][3];                    // state sets (initial, ping, pong) x (h, b_prev, x_prev)
     size_t slot[2][8];                  // x, B, C, dt, lam, theta, A, y of each slot
@@ -109,6 +111,15 @@ m3_status plan_layout(const m3_dims *d, Layout *L) {
     L->nslice = T <= kSliceAlign ? 1 : std::min(cdiv(T, kSliceAlign), want);
     L->slice = T <= kSliceAlign ? T : cdiv(cdiv(T, L->nslice), kSliceAlign) * kSliceAlign;
     if (T > kSliceAlign) L->nslice = cdiv(T, L->slice);
+    // What is left after the last copy-in -- the last unit's kernels and its
+    // copy-out -- is the pipeline's exposed tail: cut the last group finer.
+    L->slice_last = L->slice;
+    L->nslice_last = L->nslice;
+    if (T > kSliceAlign) {
+        const int64_t n = std::min(cdiv(T, kSliceAlign), std::max(L->nslice, kTailSlices));
+        L->slice_last = cdiv(cdiv(T, n), kSliceAlign) * kSliceAlign;
+        L->nslice_last = cdiv(T, L->slice_last);
+    }
 
     const size_t es = d->io == M3_BF16 ? 2 : 4;
     const size_t H = d->nheads, R = d->rank, P = d->headdim, N = d->dstate;
@@ -133,7 +144,8 @@ m3_status plan_layout(const m3_dims *d, Layout *L) {
         for (int t = 0; t < 8; ++t) L->slot[j][t] = rows.b[t] ? take(toks * rows.b[t]) : 0;
     // the scan's workspace: the largest any unit's shape asks for
     size_t need = 0;
-    const int64_t Ts[2] = {L->slice, T - (L->nslice - 1) * L->slice};
+    const int64_t Ts[4] = {L->slice, T - (L->nslice - 1) * L->slice, L->slice_last,
+                           T - (L->nslice_last - 1) * L->slice_last};
     const int64_t Bs[2] = {L->group, Bt - (L->ngroup - 1) * L->group};
     for (int64_t b : Bs)
         for (int64_t t : Ts) {
@@ -273,8 +285,10 @@ m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *
     int64_t k = 0;
     for (int64_t g = 0; g < L.ngroup; ++g) {
         const int64_t b0 = g * L.group, nb = std::min(L.group, Bt - b0);
-        for (int64_t i = 0; i < L.nslice; ++i, ++k) {
-            const int64_t t0 = i * L.slice, tl = std::min(L.slice, T - t0);
+        const bool last_group = g == L.ngroup - 1;
+        const int64_t ns = last_group ? L.nslice_last : L.nslice, sl = last_group ? L.slice_last : L.slice;
+        for (int64_t i = 0; i < ns; ++i, ++k) {
+            const int64_t t0 = i * sl, tl = std::min(sl, T - t0);
             const int j = (int)(k & 1);
             // copy-in: wait until unit k-2 no longer reads this slot
             if (k >= 2) M3_TRY(cudaStreamWaitEvent(S->in, S->computed[j], 0), "m3_scan_fwd_host (copy-in wait)");
@@ -324,7 +338,7 @@ m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *
             M3_TRY(copy_tokens(w + L.slot[j][7], nullptr, static_cast<char *>(y), rows.b[7], b0, nb, T, t0, tl,
                                S->out),
                    "m3_scan_fwd_host (copy-out)");
-            if (i == L.nslice - 1 && fin) {
+            if (i == ns - 1 && fin) {
                 void *dst[3] = {fin->h, fin->b_prev, fin->x_prev};
                 for (int q = 0; q < 3; ++q) {
                     const size_t per = sbytes[q] / (size_t)Bt;
@@ -347,7 +361,7 @@ m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *
 extern "C" {
 
 m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *slice_tokens,
-                            int64_t *group_batch, int64_t *units) {
+                            int64_t *last_slice_tokens, int64_t *group_batch, int64_t *units) {
     try {
         m3_status st = m3_scan_plan(M3_ALGO_AUTO, d, nullptr, nullptr, nullptr);
         if (st != M3_OK) return st;
@@ -355,8 +369,9 @@ m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *
         if ((st = plan_layout(d, &L)) != M3_OK) return st;
         if (workspace_bytes) *workspace_bytes = d->batch > 0 ? L.total : 0;
         if (slice_tokens) *slice_tokens = L.slice;
+        if (last_slice_tokens) *last_slice_tokens = L.slice_last;
         if (group_batch) *group_batch = L.group;
-        if (units) *units = L.nslice * L.ngroup;
+        if (units) *units = d->batch > 0 ? L.nslice * (L.ngroup - 1) + L.nslice_last : 0;
         return M3_OK;
     } catch (...) {
         return m3::set_error(M3_ERR_INVALID_ARG, "internal error");

@@ -168,19 +168,25 @@ def test_host_plan_units_and_staging(m3, Bt, T, H, P, N, R, io, flags):
     the whole sequence), the units cover the problem, and the workspace holds
     at least two staging slots and three state sets of one unit's size."""
     d = dims(m3, Bt=Bt, T=T, H=H, P=P, N=N, R=R, io=io, flags=flags)
-    ws, ts, gb, u = ctypes.c_size_t(0), ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
-    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), ctypes.byref(ts), ctypes.byref(gb),
-                                    ctypes.byref(u)) == 0
-    ts, gb, u = ts.value, gb.value, u.value
-    assert ts == T if T <= 128 else (ts % 128 == 0 and ts <= T + 127)
+    ws = ctypes.c_size_t(0)
+    ts, tl, gb, u = (ctypes.c_int64(0) for _ in range(4))
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), ctypes.byref(ts), ctypes.byref(tl),
+                                    ctypes.byref(gb), ctypes.byref(u)) == 0
+    ts, tl, gb, u = ts.value, tl.value, gb.value, u.value
+    for s in (ts, tl):
+        assert s == T if T <= 128 else (s % 128 == 0 and s <= T + 127)
     nslice = 1 if T <= 128 else -(-T // ts)
-    assert u == nslice * -(-Bt // gb)
-    # the documented rule: up to 8 groups of whole sequences, then time slices toward 8 units
-    groups = -(-Bt // -(-Bt // min(Bt, 8)))
+    nlast = 1 if T <= 128 else -(-T // tl)
+    groups = -(-Bt // gb)
+    assert u == nslice * (groups - 1) + nlast
+    # the documented rule: up to 8 groups of whole sequences, then time slices toward 8 units;
+    # the last group in at least 4 slices where the sequence has 4 chunks of 128 tokens
     assert gb == -(-Bt // min(Bt, 8))
     want = -(-8 // groups)
     if T > 128:
         assert ts == -(-(-(-T // min(-(-T // 128), want))) // 128) * 128
+        assert tl == -(-(-(-T // min(-(-T // 128), max(nslice, 4)))) // 128) * 128
+        assert tl <= ts
     es = 2 if io == 1 else 4
     per_tok = H * (2 * R * P * es + 2 * R * N * es + 2 * es + (0 if flags & 2 else N // 2 * es)
                    + (4 if flags & 1 else 0))
@@ -191,10 +197,10 @@ def test_host_plan_units_and_staging(m3, Bt, T, H, P, N, R, io, flags):
 def test_host_plan_empty_batch_and_bad_dims(m3):
     ws = ctypes.c_size_t(7)
     d = dims(m3, Bt=0, T=500)
-    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), None, None, None) == 0
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), None, None, None, None) == 0
     assert ws.value == 0
     bad = dims(m3, N=7)
-    assert m3.lib.m3_scan_host_plan(ctypes.byref(bad), None, None, None, None) == 1
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(bad), None, None, None, None, None) == 1
     # the host entry point validates before touching the device
     assert m3.lib.m3_scan_fwd_host(None, *([None] * 8), None, None, None, None, 0, None) == 1
 

@@ -44,9 +44,10 @@ def by_units(inp, init, plan, shape):
         ({"A"} if inp["A"].dim() == 3 else set())
     for b0 in range(0, Bt, plan.group_batch):
         b1 = min(Bt, b0 + plan.group_batch)
+        sl = plan.last_slice_tokens if b1 == Bt else plan.slice_tokens
         st = None if init is None else m3.State(*(t[b0:b1].cuda() for t in init))
-        for t0 in range(0, max(T, 1), max(plan.slice_tokens, 1)):
-            t1 = min(T, t0 + plan.slice_tokens)
+        for t0 in range(0, max(T, 1), max(sl, 1)):
+            t1 = min(T, t0 + sl)
             args = [(inp[k][b0:b1, t0:t1] if k in per_tok else inp[k]).contiguous().cuda() for k in KEYS]
             ys, st = m3.scan_fwd(*args, st)
             y[b0:b1, t0:t1] = ys.cpu()
@@ -59,10 +60,10 @@ CASES = [
     # (shape, per-token A, theta per head, with init)
     (Shape(2, 1000, 2, 64, 128, 1, "bf16", 301), False, False, True),    # 2 sequences x 4 slices, ragged last
     (Shape(2, 1000, 2, 64, 128, 1, "bf16", 302), False, False, False),
-    (Shape(5, 300, 2, 64, 128, 2, "bf16", 303), False, False, True),     # 5 x 2 slices (256 + 44 tokens)
+    (Shape(5, 300, 2, 64, 128, 2, "bf16", 303), False, False, True),     # 4 x 2 slices (256 + 44), last x 3
     (Shape(3, 300, 2, 64, 64, 4, "bf16", 304), True, True, True),        # MIMO, both optional features
     (Shape(16, 100, 2, 64, 64, 1, "f32", 305), False, False, True),      # 8 groups of 2, one slice each
-    (Shape(12, 300, 1, 64, 64, 1, "bf16", 307), False, False, True),     # groups of 2 x 2 slices: strided copies
+    (Shape(12, 300, 1, 64, 64, 1, "bf16", 307), False, False, True),     # groups of 2 x 2-3 slices: strided copies
     (Shape(1, 2600, 1, 64, 128, 1, "bf16", 306), True, False, False),    # 7 slices of 384 tokens
 ]
 
