@@ -45,7 +45,9 @@
  *
  * Execution: every call is asynchronous on the given CUDA stream (a
  * cudaStream_t passed as void*, NULL = legacy default stream) and never
- * synchronises the device.  Errors are returned as m3_status; the message of
+ * synchronises the device.  m3_scan_fwd / m3_scan_fwd_algo (whole and split
+ * sequences) and m3_step can be captured into a CUDA graph and replayed; the
+ * arguments (pointers included) are fixed at capture.  Errors are returned as m3_status; the message of
  * the calling thread's last failure is available from m3_last_error().  No
  * C++ exception crosses this boundary and no kernel traps.
  */

@@ -151,6 +151,16 @@ def _require_cuda(*ts):
                 raise ValueError("m3: tensors must be contiguous")
 
 
+def _scratch(nbytes: int, device, stream):
+    """A workspace the binding allocates for one call: marked as used by the
+    call's stream, so that the caching allocator does not hand it out again
+    before that stream has finished with it."""
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if stream is not None:
+        ws.record_stream(stream)
+    return ws
+
+
 def make_dims(Bt, T, H, P, N, R, dtype, a_per_token: bool = False, theta_per_head: bool = False) -> Dims:
     io = M3_BF16 if dtype == torch.bfloat16 else M3_F32
     if dtype not in (torch.bfloat16, torch.float32):
@@ -207,7 +217,7 @@ def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_s
                       torch.empty(Bt, H, R, P, device=x.device))
     ws_need = workspace_size(dims, algo) if algo != ALGO_SIMT else 0
     if workspace is None and ws_need:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=x.device)
+        workspace = _scratch(ws_need, x.device, stream)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(init), _ptr(y), _cstate(final), _ptr(workspace),
             ws_bytes, _stream(stream))
@@ -288,8 +298,7 @@ def scan_fwd_host(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, w
         f = dict(dtype=torch.float32, pin_memory=True)
         final = State(torch.empty(Bt, H, N, P, **f), torch.empty(Bt, H, R, N, **f), torch.empty(Bt, H, R, P, **f))
     if workspace is None:
-        need = scan_host_plan(dims).workspace_bytes
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+        workspace = _scratch(max(scan_host_plan(dims).workspace_bytes, 1), torch.device("cuda"), stream)
     _require_cuda(workspace)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(get_lib().m3_scan_fwd_host(ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
