@@ -544,9 +544,7 @@ template <typename IO, int R, bool GEN>
 cudaError_t dispatch_np(const StepArgs<IO> &a, const StepFeat &f, cudaStream_t s, bool *done) {
     *done = true;
     // rank 1: one CTA per slice (measured faster); rank >= 2: the persistent
-    // streaming kernel (its heavier per-element work overlaps the next slice's
-    // load; measured at rank 4, N 128: 103 us per step against 176 us for one
-    // CTA per slice)
+    // streaming kernel (its heavier per-element work overlaps the next slice's load)
     // (BC-norm: the tiled kernel, which normalises its staged rows in place)
     const bool tiled = R == 1 || f.wB;
     if (a.N == 128 && a.P == 64)
