@@ -433,8 +433,11 @@ def run_ours(args):
     if not args.no_decode:
         del inp, y, fin
         torch.cuda.empty_cache()
+        # the long-context workload continues its own sequences (its prefill's
+        # state, then 256 steps); every other line reports the batch-256 decode workloads
+        names = [args.workload] if args.workload.startswith("long") else DECODE_WORKLOADS
         line["decode"] = [run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
-                                     peak_src, keys) for name in DECODE_WORKLOADS]
+                                     peak_src, keys) for name in names]
 
     # ---- CPU baseline: the oracle as it stands on this machine's host cores (rank 0, N = 1)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -513,7 +516,7 @@ def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_p
 
 def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys):
     import torch
-    from m3_inputs import WORKLOADS, make_prefill, make_steps
+    from m3_inputs import LONG_DECODE_STEPS, WORKLOADS, make_prefill, make_steps
 
     s = replica_shape(name, rank)
     pre = make_prefill(s, device=dev)
@@ -521,7 +524,7 @@ def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_pe
     A, D = pre["A"], pre["D"]
     del pre
     torch.cuda.empty_cache()
-    S = args.decode_steps
+    S = LONG_DECODE_STEPS if name.startswith("long") else args.decode_steps
     steps = make_steps(s, S, device=dev)
     y = torch.empty(s.batch, s.nheads, s.rank, s.headdim, dtype=s.torch_io, device=dev)
     stream = torch.cuda.Stream(device=dev)

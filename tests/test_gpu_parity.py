@@ -198,16 +198,21 @@ def test_full_size_prefill_sampled(name, nslices):
     check_full_prefill(name, m3.ALGO_AUTO, nslices)
 
 
-@pytest.mark.parametrize("name", ["decode_bf16_b256_h32_p64_n128_r1", "decode_bf16_b256_h32_p64_n128_r4"])
-def test_full_size_decode_sampled(name):
-    """1024-token prefill, then 1000 decode steps on every slice; sampled
-    slices checked against the oracle's prefill + steps."""
-    from m3_inputs import DECODE_STEPS
+@pytest.mark.parametrize("name,nsteps,nslices", [
+    ("decode_bf16_b256_h32_p64_n128_r1", 1000, 3),
+    ("decode_bf16_b256_h32_p64_n128_r4", 1000, 3),
+    ("long_mimo_bf16_b1_t65536_h64_p64_n128_r4", 256, 1),
+])
+def test_full_size_decode_sampled(name, nsteps, nslices):
+    """The workload's prefill (1024 tokens; 65,536 for the long-context
+    one), then its decode steps on every slice; sampled slices checked against
+    the oracle's prefill + steps."""
+    DECODE_STEPS = nsteps
     shape = WORKLOADS[name]
     inp = make_prefill(shape, device=DEV)
     _, st = m3.scan_fwd(*(inp[k] for k in KEYS), None)
     steps = make_steps(shape, DECODE_STEPS, device=DEV)
-    picks = sampled_slices(shape, 3)
+    picks = sampled_slices(shape, nslices)
     bi = torch.tensor([b for b, _ in picks], device=DEV)
     hi = torch.tensor([h for _, h in picks], device=DEV)
     ys = []
