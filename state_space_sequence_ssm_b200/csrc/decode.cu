@@ -44,34 +44,6 @@ template <>
 __device__ __forceinline__ void stv<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float v) {
     p[i] = __float2bfloat16_rn(v);
 }
-// 4 consecutive io values starting at element i (i multiple of 4)
-template <typename T>
-__device__ __forceinline__ float4 ld4(const T *p, int64_t i);
-template <>
-__device__ __forceinline__ float4 ld4<float>(const float *p, int64_t i) {
-    return __ldg(reinterpret_cast<const float4 *>(p + i));
-}
-template <>
-__device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
-    const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p + i));
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
-    const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-// 2 consecutive io values starting at element i (i even)
-template <typename T>
-__device__ __forceinline__ float2 ld2(const T *p, int64_t i);
-template <>
-__device__ __forceinline__ float2 ld2<float>(const float *p, int64_t i) {
-    return __ldg(reinterpret_cast<const float2 *>(p + i));
-}
-template <>
-__device__ __forceinline__ float2 ld2<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(p + i);
-    return __bfloat1622float2(v);
-}
-
 template <typename IO>
 struct StepArgs {
     int64_t BH, H;
@@ -346,14 +318,6 @@ template <>
 __device__ __forceinline__ float sv<float>(const float *p, int i) { return p[i]; }
 template <>
 __device__ __forceinline__ float sv<__nv_bfloat16>(const __nv_bfloat16 *p, int i) { return __bfloat162float(p[i]); }
-template <typename T>
-__device__ __forceinline__ float2 sv2(const T *p, int i);
-template <>
-__device__ __forceinline__ float2 sv2<float>(const float *p, int i) { return *reinterpret_cast<const float2 *>(p + i); }
-template <>
-__device__ __forceinline__ float2 sv2<__nv_bfloat16>(const __nv_bfloat16 *p, int i) {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p + i));
-}
 template <typename T>
 __device__ __forceinline__ float4 sv4(const T *p, int i);
 template <>

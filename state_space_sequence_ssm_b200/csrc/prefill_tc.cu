@@ -158,20 +158,6 @@ __device__ __forceinline__ bool bar_any(bool pred) {
     return r != 0;
 }
 
-// bf16 copy of the 64 fp32 values of state row n into the 128B-swizzled
-// MN-major operand tile (row n = K index of the readout MMA).
-__device__ __forceinline__ void store_state_row(uint8_t *hb, int n, const float (&h)[64]) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        uint4 v;
-        v.x = pack_bf16(h[8 * j + 0], h[8 * j + 1]);
-        v.y = pack_bf16(h[8 * j + 2], h[8 * j + 3]);
-        v.z = pack_bf16(h[8 * j + 4], h[8 * j + 5]);
-        v.w = pack_bf16(h[8 * j + 6], h[8 * j + 7]);
-        *reinterpret_cast<uint4 *>(hb + sw128(n, j)) = v;
-    }
-}
-
 // bf16 copy of 32 fp32 values (columns 32*half ..) of state row n into the
 // 128B-swizzled MN-major operand tile (row n = K index of the readout MMA).
 __device__ __forceinline__ void store_state_half(uint8_t *hb, int n, int half, const float (&h)[32]) {
