@@ -17,10 +17,8 @@ from __future__ import annotations
 
 import argparse
 import datetime
-import glob
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -231,7 +229,6 @@ def job_tokens_per_s(world, steps, shape, elapsed_s):
 
 # ---------------------------------------------------------------- reference arm (the oracle)
 def run_reference(args):
-    import numpy as np
     import torch
 
     import oracle
@@ -269,7 +266,6 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- our arm
 def run_ours(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -568,8 +564,6 @@ def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_pe
 
 
 def cpu_baseline(s, keys):
-    import numpy as np
-
     import oracle
     from m3_inputs import make_prefill
 

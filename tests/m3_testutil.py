@@ -7,7 +7,6 @@ import numpy as np
 import torch
 
 import oracle
-from m3_inputs import Shape, make_prefill, make_state, make_steps
 
 # tolerances: fp32 I/O path and bf16 I/O path (fp32 state)
 TOL_F32 = 1e-4

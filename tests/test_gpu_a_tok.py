@@ -1,7 +1,6 @@
 """GPU parity with a data-dependent A_t (one fp32 value per token-head,
 M3_FLAG_A_PER_TOKEN) against the fp64 oracle: tensor-core and SIMT prefill,
 split sequences, decode steps, and the full-size SISO workload sampled."""
-import numpy as np
 import pytest
 import torch
 

@@ -1,12 +1,11 @@
 """GPU parity of the tensor-core prefill with sequences split into segments
 (summary pass, segment scan, main pass) against the fp64 oracle, and against
 the same path unsplit."""
-import numpy as np
 import pytest
 import torch
 
 from m3_inputs import WORKLOADS, Shape, make_prefill, make_state
-from m3_testutil import KEYS, TOL_BF16, host64, max_rel_l2_state, max_rel_l2_y
+from m3_testutil import KEYS, host64, max_rel_l2_state, max_rel_l2_y
 
 from test_gpu_parity import check_scan, to_dev
 
