@@ -35,24 +35,25 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 def parse():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=PREFILL_WORKLOAD)
-    ap.add_argument("--algo", choices=["auto", "simt", "tc"], default="auto")
-    ap.add_argument("--decode-steps", type=int, default=1000)
-    ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
+    ap = argparse.ArgumentParser(description="Mamba-3 SSM forward benchmark: one JSON line on stdout (rank 0).")
+    ap.add_argument("--gpus", type=int, default=1, help="GPUs (one process each, launched by torchrun for N > 1)")
+    ap.add_argument("--steps", type=int, default=20, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
+                    help="ours: the CUDA library; reference: the fp64 oracle on the host cores")
+    ap.add_argument("--workload", default=PREFILL_WORKLOAD, help="prefill workload (a name in m3_inputs.WORKLOADS)")
+    ap.add_argument("--algo", choices=["auto", "simt", "tc"], default="auto", help="prefill kernel choice")
+    ap.add_argument("--decode-steps", type=int, default=1000, help="graph-captured steps of the decode lines")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-variants", action="store_true",
-                    help="skip the data-dependent-A variant of the prefill workload")
+                    help="skip the variant lines (per-token A, per-head theta, BC-norm) of the prefill workload")
     ap.add_argument("--case", choices=["prefill", "decode"], default=None,
                     help="profiling case: only run --case-launches launches of one kernel at --case-batch "
                          "(for ncu captures; prints no bench line)")
-    ap.add_argument("--case-batch", type=int, default=None)
-    ap.add_argument("--case-launches", type=int, default=3)
+    ap.add_argument("--case-batch", type=int, default=None, help="batch of the profiling case")
+    ap.add_argument("--case-launches", type=int, default=3, help="launches of the profiling case")
     return ap.parse_args()
 
 
