@@ -31,7 +31,8 @@
 //   warp 16     TMA producers: lane 0 fills a 2-stage ring of B and C tiles
 //               (freed as soon as S, G and Yo have read them), lane 1 a
 //               3-stage ring of x tiles (freed after the epilogue), both
-//               128B-swizzled, with L2 prefetches of the chunks ahead;
+//               128B-swizzled (for N = 64 also L2 prefetches of the chunks
+//               ahead);
 //   warp 17     TMEM owner and single-thread MMA issuer.
 // A sequence too long for the grid to fill the GPU is split into segments
 // (a summary pass, a scan over the segments, then this pass per segment:
