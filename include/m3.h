@@ -222,7 +222,8 @@ M3_API m3_status m3_scan_fwd_static(int algo, const m3_dims *d,
                              const m3_state *init, void *y, const m3_state *final_state,
                              void *stream);
 
-/* How m3_scan_fwd_host will run `d` on the current device: the device
+/* How m3_scan_fwd_host will run `d` (with the BC-norm prologue when
+ * `with_bcnorm` is non-zero) on the current device: the device
  * workspace it needs (bytes), the tokens per time slice (of every group but
  * the last, and of the last), the sequences per group and the number of
  * (group, slice) units.  Any output pointer may be NULL.  Slices are
@@ -230,14 +231,17 @@ M3_API m3_status m3_scan_fwd_static(int algo, const m3_dims *d,
  * units: groups of whole sequences first, then time slices when there are
  * fewer than 8 groups; the last group is cut into at least 4 slices (when
  * seqlen allows), so that little work is left once the last copy-in ends. */
-M3_API m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *slice_tokens,
-                                   int64_t *last_slice_tokens, int64_t *group_batch, int64_t *units);
+M3_API m3_status m3_scan_host_plan(const m3_dims *d, int with_bcnorm, size_t *workspace_bytes,
+                                   int64_t *slice_tokens, int64_t *last_slice_tokens, int64_t *group_batch,
+                                   int64_t *units);
 
 /* m3_scan_fwd for sequences held in HOST memory: x, B, C, dt, lam, theta, A,
  * D, y and the optional init / final_state buffers are host pointers (same
  * shapes, dtypes and m3_dims flags as m3_scan_fwd); `workspace` is DEVICE
  * memory of at least m3_scan_host_plan's size, 16-byte aligned.  The result
- * is the scan of the whole sequence, as m3_scan_fwd computes it.
+ * is the scan of the whole sequence, as m3_scan_fwd computes it (as
+ * m3_scan_fwd_bcnorm when `bcn` is non-NULL: its four arrays are then host
+ * memory too, copied to the device once per call).
  *   - Pipelining: the call cuts the problem into (group of sequences) x
  *     (time slice) units and chains the slices of a group through the
  *     recurrent state (each slice resumes from the state the previous one
@@ -256,10 +260,10 @@ M3_API m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, in
  *   - Host buffers: y must not overlap an input; final_state must not overlap
  *     the inputs or y; init and final_state may be identical (in-place
  *     resume), not partially overlapping.
- *   - No BC-norm prologue and no explicit kernel choice (m3_scan_fwd's
- *     automatic choice runs every unit).  On an error returned after some
- *     units were queued, y and final_state are undefined. */
-M3_API m3_status m3_scan_fwd_host(const m3_dims *d,
+ *   - No explicit kernel choice (m3_scan_fwd's automatic choice runs every
+ *     unit).  On an error returned after some units were queued, y and
+ *     final_state are undefined. */
+M3_API m3_status m3_scan_fwd_host(const m3_dims *d, const m3_bcnorm *bcn,
                            const void *x, const void *B, const void *C,
                            const void *dt, const void *lam, const void *theta,
                            const float *A, const float *D,

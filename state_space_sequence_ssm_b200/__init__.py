@@ -94,9 +94,9 @@ def _load():
     lib.m3_scan_fwd_static.restype = ctypes.c_int
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
     i64p = ctypes.POINTER(ctypes.c_int64)
-    lib.m3_scan_host_plan.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t), i64p, i64p, i64p, i64p]
+    lib.m3_scan_host_plan.argtypes = [dp, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t), i64p, i64p, i64p, i64p]
     lib.m3_scan_host_plan.restype = ctypes.c_int
-    lib.m3_scan_fwd_host.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_scan_fwd_host.argtypes = [dp, ctypes.POINTER(CBCNorm)] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     lib.m3_scan_fwd_host.restype = ctypes.c_int
     for f in (lib.m3_scan_workspace_size, lib.m3_scan_plan, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
         f.restype = ctypes.c_int
@@ -254,12 +254,12 @@ class HostPlan(NamedTuple):
     units: int              # (group, slice) units of one call
 
 
-def scan_host_plan(dims: Dims) -> HostPlan:
+def scan_host_plan(dims: Dims, bcnorm: bool = False) -> HostPlan:
     """How scan_fwd_host cuts a problem of these dims into pipelined units."""
     n = ctypes.c_size_t(0)
     ts, tl, gb, u = (ctypes.c_int64(0) for _ in range(4))
-    _check(get_lib().m3_scan_host_plan(ctypes.byref(dims), ctypes.byref(n), ctypes.byref(ts), ctypes.byref(tl),
-                                       ctypes.byref(gb), ctypes.byref(u)))
+    _check(get_lib().m3_scan_host_plan(ctypes.byref(dims), int(bool(bcnorm)), ctypes.byref(n), ctypes.byref(ts),
+                                       ctypes.byref(tl), ctypes.byref(gb), ctypes.byref(u)))
     return HostPlan(n.value, ts.value, tl.value, gb.value, u.value)
 
 
@@ -280,15 +280,21 @@ def _hstate(s: State | None):
 
 
 def scan_fwd_host(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
-                  y=None, final: State | None = None, workspace=None, stream=None):
+                  y=None, final: State | None = None, workspace=None, stream=None, bcnorm: BCNorm | None = None):
     """scan_fwd over host tensors (same shapes as scan_fwd; pinned memory lets
     the copies overlap): the library copies the inputs in, runs the scan and
     copies y (and the final state) back, pipelined over time slices, all
     ordered on `stream`.  `workspace` is a CUDA uint8 tensor of at least
     scan_host_plan(dims).workspace_bytes (allocated when None).  Returns
     (y, final State or None) as host tensors, complete once `stream` has
-    reached the end of the call."""
+    reached the end of the call.  `bcnorm` (host fp32 tensors) adds the
+    BC-norm prologue."""
     _require_host(x, B, C, dt, lam, theta, A, D, y)
+    cb = None
+    if bcnorm is not None:
+        _require_host(bcnorm.wB, bcnorm.wC, bcnorm.bB, bcnorm.bC)
+        cb = ctypes.byref(CBCNorm(bcnorm.wB.data_ptr(), bcnorm.wC.data_ptr(), bcnorm.bB.data_ptr(),
+                                  bcnorm.bC.data_ptr(), float(bcnorm.eps)))
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
     dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
@@ -298,10 +304,11 @@ def scan_fwd_host(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, w
         f = dict(dtype=torch.float32, pin_memory=True)
         final = State(torch.empty(Bt, H, N, P, **f), torch.empty(Bt, H, R, N, **f), torch.empty(Bt, H, R, P, **f))
     if workspace is None:
-        workspace = _scratch(max(scan_host_plan(dims).workspace_bytes, 1), torch.device("cuda"), stream)
+        workspace = _scratch(max(scan_host_plan(dims, bcnorm is not None).workspace_bytes, 1), torch.device("cuda"),
+                             stream)
     _require_cuda(workspace)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(get_lib().m3_scan_fwd_host(ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
+    _check(get_lib().m3_scan_fwd_host(ctypes.byref(dims), cb, *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
                                       _hstate(init), _ptr(y), _hstate(final), _ptr(workspace), ws_bytes,
                                       _stream(stream)))
     return y, final

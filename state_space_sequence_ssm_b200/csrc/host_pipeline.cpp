@@ -77,6 +77,7 @@ struct Layout {
     int64_t slice, group, nslice, ngroup;
     int64_t slice_last, nslice_last;    // the last group's slicing (finer: a short pipeline tail)
     size_t A, D, theta;                 // per-head constants (theta only when fixed per head)
+    size_t wB, wC, bB, bC;              // BC-norm parameters (when the call has them)
     size_t st[3][3];                    // state sets (initial, ping, pong) x (h, b_prev, x_prev)
     size_t slot[2][8];                  // x, B, C, dt, lam, theta, A, y of each slot
     size_t ws, ws_bytes;                // the scan's own workspace and its size
@@ -100,7 +101,7 @@ Rows token_rows(const m3_dims *d) {
     return r;
 }
 
-m3_status plan_layout(const m3_dims *d, Layout *L) {
+m3_status plan_layout(const m3_dims *d, bool bcn, Layout *L) {
     const int64_t T = d->seqlen, Bt = d->batch;
     // Whole sequences first (their copies are contiguous: measured 1 % faster
     // than time slices of the full batch), time slices only for the rest.
@@ -132,6 +133,10 @@ m3_status plan_layout(const m3_dims *d, Layout *L) {
     L->A = (d->flags & M3_FLAG_A_PER_TOKEN) ? 0 : take(H * 4);
     L->D = take(H * 4);
     L->theta = (d->flags & M3_FLAG_THETA_PER_HEAD) ? take(H * (N / 2) * es) : 0;
+    L->wB = bcn ? take(N * 4) : 0;
+    L->wC = bcn ? take(N * 4) : 0;
+    L->bB = bcn ? take(H * R * N * 4) : 0;
+    L->bC = bcn ? take(H * R * N * 4) : 0;
     const size_t gh = (size_t)L->group * H;
     for (int s = 0; s < 3; ++s) {
         L->st[s][0] = take(gh * N * P * 4);
@@ -196,13 +201,13 @@ cudaError_t copy_tokens(char *dev, const char *host_in, char *host_out, size_t r
     return cudaSuccess;
 }
 
-m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
-                    const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
-                    void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream) {
+m3_status host_impl(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B, const void *C,
+                    const void *dt, const void *lam, const void *theta, const float *A, const float *D,
+                    const m3_state *init, void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream) {
     Layout L{};
     m3_status st = m3_scan_plan(M3_ALGO_AUTO, d, nullptr, nullptr, nullptr);  // validates dims
     if (st != M3_OK) return st;
-    if ((st = plan_layout(d, &L)) != M3_OK) return st;
+    if ((st = plan_layout(d, bcn != nullptr, &L)) != M3_OK) return st;
     const int64_t Bt = d->batch, T = d->seqlen, H = d->nheads;
     const int64_t N = d->dstate, P = d->headdim, R = d->rank;
     const size_t es = d->io == M3_BF16 ? 2 : 4;
@@ -214,6 +219,9 @@ m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *
     if (tok > 0 && (!x || !B || !C || !dt || !lam || !theta || !y))
         return m3::set_error(M3_ERR_INVALID_ARG, "x, B, C, dt, lam, theta and y are required");
     if (!A || !D) return m3::set_error(M3_ERR_INVALID_ARG, "A and D are required");
+    if (bcn && (!bcn->wB || !bcn->wC || !bcn->bB || !bcn->bC))
+        return m3::set_error(M3_ERR_INVALID_ARG, "bcn: wB, wC, bB and bC are all required");
+    if (bcn && !(bcn->eps > 0.f)) return m3::set_error(M3_ERR_INVALID_ARG, "bcn eps must be > 0");
     const Rows rows = token_rows(d);
     const Span ins[8] = {span(x, tok / H * rows.b[0]), span(B, tok / H * rows.b[1]), span(C, tok / H * rows.b[2]),
                          span(dt, tok / H * rows.b[3]), span(lam, tok / H * rows.b[4]),
@@ -281,6 +289,17 @@ m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *
     if (th_head)
         M3_TRY(cudaMemcpyAsync(w + L.theta, theta, H * (N / 2) * es, cudaMemcpyHostToDevice, S->in),
                "m3_scan_fwd_host (theta)");
+    m3_bcnorm dbcn{};  // the BC-norm parameters' device copies
+    if (bcn) {
+        const size_t nb = (size_t)N * 4, hb = (size_t)H * R * N * 4;
+        M3_TRY(cudaMemcpyAsync(w + L.wB, bcn->wB, nb, cudaMemcpyHostToDevice, S->in), "m3_scan_fwd_host (bcn)");
+        M3_TRY(cudaMemcpyAsync(w + L.wC, bcn->wC, nb, cudaMemcpyHostToDevice, S->in), "m3_scan_fwd_host (bcn)");
+        M3_TRY(cudaMemcpyAsync(w + L.bB, bcn->bB, hb, cudaMemcpyHostToDevice, S->in), "m3_scan_fwd_host (bcn)");
+        M3_TRY(cudaMemcpyAsync(w + L.bC, bcn->bC, hb, cudaMemcpyHostToDevice, S->in), "m3_scan_fwd_host (bcn)");
+        dbcn = m3_bcnorm{reinterpret_cast<const float *>(w + L.wB), reinterpret_cast<const float *>(w + L.wC),
+                         reinterpret_cast<const float *>(w + L.bB), reinterpret_cast<const float *>(w + L.bC),
+                         bcn->eps};
+    }
     const void *hin[8] = {x, B, C, dt, lam, theta, A, nullptr};
     int64_t k = 0;
     for (int64_t g = 0; g < L.ngroup; ++g) {
@@ -325,11 +344,16 @@ m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *
             m3_state sout{reinterpret_cast<float *>(w + L.st[pout][0]), reinterpret_cast<float *>(w + L.st[pout][1]),
                           reinterpret_cast<float *>(w + L.st[pout][2])};
             const bool zero_init = i == 0 && !init;
-            st = m3_scan_fwd(&u, w + L.slot[j][0], w + L.slot[j][1], w + L.slot[j][2], w + L.slot[j][3],
-                             w + L.slot[j][4], th_head ? w + L.theta : w + L.slot[j][5],
-                             reinterpret_cast<const float *>(a_tok ? w + L.slot[j][6] : w + L.A),
-                             reinterpret_cast<const float *>(w + L.D), zero_init ? nullptr : &sin, w + L.slot[j][7],
-                             &sout, w + L.ws, L.ws_bytes, cs);
+            const void *uth = th_head ? w + L.theta : w + L.slot[j][5];
+            const float *uA = reinterpret_cast<const float *>(a_tok ? w + L.slot[j][6] : w + L.A);
+            const float *uD = reinterpret_cast<const float *>(w + L.D);
+            st = bcn ? m3_scan_fwd_bcnorm(M3_ALGO_AUTO, &u, &dbcn, w + L.slot[j][0], w + L.slot[j][1],
+                                          w + L.slot[j][2], w + L.slot[j][3], w + L.slot[j][4], uth, uA, uD,
+                                          zero_init ? nullptr : &sin, w + L.slot[j][7], &sout, w + L.ws,
+                                          L.ws_bytes, cs)
+                     : m3_scan_fwd(&u, w + L.slot[j][0], w + L.slot[j][1], w + L.slot[j][2], w + L.slot[j][3],
+                                   w + L.slot[j][4], uth, uA, uD, zero_init ? nullptr : &sin, w + L.slot[j][7],
+                                   &sout, w + L.ws, L.ws_bytes, cs);
             if (st != M3_OK) return st;
             M3_TRY(cudaEventRecord(S->computed[j], cs), "m3_scan_fwd_host (compute)");
 
@@ -360,13 +384,13 @@ m3_status host_impl(const m3_dims *d, const void *x, const void *B, const void *
 
 extern "C" {
 
-m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *slice_tokens,
+m3_status m3_scan_host_plan(const m3_dims *d, int with_bcnorm, size_t *workspace_bytes, int64_t *slice_tokens,
                             int64_t *last_slice_tokens, int64_t *group_batch, int64_t *units) {
     try {
         m3_status st = m3_scan_plan(M3_ALGO_AUTO, d, nullptr, nullptr, nullptr);
         if (st != M3_OK) return st;
         Layout L{};
-        if ((st = plan_layout(d, &L)) != M3_OK) return st;
+        if ((st = plan_layout(d, with_bcnorm != 0, &L)) != M3_OK) return st;
         if (workspace_bytes) *workspace_bytes = d->batch > 0 ? L.total : 0;
         if (slice_tokens) *slice_tokens = L.slice;
         if (last_slice_tokens) *last_slice_tokens = L.slice_last;
@@ -378,12 +402,12 @@ m3_status m3_scan_host_plan(const m3_dims *d, size_t *workspace_bytes, int64_t *
     }
 }
 
-m3_status m3_scan_fwd_host(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
-                           const void *lam, const void *theta, const float *A, const float *D,
+m3_status m3_scan_fwd_host(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B, const void *C,
+                           const void *dt, const void *lam, const void *theta, const float *A, const float *D,
                            const m3_state *init, void *y, const m3_state *final_state, void *workspace,
                            size_t workspace_bytes, void *stream) {
     try {
-        return host_impl(d, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace, workspace_bytes,
+        return host_impl(d, bcn, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace, workspace_bytes,
                          stream);
     } catch (...) {
         return m3::set_error(M3_ERR_INVALID_ARG, "internal error");

@@ -170,7 +170,7 @@ def test_host_plan_units_and_staging(m3, Bt, T, H, P, N, R, io, flags):
     d = dims(m3, Bt=Bt, T=T, H=H, P=P, N=N, R=R, io=io, flags=flags)
     ws = ctypes.c_size_t(0)
     ts, tl, gb, u = (ctypes.c_int64(0) for _ in range(4))
-    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), ctypes.byref(ts), ctypes.byref(tl),
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), 0, ctypes.byref(ws), ctypes.byref(ts), ctypes.byref(tl),
                                     ctypes.byref(gb), ctypes.byref(u)) == 0
     ts, tl, gb, u = ts.value, tl.value, gb.value, u.value
     for s in (ts, tl):
@@ -197,12 +197,18 @@ def test_host_plan_units_and_staging(m3, Bt, T, H, P, N, R, io, flags):
 def test_host_plan_empty_batch_and_bad_dims(m3):
     ws = ctypes.c_size_t(7)
     d = dims(m3, Bt=0, T=500)
-    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), ctypes.byref(ws), None, None, None, None) == 0
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), 0, ctypes.byref(ws), None, None, None, None) == 0
     assert ws.value == 0
     bad = dims(m3, N=7)
-    assert m3.lib.m3_scan_host_plan(ctypes.byref(bad), None, None, None, None, None) == 1
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(bad), 0, None, None, None, None, None) == 1
+    # the BC-norm parameters take room in the staging area
+    d = dims(m3, Bt=2, T=300, H=2, P=8, N=8, R=2)
+    w0, w1 = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), 0, ctypes.byref(w0), None, None, None, None) == 0
+    assert m3.lib.m3_scan_host_plan(ctypes.byref(d), 1, ctypes.byref(w1), None, None, None, None) == 0
+    assert w1.value >= w0.value + 2 * 8 * 4 + 2 * 2 * 2 * 8 * 4
     # the host entry point validates before touching the device
-    assert m3.lib.m3_scan_fwd_host(None, *([None] * 8), None, None, None, None, 0, None) == 1
+    assert m3.lib.m3_scan_fwd_host(None, None, *([None] * 8), None, None, None, None, 0, None) == 1
 
 
 def test_library_has_no_unresolved_internal_symbols(m3):

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle
-from m3_inputs import Shape, make_prefill, make_state
+from m3_inputs import Shape, make_bcnorm, make_prefill, make_state
 from m3_testutil import KEYS, host64, max_rel_l2_state, max_rel_l2_y, tol_for
 
 pytestmark = pytest.mark.gpu
@@ -34,7 +34,7 @@ def dims_of(shape, a_tok=False, th_head=False):
                         shape.torch_io, a_per_token=a_tok, theta_per_head=th_head)
 
 
-def by_units(inp, init, plan, shape):
+def by_units(inp, init, plan, shape, bcnorm=None):
     """The plan's units run one at a time on device tensors: each slice
     resumes from the previous slice's final state."""
     Bt, T = shape.batch, shape.seqlen
@@ -49,7 +49,7 @@ def by_units(inp, init, plan, shape):
         for t0 in range(0, max(T, 1), max(sl, 1)):
             t1 = min(T, t0 + sl)
             args = [(inp[k][b0:b1, t0:t1] if k in per_tok else inp[k]).contiguous().cuda() for k in KEYS]
-            ys, st = m3.scan_fwd(*args, st)
+            ys, st = m3.scan_fwd(*args, st, bcnorm=bcnorm)
             y[b0:b1, t0:t1] = ys.cpu()
         for f, s in zip(fin, st):
             f[b0:b1] = s.cpu()
@@ -91,6 +91,31 @@ def test_host_scan_matches_oracle_and_units(shape, a_tok, th_head, with_init):
     assert torch.equal(y, yu)
     for a, b in zip(fin, fu):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("shape", [Shape(3, 700, 2, 64, 128, 1, "bf16", 320), Shape(2, 300, 2, 64, 64, 4, "bf16", 321)],
+                         ids=lambda s: f"b{s.batch}t{s.seqlen}n{s.dstate}r{s.rank}")
+def test_host_scan_bcnorm(shape):
+    """The BC-norm prologue from host parameters: parity with the oracle and
+    the same bits as the units run one by one with device parameters."""
+    inp = pinned(make_prefill(shape))
+    init = host_state(shape)
+    p = make_bcnorm(shape)
+    hb = m3.BCNorm(p["wB"], p["wC"], p["bB"], p["bC"], p["eps"])
+    y, fin = m3.scan_fwd_host(*(inp[k] for k in KEYS), init, bcnorm=hb)
+    torch.cuda.synchronize()
+    m3.stream_status()
+    ref = oracle.BCNorm(*(host64(p[k]) for k in ("wB", "wC", "bB", "bC")), p["eps"])
+    yr, sr = oracle.scan(*(host64(inp[k]) for k in KEYS), oracle.State(*(host64(t) for t in init)), bcnorm=ref)
+    tol = tol_for(shape.io)
+    ey, eh = max_rel_l2_y(host64(y), yr), max_rel_l2_state(host64(fin.h), sr.h)
+    assert ey < tol and eh < tol, f"y {ey:.3e} state {eh:.3e}"
+    plan = m3.scan_host_plan(dims_of(shape), bcnorm=True)
+    db = m3.BCNorm(*(t.cuda() for t in (p["wB"], p["wC"], p["bB"], p["bC"])), p["eps"])
+    yu, fu = by_units(inp, init, plan, shape, bcnorm=db)
+    assert torch.equal(y, yu)
+    for a, c in zip(fin, fu):
+        assert torch.equal(a, c)
 
 
 def test_host_scan_agrees_with_device_scan():
