@@ -241,7 +241,12 @@ M3_API m3_status m3_scan_host_plan(const m3_dims *d, int with_bcnorm, size_t *wo
  * memory of at least m3_scan_host_plan's size, 16-byte aligned.  The result
  * is the scan of the whole sequence, as m3_scan_fwd computes it (as
  * m3_scan_fwd_bcnorm when `bcn` is non-NULL: its four arrays are then host
- * memory too, copied to the device once per call).
+ * memory too, copied to the device once per call).  The pages have no
+ * counterpart to this entry point: it is the end-to-end call for data that
+ * starts and ends in host memory.  Errors: M3_ERR_INVALID_ARG for missing or
+ * overlapping host buffers or a small or misaligned workspace (nothing is
+ * queued then), the scan's own errors for its units, M3_ERR_CUDA for a failed
+ * copy, event or stream call.
  *   - Pipelining: the call cuts the problem into (group of sequences) x
  *     (time slice) units and chains the slices of a group through the
  *     recurrent state (each slice resumes from the state the previous one
