@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -134,16 +135,17 @@ class ClockSampler:
         self.path = None
 
     def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="m3_clocks_", suffix=".csv")
+        self.fh = os.fdopen(fd, "w")
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
-            self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
             self.proc = None
+            self.fh.close()
+            os.unlink(self.path)
 
     def stop(self):
         if self.proc is None:
@@ -155,7 +157,16 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
+        with open(self.path) as f:
+            text = f.read()
+        os.unlink(self.path)
+        return self.summarise(text)
+
+    @staticmethod
+    def summarise(text):
+        """Median SM clock under load, max clock, throttle reasons seen and
+        peak power from the sampled CSV rows (None if there are none)."""
+        rows = [l.split(",") for l in text.strip().splitlines() if l.strip()]
         rows = [[c.strip() for c in r] for r in rows if len(r) >= 10]
         if not rows:
             return None

@@ -264,3 +264,21 @@ def _undefined_names(path):
 def test_bench_has_no_undefined_names():
     """bench.py's GPU legs cannot run here; at least every name they load is bound."""
     assert _undefined_names(os.path.join(ROOT, "bench.py")) == set()
+
+
+def test_bench_clock_summary():
+    """The bench's clock record: median SM clock of the loaded samples, the
+    throttle reasons any sample showed, and no reasons when none was active."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    row = "0, GPU-x, {sm}, 1965, {pw}, 0x0, Not Active, Not Active, Not Active, {cap}"
+    text = "\n".join([row.format(sm=1965, pw=600, cap="Not Active"), row.format(sm=1950, pw=900, cap="Active"),
+                      row.format(sm=1965, pw=950, cap="Not Active"), row.format(sm=210, pw=80, cap="Not Active")])
+    s = bench.ClockSampler.summarise(text)
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965 and s["samples"] == 4
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_max"] == 950
+    quiet = bench.ClockSampler.summarise(row.format(sm=1965, pw=500, cap="Not Active"))
+    assert quiet["reasons"] == []
+    assert bench.ClockSampler.summarise("") is None
