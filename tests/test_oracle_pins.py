@@ -586,3 +586,33 @@ def test_bcnorm_decode_continues_the_scan():
         yt, fs = oracle.step(*args, d["A"], d["D"], fs, bcnorm=bcn)
         ys.append(yt)
     assert rel(np.stack(ys, 1), y_full[:, k:]) < TOL and rel(fs.h, f_full.h) < TOL
+
+
+def test_bcnorm_eps_inside_the_root_with_both_options():
+    """With eps comparable to the rows' mean square, the prologue is
+    B / sqrt(mean_n B^2 + eps) * w + b (eps inside the root, as the header
+    states), written out here in numpy; checked with per-token A and angle
+    rates fixed per head at the same time."""
+    from m3_inputs import make_bcnorm
+    s = Shape(2, 19, 2, 5, 8, 2, "f32", 15)
+    d = {k: v.double().numpy() for k, v in make_prefill(s, a_per_token=True, theta_per_head=True).items()}
+    assert d["A"].shape == (2, 19, 2) and d["theta"].shape == (2, 4)
+    bn = {k: (v.double().numpy() if hasattr(v, "double") else v) for k, v in make_bcnorm(s).items()}
+    eps = 0.3  # the rows' mean square is about 1/N = 0.125
+    bcn = oracle.BCNorm(bn["wB"], bn["wC"], bn["bB"], bn["bC"], eps)
+    st = oracle.State(*(t.double().numpy() for t in make_state(s)))
+    y1, f1 = run_bcn(d, bcn, st)
+
+    def norm(a, w, b):
+        return a / np.sqrt(np.mean(a * a, axis=-1, keepdims=True) + eps) * w + b[None, None]
+
+    d2 = dict(d)
+    d2["B"], d2["C"] = norm(d["B"], bn["wB"], bn["bB"]), norm(d["C"], bn["wC"], bn["bC"])
+    y2, f2 = run(d2, st)
+    assert rel(y1, y2) < 1e-12 and rel(f1.h, f2.h) < 1e-12 and rel(f1.b_prev, f2.b_prev) < 1e-12
+    # and eps does matter at this size: outside the root it gives another answer
+    d3 = dict(d)
+    d3["B"] = d["B"] / (np.sqrt(np.mean(d["B"] ** 2, axis=-1, keepdims=True)) + eps) * bn["wB"] + bn["bB"][None, None]
+    d3["C"] = d["C"] / (np.sqrt(np.mean(d["C"] ** 2, axis=-1, keepdims=True)) + eps) * bn["wC"] + bn["bC"][None, None]
+    y3, _ = run(d3, st)
+    assert rel(y3, y1) > 1e-3
