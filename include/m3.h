@@ -276,11 +276,16 @@ M3_API m3_status m3_scan_fwd_host(const m3_dims *d, const m3_bcnorm *bcn,
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /* Decode: one token per (batch, head) against a resident state, updated in
- * place (the recurrent form of the same method, one token at a time).
+ * place -- the three-term recurrence of "Знакомство с Mamba-3", section 1,
+ * applied to a single token: h += beta' b_prev x_prev^T, h <- a Rot(-dt theta) h,
+ * h += gamma B x^T, y = h^T C + D x, then b_prev <- B, x_prev <- x.
  * x [batch,nheads,rank,headdim], B/C [batch,nheads,rank,dstate],
  * dt/lam [batch,nheads], theta [batch,nheads,dstate/2] (io dtype);
  * y [batch,nheads,rank,headdim] (io).  `state` buffers are read and written
- * once each; y must not overlap anything else. */
+ * once each; y must not overlap anything else.  Errors: M3_ERR_INVALID_ARG
+ * (null, misaligned or overlapping buffers, bad dims), M3_ERR_UNSUPPORTED
+ * (sizes outside the compiled set), M3_ERR_CUDA (launch failure); nothing
+ * is queued on an error. */
 M3_API m3_status m3_step(const m3_dims *d,
                   const void *x, const void *B, const void *C,
                   const void *dt, const void *lam, const void *theta,
