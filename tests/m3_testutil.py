@@ -69,3 +69,23 @@ def oracle_scan_slices(inp: dict, bh_list, init=None):
 
 def rel_l2(a: np.ndarray, ref: np.ndarray) -> float:
     return float(np.linalg.norm(a - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+def max_rel_l2_step(y: np.ndarray, yref: np.ndarray) -> float:
+    """One decode step, y, yref [Bt, H, R, P]: per (b,h) slice relative L2
+    over (r, p), max over slices (the same metric as the prefill's)."""
+    if y.size == 0:
+        return 0.0
+    d = (y - yref).reshape(y.shape[0] * y.shape[1], -1)
+    r = yref.reshape(d.shape)
+    return float(np.max(np.linalg.norm(d, axis=1) / np.maximum(np.linalg.norm(r, axis=1), 1e-30)))
+
+
+# Worst per-slice errors of the parity tests that record them, printed at the
+# end of the session (tests/conftest.py), so the margin against the bar is on
+# record in every run's output: (test, worst error, bar).
+MARGINS: list = []
+
+
+def record_margin(name: str, err: float, tol: float):
+    MARGINS.append((name, float(err), float(tol)))

@@ -6,7 +6,7 @@ import torch
 
 import oracle
 from m3_inputs import WORKLOADS, Shape, make_prefill, make_state, make_steps
-from m3_testutil import (KEYS, TOL_BF16, host64, max_rel_l2_state, max_rel_l2_y, oracle_scan_slices, rel_l2,
+from m3_testutil import (max_rel_l2_step, KEYS, TOL_BF16, host64, max_rel_l2_state, max_rel_l2_y, oracle_scan_slices, rel_l2,
                          tol_for)
 
 pytestmark = pytest.mark.gpu
@@ -82,7 +82,7 @@ def test_decode_a_per_token(shape):
     for i in range(6):
         args = [host64(steps[k][i]) for k in ("x", "B", "C", "dt", "lam", "theta")]
         yo, ost = oracle.step(*args, host64(steps["A"][i]), host64(pre["D"]), ost)
-        assert rel_l2(host64(ys[i]), yo) < tol, f"step {i}"
+        assert max_rel_l2_step(host64(ys[i]), yo) < tol, f"step {i} (worst slice)"
     assert max_rel_l2_state(host64(st.h), ost.h) < tol
 
 

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from m3_inputs import WORKLOADS, Shape, make_bcnorm, make_prefill, make_state, make_steps
-from m3_testutil import KEYS, TOL_BF16, host64, max_rel_l2_state, max_rel_l2_y, rel_l2, tol_for
+from m3_testutil import max_rel_l2_step, KEYS, TOL_BF16, host64, max_rel_l2_state, max_rel_l2_y, rel_l2, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -80,7 +80,7 @@ def test_decode_bcnorm(shape):
     for i in range(5):
         args = [host64(steps[k][i]) for k in ("x", "B", "C", "dt", "lam", "theta")]
         yo, ost = oracle.step(*args, host64(pre["A"]), host64(pre["D"]), ost, bcnorm=bref)
-        assert rel_l2(host64(ys[i]), yo) < tol, f"step {i}"
+        assert max_rel_l2_step(host64(ys[i]), yo) < tol, f"step {i} (worst slice)"
     assert max_rel_l2_state(host64(st.h), ost.h) < tol
     assert max_rel_l2_state(host64(st.b_prev), ost.b_prev) < 1e-5
 
