@@ -12,6 +12,15 @@ the (batch, head) slices are independent, there is no collective on the data
 path); time is the max over ranks of CUDA-event time.  Rank 0 prints one JSON
 line.  `--impl reference` times the fp64 CPU oracle on bounded samples of the
 same workload instead (rank 0 only).
+
+Besides the headline the line carries `configs`: every workload the method is
+measured on, each timed on its own with CUDA events and its own roofline --
+the small fp32 scan (batch 1, T=256, 4 heads, P=N=64; smaller than L2, so
+L2 is flushed between calls), the SISO prefill (the headline itself), the
+MIMO rank-4 prefill (batch 8, T=4096, 32 heads, N=64), the batch-256 decode
+steps (rank 1 and rank 4, 1000 graph-captured steps from a 1024-token
+prefill) and the long-context MIMO prefill (batch 1, T=65536, 64 heads,
+N=128, R=4) followed by 256 decode steps of its own sequences.
 """
 from __future__ import annotations
 
@@ -32,6 +41,10 @@ sys.path.insert(0, ROOT)
 METRIC = "Mamba-3 SSM tokens/s (prefill scan, decode step) and % of roofline, 1 B200"
 PREFILL_WORKLOAD = "siso_bf16_b8_t4096_h32_p64_n128"
 DECODE_WORKLOADS = ["decode_bf16_b256_h32_p64_n128_r1", "decode_bf16_b256_h32_p64_n128_r4"]
+# the five workloads the method is measured on, in order (the decode entry
+# stands for both ranks of DECODE_WORKLOADS)
+CONFIG_WORKLOADS = ["siso_f32_b1_t256_h4_p64_n64", PREFILL_WORKLOAD, "mimo_bf16_b8_t4096_h32_p64_n64_r4",
+                    DECODE_WORKLOADS[0], "long_mimo_bf16_b1_t65536_h64_p64_n128_r4"]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -50,6 +63,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the variant lines (per-token A, per-head theta, BC-norm) of the prefill workload")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' lines (small fp32 scan, MIMO, decode, long context)")
     ap.add_argument("--case", choices=["prefill", "decode"], default=None,
                     help="profiling case: only run --case-launches launches of one kernel at --case-batch "
                          "(for ncu captures; prints no bench line)")
@@ -234,6 +249,17 @@ def replica_shape(name, rank):
     return WORKLOADS[name].with_(seed=WORKLOADS[name].seed + rank)
 
 
+def workload_config(name, s, world):
+    """The `config` of the JSON line: the workload by name and sizes, the same
+    dict in both arms."""
+    ab = prefill_bytes(s)
+    return {"workload": name, "batch": s.batch, "seq_len": s.seqlen, "nheads": s.nheads, "headdim": s.headdim,
+            "dstate": s.dstate, "rank": s.rank, "io": s.io, "global_batch": world * s.batch,
+            "parallelism": f"replicas x{world} (no collective)",
+            "l2": (f"inputs larger than L2 ({ab / 1e6:.0f} MB per step), no flush" if ab > (200 << 20) else
+                   f"inputs ({ab / 1e6:.1f} MB) smaller than L2")}
+
+
 def job_tokens_per_s(world, steps, shape, elapsed_s):
     """Whole-job throughput: tokens of all ranks over the max-over-ranks time."""
     return world * steps * shape.batch * shape.seqlen / elapsed_s
@@ -266,9 +292,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "batch": s.batch, "seq_len": s.seqlen,
-                                            "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
-                                            "rank": s.rank, "io": s.io},
+            "data": "synthetic", "config": workload_config(args.workload, s, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{nslices} (batch, head) slices x {s.seqlen} tokens per step, "
                                        f"scaled to tokens of all {s.nheads} heads"},
@@ -277,12 +301,81 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our arm
+def time_prefill(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys, stream,
+                 algo, steps, flush_l2=False):
+    """Time `steps` prefill calls of workload `name` (inputs resident in HBM)
+    with CUDA events on the launching stream: the whole timed region (max
+    over ranks) and each call alone (mean, for the roofline).  With flush_l2
+    (inputs smaller than L2) a 256 MiB buffer is written between calls,
+    outside the per-call events.  Returns the entry, the state after the last
+    call and the workload's (A, D)."""
+    import torch
+    from m3_inputs import make_prefill
+
+    s = replica_shape(name, rank)
+    inp = make_prefill(s, device=dev)
+    dims = m3.make_dims(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.rank, s.torch_io)
+    info = m3.scan_plan_info(dims, algo)
+    kernel = info.kernel_name
+    y = torch.empty_like(inp["x"])
+    fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device=dev)
+    ws = torch.empty(max(info.workspace_bytes, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
+
+    def call():
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, workspace=ws, algo=algo, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(i & 0xff)
+        ev[2 * i].record(stream)
+        call()
+        ev[2 * i + 1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    m3.stream_status(stream)
+    elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    launch = statistics.mean(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)) / 1e3
+    abytes = prefill_bytes(s)
+    achieved = abytes / launch / 1e9
+    per_call = max_over_ranks(launch) if flush_l2 else elapsed / steps
+    entry = {"workload": name, "kind": "prefill", "value": world * s.batch * s.seqlen / per_call,
+             "unit": "tokens/s", "steps": steps, "ms_per_step": 1e3 * per_call,
+             "gpu_launches": steps * info.launches, "dtype": "bf16" if s.io == "bf16" else "f32",
+             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                          "frac": achieved / hbm_peak, "traffic": recorded_traffic(kernel, name),
+                          "kernel": kernel, "algorithmic_bytes_per_launch": abytes, "launch_ms": launch * 1e3,
+                          "peak_source": peak_src},
+             "schedule": {"balanced": info.balanced, "ctas": info.ctas, "segments_per_sequence": info.segments,
+                          "kernel_launches_per_call": info.launches}}
+    if info.launches > 1:
+        entry["roofline"]["note"] = ("sequences split into segments: summary pass, segment scan and main pass; "
+                                     "launch_ms and achieved cover the whole call")
+    if flush_l2:
+        entry["l2"] = f"inputs ({abytes / 1e6:.1f} MB) smaller than L2: 256 MiB written between calls, " \
+                      "value from the per-call events"
+    else:
+        entry["l2"] = f"inputs larger than L2 ({abytes / 1e6:.0f} MB per step), no flush"
+    AD = (inp["A"], inp["D"])
+    del inp, y, ws, flush
+    return entry, fin, AD
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
     import state_space_sequence_ssm_b200 as m3
-    from m3_inputs import WORKLOADS, make_prefill, make_steps
+    from m3_inputs import WORKLOADS, make_prefill
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -300,13 +393,12 @@ def run_ours(args):
     s = replica_shape(args.workload, rank)
     inp = make_prefill(s, device=dev)
     dims = m3.make_dims(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.rank, s.torch_io)
-    use_tc = algo != m3.ALGO_SIMT and m3.workspace_size(dims) >= 0 and _tc_supported(m3, inp, keys, algo)
-    kernel = "prefill_tc_kernel" if use_tc else "prefill_simt_kernel"
+    info = m3.scan_plan_info(dims, algo)
+    kernel = info.kernel_name
+    use_tc = info.kernel == m3.KERNEL_TC
     y = torch.empty_like(inp["x"])
     fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device=dev)
-    plan = m3.scan_plan(dims, algo)
-    wsn = plan.workspace_bytes if use_tc else 0
-    ws = torch.empty(max(wsn, 1), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(info.workspace_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def prefill():
@@ -334,6 +426,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
+    m3.stream_status(stream)
     elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     launch = statistics.mean(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)) / 1e3
     value = job_tokens_per_s(world, K, s, elapsed)
@@ -343,17 +436,15 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if use_tc else "f32",
             "data": "synthetic",
-            "config": {"workload": args.workload, "batch": s.batch, "seq_len": s.seqlen, "nheads": s.nheads,
-                       "headdim": s.headdim, "dstate": s.dstate, "rank": s.rank, "io": s.io,
-                       "global_batch": world * s.batch, "parallelism": f"replicas x{world} (no collective)",
-                       "l2": f"inputs larger than L2 ({abytes / 1e6:.0f} MB per step), no flush"},
+            "config": workload_config(args.workload, s, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": recorded_traffic(kernel, args.workload),
                          "kernel": kernel, "algorithmic_bytes_per_launch": abytes,
                          "launch_ms": launch * 1e3, "peak_source": peak_src,
-                         "segments_per_sequence": plan.segments, "kernel_launches_per_call": plan.launches},
-            "gpu_launches": K * plan.launches, "clocks": clk}
-    if plan.launches > 1:
+                         "segments_per_sequence": info.segments, "kernel_launches_per_call": info.launches,
+                         "balanced_schedule": info.balanced, "ctas": info.ctas},
+            "gpu_launches": K * info.launches, "clocks": clk}
+    if info.launches > 1:
         line["roofline"]["note"] = ("sequences split into segments: summary pass, segment scan and main pass; "
                                     "launch_ms and achieved cover the whole call")
 
@@ -434,15 +525,45 @@ def run_ours(args):
                                     "group_batch": hplan.group_batch}}
         del host, yh, fh, hws
 
-    # ---- decode step: state from a 1024-token prefill, then single-token steps in one CUDA graph
     if not args.no_variants and use_tc:
         line["variants"] = [run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
                                         peak_src, keys, stream) for kind in VARIANTS]
-    if not args.no_decode:
-        del inp, y, fin
-        torch.cuda.empty_cache()
-        # the long-context workload continues its own sequences (its prefill's
-        # state, then 256 steps); every other line reports the batch-256 decode workloads
+    del inp, y, fin, ws
+    torch.cuda.empty_cache()
+
+    # ---- every workload the method is measured on, each timed on its own:
+    #      the small fp32 scan, the SISO prefill (the line above), the MIMO
+    #      prefill, the batch-256 decode steps and the long-context prefill
+    #      followed by 256 decode steps of its own sequences
+    if not args.no_configs and args.workload == PREFILL_WORKLOAD:
+        configs = []
+        for idx, name in enumerate(CONFIG_WORKLOADS):
+            if name == PREFILL_WORKLOAD:
+                configs.append({"config": idx, "workload": name, "kind": "prefill", "value": value,
+                                "unit": "tokens/s", "ms_per_step": line["ms_per_step"], "steps": K,
+                                "gpu_launches": line["gpu_launches"], "roofline": line["roofline"],
+                                "note": "the headline line itself"})
+            elif name.startswith("decode"):
+                if not args.no_decode:
+                    for dname in DECODE_WORKLOADS:
+                        e = run_decode(m3, dname, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
+                                       peak_src, keys)
+                        configs.append({"config": idx, **e})
+            else:
+                small = WORKLOADS[name].seqlen * WORKLOADS[name].batch * WORKLOADS[name].nheads < (1 << 20)
+                e, st, AD = time_prefill(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
+                                         peak_src, keys, stream, m3.ALGO_AUTO, K, flush_l2=small)
+                configs.append({"config": idx, **e})
+                if name.startswith("long") and not args.no_decode:
+                    e = run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src,
+                                   keys, state=st, AD=AD)
+                    configs.append({"config": idx, **e})
+                del st, AD
+                torch.cuda.empty_cache()
+        line["configs"] = configs
+    elif not args.no_decode:
+        # another --workload: the long-context one continues its own sequences
+        # (its prefill's state, then 256 steps); every other reports the batch-256 decode workloads
         names = [args.workload] if args.workload.startswith("long") else DECODE_WORKLOADS
         line["decode"] = [run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak,
                                      peak_src, keys) for name in names]
@@ -455,21 +576,6 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
-
-
-def _tc_supported(m3, inp, keys, algo):
-    if algo == m3.ALGO_SIMT:
-        return False
-    try:
-        import torch
-        sub = {k: (v[:1, :1].contiguous() if v.dim() >= 3 else v) for k, v in inp.items()}
-        m3.scan_fwd(*(sub[k] for k in keys), None, algo=m3.ALGO_TC)
-        torch.cuda.synchronize()
-        return True
-    except m3.M3Error as e:
-        if e.status == m3.M3_ERR_UNSUPPORTED:
-            return False
-        raise
 
 
 VARIANTS = {"a_per_token": "data-dependent A_t (M3_FLAG_A_PER_TOKEN)",
@@ -522,20 +628,30 @@ def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_p
                          "peak_source": peak_src}}
 
 
-def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys):
+def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys, state=None,
+               AD=None):
+    """Decode steps of workload `name`, all captured in one CUDA graph: from
+    the state of its own prefill (`state` with the prefill's (A, D) `AD`, or a
+    prefill run here), 256 steps for the long-context workload,
+    --decode-steps for the others."""
     import torch
-    from m3_inputs import LONG_DECODE_STEPS, WORKLOADS, make_prefill, make_steps
+    from m3_inputs import LONG_DECODE_STEPS, make_prefill, make_steps
 
     s = replica_shape(name, rank)
-    pre = make_prefill(s, device=dev)
-    _, st = m3.scan_fwd(*(pre[k] for k in keys), None)
-    A, D = pre["A"], pre["D"]
-    del pre
+    if state is None:
+        pre = make_prefill(s, device=dev)
+        _, st = m3.scan_fwd(*(pre[k] for k in keys), None)
+        A, D = pre["A"], pre["D"]
+        del pre
+    else:
+        st = state
+        A, D = AD
     torch.cuda.empty_cache()
     S = LONG_DECODE_STEPS if name.startswith("long") else args.decode_steps
     steps = make_steps(s, S, device=dev)
     y = torch.empty(s.batch, s.nheads, s.rank, s.headdim, dtype=s.torch_io, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
     sk = ("x", "B", "C", "dt", "lam", "theta")
     # warm-up launches (they advance the state, as real decode would)
     with torch.cuda.stream(stream):
@@ -558,21 +674,27 @@ def run_decode(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_pe
         e1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    m3.stream_status(stream)
     el = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     per = el / S
     ab = step_bytes(s)
-    # the library runs rank 1 (and P = 128 or N = 256) on the one-CTA-per-slice
-    # kernel and rank >= 2 with P = 64, N in {64, 128} on the persistent one
-    kernel = "step_stream_kernel" if (s.rank >= 2 and s.headdim == 64 and s.dstate in (64, 128)) else "step_kernel"
+    kernel = decode_kernel_name(s)
     ach = ab / per / 1e9
     del g, steps
     torch.cuda.empty_cache()
-    return {"workload": name, "value": world * s.batch / per, "unit": "tokens/s", "steps": S,
+    return {"workload": name, "kind": "decode", "value": world * s.batch / per, "unit": "tokens/s", "steps": S,
             "us_per_step": per * 1e6, "gpu_launches": S,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                          "frac": ach / hbm_peak, "traffic": recorded_traffic(kernel, name),
                          "kernel": kernel, "algorithmic_bytes_per_launch": ab,
                          "note": "per-step time includes graph launch gaps", "peak_source": peak_src}}
+
+
+def decode_kernel_name(s):
+    """The decode kernel the library runs for this shape: rank 1 (and P = 128
+    or N = 256) one CTA per slice, rank >= 2 with P = 64, N in {64, 128} the
+    persistent streaming kernel."""
+    return "step_stream_kernel" if (s.rank >= 2 and s.headdim == 64 and s.dstate in (64, 128)) else "step_kernel"
 
 
 def cpu_baseline(s, keys):

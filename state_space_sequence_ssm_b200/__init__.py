@@ -22,6 +22,8 @@ M3_F32, M3_BF16 = 0, 1
 M3_FLAG_A_PER_TOKEN = 1
 M3_FLAG_THETA_PER_HEAD = 2
 ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
+KERNEL_NONE, KERNEL_SIMT, KERNEL_TC = 0, 1, 2
+PLAN_STATIC, PLAN_NO_WORKSPACE = 1, 2
 
 
 def ALGO_TC_SEGMENTS(s: int) -> int:
@@ -53,8 +55,12 @@ class BCNorm(NamedTuple):
 
 
 def _cbcn(b: BCNorm):
-    _require_cuda(b.wB, b.wC, b.bB, b.bC)
     return ctypes.byref(CBCNorm(b.wB.data_ptr(), b.wC.data_ptr(), b.bB.data_ptr(), b.bC.data_ptr(), float(b.eps)))
+
+
+class CPlanInfo(ctypes.Structure):
+    _fields_ = [("workspace_bytes", ctypes.c_size_t), ("kernel", ctypes.c_int32), ("segments", ctypes.c_int32),
+                ("launches", ctypes.c_int32), ("balanced", ctypes.c_int32), ("ctas", ctypes.c_int64)]
 
 
 class CState(ctypes.Structure):
@@ -83,6 +89,8 @@ def _load():
     lib.m3_scan_workspace_size.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t)]
     lib.m3_scan_plan.argtypes = [ctypes.c_int, dp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_int),
                                  ctypes.POINTER(ctypes.c_int)]
+    lib.m3_scan_plan_info.argtypes = [ctypes.c_int, dp, ctypes.c_int, ctypes.POINTER(CPlanInfo)]
+    lib.m3_scan_plan_info.restype = ctypes.c_int
     lib.m3_scan_fwd.argtypes = [dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     lib.m3_scan_fwd_algo.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
     bp_ = ctypes.POINTER(CBCNorm)
@@ -136,19 +144,35 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, device=None):
+    """The call's stream as a cudaStream_t: `stream`, else the current stream
+    of `device` (the tensors' GPU).  A given stream must belong to `device`."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise ValueError(f"m3: stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _require_cuda(*ts):
+    """Check that every given tensor is a contiguous CUDA tensor and that they
+    all sit on one GPU; return that device (None if no tensor was given).
+
+    The C library launches on the CUDA runtime's current device, so each call
+    below runs with this device made current: pointers of a tensor on another
+    GPU never reach a kernel on this one."""
+    dev = None
     for t in ts:
         if t is not None:
             if not t.is_cuda:
                 raise ValueError("m3: tensors must be on a CUDA device (no CPU path)")
             if not t.is_contiguous():
                 raise ValueError("m3: tensors must be contiguous")
+            if dev is None:
+                dev = t.device
+            elif t.device != dev:
+                raise ValueError(f"m3: tensors on different devices ({dev} and {t.device})")
+    return dev
 
 
 def _scratch(nbytes: int, device, stream):
@@ -172,7 +196,6 @@ def make_dims(Bt, T, H, P, N, R, dtype, a_per_token: bool = False, theta_per_hea
 def _cstate(s: State | None):
     if s is None:
         return None
-    _require_cuda(*s)
     return ctypes.pointer(CState(s.h.data_ptr(), s.b_prev.data_ptr(), s.x_prev.data_ptr()))
 
 
@@ -199,6 +222,28 @@ def scan_plan(dims: Dims, algo: int = ALGO_AUTO) -> Plan:
     return Plan(n.value, sg.value, ln.value)
 
 
+class PlanInfo(NamedTuple):
+    workspace_bytes: int
+    kernel: int     # KERNEL_SIMT or KERNEL_TC (KERNEL_NONE: nothing to run)
+    segments: int   # per sequence (1 = not split)
+    launches: int   # kernel launches of one call
+    balanced: bool  # one CTA per SM over equal runs of chunks
+    ctas: int       # CTAs of the (main) launch
+
+    @property
+    def kernel_name(self) -> str:
+        return {KERNEL_NONE: "none", KERNEL_SIMT: "prefill_simt_kernel", KERNEL_TC: "prefill_tc_kernel"}[self.kernel]
+
+
+def scan_plan_info(dims: Dims, algo: int = ALGO_AUTO, flags: int = 0) -> PlanInfo:
+    """Which kernel and schedule one prefill call runs on the current device
+    (flags: PLAN_STATIC for scan_fwd_static, PLAN_NO_WORKSPACE for a call
+    without a workspace)."""
+    info = CPlanInfo()
+    _check(get_lib().m3_scan_plan_info(algo, ctypes.byref(dims), flags, ctypes.byref(info)))
+    return PlanInfo(info.workspace_bytes, info.kernel, info.segments, info.launches, bool(info.balanced), info.ctas)
+
+
 def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
              y=None, final: State | None = None, workspace=None, algo: int = ALGO_AUTO, stream=None,
              bcnorm: BCNorm | None = None):
@@ -206,25 +251,27 @@ def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_s
     theta [Bt,T,H,N/2] (or [H,N/2]: fixed per head) in one io dtype (fp32 or
     bf16); D [H] fp32; A [H] fp32, or [Bt,T,H] fp32 for a data-dependent A_t.
     Returns (y, final State or None)."""
-    _require_cuda(x, B, C, dt, lam, theta, A, D, y, workspace)
+    dev = _require_cuda(x, B, C, dt, lam, theta, A, D, y, workspace, *(init or ()), *(final or ()),
+                        *(bcnorm[:4] if bcnorm is not None else ()))
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
     dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
-    if y is None:
-        y = torch.empty_like(x)
-    if final is None and want_state:
-        final = State(torch.empty(Bt, H, N, P, device=x.device), torch.empty(Bt, H, R, N, device=x.device),
-                      torch.empty(Bt, H, R, P, device=x.device))
-    ws_need = workspace_size(dims, algo) if algo != ALGO_SIMT else 0
-    if workspace is None and ws_need:
-        workspace = _scratch(ws_need, x.device, stream)
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(init), _ptr(y), _cstate(final), _ptr(workspace),
-            ws_bytes, _stream(stream))
-    if bcnorm is None:
-        _check(get_lib().m3_scan_fwd_algo(algo, ctypes.byref(dims), *args))
-    else:
-        _check(get_lib().m3_scan_fwd_bcnorm(algo, ctypes.byref(dims), _cbcn(bcnorm), *args))
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty_like(x)
+        if final is None and want_state:
+            final = State(torch.empty(Bt, H, N, P, device=dev), torch.empty(Bt, H, R, N, device=dev),
+                          torch.empty(Bt, H, R, P, device=dev))
+        ws_need = workspace_size(dims, algo) if algo != ALGO_SIMT else 0
+        if workspace is None and ws_need:
+            workspace = _scratch(ws_need, dev, stream)
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(init), _ptr(y), _cstate(final),
+                _ptr(workspace), ws_bytes, _stream(stream, dev))
+        if bcnorm is None:
+            _check(get_lib().m3_scan_fwd_algo(algo, ctypes.byref(dims), *args))
+        else:
+            _check(get_lib().m3_scan_fwd_bcnorm(algo, ctypes.byref(dims), _cbcn(bcnorm), *args))
     return y, final
 
 
@@ -232,17 +279,18 @@ def scan_fwd_static(x, B, C, dt, lam, theta, A, D, init: State | None = None, *,
                     y=None, final: State | None = None, algo: int = ALGO_AUTO, stream=None):
     """scan_fwd without a workspace: split sequences use the library's own
     device scratch (see m3_scan_fwd_static in include/m3.h for its limits)."""
-    _require_cuda(x, B, C, dt, lam, theta, A, D, y)
+    dev = _require_cuda(x, B, C, dt, lam, theta, A, D, y, *(init or ()), *(final or ()))
     Bt, T, H, R, P = x.shape
     N = B.shape[-1]
     dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
-    if y is None:
-        y = torch.empty_like(x)
-    if final is None and want_state:
-        final = State(torch.empty(Bt, H, N, P, device=x.device), torch.empty(Bt, H, R, N, device=x.device),
-                      torch.empty(Bt, H, R, P, device=x.device))
-    _check(get_lib().m3_scan_fwd_static(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
-                                        _cstate(init), _ptr(y), _cstate(final), _stream(stream)))
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty_like(x)
+        if final is None and want_state:
+            final = State(torch.empty(Bt, H, N, P, device=dev), torch.empty(Bt, H, R, N, device=dev),
+                          torch.empty(Bt, H, R, P, device=dev))
+        _check(get_lib().m3_scan_fwd_static(algo, ctypes.byref(dims), *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
+                                            _cstate(init), _ptr(y), _cstate(final), _stream(stream, dev)))
     return y, final
 
 
@@ -303,41 +351,49 @@ def scan_fwd_host(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, w
     if final is None and want_state:
         f = dict(dtype=torch.float32, pin_memory=True)
         final = State(torch.empty(Bt, H, N, P, **f), torch.empty(Bt, H, R, N, **f), torch.empty(Bt, H, R, P, **f))
-    if workspace is None:
-        workspace = _scratch(max(scan_host_plan(dims, bcnorm is not None).workspace_bytes, 1), torch.device("cuda"),
-                             stream)
-    _require_cuda(workspace)
-    ws_bytes = workspace.numel() * workspace.element_size()
-    _check(get_lib().m3_scan_fwd_host(ctypes.byref(dims), cb, *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
-                                      _hstate(init), _ptr(y), _hstate(final), _ptr(workspace), ws_bytes,
-                                      _stream(stream)))
+    # the device: the workspace's, else the stream's, else the current one
+    dev = _require_cuda(workspace) or (stream.device if stream is not None else
+                                       torch.device("cuda", torch.cuda.current_device()))
+    with torch.cuda.device(dev):
+        if workspace is None:
+            workspace = _scratch(max(scan_host_plan(dims, bcnorm is not None).workspace_bytes, 1), dev, stream)
+        ws_bytes = workspace.numel() * workspace.element_size()
+        _check(get_lib().m3_scan_fwd_host(ctypes.byref(dims), cb, *map(_ptr, (x, B, C, dt, lam, theta, A, D)),
+                                          _hstate(init), _ptr(y), _hstate(final), _ptr(workspace), ws_bytes,
+                                          _stream(stream, dev)))
     return y, final
 
 
 def selftest_wait_timeout(stream=None):
     """Queue a kernel whose bounded device wait gives up; the next
     stream_status() on that stream raises M3Error(M3_ERR_TIMEOUT)."""
-    _check(get_lib().m3_selftest_wait_timeout(_stream(stream)))
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(get_lib().m3_selftest_wait_timeout(_stream(stream, dev)))
 
 
 def stream_status(stream=None):
-    """Synchronise the stream and raise if a kernel's bounded wait gave up."""
-    _check(get_lib().m3_stream_status(_stream(stream)))
+    """Synchronise the stream and raise if a kernel's bounded wait gave up
+    (on any stream of the stream's device since the previous check)."""
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(get_lib().m3_stream_status(_stream(stream, dev)))
 
 
 def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None, bcnorm: BCNorm | None = None):
     """One decode step in place on `state`.  x [Bt,H,R,P], B/C [Bt,H,R,N],
     dt/lam [Bt,H], theta [Bt,H,N/2] (or [H,N/2]: fixed per head); A [H] fp32,
     or [Bt,H] fp32 for a data-dependent A_t.  Returns y [Bt,H,R,P]."""
-    _require_cuda(x, B, C, dt, lam, theta, A, D, y)
+    dev = _require_cuda(x, B, C, dt, lam, theta, A, D, y, *state, *(bcnorm[:4] if bcnorm is not None else ()))
     Bt, H, R, P = x.shape
     N = B.shape[-1]
     dims = make_dims(Bt, 1, H, P, N, R, x.dtype, a_per_token=A.dim() == 2, theta_per_head=theta.dim() == 2)
-    if y is None:
-        y = torch.empty_like(x)
-    args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state), _ptr(y), _stream(stream))
-    if bcnorm is None:
-        _check(get_lib().m3_step(ctypes.byref(dims), *args))
-    else:
-        _check(get_lib().m3_step_bcnorm(ctypes.byref(dims), _cbcn(bcnorm), *args))
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty_like(x)
+        args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state), _ptr(y), _stream(stream, dev))
+        if bcnorm is None:
+            _check(get_lib().m3_step(ctypes.byref(dims), *args))
+        else:
+            _check(get_lib().m3_step_bcnorm(ctypes.byref(dims), _cbcn(bcnorm), *args))
     return y

@@ -219,9 +219,16 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
                 if (e != cudaSuccess) return cuda_fail(e, "m3_scan_fwd_static (scratch address)");
             }
         } else {
-            const size_t need = m3::prefill_tc_workspace(p);
+            size_t need = m3::prefill_tc_workspace(p);
+            if (need > ws_bytes || (need && !ws)) {
+                // without room for the balanced schedule's hand-off slots the
+                // call runs one CTA per sequence (which needs none)
+                p.no_balance = true;
+                need = m3::prefill_tc_workspace(p);
+            }
             if (need > ws_bytes || (need && !ws))
                 return fail(M3_ERR_INVALID_ARG, "workspace too small (query m3_scan_workspace_size)");
+            if (need && !aligned16(ws)) return fail(M3_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
         }
     }
     cudaError_t e = use_tc ? m3::launch_prefill_tc(p, &why) : m3::launch_prefill_simt(p, &why);
@@ -239,26 +246,25 @@ m3_status set_cuda_error(cudaError_t e, const char *where) { return cuda_fail(e,
 
 extern "C" {
 
-int m3_version(void) { return 100; }
+int m3_version(void) { return 101; }
 
 const char *m3_last_error(void) { return g_err.c_str(); }
 
-m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_bytes, int *segments, int *launches) {
+m3_status m3_scan_plan_info(int algo, const m3_dims *d, int flags, m3_plan_info *info) {
     try {
+        if (!info) return fail(M3_ERR_INVALID_ARG, "info is NULL");
         m3_status s = check_dims(d, false);
         if (s != M3_OK) return s;
+        if (flags & ~(M3_PLAN_STATIC | M3_PLAN_NO_WORKSPACE)) return fail(M3_ERR_INVALID_ARG, "unknown plan flags");
         const int forced = algo >> 8;
         const int base = algo & 0xff;
         if (base != M3_ALGO_AUTO && base != M3_ALGO_SIMT && base != M3_ALGO_TC)
             return fail(M3_ERR_INVALID_ARG, "unknown algo");
         if (forced < 0 || forced > kMaxForcedSegments || (forced && base != M3_ALGO_TC))
             return fail(M3_ERR_INVALID_ARG, "bad segment count in algo");
-        if (d->batch == 0) {  // nothing to run, whichever kernel was asked for
-            if (workspace_bytes) *workspace_bytes = 0;
-            if (segments) *segments = 1;
-            if (launches) *launches = 0;
-            return M3_OK;
-        }
+        *info = m3_plan_info{};
+        info->segments = 1;
+        if (d->batch == 0) return M3_OK;  // nothing to run, whichever kernel was asked for
         m3::Problem p{};
         p.Bt = d->batch; p.T = d->seqlen; p.H = d->nheads; p.P = d->headdim; p.N = d->dstate; p.R = d->rank;
         p.bf16 = d->io == M3_BF16;
@@ -267,17 +273,42 @@ m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_bytes, int 
         const bool tc = base != M3_ALGO_SIMT && m3::prefill_tc_supported(p, &why);
         if (base == M3_ALGO_TC && !tc)
             return fail(M3_ERR_UNSUPPORTED, "%s", why ? why : "tensor-core path unsupported");
-        m3::TcPlan plan{};
-        if (tc) plan = m3::prefill_tc_plan(p);
-        if (workspace_bytes) *workspace_bytes = tc ? plan.ws_bytes : 0;
-        if (segments) *segments = tc ? plan.nseg : 1;
-        if (launches) *launches = (d->batch == 0 || d->nheads == 0) ? 0 : (tc ? plan.launches : 1);
+        if (!tc) {
+            info->kernel = M3_KERNEL_SIMT;
+            info->launches = 1;
+            info->ctas = d->batch * d->nheads;
+            return M3_OK;
+        }
+        if (flags & M3_PLAN_STATIC) p.ws_cap = m3::static_scratch_bytes();
+        if (flags & M3_PLAN_NO_WORKSPACE) p.no_balance = true;
+        const m3::TcPlan plan = m3::prefill_tc_plan(p);
+        if ((flags & M3_PLAN_STATIC) && plan.ws_bytes > p.ws_cap)
+            return fail(M3_ERR_UNSUPPORTED, "m3_scan_fwd_static: this segment count needs more than the "
+                                            "library's 24 MiB scratch");
+        if ((flags & M3_PLAN_NO_WORKSPACE) && plan.ws_bytes)
+            return fail(M3_ERR_INVALID_ARG, "this split needs a workspace");
+        info->kernel = M3_KERNEL_TC;
+        info->workspace_bytes = plan.ws_bytes;
+        info->segments = plan.nseg;
+        info->launches = plan.launches;
+        info->balanced = plan.balanced ? 1 : 0;
+        info->ctas = plan.ctas;
         return M3_OK;
     } catch (const std::exception &ex) {
         return fail(M3_ERR_INVALID_ARG, "internal error: %s", ex.what());
     } catch (...) {
         return fail(M3_ERR_INVALID_ARG, "internal error");
     }
+}
+
+m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_bytes, int *segments, int *launches) {
+    m3_plan_info info{};
+    const m3_status s = m3_scan_plan_info(algo, d, 0, &info);
+    if (s != M3_OK) return s;
+    if (workspace_bytes) *workspace_bytes = info.workspace_bytes;
+    if (segments) *segments = info.segments;
+    if (launches) *launches = info.launches;
+    return M3_OK;
 }
 
 m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes) {

@@ -17,9 +17,8 @@ enum : unsigned {
     kErrWaitTma = 1u << 0,
     kErrWaitMma = 1u << 1,
     kErrWaitCompute = 1u << 2,
-    kErrWaitProducer = 1u << 3,
+    kErrWaitHandoff = 1u << 3,   // a slice hand-off between two CTAs of the balanced schedule
     kErrWaitSelftest = 1u << 4,  // the self-test wait of m3_selftest_wait_timeout
-    kErrTmemAlloc = 1u << 4,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -271,16 +270,6 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// sin and cos of x: Cody-Waite reduction of x by 2*pi (two-term split of
-// 2*pi, hi part exact in 13 bits), then the hardware approximations on
-// [-pi, pi].
-__device__ __forceinline__ void sincos_reduced(float x, float *s, float *c) {
-    const float k = rintf(x * 0.15915494309189535f);  // x / (2 pi)
-    float r = fmaf(-k, 6.28125f, x);                   // 2 pi hi = 6.28125 (exact)
-    r = fmaf(-k, 1.9353071795864769e-3f, r);          // 2 pi lo
-    __sincosf(r, s, c);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);

@@ -130,7 +130,24 @@ def test_workspace_query_is_host_only(m3):
 
 
 def test_version(m3):
-    assert m3.lib.m3_version() == 100
+    assert m3.lib.m3_version() == 101
+
+
+def test_scan_plan_info_host_side(m3):
+    """m3_scan_plan_info on the host: the kernel that runs is reported (fp32
+    I/O: the SIMT kernel, one CTA per slice, no workspace), bad flags and a
+    NULL result are refused, an empty batch runs nothing."""
+    d = dims(m3, Bt=3, H=5, io=0)
+    info = m3.scan_plan_info(d)
+    assert info == m3.PlanInfo(0, m3.KERNEL_SIMT, 1, 1, False, 15)
+    assert info.kernel_name == "prefill_simt_kernel"
+    assert m3.scan_plan_info(d, flags=m3.PLAN_STATIC).kernel == m3.KERNEL_SIMT
+    assert m3.scan_plan_info(dims(m3, Bt=0)) == m3.PlanInfo(0, m3.KERNEL_NONE, 1, 0, False, 0)
+    out = m3.CPlanInfo()
+    assert m3.lib.m3_scan_plan_info(0, ctypes.byref(d), 4, ctypes.byref(out)) == 1
+    assert "flags" in m3.lib.m3_last_error().decode()
+    assert m3.lib.m3_scan_plan_info(0, ctypes.byref(d), 0, None) == 1
+    assert m3.lib.m3_scan_plan_info(m3.ALGO_TC, ctypes.byref(d), 0, ctypes.byref(out)) == 2
 
 
 def test_segment_count_only_with_tc(m3):
@@ -282,3 +299,43 @@ def test_bench_clock_summary():
     quiet = bench.ClockSampler.summarise(row.format(sm=1965, pw=500, cap="Not Active"))
     assert quiet["reasons"] == []
     assert bench.ClockSampler.summarise("") is None
+
+
+class _FakeCudaTensor:
+    """Stand-in for a CUDA tensor (no GPU here): only what the binding's
+    device check reads."""
+
+    def __init__(self, index, contiguous=True):
+        import torch
+        self.device = torch.device("cuda", index)
+        self.is_cuda = True
+        self._contiguous = contiguous
+
+    def is_contiguous(self):
+        return self._contiguous
+
+
+def test_binding_refuses_tensors_on_two_gpus(m3):
+    """Tensors of one call on different GPUs are refused before any pointer
+    reaches the library; the common device is returned otherwise."""
+    a, b = _FakeCudaTensor(0), _FakeCudaTensor(1)
+    assert m3._require_cuda(a, None, _FakeCudaTensor(0)) == a.device
+    with pytest.raises(ValueError, match="different devices"):
+        m3._require_cuda(a, b)
+    with pytest.raises(ValueError, match="contiguous"):
+        m3._require_cuda(_FakeCudaTensor(0, contiguous=False))
+    with pytest.raises(ValueError, match="different devices"):
+        m3.scan_fwd(a, a, a, a, a, a, a, b)
+    with pytest.raises(ValueError, match="different devices"):
+        m3.step(a, a, a, a, a, a, a, a, m3.State(a, a, b))
+
+
+def test_binding_refuses_a_stream_of_another_gpu(m3):
+    import torch
+
+    class _S:
+        device = torch.device("cuda", 1)
+        cuda_stream = 0
+
+    with pytest.raises(ValueError, match="stream is on"):
+        m3._stream(_S(), torch.device("cuda", 0))
