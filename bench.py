@@ -355,7 +355,7 @@ def time_prefill(m3, name, args, dev, rank, world, barrier, max_over_ranks, hbm_
                           "frac": achieved / hbm_peak, "traffic": recorded_traffic(kernel, name),
                           "kernel": kernel, "algorithmic_bytes_per_launch": abytes, "launch_ms": launch * 1e3,
                           "peak_source": peak_src},
-             "schedule": {"balanced": info.balanced, "ctas": info.ctas, "segments_per_sequence": info.segments,
+             "schedule": {"ctas": info.ctas, "segments_per_sequence": info.segments,
                           "kernel_launches_per_call": info.launches}}
     if info.launches > 1:
         entry["roofline"]["note"] = ("sequences split into segments: summary pass, segment scan and main pass; "
@@ -442,7 +442,7 @@ def run_ours(args):
                          "kernel": kernel, "algorithmic_bytes_per_launch": abytes,
                          "launch_ms": launch * 1e3, "peak_source": peak_src,
                          "segments_per_sequence": info.segments, "kernel_launches_per_call": info.launches,
-                         "balanced_schedule": info.balanced, "ctas": info.ctas},
+                         "ctas": info.ctas},
             "gpu_launches": K * info.launches, "clocks": clk}
     if info.launches > 1:
         line["roofline"]["note"] = ("sequences split into segments: summary pass, segment scan and main pass; "

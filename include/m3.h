@@ -149,26 +149,19 @@ typedef enum m3_algo {
 
 /* Bytes of device workspace m3_scan_fwd needs for these dims (0 = none; the
  * workspace pointer may then be NULL).  Host function; the answer depends on
- * the current CUDA device's SM count (it sets how the work is scheduled).  The
- * workspace (16-byte aligned) holds either the fp32 per-segment states of
- * split sequences, [segments][batch*nheads][dstate][headdim + 1], or -- with
- * more (batch, head) slices than SMs, where the tensor-core path runs one CTA
- * per SM over equal runs of chunks -- one fp32 [dstate][headdim] state per SM
- * for the slices cut between two CTAs and one flag word per SM, which the
- * call clears itself (a 4-byte-per-SM memset queued on the stream before its
- * kernel).  It needs no initialisation, its contents are meaningless after
- * the call, and calls that may run at the same time (other streams) must not
- * share one.  A workspace smaller than this answer (NULL included) is
- * refused only where sequences are split; otherwise the call then runs one
- * CTA per (batch, head) slice, which needs none. */
+ * the current CUDA device's SM count (it sets how sequences are split).  The
+ * workspace (16-byte aligned) holds fp32 per-segment states of split
+ * sequences, [segments][batch*nheads][dstate][headdim + 1]; it needs no
+ * initialisation, its contents are meaningless after the call, and calls that
+ * may run at the same time (other streams) must not share one. */
 M3_API m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes);
 
-/* How m3_scan_fwd_algo(algo, d, ...) will run on the current device, given
- * the workspace it asks for: workspace bytes, segments per sequence (1 = not
- * split) and the number of kernel launches of one call.  Any output pointer
- * may be NULL.  M3_ERR_UNSUPPORTED if `algo` names the tensor-core path for
- * sizes it does not cover.  (m3_scan_plan_info tells more, and also how
- * m3_scan_fwd_static and workspace-less calls run.) */
+/* How m3_scan_fwd_algo(algo, d, ...) will run on the current device:
+ * workspace bytes, segments per sequence (1 = not split) and the number of
+ * kernel launches of one call.  Any output pointer may be NULL.
+ * M3_ERR_UNSUPPORTED if `algo` names the tensor-core path for sizes it does
+ * not cover.  (m3_scan_plan_info also names the kernel, and tells how
+ * m3_scan_fwd_static runs.) */
 M3_API m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_bytes, int *segments,
                               int *launches);
 
@@ -184,22 +177,20 @@ typedef struct m3_plan_info {
     int32_t kernel;          /* m3_kernel that runs                                 */
     int32_t segments;        /* segments per sequence (1 = not split)               */
     int32_t launches;        /* kernel launches of one call                         */
-    int32_t balanced;        /* 1: one CTA per SM over equal runs of chunks         */
+    int32_t reserved;        /* 0                                                   */
     int64_t ctas;            /* CTAs of the (main) launch                           */
 } m3_plan_info;
 
-/* Flags of m3_scan_plan_info: describe the call as m3_scan_fwd_static runs it
- * (the library's scratch bounds the schedule), or as m3_scan_fwd runs it
- * with no workspace (one CTA per slice; M3_ERR_INVALID_ARG where the
- * sequences must be split and so need one). */
+/* Flag of m3_scan_plan_info: describe the call as m3_scan_fwd_static runs it
+ * (the library's 24 MiB scratch bounds its choice of segments, so it may
+ * differ from m3_scan_fwd's). */
 #define M3_PLAN_STATIC 1
-#define M3_PLAN_NO_WORKSPACE 2
 
 /* Which kernel and schedule m3_scan_fwd_algo(algo, d, ...) -- or, with
- * `flags`, m3_scan_fwd_static or a workspace-less call -- runs on the current
- * device.  Host function.  So that a bf16 call that runs the SIMT kernel (for
- * sizes the tensor-core kernel does not cover: headdim != 64, dstate not 64
- * or 128, rank not 1, 2 or 4) is visible to the caller. */
+ * M3_PLAN_STATIC, m3_scan_fwd_static -- runs on the current device.  Host
+ * function.  So that a bf16 call that runs the SIMT kernel (for sizes the
+ * tensor-core kernel does not cover: headdim != 64, dstate not 64 or 128,
+ * rank not 1, 2 or 4) is visible to the caller. */
 M3_API m3_status m3_scan_plan_info(int algo, const m3_dims *d, int flags, m3_plan_info *info);
 
 /* Prefill: the chunked scan over a whole sequence (the four-piece chunked
@@ -239,8 +230,7 @@ M3_API m3_status m3_scan_fwd_bcnorm(int algo, const m3_dims *d, const m3_bcnorm 
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /* m3_scan_fwd_algo without a workspace argument: the per-segment states of
- * split sequences (and the hand-off states and flags of the balanced
- * schedule) go to a scratch area the library itself holds in device
+ * split sequences go to a scratch area the library itself holds in device
  * memory (a static 24 MiB array, reserved on each device when the library's
  * code is loaded there).  The pages have no counterpart to this entry point;
  * it exists for callers that cannot hand over device memory.
@@ -349,12 +339,10 @@ M3_API m3_status m3_step_bcnorm(const m3_dims *d, const m3_bcnorm *bcn,
  * stream: the call reports (and clears) a wait that gave up in a kernel of
  * any stream of the current device, whatever `stream` is.  The code in the
  * message tells which wait: 0x1 a tile copy, 0x2 a tensor-core MMA, 0x4 the
- * other warps of the prefill CTA, 0x8 a slice hand-off between two CTAs of
- * the balanced schedule, 0x10 the self-test; the same bits shifted left by 8
- * come from the decode kernels.  A device-side wait gives up only on a
- * library bug (or when another kernel occupies SMs for seconds while a CTA
- * of the balanced schedule waits for one that has not started); this call
- * exists so that such a failure surfaces as a status instead of a hang.
+ * other warps of the prefill CTA, 0x10 the self-test; the same bits shifted
+ * left by 8 come from the decode kernels.  A device-side wait gives up only on
+ * a library bug; this call exists so that such a failure surfaces as a status
+ * instead of a hang.
  * The library keeps, per device and for the life of the process, the
  * address of its scratch array and the host-buffer entry point's two streams
  * and events: do not use it across a cudaDeviceReset (or other teardown of

@@ -23,7 +23,7 @@ M3_FLAG_A_PER_TOKEN = 1
 M3_FLAG_THETA_PER_HEAD = 2
 ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
 KERNEL_NONE, KERNEL_SIMT, KERNEL_TC = 0, 1, 2
-PLAN_STATIC, PLAN_NO_WORKSPACE = 1, 2
+PLAN_STATIC = 1
 
 
 def ALGO_TC_SEGMENTS(s: int) -> int:
@@ -60,7 +60,7 @@ def _cbcn(b: BCNorm):
 
 class CPlanInfo(ctypes.Structure):
     _fields_ = [("workspace_bytes", ctypes.c_size_t), ("kernel", ctypes.c_int32), ("segments", ctypes.c_int32),
-                ("launches", ctypes.c_int32), ("balanced", ctypes.c_int32), ("ctas", ctypes.c_int64)]
+                ("launches", ctypes.c_int32), ("reserved", ctypes.c_int32), ("ctas", ctypes.c_int64)]
 
 
 class CState(ctypes.Structure):
@@ -227,7 +227,6 @@ class PlanInfo(NamedTuple):
     kernel: int     # KERNEL_SIMT or KERNEL_TC (KERNEL_NONE: nothing to run)
     segments: int   # per sequence (1 = not split)
     launches: int   # kernel launches of one call
-    balanced: bool  # one CTA per SM over equal runs of chunks
     ctas: int       # CTAs of the (main) launch
 
     @property
@@ -237,11 +236,10 @@ class PlanInfo(NamedTuple):
 
 def scan_plan_info(dims: Dims, algo: int = ALGO_AUTO, flags: int = 0) -> PlanInfo:
     """Which kernel and schedule one prefill call runs on the current device
-    (flags: PLAN_STATIC for scan_fwd_static, PLAN_NO_WORKSPACE for a call
-    without a workspace)."""
+    (flags: PLAN_STATIC for scan_fwd_static)."""
     info = CPlanInfo()
     _check(get_lib().m3_scan_plan_info(algo, ctypes.byref(dims), flags, ctypes.byref(info)))
-    return PlanInfo(info.workspace_bytes, info.kernel, info.segments, info.launches, bool(info.balanced), info.ctas)
+    return PlanInfo(info.workspace_bytes, info.kernel, info.segments, info.launches, info.ctas)
 
 
 def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,

@@ -219,13 +219,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
                 if (e != cudaSuccess) return cuda_fail(e, "m3_scan_fwd_static (scratch address)");
             }
         } else {
-            size_t need = m3::prefill_tc_workspace(p);
-            if (need > ws_bytes || (need && !ws)) {
-                // without room for the balanced schedule's hand-off slots the
-                // call runs one CTA per sequence (which needs none)
-                p.no_balance = true;
-                need = m3::prefill_tc_workspace(p);
-            }
+            const size_t need = m3::prefill_tc_workspace(p);
             if (need > ws_bytes || (need && !ws))
                 return fail(M3_ERR_INVALID_ARG, "workspace too small (query m3_scan_workspace_size)");
             if (need && !aligned16(ws)) return fail(M3_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
@@ -255,7 +249,7 @@ m3_status m3_scan_plan_info(int algo, const m3_dims *d, int flags, m3_plan_info 
         if (!info) return fail(M3_ERR_INVALID_ARG, "info is NULL");
         m3_status s = check_dims(d, false);
         if (s != M3_OK) return s;
-        if (flags & ~(M3_PLAN_STATIC | M3_PLAN_NO_WORKSPACE)) return fail(M3_ERR_INVALID_ARG, "unknown plan flags");
+        if (flags & ~M3_PLAN_STATIC) return fail(M3_ERR_INVALID_ARG, "unknown plan flags");
         const int forced = algo >> 8;
         const int base = algo & 0xff;
         if (base != M3_ALGO_AUTO && base != M3_ALGO_SIMT && base != M3_ALGO_TC)
@@ -280,18 +274,14 @@ m3_status m3_scan_plan_info(int algo, const m3_dims *d, int flags, m3_plan_info 
             return M3_OK;
         }
         if (flags & M3_PLAN_STATIC) p.ws_cap = m3::static_scratch_bytes();
-        if (flags & M3_PLAN_NO_WORKSPACE) p.no_balance = true;
         const m3::TcPlan plan = m3::prefill_tc_plan(p);
         if ((flags & M3_PLAN_STATIC) && plan.ws_bytes > p.ws_cap)
             return fail(M3_ERR_UNSUPPORTED, "m3_scan_fwd_static: this segment count needs more than the "
                                             "library's 24 MiB scratch");
-        if ((flags & M3_PLAN_NO_WORKSPACE) && plan.ws_bytes)
-            return fail(M3_ERR_INVALID_ARG, "this split needs a workspace");
         info->kernel = M3_KERNEL_TC;
         info->workspace_bytes = plan.ws_bytes;
         info->segments = plan.nseg;
         info->launches = plan.launches;
-        info->balanced = plan.balanced ? 1 : 0;
         info->ctas = plan.ctas;
         return M3_OK;
     } catch (const std::exception &ex) {

@@ -365,6 +365,14 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
         tc::fence_mbar_init();
     }
     __syncthreads();
+    // With fewer slices than resident CTAs the kernel is launched as a
+    // programmatic dependent of the previous kernel on the stream: its CTAs are
+    // scheduled while that kernel still runs, nothing is read before that
+    // kernel has completed (the wait below), and the next step may launch as
+    // soon as every CTA here has started.  Without the launch attribute both
+    // instructions do nothing.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         if ((int64_t)blockIdx.x < BH) issue(blockIdx.x, 0);
         if ((int64_t)blockIdx.x + step < BH) issue(blockIdx.x + step, 1);
@@ -493,8 +501,24 @@ cudaError_t launch_stream(const StepArgs<IO> &a, const StepFeat &f, cudaStream_t
                              (int)Cfg::SMEM);
     if (e != cudaSuccess) return e;
     int64_t grid = (int64_t)sms * Cfg::CTAS_PER_SM;
+    // programmatic dependent launch only where the grid leaves SMs free (few
+    // slices: it hides the launch gap of a latency-bound step; measured: the
+    // long-context decode's 64 slices 3.44 -> 3.27 us per step, while a grid
+    // that fills every SM ran 1.6 % slower with it)
+    const bool pdl = grid > a.BH;
     if (grid > a.BH) grid = a.BH;
-    step_stream_kernel<N, P, R, IO, GEN><<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, s>>>(a, f);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, step_stream_kernel<N, P, R, IO, GEN>, a, f);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

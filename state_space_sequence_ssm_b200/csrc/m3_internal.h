@@ -25,20 +25,16 @@ struct Problem {
     size_t ws_bytes;
     int segments;                 // tensor-core prefill: segments per sequence (0 = chosen by the library)
     size_t ws_cap;                // > 0: the library's choice of segments must fit this workspace
-    bool no_balance;              // tensor-core prefill: one CTA per slice even with more slices than SMs
     cudaStream_t stream;
 };
 
 // How the tensor-core prefill runs one problem: every sequence in `nseg`
-// segments of `cpseg` chunks (nseg > 1: summary pass, segment scan, main pass
-// = three launches and a workspace of ws_bytes), or (nseg = 1) one launch of
-// `ctas` CTAs: one per sequence, or -- balanced, with more sequences than SMs
-// -- one per SM, each taking an equal run of all chunks (a workspace of
-// ws_bytes for the states of sequences cut between two CTAs).
+// segments of `cpseg` chunks (nseg = 1: one CTA per sequence, one launch;
+// nseg > 1: summary pass, segment scan, main pass = three launches and a
+// workspace of ws_bytes); `ctas` CTAs in the (main) launch.
 struct TcPlan {
     int nchunks, cpseg, nseg, launches;
     int64_t ctas;
-    bool balanced;
     size_t ws_bytes;
 };
 

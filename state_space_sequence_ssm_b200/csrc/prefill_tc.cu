@@ -8,13 +8,8 @@
 // gamma_hat_s = lam_s dt_s + (1 - lam_{s+1}) dt_{s+1}, the pair rotations
 // of B and C by the chunk-local cumulative angle, and rank-R MIMO rows.
 //
-// Every CTA walks a run of chunks of 128 rows (Q = 128 / R tokens x R
-// ranks), the M = 128 shape of one tcgen05 MMA.  With more (batch, head)
-// slices than SMs, one CTA per SM takes an equal share of all chunks (slice
-// after slice, its pipeline running on from one into the next); a slice cut
-// between two CTAs is continued by the second from the state the first
-// publishes (see "Balanced schedule" below).  Otherwise one CTA takes one
-// slice.
+// One CTA per (batch, head) walks its sequence in chunks of 128 rows
+// (Q = 128 / R tokens x R ranks), the M = 128 shape of one tcgen05 MMA.
 // Per chunk c the tensor cores compute (bf16 operands in shared memory,
 // fp32 accumulators in TMEM)
 //   S  = C~ B~^T          (128 x 128, K = N)        masked into P (bf16)
@@ -42,16 +37,6 @@
 // A sequence too long for the grid to fill the GPU is split into segments
 // (a summary pass, a scan over the segments, then this pass per segment:
 // the MODE template argument).
-//
-// Balanced schedule (MODE kFlow with fewer CTAs than slices): the chunks of
-// all slices, slice-major, are cut into gridDim.x runs of equal length (to
-// one chunk); each run is at least a slice long, so it holds at most the
-// tail of one slice (its first chunks), whole slices, and the head of
-// another slice (its last chunks).  A CTA runs the head first, then the
-// whole slices, then the tail: the head's pending-inclusive end state goes to
-// the CTA's slot of the workspace with a release flag, and the next CTA,
-// whose tail it is, takes it from there long after it was written -- its
-// wait is short or none, and no CTA waits on a CTA that waits.
 // Every wait is bounded; a wait that gives up records a code that the host
 // reads back with m3_stream_status() and the CTA drains and returns.
 #include <cuda.h>
@@ -128,10 +113,8 @@ struct Cfg {
     static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16 + 2 * R * K2 + 2 * kRows;
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
     static constexpr uint32_t NBARS = 19;
-    // TMEM base, abort flag, first chunk (16 B), FlowMap (48 B), the prologue's
-    // and the state warps' current piece (32 B each)
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
-    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 128 + 1024;  // + slack for 1024 alignment
+    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024 alignment
     static_assert(K2 % 4 == 0 && kPro % G4 == 0, "pair groups must tile the prologue threads");
     static_assert(Q % NPART == 0 && TPT % TB == 0, "tokens must split across the angle-pass parts");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -142,12 +125,6 @@ struct TcArgs {
     int nchunks;
     int cpseg;         // chunks per segment (nchunks when the sequence is not split)
     int nseg;          // segments per sequence
-    // kFlow with gridDim.x < BH: hand-off slots [gridDim.x][N][P] fp32 of the
-    // pending-inclusive states of slices cut between two CTAs, then
-    // gridDim.x flags (zeroed before the launch); unused when every CTA
-    // takes whole slices
-    float *flow_h;
-    unsigned *flow_flag;
     const __nv_bfloat16 *x, *B, *dt, *lam, *theta;
     const float *A, *D, *h0, *bp0, *xp0;
     const float *A_tok;  // non-null: A per token-head [Bt, T, H] (A unused)
@@ -338,63 +315,13 @@ struct Bars {
     uint64_t *full_bc, *empty_bc, *full_x, *empty_x, *ops, *sg, *hrdy, *p, *yd, *drain, *sc;
 };
 
-// Pass kinds.  kFlow: the full forward pass over this CTA's run of chunks --
-// one whole slice per CTA when the grid has one CTA per slice, else the
-// balanced schedule described at the top of this file.  kSummary: the
-// summary pass of a split sequence -- only the chunk states and the
-// carried-state chain over one segment, from a zero state (segment 0: the
+// Pass kinds.  kWhole: the full forward pass, one CTA per sequence.
+// kSummary: the summary pass of a split sequence -- only the chunk states and
+// the carried-state chain over one segment, from a zero state (segment 0: the
 // caller's initial state), ending in the segment's local end state and its
 // transition, for the segment scan.  kSegment: the full forward pass over one
 // segment, from the scanned state.
-constexpr int kFlow = 0, kSummary = 1, kSegment = 2;
-
-// A CTA's run of chunks under kFlow, in the order it processes them: hl
-// chunks of slice sb (its head: chunks 0 .. hl-1), nf whole slices sf0,
-// sf0 + 1, ... (nfc chunks), then tl chunks of slice sa (its tail: chunks
-// ca0 .. nchunks-1); n chunks in np pieces.  Written by thread 0 into shared
-// memory.
-struct FlowMap {
-    int hl, sb, nfc, sf0, tl, sa, ca0, n, nf, np;
-};
-
-// A piece of a CTA's run: chunks [c0, c1) of slice bh = b * H + h, the
-// piece's index pc, and the head's A (log2 units) and D.  The prologue and
-// the state warps each keep their current piece in shared memory and read
-// its fields where they use them, so that their chunk loops hold no more
-// registers than a CTA bound to one slice.
-struct Piece {
-    int b, h, bh, c0, c1, pc;
-    float Ah2, Dh;
-};
-
-__device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Bounded wait for a hand-off flag another CTA sets (same rules as
-// mbar_wait: gives up after `budget` cycles, or when `abort` is raised).
-__device__ __forceinline__ bool flag_wait(const unsigned *flag, volatile int *abort, unsigned *err_word,
-                                          unsigned code, long long budget = 4000000000LL) {
-    if (ld_acquire_gpu(flag)) return true;
-    const long long t0 = clock64();
-    for (uint32_t it = 1;; ++it) {
-        __nanosleep(128);
-        if (ld_acquire_gpu(flag)) return true;
-        if ((it & 15u) == 0) {
-            if (*abort) return false;
-            if (clock64() - t0 > budget) {
-                *abort = 1;
-                atomicOr(err_word, code);
-                return false;
-            }
-        }
-    }
-}
+constexpr int kWhole = 0, kSummary = 1, kSegment = 2;
 
 // GEN = false: the plain method (A per head, theta per token), compiled
 // without the optional features' branches; GEN = true reads A_tok and th_head
@@ -406,7 +333,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                   const TcArgs a) {
     using C = Cfg<N, R>;
     constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, G4 = C::G4, NPART = C::NPART, TPT = C::TPT, TB = C::TB;
-    constexpr bool SUM = MODE == kSummary, SEGD = MODE != kFlow, FLOW = MODE == kFlow;
+    constexpr bool SUM = MODE == kSummary, SEGD = MODE != kWhole;
     const float *const A_tok = GEN ? a.A_tok : nullptr;  // A per token-head, or none
     const bool th_head = GEN && a.th_head;               // theta fixed per head
     extern __shared__ uint8_t smem_raw[];
@@ -433,19 +360,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     // first chunk of this CTA's segment, re-read where needed (a register
     // held across the prologue warps' loop would spill)
     volatile int *chunk0 = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
-    // read through a volatile pointer at every use, so that no role keeps its
-    // fields in registers across its chunk loop (the prologue and state warps
-    // have none to spare)
-    volatile FlowMap *fmap = reinterpret_cast<volatile FlowMap *>(smem + C::OFF_MISC + 16);
     unsigned *err = &g_device_error;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // segment-major CTA order: CTAs of neighbouring heads share dt/lam sectors
-    const uint32_t BH = (uint32_t)a.BH;
+    const uint32_t BH = SEGD ? (uint32_t)a.BH : gridDim.x;
     const int seg = SEGD ? (int)(blockIdx.x / BH) : 0;
+    const int64_t bh = SEGD ? blockIdx.x % BH : blockIdx.x;
     const int64_t T = a.T, H = a.H;
-    // token-head index of token t of slice (b, h)
-    auto tok = [&](int64_t b, int64_t h, int64_t t) { return (b * T + t) * H + h; };
+    const int64_t b = bh / H, h = bh % H;
+    auto tok = [&](int64_t t) { return (b * T + t) * H + h; };
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -465,32 +389,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         mbar_init(bb.drain, 1);
         *abort_flag = 0;
         *chunk0 = SEGD ? (int)(blockIdx.x / (uint32_t)a.BH) * a.cpseg : 0;
-        if (FLOW) {  // this CTA's run [lo, hi) of all BH * nchunks chunks, slice-major
-            const int64_t nch = a.nchunks, W = (int64_t)a.BH * nch, G = gridDim.x;
-            const int64_t lo = (int64_t)blockIdx.x * W / G, hi = ((int64_t)blockIdx.x + 1) * W / G;
-            FlowMap f;
-            f.hl = (int)(hi % nch);
-            f.sb = (int)(hi / nch);
-            const int64_t sf0 = (lo + nch - 1) / nch;
-            f.sf0 = (int)sf0;
-            f.nfc = (int)((hi / nch - sf0) * nch);
-            f.ca0 = (int)(lo % nch);
-            f.tl = f.ca0 ? (int)(nch - f.ca0) : 0;
-            f.sa = (int)(lo / nch);
-            f.n = (int)(hi - lo);
-            f.nf = f.nfc / a.nchunks;
-            f.np = (f.hl > 0) + f.nf + (f.tl > 0);
-            fmap->nf = f.nf;
-            fmap->np = f.np;
-            fmap->hl = f.hl;
-            fmap->sb = f.sb;
-            fmap->nfc = f.nfc;
-            fmap->sf0 = f.sf0;
-            fmap->tl = f.tl;
-            fmap->sa = f.sa;
-            fmap->ca0 = f.ca0;
-            fmap->n = f.n;
-        }
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -507,108 +405,41 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    // this CTA's nloc chunks, local index i (ring stages and mbarrier phases
-    // count from it): a segment [cb, cb + nloc) of one slice, or the run of
-    // the balanced schedule
+    // this CTA's chunks [cb, cb + nloc); ring stages and mbarrier phases
+    // count from the segment's first chunk (local index i)
     const int cb = SEGD ? seg * a.cpseg : 0;
-    const int nloc = SEGD ? ((a.nchunks - cb < a.cpseg) ? a.nchunks - cb : a.cpseg) : fmap->n;
-    // Piece pc of this CTA's run (kFlow: head, whole slices, tail; a segment
-    // pass: its one segment).
-    const int npieces = FLOW ? fmap->np : 1;
-    auto piece = [&](int pc) {
-        Piece P;
-        if (FLOW) {
-            const int hl = fmap->hl, k = pc - (hl > 0 ? 1 : 0);
-            if (hl > 0 && pc == 0) {
-                P.bh = fmap->sb;
-                P.c0 = 0;
-                P.c1 = hl;
-            } else if (k < fmap->nf) {
-                P.bh = fmap->sf0 + k;
-                P.c0 = 0;
-                P.c1 = a.nchunks;
-            } else {
-                P.bh = fmap->sa;
-                P.c0 = fmap->ca0;
-                P.c1 = a.nchunks;
-            }
-        } else {
-            P.bh = (int)(blockIdx.x % BH);
-            P.c0 = *chunk0;
-            P.c1 = *chunk0 + nloc;
-        }
-        P.b = P.bh / (int)H;
-        P.h = P.bh - P.b * (int)H;
-        P.pc = pc;
-        P.Ah2 = A_tok ? 0.f : a.A[P.h] * kLog2e;
-        P.Dh = a.D[P.h];
-        return P;
-    };
-    auto put_piece = [](volatile Piece *dst, const Piece &P) {
-        dst->b = P.b;
-        dst->h = P.h;
-        dst->bh = P.bh;
-        dst->c0 = P.c0;
-        dst->c1 = P.c1;
-        dst->pc = P.pc;
-        dst->Ah2 = P.Ah2;
-        dst->Dh = P.Dh;
-    };
-
-    // A walk over this CTA's chunks in order, for the single-thread TMA
-    // producers (registers to spare, and no division per chunk on the path
-    // that issues the copies): slice (b, h), chunk c, the piece's end c1.
-    struct Walk {
-        int b, h, c, c1, pc;
-    };
-    auto walk_start = [&]() {
-        const Piece P = piece(0);
-        return Walk{P.b, P.h, P.c0, P.c1, 0};
-    };
-    auto walk_next = [&](Walk &w) {
-        if (++w.c < w.c1 || w.pc + 1 >= npieces) return;
-        const Piece P = piece(++w.pc);
-        w.b = P.b;
-        w.h = P.h;
-        w.c = P.c0;
-        w.c1 = P.c1;
-    };
+    const int nloc = SEGD ? ((a.nchunks - cb < a.cpseg) ? a.nchunks - cb : a.cpseg) : a.nchunks;
+    auto first_chunk = [&]() { return SEGD ? *chunk0 : 0; };
 
     if (warp == kWarpTma) {
         // ============================================================ TMA producers
         if (lane == 0) {
             // B/C ring (2 stages), plus L2 prefetches of everything a chunk needs
-            auto prefetch_chunk = [&](const Walk &l) {
-                const int t0 = l.c * Q;
-                tma_prefetch_5d(&tmX, 0, 0, l.h, t0, l.b);
+            auto prefetch_chunk = [&](int c) {
+                const int t0 = c * Q;
+                tma_prefetch_5d(&tmX, 0, 0, (int)h, t0, (int)b);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_prefetch_5d(&tmB, kb * 64, 0, l.h, t0, l.b);
-                    if (!SUM) tma_prefetch_5d(&tmC, kb * 64, 0, l.h, t0, l.b);
+                    tma_prefetch_5d(&tmB, kb * 64, 0, (int)h, t0, (int)b);
+                    if (!SUM) tma_prefetch_5d(&tmC, kb * 64, 0, (int)h, t0, (int)b);
                 }
-                if (!th_head) tma_prefetch_4d(&tmT, 0, l.h, t0, l.b);  // read straight into registers
+                if (!th_head) tma_prefetch_4d(&tmT, 0, (int)h, t0, (int)b);  // read straight into registers
             };
             int issued = 0;
-            Walk l = walk_start(), lp = walk_start();  // the chunk to load, the chunk to prefetch
-            for (int i = 0; i < C::PREFETCH && i < nloc; ++i) {
-                prefetch_chunk(lp);
-                walk_next(lp);
-            }
-            for (int i = 0; i < nloc; ++i, walk_next(l)) {
-                if (i + C::PREFETCH < nloc) {
-                    prefetch_chunk(lp);
-                    walk_next(lp);
-                }
+            for (int i = 0; i < C::PREFETCH && i < nloc; ++i) prefetch_chunk(cb + i);
+            for (int i = 0; i < nloc; ++i) {
+                if (i + C::PREFETCH < nloc) prefetch_chunk(cb + i + C::PREFETCH);
                 const int s = i & 1;
                 if (i >= 2 && !mbar_wait(&bb.empty_bc[s], ((i >> 1) - 1) & 1, abort_flag, err, kErrWaitMma)) break;
                 uint8_t *st = smem + C::OFF_BC + s * C::BCS_BYTES;
-                const int t0 = l.c * Q;
+                const int t0 = (cb + i) * Q;
                 mbar_arrive_expect_tx(&bb.full_bc[s], SUM ? C::BC_BYTES : C::BCS_BYTES);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_5d(st + kb * 16384, &tmB, &bb.full_bc[s], kb * 64, 0, l.h, t0, l.b);
+                    tma_load_5d(st + kb * 16384, &tmB, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
                     if (!SUM)
-                        tma_load_5d(st + C::BC_BYTES + kb * 16384, &tmC, &bb.full_bc[s], kb * 64, 0, l.h, t0, l.b);
+                        tma_load_5d(st + C::BC_BYTES + kb * 16384, &tmC, &bb.full_bc[s], kb * 64, 0, (int)h, t0,
+                                    (int)b);
                 }
                 issued = i + 1;
             }
@@ -620,13 +451,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             // x ring (kNX stages), freed by the epilogue (the summary pass: by the
             // state update, once w o X has been formed from it)
             int issued = 0;
-            Walk l = walk_start();
-            for (int i = 0; i < nloc; ++i, walk_next(l)) {
+            for (int i = 0; i < nloc; ++i) {
                 const int s = i % kNX;
                 if (i >= kNX && !mbar_wait(&bb.empty_x[s], ((i / kNX) - 1) & 1, abort_flag, err, kErrWaitCompute))
                     break;
                 mbar_arrive_expect_tx(&bb.full_x[s], C::X_BYTES);
-                tma_load_5d(smem + C::OFF_X + s * C::X_BYTES, &tmX, &bb.full_x[s], 0, 0, l.h, l.c * Q, l.b);
+                tma_load_5d(smem + C::OFF_X + s * C::X_BYTES, &tmX, &bb.full_x[s], 0, 0, (int)h, (cb + i) * Q,
+                            (int)b);
                 issued = i + 1;
             }
             if (*abort_flag) {
@@ -709,26 +540,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
     } else if (warp < 8) {
         // ============================================================ prologue warps (0-7)
+        const float Ah2 = A_tok ? 0.f : a.A[h] * kLog2e;
         uint8_t *xw = smem + C::OFF_XW;
         const unsigned short *dtr = reinterpret_cast<const unsigned short *>(a.dt);
         const unsigned short *lmr = reinterpret_cast<const unsigned short *>(a.lam);
         const int g = tid % G4, part = tid / G4;  // angle pass: 4 pairs x TPT tokens per thread
-        volatile Piece *cur = reinterpret_cast<volatile Piece *>(smem + C::OFF_MISC + 64);  // this role's piece
         // raw bf16 bits of dt, lam for this thread's token and the one after it,
         // loaded one chunk ahead and converted only when used
         unsigned short pd = 0, pl = 0, pd1 = 0, pl1 = 0;
         float pa = 0.f;  // A of this thread's token (per-token A only)
-        auto prefetch_scalars = [&](int b, int h, int64_t t0s) {
+        auto prefetch_scalars = [&](int64_t t0s) {
             const int64_t t = t0s + tid;
             pd = pl = pd1 = pl1 = 0;
             if (tid < Q && t < T) {
-                const int64_t k = tok(b, h, t);
-                pd = __ldg(dtr + k);
-                pl = __ldg(lmr + k);
-                if (A_tok) pa = __ldg(A_tok + k);
+                pd = __ldg(dtr + tok(t));
+                pl = __ldg(lmr + tok(t));
+                if (A_tok) pa = __ldg(A_tok + tok(t));
                 if (t + 1 < T) {
-                    pd1 = __ldg(dtr + k + H);
-                    pl1 = __ldg(lmr + k + H);
+                    pd1 = __ldg(dtr + tok(t + 1));
+                    pl1 = __ldg(lmr + tok(t + 1));
                 }
             }
         };
@@ -745,45 +575,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 wB2[e] = pack_bf16(a.wB[n], a.wB[n + 1]);
                 wC2[e] = pack_bf16(a.wC[n], a.wC[n + 1]);
             }
+            for (int i = tid; i < 2 * R * K2; i += kPro) {
+                const int which = i / (R * K2), rk = i % (R * K2);
+                const float *src = (which ? a.bC : a.bB) + (h * R + rk / K2) * N + 2 * (rk % K2);
+                sbias[i] = pack_bf16(src[0], src[1]);
+            }
         }
-        // angle rates fixed per head: the thread's 4 pairs of the current slice's head
+        // angle rates fixed per head: the thread's 4 pairs, for the whole sequence
         float thh[4] = {0.f, 0.f, 0.f, 0.f};
-        auto prefetch_theta = [&](int b, int h, int64_t t0s) {
+        if (th_head) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) thh[e] = bf(a.theta, h * K2 + 4 * g + e);
+        }
+        auto prefetch_theta = [&](int64_t t0s) {
             if (th_head) return;
 #pragma unroll
             for (int j = 0; j < TPT; ++j) {
                 const int64_t t = t0s + part * TPT + j;
-                thr[j] = t < T ? __ldg(reinterpret_cast<const uint2 *>(a.theta + tok(b, h, t) * K2 + 4 * g))
+                thr[j] = t < T ? __ldg(reinterpret_cast<const uint2 *>(a.theta + tok(t) * K2 + 4 * g))
                                : make_uint2(0u, 0u);
             }
         };
-        {
-            const Piece P0 = piece(0);
-            prefetch_scalars(P0.b, P0.h, (int64_t)P0.c0 * Q);
-            prefetch_theta(P0.b, P0.h, (int64_t)P0.c0 * Q);
-        }
-        int lc = 0;  // local chunk index (ring stages, barrier phases)
-        bool go = true;
-        for (int pc = 0; pc < npieces && go; ++pc) {
-            // the piece's slice and its per-head values (the previous chunk's
-            // rotation, their last reader, ended before the barrier that closed
-            // it; the first barrier keeps every thread's last reads of the
-            // previous piece before the update)
-            named_bar(kBarPro, kPro);
-            if (tid == 0) put_piece(cur, piece(pc));
-            named_bar(kBarPro, kPro);
-            if (BCN) {
-                for (int i = tid; i < 2 * R * K2; i += kPro) {
-                    const int which = i / (R * K2), rk = i % (R * K2);
-                    const float *src = (which ? a.bC : a.bB) + (cur->h * R + rk / K2) * N + 2 * (rk % K2);
-                    sbias[i] = pack_bf16(src[0], src[1]);
-                }
-            }
-            if (th_head) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) thh[e] = bf(a.theta, cur->h * K2 + 4 * g + e);
-            }
-          for (int c = cur->c0; c < cur->c1; ++c, ++lc) {
+        prefetch_scalars((int64_t)cb * Q);
+        prefetch_theta((int64_t)cb * Q);
+        for (int lc = 0; lc < nloc; ++lc) {
             const int s = lc & 1, sx = lc % kNX;
             float *cAl2 = sbuf + sx * C::SB;
             float *gam = cAl2 + Q;
@@ -796,23 +611,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
             // the scalar buffer lc % kNX is free once the epilogue of lc - kNX is done
             if (lc >= kNX && bar_any<kBarPro, kPro>(!mbar_wait(&bb.empty_x[sx], ((lc / kNX) - 1) & 1, abort_flag,
-                                                              err, kErrWaitCompute))) {
-                go = false;
+                                                              err, kErrWaitCompute)))
                 break;
-            }
 
             // ---- A. per-token scalars and the chunk-local scan of dt*A
             float acc = 0.f, acd = 0.f;
             {
                 const float d = bf16_bits(pd), l = bf16_bits(pl);
                 const float nx = (1.f - bf16_bits(pl1)) * bf16_bits(pd1);  // 0 past the sequence end
-                const float a2 = A_tok ? pa * kLog2e : cur->Ah2;           // A_t in log2 units
-                if (c + 1 < cur->c1) {  // the next chunk: this piece's, or the next piece's first
-                    prefetch_scalars(cur->b, cur->h, (int64_t)(c + 1) * Q);
-                } else if (cur->pc + 1 < npieces) {
-                    const Piece Pn = piece(cur->pc + 1);
-                    prefetch_scalars(Pn.b, Pn.h, (int64_t)Pn.c0 * Q);
-                }
+                const float a2 = A_tok ? pa * kLog2e : Ah2;                // A_t in log2 units
+                if (lc + 1 < nloc) prefetch_scalars((int64_t)(first_chunk() + lc + 1) * Q);
                 if (tid < Q) {
                     dts[tid] = d;
                     gam[tid] = l * d;
@@ -875,10 +683,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
                 *reinterpret_cast<float4 *>(phis + part * K2 + 4 * g) = make_float4(loc[0], loc[1], loc[2], loc[3]);
                 // the B/C tiles of this chunk
-                if (bar_any<kBarPro, kPro>(!mbar_wait(&bb.full_bc[s], (lc >> 1) & 1, abort_flag, err, kErrWaitTma))) {
-                    go = false;
+                if (bar_any<kBarPro, kPro>(!mbar_wait(&bb.full_bc[s], (lc >> 1) & 1, abort_flag, err, kErrWaitTma)))
                     break;
-                }
                 if (BCN) {  // one row scale per thread: B rows (tid < 128), then C rows
                     if (!SUM || tid < kRows)
                         rsc[tid] = bc_row_scale<KB>(tid < kRows ? bst : cst, (uint32_t)(tid % kRows), 1.f / N, a.eps);
@@ -975,20 +781,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         sinE[4 * g + e] = sn;
                     }
                 }
-                if (c + 1 < cur->c1) {
-                    prefetch_theta(cur->b, cur->h, (int64_t)(c + 1) * Q);
-                } else if (cur->pc + 1 < npieces) {
-                    const Piece Pn = piece(cur->pc + 1);
-                    prefetch_theta(Pn.b, Pn.h, (int64_t)Pn.c0 * Q);
-                }
+                if (lc + 1 < nloc) prefetch_theta((int64_t)(first_chunk() + lc + 1) * Q);
             }
             // ---- C. w o X (chunk-state weights on the value rows), once G(c-1)
             //      has finished reading the previous w o X and x of chunk c is in
             if (bar_any<kBarPro, kPro>((lc >= 1 && !mbar_wait(bb.sg, (lc - 1) & 1, abort_flag, err, kErrWaitMma)) ||
-                                       !mbar_wait(&bb.full_x[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitTma))) {
-                go = false;
+                                       !mbar_wait(&bb.full_x[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitTma)))
                 break;
-            }
             {
                 const int row = tid >> 1, j0 = (tid & 1) * 4;  // half a row per thread
                 const float wv = wst[row / R];
@@ -1011,7 +810,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 mbar_arrive(bb.ops);
                 mbar_arrive(&bb.sc[sx]);
             }
-          }
         }
     } else {
         // ============================================================ state warps (8-15)
@@ -1024,137 +822,49 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const bool own_state = (N == 128) || (lane < 16);
         const int srow = (N == 128) ? lq : (wq * 16 + lane);  // TMEM lane layout of G (M = N)
         uint8_t *hbuf = smem + C::OFF_HB;
+        const float Dh = a.D[h];
         const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
         const int c0 = 32 * hf;            // first column of this thread's half
-        volatile Piece *cur = reinterpret_cast<volatile Piece *>(smem + C::OFF_MISC + 96);  // this role's piece
         float hreg[32];
-        // The caller's state entering slice (b, h), pending-inclusive:
-        // h0 + beta'_0 b_prev x_prev^T (the pending write of token -1).
-        auto caller_state = [&](int64_t b, int64_t h) {
-#pragma unroll
-            for (int p = 0; p < 32; ++p) hreg[p] = 0.f;
-            const int64_t bh = b * H + h;
-            const float betap0 = (1.f - bf(a.lam, tok(b, h, 0))) * bf(a.dt, tok(b, h, 0));
-            if (own_state) {
-                if (a.h0) {
-#pragma unroll
-                    for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * N + srow) * kP + c0 + p];
-                }
-                if (a.bp0 && a.xp0) {
-                    for (int r = 0; r < R; ++r) {
-                        const float cw = betap0 * a.bp0[(bh * R + r) * N + srow];
-#pragma unroll
-                        for (int p = 0; p < 32; ++p) hreg[p] = fmaf(cw, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
-                    }
-                }
-            }
-        };
-        // Balanced schedule: the state the previous CTA published for the
-        // slice this CTA ends with (bounded wait on its flag; false if it gave up).
-        auto handoff_state = [&]() {
-            bool got = true;
-            if (lt == 0) got = flag_wait(a.flow_flag + blockIdx.x - 1, abort_flag, err, kErrWaitHandoff);
-            if (bar_any<kBarState, kSt>(!got)) return false;
-            if (own_state) {
-                const float4 *src =
-                    reinterpret_cast<const float4 *>(a.flow_h + ((int64_t)(blockIdx.x - 1) * N + srow) * kP + c0);
-#pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    const float4 v = __ldcg(src + p);
-                    hreg[4 * p] = v.x;
-                    hreg[4 * p + 1] = v.y;
-                    hreg[4 * p + 2] = v.z;
-                    hreg[4 * p + 3] = v.w;
-                }
-            }
-            return true;
-        };
-        // Balanced schedule: publish the pending-inclusive state after this
-        // CTA's head chunks for the next CTA (slot blockIdx.x, then its flag).
-        auto publish_state = [&]() {
-            if (own_state) {
-                float4 *dst = reinterpret_cast<float4 *>(a.flow_h + ((int64_t)blockIdx.x * N + srow) * kP + c0);
-#pragma unroll
-                for (int p = 0; p < 8; ++p)
-                    __stcg(dst + p, make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]));
-                __threadfence();
-            }
-            named_bar(kBarState, kSt);
-            if (lt == 0) {
-                __threadfence();
-                st_release_gpu(a.flow_flag + blockIdx.x, 1u);
-            }
-        };
-        // Final state of slice (b, h): plain-frame h_{T-1}, the raw last token
-        // as the pending term (the BC-norm variant: its normalised B).
-        auto final_state = [&](int64_t b, int64_t h) {
-            const int64_t bh = b * H + h;
-            const int64_t last = tok(b, h, T - 1);
-            if (a.hT && own_state) {
-                float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * N + srow) * kP + c0);
-#pragma unroll
-                for (int p = 0; p < 8; ++p)
-                    dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
-            }
-            if (a.bpT && BCN) {  // the last token's normalised B, one state warp per rank row
-                const int wl = lt >> 5;
-                if (wl < R) {
-                    const int64_t src = last * R * N + wl * N;
-                    float ss = 0.f;
-                    for (int n = lane; n < N; n += 32) ss = fmaf(bf(a.B, src + n), bf(a.B, src + n), ss);
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                    const float sc = rsqrtf(ss / N + a.eps);
-                    for (int n = lane; n < N; n += 32)
-                        a.bpT[(bh * R + wl) * N + n] = fmaf(bf(a.B, src + n) * sc, a.wB[n], a.bB[(h * R + wl) * N + n]);
-                }
-            } else if (a.bpT) {
-                for (int i = lt; i < R * N; i += kSt) a.bpT[bh * R * N + i] = bf(a.B, last * R * N + i);
-            }
-            if (a.xpT)
-                for (int i = lt; i < R * kP; i += kSt) a.xpT[bh * R * kP + i] = bf(a.x, last * R * kP + i);
-        };
-        // summary pass: the segment's transition exp(cA) Rot(-Phi) on this row's pair
-        float m_l2 = 0.f, m_cs = 1.f, m_sn = 0.f;
-        bool ok = true;
-        int lc = 0;  // local chunk index (ring stages, barrier phases)
-        for (int pc = 0; pc < npieces && ok; ++pc) {
-            named_bar(kBarState, kSt);  // every thread is done with the previous piece
-            if (lt == 0) put_piece(cur, piece(pc));
-            named_bar(kBarState, kSt);
-            // Pending-inclusive state entering the piece.  A slice's first
-            // chunk (kFlow, segment 0 of the summary pass): the caller's state;
-            // a tail of the balanced schedule: the previous CTA's hand-off;
-            // later summary segments: zero (their local state); segments of
-            // the main pass: the scanned state.
+        // Pending-inclusive state entering the segment.  The whole sequence and
+        // segment 0 of the summary pass: the caller's h0 + beta'_0 b_prev
+        // x_prev^T (pending write of token -1); later summary segments: zero
+        // (their local state); segments of the main pass: the scanned state.
+        {
 #pragma unroll
             for (int p = 0; p < 32; ++p) hreg[p] = 0.f;
             if (MODE == kSegment) {
                 if (own_state) {
-                    const float4 *hin = reinterpret_cast<const float4 *>(
-                        a.ws_h + (((int64_t)seg * BH + cur->bh) * N + srow) * kP + c0);
+                    const float *hin = a.ws_h + ((int64_t)seg * BH + bh) * N * kP;
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const float4 v = hin[p];
-                        hreg[4 * p] = v.x;
-                        hreg[4 * p + 1] = v.y;
-                        hreg[4 * p + 2] = v.z;
-                        hreg[4 * p + 3] = v.w;
+                    for (int p = 0; p < 32; ++p) hreg[p] = hin[srow * kP + c0 + p];
+                }
+            } else if (seg == 0) {
+                const float betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
+                if (own_state) {
+                    if (a.h0) {
+#pragma unroll
+                        for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * N + srow) * kP + c0 + p];
+                    }
+                    if (a.bp0 && a.xp0) {
+                        for (int r = 0; r < R; ++r) {
+                            const float cw = betap0 * a.bp0[(bh * R + r) * N + srow];
+#pragma unroll
+                            for (int p = 0; p < 32; ++p)
+                                hreg[p] = fmaf(cw, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
+                        }
                     }
                 }
-            } else if (cur->c0 == 0) {
-                caller_state(cur->b, cur->h);
-            } else if (FLOW) {
-                ok = handoff_state();
-                if (!ok) break;
             }
             if (!SUM && own_state) store_state_half(hbuf, srow, hf, hreg);
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(kBarState, kSt);
-            if (lt == 0) mbar_arrive(bb.hrdy);  // h* for the piece's first chunk
-
-          for (int c = cur->c0; c < cur->c1; ++c, ++lc) {
+        }
+        // summary pass: the segment's transition exp(cA) Rot(-Phi) on this row's pair
+        float m_l2 = 0.f, m_cs = 1.f, m_sn = 0.f;
+        fence_proxy_async_smem();
+        named_bar(kBarState, kSt);
+        if (lt == 0) mbar_arrive(bb.hrdy);
+        bool ok = true;
+        for (int lc = 0; lc < nloc; ++lc) {
             const int sx = lc % kNX;
             const float *cAl2 = sbuf + sx * C::SB;
             const float *gam = cAl2 + Q;
@@ -1171,9 +881,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 break;
             }
             tc_fence_after();
-            // another chunk of this piece follows (else the piece's end, below,
-            // publishes h* for the next chunk)
-            const bool more = c + 1 < cur->c1;
             // ---- E. carried state: h* <- Rot(-Phi)(exp(cA_end) h* + G), fp32 in registers
             {
                 const float eA = ex2(cAl2[Q - 1]);
@@ -1194,7 +901,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const float ncs = m_cs * cs - m_sn * sn;
                     m_sn = fmaf(m_sn, cs, m_cs * sn);
                     m_cs = ncs;
-                } else if (own_state && more) {
+                } else if (own_state) {
                     store_state_half(hbuf, srow, hf, hreg);
                 }
             }
@@ -1202,7 +909,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             tc_fence_before();
             named_bar(kBarState, kSt);
             if (lt == 0) {
-                if (more) mbar_arrive(bb.hrdy);
+                mbar_arrive(bb.hrdy);
                 if (SUM) mbar_arrive(&bb.empty_x[sx]);  // x tile and scalars consumed
             }
             if (SUM) continue;
@@ -1223,9 +930,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             {
                 const int row = lq;
                 const int ti = row / R, r = row % R;
-                const int64_t t = (int64_t)c * Q + ti;
+                const int64_t t = (int64_t)(first_chunk() + lc) * Q + ti;
                 const float sc = ex2(cAl2[ti]);
-                const float Dh = cur->Dh;
                 const uint32_t yo = kColYo + (uint32_t)(lc & 1) * 64u;
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
@@ -1234,7 +940,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     tmem_ld16(tl + yo + c0 + 16 * qq, yv);
                     tmem_wait_ld();
                     if (t < T) {
-                        __nv_bfloat16 *yrow = a.y + (tok(cur->b, cur->h, t) * R + r) * kP + c0 + 16 * qq;
+                        __nv_bfloat16 *yrow = a.y + (tok(t) * R + r) * kP + c0 + 16 * qq;
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
                             const uint4 xv =
@@ -1257,29 +963,47 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             tc_fence_before();
             named_bar(kBarState, kSt);
             if (lt == 0) mbar_arrive(&bb.empty_x[sx]);
-          }
-            if (!ok) break;
-            // ---- the piece's end
-            if (SUM) {
-                // summary: the segment's local end state (pending-inclusive) into
-                // slot seg + 1, its transition exp(cA) Rot(-Phi) per pair
-                if (own_state) {
-                    float4 *dst = reinterpret_cast<float4 *>(a.ws_h + (((int64_t)seg + 1) * BH + cur->bh) * N * kP +
-                                                             srow * kP + c0);
+        }
+        if (SUM) {
+            // ---- summary: the segment's local end state (pending-inclusive) into
+            //      slot seg + 1, its transition exp(cA) Rot(-Phi) per pair
+            if (ok && own_state) {
+                float4 *dst = reinterpret_cast<float4 *>(a.ws_h + (((int64_t)seg + 1) * BH + bh) * N * kP +
+                                                         srow * kP + c0);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p)
-                        dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
-                    if (hf == 0 && (srow & 1) == 0) {
-                        const float e = ex2(m_l2);
-                        *reinterpret_cast<float2 *>(a.ws_m + ((int64_t)seg * BH + cur->bh) * N + srow) =
-                            make_float2(e * m_cs, e * m_sn);
-                    }
+                for (int p = 0; p < 8; ++p)
+                    dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
+                if (hf == 0 && (srow & 1) == 0) {
+                    const float e = ex2(m_l2);
+                    *reinterpret_cast<float2 *>(a.ws_m + ((int64_t)seg * BH + bh) * N + srow) =
+                        make_float2(e * m_cs, e * m_sn);
                 }
-            } else if (cur->c1 == a.nchunks) {
-                if (MODE == kFlow || seg == a.nseg - 1) final_state(cur->b, cur->h);  // the sequence's end
-            } else if (FLOW) {
-                publish_state();  // this CTA's head: the next CTA continues the slice
             }
+        } else if (ok && (!SEGD || seg == a.nseg - 1)) {
+            // ---- final state: plain-frame h_{T-1}, raw last token as the pending term
+            if (a.hT && own_state) {
+                float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * N + srow) * kP + c0);
+#pragma unroll
+                for (int p = 0; p < 8; ++p)
+                    dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
+            }
+            if (a.bpT && BCN) {  // the last token's normalised B, one state warp per rank row
+                const int wl = lt >> 5;
+                if (wl < R) {
+                    const int64_t src = tok(T - 1) * R * N + wl * N;
+                    float ss = 0.f;
+                    for (int n = lane; n < N; n += 32) ss = fmaf(bf(a.B, src + n), bf(a.B, src + n), ss);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    const float sc = rsqrtf(ss / N + a.eps);
+                    for (int n = lane; n < N; n += 32)
+                        a.bpT[(bh * R + wl) * N + n] = fmaf(bf(a.B, src + n) * sc, a.wB[n], a.bB[(h * R + wl) * N + n]);
+                }
+            } else if (a.bpT) {
+                for (int i = lt; i < R * N; i += kSt) a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
+            }
+            if (a.xpT)
+                for (int i = lt; i < R * kP; i += kSt) a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
         }
     }
     __syncwarp();  // reconverge the single-lane roles before the block barrier
@@ -1453,13 +1177,7 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
         a.hT = p.hT;
         a.bpT = p.bpT;
         a.xpT = p.xpT;
-        if (plan.balanced) {  // hand-off slots, then the flags (cleared here: a fresh wait per call)
-            a.flow_h = static_cast<float *>(p.ws);
-            a.flow_flag = reinterpret_cast<unsigned *>(a.flow_h + (size_t)plan.ctas * N * kP);
-            const cudaError_t e = cudaMemsetAsync(a.flow_flag, 0, (size_t)plan.ctas * sizeof(unsigned), p.stream);
-            if (e != cudaSuccess) return e;
-        }
-        return launch_pass<N, R, kFlow, GEN, BCN>(mx, mb, mc, mt, a, plan.ctas, p.stream);
+        return launch_pass<N, R, kWhole, GEN, BCN>(mx, mb, mc, mt, a, BH, p.stream);
     }
     // split sequences: summary pass over segments 0 .. nseg-2, segment scan,
     // then the main pass over all segments from the scanned states
@@ -1515,23 +1233,6 @@ TcPlan prefill_tc_plan(const Problem &p) {
     const int64_t Q = kRows / p.R;
     const int64_t nch = (p.T + Q - 1) / Q;
     const int64_t BH = p.Bt * p.H;
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    if (nsm < 1) nsm = 1;
-    // Balanced schedule: more slices than SMs (every CTA's run then spans at
-    // least one slice), indices within int, and room for the hand-off slots.
-    const size_t bal_ws = (size_t)nsm * p.N * p.P * sizeof(float) + (((size_t)nsm * 4 + 255) / 256) * 256;
-    if (p.segments == 0 && !p.no_balance && BH > nsm && BH * nch < ((int64_t)1 << 31) &&
-        (!p.ws_cap || bal_ws <= p.ws_cap)) {
-        plan.nchunks = (int)nch;
-        plan.cpseg = (int)nch;
-        plan.nseg = 1;
-        plan.launches = 1;
-        plan.ctas = nsm;
-        plan.balanced = true;
-        plan.ws_bytes = bal_ws;
-        return plan;
-    }
     int64_t S = 1;
     if (p.segments > 0) {
         S = p.segments;
@@ -1539,6 +1240,9 @@ TcPlan prefill_tc_plan(const Problem &p) {
         // Split a sequence only when it shortens the estimated critical path:
         // waves of one CTA per SM, a summary chunk costing kSumCost of a full
         // one, segments of at least kMinSegChunks chunks.
+        int dev = 0, nsm = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (nsm < 1) nsm = 1;
         auto waves = [&](int64_t ctas) { return (double)((ctas + nsm - 1) / nsm); };
         double best = waves(BH) * (double)nch;
         for (int64_t s = 2; s <= kMaxSegments && s * kMinSegChunks <= nch; ++s) {
@@ -1561,7 +1265,6 @@ TcPlan prefill_tc_plan(const Problem &p) {
     plan.nseg = (int)S;
     plan.launches = S > 1 ? 3 : 1;
     plan.ctas = BH * S;
-    plan.balanced = false;
     plan.ws_bytes = S > 1 ? (size_t)S * BH * p.N * (p.P + 1) * sizeof(float) : 0;
     return plan;
 }
@@ -1570,8 +1273,8 @@ size_t prefill_tc_workspace(const Problem &p) { return prefill_tc_plan(p).ws_byt
 
 cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
     const TcPlan plan = prefill_tc_plan(p);
-    if (plan.ws_bytes && (!p.ws || p.ws_bytes < plan.ws_bytes)) {
-        *why = "tensor-core prefill: workspace too small for this schedule";
+    if (plan.nseg > 1 && (!p.ws || p.ws_bytes < plan.ws_bytes)) {
+        *why = "tensor-core prefill: workspace too small for the split sequence";
         return cudaErrorNotSupported;
     }
     // plain instantiations unless an optional feature is on

@@ -17,7 +17,6 @@ enum : unsigned {
     kErrWaitTma = 1u << 0,
     kErrWaitMma = 1u << 1,
     kErrWaitCompute = 1u << 2,
-    kErrWaitHandoff = 1u << 3,   // a slice hand-off between two CTAs of the balanced schedule
     kErrWaitSelftest = 1u << 4,  // the self-test wait of m3_selftest_wait_timeout
 };
 

@@ -139,12 +139,12 @@ def test_scan_plan_info_host_side(m3):
     NULL result are refused, an empty batch runs nothing."""
     d = dims(m3, Bt=3, H=5, io=0)
     info = m3.scan_plan_info(d)
-    assert info == m3.PlanInfo(0, m3.KERNEL_SIMT, 1, 1, False, 15)
+    assert info == m3.PlanInfo(0, m3.KERNEL_SIMT, 1, 1, 15)
     assert info.kernel_name == "prefill_simt_kernel"
     assert m3.scan_plan_info(d, flags=m3.PLAN_STATIC).kernel == m3.KERNEL_SIMT
-    assert m3.scan_plan_info(dims(m3, Bt=0)) == m3.PlanInfo(0, m3.KERNEL_NONE, 1, 0, False, 0)
+    assert m3.scan_plan_info(dims(m3, Bt=0)) == m3.PlanInfo(0, m3.KERNEL_NONE, 1, 0, 0)
     out = m3.CPlanInfo()
-    assert m3.lib.m3_scan_plan_info(0, ctypes.byref(d), 4, ctypes.byref(out)) == 1
+    assert m3.lib.m3_scan_plan_info(0, ctypes.byref(d), 2, ctypes.byref(out)) == 1
     assert "flags" in m3.lib.m3_last_error().decode()
     assert m3.lib.m3_scan_plan_info(0, ctypes.byref(d), 0, None) == 1
     assert m3.lib.m3_scan_plan_info(m3.ALGO_TC, ctypes.byref(d), 0, ctypes.byref(out)) == 2

@@ -20,7 +20,8 @@ error over (t, r, p); bars 2e-2 for bf16 I/O, 1e-4 for fp32 I/O):
 
 Paths: the tensor-core prefill (N = 128 R = 1, N = 64 R = 4, and N = 128
 R = 4 split into segments), the SIMT prefill (fp32 I/O), and the decode
-kernels (one CTA per slice, the persistent rank-4 kernel, fp32 I/O)."""
+kernels (one CTA per slice, the persistent rank >= 2 kernel with a full grid
+and with few slices, bf16 and fp32 I/O)."""
 import math
 
 import numpy as np
@@ -165,9 +166,11 @@ def test_prefill_edge_case(name, shape, path, kind):
 
 
 DECODE_CASES = [
-    ("tiled_n128_r1", Shape(3, 40, 2, 64, 128, 1, "bf16", 71)),
-    ("stream_n128_r4", Shape(3, 40, 2, 64, 128, 4, "bf16", 72)),
-    ("f32_n64_r2", Shape(2, 40, 2, 64, 64, 2, "f32", 73)),
+    ("tiled_n128_r1", Shape(5, 40, 32, 64, 128, 1, "bf16", 71)),       # one CTA per slice
+    ("stream_n128_r4", Shape(5, 40, 32, 64, 128, 4, "bf16", 72)),      # the persistent kernel
+    ("stream_few_n128_r4", Shape(1, 40, 16, 64, 128, 4, "bf16", 74)),  # 16 slices: dependent launch
+    ("tiled_few_n64_r1", Shape(3, 40, 2, 64, 64, 1, "bf16", 75)),
+    ("stream_f32_n64_r2", Shape(2, 40, 2, 64, 64, 2, "f32", 73)),
 ]
 
 

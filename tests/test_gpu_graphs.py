@@ -54,8 +54,9 @@ def test_prefill_graph_replay_matches_eager(algo_name, segs):
 
 
 @pytest.mark.parametrize("rank", [1, 4])
-def test_decode_graph_replay_matches_eager(rank):
-    s = Shape(8, 64, 4, 64, 128, rank, "bf16", 402)
+@pytest.mark.parametrize("batch", [8, 40])  # 32 and 160 slices: rank 4 with and without dependent launch
+def test_decode_graph_replay_matches_eager(rank, batch):
+    s = Shape(batch, 64, 4, 64, 128, rank, "bf16", 402)
     pre = dev(make_prefill(s))
     nsteps = 4
     steps = make_steps(s, nsteps, device="cuda")

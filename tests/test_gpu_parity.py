@@ -112,6 +112,9 @@ DECODE = [
     Shape(2, 1, 3, 64, 64, 2, "f32", 23),
     Shape(2, 1, 2, 128, 128, 1, "f32", 24),
     Shape(2, 1, 2, 64, 256, 4, "bf16", 25),
+    Shape(5, 1, 32, 64, 64, 2, "f32", 28),      # 160 slices: the persistent kernel, fp32 I/O
+    Shape(5, 1, 32, 64, 128, 1, "f32", 29),     # 160 slices: one CTA per slice, fp32 I/O
+    Shape(1, 1, 1, 64, 128, 2, "bf16", 30),     # one slice: the persistent kernel, one CTA
     Shape(2, 1, 2, 12, 10, 3, "f32", 26),       # generic kernel
     Shape(1, 1, 2, 2, 6, 1, "f32", 27),         # generic kernel, tiny head
 ]
