@@ -32,6 +32,21 @@ template <>
 __device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
     return __bfloat162float(p[i]);
 }
+// Four consecutive values (i a multiple of 4; the row they lie in starts
+// 16-byte aligned for fp32, 8-byte aligned for bf16).
+template <typename T>
+__device__ __forceinline__ float4 ldv4(const T *p, int64_t i);
+template <>
+__device__ __forceinline__ float4 ldv4<float>(const float *p, int64_t i) {
+    return __ldg(reinterpret_cast<const float4 *>(p + i));
+}
+template <>
+__device__ __forceinline__ float4 ldv4<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p + i));
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
 template <typename T>
 __device__ __forceinline__ void stv(T *p, int64_t i, float v);
 template <>
@@ -58,20 +73,23 @@ struct SimtArgs {
 
 constexpr int kThreads = 256;
 
+// B and C rows are N + 1 floats apart in shared memory: with an odd stride,
+// threads that read the same column of consecutive rows hit distinct banks.
 __host__ __device__ inline size_t simt_smem_floats(int P, int N, int R, int Q) {
     const size_t rows = (size_t)Q * R;
-    return rows * P + 2 * rows * N + rows * rows + (size_t)N * P + 6 * (size_t)Q + 3 * (size_t)(N / 2);
+    return rows * P + 2 * rows * (N + 1) + rows * rows + (size_t)N * P + 6 * (size_t)Q + 3 * (size_t)(N / 2) +
+           (size_t)Q * (N / 2);
 }
 
 template <typename IO>
 __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<IO> a) {
     extern __shared__ float smem[];
-    const int P = a.P, N = a.N, R = a.R, Q = a.Q, K2 = N / 2;
+    const int P = a.P, N = a.N, R = a.R, Q = a.Q, K2 = N / 2, NS = N + 1;
     const int rowsmax = Q * R;
     float *Xs = smem;                       // [rows][P]
-    float *Bs = Xs + rowsmax * P;           // [rows][N]  (rotated in place)
-    float *Cs = Bs + rowsmax * N;           // [rows][N]  (rotated in place)
-    float *Pm = Cs + rowsmax * N;           // [rows][rows] masked scores
+    float *Bs = Xs + rowsmax * P;           // [rows][NS]  (rotated in place)
+    float *Cs = Bs + rowsmax * NS;          // [rows][NS]  (rotated in place)
+    float *Pm = Cs + rowsmax * NS;          // [rows][rows] masked scores
     float *hs = Pm + rowsmax * rowsmax;     // [N][P] carried plain-frame state
     float *dts = hs + N * P;                // [Q] dt
     float *cA = dts + Q;                    // [Q] chunk-local cumulative dt*A
@@ -82,6 +100,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
     float *phiE = scr + Q;                  // [N/2] chunk-end angle
     float *cosE = phiE + K2;                // [N/2]
     float *sinE = cosE + K2;                // [N/2]
+    float *phis = sinE + K2;                // [Q][N/2] chunk-local cumulative angles
 
     const int tid = threadIdx.x;
     const int64_t bh = blockIdx.x;
@@ -113,16 +132,39 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
         const int rows = L * R;
         const bool last_chunk = (t0 + L == T);
 
-        // ---- load the chunk (rows = (token, rank))
-        for (int idx = tid; idx < rows * P; idx += kThreads) {
-            const int i = idx / P, p = idx % P;
-            Xs[idx] = ldv(a.x, (tok(t0 + i / R) * R + i % R) * P + p);
+        // ---- load the chunk (rows = (token, rank)), four values per load where
+        //      the rows allow it (every load of a loop is independent)
+        if (P % 4 == 0) {
+            const int P4 = P / 4;
+#pragma unroll 4
+            for (int idx = tid; idx < rows * P4; idx += kThreads) {
+                const int i = idx / P4, p = 4 * (idx % P4);
+                *reinterpret_cast<float4 *>(Xs + i * P + p) = ldv4(a.x, (tok(t0 + i / R) * R + i % R) * P + p);
+            }
+        } else {
+            for (int idx = tid; idx < rows * P; idx += kThreads) {
+                const int i = idx / P, p = idx % P;
+                Xs[idx] = ldv(a.x, (tok(t0 + i / R) * R + i % R) * P + p);
+            }
         }
-        for (int idx = tid; idx < rows * N; idx += kThreads) {
-            const int i = idx / N, n = idx % N;
-            const int64_t g = (tok(t0 + i / R) * R + i % R) * N + n;
-            Bs[idx] = ldv(a.B, g);
-            Cs[idx] = ldv(a.C, g);
+        if (N % 4 == 0) {
+            const int N4 = N / 4;
+#pragma unroll 4
+            for (int idx = tid; idx < rows * N4; idx += kThreads) {
+                const int i = idx / N4, n = 4 * (idx % N4);
+                const int64_t g = (tok(t0 + i / R) * R + i % R) * N + n;
+                const float4 vb = ldv4(a.B, g), vc = ldv4(a.C, g);
+                float *bd = Bs + i * NS + n, *cd = Cs + i * NS + n;
+                bd[0] = vb.x; bd[1] = vb.y; bd[2] = vb.z; bd[3] = vb.w;
+                cd[0] = vc.x; cd[1] = vc.y; cd[2] = vc.z; cd[3] = vc.w;
+            }
+        } else {
+            for (int idx = tid; idx < rows * N; idx += kThreads) {
+                const int i = idx / N, n = idx % N;
+                const int64_t g = (tok(t0 + i / R) * R + i % R) * N + n;
+                Bs[i * NS + n] = ldv(a.B, g);
+                Cs[i * NS + n] = ldv(a.C, g);
+            }
         }
         for (int s = tid; s < L; s += kThreads) {
             const int64_t t = t0 + s;
@@ -142,7 +184,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             const int warp = tid >> 5, lane = tid & 31;
             for (int row = warp; row < 2 * rows; row += kThreads / 32) {
                 const bool isB = row < rows;
-                float *v = isB ? Bs + row * N : Cs + (row - rows) * N;
+                float *v = isB ? Bs + row * NS : Cs + (row - rows) * NS;
                 const int r = (isB ? row : row - rows) % R;
                 const float *w = isB ? a.wB : a.wC;
                 const float *bias = (isB ? a.bB : a.bC) + (h * R + r) * N;
@@ -155,29 +197,40 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             float run = 0.f;
             for (int s = 0; s < L; ++s) { run += cA[s]; cA[s] = run; }
         }
-        // ---- rotate B and C by the chunk-local cumulative angle (one thread per pair)
+        // ---- rotate B and C by the chunk-local cumulative angle: the angle
+        //      increments dt_s theta_s[k], their running sum over the chunk's
+        //      tokens (one thread per pair, in token order), then every (row,
+        //      pair) rotated by its token's angle in parallel
+#pragma unroll 4
+        for (int idx = tid; idx < L * K2; idx += kThreads) {
+            const int s = idx / K2, k = idx % K2;
+            phis[idx] = dts[s] * ldv(a.theta, (a.th_head ? (int64_t)h : tok(t0 + s)) * K2 + k);
+        }
+        __syncthreads();
         for (int k = tid; k < K2; k += kThreads) {
             float phi = 0.f;
             for (int s = 0; s < L; ++s) {
-                phi += dts[s] * ldv(a.theta, (a.th_head ? (int64_t)h : tok(t0 + s)) * K2 + k);
-                float sn, cs;
-                sincosf(phi, &sn, &cs);
-                for (int r = 0; r < R; ++r) {
-                    const int i = s * R + r;
-                    float u = Bs[i * N + 2 * k], v = Bs[i * N + 2 * k + 1];
-                    Bs[i * N + 2 * k] = u * cs - v * sn;
-                    Bs[i * N + 2 * k + 1] = u * sn + v * cs;
-                    u = Cs[i * N + 2 * k];
-                    v = Cs[i * N + 2 * k + 1];
-                    Cs[i * N + 2 * k] = u * cs - v * sn;
-                    Cs[i * N + 2 * k + 1] = u * sn + v * cs;
-                }
+                phi += phis[s * K2 + k];
+                phis[s * K2 + k] = phi;
             }
             phiE[k] = phi;
             float sn, cs;
             sincosf(phi, &sn, &cs);
             cosE[k] = cs;
             sinE[k] = sn;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < rows * K2; idx += kThreads) {
+            const int i = idx / K2, k = idx % K2;
+            float sn, cs;
+            sincosf(phis[(i / R) * K2 + k], &sn, &cs);
+            float u = Bs[i * NS + 2 * k], v = Bs[i * NS + 2 * k + 1];
+            Bs[i * NS + 2 * k] = u * cs - v * sn;
+            Bs[i * NS + 2 * k + 1] = u * sn + v * cs;
+            u = Cs[i * NS + 2 * k];
+            v = Cs[i * NS + 2 * k + 1];
+            Cs[i * NS + 2 * k] = u * cs - v * sn;
+            Cs[i * NS + 2 * k + 1] = u * sn + v * cs;
         }
         __syncthreads();
         const float cAe = cA[L - 1];
@@ -187,46 +240,133 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             const float g = (last_chunk && s == L - 1) ? gam[s] : ghat[s];
             wst[s] = expf(cAe - cA[s]) * g;
         }
-        // ---- (i) masked decay-weighted scores: mask applied before exp
-        for (int idx = tid; idx < rows * rows; idx += kThreads) {
-            const int i = idx / rows, j = idx % rows;
-            const int ti = i / R, tj = j / R;
-            float v = 0.f;
-            if (tj <= ti) {
-                float dot = 0.f;
-                for (int n = 0; n < N; ++n) dot += Cs[i * N + n] * Bs[j * N + n];
-                const float coef = (ti == tj) ? gam[ti] : ghat[tj];
-                v = dot * expf(cA[ti] - cA[tj]) * coef;
+        // ---- (i) masked decay-weighted scores: mask applied before exp.  Each
+        //      thread owns a 4 x 4 tile of rows i = it + TI a, columns
+        //      j = jt + TI b (a, b < 4): 16 products per 8 shared-memory loads
+        const int TI = (rows + 3) / 4;
+        for (int tt = tid; tt < TI * TI; tt += kThreads) {
+            const int it = tt / TI, jt = tt % TI;
+            float acc[4][4] = {};
+            for (int n = 0; n < N; ++n) {
+                float c[4], bv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = it + TI * q, j = jt + TI * q;
+                    c[q] = i < rows ? Cs[i * NS + n] : 0.f;
+                    bv[q] = j < rows ? Bs[j * NS + n] : 0.f;
+                }
+#pragma unroll
+                for (int qa = 0; qa < 4; ++qa)
+#pragma unroll
+                    for (int qb = 0; qb < 4; ++qb) acc[qa][qb] = fmaf(c[qa], bv[qb], acc[qa][qb]);
             }
-            Pm[idx] = v;
+#pragma unroll
+            for (int qa = 0; qa < 4; ++qa)
+#pragma unroll
+                for (int qb = 0; qb < 4; ++qb) {
+                    const int i = it + TI * qa, j = jt + TI * qb;
+                    if (i >= rows || j >= rows) continue;
+                    const int ti = i / R, tj = j / R;
+                    float v = 0.f;
+                    if (tj <= ti) {
+                        const float coef = (ti == tj) ? gam[ti] : ghat[tj];
+                        v = acc[qa][qb] * expf(cA[ti] - cA[tj]) * coef;
+                    }
+                    Pm[i * rows + j] = v;
+                }
         }
         __syncthreads();
-        // ---- outputs: (i) diagonal block + (iv) carried-state readout + skip
-        for (int idx = tid; idx < rows * P; idx += kThreads) {
-            const int i = idx / P, p = idx % P;
-            float acc = 0.f;
-            for (int j = 0; j < rows; ++j) acc += Pm[i * rows + j] * Xs[j * P + p];
-            float off = 0.f;
-            for (int n = 0; n < N; ++n) off += Cs[i * N + n] * hs[n * P + p];
-            const float yv = acc + expf(cA[i / R]) * off + Dh * Xs[idx];
-            stv(a.y, (tok(t0 + i / R) * R + i % R) * P + p, yv);
-        }
-        __syncthreads();
-        // ---- (ii)+(iii): h* <- Rot(-Phi)(exp(cA_end) h* + G)
-        const float eA = expf(cAe);
-        for (int idx = tid; idx < K2 * P; idx += kThreads) {
-            const int k = idx / P, p = idx % P;
-            float g0 = 0.f, g1 = 0.f;
+        // ---- outputs: (i) diagonal block + (iv) carried-state readout + skip,
+        //      4 x 4 tiles of rows i = it + TI a and columns p = pt + TP b
+        const int TP = (P + 3) / 4;
+        for (int tt = tid; tt < TI * TP; tt += kThreads) {
+            const int it = tt / TP, pt = tt % TP;
+            float dg[4][4] = {}, of[4][4] = {};
             for (int j = 0; j < rows; ++j) {
-                const float wx = wst[j / R] * Xs[j * P + p];
-                g0 += Bs[j * N + 2 * k] * wx;
-                g1 += Bs[j * N + 2 * k + 1] * wx;
+                float pm[4], xv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = it + TI * q, p = pt + TP * q;
+                    pm[q] = i < rows ? Pm[i * rows + j] : 0.f;
+                    xv[q] = p < P ? Xs[j * P + p] : 0.f;
+                }
+#pragma unroll
+                for (int qa = 0; qa < 4; ++qa)
+#pragma unroll
+                    for (int qb = 0; qb < 4; ++qb) dg[qa][qb] = fmaf(pm[qa], xv[qb], dg[qa][qb]);
             }
-            const float u = eA * hs[(2 * k) * P + p] + g0;
-            const float v = eA * hs[(2 * k + 1) * P + p] + g1;
-            const float cs = cosE[k], sn = sinE[k];
-            hs[(2 * k) * P + p] = u * cs + v * sn;
-            hs[(2 * k + 1) * P + p] = -u * sn + v * cs;
+            for (int n = 0; n < N; ++n) {
+                float c[4], hv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = it + TI * q, p = pt + TP * q;
+                    c[q] = i < rows ? Cs[i * NS + n] : 0.f;
+                    hv[q] = p < P ? hs[n * P + p] : 0.f;
+                }
+#pragma unroll
+                for (int qa = 0; qa < 4; ++qa)
+#pragma unroll
+                    for (int qb = 0; qb < 4; ++qb) of[qa][qb] = fmaf(c[qa], hv[qb], of[qa][qb]);
+            }
+#pragma unroll
+            for (int qa = 0; qa < 4; ++qa) {
+                const int i = it + TI * qa;
+                if (i >= rows) continue;
+                const float ei = expf(cA[i / R]);
+#pragma unroll
+                for (int qb = 0; qb < 4; ++qb) {
+                    const int p = pt + TP * qb;
+                    if (p >= P) continue;
+                    const float yv = dg[qa][qb] + ei * of[qa][qb] + Dh * Xs[i * P + p];
+                    stv(a.y, (tok(t0 + i / R) * R + i % R) * P + p, yv);
+                }
+            }
+        }
+        __syncthreads();
+        // ---- (ii)+(iii): h* <- Rot(-Phi)(exp(cA_end) h* + G), tiles of 2 pairs
+        //      k = kt + TK a (a < 2) by 4 columns p = pt + TP b
+        const float eA = expf(cAe);
+        const int TK = (K2 + 1) / 2;
+        for (int tt = tid; tt < TK * TP; tt += kThreads) {
+            const int kt = tt / TP, pt = tt % TP;
+            float g[2][2][4] = {};  // [pair][row of the pair][column]
+            for (int j = 0; j < rows; ++j) {
+                const float w = wst[j / R];
+                float wx[4], bu[2], bv[2];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int p = pt + TP * q;
+                    wx[q] = p < P ? w * Xs[j * P + p] : 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int k = kt + TK * q;
+                    bu[q] = k < K2 ? Bs[j * NS + 2 * k] : 0.f;
+                    bv[q] = k < K2 ? Bs[j * NS + 2 * k + 1] : 0.f;
+                }
+#pragma unroll
+                for (int qa = 0; qa < 2; ++qa)
+#pragma unroll
+                    for (int qb = 0; qb < 4; ++qb) {
+                        g[qa][0][qb] = fmaf(bu[qa], wx[qb], g[qa][0][qb]);
+                        g[qa][1][qb] = fmaf(bv[qa], wx[qb], g[qa][1][qb]);
+                    }
+            }
+#pragma unroll
+            for (int qa = 0; qa < 2; ++qa) {
+                const int k = kt + TK * qa;
+                if (k >= K2) continue;
+                const float cs = cosE[k], sn = sinE[k];
+#pragma unroll
+                for (int qb = 0; qb < 4; ++qb) {
+                    const int p = pt + TP * qb;
+                    if (p >= P) continue;
+                    const float u = eA * hs[(2 * k) * P + p] + g[qa][0][qb];
+                    const float v = eA * hs[(2 * k + 1) * P + p] + g[qa][1][qb];
+                    hs[(2 * k) * P + p] = u * cs + v * sn;
+                    hs[(2 * k + 1) * P + p] = -u * sn + v * cs;
+                }
+            }
         }
         __syncthreads();
     }
