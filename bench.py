@@ -69,6 +69,7 @@ def parse():
                     help="profiling case: only run --case-launches launches of one kernel at --case-batch "
                          "(for ncu captures; prints no bench line)")
     ap.add_argument("--case-batch", type=int, default=None, help="batch of the profiling case")
+    ap.add_argument("--case-seqlen", type=int, default=None, help="sequence length of the profiling case")
     ap.add_argument("--case-launches", type=int, default=3, help="launches of the profiling case")
     return ap.parse_args()
 
@@ -84,7 +85,7 @@ def run_case(args):
     keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
     if args.case == "prefill":
         s = WORKLOADS[args.workload]
-        s = s.with_(batch=args.case_batch or s.batch)
+        s = s.with_(batch=args.case_batch or s.batch, seqlen=args.case_seqlen or s.seqlen)
         inp = make_prefill(s, device="cuda")
         for _ in range(args.case_launches):
             m3.scan_fwd(*(inp[k] for k in keys), None)

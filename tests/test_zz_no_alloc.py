@@ -50,3 +50,24 @@ def test_static_scratch_refuses_oversize():
     y_ref, _ = m3.scan_fwd(*(inp[k] for k in KEYS), None)
     m3.stream_status()
     assert torch.equal(y, y_ref)
+
+
+def test_static_plan_reports_the_capped_segment_choice():
+    """Where the workspace entry point's own segment choice would not fit the
+    scratch, the static entry point splits into fewer segments; the plan
+    query with M3_PLAN_STATIC says so, and both calls agree within the bf16
+    bar (they differ only in where the sequence is cut)."""
+    # 30 sequences of 2048 chunks: the free choice is 29 segments (27 MiB of
+    # per-segment states), the scratch admits 14
+    s = Shape(1, 65536, 30, 64, 128, 4, "bf16", 75)
+    free = m3.scan_plan_info(_dims(s))
+    capped = m3.scan_plan_info(_dims(s), flags=m3.PLAN_STATIC)
+    assert free.workspace_bytes > 24 << 20 >= capped.workspace_bytes > 0
+    assert 1 < capped.segments < free.segments
+    inp = {k: v.to(DEV) for k, v in make_prefill(s).items()}
+    y_ref, f_ref = m3.scan_fwd(*(inp[k] for k in KEYS), None)
+    y, f = m3.scan_fwd_static(*(inp[k] for k in KEYS), None)
+    m3.stream_status()
+    ey = ((y.float() - y_ref.float()).norm() / y_ref.float().norm()).item()
+    eh = ((f.h - f_ref.h).norm() / f_ref.h.norm()).item()
+    assert ey < 1e-2 and eh < 1e-2, (ey, eh)
