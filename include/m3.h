@@ -131,9 +131,12 @@ typedef struct m3_bcnorm {
 
 /* Prefill kernel selection for m3_scan_fwd_algo. */
 typedef enum m3_algo {
-    M3_ALGO_AUTO = 0,   /* tensor-core path for bf16 where supported, else SIMT */
+    M3_ALGO_AUTO = 0,   /* tensor-core path where supported, else SIMT            */
     M3_ALGO_SIMT = 1,   /* fp32 CUDA-core chunked scan (any supported size)      */
-    M3_ALGO_TC = 2      /* tcgen05/TMEM/TMA chunked scan (bf16 only)             */
+    M3_ALGO_TC = 2      /* tcgen05/TMEM chunked scan: bf16 I/O (headdim 64,
+                         * dstate 64 or 128, rank 1, 2 or 4), or fp32 I/O
+                         * (headdim 64, dstate 64, rank 1, 2 or 4, no forced
+                         * segments)                                           */
 } m3_algo;
 
 /* The tensor-core path forced to split every sequence into s >= 1 segments
@@ -169,7 +172,12 @@ M3_API m3_status m3_scan_plan(int algo, const m3_dims *d, size_t *workspace_byte
 typedef enum m3_kernel {
     M3_KERNEL_NONE = 0,  /* nothing to run (batch = 0)                    */
     M3_KERNEL_SIMT = 1,  /* the fp32 CUDA-core chunked scan               */
-    M3_KERNEL_TC = 2     /* the tcgen05/TMEM/TMA chunked scan (bf16 I/O)  */
+    M3_KERNEL_TC = 2,    /* the tcgen05/TMEM/TMA chunked scan (bf16 I/O)  */
+    M3_KERNEL_TC32 = 3   /* the tcgen05/TMEM chunked scan for fp32 I/O:
+                          * every product operand split into bf16 high and
+                          * low halves, three MMAs per product (about 2^-16
+                          * relative error), one CTA per sequence and head,
+                          * no workspace                                    */
 } m3_kernel;
 
 typedef struct m3_plan_info {
@@ -338,8 +346,9 @@ M3_API m3_status m3_step_bcnorm(const m3_dims *d, const m3_bcnorm *bcn,
  * recorded failure is cleared.  Failures are recorded per device, not per
  * stream: the call reports (and clears) a wait that gave up in a kernel of
  * any stream of the current device, whatever `stream` is.  The code in the
- * message tells which wait: 0x1 a tile copy, 0x2 a tensor-core MMA, 0x4 the
- * other warps of the prefill CTA, 0x10 the self-test; the same bits shifted
+ * message tells which wait: 0x1 a tile copy, 0x2 a tensor-core MMA (of either
+ * prefill kernel), 0x4 the other warps of the prefill CTA, 0x10 the
+ * self-test; the same bits shifted
  * left by 8 come from the decode kernels.  A device-side wait gives up only on
  * a library bug; this call exists so that such a failure surfaces as a status
  * instead of a hang.
@@ -360,7 +369,8 @@ M3_API m3_status m3_selftest_wait_timeout(void *stream);
 /* Message describing the calling thread's most recent failure ("" if none). */
 M3_API const char *m3_last_error(void);
 
-/* ABI version of this header (major * 100 + minor): 101 adds m3_scan_plan_info. */
+/* ABI version of this header (major * 100 + minor): 101 adds m3_scan_plan_info,
+ * 102 the fp32 tensor-core prefill (M3_KERNEL_TC32). */
 M3_API int m3_version(void);
 
 #ifdef __cplusplus

@@ -22,7 +22,7 @@ M3_F32, M3_BF16 = 0, 1
 M3_FLAG_A_PER_TOKEN = 1
 M3_FLAG_THETA_PER_HEAD = 2
 ALGO_AUTO, ALGO_SIMT, ALGO_TC = 0, 1, 2
-KERNEL_NONE, KERNEL_SIMT, KERNEL_TC = 0, 1, 2
+KERNEL_NONE, KERNEL_SIMT, KERNEL_TC, KERNEL_TC32 = 0, 1, 2, 3
 PLAN_STATIC = 1
 
 
@@ -224,14 +224,15 @@ def scan_plan(dims: Dims, algo: int = ALGO_AUTO) -> Plan:
 
 class PlanInfo(NamedTuple):
     workspace_bytes: int
-    kernel: int     # KERNEL_SIMT or KERNEL_TC (KERNEL_NONE: nothing to run)
+    kernel: int     # KERNEL_SIMT, KERNEL_TC or KERNEL_TC32 (KERNEL_NONE: nothing to run)
     segments: int   # per sequence (1 = not split)
     launches: int   # kernel launches of one call
     ctas: int       # CTAs of the (main) launch
 
     @property
     def kernel_name(self) -> str:
-        return {KERNEL_NONE: "none", KERNEL_SIMT: "prefill_simt_kernel", KERNEL_TC: "prefill_tc_kernel"}[self.kernel]
+        return {KERNEL_NONE: "none", KERNEL_SIMT: "prefill_simt_kernel", KERNEL_TC: "prefill_tc_kernel",
+                KERNEL_TC32: "prefill_tc32_kernel"}[self.kernel]
 
 
 def scan_plan_info(dims: Dims, algo: int = ALGO_AUTO, flags: int = 0) -> PlanInfo:

@@ -154,6 +154,12 @@ m3_status check_bcnorm(const m3_dims *d, const m3_bcnorm *bcn, Range yr) {
     return M3_OK;
 }
 
+// The tensor-core kernel for p's I/O type (bf16: prefill_tc, fp32:
+// prefill_tc32) and whether it covers p.
+bool tc_supported(const m3::Problem &p, const char **why) {
+    return p.bf16 ? m3::prefill_tc_supported(p, why) : m3::prefill_tc32_supported(p, why);
+}
+
 m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
                     const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
                     void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream,
@@ -198,7 +204,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
 
     const char *why = nullptr;
     const char *tc_why = nullptr;
-    const bool tc_ok = m3::prefill_tc_supported(p, &tc_why);
+    const bool tc_ok = tc_supported(p, &tc_why);
     bool use_tc = false;
     if (algo == M3_ALGO_TC) {
         if (!tc_ok) return fail(M3_ERR_UNSUPPORTED, "%s", tc_why ? tc_why : "tensor-core path unsupported");
@@ -206,7 +212,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
     } else if (algo == M3_ALGO_AUTO) {
         use_tc = tc_ok;
     }
-    if (use_tc) {
+    if (use_tc && p.bf16) {  // the fp32 kernel needs no workspace
         if (static_ws) {
             p.ws_cap = m3::static_scratch_bytes();
             const size_t need = m3::prefill_tc_workspace(p);
@@ -225,9 +231,14 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
             if (need && !aligned16(ws)) return fail(M3_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
         }
     }
-    cudaError_t e = use_tc ? m3::launch_prefill_tc(p, &why) : m3::launch_prefill_simt(p, &why);
+    cudaError_t e = !use_tc ? m3::launch_prefill_simt(p, &why)
+                    : p.bf16 ? m3::launch_prefill_tc(p, &why)
+                             : m3::launch_prefill_tc32(p, &why);
     if (e == cudaErrorNotSupported && why) return fail(M3_ERR_UNSUPPORTED, "%s", why);
-    if (e != cudaSuccess) return cuda_fail(e, use_tc ? "m3_scan_fwd (tensor-core kernel)" : "m3_scan_fwd (SIMT kernel)");
+    if (e != cudaSuccess)
+        return cuda_fail(e, !use_tc ? "m3_scan_fwd (SIMT kernel)"
+                            : p.bf16 ? "m3_scan_fwd (tensor-core kernel)"
+                                     : "m3_scan_fwd (fp32 tensor-core kernel)");
     return M3_OK;
 }
 
@@ -240,7 +251,7 @@ m3_status set_cuda_error(cudaError_t e, const char *where) { return cuda_fail(e,
 
 extern "C" {
 
-int m3_version(void) { return 101; }
+int m3_version(void) { return 102; }
 
 const char *m3_last_error(void) { return g_err.c_str(); }
 
@@ -264,11 +275,17 @@ m3_status m3_scan_plan_info(int algo, const m3_dims *d, int flags, m3_plan_info 
         p.bf16 = d->io == M3_BF16;
         p.segments = forced;
         const char *why = nullptr;
-        const bool tc = base != M3_ALGO_SIMT && m3::prefill_tc_supported(p, &why);
+        const bool tc = base != M3_ALGO_SIMT && tc_supported(p, &why);
         if (base == M3_ALGO_TC && !tc)
             return fail(M3_ERR_UNSUPPORTED, "%s", why ? why : "tensor-core path unsupported");
         if (!tc) {
             info->kernel = M3_KERNEL_SIMT;
+            info->launches = 1;
+            info->ctas = d->batch * d->nheads;
+            return M3_OK;
+        }
+        if (!p.bf16) {  // fp32 tensor-core kernel: one CTA per sequence and head, no workspace
+            info->kernel = M3_KERNEL_TC32;
             info->launches = 1;
             info->ctas = d->batch * d->nheads;
             return M3_OK;
@@ -371,7 +388,10 @@ m3_status m3_stream_status(void *stream) {
         unsigned dcode = 0;
         e = m3::read_decode_error(&dcode);
         if (e != cudaSuccess) return cuda_fail(e, "m3_stream_status");
-        code |= dcode << 8;
+        unsigned tcode = 0;
+        e = m3::read_tc32_error(&tcode);
+        if (e != cudaSuccess) return cuda_fail(e, "m3_stream_status");
+        code |= tcode | (dcode << 8);
         if (code) {
             char buf[128];
             std::snprintf(buf, sizeof buf, "a bounded device-side wait gave up (code 0x%x)", code);

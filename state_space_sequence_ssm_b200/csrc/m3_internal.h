@@ -46,6 +46,9 @@ bool prefill_tc_supported(const Problem &p, const char **why);
 TcPlan prefill_tc_plan(const Problem &p);
 size_t prefill_tc_workspace(const Problem &p);
 cudaError_t launch_prefill_tc(const Problem &p, const char **why);
+// fp32 I/O on the tensor cores (bf16 hi/lo operand halves); no workspace.
+bool prefill_tc32_supported(const Problem &p, const char **why);
+cudaError_t launch_prefill_tc32(const Problem &p, const char **why);
 cudaError_t launch_step(const Problem &p, const char **why);
 // The library's own device scratch for m3_scan_fwd_static: its address on the
 // current device (looked up once per device) and its size.
@@ -58,6 +61,8 @@ cudaError_t launch_wait_selftest(cudaStream_t stream);
 cudaError_t read_device_error(unsigned *code, cudaStream_t stream);
 // Read and clear the decode kernels' device error word (after a sync).
 cudaError_t read_decode_error(unsigned *code);
+// Read and clear the fp32 tensor-core prefill's device error word (after a sync).
+cudaError_t read_tc32_error(unsigned *code);
 // Record the calling thread's failure message (m3_last_error) and return `s`.
 m3_status set_error(m3_status s, const char *msg);
 m3_status set_cuda_error(cudaError_t e, const char *where);

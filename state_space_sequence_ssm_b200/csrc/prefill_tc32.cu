@@ -1,0 +1,562 @@
+// prefill_tc32.cu -- tcgen05 chunked prefill for fp32 I/O at the fp32 bar.
+//
+// The chunked algorithm of "La dualità: Mamba-2 e Mamba-3" (section "Perché
+// conviene: i tensor core": the masked block inside a chunk, the chunk state,
+// the recurrence between chunks and the carried state read out through the
+// decay), with the Mamba-3 pieces of "Знакомство с Mamba-3" (sections 1-3):
+// the trapezoid's previous-token write folded into the off-diagonal weight
+// gamma_hat_s = lam_s dt_s + (1 - lam_{s+1}) dt_{s+1}, the pair rotations of
+// B and C by the chunk-local cumulative angle, and rank-R MIMO rows -- the
+// same algebra as the bf16 tensor-core kernel, for fp32 inputs and outputs.
+//
+// The page's case for moving this work onto tensor cores is their throughput
+// over generic fp32 units (same page, same section).  To keep fp32 accuracy on
+// bf16 tensor cores every operand v of the four chunk products is split into
+// two bf16 values, hi = bf16(v) and lo = bf16(v - hi) (v - hi - lo is below
+// 2^-17 of v), and every product A B is taken as hi.hi + hi.lo + lo.hi in the
+// fp32 accumulators: three MMAs where the bf16 kernel takes one, the dropped
+// lo.lo term and the splits' rounding about 2^-16 of the product.  Angles,
+// decays, the decay mask, the carried state and the epilogue stay fp32.
+//
+// One CTA of 256 threads per (batch, head) walks its sequence in chunks of
+// 128 rows (Q = 128 / R tokens x R ranks), in synchronous phases per chunk:
+//   1. per-token scalars, the chunk-local scan of dt*A, the angle table;
+//   2. B, C (BC-normed first when the prologue is on) rotated in fp32 and
+//      split into 128B-swizzled bf16 hi/lo tiles (K-major), x and w o x
+//      split likewise (MN-major);
+//   3. one thread issues S = C~ B~^T, G = B~^T (w o X) and Yo = C~ h* (three
+//      terms each);
+//   4. the decay mask S -> P in fp32, written back to TMEM as hi and lo bf16;
+//      Yd = P X (three terms, P read from TMEM);
+//   5. the carried state h* <- Rot(-Phi)(exp(cA_end) h* + G) in fp32
+//      registers, its hi/lo tiles for the next chunk's Yo;
+//   6. y = Yd + exp(cA_t) Yo + D x, stored in fp32.
+// Built for headdim 64 and dstate 64 (the tiles of one chunk then take
+// 160 KB of shared memory); other fp32 sizes run the SIMT kernel.  Every wait
+// is bounded and reports through the library's device error word.
+#include <cuda_bf16.h>
+
+#include "bcnorm.cuh"
+#include "m3_internal.h"
+#include "tc_primitives.cuh"
+
+namespace m3 {
+
+// This kernel's failure word (an MMA wait that gave up: kErrWaitMma), read and
+// cleared by read_tc32_error() on the host.
+__device__ unsigned g_tc32_error;
+
+namespace {
+using namespace tc;
+
+constexpr int kP = 64, kN = 64, kK2 = kN / 2;
+constexpr int kRows = 128;   // rows per chunk = MMA M
+constexpr int kThreads = 256;
+constexpr uint32_t kTile = kRows * 128;  // one bf16 tile of 128 rows x 64 columns (16 KB)
+// TMEM columns: S [0,128), G [128,192), Yo [192,256), Yd [256,320),
+// P hi [320,384), P lo [384,448) (P as packed bf16 pairs)
+constexpr uint32_t kColS = 0, kColG = 128, kColYo = 192, kColYd = 256, kColPh = 320, kColPl = 384;
+constexpr uint32_t kTmemCols = 512;
+
+// shared memory: tiles (hi, lo) of C~, B~, X, w o X (each 128 x 64 bf16),
+// h* (64 x 64 bf16), the angle table, the per-token scalars, barriers
+constexpr uint32_t OFF_C = 0, OFF_B = OFF_C + 2 * kTile, OFF_X = OFF_B + 2 * kTile, OFF_XW = OFF_X + 2 * kTile;
+constexpr uint32_t H_TILE = kN * 128;
+constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;
+constexpr uint32_t OFF_PHI = OFF_H + 2 * H_TILE;                  // phi [128][K2] fp32
+constexpr uint32_t OFF_SCAL = OFF_PHI + kRows * kK2 * 4;          // dts, gam, ghat, cA, wst [128]; cos, sin [K2]; wtot [8]
+constexpr uint32_t OFF_BAR = OFF_SCAL + (5 * kRows + 2 * kK2 + 8) * 4;
+constexpr uint32_t OFF_MISC = OFF_BAR + 4 * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct Tc32Args {
+    int64_t T, H;
+    const float *x, *B, *C, *dt, *lam, *theta, *A, *D;
+    int a_tok, th_head;
+    const float *h0, *bp0, *xp0;
+    const float *wB, *wC, *bB, *bC;  // BC-norm prologue (wB == nullptr: off)
+    float eps;
+    float *y, *hT, *bpT, *xpT;
+};
+
+// v = hi + lo, both bf16: the pair for 8 consecutive values (two uint4 of packed pairs)
+__device__ __forceinline__ void split8(const float (&v)[8], uint4 &hi, uint4 &lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        const float2 hf = __bfloat1622float2(hh);
+        const __nv_bfloat162 ll = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+        h[e] = *reinterpret_cast<const uint32_t *>(&hh);
+        l[e] = *reinterpret_cast<const uint32_t *>(&ll);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// hi and lo of a pair, packed (low half = first value)
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(hh);
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&hh);
+    lo = *reinterpret_cast<const uint32_t *>(&ll);
+}
+
+// hi/lo of 32 state values (row n, columns 32 half ..) into the MN-major h* tiles
+__device__ __forceinline__ void store_state32(uint8_t *hhi, uint8_t *hlo, int n, int half, const float (&h)[32]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = h[8 * j + e];
+        uint4 hi, lo;
+        split8(v, hi, lo);
+        *reinterpret_cast<uint4 *>(hhi + sw128(n, 4 * half + j)) = hi;
+        *reinterpret_cast<uint4 *>(hlo + sw128(n, 4 * half + j)) = lo;
+    }
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Args a) {
+    constexpr int Q = kRows / R;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *Chi = smem + OFF_C, *Clo = Chi + kTile, *Bhi = smem + OFF_B, *Blo = Bhi + kTile;
+    uint8_t *Xhi = smem + OFF_X, *Xlo = Xhi + kTile, *XWhi = smem + OFF_XW, *XWlo = XWhi + kTile;
+    uint8_t *Hhi = smem + OFF_H, *Hlo = Hhi + H_TILE;
+    float *phi = reinterpret_cast<float *>(smem + OFF_PHI);
+    float *dts = reinterpret_cast<float *>(smem + OFF_SCAL), *gam = dts + kRows, *ghat = gam + kRows;
+    float *cA = ghat + kRows, *wst = cA + kRows, *cosE = wst + kRows, *sinE = cosE + kK2, *wtot = sinE + kK2;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);  // [0] S/G/Yo, [1] Yd, [2] drain
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    unsigned *err = &g_tc32_error;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, hf = warp >> 2;  // TMEM lane quarter, column half
+    const int lq = 32 * wq + lane;            // TMEM lane = chunk row
+    const int c0 = 32 * hf;                   // first of this thread's 32 columns
+    const bool own_state = lane < 16;         // G (M = 64): lanes 0-15 of each quarter
+    const int srow = wq * 16 + lane;          // its state row
+    const int64_t bh = blockIdx.x, T = a.T, H = a.H;
+    const int64_t b = bh / H, h = bh % H;
+    auto tok = [&](int64_t t) { return (b * T + t) * H + h; };
+    const float Dh = a.D[h];
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
+
+    // carried state (plain frame, pending-inclusive): h0 + beta'_0 b_prev x_prev^T
+    float hreg[32];
+#pragma unroll
+    for (int p = 0; p < 32; ++p) hreg[p] = 0.f;
+    if (own_state && T > 0) {
+        const float betap0 = (1.f - a.lam[tok(0)]) * a.dt[tok(0)];
+        if (a.h0) {
+#pragma unroll
+            for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * kN + srow) * kP + c0 + p];
+        }
+        if (a.bp0 && a.xp0) {
+            for (int r = 0; r < R; ++r) {
+                const float cw = betap0 * a.bp0[(bh * R + r) * kN + srow];
+#pragma unroll
+                for (int p = 0; p < 32; ++p) hreg[p] = fmaf(cw, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
+            }
+        }
+    }
+    if (own_state) store_state32(Hhi, Hlo, srow, hf, hreg);
+
+    constexpr uint32_t idS = idesc_bf16(kRows, kRows, 0, 0);
+    constexpr uint32_t idG = idesc_bf16(kN, kP, 1, 1);
+    constexpr uint32_t idY = idesc_bf16(kRows, kP, 0, 1);
+    const int nch = (int)((T + Q - 1) / Q);
+    bool ok = true;
+    bool issued = false;  // MMAs may be in flight
+    for (int c = 0; c < nch && ok; ++c) {
+        const int64_t t0 = (int64_t)c * Q;
+        // ---- 1. per-token scalars and the chunk-local scan of dt*A
+        float acc = 0.f;
+        if (tid < Q) {
+            const int64_t t = t0 + tid;
+            float d = 0.f, l = 0.f, nx = 0.f, av = 0.f;
+            if (t < T) {
+                d = a.dt[tok(t)];
+                l = a.lam[tok(t)];
+                av = a.a_tok ? a.A[tok(t)] : a.A[h];
+                if (t + 1 < T) nx = (1.f - a.lam[tok(t + 1)]) * a.dt[tok(t + 1)];
+            }
+            dts[tid] = d;
+            gam[tid] = l * d;
+            ghat[tid] = l * d + nx;
+            acc = d * av;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, acc, off);
+                if (lane >= off) acc += v;
+            }
+            if (lane == 31) wtot[warp] = acc;
+        }
+        __syncthreads();
+        if (tid < Q) {
+            float off = 0.f;
+            for (int w = 0; w < warp; ++w) off += wtot[w];
+            cA[tid] = acc + off;
+        }
+        // angle increments dt_s theta_s[k]
+        for (int idx = tid; idx < Q * kK2; idx += kThreads) {
+            const int s = idx / kK2, k = idx % kK2;
+            const int64_t t = t0 + s;
+            phi[idx] = t < T ? dts[s] * a.theta[(a.th_head ? (int64_t)h : tok(t)) * kK2 + k] : 0.f;
+        }
+        __syncthreads();
+        // their running sum per pair; the chunk's total angle
+        if (tid < kK2) {
+            float run = 0.f;
+            for (int s = 0; s < Q; ++s) {
+                run += phi[s * kK2 + tid];
+                phi[s * kK2 + tid] = run;
+            }
+            float sn, cs;
+            sincosf(run, &sn, &cs);
+            cosE[tid] = cs;
+            sinE[tid] = sn;
+        }
+        if (tid >= kThreads - Q) {  // chunk-state weights exp(cA_end - cA_s) ghat_s
+            const int s = tid - (kThreads - Q);
+            wst[s] = expf(cA[Q - 1] - cA[s]) * ghat[s];
+        }
+        __syncthreads();
+
+        // ---- 2. rotated B, C and the value rows as hi/lo tiles (16-byte chunk j of row i)
+        for (int it = tid; it < kRows * 8; it += kThreads) {
+            const int i = it >> 3, j = it & 7;
+            const int s = i / R, r = i % R;
+            const int64_t t = t0 + s;
+            float vb[8], vc[8], vx[8], vw[8];
+            if (t < T) {
+                const int64_t row = tok(t) * R + r;
+                const float4 b0 = *reinterpret_cast<const float4 *>(a.B + row * kN + 8 * j);
+                const float4 b1 = *reinterpret_cast<const float4 *>(a.B + row * kN + 8 * j + 4);
+                const float4 q0 = *reinterpret_cast<const float4 *>(a.C + row * kN + 8 * j);
+                const float4 q1 = *reinterpret_cast<const float4 *>(a.C + row * kN + 8 * j + 4);
+                const float4 x0 = *reinterpret_cast<const float4 *>(a.x + row * kP + 8 * j);
+                const float4 x1 = *reinterpret_cast<const float4 *>(a.x + row * kP + 8 * j + 4);
+                float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                float cc[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                if (a.wB) {  // BC-norm: the row's RMS over its 8 lanes, weight and bias
+                    const unsigned grp = 0xffu << (lane & 24);
+                    float sb = 0.f, sq = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        sb = fmaf(bb[e], bb[e], sb);
+                        sq = fmaf(cc[e], cc[e], sq);
+                    }
+#pragma unroll
+                    for (int o = 1; o < 8; o <<= 1) {
+                        sb += __shfl_xor_sync(grp, sb, o);
+                        sq += __shfl_xor_sync(grp, sq, o);
+                    }
+                    const float kb = rsqrtf(sb / (float)kN + a.eps), kc = rsqrtf(sq / (float)kN + a.eps);
+                    const float *biB = a.bB + (h * R + r) * kN + 8 * j, *biC = a.bC + (h * R + r) * kN + 8 * j;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        bb[e] = fmaf(bb[e] * kb, a.wB[8 * j + e], biB[e]);
+                        cc[e] = fmaf(cc[e] * kc, a.wC[8 * j + e], biC[e]);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {  // pair k = 4 j + e: rotate by +phi_s[k]
+                    float sn, cs;
+                    sincosf(phi[s * kK2 + 4 * j + e], &sn, &cs);
+                    vb[2 * e] = bb[2 * e] * cs - bb[2 * e + 1] * sn;
+                    vb[2 * e + 1] = bb[2 * e] * sn + bb[2 * e + 1] * cs;
+                    vc[2 * e] = cc[2 * e] * cs - cc[2 * e + 1] * sn;
+                    vc[2 * e + 1] = cc[2 * e] * sn + cc[2 * e + 1] * cs;
+                }
+                const float w = wst[s];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    vx[e] = xx[e];
+                    vw[e] = w * xx[e];
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) vb[e] = vc[e] = vx[e] = vw[e] = 0.f;
+            }
+            const uint32_t off = sw128((uint32_t)i, (uint32_t)j);
+            uint4 hi, lo;
+            split8(vb, hi, lo);
+            *reinterpret_cast<uint4 *>(Bhi + off) = hi;
+            *reinterpret_cast<uint4 *>(Blo + off) = lo;
+            split8(vc, hi, lo);
+            *reinterpret_cast<uint4 *>(Chi + off) = hi;
+            *reinterpret_cast<uint4 *>(Clo + off) = lo;
+            split8(vx, hi, lo);
+            *reinterpret_cast<uint4 *>(Xhi + off) = hi;
+            *reinterpret_cast<uint4 *>(Xlo + off) = lo;
+            split8(vw, hi, lo);
+            *reinterpret_cast<uint4 *>(XWhi + off) = hi;
+            *reinterpret_cast<uint4 *>(XWlo + off) = lo;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- 3. S = C~ B~^T, G = B~^T (w o X), Yo = C~ h*: hi.hi + hi.lo + lo.hi
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t ch[2] = {smem_u32(Chi), smem_u32(Clo)}, bv[2] = {smem_u32(Bhi), smem_u32(Blo)};
+            const uint32_t xw[2] = {smem_u32(XWhi), smem_u32(XWlo)}, hh[2] = {smem_u32(Hhi), smem_u32(Hlo)};
+            const int ta[3] = {0, 0, 1}, tb[3] = {0, 1, 0};  // (a, b) halves of the three terms
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const uint64_t dCk = sdesc_sw128(ch[ta[q]], 16, 1024), dBk = sdesc_sw128(bv[tb[q]], 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tbase + kColS, dCk + (uint64_t)((kk * 32) >> 4), dBk + (uint64_t)((kk * 32) >> 4), idS,
+                             (q | kk) != 0);
+            }
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const uint64_t dBm = sdesc_sw128(bv[ta[q]], 16384, 1024), dXw = sdesc_sw128(xw[tb[q]], 16384, 1024);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16(tbase + kColG, dBm + (uint64_t)((ks * 2048) >> 4), dXw + (uint64_t)((ks * 2048) >> 4),
+                             idG, (q | ks) != 0);
+            }
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const uint64_t dCk = sdesc_sw128(ch[ta[q]], 16, 1024), dH = sdesc_sw128(hh[tb[q]], 16384, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tbase + kColYo, dCk + (uint64_t)((kk * 32) >> 4), dH + (uint64_t)((kk * 2048) >> 4), idY,
+                             (q | kk) != 0);
+            }
+            mma_commit(&bars[0]);
+        }
+        issued = true;
+        ok = !__syncthreads_or(!mbar_wait(&bars[0], c & 1, abort_flag, err, kErrWaitMma));
+        if (!ok) break;
+        tc_fence_after();
+
+        // ---- 4. decay mask S -> P (fp32), written to TMEM as hi and lo bf16
+        {
+            const int ti = lq / R;
+            const float cai = cA[ti], gi = gam[ti];
+#pragma unroll 1
+            for (int g = 0; g < 4; ++g) {  // this thread's 64 columns, 16 at a time
+                const int j0 = 64 * hf + 16 * g;
+                float v[16];
+                tmem_ld16(tl + kColS + j0, v);
+                tmem_wait_ld();
+                uint32_t ph[8], pl[8];
+#pragma unroll
+                for (int e = 0; e < 16; e += 2) {
+                    float pv[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int tj = (j0 + e + u) / R;
+                        pv[u] = tj < ti ? v[e + u] * expf(cai - cA[tj]) * ghat[tj] : (tj == ti ? v[e + u] * gi : 0.f);
+                    }
+                    split2(pv[0], pv[1], ph[e >> 1], pl[e >> 1]);
+                }
+                tmem_st8(tl + kColPh + (uint32_t)(j0 >> 1), ph);
+                tmem_st8(tl + kColPl + (uint32_t)(j0 >> 1), pl);
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncthreads();
+        // Yd = P X: P hi.X hi + P hi.X lo + P lo.X hi, P read from TMEM
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t pa[3] = {kColPh, kColPh, kColPl};
+            const uint32_t xb[3] = {smem_u32(Xhi), smem_u32(Xlo), smem_u32(Xhi)};
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const uint64_t dX = sdesc_sw128(xb[q], 16384, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tbase + kColYd, tbase + pa[q] + (uint32_t)kk * 8u, dX + (uint64_t)((kk * 2048) >> 4),
+                                idY, (q | kk) != 0);
+            }
+            mma_commit(&bars[1]);
+        }
+
+        // ---- 5. carried state: h* <- Rot(-Phi)(exp(cA_end) h* + G), fp32 in registers
+        //      (Yo, the last reader of the h* tiles, completed before the mask)
+        {
+            const float eA = expf(cA[Q - 1]);
+            const int kp = (own_state ? srow : 0) >> 1;
+            const float cs = cosE[kp], sn = sinE[kp];
+            const float sgn = (srow & 1) ? -sn : sn;
+            float gv[32];
+            tmem_ld32(tl + kColG + c0, gv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int p = 0; p < 32; ++p) {
+                const float u = fmaf(eA, hreg[p], gv[p]);
+                const float o = __shfl_xor_sync(0xffffffffu, u, 1);
+                hreg[p] = fmaf(u, cs, o * sgn);
+            }
+            if (own_state) store_state32(Hhi, Hlo, srow, hf, hreg);
+        }
+
+        // ---- 6. y = Yd + exp(cA_t) Yo + D x
+        ok = !__syncthreads_or(!mbar_wait(&bars[1], c & 1, abort_flag, err, kErrWaitMma));
+        if (!ok) break;
+        tc_fence_after();
+        {
+            const int ti = lq / R, r = lq % R;
+            const int64_t t = t0 + ti;
+            const float sc = expf(cA[ti]);
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                float yd[16], yo[16];
+                tmem_ld16(tl + kColYd + c0 + 16 * qq, yd);
+                tmem_ld16(tl + kColYo + c0 + 16 * qq, yo);
+                tmem_wait_ld();
+                if (t < T) {
+                    const int64_t row = tok(t) * R + r;
+                    const float4 *xr = reinterpret_cast<const float4 *>(a.x + row * kP + c0 + 16 * qq);
+                    float4 *yr = reinterpret_cast<float4 *>(a.y + row * kP + c0 + 16 * qq);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 xv = xr[e];
+                        yr[e] = make_float4(fmaf(Dh, xv.x, fmaf(sc, yo[4 * e], yd[4 * e])),
+                                            fmaf(Dh, xv.y, fmaf(sc, yo[4 * e + 1], yd[4 * e + 1])),
+                                            fmaf(Dh, xv.z, fmaf(sc, yo[4 * e + 2], yd[4 * e + 2])),
+                                            fmaf(Dh, xv.w, fmaf(sc, yo[4 * e + 3], yd[4 * e + 3])));
+                    }
+                }
+            }
+        }
+        issued = false;  // both batches of MMAs have completed
+        fence_proxy_async_smem();  // the new h* tiles, before the next chunk's MMAs
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (ok) {  // final state: plain-frame h_{T-1}, the raw last token as the pending term
+        if (a.hT && own_state) {
+            float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * kN + srow) * kP + c0);
+#pragma unroll
+            for (int p = 0; p < 8; ++p) dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
+        }
+        if (T > 0) {
+            const int64_t last = tok(T - 1);
+            if (a.bpT && a.wB) {  // the last token's normalised B, one warp per rank row
+                for (int r = warp; r < R; r += kThreads / 32) {
+                    const float *src = a.B + (last * R + r) * kN;
+                    const float sc = bcn_row_scale_warp([&](int n) { return src[n]; }, kN, a.eps);
+                    for (int n = lane; n < kN; n += 32)
+                        a.bpT[(bh * R + r) * kN + n] = fmaf(src[n] * sc, a.wB[n], a.bB[(h * R + r) * kN + n]);
+                }
+            } else if (a.bpT) {
+                for (int i = tid; i < R * kN; i += kThreads) a.bpT[bh * R * kN + i] = a.B[last * R * kN + i];
+            }
+            if (a.xpT)
+                for (int i = tid; i < R * kP; i += kThreads) a.xpT[bh * R * kP + i] = a.x[last * R * kP + i];
+        }
+    } else if (issued && tid == 0) {  // no MMA may still run when TMEM is released
+        mma_commit(&bars[2]);
+        mbar_wait(&bars[2], 0, nullptr, err, 0, 400000000LL);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+template <int R>
+cudaError_t launch_r(const Tc32Args &a, int64_t grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc32_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    prefill_tc32_kernel<R><<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_tc32_supported(const Problem &p, const char **why) {
+    if (p.bf16) { *why = "fp32 tensor-core prefill: fp32 I/O only"; return false; }
+    if (p.P != kP || p.N != kN) { *why = "fp32 tensor-core prefill: headdim 64 and dstate 64 only"; return false; }
+    if (p.R != 1 && p.R != 2 && p.R != 4) { *why = "fp32 tensor-core prefill: rank 1, 2 or 4 only"; return false; }
+    if (p.segments > 0) { *why = "fp32 tensor-core prefill: sequences are not split"; return false; }
+    if (p.T < 1 || p.Bt < 1) { *why = "fp32 tensor-core prefill: empty problem"; return false; }
+    if (p.T > (int64_t)1 << 30) { *why = "fp32 tensor-core prefill: seqlen too long"; return false; }
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess || major != 10 ||
+        minor != 0) {
+        *why = "fp32 tensor-core prefill: needs an sm_100 device";
+        return false;
+    }
+    return true;
+}
+
+cudaError_t launch_prefill_tc32(const Problem &p, const char **) {
+    Tc32Args a{};
+    a.T = p.T;
+    a.H = p.H;
+    a.x = static_cast<const float *>(p.x);
+    a.B = static_cast<const float *>(p.B);
+    a.C = static_cast<const float *>(p.C);
+    a.dt = static_cast<const float *>(p.dt);
+    a.lam = static_cast<const float *>(p.lam);
+    a.theta = static_cast<const float *>(p.theta);
+    a.A = p.A;
+    a.D = p.D;
+    a.a_tok = p.a_tok;
+    a.th_head = p.th_head;
+    a.h0 = p.h0;
+    a.bp0 = p.bp0;
+    a.xp0 = p.xp0;
+    a.wB = p.wB;
+    a.wC = p.wC;
+    a.bB = p.bB;
+    a.bC = p.bC;
+    a.eps = p.eps;
+    a.y = static_cast<float *>(p.y);
+    a.hT = p.hT;
+    a.bpT = p.bpT;
+    a.xpT = p.xpT;
+    const int64_t grid = p.Bt * p.H;
+    if (grid == 0) return cudaSuccess;
+    if (p.R == 1) return launch_r<1>(a, grid, p.stream);
+    if (p.R == 2) return launch_r<2>(a, grid, p.stream);
+    return launch_r<4>(a, grid, p.stream);
+}
+
+cudaError_t read_tc32_error(unsigned *code) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_tc32_error, sizeof v);
+    if (e != cudaSuccess) return e;
+    if (v) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_tc32_error, &zero, sizeof zero);
+    }
+    *code = v;
+    return e;
+}
+
+}  // namespace m3

@@ -41,6 +41,8 @@ TC_CASES = [
     (Shape(1, 300, 2, 64, 64, 4, "bf16", 95), "split4"),
     (Shape(1, 130, 2, 64, 64, 1, "f32", 96), "simt"),
     (Shape(1, 70, 2, 64, 128, 4, "f32", 97), "simt"),
+    (Shape(1, 130, 2, 64, 64, 1, "f32", 96), "tc"),
+    (Shape(2, 77, 2, 64, 64, 4, "f32", 99), "tc"),
 ]
 
 

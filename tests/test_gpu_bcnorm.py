@@ -50,6 +50,8 @@ CASES = [
     (Shape(1, 130, 2, 64, 64, 1, "f32", 136), "simt"),
     (Shape(1, 70, 2, 64, 128, 4, "f32", 137), "simt"),
     (Shape(2, 37, 3, 8, 8, 1, "f32", 138), "simt"),
+    (Shape(1, 130, 2, 64, 64, 1, "f32", 136), "tc"),
+    (Shape(2, 77, 2, 64, 64, 2, "f32", 143), "tc"),
 ]
 
 

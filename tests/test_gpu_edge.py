@@ -19,7 +19,8 @@ error over (t, r, p); bars 2e-2 for bf16 I/O, 1e-4 for fp32 I/O):
   carries over many chunks.
 
 Paths: the tensor-core prefill (N = 128 R = 1, N = 64 R = 4, and N = 128
-R = 4 split into segments), the SIMT prefill (fp32 I/O), and the decode
+R = 4 split into segments), the fp32 tensor-core prefill (N = 64, R = 1 and
+2), the SIMT prefill (fp32 I/O), and the decode
 kernels (one CTA per slice, the persistent rank >= 2 kernel with a full grid
 and with few slices, bf16 and fp32 I/O)."""
 import math
@@ -133,6 +134,8 @@ PREFILL_CASES = [
     ("tc_n64_r4", Shape(1, 200, 3, 64, 64, 4, "bf16", 62), "tc"),
     ("tc_split_n128_r4", Shape(1, 600, 2, 64, 128, 4, "bf16", 63), "split"),
     ("simt_f32_n64_r2", Shape(1, 150, 2, 64, 64, 2, "f32", 64), "simt"),
+    ("tc32_n64_r1", Shape(2, 300, 2, 64, 64, 1, "f32", 65), "tc"),
+    ("tc32_n64_r2", Shape(1, 150, 2, 64, 64, 2, "f32", 66), "tc"),
 ]
 
 

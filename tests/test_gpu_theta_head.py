@@ -39,6 +39,8 @@ CASES = [
     (Shape(1, 1100, 2, 64, 128, 1, "bf16", 114), "split3"),
     (Shape(1, 130, 2, 64, 64, 1, "f32", 115), "simt"),
     (Shape(1, 70, 2, 64, 128, 4, "f32", 116), "simt"),
+    (Shape(1, 130, 2, 64, 64, 1, "f32", 115), "tc"),
+    (Shape(2, 77, 2, 64, 64, 4, "f32", 119), "tc"),
 ]
 
 
