@@ -18,7 +18,7 @@
 // lo.lo term and the splits' rounding about 2^-16 of the product.  Angles,
 // decays, the decay mask, the carried state and the epilogue stay fp32.
 //
-// One CTA of 256 threads per (batch, head) walks its sequence in chunks of
+// One CTA of 512 threads per (batch, head) walks its sequence in chunks of
 // 128 rows (Q = 128 / R tokens x R ranks), in synchronous phases per chunk:
 //   1. per-token scalars, the chunk-local scan of dt*A, the angle table;
 //   2. B, C (BC-normed first when the prologue is on) rotated in fp32 and
@@ -51,7 +51,13 @@ using namespace tc;
 
 constexpr int kP = 64, kN = 64, kK2 = kN / 2;
 constexpr int kRows = 128;   // rows per chunk = MMA M
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+// Thread roles on TMEM: warp w reads lanes 32 (w % 4) .. +31 (one chunk row per
+// thread) and takes column quarter w / 4 of each accumulator.
+constexpr int kCQ = kWarps / 4;    // column quarters
+constexpr int kTC = kP / kCQ;      // state / output columns per thread (16)
+constexpr int kSC = kRows / kCQ;   // S columns per thread in the mask (32)
 constexpr uint32_t kTile = kRows * 128;  // one bf16 tile of 128 rows x 64 columns (16 KB)
 // TMEM columns: S [0,128), G [128,192), Yo [192,256), Yd [256,320),
 // P hi [320,384), P lo [384,448) (P as packed bf16 pairs)
@@ -64,8 +70,9 @@ constexpr uint32_t OFF_C = 0, OFF_B = OFF_C + 2 * kTile, OFF_X = OFF_B + 2 * kTi
 constexpr uint32_t H_TILE = kN * 128;
 constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;
 constexpr uint32_t OFF_PHI = OFF_H + 2 * H_TILE;                  // phi [128][K2] fp32
-constexpr uint32_t OFF_SCAL = OFF_PHI + kRows * kK2 * 4;          // dts, gam, ghat, cA, wst [128]; cos, sin [K2]; wtot [8]
-constexpr uint32_t OFF_BAR = OFF_SCAL + (5 * kRows + 2 * kK2 + 8) * 4;
+constexpr uint32_t OFF_SCAL = OFF_PHI + kRows * kK2 * 4;
+// gam, ghat, cA, wst, colf [128]; cos, sin [K2]; wtot [8]; segment angle totals [kWarps][K2]; cA_0
+constexpr uint32_t OFF_BAR = OFF_SCAL + (5 * kRows + 2 * kK2 + 8 + kWarps * kK2 + 8) * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 4 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -104,17 +111,18 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
     lo = *reinterpret_cast<const uint32_t *>(&ll);
 }
 
-// hi/lo of 32 state values (row n, columns 32 half ..) into the MN-major h* tiles
-__device__ __forceinline__ void store_state32(uint8_t *hhi, uint8_t *hlo, int n, int half, const float (&h)[32]) {
+// hi/lo of this thread's kTC state values (row n, columns c0 ..) into the
+// MN-major h* tiles
+__device__ __forceinline__ void store_state(uint8_t *hhi, uint8_t *hlo, int n, int c0, const float (&h)[kTC]) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kTC / 8; ++j) {
         float v[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[e] = h[8 * j + e];
         uint4 hi, lo;
         split8(v, hi, lo);
-        *reinterpret_cast<uint4 *>(hhi + sw128(n, 4 * half + j)) = hi;
-        *reinterpret_cast<uint4 *>(hlo + sw128(n, 4 * half + j)) = lo;
+        *reinterpret_cast<uint4 *>(hhi + sw128(n, c0 / 8 + j)) = hi;
+        *reinterpret_cast<uint4 *>(hlo + sw128(n, c0 / 8 + j)) = lo;
     }
 }
 
@@ -127,17 +135,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
     uint8_t *Xhi = smem + OFF_X, *Xlo = Xhi + kTile, *XWhi = smem + OFF_XW, *XWlo = XWhi + kTile;
     uint8_t *Hhi = smem + OFF_H, *Hlo = Hhi + H_TILE;
     float *phi = reinterpret_cast<float *>(smem + OFF_PHI);
-    float *dts = reinterpret_cast<float *>(smem + OFF_SCAL), *gam = dts + kRows, *ghat = gam + kRows;
-    float *cA = ghat + kRows, *wst = cA + kRows, *cosE = wst + kRows, *sinE = cosE + kK2, *wtot = sinE + kK2;
+    float *gam = reinterpret_cast<float *>(smem + OFF_SCAL), *ghat = gam + kRows, *cA = ghat + kRows;
+    float *wst = cA + kRows, *colf = wst + kRows, *cosE = colf + kRows, *sinE = cosE + kK2, *wtot = sinE + kK2;
+    float *segtot = wtot + 8, *cA0 = segtot + kWarps * kK2;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);  // [0] S/G/Yo, [1] Yd, [2] drain
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
     unsigned *err = &g_tc32_error;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, hf = warp >> 2;  // TMEM lane quarter, column half
+    const int wq = warp & 3, cq = warp >> 2;  // TMEM lane quarter, column quarter
     const int lq = 32 * wq + lane;            // TMEM lane = chunk row
-    const int c0 = 32 * hf;                   // first of this thread's 32 columns
+    const int c0 = kTC * cq;                  // first of this thread's state / output columns
     const bool own_state = lane < 16;         // G (M = 64): lanes 0-15 of each quarter
     const int srow = wq * 16 + lane;          // its state row
     const int64_t bh = blockIdx.x, T = a.T, H = a.H;
@@ -161,24 +170,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
     const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
 
     // carried state (plain frame, pending-inclusive): h0 + beta'_0 b_prev x_prev^T
-    float hreg[32];
+    float hreg[kTC];
 #pragma unroll
-    for (int p = 0; p < 32; ++p) hreg[p] = 0.f;
+    for (int p = 0; p < kTC; ++p) hreg[p] = 0.f;
     if (own_state && T > 0) {
         const float betap0 = (1.f - a.lam[tok(0)]) * a.dt[tok(0)];
         if (a.h0) {
 #pragma unroll
-            for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * kN + srow) * kP + c0 + p];
+            for (int p = 0; p < kTC; ++p) hreg[p] = a.h0[(bh * kN + srow) * kP + c0 + p];
         }
         if (a.bp0 && a.xp0) {
             for (int r = 0; r < R; ++r) {
                 const float cw = betap0 * a.bp0[(bh * R + r) * kN + srow];
 #pragma unroll
-                for (int p = 0; p < 32; ++p) hreg[p] = fmaf(cw, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
+                for (int p = 0; p < kTC; ++p) hreg[p] = fmaf(cw, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
             }
         }
     }
-    if (own_state) store_state32(Hhi, Hlo, srow, hf, hreg);
+    if (own_state) store_state(Hhi, Hlo, srow, c0, hreg);
 
     constexpr uint32_t idS = idesc_bf16(kRows, kRows, 0, 0);
     constexpr uint32_t idG = idesc_bf16(kN, kP, 1, 1);
@@ -188,8 +197,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
     bool issued = false;  // MMAs may be in flight
     for (int c = 0; c < nch && ok; ++c) {
         const int64_t t0 = (int64_t)c * Q;
-        // ---- 1. per-token scalars and the chunk-local scan of dt*A
-        float acc = 0.f;
+        // ---- 1. per-token scalars, the chunk-local scan of dt*A and the angles.
+        //      Every thread also takes one state pair k and one of kWarps segments
+        //      of TPS tokens: the angle increments dt_s theta_s[k], their running
+        //      sum in registers, then the earlier segments' totals added.
+        constexpr int TPS = Q / kWarps;
+        const int kq = tid & 31, sg = tid >> 5;
+        float dtv[TPS], thv[TPS];
+#pragma unroll
+        for (int u = 0; u < TPS; ++u) {
+            const int64_t t = t0 + sg * TPS + u;
+            dtv[u] = t < T ? a.dt[tok(t)] : 0.f;
+            thv[u] = t < T ? a.theta[(a.th_head ? (int64_t)h : tok(t)) * kK2 + kq] : 0.f;
+        }
+        float acc = 0.f, gh = 0.f;
         if (tid < Q) {
             const int64_t t = t0 + tid;
             float d = 0.f, l = 0.f, nx = 0.f, av = 0.f;
@@ -199,9 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
                 av = a.a_tok ? a.A[tok(t)] : a.A[h];
                 if (t + 1 < T) nx = (1.f - a.lam[tok(t + 1)]) * a.dt[tok(t + 1)];
             }
-            dts[tid] = d;
             gam[tid] = l * d;
-            ghat[tid] = l * d + nx;
+            gh = l * d + nx;
+            ghat[tid] = gh;
             acc = d * av;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -209,56 +230,85 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
                 if (lane >= off) acc += v;
             }
             if (lane == 31) wtot[warp] = acc;
+            if (tid == 0) *cA0 = acc;
         }
-        __syncthreads();
-        if (tid < Q) {
-            float off = 0.f;
-            for (int w = 0; w < warp; ++w) off += wtot[w];
-            cA[tid] = acc + off;
-        }
-        // angle increments dt_s theta_s[k]
-        for (int idx = tid; idx < Q * kK2; idx += kThreads) {
-            const int s = idx / kK2, k = idx % kK2;
-            const int64_t t = t0 + s;
-            phi[idx] = t < T ? dts[s] * a.theta[(a.th_head ? (int64_t)h : tok(t)) * kK2 + k] : 0.f;
-        }
-        __syncthreads();
-        // their running sum per pair; the chunk's total angle
-        if (tid < kK2) {
+        float pre[TPS];
+        {
             float run = 0.f;
-            for (int s = 0; s < Q; ++s) {
-                run += phi[s * kK2 + tid];
-                phi[s * kK2 + tid] = run;
+#pragma unroll
+            for (int u = 0; u < TPS; ++u) {
+                run = fmaf(dtv[u], thv[u], run);
+                pre[u] = run;
             }
-            float sn, cs;
-            sincosf(run, &sn, &cs);
-            cosE[tid] = cs;
-            sinE[tid] = sn;
+            segtot[sg * kK2 + kq] = run;
         }
-        if (tid >= kThreads - Q) {  // chunk-state weights exp(cA_end - cA_s) ghat_s
-            const int s = tid - (kThreads - Q);
-            wst[s] = expf(cA[Q - 1] - cA[s]) * ghat[s];
+        __syncthreads();
+        if (tid < Q) {  // cA_t, the chunk-state weight exp(cA_end - cA_t) ghat_t, the column factor
+            constexpr int NW = Q / 32;
+            float off = 0.f, offl = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                if (w < warp) off += wtot[w];
+                if (w < NW - 1) offl += wtot[w];
+            }
+            const float ca = acc + off, cend = wtot[NW - 1] + offl;  // cend: the same sum as cA_{Q-1}
+            cA[tid] = ca;
+            wst[tid] = expf(cend - ca) * gh;
+            colf[tid] = expf(*cA0 - ca) * gh;
+        }
+        {
+            float off = 0.f;
+            for (int s2 = 0; s2 < sg; ++s2) off += segtot[s2 * kK2 + kq];
+#pragma unroll
+            for (int u = 0; u < TPS; ++u) phi[(sg * TPS + u) * kK2 + kq] = pre[u] + off;
+            if (sg == kWarps - 1) {  // the chunk's total angle of pair kq
+                float sn, cs;
+                sincosf(pre[TPS - 1] + off, &sn, &cs);
+                cosE[kq] = cs;
+                sinE[kq] = sn;
+            }
         }
         __syncthreads();
 
-        // ---- 2. rotated B, C and the value rows as hi/lo tiles (16-byte chunk j of row i)
-        for (int it = tid; it < kRows * 8; it += kThreads) {
-            const int i = it >> 3, j = it & 7;
-            const int s = i / R, r = i % R;
-            const int64_t t = t0 + s;
-            float vb[8], vc[8], vx[8], vw[8];
-            if (t < T) {
-                const int64_t row = tok(t) * R + r;
-                const float4 b0 = *reinterpret_cast<const float4 *>(a.B + row * kN + 8 * j);
-                const float4 b1 = *reinterpret_cast<const float4 *>(a.B + row * kN + 8 * j + 4);
-                const float4 q0 = *reinterpret_cast<const float4 *>(a.C + row * kN + 8 * j);
-                const float4 q1 = *reinterpret_cast<const float4 *>(a.C + row * kN + 8 * j + 4);
-                const float4 x0 = *reinterpret_cast<const float4 *>(a.x + row * kP + 8 * j);
-                const float4 x1 = *reinterpret_cast<const float4 *>(a.x + row * kP + 8 * j + 4);
-                float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                float cc[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                if (a.wB) {  // BC-norm: the row's RMS over its 8 lanes, weight and bias
+        // ---- 2. rotated B, C and the value rows as hi/lo tiles: thread (row i,
+        //      16-byte chunk j) for rows i = tid / 8 + 64 u, u = 0, 1, the loads
+        //      of both rows issued together
+        const int j = tid & 7;
+        {
+            float4 ld[2][6];
+            bool valid[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = (tid >> 3) + 64 * u;
+                const int64_t t = t0 + i / R;
+                valid[u] = t < T;
+                if (valid[u]) {
+                    const int64_t row = tok(t) * R + i % R;
+                    const float4 *pb = reinterpret_cast<const float4 *>(a.B + row * kN + 8 * j);
+                    const float4 *pc = reinterpret_cast<const float4 *>(a.C + row * kN + 8 * j);
+                    const float4 *px = reinterpret_cast<const float4 *>(a.x + row * kP + 8 * j);
+                    ld[u][0] = pb[0];
+                    ld[u][1] = pb[1];
+                    ld[u][2] = pc[0];
+                    ld[u][3] = pc[1];
+                    ld[u][4] = px[0];
+                    ld[u][5] = px[1];
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 6; ++e) ld[u][e] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = (tid >> 3) + 64 * u;
+                const int si = i / R, r = i % R;
+                float bb[8] = {ld[u][0].x, ld[u][0].y, ld[u][0].z, ld[u][0].w,
+                               ld[u][1].x, ld[u][1].y, ld[u][1].z, ld[u][1].w};
+                float cc[8] = {ld[u][2].x, ld[u][2].y, ld[u][2].z, ld[u][2].w,
+                               ld[u][3].x, ld[u][3].y, ld[u][3].z, ld[u][3].w};
+                const float xx[8] = {ld[u][4].x, ld[u][4].y, ld[u][4].z, ld[u][4].w,
+                                     ld[u][5].x, ld[u][5].y, ld[u][5].z, ld[u][5].w};
+                if (a.wB && valid[u]) {  // BC-norm: the row's RMS over its 8 lanes, weight and bias
                     const unsigned grp = 0xffu << (lane & 24);
                     float sb = 0.f, sq = 0.f;
 #pragma unroll
@@ -279,39 +329,34 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
                         cc[e] = fmaf(cc[e] * kc, a.wC[8 * j + e], biC[e]);
                     }
                 }
+                float vb[8], vc[8], vw[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {  // pair k = 4 j + e: rotate by +phi_s[k]
                     float sn, cs;
-                    sincosf(phi[s * kK2 + 4 * j + e], &sn, &cs);
+                    sincosf(phi[si * kK2 + 4 * j + e], &sn, &cs);
                     vb[2 * e] = bb[2 * e] * cs - bb[2 * e + 1] * sn;
                     vb[2 * e + 1] = bb[2 * e] * sn + bb[2 * e + 1] * cs;
                     vc[2 * e] = cc[2 * e] * cs - cc[2 * e + 1] * sn;
                     vc[2 * e + 1] = cc[2 * e] * sn + cc[2 * e + 1] * cs;
                 }
-                const float w = wst[s];
+                const float w = wst[si];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    vx[e] = xx[e];
-                    vw[e] = w * xx[e];
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) vb[e] = vc[e] = vx[e] = vw[e] = 0.f;
+                for (int e = 0; e < 8; ++e) vw[e] = w * xx[e];
+                const uint32_t off = sw128((uint32_t)i, (uint32_t)j);
+                uint4 hi, lo;
+                split8(vb, hi, lo);
+                *reinterpret_cast<uint4 *>(Bhi + off) = hi;
+                *reinterpret_cast<uint4 *>(Blo + off) = lo;
+                split8(vc, hi, lo);
+                *reinterpret_cast<uint4 *>(Chi + off) = hi;
+                *reinterpret_cast<uint4 *>(Clo + off) = lo;
+                split8(xx, hi, lo);
+                *reinterpret_cast<uint4 *>(Xhi + off) = hi;
+                *reinterpret_cast<uint4 *>(Xlo + off) = lo;
+                split8(vw, hi, lo);
+                *reinterpret_cast<uint4 *>(XWhi + off) = hi;
+                *reinterpret_cast<uint4 *>(XWlo + off) = lo;
             }
-            const uint32_t off = sw128((uint32_t)i, (uint32_t)j);
-            uint4 hi, lo;
-            split8(vb, hi, lo);
-            *reinterpret_cast<uint4 *>(Bhi + off) = hi;
-            *reinterpret_cast<uint4 *>(Blo + off) = lo;
-            split8(vc, hi, lo);
-            *reinterpret_cast<uint4 *>(Chi + off) = hi;
-            *reinterpret_cast<uint4 *>(Clo + off) = lo;
-            split8(vx, hi, lo);
-            *reinterpret_cast<uint4 *>(Xhi + off) = hi;
-            *reinterpret_cast<uint4 *>(Xlo + off) = lo;
-            split8(vw, hi, lo);
-            *reinterpret_cast<uint4 *>(XWhi + off) = hi;
-            *reinterpret_cast<uint4 *>(XWlo + off) = lo;
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -354,13 +399,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
         if (!ok) break;
         tc_fence_after();
 
-        // ---- 4. decay mask S -> P (fp32), written to TMEM as hi and lo bf16
+        // ---- 4. decay mask S -> P (fp32), written to TMEM as hi and lo bf16:
+        //      P(t,s) = S(t,s) exp(cA_t - cA_s) (s < t ? ghat_s : gam_t), 0 for s > t.
+        //      While the chunk's decay stays within e^60 the exponential is a row
+        //      factor exp(cA_t - cA_0) times the column factor exp(cA_0 - cA_s)
+        //      ghat_s (both in fp32 range); deeper chunks take one exp per element.
         {
             const int ti = lq / R;
             const float cai = cA[ti], gi = gam[ti];
+            const bool fact = (cA[0] - cA[Q - 1]) < 60.f;  // uniform across the CTA
+            const float rowf = expf(cai - cA[0]);
 #pragma unroll 1
-            for (int g = 0; g < 4; ++g) {  // this thread's 64 columns, 16 at a time
-                const int j0 = 64 * hf + 16 * g;
+            for (int g = 0; g < kSC / 16; ++g) {  // this thread's kSC columns, 16 at a time
+                const int j0 = kSC * cq + 16 * g;
                 float v[16];
                 tmem_ld16(tl + kColS + j0, v);
                 tmem_wait_ld();
@@ -371,7 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int tj = (j0 + e + u) / R;
-                        pv[u] = tj < ti ? v[e + u] * expf(cai - cA[tj]) * ghat[tj] : (tj == ti ? v[e + u] * gi : 0.f);
+                        const float f = tj < ti ? (fact ? rowf * colf[tj] : expf(cai - cA[tj]) * ghat[tj])
+                                                : (tj == ti ? gi : 0.f);
+                        pv[u] = v[e + u] * f;
                     }
                     split2(pv[0], pv[1], ph[e >> 1], pl[e >> 1]);
                 }
@@ -397,6 +450,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
             }
             mma_commit(&bars[1]);
         }
+        // this thread's x row segment for the epilogue, loaded while the state update runs
+        const int ty = lq / R, ry = lq % R;
+        const int64_t t_y = t0 + ty;
+        float4 xv[kTC / 4];
+        if (t_y < T) {
+            const float4 *xr = reinterpret_cast<const float4 *>(a.x + (tok(t_y) * R + ry) * kP + c0);
+#pragma unroll
+            for (int e = 0; e < kTC / 4; ++e) xv[e] = xr[e];
+        } else {
+#pragma unroll
+            for (int e = 0; e < kTC / 4; ++e) xv[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 
         // ---- 5. carried state: h* <- Rot(-Phi)(exp(cA_end) h* + G), fp32 in registers
         //      (Yo, the last reader of the h* tiles, completed before the mask)
@@ -405,16 +470,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
             const int kp = (own_state ? srow : 0) >> 1;
             const float cs = cosE[kp], sn = sinE[kp];
             const float sgn = (srow & 1) ? -sn : sn;
-            float gv[32];
-            tmem_ld32(tl + kColG + c0, gv);
+            float gv[kTC];
+            tmem_ld16(tl + kColG + c0, gv);
             tmem_wait_ld();
 #pragma unroll
-            for (int p = 0; p < 32; ++p) {
+            for (int p = 0; p < kTC; ++p) {
                 const float u = fmaf(eA, hreg[p], gv[p]);
                 const float o = __shfl_xor_sync(0xffffffffu, u, 1);
                 hreg[p] = fmaf(u, cs, o * sgn);
             }
-            if (own_state) store_state32(Hhi, Hlo, srow, hf, hreg);
+            if (own_state) store_state(Hhi, Hlo, srow, c0, hreg);
         }
 
         // ---- 6. y = Yd + exp(cA_t) Yo + D x
@@ -422,26 +487,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
         if (!ok) break;
         tc_fence_after();
         {
-            const int ti = lq / R, r = lq % R;
-            const int64_t t = t0 + ti;
-            const float sc = expf(cA[ti]);
+            const float sc = expf(cA[ty]);
 #pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
+            for (int qq = 0; qq < kTC / 16; ++qq) {
                 float yd[16], yo[16];
                 tmem_ld16(tl + kColYd + c0 + 16 * qq, yd);
                 tmem_ld16(tl + kColYo + c0 + 16 * qq, yo);
                 tmem_wait_ld();
-                if (t < T) {
-                    const int64_t row = tok(t) * R + r;
-                    const float4 *xr = reinterpret_cast<const float4 *>(a.x + row * kP + c0 + 16 * qq);
-                    float4 *yr = reinterpret_cast<float4 *>(a.y + row * kP + c0 + 16 * qq);
+                if (t_y < T) {
+                    float4 *yr = reinterpret_cast<float4 *>(a.y + (tok(t_y) * R + ry) * kP + c0 + 16 * qq);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float4 xv = xr[e];
-                        yr[e] = make_float4(fmaf(Dh, xv.x, fmaf(sc, yo[4 * e], yd[4 * e])),
-                                            fmaf(Dh, xv.y, fmaf(sc, yo[4 * e + 1], yd[4 * e + 1])),
-                                            fmaf(Dh, xv.z, fmaf(sc, yo[4 * e + 2], yd[4 * e + 2])),
-                                            fmaf(Dh, xv.w, fmaf(sc, yo[4 * e + 3], yd[4 * e + 3])));
+                        const float4 x4 = xv[4 * qq + e];
+                        yr[e] = make_float4(fmaf(Dh, x4.x, fmaf(sc, yo[4 * e], yd[4 * e])),
+                                            fmaf(Dh, x4.y, fmaf(sc, yo[4 * e + 1], yd[4 * e + 1])),
+                                            fmaf(Dh, x4.z, fmaf(sc, yo[4 * e + 2], yd[4 * e + 2])),
+                                            fmaf(Dh, x4.w, fmaf(sc, yo[4 * e + 3], yd[4 * e + 3])));
                     }
                 }
             }
@@ -456,7 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
         if (a.hT && own_state) {
             float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * kN + srow) * kP + c0);
 #pragma unroll
-            for (int p = 0; p < 8; ++p) dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
+            for (int p = 0; p < kTC / 4; ++p)
+                dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
         }
         if (T > 0) {
             const int64_t last = tok(T - 1);
