@@ -71,6 +71,9 @@ def parse():
     ap.add_argument("--case-batch", type=int, default=None, help="batch of the profiling case")
     ap.add_argument("--case-seqlen", type=int, default=None, help="sequence length of the profiling case")
     ap.add_argument("--case-launches", type=int, default=3, help="launches of the profiling case")
+    ap.add_argument("--compare-fp32", action="store_true",
+                    help="kernel study: the fp32 tensor-core prefill against the SIMT kernel on fp32 shapes "
+                         "(one JSON line per shape; prints no bench line)")
     return ap.parse_args()
 
 
@@ -103,6 +106,53 @@ def run_case(args):
     print(f"case {args.case} {s} x{args.case_launches} done")
 
 
+def run_compare_fp32(args):
+    """Both prefill kernels that take fp32 I/O on the same inputs: the small
+    fp32 workload and the SISO workload's batch, length and heads at
+    dstate 64 (ranks 1, 2, 4).  Median of --steps calls, each timed alone
+    with CUDA events after a 256 MiB write that flushes L2."""
+    import dataclasses
+
+    import torch
+
+    import state_space_sequence_ssm_b200 as m3
+    from m3_inputs import WORKLOADS, make_prefill
+
+    keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
+    hbm, src = peaks()
+    big = WORKLOADS[PREFILL_WORKLOAD]
+    shapes = [WORKLOADS["siso_f32_b1_t256_h4_p64_n64"]] + [
+        big.with_(dstate=64, rank=r, io="f32") for r in (1, 2, 4)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for s in shapes:
+        inp = make_prefill(s, device="cuda")
+        y = torch.empty_like(inp["x"])
+        fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device="cuda")
+        dims = m3.make_dims(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.rank, s.torch_io)
+        line = {"study": "fp32 prefill kernels", "shape": dataclasses.asdict(s),
+                "algorithmic_bytes": prefill_bytes(s), "peak_gbs": hbm, "peak_source": src}
+        for name, algo in (("tc", m3.ALGO_TC), ("simt", m3.ALGO_SIMT)):
+            line[name + "_kernel"] = m3.scan_plan_info(dims, algo).kernel_name
+            for _ in range(max(args.warmup, 3)):
+                m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, algo=algo)
+            ts = []
+            for i in range(args.steps):
+                flush.fill_(i & 0xff)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, algo=algo)
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            m3.stream_status()
+            ms = statistics.median(ts)
+            line[name + "_ms"] = ms
+            line[name + "_frac"] = prefill_bytes(s) / (ms * 1e-3) / 1e9 / hbm
+        line["speedup"] = line["simt_ms"] / line["tc_ms"]
+        print(json.dumps(line, default=str), flush=True)
+        del inp, y, fin
+
+
 # ---------------------------------------------------------------- helpers
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -123,7 +173,8 @@ def kernel_sources(kernel):
     csrc = os.path.join(ROOT, "state_space_sequence_ssm_b200", "csrc")
     files = {"prefill_simt_kernel": ["prefill_simt.cu"], "step_kernel": ["decode.cu"],
              "step_stream_kernel": ["decode.cu"],
-             "prefill_tc_kernel": ["prefill_tc.cu", "tc_primitives.cuh"]}[kernel]
+             "prefill_tc_kernel": ["prefill_tc.cu", "tc_primitives.cuh"],
+             "prefill_tc32_kernel": ["prefill_tc32.cu", "tc_primitives.cuh", "bcnorm.cuh"]}[kernel]
     return [os.path.join(csrc, f) for f in files if os.path.exists(os.path.join(csrc, f))]
 
 
@@ -756,6 +807,8 @@ def main():
     args = parse()
     if args.case:
         run_case(args)
+    elif args.compare_fp32:
+        run_compare_fp32(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
