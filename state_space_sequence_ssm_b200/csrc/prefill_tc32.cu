@@ -102,6 +102,22 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4 &hi, uint4 &lo
     lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// sin and cos of a chunk-local angle (|x| < 2^16 * 2 pi): Cody and Waite's
+// reduction by 2 pi in two parts (the first, 6.28125, has 8 significant bits,
+// so n times it is exact; the second is the rest of 2 pi in fp32), then the
+// hardware approximation on [-pi, pi], whose absolute error there is about
+// 4e-7.  Used where each angle rotates one chunk's B and C rows only; the
+// chunk's total angle, which rotates the carried state once per chunk (so its
+// error would compound), takes the full-accuracy sincosf.
+__device__ __forceinline__ void sincos_reduced(float x, float *s, float *c) {
+    constexpr float kInv2Pi = 0.15915494309189535f;
+    constexpr float k2PiHi = 6.28125f;
+    constexpr float k2PiLo = 1.9353071795864769e-3f;  // 2 pi - 6.28125
+    const float n = rintf(x * kInv2Pi);
+    const float r = fmaf(-n, k2PiLo, fmaf(-n, k2PiHi, x));
+    __sincosf(r, s, c);
+}
+
 // hi and lo of a pair, packed (low half = first value)
 __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
     const __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
@@ -257,8 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
             colf[tid] = expf(*cA0 - ca) * gh;
         }
         {
-            float off = 0.f;
-            for (int s2 = 0; s2 < sg; ++s2) off += segtot[s2 * kK2 + kq];
+            float off = 0.f;  // the earlier segments' totals: independent loads, no serial chain
+#pragma unroll
+            for (int s2 = 0; s2 < kWarps - 1; ++s2)
+                if (s2 < sg) off += segtot[s2 * kK2 + kq];
 #pragma unroll
             for (int u = 0; u < TPS; ++u) phi[(sg * TPS + u) * kK2 + kq] = pre[u] + off;
             if (sg == kWarps - 1) {  // the chunk's total angle of pair kq
@@ -333,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {  // pair k = 4 j + e: rotate by +phi_s[k]
                     float sn, cs;
-                    sincosf(phi[si * kK2 + 4 * j + e], &sn, &cs);
+                    sincos_reduced(phi[si * kK2 + 4 * j + e], &sn, &cs);
                     vb[2 * e] = bb[2 * e] * cs - bb[2 * e + 1] * sn;
                     vb[2 * e + 1] = bb[2 * e] * sn + bb[2 * e + 1] * cs;
                     vc[2 * e] = cc[2 * e] * cs - cc[2 * e + 1] * sn;
