@@ -29,7 +29,8 @@ def test_context_usable_after_timeout():
     m3.selftest_wait_timeout(stream=s)
     with pytest.raises(m3.M3Error):
         m3.stream_status(stream=s)
-    # both kernel families still run and still match the oracle
+    # every prefill kernel still runs and still matches the oracle
     check_scan(Shape(1, 300, 2, 64, 128, 1, "bf16", 81), m3.ALGO_TC, with_init=True)
+    check_scan(Shape(1, 300, 2, 64, 64, 2, "f32", 83), m3.ALGO_TC, with_init=True)
     check_scan(Shape(1, 100, 2, 16, 32, 2, "f32", 82), m3.ALGO_SIMT, with_init=True)
     m3.stream_status()

@@ -1,5 +1,6 @@
 """GPU tests of the library inside CUDA graphs and under concurrent host
-threads: prefill (whole and split sequences) and decode steps captured once
+threads: prefill (whole and split sequences, the SIMT kernel, fp32 I/O on
+the tensor cores) and decode steps captured once
 and replayed give the same bits as eager calls; two host threads driving
 m3_scan_fwd_host on their own streams give the same bits as one at a time."""
 import threading
@@ -22,10 +23,13 @@ def dev(d):
     return {k: v.cuda() for k, v in d.items()}
 
 
-@pytest.mark.parametrize("algo_name,segs", [("auto", 0), ("split", 3), ("simt", 0)])
+@pytest.mark.parametrize("algo_name,segs", [("auto", 0), ("split", 3), ("simt", 0), ("tc32", 0)])
 def test_prefill_graph_replay_matches_eager(algo_name, segs):
     s = Shape(2, 700, 4, 64, 128, 1, "bf16", 401)
-    algo = {"auto": m3.ALGO_AUTO, "split": m3.ALGO_TC_SEGMENTS(segs), "simt": m3.ALGO_SIMT}[algo_name]
+    if algo_name == "tc32":  # fp32 I/O on the tensor cores (split operands)
+        s = Shape(2, 700, 4, 64, 64, 2, "f32", 405)
+    algo = {"auto": m3.ALGO_AUTO, "split": m3.ALGO_TC_SEGMENTS(segs), "simt": m3.ALGO_SIMT,
+            "tc32": m3.ALGO_TC}[algo_name]
     inp = dev(make_prefill(s))
     init = m3.State(*(t.cuda() for t in make_state(s)))
     dims = m3.make_dims(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.rank, s.torch_io)
