@@ -20,7 +20,8 @@
 //
 // One CTA of 512 threads per (batch, head) walks its sequence in chunks of
 // 128 rows (Q = 128 / R tokens x R ranks), in synchronous phases per chunk:
-//   1. per-token scalars, the chunk-local scan of dt*A, the angle table;
+//   1. per-token scalars, the chunk-local scan of dt*A, the angle table
+//      (for chunk c + 1, while the tensor cores run step 3 of chunk c);
 //   2. B, C (BC-normed first when the prologue is on) rotated in fp32 and
 //      split into 128B-swizzled bf16 hi/lo tiles (K-major), x and w o x
 //      split likewise (MN-major);
@@ -71,8 +72,10 @@ constexpr uint32_t H_TILE = kN * 128;
 constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;
 constexpr uint32_t OFF_PHI = OFF_H + 2 * H_TILE;                  // phi [128][K2] fp32
 constexpr uint32_t OFF_SCAL = OFF_PHI + kRows * kK2 * 4;
-// gam, ghat, cA, wst, colf [128]; cos, sin [K2]; wtot [8]; segment angle totals [kWarps][K2]; cA_0
-constexpr uint32_t OFF_BAR = OFF_SCAL + (5 * kRows + 2 * kK2 + 8 + kWarps * kK2 + 8) * 4;
+// two buffers (chunk c and c + 1) of {gam, ghat, cA, wst, colf}[128] + {cos, sin}[K2];
+// then wtot [8], segment angle totals [kWarps][K2], cA_0
+constexpr uint32_t SB32 = 5 * kRows + 2 * kK2;
+constexpr uint32_t OFF_BAR = OFF_SCAL + (2 * SB32 + 8 + kWarps * kK2 + 8) * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 4 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -151,9 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
     uint8_t *Xhi = smem + OFF_X, *Xlo = Xhi + kTile, *XWhi = smem + OFF_XW, *XWlo = XWhi + kTile;
     uint8_t *Hhi = smem + OFF_H, *Hlo = Hhi + H_TILE;
     float *phi = reinterpret_cast<float *>(smem + OFF_PHI);
-    float *gam = reinterpret_cast<float *>(smem + OFF_SCAL), *ghat = gam + kRows, *cA = ghat + kRows;
-    float *wst = cA + kRows, *colf = wst + kRows, *cosE = colf + kRows, *sinE = cosE + kK2, *wtot = sinE + kK2;
-    float *segtot = wtot + 8, *cA0 = segtot + kWarps * kK2;
+    float *sbuf = reinterpret_cast<float *>(smem + OFF_SCAL);  // two chunks' scalars, SB32 floats each
+    float *wtot = sbuf + 2 * SB32, *segtot = wtot + 8, *cA0 = segtot + kWarps * kK2;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);  // [0] S/G/Yo, [1] Yd, [2] drain
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
@@ -208,15 +210,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
     constexpr uint32_t idS = idesc_bf16(kRows, kRows, 0, 0);
     constexpr uint32_t idG = idesc_bf16(kN, kP, 1, 1);
     constexpr uint32_t idY = idesc_bf16(kRows, kP, 0, 1);
-    const int nch = (int)((T + Q - 1) / Q);
-    bool ok = true;
-    bool issued = false;  // MMAs may be in flight
-    for (int c = 0; c < nch && ok; ++c) {
-        const int64_t t0 = (int64_t)c * Q;
-        // ---- 1. per-token scalars, the chunk-local scan of dt*A and the angles.
-        //      Every thread also takes one state pair k and one of kWarps segments
-        //      of TPS tokens: the angle increments dt_s theta_s[k], their running
-        //      sum in registers, then the earlier segments' totals added.
+    // ---- 1. per-token scalars of the chunk starting at token t0 into the scalar
+    //      buffer sb, the chunk-local scan of dt*A and the angle table.  Every
+    //      thread also takes one state pair k and one of kWarps segments of TPS
+    //      tokens: the angle increments dt_s theta_s[k], their running sum in
+    //      registers, then the earlier segments' totals added.  Two CTA barriers.
+    auto phase1 = [&](const int64_t t0, float *sb) {
+        float *gam = sb, *ghat = sb + kRows, *cA = sb + 2 * kRows, *wst = sb + 3 * kRows, *colf = sb + 4 * kRows;
+        float *cosE = sb + 5 * kRows, *sinE = cosE + kK2;
         constexpr int TPS = Q / kWarps;
         const int kq = tid & 31, sg = tid >> 5;
         float dtv[TPS], thv[TPS];
@@ -287,7 +288,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
             }
         }
         __syncthreads();
-
+    };
+    const int nch = (int)((T + Q - 1) / Q);
+    bool ok = true;
+    bool issued = false;  // MMAs may be in flight
+    phase1(0, sbuf);
+    for (int c = 0; c < nch && ok; ++c) {
+        const int64_t t0 = (int64_t)c * Q;
+        // this chunk's scalars (phase 1 of chunk c + 1 fills the other buffer
+        // while the tensor cores run S, G and Yo of chunk c)
+        float *sb = sbuf + (c & 1) * SB32;
+        float *gam = sb, *ghat = sb + kRows, *cA = sb + 2 * kRows, *wst = sb + 3 * kRows, *colf = sb + 4 * kRows;
+        float *cosE = sb + 5 * kRows, *sinE = cosE + kK2;
         // ---- 2. rotated B, C and the value rows as hi/lo tiles: thread (row i,
         //      16-byte chunk j) for rows i = tid / 8 + 64 u, u = 0, 1, the loads
         //      of both rows issued together
@@ -413,6 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
             mma_commit(&bars[0]);
         }
         issued = true;
+        // phase 1 of the next chunk while the MMAs run: the angle table is free
+        // (phase 2 above was its last reader) and the other scalar buffer was
+        // last read by the previous chunk's epilogue
+        if (c + 1 < nch) phase1(t0 + Q, sbuf + ((c + 1) & 1) * SB32);
         ok = !__syncthreads_or(!mbar_wait(&bars[0], c & 1, abort_flag, err, kErrWaitMma));
         if (!ok) break;
         tc_fence_after();
