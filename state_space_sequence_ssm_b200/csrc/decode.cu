@@ -181,10 +181,10 @@ step_kernel(const StepArgs<IO> a, const StepFeat f) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const float2 ck = *reinterpret_cast<const float2 *>(&sC[r][2 * k]);
-            yacc[r].x += nu.x * ck.x + nv.x * ck.y;
-            yacc[r].y += nu.y * ck.x + nv.y * ck.y;
-            yacc[r].z += nu.z * ck.x + nv.z * ck.y;
-            yacc[r].w += nu.w * ck.x + nv.w * ck.y;
+            yacc[r].x = fmaf(nu.x, ck.x, fmaf(nv.x, ck.y, yacc[r].x));
+            yacc[r].y = fmaf(nu.y, ck.x, fmaf(nv.y, ck.y, yacc[r].y));
+            yacc[r].z = fmaf(nu.z, ck.x, fmaf(nv.z, ck.y, yacc[r].z));
+            yacc[r].w = fmaf(nu.w, ck.x, fmaf(nv.w, ck.y, yacc[r].w));
         }
     }
     // ---- readout: sum over pair groups (same cg) -- shuffle within the warp
@@ -448,10 +448,10 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const float2 ck = *reinterpret_cast<const float2 *>(vC + r * N + 2 * k);
-                yacc[r].x += nu.x * ck.x + nv.x * ck.y;
-                yacc[r].y += nu.y * ck.x + nv.y * ck.y;
-                yacc[r].z += nu.z * ck.x + nv.z * ck.y;
-                yacc[r].w += nu.w * ck.x + nv.w * ck.y;
+                yacc[r].x = fmaf(nu.x, ck.x, fmaf(nv.x, ck.y, yacc[r].x));
+                yacc[r].y = fmaf(nu.y, ck.x, fmaf(nv.y, ck.y, yacc[r].y));
+                yacc[r].z = fmaf(nu.z, ck.x, fmaf(nv.z, ck.y, yacc[r].z));
+                yacc[r].w = fmaf(nu.w, ck.x, fmaf(nv.w, ck.y, yacc[r].w));
             }
         }
 #pragma unroll
