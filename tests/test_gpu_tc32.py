@@ -142,3 +142,25 @@ def test_tc32_resume_equals_one_call():
     yb, _ = m3.scan_fwd(*part(cut, s.seqlen), st)
     torch.cuda.synchronize()
     assert rel_l2(host64(torch.cat([ya, yb], dim=1)), host64(y)) < TOL_F32
+
+
+@pytest.mark.parametrize("rank", [1, 4])
+def test_tc32_long_weak_decay_large_angles(rank):
+    """16,384 tokens with almost no decay (A = -0.002) and large angle rates:
+    the carried state is rotated once per chunk for 128 (rank 1) or 512 (rank
+    4) chunks and keeps nearly all of its history, so errors of the chunk
+    rotation and of the split products would compound; the result must stay
+    within the fp32 bar."""
+    s = Shape(1, 16384, 2, 64, 64, rank, "f32", 330 + rank)
+    inp = make_prefill(s)
+    inp["A"] = torch.full_like(inp["A"], -0.002)
+    inp["theta"] = inp["theta"] * 3.0  # |theta| up to 3 pi
+    inp = {k: v.to(DEV) for k, v in inp.items()}
+    init = m3.State(*(t.to(DEV) for t in make_state(s)))
+    y, fs = m3.scan_fwd(*(inp[k] for k in KEYS), init, algo=m3.ALGO_TC)
+    m3.stream_status()
+    yr, sr = oracle.scan(*(host64(inp[k]) for k in KEYS), oracle.State(*(host64(t) for t in init)))
+    ey, eh = max_rel_l2_y(host64(y), yr), max_rel_l2_state(host64(fs.h), sr.h)
+    record_margin(f"tc32 long weak decay r{rank}", max(ey, eh), TOL_F32)
+    assert ey < TOL_F32, f"y rel-L2 {ey:.3e}"
+    assert eh < TOL_F32, f"state rel-L2 {eh:.3e}"
