@@ -32,9 +32,11 @@
 //   5. the carried state h* <- Rot(-Phi)(exp(cA_end) h* + G) in fp32
 //      registers, its hi/lo tiles for the next chunk's Yo;
 //   6. y = Yd + exp(cA_t) Yo + D x, stored in fp32.
-// Built for headdim 64 and dstate 64 (the tiles of one chunk then take
-// 160 KB of shared memory); other fp32 sizes run the SIMT kernel.  Every wait
-// is bounded and reports through the library's device error word.
+// Built for headdim 64 and dstate 64 (the hi/lo tiles of one chunk take
+// 144 KB of shared memory, 173 KB with the angle table and the scalars; all
+// 512 TMEM columns); other fp32 sizes run the SIMT kernel.  Every wait is
+// bounded and reports through this kernel's device error word, which
+// m3_stream_status reads.
 #include <cuda_bf16.h>
 
 #include "bcnorm.cuh"
