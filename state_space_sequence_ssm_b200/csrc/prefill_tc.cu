@@ -881,14 +881,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 break;
             }
             tc_fence_after();
-            if (!SUM) {
-                // ---- D. decay mask S -> P (TMEM): half 0 takes column blocks 0 and 3,
-                //      half 1 blocks 1 and 2 (balances the lower triangle)
+            // ---- D. decay mask S -> P (TMEM): half 0 takes column blocks 0 and 3,
+            //      half 1 blocks 1 and 2 (balances the lower triangle).  The plain
+            //      kernel takes it before the carried-state update, so that Yd runs
+            //      under the update; the optional features' instantiations measured
+            //      2 % slower that way (register allocation) and take it after.
+            constexpr bool kMaskFirst = !GEN && !BCN;
+            auto decay_mask = [&]() {
                 mask_to_tmem<R, Q>(hf == 0 ? 0 : 1, hf == 0 ? 3 : 2, wq, lq, tl, cAl2, gam, ghat, colf);
                 tc_fence_before();
                 named_bar(kBarState, kSt);
                 if (lt == 0) mbar_arrive(bb.p);
-            }
+            };
+            if (kMaskFirst && !SUM) decay_mask();
             // ---- E. carried state: h* <- Rot(-Phi)(exp(cA_end) h* + G), fp32 in registers
             {
                 const float eA = ex2(cAl2[Q - 1]);
@@ -921,6 +926,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (SUM) mbar_arrive(&bb.empty_x[sx]);  // x tile and scalars consumed
             }
             if (SUM) continue;
+            if (!kMaskFirst) decay_mask();
 
             // ---- F. epilogue: y = Yd + exp(cA_t) Yo + D x, this thread's 32 columns
             if (bar_any<kBarState, kSt>(!mbar_wait(bb.yd, lc & 1, abort_flag, err, kErrWaitMma))) {
