@@ -112,7 +112,7 @@ struct Cfg {
     // scales of the chunk's B and C tiles [2][128]
     static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16 + 2 * R * K2 + 2 * kRows;
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
-    static constexpr uint32_t NBARS = 19;
+    static constexpr uint32_t NBARS = 20;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024 alignment
     static_assert(K2 % 4 == 0 && kPro % G4 == 0, "pair groups must tile the prologue threads");
@@ -313,6 +313,7 @@ __device__ __forceinline__ void mask_to_tmem(int cbA, int cbB, int wq, int row, 
 
 struct Bars {
     uint64_t *full_bc, *empty_bc, *full_x, *empty_x, *ops, *sg, *hrdy, *p, *yd, *drain, *sc;
+    uint64_t *sd;  // S of the chunk done (the plain kernel's mask starts on it, before G and Yo)
 };
 
 // Pass kinds.  kWhole: the full forward pass, one CTA per sequence.
@@ -354,7 +355,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     float *rsc = reinterpret_cast<float *>(sbias + 2 * R * C::K2);  // BC-norm row scales [B, C][128]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     Bars bb{bars, bars + 2, bars + 4, bars + 7, bars + 10, bars + 11, bars + 12, bars + 13, bars + 14, bars + 15,
-            bars + 16};
+            bars + 16, bars + 19};
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     // first chunk of this CTA's segment, re-read where needed (a register
@@ -387,6 +388,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         mbar_init(bb.p, 1);
         mbar_init(bb.yd, 1);
         mbar_init(bb.drain, 1);
+        mbar_init(bb.sd, 1);
         *abort_flag = 0;
         *chunk0 = SEGD ? (int)(blockIdx.x / (uint32_t)a.BH) * a.cpseg : 0;
         fence_mbar_init();
@@ -499,6 +501,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                             const uint64_t o = (uint64_t)((kb * 16384 + kk * 32) >> 4);
                             mma_bf16(tbase + kColS, dCk + o, dBk + o, idS, (kb | kk) != 0);
                         }
+                    mma_commit(bb.sd);
                 }
                 // G(i) and Yo(i) once the state warpgroup has consumed G(i-1) and
                 // published h*_{i-1} (completion i of hrdy; the first is the initial state)
@@ -873,27 +876,39 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const float *cosE = colf + Q;
             const float *sinE = cosE + K2;
             const uint8_t *xst = smem + C::OFF_X + sx * C::X_BYTES;
-            // scalars of chunk c (release/acquire through sc), its x tile, and G(c)
+            // ---- D. decay mask S -> P (TMEM): half 0 takes column blocks 0 and 3,
+            //      half 1 blocks 1 and 2 (balances the lower triangle).  The plain
+            //      kernel takes it before the carried-state update, so that Yd runs
+            //      under the update; for N = 64 it starts as soon as S is done (G
+            //      and Yo finish meanwhile; for N = 128 that measured slower).  The
+            //      optional features' instantiations measured 2 % slower with the
+            //      mask first (register allocation) and take it after the update.
+            constexpr bool kMaskFirst = !GEN && !BCN && !SUM;
+            constexpr bool kMaskOnS = kMaskFirst && N == 64;
+            // scalars of chunk c (release/acquire through sc), its x tile, and
+            // S(c) (mask on S alone) or S, G and Yo of chunk c
             if (bar_any<kBarState, kSt>(!mbar_wait(&bb.sc[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
                                         !mbar_wait(&bb.full_x[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitTma) ||
-                                        !mbar_wait(bb.sg, lc & 1, abort_flag, err, kErrWaitMma))) {
+                                        !mbar_wait(kMaskOnS ? bb.sd : bb.sg, lc & 1, abort_flag, err,
+                                                   kErrWaitMma))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            // ---- D. decay mask S -> P (TMEM): half 0 takes column blocks 0 and 3,
-            //      half 1 blocks 1 and 2 (balances the lower triangle).  The plain
-            //      kernel takes it before the carried-state update, so that Yd runs
-            //      under the update; the optional features' instantiations measured
-            //      2 % slower that way (register allocation) and take it after.
-            constexpr bool kMaskFirst = !GEN && !BCN;
             auto decay_mask = [&]() {
                 mask_to_tmem<R, Q>(hf == 0 ? 0 : 1, hf == 0 ? 3 : 2, wq, lq, tl, cAl2, gam, ghat, colf);
                 tc_fence_before();
                 named_bar(kBarState, kSt);
                 if (lt == 0) mbar_arrive(bb.p);
             };
-            if (kMaskFirst && !SUM) decay_mask();
+            if (kMaskFirst) decay_mask();
+            if (kMaskOnS) {  // G(c) and Yo(c), for the update below and the epilogue
+                if (bar_any<kBarState, kSt>(!mbar_wait(bb.sg, lc & 1, abort_flag, err, kErrWaitMma))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
             // ---- E. carried state: h* <- Rot(-Phi)(exp(cA_end) h* + G), fp32 in registers
             {
                 const float eA = ex2(cAl2[Q - 1]);
