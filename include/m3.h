@@ -141,22 +141,28 @@ typedef enum m3_algo {
 
 /* The tensor-core path forced to split every sequence into s >= 1 segments
  * (fewer if the sequence has fewer chunks); M3_ALGO_TC and M3_ALGO_AUTO
- * choose the number themselves.  A split sequence runs as three launches:
- * a summary pass (each segment's local end state from a zero state and its
- * transition exp(sum dt A) Rot(-sum dt theta)), a scan of those summaries
- * across the segments -- the chunk-state recurrence of "La dualità: Mamba-2
- * e Mamba-3", section "Perché conviene: i tensor core", applied one level up
- * -- and the full pass of every segment from its scanned initial state, so
- * that a few long sequences still fill every SM. */
+ * choose the number themselves.  A split sequence runs as two launches, so
+ * that a few long sequences still fill every SM: a summary pass (each
+ * segment's local end state from a zero state and its transition
+ * exp(sum dt A) Rot(-sum dt theta), published with a release flag) and the
+ * full pass of every segment, launched as a programmatic dependent of the
+ * summary pass (its CTAs take SMs as summary CTAs finish), in which the CTA
+ * of segment j first scans the published summaries of segments 0 .. j-1
+ * into its initial state -- the chunk-state recurrence of "La dualità:
+ * Mamba-2 e Mamba-3", section "Perché conviene: i tensor core", applied one
+ * level up -- waiting (bounded, error 0x8 on expiry) for any not yet
+ * published. */
 #define M3_ALGO_TC_SEGMENTS(s) (M3_ALGO_TC | ((int)(s) << 8))
 
 /* Bytes of device workspace m3_scan_fwd needs for these dims (0 = none; the
  * workspace pointer may then be NULL).  Host function; the answer depends on
  * the current CUDA device's SM count (it sets how sequences are split).  The
  * workspace (16-byte aligned) holds fp32 per-segment states of split
- * sequences, [segments][batch*nheads][dstate][headdim + 1]; it needs no
- * initialisation, its contents are meaningless after the call, and calls that
- * may run at the same time (other streams) must not share one. */
+ * sequences, [segments][batch*nheads][dstate][headdim + 1], and one 32-bit
+ * flag per segment and sequence (zeroed by the call itself, on its stream);
+ * it needs no initialisation, its contents are meaningless after the call,
+ * and calls that may run at the same time (other streams) must not share
+ * one. */
 M3_API m3_status m3_scan_workspace_size(const m3_dims *d, size_t *bytes);
 
 /* How m3_scan_fwd_algo(algo, d, ...) will run on the current device:
@@ -347,7 +353,9 @@ M3_API m3_status m3_step_bcnorm(const m3_dims *d, const m3_bcnorm *bcn,
  * stream: the call reports (and clears) a wait that gave up in a kernel of
  * any stream of the current device, whatever `stream` is.  The code in the
  * message tells which wait: 0x1 a tile copy, 0x2 a tensor-core MMA (of either
- * prefill kernel), 0x4 the other warps of the prefill CTA, 0x10 the
+ * prefill kernel), 0x4 the other warps of the prefill CTA, 0x8 a split
+ * sequence's wait for an earlier segment (or, in its last segment, for the
+ * first to have read the initial state), 0x10 the
  * self-test; the same bits shifted
  * left by 8 come from the decode kernels.  A device-side wait gives up only on
  * a library bug; this call exists so that such a failure surfaces as a status

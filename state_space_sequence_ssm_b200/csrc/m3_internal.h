@@ -30,8 +30,8 @@ struct Problem {
 
 // How the tensor-core prefill runs one problem: every sequence in `nseg`
 // segments of `cpseg` chunks (nseg = 1: one CTA per sequence, one launch;
-// nseg > 1: summary pass, segment scan, main pass = three launches and a
-// workspace of ws_bytes); `ctas` CTAs in the (main) launch.
+// nseg > 1: summary pass, then the main pass with its look-back = two
+// launches and a workspace of ws_bytes); `ctas` CTAs in the (main) launch.
 struct TcPlan {
     int nchunks, cpseg, nseg, launches;
     int64_t ctas;

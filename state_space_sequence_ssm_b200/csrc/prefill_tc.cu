@@ -35,8 +35,8 @@
 //               ahead);
 //   warp 17     TMEM owner and single-thread MMA issuer.
 // A sequence too long for the grid to fill the GPU is split into segments
-// (a summary pass, a scan over the segments, then this pass per segment:
-// the MODE template argument).
+// (a summary pass, then this pass per segment, which first scans the
+// summaries of the segments before its own: the MODE template argument).
 // Every wait is bounded; a wait that gives up records a code that the host
 // reads back with m3_stream_status() and the CTA drains and returns.
 #include <cuda.h>
@@ -77,10 +77,11 @@ constexpr int kNX = 3;   // x tile stages (also the number of per-chunk scalar b
 constexpr uint32_t kBarPro = 1, kBarState = 2;  // named barriers of the two warpgroups
 constexpr float kLog2e = 1.4426950408889634f;
 // Sequence splitting (host policy): at most kMaxSegments segments of at least
-// kMinSegChunks chunks; the summary pass costs about kSumCost of the full pass
-// per chunk and the segment scan about kScanCost chunk-times.
+// kMinSegChunks chunks; a summary-pass chunk costs about kSumCost of a
+// main-pass chunk, and every CTA about kCtaCost chunk-times of its own
+// (launch, set-up, pipeline fill and drain).
 constexpr int64_t kMaxSegments = 64, kMinSegChunks = 8;
-constexpr double kSumCost = 0.55, kScanCost = 2.0;
+constexpr double kSumCost = 0.55, kCtaCost = 2.0;
 
 template <int N, int R>
 struct Cfg {
@@ -133,11 +134,15 @@ struct TcArgs {
     float eps;
     __nv_bfloat16 *y;
     float *hT, *bpT, *xpT;
-    // Split sequences: ws_h [nseg][BH][N][P] fp32 holds, per segment j, the
-    // summary pass's local end state (slot j + 1) and after the segment scan the
-    // pending-inclusive state entering segment j (slot j); ws_m [nseg][BH][N]
-    // holds segment j's transition exp(cA) Rot(-Phi) as (e cos, e sin) per pair.
+    // Split sequences: ws_h [nseg][BH][N][P] fp32 holds in slot j + 1 the
+    // summary pass's local end state of segment j; ws_m [nseg][BH][N] holds
+    // segment j's transition exp(cA) Rot(-Phi) as (e cos, e sin) per pair;
+    // flags [nseg][BH] (zeroed before the summary pass): [j][bh] for j <
+    // nseg - 1 is set to 1 once segment j's summary is published (2 if that
+    // CTA gave up), [nseg - 1][bh] once the main pass has read the caller's
+    // initial state (the last segment overwrites it when resumed in place).
     float *ws_h, *ws_m;
+    unsigned *flags;
 };
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
@@ -320,8 +325,8 @@ struct Bars {
 // kSummary: the summary pass of a split sequence -- only the chunk states and
 // the carried-state chain over one segment, from a zero state (segment 0: the
 // caller's initial state), ending in the segment's local end state and its
-// transition, for the segment scan.  kSegment: the full forward pass over one
-// segment, from the scanned state.
+// transition, published for the main pass.  kSegment: the full forward pass
+// over one segment, from the scan of the summaries before it (look-back).
 constexpr int kWhole = 0, kSummary = 1, kSegment = 2;
 
 // GEN = false: the plain method (A per head, theta per token), compiled
@@ -372,6 +377,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int64_t b = bh / H, h = bh % H;
     auto tok = [&](int64_t t) { return (b * T + t) * H + h; };
 
+    // the main pass is launched as a programmatic dependent of the summary
+    // pass: its CTAs take SMs as summary CTAs leave them, and all summary CTAs
+    // are resident (or done) before any of them starts, so its bounded waits
+    // on their flags always wait on running CTAs
+    if (SUM && tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bb.full_bc[i], 1);
@@ -830,17 +840,57 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const int c0 = 32 * hf;            // first column of this thread's half
         float hreg[32];
         // Pending-inclusive state entering the segment.  The whole sequence and
-        // segment 0 of the summary pass: the caller's h0 + beta'_0 b_prev
-        // x_prev^T (pending write of token -1); later summary segments: zero
-        // (their local state); segments of the main pass: the scanned state.
+        // segment 0 of either pass: the caller's h0 + beta'_0 b_prev x_prev^T
+        // (pending write of token -1); later summary segments: zero (their
+        // local state); later segments of the main pass: the scan of the
+        // published summaries of the segments before it (look-back).
+        bool ok = true;
         {
 #pragma unroll
             for (int p = 0; p < 32; ++p) hreg[p] = 0.f;
-            if (MODE == kSegment) {
-                if (own_state) {
-                    const float *hin = a.ws_h + ((int64_t)seg * BH + bh) * N * kP;
+            if (MODE == kSegment && seg > 0) {
+                // Every earlier segment's summary (bounded waits; the summary
+                // CTAs are all resident or done), then S_1 = L_0 and S_{j+1} =
+                // M_j S_j + L_j, with L_j in slot j + 1 and M_j acting on row pairs
+                // exactly like the chunk-to-chunk update.
+                if (bar_any<kBarState, kSt>(lt == 0 && [&] {
+                        for (int j = 0; j < seg; ++j)
+                            if (!flag_wait(a.flags + (int64_t)j * BH + bh, abort_flag, err, kErrWaitSegment))
+                                return true;
+                        return false;
+                    }())) {
+                    ok = false;
+                } else {
+                    const int rr = own_state ? srow : 0;
+                    const int64_t slot = (int64_t)BH * N * kP;
+                    const float *hs = a.ws_h + slot + bh * N * kP + rr * kP + c0;
 #pragma unroll
-                    for (int p = 0; p < 32; ++p) hreg[p] = hin[srow * kP + c0 + p];
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(hs) + q);
+                        hreg[4 * q] = v.x;
+                        hreg[4 * q + 1] = v.y;
+                        hreg[4 * q + 2] = v.z;
+                        hreg[4 * q + 3] = v.w;
+                    }
+                    for (int j = 1; j < seg; ++j) {
+                        const float2 m =
+                            __ldcg(reinterpret_cast<const float2 *>(a.ws_m + ((int64_t)j * BH + bh) * N + (rr & ~1)));
+                        const float ms = (rr & 1) ? -m.y : m.y;
+                        float4 l[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            l[q] = __ldcg(reinterpret_cast<const float4 *>(hs + (int64_t)j * slot) + q);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float lv[4] = {l[q].x, l[q].y, l[q].z, l[q].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float u = hreg[4 * q + e];
+                                const float o = __shfl_xor_sync(0xffffffffu, u, 1);
+                                hreg[4 * q + e] = fmaf(m.x, u, fmaf(ms, o, lv[e]));
+                            }
+                        }
+                    }
                 }
             } else if (seg == 0) {
                 const float betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
@@ -865,9 +915,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         float m_l2 = 0.f, m_cs = 1.f, m_sn = 0.f;
         fence_proxy_async_smem();
         named_bar(kBarState, kSt);
-        if (lt == 0) mbar_arrive(bb.hrdy);
-        bool ok = true;
-        for (int lc = 0; lc < nloc; ++lc) {
+        if (lt == 0) {
+            mbar_arrive(bb.hrdy);
+            // the caller's initial state is read (the last segment may now overwrite it)
+            if (MODE == kSegment && seg == 0) flag_release(a.flags + (int64_t)(a.nseg - 1) * BH + bh, 1u);
+        }
+        for (int lc = 0; ok && lc < nloc; ++lc) {
             const int sx = lc % kNX;
             const float *cAl2 = sbuf + sx * C::SB;
             const float *gam = cAl2 + Q;
@@ -1001,8 +1054,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         make_float2(e * m_cs, e * m_sn);
                 }
             }
-        } else if (ok && (!SEGD || seg == a.nseg - 1)) {
+            __threadfence();  // before the flag release below
+        } else if (ok && (!SEGD || seg == a.nseg - 1) &&
+                   !(MODE == kSegment &&
+                     bar_any<kBarState, kSt>(lt == 0 && !flag_wait(a.flags + (int64_t)(a.nseg - 1) * BH + bh,
+                                                                   abort_flag, err, kErrWaitSegment)))) {
             // ---- final state: plain-frame h_{T-1}, raw last token as the pending term
+            //      (the last segment of a split sequence: once segment 0 has read
+            //      the initial state, which this may overwrite)
             if (a.hT && own_state) {
                 float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * N + srow) * kP + c0);
 #pragma unroll
@@ -1031,74 +1090,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     __syncwarp();  // reconverge the single-lane roles before the block barrier
     tc_fence_before();
     __syncthreads();
+    if (SUM && tid == 0) flag_release(a.flags + (int64_t)seg * BH + bh, *abort_flag ? 2u : 1u);
     if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
     }
-}
-
-// ---------------------------------------------------------------- segment scan
-// Exclusive scan over the segments of each split sequence, element-wise on the
-// N x P state: slot 0 <- h0 + beta'_0 b_prev x_prev^T (the pending-inclusive
-// state before token 0); slot 1 already holds segment 0's end state (its
-// summary pass started from the caller's state); slot j >= 2 <- M_{j-1}
-// slot(j-1) + slot j, M_{j-1} = exp(cA) Rot(-Phi) of segment j-1.  The same
-// linear recurrence as the carried state between chunks, one level up.
-struct ScanArgs {
-    int64_t BH, H, T;
-    int nseg;
-    const __nv_bfloat16 *dt, *lam;
-    const float *h0, *bp0, *xp0;
-    float *ws_h;
-    const float *ws_m;
-};
-
-template <int N, int R>
-__global__ void __launch_bounds__(256) segment_scan_kernel(const ScanArgs a) {
-    constexpr int QD = kP / 4;  // column quads of a state row
-    const int64_t bh = blockIdx.x;
-    const int64_t b = bh / a.H, h = bh % a.H;
-    const bool pend = a.bp0 && a.xp0;
-    const int64_t t0 = (b * a.T) * a.H + h;  // token 0 of this sequence
-    const float betap0 = pend ? (1.f - bf(a.lam, t0)) * bf(a.dt, t0) : 0.f;
-    const int64_t slot = a.BH * N * kP;
-    float *base = a.ws_h + bh * N * kP;
-    for (int it = threadIdx.x; it < (N / 2) * QD; it += blockDim.x) {
-        const int k = it / QD, col = 4 * (it % QD);
-        const int ru = 2 * k, rv = 2 * k + 1;
-        float4 u = make_float4(0.f, 0.f, 0.f, 0.f), v = u;
-        if (a.h0) {
-            u = *reinterpret_cast<const float4 *>(a.h0 + (bh * N + ru) * kP + col);
-            v = *reinterpret_cast<const float4 *>(a.h0 + (bh * N + rv) * kP + col);
-        }
-        if (pend) {
-            for (int r = 0; r < R; ++r) {
-                const float wu = betap0 * a.bp0[(bh * R + r) * N + ru];
-                const float wv = betap0 * a.bp0[(bh * R + r) * N + rv];
-                const float4 xq = *reinterpret_cast<const float4 *>(a.xp0 + (bh * R + r) * kP + col);
-                u = make_float4(fmaf(wu, xq.x, u.x), fmaf(wu, xq.y, u.y), fmaf(wu, xq.z, u.z), fmaf(wu, xq.w, u.w));
-                v = make_float4(fmaf(wv, xq.x, v.x), fmaf(wv, xq.y, v.y), fmaf(wv, xq.z, v.z), fmaf(wv, xq.w, v.w));
-            }
-        }
-        *reinterpret_cast<float4 *>(base + ru * kP + col) = u;
-        *reinterpret_cast<float4 *>(base + rv * kP + col) = v;
-        if (a.nseg < 2) continue;
-        u = *reinterpret_cast<const float4 *>(base + slot + ru * kP + col);
-        v = *reinterpret_cast<const float4 *>(base + slot + rv * kP + col);
-        for (int j = 2; j < a.nseg; ++j) {
-            const float2 m = *reinterpret_cast<const float2 *>(a.ws_m + ((int64_t)(j - 1) * a.BH + bh) * N + ru);
-            float *pu = base + j * slot + ru * kP + col, *pv = base + j * slot + rv * kP + col;
-            const float4 cu = *reinterpret_cast<const float4 *>(pu), cv = *reinterpret_cast<const float4 *>(pv);
-            const float4 nu = make_float4(fmaf(m.x, u.x, fmaf(m.y, v.x, cu.x)), fmaf(m.x, u.y, fmaf(m.y, v.y, cu.y)),
-                                          fmaf(m.x, u.z, fmaf(m.y, v.z, cu.z)), fmaf(m.x, u.w, fmaf(m.y, v.w, cu.w)));
-            const float4 nv = make_float4(fmaf(m.x, v.x, fmaf(-m.y, u.x, cv.x)), fmaf(m.x, v.y, fmaf(-m.y, u.y, cv.y)),
-                                          fmaf(m.x, v.z, fmaf(-m.y, u.z, cv.z)), fmaf(m.x, v.w, fmaf(-m.y, u.w, cv.w)));
-            *reinterpret_cast<float4 *>(pu) = nu;
-            *reinterpret_cast<float4 *>(pv) = nv;
-            u = nu;
-            v = nv;
-        }
-    }
+    // the main pass completes only after the summary pass (so that later work
+    // on the stream finds both done)
+    if (MODE == kSegment && tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- host side
@@ -1147,14 +1146,27 @@ bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// `dependent`: launched as a programmatic dependent of the previous kernel on
+// the stream (the main pass of a split sequence after its summary pass).
 template <int N, int R, int MODE, bool GEN, bool BCN>
 cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc, const CUtensorMap &mt,
-                        const TcArgs &a, int64_t ctas, cudaStream_t stream) {
+                        const TcArgs &a, int64_t ctas, cudaStream_t stream, bool dependent = false) {
     using C = Cfg<N, R>;
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, GEN, BCN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<N, R, MODE, GEN, BCN><<<(unsigned)ctas, kThreads, C::SMEM_BYTES, stream>>>(mx, mb, mc, mt, a);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<N, R, MODE, GEN, BCN>, mx, mb, mc, mt, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -1201,32 +1213,22 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
         a.xpT = p.xpT;
         return launch_pass<N, R, kWhole, GEN, BCN>(mx, mb, mc, mt, a, BH, p.stream);
     }
-    // split sequences: summary pass over segments 0 .. nseg-2, segment scan,
-    // then the main pass over all segments from the scanned states
+    // split sequences: the summary pass over segments 0 .. nseg-2 publishes
+    // each segment's local end state and transition; the main pass over all
+    // segments, launched as its programmatic dependent, scans the published
+    // summaries of the segments before its own (look-back)
     a.ws_h = static_cast<float *>(p.ws);
     a.ws_m = a.ws_h + (size_t)plan.nseg * BH * N * kP;
-    cudaError_t e = launch_pass<N, R, kSummary, GEN, BCN>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
+    a.flags = reinterpret_cast<unsigned *>(a.ws_m + (size_t)plan.nseg * BH * N);
+    cudaError_t e = cudaMemsetAsync(a.flags, 0, (size_t)plan.nseg * BH * sizeof(unsigned), p.stream);
     if (e != cudaSuccess) return e;
-    ScanArgs sa{};
-    sa.BH = BH;
-    sa.H = p.H;
-    sa.T = p.T;
-    sa.nseg = plan.nseg;
-    sa.dt = a.dt;
-    sa.lam = a.lam;
-    sa.h0 = p.h0;
-    sa.bp0 = p.bp0;
-    sa.xp0 = p.xp0;
-    sa.ws_h = a.ws_h;
-    sa.ws_m = a.ws_m;
-    segment_scan_kernel<N, R><<<(unsigned)BH, 256, 0, p.stream>>>(sa);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    a.h0 = a.bp0 = a.xp0 = nullptr;  // the main pass reads only the scanned states
+    e = launch_pass<N, R, kSummary, GEN, BCN>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
+    if (e != cudaSuccess) return e;
     a.y = (__nv_bfloat16 *)p.y;
     a.hT = p.hT;
     a.bpT = p.bpT;
     a.xpT = p.xpT;
-    return launch_pass<N, R, kSegment, GEN, BCN>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream);
+    return launch_pass<N, R, kSegment, GEN, BCN>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream, true);
 }
 
 bool device_is_sm100() {
@@ -1250,6 +1252,11 @@ bool prefill_tc_supported(const Problem &p, const char **why) {
     return true;
 }
 
+// workspace of a split call: the local end states, the transitions and the flags
+static size_t split_ws_bytes(int64_t S, int64_t BH, int64_t N, int64_t P) {
+    return (size_t)S * BH * (N * (P + 1) * sizeof(float) + sizeof(unsigned));
+}
+
 TcPlan prefill_tc_plan(const Problem &p) {
     TcPlan plan{};
     const int64_t Q = kRows / p.R;
@@ -1259,19 +1266,39 @@ TcPlan prefill_tc_plan(const Problem &p) {
     if (p.segments > 0) {
         S = p.segments;
     } else {
-        // Split a sequence only when it shortens the estimated critical path:
-        // waves of one CTA per SM, a summary chunk costing kSumCost of a full
-        // one, segments of at least kMinSegChunks chunks.
+        // Split a sequence only when it shortens the estimated time: one CTA
+        // per SM taken in launch order, the BH (S - 1) summary CTAs first, then
+        // the BH S main-pass CTAs as SMs come free; segments of at least
+        // kMinSegChunks chunks.
         int dev = 0, nsm = 148;
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
         if (nsm < 1) nsm = 1;
-        auto waves = [&](int64_t ctas) { return (double)((ctas + nsm - 1) / nsm); };
-        double best = waves(BH) * (double)nch;
+        // finishing time of n1 CTAs of length t1 followed by n2 of length t2:
+        // after the first kind the SMs form two groups (the last, partial wave
+        // of summary CTAs and the rest) that stay in lock step
+        auto makespan = [&](int64_t n1, double t1, int64_t n2, double t2) {
+            const int64_t w1 = n1 / nsm, r1 = n1 % nsm;
+            double ta = (double)w1 * t1, tb = (double)(w1 + 1) * t1, end = r1 ? tb : ta;
+            int64_t ca = nsm - r1, cb = r1, rem = n2;
+            while (rem > 0) {
+                if (cb == 0 || (ca > 0 && ta <= tb)) {
+                    rem -= ca < rem ? ca : rem;
+                    ta += t2;
+                    end = end > ta ? end : ta;
+                } else {
+                    rem -= cb < rem ? cb : rem;
+                    tb += t2;
+                    end = end > tb ? end : tb;
+                }
+            }
+            return end;
+        };
+        double best = makespan(0, 0.0, BH, (double)nch + kCtaCost);
         for (int64_t s = 2; s <= kMaxSegments && s * kMinSegChunks <= nch; ++s) {
             const int64_t L = (nch + s - 1) / s, Se = (nch + L - 1) / L;
             if (Se != s) continue;
-            if (p.ws_cap && (size_t)Se * BH * p.N * (p.P + 1) * sizeof(float) > p.ws_cap) break;
-            const double cost = waves(BH * Se) * L + waves(BH * (Se - 1)) * L * kSumCost + kScanCost;
+            if (p.ws_cap && split_ws_bytes(Se, BH, p.N, p.P) > p.ws_cap) break;
+            const double cost = makespan(BH * (Se - 1), L * kSumCost + kCtaCost, BH * Se, (double)L + kCtaCost);
             if (cost < best * 0.97) {
                 best = cost;
                 S = s;
@@ -1285,9 +1312,9 @@ TcPlan prefill_tc_plan(const Problem &p) {
     plan.nchunks = (int)nch;
     plan.cpseg = (int)L;
     plan.nseg = (int)S;
-    plan.launches = S > 1 ? 3 : 1;
+    plan.launches = S > 1 ? 2 : 1;
     plan.ctas = BH * S;
-    plan.ws_bytes = S > 1 ? (size_t)S * BH * p.N * (p.P + 1) * sizeof(float) : 0;
+    plan.ws_bytes = S > 1 ? split_ws_bytes(S, BH, p.N, p.P) : 0;
     return plan;
 }
 

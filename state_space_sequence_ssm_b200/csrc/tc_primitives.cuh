@@ -17,6 +17,7 @@ enum : unsigned {
     kErrWaitTma = 1u << 0,
     kErrWaitMma = 1u << 1,
     kErrWaitCompute = 1u << 2,
+    kErrWaitSegment = 1u << 3,   // a split sequence's wait for an earlier segment's summary
     kErrWaitSelftest = 1u << 4,  // the self-test wait of m3_selftest_wait_timeout
 };
 
@@ -70,6 +71,40 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             }
         }
     }
+}
+
+// ---------------------------------------------------------------- flags in global memory
+// Publication of a result to other CTAs of the device: the writer's stores,
+// then a release store of the flag; the reader acquires the flag and reads the
+// result past L1 (ld.global.cg).
+__device__ __forceinline__ void flag_release(unsigned *f, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned flag_acquire(const unsigned *f) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+// Bounded wait for a flag to leave 0.  Returns true when it reads 1; false
+// when it reads anything else (the writer gave up and recorded its own
+// failure), when another role has raised `abort`, or after `budget` cycles
+// (then it raises `abort` and records `code`).
+__device__ __forceinline__ bool flag_wait(const unsigned *f, volatile int *abort, unsigned *err_word,
+                                          unsigned code, long long budget = 4000000000LL) {
+    unsigned v = flag_acquire(f);
+    const long long t0 = clock64();
+    while (v == 0u) {
+        __nanosleep(128);
+        if (abort && *abort) return false;
+        if (clock64() - t0 > budget) {
+            if (abort) *abort = 1;
+            atomicOr(err_word, code);
+            return false;
+        }
+        v = flag_acquire(f);
+    }
+    if (v != 1u && abort) *abort = 1;
+    return v == 1u;
 }
 
 // ---------------------------------------------------------------- fences

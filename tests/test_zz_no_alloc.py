@@ -57,9 +57,9 @@ def test_static_plan_reports_the_capped_segment_choice():
     scratch, the static entry point splits into fewer segments; the plan
     query with M3_PLAN_STATIC says so, and both calls agree within the bf16
     bar (they differ only in where the sequence is cut)."""
-    # 30 sequences of 2048 chunks: the free choice is 29 segments (27 MiB of
-    # per-segment states), the scratch admits 14
-    s = Shape(1, 65536, 30, 64, 128, 4, "bf16", 75)
+    # 50 sequences of 1280 chunks: the free choice is 21 segments (33 MiB of
+    # per-segment states), the scratch admits 9
+    s = Shape(1, 40960, 50, 64, 128, 4, "bf16", 75)
     free = m3.scan_plan_info(_dims(s))
     capped = m3.scan_plan_info(_dims(s), flags=m3.PLAN_STATIC)
     assert free.workspace_bytes > 24 << 20 >= capped.workspace_bytes > 0
