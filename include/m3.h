@@ -72,7 +72,8 @@ typedef enum m3_status {
     M3_ERR_INVALID_ARG = 1,  /* null/misaligned/overlapping pointer, bad size */
     M3_ERR_UNSUPPORTED = 2,  /* valid sizes outside what the kernels support   */
     M3_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed          */
-    M3_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up            */
+    M3_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up            */
+    M3_ERR_BOUNDS = 5        /* a device-side index check failed (bounds build) */
 } m3_status;
 
 typedef enum m3_dtype { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
@@ -357,7 +358,9 @@ M3_API m3_status m3_step_bcnorm(const m3_dims *d, const m3_bcnorm *bcn,
  * sequence's wait for an earlier segment (or, in its last segment, for the
  * first to have read the initial state), 0x10 the
  * self-test; the same bits shifted
- * left by 8 come from the decode kernels.  A device-side wait gives up only on
+ * left by 8 come from the decode kernels.  In the bounds build it also
+ * returns M3_ERR_BOUNDS (after any timeout) if a device index check failed
+ * (m3_device_checks).  A device-side wait gives up only on
  * a library bug; this call exists so that such a failure surfaces as a status
  * instead of a hang.
  * The library keeps, per device and for the life of the process, the
@@ -377,8 +380,21 @@ M3_API m3_status m3_selftest_wait_timeout(void *stream);
 /* Message describing the calling thread's most recent failure ("" if none). */
 M3_API const char *m3_last_error(void);
 
+/* 1 in the bounds build of the library (libm3_bounds.so, compiled with
+ * M3_DEVICE_CHECKS), 0 in the normal build.  In the bounds build every
+ * kernel checks each global-memory access it makes through a plain pointer
+ * against the extent of its buffer (computed from the call's dims); a failed
+ * check skips the access (a read gives 0; a bulk copy reads from the
+ * buffer's start instead) and records the site, the index and the extent of
+ * the first failure, and m3_stream_status then returns M3_ERR_BOUNDS with
+ * them in m3_last_error (and clears the record).  Tile copies (TMA) carry
+ * their own extents and are not checked.  Same ABI and results as the normal
+ * build, slower.  The pages have no counterpart to it. */
+M3_API int m3_device_checks(void);
+
 /* ABI version of this header (major * 100 + minor): 101 adds m3_scan_plan_info,
- * 102 the fp32 tensor-core prefill (M3_KERNEL_TC32). */
+ * 102 the fp32 tensor-core prefill (M3_KERNEL_TC32), 103 the bounds build
+ * (m3_device_checks, M3_ERR_BOUNDS) and split sequences in two launches. */
 M3_API int m3_version(void);
 
 #ifdef __cplusplus

@@ -4,7 +4,9 @@ Argument marshalling only: every step of the method runs in the CUDA
 library ``libm3.so`` built from ``csrc/``.  PyTorch supplies device memory and
 streams.  There is no fallback: if the library is missing, the first call
 raises ImportError, and every call checks that its tensors live on a CUDA
-device.
+device.  With ``M3_BOUNDS=1`` in the environment when the library is first
+loaded, the binding loads the bounds build ``libm3_bounds.so`` instead (the
+same ABI with device-side index checks; ``device_checks()`` tells which).
 """
 from __future__ import annotations
 
@@ -16,8 +18,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libm3.so")
+BOUNDS_LIB_PATH = os.path.join(_HERE, "libm3_bounds.so")
 
-M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
+M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT, M3_ERR_BOUNDS = range(6)
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_A_PER_TOKEN = 1
 M3_FLAG_THETA_PER_HEAD = 2
@@ -30,7 +33,8 @@ def ALGO_TC_SEGMENTS(s: int) -> int:
     """The tensor-core path with every sequence split into `s` segments."""
     return ALGO_TC | (int(s) << 8)
 
-_STATUS = {0: "M3_OK", 1: "M3_ERR_INVALID_ARG", 2: "M3_ERR_UNSUPPORTED", 3: "M3_ERR_CUDA", 4: "M3_ERR_TIMEOUT"}
+_STATUS = {0: "M3_OK", 1: "M3_ERR_INVALID_ARG", 2: "M3_ERR_UNSUPPORTED", 3: "M3_ERR_CUDA", 4: "M3_ERR_TIMEOUT",
+           5: "M3_ERR_BOUNDS"}
 
 
 class Dims(ctypes.Structure):
@@ -79,11 +83,17 @@ class State(NamedTuple):
     x_prev: torch.Tensor  # [Bt, H, R, P] fp32
 
 
+def lib_path() -> str:
+    """The library the binding loads: the bounds build if M3_BOUNDS=1."""
+    return BOUNDS_LIB_PATH if os.environ.get("M3_BOUNDS", "") == "1" else LIB_PATH
+
+
 def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"m3 CUDA library not built ({LIB_PATH} missing); "
+    path = lib_path()
+    if not os.path.exists(path):
+        raise ImportError(f"m3 CUDA library not built ({path} missing); "
                           "run `python -m state_space_sequence_ssm_b200.build`")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     vp, dp = ctypes.c_void_p, ctypes.POINTER(Dims)
     sp = ctypes.POINTER(CState)
     lib.m3_scan_workspace_size.argtypes = [dp, ctypes.POINTER(ctypes.c_size_t)]
@@ -115,6 +125,7 @@ def _load():
     lib.m3_last_error.argtypes = []
     lib.m3_last_error.restype = ctypes.c_char_p
     lib.m3_version.restype = ctypes.c_int
+    lib.m3_device_checks.restype = ctypes.c_int
     return lib
 
 
@@ -122,7 +133,7 @@ _lib = None
 
 
 def get_lib():
-    """The loaded libm3.so (raises ImportError if it has not been built)."""
+    """The loaded library (raises ImportError if it has not been built)."""
     global _lib
     if _lib is None:
         _lib = _load()
@@ -371,9 +382,15 @@ def selftest_wait_timeout(stream=None):
         _check(get_lib().m3_selftest_wait_timeout(_stream(stream, dev)))
 
 
+def device_checks() -> bool:
+    """True when the loaded library is the bounds build (device index checks)."""
+    return bool(get_lib().m3_device_checks())
+
+
 def stream_status(stream=None):
     """Synchronise the stream and raise if a kernel's bounded wait gave up
-    (on any stream of the stream's device since the previous check)."""
+    (on any stream of the stream's device since the previous check), or, in
+    the bounds build, if a device index check failed (M3_ERR_BOUNDS)."""
     dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
     with torch.cuda.device(dev):
         _check(get_lib().m3_stream_status(_stream(stream, dev)))

@@ -251,7 +251,15 @@ m3_status set_cuda_error(cudaError_t e, const char *where) { return cuda_fail(e,
 
 extern "C" {
 
-int m3_version(void) { return 102; }
+int m3_version(void) { return 103; }
+
+int m3_device_checks(void) {
+#ifdef M3_DEVICE_CHECKS
+    return 1;
+#else
+    return 0;
+#endif
+}
 
 const char *m3_last_error(void) { return g_err.c_str(); }
 
@@ -392,11 +400,29 @@ m3_status m3_stream_status(void *stream) {
         e = m3::read_tc32_error(&tcode);
         if (e != cudaSuccess) return cuda_fail(e, "m3_stream_status");
         code |= tcode | (dcode << 8);
+        // the bounds build's index-check records (all read, so all cleared)
+        m3::DcheckRecord rec[4], first{0u, 0u, 0, 0};
+        unsigned fails = 0;
+        cudaError_t (*const readers[4])(m3::DcheckRecord *) = {m3::read_dcheck_tc, m3::read_dcheck_tc32,
+                                                                m3::read_dcheck_simt, m3::read_dcheck_decode};
+        for (int i = 0; i < 4; ++i) {
+            if ((e = readers[i](&rec[i])) != cudaSuccess) return cuda_fail(e, "m3_stream_status");
+            if (rec[i].count && !fails) first = rec[i];
+            fails += rec[i].count;
+        }
         if (code) {
             char buf[128];
             std::snprintf(buf, sizeof buf, "a bounded device-side wait gave up (code 0x%x)", code);
             g_err = buf;
             return M3_ERR_TIMEOUT;
+        }
+        if (fails) {
+            char buf[192];
+            std::snprintf(buf, sizeof buf,
+                          "device index check failed: site 0x%x, index %lld, extent %lld (%u failed checks)",
+                          first.site, first.index, first.extent, fails);
+            g_err = buf;
+            return M3_ERR_BOUNDS;
         }
         return M3_OK;
     } catch (...) {

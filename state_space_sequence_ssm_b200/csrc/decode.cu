@@ -18,6 +18,7 @@
 #include <cuda_bf16.h>
 
 #include "bcnorm.cuh"
+#include "dcheck.cuh"
 #include "m3_internal.h"
 #include "tc_primitives.cuh"
 
@@ -28,21 +29,42 @@ __device__ unsigned g_decode_error;
 
 namespace {
 
+// Index-check sites of this file (bounds build).
+enum : unsigned {
+    kSiteScalars = 0x401,  // dt, lam, A, D
+    kSiteTheta = 0x402,    // angle rates
+    kSiteVec = 0x403,      // x, B, C of the step
+    kSiteNorm = 0x404,     // BC-norm weights and biases
+    kSiteState = 0x405,    // the state h
+    kSitePend = 0x406,     // b_prev, x_prev
+    kSiteY = 0x407,        // output
+};
+
+// Element i of a buffer of n elements (the bounds build checks i and reads 0
+// outside; `site` names the access).
 template <typename T>
-__device__ __forceinline__ float ldv(const T *p, int64_t i);
+__device__ __forceinline__ float ldv(const T *p, int64_t i, int64_t n, unsigned site);
 template <>
-__device__ __forceinline__ float ldv<float>(const float *p, int64_t i) { return __ldg(p + i); }
+__device__ __forceinline__ float ldv<float>(const float *p, int64_t i, int64_t n, unsigned site) {
+    return dchk::in(site, i, 1, n) ? __ldg(p + i) : 0.f;
+}
 template <>
-__device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
-    return __bfloat162float(p[i]);
+__device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i, int64_t n, unsigned site) {
+    return dchk::in(site, i, 1, n) ? __bfloat162float(p[i]) : 0.f;
 }
 template <typename T>
-__device__ __forceinline__ void stv(T *p, int64_t i, float v);
+__device__ __forceinline__ void stv(T *p, int64_t i, int64_t n, unsigned site, float v);
 template <>
-__device__ __forceinline__ void stv<float>(float *p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void stv<float>(float *p, int64_t i, int64_t n, unsigned site, float v) {
+    if (dchk::in(site, i, 1, n)) p[i] = v;
+}
 template <>
-__device__ __forceinline__ void stv<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float v) {
-    p[i] = __float2bfloat16_rn(v);
+__device__ __forceinline__ void stv<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, int64_t n, unsigned site, float v) {
+    if (dchk::in(site, i, 1, n)) p[i] = __float2bfloat16_rn(v);
+}
+// Plain fp32 element (state side buffers, per-head parameters), checked like ldv.
+__device__ __forceinline__ float ldf(const float *p, int64_t i, int64_t n, unsigned site) {
+    return dchk::in(site, i, 1, n) ? p[i] : 0.f;
 }
 template <typename IO>
 struct StepArgs {
@@ -101,31 +123,36 @@ step_kernel(const StepArgs<IO> a, const StepFeat f) {
     const int h = (int)(bh % a.H);
     const int p0 = cg * 4;
 
+    // buffer extents in elements, for the bounds build's index checks
+    const int64_t nSt = a.BH * N * P, nBN = a.BH * R * N, nBP = a.BH * R * P;
     float4 *hst = reinterpret_cast<float4 *>(a.h + bh * N * P);
     // ---- issue the state loads first (the bulk of the bytes)
     float4 hu[PT], hv[PT];
 #pragma unroll
     for (int j = 0; j < PT; ++j) {
         const int k = kk + j * KK;
-        hu[j] = __ldcs(hst + ((2 * k) * P + p0) / 4);
-        hv[j] = __ldcs(hst + ((2 * k + 1) * P + p0) / 4);
+        const bool in = dchk::in(kSiteState, bh * N * P + (2 * k) * P + p0, P + 4, nSt);
+        hu[j] = in ? __ldcs(hst + ((2 * k) * P + p0) / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        hv[j] = in ? __ldcs(hst + ((2 * k + 1) * P + p0) / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
-    const float alpha = __expf(dtv * a.A[(GEN && f.a_tok) ? bh : h]);
+    const float dtv = ldv(a.dt, bh, a.BH, kSiteScalars), lamv = ldv(a.lam, bh, a.BH, kSiteScalars);
+    const float alpha = __expf(dtv * ldf(a.A, (GEN && f.a_tok) ? bh : h, (GEN && f.a_tok) ? a.BH : a.H, kSiteScalars));
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
     // ---- stage the slice's small vectors
     for (int i = tid; i < R * N; i += NT) {
-        (&sBp[0][0])[i] = a.bp[bh * R * N + i];
-        (&sB[0][0])[i] = ldv(a.B, bh * R * N + i);
-        (&sC[0][0])[i] = ldv(a.C, bh * R * N + i);
+        (&sBp[0][0])[i] = ldf(a.bp, bh * R * N + i, nBN, kSitePend);
+        (&sB[0][0])[i] = ldv(a.B, bh * R * N + i, nBN, kSiteVec);
+        (&sC[0][0])[i] = ldv(a.C, bh * R * N + i, nBN, kSiteVec);
     }
     for (int i = tid; i < R * P; i += NT) {
-        (&sXp[0][0])[i] = a.xp[bh * R * P + i];
-        (&sX[0][0])[i] = ldv(a.x, bh * R * P + i);
+        (&sXp[0][0])[i] = ldf(a.xp, bh * R * P + i, nBP, kSitePend);
+        (&sX[0][0])[i] = ldv(a.x, bh * R * P + i, nBP, kSiteVec);
     }
     for (int k = tid; k < K2; k += NT) {
         float sn, cs;
-        sincosf(dtv * ldv(a.theta, ((GEN && f.th_head) ? (int64_t)h : bh) * K2 + k), &sn, &cs);
+        sincosf(dtv * ldv(a.theta, ((GEN && f.th_head) ? (int64_t)h : bh) * K2 + k,
+                          ((GEN && f.th_head) ? a.H : a.BH) * K2, kSiteTheta),
+                &sn, &cs);
         sAc[k] = alpha * cs;
         sAs[k] = alpha * sn;
     }
@@ -137,9 +164,10 @@ step_kernel(const StepArgs<IO> a, const StepFeat f) {
             const int r = isB ? row : row - R;
             float *v = isB ? sB[r] : sC[r];
             const float *w = isB ? f.wB : f.wC;
-            const float *bias = (isB ? f.bB : f.bC) + (h * R + r) * N;
+            const float *bias = isB ? f.bB : f.bC;
             const float sc = bcn_row_scale_warp([&](int n) { return v[n]; }, N, f.eps);
-            for (int n = lane; n < N; n += 32) v[n] = fmaf(v[n] * sc, w[n], bias[n]);
+            for (int n = lane; n < N; n += 32)
+                v[n] = fmaf(v[n] * sc, ldf(w, n, N, kSiteNorm), ldf(bias, (h * R + r) * N + n, a.H * R * N, kSiteNorm));
         }
         __syncthreads();
     }
@@ -176,8 +204,10 @@ step_kernel(const StepArgs<IO> a, const StepFeat f) {
             nu.x = fmaf(cu, xv.x, nu.x); nu.y = fmaf(cu, xv.y, nu.y); nu.z = fmaf(cu, xv.z, nu.z); nu.w = fmaf(cu, xv.w, nu.w);
             nv.x = fmaf(cv, xv.x, nv.x); nv.y = fmaf(cv, xv.y, nv.y); nv.z = fmaf(cv, xv.z, nv.z); nv.w = fmaf(cv, xv.w, nv.w);
         }
-        __stcs(hst + ((2 * k) * P + p0) / 4, nu);
-        __stcs(hst + ((2 * k + 1) * P + p0) / 4, nv);
+        if (dchk::in(kSiteState, bh * N * P + (2 * k) * P + p0, P + 4, nSt)) {
+            __stcs(hst + ((2 * k) * P + p0) / 4, nu);
+            __stcs(hst + ((2 * k + 1) * P + p0) / 4, nv);
+        }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const float2 ck = *reinterpret_cast<const float2 *>(&sC[r][2 * k]);
@@ -204,17 +234,17 @@ step_kernel(const StepArgs<IO> a, const StepFeat f) {
         for (int r = 0; r < R; ++r) *reinterpret_cast<float4 *>(&ypart[warp][r][p0]) = yacc[r];
     }
     __syncthreads();
-    const float Dh = a.D[h];
+    const float Dh = ldf(a.D, h, a.H, kSiteScalars);
     for (int idx = tid; idx < R * P; idx += NT) {
         const int r = idx / P, p = idx % P;
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < Cfg::WARPS; ++w) s += ypart[w][r][p];
         const float xval = sX[r][p];
-        stv(a.y, (bh * R + r) * P + p, s + Dh * xval);
-        a.xp[(bh * R + r) * P + p] = xval;
+        stv(a.y, (bh * R + r) * P + p, nBP, kSiteY, s + Dh * xval);
+        stv(a.xp, (bh * R + r) * P + p, nBP, kSitePend, xval);
     }
-    for (int i = tid; i < R * N; i += NT) a.bp[bh * R * N + i] = (&sB[0][0])[i];
+    for (int i = tid; i < R * N; i += NT) stv(a.bp, bh * R * N + i, nBN, kSitePend, (&sB[0][0])[i]);
 }
 
 // Generic kernel for any even N and any P: one thread per (pair, column),
@@ -225,6 +255,8 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a,
     const int N = a.N, P = a.P, R = a.R, K2 = N / 2;
     const int64_t bh = blockIdx.x;
     const int h = (int)(bh % a.H);
+    // buffer extents in elements, for the bounds build's index checks
+    const int64_t nSt = a.BH * N * P, nBN = a.BH * R * N, nBP = a.BH * R * P;
     float *nB = ysum + R * P, *nC = nB + R * N;
     for (int i = threadIdx.x; i < R * P; i += blockDim.x) ysum[i] = 0.f;
     if (f.wB) {  // BC-norm prologue: one warp per row of B, then of C
@@ -232,50 +264,55 @@ __global__ void __launch_bounds__(256) step_generic_kernel(const StepArgs<IO> a,
         for (int row = warp; row < 2 * R; row += blockDim.x / 32) {
             const bool isB = row < R;
             const int r = isB ? row : row - R;
-            const IO *src = (isB ? a.B : a.C) + (bh * R + r) * N;
+            const IO *src = isB ? a.B : a.C;
+            const int64_t o = (bh * R + r) * N;
             const float *w = isB ? f.wB : f.wC;
-            const float *bias = (isB ? f.bB : f.bC) + (h * R + r) * N;
+            const float *bias = isB ? f.bB : f.bC;
             float *dst = (isB ? nB : nC) + r * N;
-            const float sc = bcn_row_scale_warp([&](int n) { return ldv(src, n); }, N, f.eps);
-            for (int n = lane; n < N; n += 32) dst[n] = fmaf(ldv(src, n) * sc, w[n], bias[n]);
+            const float sc = bcn_row_scale_warp([&](int n) { return ldv(src, o + n, nBN, kSiteVec); }, N, f.eps);
+            for (int n = lane; n < N; n += 32)
+                dst[n] = fmaf(ldv(src, o + n, nBN, kSiteVec) * sc, ldf(w, n, N, kSiteNorm),
+                              ldf(bias, (h * R + r) * N + n, a.H * R * N, kSiteNorm));
         }
     }
     __syncthreads();
-    auto Bv = [&](int i) { return f.wB ? nB[i] : ldv(a.B, bh * R * N + i); };  // i = r * N + n
-    auto Cv = [&](int i) { return f.wB ? nC[i] : ldv(a.C, bh * R * N + i); };
-    const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
-    const float alpha = expf(dtv * a.A[f.a_tok ? bh : h]);
+    auto Bv = [&](int i) { return f.wB ? nB[i] : ldv(a.B, bh * R * N + i, nBN, kSiteVec); };  // i = r * N + n
+    auto Cv = [&](int i) { return f.wB ? nC[i] : ldv(a.C, bh * R * N + i, nBN, kSiteVec); };
+    const float dtv = ldv(a.dt, bh, a.BH, kSiteScalars), lamv = ldv(a.lam, bh, a.BH, kSiteScalars);
+    const float alpha = expf(dtv * ldf(a.A, f.a_tok ? bh : h, f.a_tok ? a.BH : a.H, kSiteScalars));
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
     float *hs = a.h + bh * N * P;
     for (int idx = threadIdx.x; idx < K2 * P; idx += blockDim.x) {
         const int k = idx / P, p = idx % P;
-        float u = hs[(2 * k) * P + p], v = hs[(2 * k + 1) * P + p];
+        const int64_t iu = bh * N * P + (2 * k) * P + p, iv = iu + P;
+        float u = ldf(a.h, iu, nSt, kSiteState), v = ldf(a.h, iv, nSt, kSiteState);
         for (int r = 0; r < R; ++r) {
-            const float xpp = a.xp[(bh * R + r) * P + p];
-            u += betap * a.bp[(bh * R + r) * N + 2 * k] * xpp;
-            v += betap * a.bp[(bh * R + r) * N + 2 * k + 1] * xpp;
+            const float xpp = ldf(a.xp, (bh * R + r) * P + p, nBP, kSitePend);
+            u += betap * ldf(a.bp, (bh * R + r) * N + 2 * k, nBN, kSitePend) * xpp;
+            v += betap * ldf(a.bp, (bh * R + r) * N + 2 * k + 1, nBN, kSitePend) * xpp;
         }
         float sn, cs;
-        sincosf(dtv * ldv(a.theta, (f.th_head ? (int64_t)h : bh) * K2 + k), &sn, &cs);
+        sincosf(dtv * ldv(a.theta, (f.th_head ? (int64_t)h : bh) * K2 + k, (f.th_head ? a.H : a.BH) * K2, kSiteTheta),
+                &sn, &cs);
         float nu = alpha * (u * cs + v * sn), nv = alpha * (-u * sn + v * cs);
         for (int r = 0; r < R; ++r) {
-            const float xx = ldv(a.x, (bh * R + r) * P + p);
+            const float xx = ldv(a.x, (bh * R + r) * P + p, nBP, kSiteVec);
             nu += gam * Bv(r * N + 2 * k) * xx;
             nv += gam * Bv(r * N + 2 * k + 1) * xx;
         }
-        hs[(2 * k) * P + p] = nu;
-        hs[(2 * k + 1) * P + p] = nv;
+        stv(a.h, iu, nSt, kSiteState, nu);
+        stv(a.h, iv, nSt, kSiteState, nv);
         for (int r = 0; r < R; ++r)
             atomicAdd(&ysum[r * P + p], nu * Cv(r * N + 2 * k) + nv * Cv(r * N + 2 * k + 1));
     }
     __syncthreads();
-    const float Dh = a.D[h];
+    const float Dh = ldf(a.D, h, a.H, kSiteScalars);
     for (int idx = threadIdx.x; idx < R * P; idx += blockDim.x) {
-        const float xval = ldv(a.x, bh * R * P + idx);
-        stv(a.y, bh * R * P + idx, ysum[idx] + Dh * xval);
-        a.xp[bh * R * P + idx] = xval;
+        const float xval = ldv(a.x, bh * R * P + idx, nBP, kSiteVec);
+        stv(a.y, bh * R * P + idx, nBP, kSiteY, ysum[idx] + Dh * xval);
+        stv(a.xp, bh * R * P + idx, nBP, kSitePend, xval);
     }
-    for (int idx = threadIdx.x; idx < R * N; idx += blockDim.x) a.bp[bh * R * N + idx] = Bv(idx);
+    for (int idx = threadIdx.x; idx < R * N; idx += blockDim.x) stv(a.bp, bh * R * N + idx, nBN, kSitePend, Bv(idx));
 }
 
 // Persistent streaming variant: each CTA walks slices bh = blockIdx.x,
@@ -346,17 +383,28 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
     const int cg = tid % CG, kk = tid / CG, p0 = cg * 4;
     const int warp = tid / 32, lane = tid % 32;
     const int64_t BH = a.BH, step = gridDim.x;
+    // buffer extents in elements, for the bounds build's index checks
+    const int64_t nSt = BH * N * P, nBN = BH * R * N, nBP = BH * R * P;
 
+    // the slice's copies; the bounds build checks each source range and
+    // copies from the buffer's start instead of outside it (so that the
+    // expected bytes still arrive)
     auto issue = [&](int64_t bh, int st) {
         uint8_t *s = sm + st * Cfg::STAGE;
+        const int64_t th = ((GEN && f.th_head) ? bh % a.H : bh) * K2;
+        const int64_t nth = ((GEN && f.th_head) ? a.H : BH) * K2;
+        const bool ist = dchk::in(kSiteState, bh * N * P, N * P, nSt);
+        const bool ibn = dchk::in(kSitePend, bh * R * N, R * N, nBN) && dchk::in(kSiteVec, bh * R * N, R * N, nBN);
+        const bool ibp = dchk::in(kSitePend, bh * R * P, R * P, nBP) && dchk::in(kSiteVec, bh * R * P, R * P, nBP);
+        const bool ith = dchk::in(kSiteTheta, th, K2, nth);
         tc::mbar_arrive_expect_tx(&full[st], Cfg::TX);
-        tc::bulk_g2s(s, a.h + bh * N * P, Cfg::B_H, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_BP, a.bp + bh * R * N, Cfg::B_BP, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_XP, a.xp + bh * R * P, Cfg::B_XP, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_B, a.B + bh * R * N, Cfg::B_B, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_C, a.C + bh * R * N, Cfg::B_B, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_X, a.x + bh * R * P, Cfg::B_X, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_TH, a.theta + ((GEN && f.th_head) ? bh % a.H : bh) * K2, Cfg::B_TH, &full[st]);
+        tc::bulk_g2s(s, a.h + (ist ? bh * N * P : 0), Cfg::B_H, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_BP, a.bp + (ibn ? bh * R * N : 0), Cfg::B_BP, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_XP, a.xp + (ibp ? bh * R * P : 0), Cfg::B_XP, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_B, a.B + (ibn ? bh * R * N : 0), Cfg::B_B, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_C, a.C + (ibn ? bh * R * N : 0), Cfg::B_B, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_X, a.x + (ibp ? bh * R * P : 0), Cfg::B_X, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_TH, a.theta + (ith ? th : 0), Cfg::B_TH, &full[st]);
     };
     if (tid == 0) {
         tc::mbar_init(&full[0], 1);
@@ -389,12 +437,13 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
         const IO *sX = reinterpret_cast<const IO *>(s + Cfg::O_X);
         const IO *sTh = reinterpret_cast<const IO *>(s + Cfg::O_TH);
         const int h = (int)(bh % a.H);
-        const float dtv = ldv(a.dt, bh), lamv = ldv(a.lam, bh);
+        const float dtv = ldv(a.dt, bh, BH, kSiteScalars), lamv = ldv(a.lam, bh, BH, kSiteScalars);
         const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
         const bool ok = tc::mbar_wait(&full[st], (it >> 1) & 1, &abort_flag, &g_decode_error, tc::kErrWaitTma);
         if (__syncthreads_or(!ok)) break;
         if (tid < K2) {
-            const float alpha = __expf(dtv * a.A[(GEN && f.a_tok) ? bh : h]);
+            const float alpha =
+                __expf(dtv * ldf(a.A, (GEN && f.a_tok) ? bh : h, (GEN && f.a_tok) ? BH : a.H, kSiteScalars));
             float sn, cs;
             sincosf(dtv * sv(sTh, tid), &sn, &cs);
             sAc[tid] = alpha * cs;
@@ -443,8 +492,10 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
                 nv.x = fmaf(cv, xv[r].x, nv.x); nv.y = fmaf(cv, xv[r].y, nv.y);
                 nv.z = fmaf(cv, xv[r].z, nv.z); nv.w = fmaf(cv, xv[r].w, nv.w);
             }
-            __stcs(hg + ((2 * k) * P + p0) / 4, nu);
-            __stcs(hg + ((2 * k + 1) * P + p0) / 4, nv);
+            if (dchk::in(kSiteState, bh * N * P + (2 * k) * P + p0, P + 4, nSt)) {
+                __stcs(hg + ((2 * k) * P + p0) / 4, nu);
+                __stcs(hg + ((2 * k + 1) * P + p0) / 4, nv);
+            }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const float2 ck = *reinterpret_cast<const float2 *>(vC + r * N + 2 * k);
@@ -470,16 +521,16 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
                 *reinterpret_cast<float4 *>(ypart + (warp * R + r) * P + p0) = yacc[r];
         }
         __syncthreads();
-        const float Dh = a.D[h];
+        const float Dh = ldf(a.D, h, a.H, kSiteScalars);
         for (int idx = tid; idx < R * P; idx += NT) {
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < Cfg::WARPS; ++w) sum += ypart[w * R * P + idx];
             const float xval = sv(sX, idx);
-            stv(a.y, bh * R * P + idx, sum + Dh * xval);
-            a.xp[bh * R * P + idx] = xval;
+            stv(a.y, bh * R * P + idx, nBP, kSiteY, sum + Dh * xval);
+            stv(a.xp, bh * R * P + idx, nBP, kSitePend, xval);
         }
-        for (int i = tid; i < R * N; i += NT) a.bp[bh * R * N + i] = sv(sB, i);
+        for (int i = tid; i < R * N; i += NT) stv(a.bp, bh * R * N + i, nBN, kSitePend, sv(sB, i));
         __syncthreads();  // every read of this stage is done: refill it
         if (tid == 0 && bh + 2 * step < BH) issue(bh + 2 * step, st);
     }
@@ -590,5 +641,7 @@ cudaError_t read_decode_error(unsigned *code) {
     *code = v;
     return e;
 }
+
+M3_DCHECK_READER(read_dcheck_decode)
 
 }  // namespace m3

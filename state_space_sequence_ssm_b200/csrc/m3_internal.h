@@ -63,6 +63,19 @@ cudaError_t read_device_error(unsigned *code, cudaStream_t stream);
 cudaError_t read_decode_error(unsigned *code);
 // Read and clear the fp32 tensor-core prefill's device error word (after a sync).
 cudaError_t read_tc32_error(unsigned *code);
+// First failed device index check recorded by one kernel file (the bounds
+// build, compiled with M3_DEVICE_CHECKS; the normal build records none).
+struct DcheckRecord {
+    unsigned count;      // failed checks since the last read
+    unsigned site;       // site code of the first failure (kernel file in the high byte)
+    long long index;     // first element index of the failed access
+    long long extent;    // elements in the buffer
+};
+// Read and clear each kernel file's record, after a sync.
+cudaError_t read_dcheck_tc(DcheckRecord *r);
+cudaError_t read_dcheck_tc32(DcheckRecord *r);
+cudaError_t read_dcheck_simt(DcheckRecord *r);
+cudaError_t read_dcheck_decode(DcheckRecord *r);
 // Record the calling thread's failure message (m3_last_error) and return `s`.
 m3_status set_error(m3_status s, const char *msg);
 m3_status set_cuda_error(cudaError_t e, const char *where);

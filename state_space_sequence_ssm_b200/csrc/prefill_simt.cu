@@ -19,41 +19,61 @@
 #include <cuda_bf16.h>
 
 #include "bcnorm.cuh"
+#include "dcheck.cuh"
 #include "m3_internal.h"
 
 namespace m3 {
 namespace {
 
+// Index-check sites of this file (bounds build).
+enum : unsigned {
+    kSiteScalars = 0x301,  // dt, lam, A, D
+    kSiteTheta = 0x302,    // angle rates
+    kSiteRows = 0x303,     // x, B, C rows
+    kSiteNorm = 0x304,     // BC-norm weights and biases
+    kSiteInit = 0x305,     // initial state h0, b_prev, x_prev
+    kSiteY = 0x306,        // output rows
+    kSiteFinal = 0x307,    // final state
+};
+
+// Element i of a buffer of n elements (the bounds build checks i and reads 0
+// outside; `site` names the access).
 template <typename T>
-__device__ __forceinline__ float ldv(const T *p, int64_t i);
+__device__ __forceinline__ float ldv(const T *p, int64_t i, int64_t n, unsigned site);
 template <>
-__device__ __forceinline__ float ldv<float>(const float *p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float ldv<float>(const float *p, int64_t i, int64_t n, unsigned site) {
+    return dchk::in(site, i, 1, n) ? p[i] : 0.f;
+}
 template <>
-__device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
-    return __bfloat162float(p[i]);
+__device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i, int64_t n, unsigned site) {
+    return dchk::in(site, i, 1, n) ? __bfloat162float(p[i]) : 0.f;
 }
 // Four consecutive values (i a multiple of 4; the row they lie in starts
 // 16-byte aligned for fp32, 8-byte aligned for bf16).
 template <typename T>
-__device__ __forceinline__ float4 ldv4(const T *p, int64_t i);
+__device__ __forceinline__ float4 ldv4(const T *p, int64_t i, int64_t n, unsigned site);
 template <>
-__device__ __forceinline__ float4 ldv4<float>(const float *p, int64_t i) {
+__device__ __forceinline__ float4 ldv4<float>(const float *p, int64_t i, int64_t n, unsigned site) {
+    if (!dchk::in(site, i, 4, n)) return make_float4(0.f, 0.f, 0.f, 0.f);
     return __ldg(reinterpret_cast<const float4 *>(p + i));
 }
 template <>
-__device__ __forceinline__ float4 ldv4<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i) {
+__device__ __forceinline__ float4 ldv4<__nv_bfloat16>(const __nv_bfloat16 *p, int64_t i, int64_t n, unsigned site) {
+    if (!dchk::in(site, i, 4, n)) return make_float4(0.f, 0.f, 0.f, 0.f);
     const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p + i));
     const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
     const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
     return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 template <typename T>
-__device__ __forceinline__ void stv(T *p, int64_t i, float v);
+__device__ __forceinline__ void stv(T *p, int64_t i, int64_t n, unsigned site, float v);
 template <>
-__device__ __forceinline__ void stv<float>(float *p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void stv<float>(float *p, int64_t i, int64_t n, unsigned site, float v) {
+    if (dchk::in(site, i, 1, n)) p[i] = v;
+}
 template <>
-__device__ __forceinline__ void stv<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float v) {
-    p[i] = __float2bfloat16_rn(v);
+__device__ __forceinline__ void stv<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, int64_t n, unsigned site, float v) {
+    if (dchk::in(site, i, 1, n)) p[i] = __float2bfloat16_rn(v);
 }
 
 template <typename IO>
@@ -106,21 +126,25 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
     const int64_t bh = blockIdx.x;
     const int64_t b = bh / a.H, h = bh % a.H;
     const int64_t T = a.T, H = a.H;
-    const float Ah = a.a_tok ? 0.f : a.A[h], Dh = a.D[h];
     auto tok = [&](int64_t t) { return (b * T + t) * H + h; };  // token-head index
+    // buffer extents in elements, for the bounds build's index checks
+    const int64_t BH = gridDim.x, nTok = BH * T, nX = nTok * R * P, nBC = nTok * R * N, nSt = BH * N * P;
+    const float Ah = a.a_tok ? 0.f : ldv(a.A, h, H, kSiteScalars), Dh = ldv(a.D, h, H, kSiteScalars);
 
     // ---- initial state: h0 + beta'_0 * b_prev x_prev^T (pending write of token -1)
     float betap0 = 0.f;
     if (T > 0) {
-        const float d0 = ldv(a.dt, tok(0)), l0 = ldv(a.lam, tok(0));
+        const float d0 = ldv(a.dt, tok(0), nTok, kSiteScalars), l0 = ldv(a.lam, tok(0), nTok, kSiteScalars);
         betap0 = (1.f - l0) * d0;
     }
     for (int idx = tid; idx < N * P; idx += kThreads) {
         const int n = idx / P, p = idx % P;
-        float v = a.h0 ? a.h0[bh * N * P + idx] : 0.f;
+        float v = a.h0 ? ldv(a.h0, bh * N * P + idx, nSt, kSiteInit) : 0.f;
         if (a.bp0 && a.xp0 && T > 0) {
             float acc = 0.f;
-            for (int r = 0; r < R; ++r) acc += a.bp0[(bh * R + r) * N + n] * a.xp0[(bh * R + r) * P + p];
+            for (int r = 0; r < R; ++r)
+                acc += ldv(a.bp0, (bh * R + r) * N + n, BH * R * N, kSiteInit) *
+                       ldv(a.xp0, (bh * R + r) * P + p, BH * R * P, kSiteInit);
             v += betap0 * acc;
         }
         hs[idx] = v;
@@ -139,12 +163,13 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
 #pragma unroll 4
             for (int idx = tid; idx < rows * P4; idx += kThreads) {
                 const int i = idx / P4, p = 4 * (idx % P4);
-                *reinterpret_cast<float4 *>(Xs + i * P + p) = ldv4(a.x, (tok(t0 + i / R) * R + i % R) * P + p);
+                *reinterpret_cast<float4 *>(Xs + i * P + p) =
+                    ldv4(a.x, (tok(t0 + i / R) * R + i % R) * P + p, nX, kSiteRows);
             }
         } else {
             for (int idx = tid; idx < rows * P; idx += kThreads) {
                 const int i = idx / P, p = idx % P;
-                Xs[idx] = ldv(a.x, (tok(t0 + i / R) * R + i % R) * P + p);
+                Xs[idx] = ldv(a.x, (tok(t0 + i / R) * R + i % R) * P + p, nX, kSiteRows);
             }
         }
         if (N % 4 == 0) {
@@ -153,7 +178,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             for (int idx = tid; idx < rows * N4; idx += kThreads) {
                 const int i = idx / N4, n = 4 * (idx % N4);
                 const int64_t g = (tok(t0 + i / R) * R + i % R) * N + n;
-                const float4 vb = ldv4(a.B, g), vc = ldv4(a.C, g);
+                const float4 vb = ldv4(a.B, g, nBC, kSiteRows), vc = ldv4(a.C, g, nBC, kSiteRows);
                 float *bd = Bs + i * NS + n, *cd = Cs + i * NS + n;
                 bd[0] = vb.x; bd[1] = vb.y; bd[2] = vb.z; bd[3] = vb.w;
                 cd[0] = vc.x; cd[1] = vc.y; cd[2] = vc.z; cd[3] = vc.w;
@@ -162,19 +187,20 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
             for (int idx = tid; idx < rows * N; idx += kThreads) {
                 const int i = idx / N, n = idx % N;
                 const int64_t g = (tok(t0 + i / R) * R + i % R) * N + n;
-                Bs[i * NS + n] = ldv(a.B, g);
-                Cs[i * NS + n] = ldv(a.C, g);
+                Bs[i * NS + n] = ldv(a.B, g, nBC, kSiteRows);
+                Cs[i * NS + n] = ldv(a.C, g, nBC, kSiteRows);
             }
         }
         for (int s = tid; s < L; s += kThreads) {
             const int64_t t = t0 + s;
-            const float d = ldv(a.dt, tok(t)), l = ldv(a.lam, tok(t));
+            const float d = ldv(a.dt, tok(t), nTok, kSiteScalars), l = ldv(a.lam, tok(t), nTok, kSiteScalars);
             dts[s] = d;
-            cA[s] = d * (a.a_tok ? a.A[tok(t)] : Ah);
+            cA[s] = d * (a.a_tok ? ldv(a.A, tok(t), nTok, kSiteScalars) : Ah);
             gam[s] = l * d;
             float nxt = 0.f;  // (1 - lam_{t+1}) dt_{t+1}; absent after the last token
             if (t + 1 < T) {
-                const float d1 = ldv(a.dt, tok(t + 1)), l1 = ldv(a.lam, tok(t + 1));
+                const float d1 = ldv(a.dt, tok(t + 1), nTok, kSiteScalars);
+                const float l1 = ldv(a.lam, tok(t + 1), nTok, kSiteScalars);
                 nxt = (1.f - l1) * d1;
             }
             ghat[s] = l * d + nxt;
@@ -187,9 +213,10 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
                 float *v = isB ? Bs + row * NS : Cs + (row - rows) * NS;
                 const int r = (isB ? row : row - rows) % R;
                 const float *w = isB ? a.wB : a.wC;
-                const float *bias = (isB ? a.bB : a.bC) + (h * R + r) * N;
+                const float *bias = isB ? a.bB : a.bC;
                 const float sc = bcn_row_scale_warp([&](int n) { return v[n]; }, N, a.eps);
-                for (int n = lane; n < N; n += 32) v[n] = fmaf(v[n] * sc, w[n], bias[n]);
+                for (int n = lane; n < N; n += 32)
+                    v[n] = fmaf(v[n] * sc, ldv(w, n, N, kSiteNorm), ldv(bias, (h * R + r) * N + n, H * R * N, kSiteNorm));
             }
             __syncthreads();
         }
@@ -204,7 +231,8 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
 #pragma unroll 4
         for (int idx = tid; idx < L * K2; idx += kThreads) {
             const int s = idx / K2, k = idx % K2;
-            phis[idx] = dts[s] * ldv(a.theta, (a.th_head ? (int64_t)h : tok(t0 + s)) * K2 + k);
+            phis[idx] = dts[s] * ldv(a.theta, (a.th_head ? (int64_t)h : tok(t0 + s)) * K2 + k,
+                                     (a.th_head ? H : nTok) * K2, kSiteTheta);
         }
         __syncthreads();
         for (int k = tid; k < K2; k += kThreads) {
@@ -318,7 +346,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
                     const int p = pt + TP * qb;
                     if (p >= P) continue;
                     const float yv = dg[qa][qb] + ei * of[qa][qb] + Dh * Xs[i * P + p];
-                    stv(a.y, (tok(t0 + i / R) * R + i % R) * P + p, yv);
+                    stv(a.y, (tok(t0 + i / R) * R + i % R) * P + p, nX, kSiteY, yv);
                 }
             }
         }
@@ -375,27 +403,31 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(const SimtArgs<I
     if (a.hT) {
         for (int idx = tid; idx < N * P; idx += kThreads) {
             float v = hs[idx];
-            if (T == 0) v = a.h0 ? a.h0[bh * N * P + idx] : 0.f;
-            a.hT[bh * N * P + idx] = v;
+            if (T == 0) v = a.h0 ? ldv(a.h0, bh * N * P + idx, nSt, kSiteInit) : 0.f;
+            stv(a.hT, bh * N * P + idx, nSt, kSiteFinal, v);
         }
     }
     if (a.bpT && a.wB && T > 0) {  // the last token's normalised B, one warp per rank row
         const int warp = tid >> 5, lane = tid & 31;
         for (int r = warp; r < R; r += kThreads / 32) {
             const int64_t src = tok(T - 1) * R * N + r * N;
-            const float sc = bcn_row_scale_warp([&](int n) { return ldv(a.B, src + n); }, N, a.eps);
+            const float sc = bcn_row_scale_warp([&](int n) { return ldv(a.B, src + n, nBC, kSiteFinal); }, N, a.eps);
             for (int n = lane; n < N; n += 32)
-                a.bpT[(bh * R + r) * N + n] = fmaf(ldv(a.B, src + n) * sc, a.wB[n], a.bB[(h * R + r) * N + n]);
+                stv(a.bpT, (bh * R + r) * N + n, BH * R * N, kSiteFinal,
+                    fmaf(ldv(a.B, src + n, nBC, kSiteFinal) * sc, ldv(a.wB, n, N, kSiteNorm),
+                         ldv(a.bB, (h * R + r) * N + n, H * R * N, kSiteNorm)));
         }
     } else if (a.bpT) {
         for (int idx = tid; idx < R * N; idx += kThreads)
-            a.bpT[bh * R * N + idx] = T > 0 ? ldv(a.B, tok(T - 1) * R * N + idx)
-                                            : (a.bp0 ? a.bp0[bh * R * N + idx] : 0.f);
+            stv(a.bpT, bh * R * N + idx, BH * R * N, kSiteFinal,
+                T > 0 ? ldv(a.B, tok(T - 1) * R * N + idx, nBC, kSiteFinal)
+                      : (a.bp0 ? ldv(a.bp0, bh * R * N + idx, BH * R * N, kSiteInit) : 0.f));
     }
     if (a.xpT) {
         for (int idx = tid; idx < R * P; idx += kThreads)
-            a.xpT[bh * R * P + idx] = T > 0 ? ldv(a.x, tok(T - 1) * R * P + idx)
-                                            : (a.xp0 ? a.xp0[bh * R * P + idx] : 0.f);
+            stv(a.xpT, bh * R * P + idx, BH * R * P, kSiteFinal,
+                T > 0 ? ldv(a.x, tok(T - 1) * R * P + idx, nX, kSiteFinal)
+                      : (a.xp0 ? ldv(a.xp0, bh * R * P + idx, BH * R * P, kSiteInit) : 0.f));
     }
 }
 
@@ -439,5 +471,7 @@ cudaError_t launch_typed(const Problem &p, const char **why) {
 cudaError_t launch_prefill_simt(const Problem &p, const char **why) {
     return p.bf16 ? launch_typed<__nv_bfloat16>(p, why) : launch_typed<float>(p, why);
 }
+
+M3_DCHECK_READER(read_dcheck_simt)
 
 }  // namespace m3

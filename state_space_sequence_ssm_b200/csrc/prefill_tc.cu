@@ -44,6 +44,7 @@
 
 #include <mutex>
 
+#include "dcheck.cuh"
 #include "m3_internal.h"
 #include "tc_primitives.cuh"
 
@@ -329,6 +330,20 @@ struct Bars {
 // over one segment, from the scan of the summaries before it (look-back).
 constexpr int kWhole = 0, kSummary = 1, kSegment = 2;
 
+// Index-check sites of this file (bounds build).
+enum : unsigned {
+    kSiteScalars = 0x101,  // dt, lam, per-token A
+    kSiteHead = 0x102,     // A, D per head
+    kSiteNorm = 0x103,     // BC-norm weights and biases
+    kSiteTheta = 0x104,    // angle rates
+    kSiteFlags = 0x105,    // split sequences: segment flags
+    kSiteWsH = 0x106,      // split sequences: segment end states
+    kSiteWsM = 0x107,      // split sequences: segment transitions
+    kSiteInit = 0x108,     // initial state h0, b_prev, x_prev
+    kSiteY = 0x109,        // output rows
+    kSiteFinal = 0x10a,    // final state and the last token's B and x
+};
+
 // GEN = false: the plain method (A per head, theta per token), compiled
 // without the optional features' branches; GEN = true reads A_tok and th_head
 // from the arguments.  BCN: the BC-norm prologue (only with GEN).
@@ -376,6 +391,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int64_t T = a.T, H = a.H;
     const int64_t b = bh / H, h = bh % H;
     auto tok = [&](int64_t t) { return (b * T + t) * H + h; };
+    // buffer extents in elements, for the bounds build's index checks
+    const int64_t nTok = (int64_t)a.BH * T, nSt = (int64_t)a.BH * N * kP, nSeg = SEGD ? (int64_t)a.nseg : 1;
 
     // the main pass is launched as a programmatic dependent of the summary
     // pass: its CTAs take SMs as summary CTAs leave them, and all summary CTAs
@@ -553,7 +570,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
     } else if (warp < 8) {
         // ============================================================ prologue warps (0-7)
-        const float Ah2 = A_tok ? 0.f : a.A[h] * kLog2e;
+        const float Ah2 = (A_tok || !dchk::in(kSiteHead, h, 1, H)) ? 0.f : a.A[h] * kLog2e;
         uint8_t *xw = smem + C::OFF_XW;
         const unsigned short *dtr = reinterpret_cast<const unsigned short *>(a.dt);
         const unsigned short *lmr = reinterpret_cast<const unsigned short *>(a.lam);
@@ -565,11 +582,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         auto prefetch_scalars = [&](int64_t t0s) {
             const int64_t t = t0s + tid;
             pd = pl = pd1 = pl1 = 0;
-            if (tid < Q && t < T) {
+            if (tid < Q && t < T && dchk::in(kSiteScalars, tok(t), 1, nTok)) {
                 pd = __ldg(dtr + tok(t));
                 pl = __ldg(lmr + tok(t));
                 if (A_tok) pa = __ldg(A_tok + tok(t));
-                if (t + 1 < T) {
+                if (t + 1 < T && dchk::in(kSiteScalars, tok(t + 1), 1, nTok)) {
                     pd1 = __ldg(dtr + tok(t + 1));
                     pl1 = __ldg(lmr + tok(t + 1));
                 }
@@ -585,28 +602,32 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int n = 8 * g + 2 * e;
+                if (!dchk::in(kSiteNorm, n, 2, N)) continue;
                 wB2[e] = pack_bf16(a.wB[n], a.wB[n + 1]);
                 wC2[e] = pack_bf16(a.wC[n], a.wC[n + 1]);
             }
             for (int i = tid; i < 2 * R * K2; i += kPro) {
                 const int which = i / (R * K2), rk = i % (R * K2);
-                const float *src = (which ? a.bC : a.bB) + (h * R + rk / K2) * N + 2 * (rk % K2);
-                sbias[i] = pack_bf16(src[0], src[1]);
+                const int64_t o = (h * R + rk / K2) * N + 2 * (rk % K2);
+                const float *src = (which ? a.bC : a.bB) + o;
+                sbias[i] = dchk::in(kSiteNorm, o, 2, H * R * N) ? pack_bf16(src[0], src[1]) : 0u;
             }
         }
         // angle rates fixed per head: the thread's 4 pairs, for the whole sequence
         float thh[4] = {0.f, 0.f, 0.f, 0.f};
         if (th_head) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) thh[e] = bf(a.theta, h * K2 + 4 * g + e);
+            for (int e = 0; e < 4; ++e)
+                thh[e] = dchk::in(kSiteTheta, h * K2 + 4 * g + e, 1, H * K2) ? bf(a.theta, h * K2 + 4 * g + e) : 0.f;
         }
         auto prefetch_theta = [&](int64_t t0s) {
             if (th_head) return;
 #pragma unroll
             for (int j = 0; j < TPT; ++j) {
                 const int64_t t = t0s + part * TPT + j;
-                thr[j] = t < T ? __ldg(reinterpret_cast<const uint2 *>(a.theta + tok(t) * K2 + 4 * g))
-                               : make_uint2(0u, 0u);
+                thr[j] = (t < T && dchk::in(kSiteTheta, tok(t) * K2 + 4 * g, 4, nTok * K2))
+                             ? __ldg(reinterpret_cast<const uint2 *>(a.theta + tok(t) * K2 + 4 * g))
+                             : make_uint2(0u, 0u);
             }
         };
         prefetch_scalars((int64_t)cb * Q);
@@ -835,7 +856,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const bool own_state = (N == 128) || (lane < 16);
         const int srow = (N == 128) ? lq : (wq * 16 + lane);  // TMEM lane layout of G (M = N)
         uint8_t *hbuf = smem + C::OFF_HB;
-        const float Dh = a.D[h];
+        const float Dh = dchk::in(kSiteHead, h, 1, H) ? a.D[h] : 0.f;
         const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
         const int c0 = 32 * hf;            // first column of this thread's half
         float hreg[32];
@@ -855,7 +876,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 // exactly like the chunk-to-chunk update.
                 if (bar_any<kBarState, kSt>(lt == 0 && [&] {
                         for (int j = 0; j < seg; ++j)
-                            if (!flag_wait(a.flags + (int64_t)j * BH + bh, abort_flag, err, kErrWaitSegment))
+                            if (!dchk::in(kSiteFlags, (int64_t)j * BH + bh, 1, nSeg * BH) ||
+                                !flag_wait(a.flags + (int64_t)j * BH + bh, abort_flag, err, kErrWaitSegment))
                                 return true;
                         return false;
                     }())) {
@@ -863,23 +885,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 } else {
                     const int rr = own_state ? srow : 0;
                     const int64_t slot = (int64_t)BH * N * kP;
-                    const float *hs = a.ws_h + slot + bh * N * kP + rr * kP + c0;
+                    const int64_t ho = slot + bh * N * kP + rr * kP + c0;
+                    const float *hs = a.ws_h + ho;
+                    const bool in1 = dchk::in(kSiteWsH, ho, 32, nSeg * slot);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(hs) + q);
+                        const float4 v =
+                            in1 ? __ldcg(reinterpret_cast<const float4 *>(hs) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
                         hreg[4 * q] = v.x;
                         hreg[4 * q + 1] = v.y;
                         hreg[4 * q + 2] = v.z;
                         hreg[4 * q + 3] = v.w;
                     }
                     for (int j = 1; j < seg; ++j) {
-                        const float2 m =
-                            __ldcg(reinterpret_cast<const float2 *>(a.ws_m + ((int64_t)j * BH + bh) * N + (rr & ~1)));
+                        const int64_t mo = ((int64_t)j * BH + bh) * N + (rr & ~1);
+                        const float2 m = dchk::in(kSiteWsM, mo, 2, nSeg * BH * N)
+                                             ? __ldcg(reinterpret_cast<const float2 *>(a.ws_m + mo))
+                                             : make_float2(0.f, 0.f);
                         const float ms = (rr & 1) ? -m.y : m.y;
+                        const bool inj = dchk::in(kSiteWsH, ho + (int64_t)j * slot, 32, nSeg * slot);
                         float4 l[8];
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
-                            l[q] = __ldcg(reinterpret_cast<const float4 *>(hs + (int64_t)j * slot) + q);
+                            l[q] = inj ? __ldcg(reinterpret_cast<const float4 *>(hs + (int64_t)j * slot) + q)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             const float lv[4] = {l[q].x, l[q].y, l[q].z, l[q].w};
@@ -893,14 +922,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     }
                 }
             } else if (seg == 0) {
-                const float betap0 = (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0));
+                const float betap0 = dchk::in(kSiteScalars, tok(0), 1, nTok)
+                                         ? (1.f - bf(a.lam, tok(0))) * bf(a.dt, tok(0)) : 0.f;
                 if (own_state) {
-                    if (a.h0) {
+                    if (a.h0 && dchk::in(kSiteInit, (bh * N + srow) * kP + c0, 32, nSt)) {
 #pragma unroll
                         for (int p = 0; p < 32; ++p) hreg[p] = a.h0[(bh * N + srow) * kP + c0 + p];
                     }
                     if (a.bp0 && a.xp0) {
                         for (int r = 0; r < R; ++r) {
+                            if (!dchk::in(kSiteInit, (bh * R + r) * N + srow, 1, (int64_t)a.BH * R * N) ||
+                                !dchk::in(kSiteInit, (bh * R + r) * kP + c0, 32, (int64_t)a.BH * R * kP))
+                                continue;
                             const float cw = betap0 * a.bp0[(bh * R + r) * N + srow];
 #pragma unroll
                             for (int p = 0; p < 32; ++p)
@@ -918,7 +951,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (lt == 0) {
             mbar_arrive(bb.hrdy);
             // the caller's initial state is read (the last segment may now overwrite it)
-            if (MODE == kSegment && seg == 0) flag_release(a.flags + (int64_t)(a.nseg - 1) * BH + bh, 1u);
+            if (MODE == kSegment && seg == 0 && dchk::in(kSiteFlags, (int64_t)(a.nseg - 1) * BH + bh, 1, nSeg * BH))
+                flag_release(a.flags + (int64_t)(a.nseg - 1) * BH + bh, 1u);
         }
         for (int lc = 0; ok && lc < nloc; ++lc) {
             const int sx = lc % kNX;
@@ -1014,7 +1048,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     tmem_ld16(tl + kColYd + c0 + 16 * qq, yd);
                     tmem_ld16(tl + yo + c0 + 16 * qq, yv);
                     tmem_wait_ld();
-                    if (t < T) {
+                    if (t < T && dchk::in(kSiteY, (tok(t) * R + r) * kP + c0 + 16 * qq, 16, nTok * R * kP)) {
                         __nv_bfloat16 *yrow = a.y + (tok(t) * R + r) * kP + c0 + 16 * qq;
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
@@ -1042,13 +1076,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (SUM) {
             // ---- summary: the segment's local end state (pending-inclusive) into
             //      slot seg + 1, its transition exp(cA) Rot(-Phi) per pair
-            if (ok && own_state) {
-                float4 *dst = reinterpret_cast<float4 *>(a.ws_h + (((int64_t)seg + 1) * BH + bh) * N * kP +
-                                                         srow * kP + c0);
+            const int64_t ho = (((int64_t)seg + 1) * BH + bh) * N * kP + srow * kP + c0;
+            if (ok && own_state && dchk::in(kSiteWsH, ho, 32, nSeg * nSt)) {
+                float4 *dst = reinterpret_cast<float4 *>(a.ws_h + ho);
 #pragma unroll
                 for (int p = 0; p < 8; ++p)
                     dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
-                if (hf == 0 && (srow & 1) == 0) {
+                if (hf == 0 && (srow & 1) == 0 &&
+                    dchk::in(kSiteWsM, ((int64_t)seg * BH + bh) * N + srow, 2, nSeg * BH * N)) {
                     const float e = ex2(m_l2);
                     *reinterpret_cast<float2 *>(a.ws_m + ((int64_t)seg * BH + bh) * N + srow) =
                         make_float2(e * m_cs, e * m_sn);
@@ -1057,12 +1092,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             __threadfence();  // before the flag release below
         } else if (ok && (!SEGD || seg == a.nseg - 1) &&
                    !(MODE == kSegment &&
-                     bar_any<kBarState, kSt>(lt == 0 && !flag_wait(a.flags + (int64_t)(a.nseg - 1) * BH + bh,
-                                                                   abort_flag, err, kErrWaitSegment)))) {
+                     bar_any<kBarState, kSt>(lt == 0 &&
+                                             (!dchk::in(kSiteFlags, (int64_t)(a.nseg - 1) * BH + bh, 1, nSeg * BH) ||
+                                              !flag_wait(a.flags + (int64_t)(a.nseg - 1) * BH + bh, abort_flag, err,
+                                                         kErrWaitSegment))))) {
             // ---- final state: plain-frame h_{T-1}, raw last token as the pending term
             //      (the last segment of a split sequence: once segment 0 has read
             //      the initial state, which this may overwrite)
-            if (a.hT && own_state) {
+            if (a.hT && own_state && dchk::in(kSiteFinal, (bh * N + srow) * kP + c0, 32, nSt)) {
                 float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * N + srow) * kP + c0);
 #pragma unroll
                 for (int p = 0; p < 8; ++p)
@@ -1070,7 +1107,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
             if (a.bpT && BCN) {  // the last token's normalised B, one state warp per rank row
                 const int wl = lt >> 5;
-                if (wl < R) {
+                if (wl < R && dchk::in(kSiteFinal, tok(T - 1) * R * N + wl * N, N, nTok * R * N) &&
+                    dchk::in(kSiteFinal, (bh * R + wl) * N, N, (int64_t)a.BH * R * N) &&
+                    dchk::in(kSiteNorm, (h * R + wl) * N, N, H * R * N)) {
                     const int64_t src = tok(T - 1) * R * N + wl * N;
                     float ss = 0.f;
                     for (int n = lane; n < N; n += 32) ss = fmaf(bf(a.B, src + n), bf(a.B, src + n), ss);
@@ -1080,17 +1119,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     for (int n = lane; n < N; n += 32)
                         a.bpT[(bh * R + wl) * N + n] = fmaf(bf(a.B, src + n) * sc, a.wB[n], a.bB[(h * R + wl) * N + n]);
                 }
-            } else if (a.bpT) {
+            } else if (a.bpT && dchk::in(kSiteFinal, tok(T - 1) * R * N, R * N, nTok * R * N) &&
+                       dchk::in(kSiteFinal, bh * R * N, R * N, (int64_t)a.BH * R * N)) {
                 for (int i = lt; i < R * N; i += kSt) a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
             }
-            if (a.xpT)
+            if (a.xpT && dchk::in(kSiteFinal, tok(T - 1) * R * kP, R * kP, nTok * R * kP) &&
+                dchk::in(kSiteFinal, bh * R * kP, R * kP, (int64_t)a.BH * R * kP))
                 for (int i = lt; i < R * kP; i += kSt) a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
         }
     }
     __syncwarp();  // reconverge the single-lane roles before the block barrier
     tc_fence_before();
     __syncthreads();
-    if (SUM && tid == 0) flag_release(a.flags + (int64_t)seg * BH + bh, *abort_flag ? 2u : 1u);
+    if (SUM && tid == 0 && dchk::in(kSiteFlags, (int64_t)seg * BH + bh, 1, nSeg * BH))
+        flag_release(a.flags + (int64_t)seg * BH + bh, *abort_flag ? 2u : 1u);
     if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
@@ -1411,5 +1453,7 @@ cudaError_t read_device_error(unsigned *code, cudaStream_t stream) {
     *code = v;
     return e;
 }
+
+M3_DCHECK_READER(read_dcheck_tc)
 
 }  // namespace m3

@@ -40,6 +40,7 @@
 #include <cuda_bf16.h>
 
 #include "bcnorm.cuh"
+#include "dcheck.cuh"
 #include "m3_internal.h"
 #include "tc_primitives.cuh"
 
@@ -81,6 +82,18 @@ constexpr uint32_t OFF_BAR = OFF_SCAL + (2 * SB32 + 8 + kWarps * kK2 + 8) * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 4 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// Index-check sites of this file (bounds build).
+enum : unsigned {
+    kSiteScalars = 0x201,  // dt, lam, A
+    kSiteTheta = 0x202,    // angle rates
+    kSiteRows = 0x203,     // B, C and x rows
+    kSiteNorm = 0x204,     // BC-norm weights and biases
+    kSiteHead = 0x205,     // D
+    kSiteInit = 0x206,     // initial state h0, b_prev, x_prev
+    kSiteY = 0x207,        // output rows
+    kSiteFinal = 0x208,    // final state and the last token's B and x
+};
 
 struct Tc32Args {
     int64_t T, H;
@@ -172,7 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
     const int64_t bh = blockIdx.x, T = a.T, H = a.H;
     const int64_t b = bh / H, h = bh % H;
     auto tok = [&](int64_t t) { return (b * T + t) * H + h; };
-    const float Dh = a.D[h];
+    // buffer extents in elements, for the bounds build's index checks
+    const int64_t BH = gridDim.x, nTok = BH * T, nSt = BH * kN * kP;
+    const float Dh = dchk::in(kSiteHead, h, 1, H) ? a.D[h] : 0.f;
 
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
@@ -194,13 +209,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
 #pragma unroll
     for (int p = 0; p < kTC; ++p) hreg[p] = 0.f;
     if (own_state && T > 0) {
-        const float betap0 = (1.f - a.lam[tok(0)]) * a.dt[tok(0)];
-        if (a.h0) {
+        const float betap0 =
+            dchk::in(kSiteScalars, tok(0), 1, nTok) ? (1.f - a.lam[tok(0)]) * a.dt[tok(0)] : 0.f;
+        if (a.h0 && dchk::in(kSiteInit, (bh * kN + srow) * kP + c0, kTC, nSt)) {
 #pragma unroll
             for (int p = 0; p < kTC; ++p) hreg[p] = a.h0[(bh * kN + srow) * kP + c0 + p];
         }
         if (a.bp0 && a.xp0) {
             for (int r = 0; r < R; ++r) {
+                if (!dchk::in(kSiteInit, (bh * R + r) * kN + srow, 1, BH * R * kN) ||
+                    !dchk::in(kSiteInit, (bh * R + r) * kP + c0, kTC, BH * R * kP))
+                    continue;
                 const float cw = betap0 * a.bp0[(bh * R + r) * kN + srow];
 #pragma unroll
                 for (int p = 0; p < kTC; ++p) hreg[p] = fmaf(cw, a.xp0[(bh * R + r) * kP + c0 + p], hreg[p]);
@@ -226,18 +245,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
 #pragma unroll
         for (int u = 0; u < TPS; ++u) {
             const int64_t t = t0 + sg * TPS + u;
-            dtv[u] = t < T ? a.dt[tok(t)] : 0.f;
-            thv[u] = t < T ? a.theta[(a.th_head ? (int64_t)h : tok(t)) * kK2 + kq] : 0.f;
+            const int64_t ti = (a.th_head ? (int64_t)h : tok(t)) * kK2 + kq;
+            dtv[u] = (t < T && dchk::in(kSiteScalars, tok(t), 1, nTok)) ? a.dt[tok(t)] : 0.f;
+            thv[u] = (t < T && dchk::in(kSiteTheta, ti, 1, (a.th_head ? H : nTok) * kK2)) ? a.theta[ti] : 0.f;
         }
         float acc = 0.f, gh = 0.f;
         if (tid < Q) {
             const int64_t t = t0 + tid;
             float d = 0.f, l = 0.f, nx = 0.f, av = 0.f;
-            if (t < T) {
+            if (t < T && dchk::in(kSiteScalars, tok(t), 1, nTok) &&
+                dchk::in(kSiteScalars, a.a_tok ? tok(t) : h, 1, a.a_tok ? nTok : H)) {
                 d = a.dt[tok(t)];
                 l = a.lam[tok(t)];
                 av = a.a_tok ? a.A[tok(t)] : a.A[h];
-                if (t + 1 < T) nx = (1.f - a.lam[tok(t + 1)]) * a.dt[tok(t + 1)];
+                if (t + 1 < T && dchk::in(kSiteScalars, tok(t + 1), 1, nTok))
+                    nx = (1.f - a.lam[tok(t + 1)]) * a.dt[tok(t + 1)];
             }
             gam[tid] = l * d;
             gh = l * d + nx;
@@ -313,9 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
             for (int u = 0; u < 2; ++u) {
                 const int i = (tid >> 3) + 64 * u;
                 const int64_t t = t0 + i / R;
-                valid[u] = t < T;
+                const int64_t row = tok(t) * R + i % R;
+                valid[u] = t < T && dchk::in(kSiteRows, row * kN + 8 * j, 8, nTok * R * kN) &&
+                           dchk::in(kSiteRows, row * kP + 8 * j, 8, nTok * R * kP);
                 if (valid[u]) {
-                    const int64_t row = tok(t) * R + i % R;
                     const float4 *pb = reinterpret_cast<const float4 *>(a.B + row * kN + 8 * j);
                     const float4 *pc = reinterpret_cast<const float4 *>(a.C + row * kN + 8 * j);
                     const float4 *px = reinterpret_cast<const float4 *>(a.x + row * kP + 8 * j);
@@ -340,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
                                ld[u][3].x, ld[u][3].y, ld[u][3].z, ld[u][3].w};
                 const float xx[8] = {ld[u][4].x, ld[u][4].y, ld[u][4].z, ld[u][4].w,
                                      ld[u][5].x, ld[u][5].y, ld[u][5].z, ld[u][5].w};
-                if (a.wB && valid[u]) {  // BC-norm: the row's RMS over its 8 lanes, weight and bias
+                if (a.wB && valid[u] && dchk::in(kSiteNorm, (h * R + r) * kN + 8 * j, 8, H * R * kN) &&
+                    dchk::in(kSiteNorm, 8 * j, 8, kN)) {  // BC-norm: the row's RMS over its 8 lanes, weight and bias
                     const unsigned grp = 0xffu << (lane & 24);
                     float sb = 0.f, sq = 0.f;
 #pragma unroll
@@ -490,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
         const int ty = lq / R, ry = lq % R;
         const int64_t t_y = t0 + ty;
         float4 xv[kTC / 4];
-        if (t_y < T) {
+        if (t_y < T && dchk::in(kSiteRows, (tok(t_y) * R + ry) * kP + c0, kTC, nTok * R * kP)) {
             const float4 *xr = reinterpret_cast<const float4 *>(a.x + (tok(t_y) * R + ry) * kP + c0);
 #pragma unroll
             for (int e = 0; e < kTC / 4; ++e) xv[e] = xr[e];
@@ -530,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
                 tmem_ld16(tl + kColYd + c0 + 16 * qq, yd);
                 tmem_ld16(tl + kColYo + c0 + 16 * qq, yo);
                 tmem_wait_ld();
-                if (t_y < T) {
+                if (t_y < T && dchk::in(kSiteY, (tok(t_y) * R + ry) * kP + c0 + 16 * qq, 16, nTok * R * kP)) {
                     float4 *yr = reinterpret_cast<float4 *>(a.y + (tok(t_y) * R + ry) * kP + c0 + 16 * qq);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -550,14 +574,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc32_kernel(const Tc32Arg
     }
 
     if (ok) {  // final state: plain-frame h_{T-1}, the raw last token as the pending term
-        if (a.hT && own_state) {
+        if (a.hT && own_state && dchk::in(kSiteFinal, (bh * kN + srow) * kP + c0, kTC, nSt)) {
             float4 *dst = reinterpret_cast<float4 *>(a.hT + (bh * kN + srow) * kP + c0);
 #pragma unroll
             for (int p = 0; p < kTC / 4; ++p)
                 dst[p] = make_float4(hreg[4 * p], hreg[4 * p + 1], hreg[4 * p + 2], hreg[4 * p + 3]);
         }
-        if (T > 0) {
-            const int64_t last = tok(T - 1);
+        const int64_t last = tok(T - 1);
+        if (T > 0 && dchk::in(kSiteFinal, last * R * kN, R * kN, nTok * R * kN) &&
+            dchk::in(kSiteFinal, last * R * kP, R * kP, nTok * R * kP) &&
+            dchk::in(kSiteFinal, bh * R * kN, R * kN, BH * R * kN) && dchk::in(kSiteFinal, bh * R * kP, R * kP, BH * R * kP) &&
+            (!a.wB || (dchk::in(kSiteNorm, h * R * kN, R * kN, H * R * kN)))) {
             if (a.bpT && a.wB) {  // the last token's normalised B, one warp per rank row
                 for (int r = warp; r < R; r += kThreads / 32) {
                     const float *src = a.B + (last * R + r) * kN;
@@ -656,5 +683,7 @@ cudaError_t read_tc32_error(unsigned *code) {
     *code = v;
     return e;
 }
+
+M3_DCHECK_READER(read_dcheck_tc32)
 
 }  // namespace m3

@@ -130,7 +130,8 @@ def test_workspace_query_is_host_only(m3):
 
 
 def test_version(m3):
-    assert m3.lib.m3_version() == 102
+    assert m3.lib.m3_version() == 103
+    assert m3.lib.m3_device_checks() == 0  # the normal build
 
 
 def test_scan_plan_info_host_side(m3):
