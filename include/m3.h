@@ -377,6 +377,22 @@ M3_API m3_status m3_stream_status(void *stream);
  * pages have no counterpart to this call. */
 M3_API m3_status m3_selftest_wait_timeout(void *stream);
 
+/* Failure-path self-test of split sequences: the same call as
+ * m3_scan_fwd_algo(M3_ALGO_TC_SEGMENTS(segments), ...) (bf16 I/O, sizes the
+ * tensor-core path covers, segments >= 2, a workspace of
+ * m3_scan_workspace_size for that algo) but without the summary pass, so
+ * that the flags the main pass's look-back waits for are never published:
+ * the CTAs of segments 1 .. segments-1 give up after their bounded wait
+ * (about 1 s), record code 0x8, drain what they issued and return.  The next
+ * m3_stream_status then returns M3_ERR_TIMEOUT, y and the final state are
+ * incomplete, and the device stays usable.  The pages have no counterpart to
+ * this call. */
+M3_API m3_status m3_selftest_segment_timeout(const m3_dims *d, int segments, const void *x, const void *B,
+                                             const void *C, const void *dt, const void *lam, const void *theta,
+                                             const float *A, const float *D, const m3_state *init, void *y,
+                                             const m3_state *final_state, void *workspace,
+                                             size_t workspace_bytes, void *stream);
+
 /* Message describing the calling thread's most recent failure ("" if none). */
 M3_API const char *m3_last_error(void);
 

@@ -118,6 +118,8 @@ def _load():
     lib.m3_scan_fwd_host.restype = ctypes.c_int
     for f in (lib.m3_scan_workspace_size, lib.m3_scan_plan, lib.m3_scan_fwd, lib.m3_scan_fwd_algo, lib.m3_step):
         f.restype = ctypes.c_int
+    lib.m3_selftest_segment_timeout.argtypes = [dp, ctypes.c_int] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_selftest_segment_timeout.restype = ctypes.c_int
     lib.m3_selftest_wait_timeout.argtypes = [vp]
     lib.m3_selftest_wait_timeout.restype = ctypes.c_int
     lib.m3_stream_status.argtypes = [vp]
@@ -380,6 +382,28 @@ def selftest_wait_timeout(stream=None):
     dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
     with torch.cuda.device(dev):
         _check(get_lib().m3_selftest_wait_timeout(_stream(stream, dev)))
+
+
+def selftest_segment_timeout(x, B, C, dt, lam, theta, A, D, segments: int, init: State | None = None, *,
+                             stream=None):
+    """The split prefill without its summary pass (m3_selftest_segment_timeout):
+    the look-back waits of segments >= 1 give up (about 1 s) and the next
+    stream_status() raises M3Error(M3_ERR_TIMEOUT) with code 0x8.  Returns the
+    (incomplete) y and final state."""
+    dev = _require_cuda(x, B, C, dt, lam, theta, A, D, *(init or ()))
+    Bt, T, H, R, P = x.shape
+    N = B.shape[-1]
+    dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
+    with torch.cuda.device(dev):
+        y = torch.empty_like(x)
+        final = State(torch.empty(Bt, H, N, P, device=dev), torch.empty(Bt, H, R, N, device=dev),
+                      torch.empty(Bt, H, R, P, device=dev))
+        need = workspace_size(dims, ALGO_TC_SEGMENTS(segments))
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        _check(get_lib().m3_selftest_segment_timeout(
+            ctypes.byref(dims), segments, *map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(init), _ptr(y),
+            _cstate(final), _ptr(ws), need, _stream(stream, dev)))
+    return y, final
 
 
 def device_checks() -> bool:

@@ -163,7 +163,7 @@ bool tc_supported(const m3::Problem &p, const char **why) {
 m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
                     const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
                     void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream,
-                    bool static_ws = false, const m3_bcnorm *bcn = nullptr) {
+                    bool static_ws = false, const m3_bcnorm *bcn = nullptr, bool skip_summary = false) {
     m3_status s = check_dims(d, false);
     if (s != M3_OK) return s;
     const int segments = algo >> 8;
@@ -201,6 +201,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
     p.ws = ws;
     p.ws_bytes = ws_bytes;
     p.segments = segments;
+    p.skip_summary = skip_summary;
 
     const char *why = nullptr;
     const char *tc_why = nullptr;
@@ -373,6 +374,20 @@ m3_status m3_scan_fwd_static(int algo, const m3_dims *d, const void *x, const vo
                              const m3_state *init, void *y, const m3_state *final_state, void *stream) {
     try {
         return scan_impl(algo, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, nullptr, 0, stream, true);
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
+m3_status m3_selftest_segment_timeout(const m3_dims *d, int segments, const void *x, const void *B, const void *C,
+                                       const void *dt, const void *lam, const void *theta, const float *A,
+                                       const float *D, const m3_state *init, void *y, const m3_state *final_state,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+    try {
+        if (segments < 2) return fail(M3_ERR_INVALID_ARG, "m3_selftest_segment_timeout: segments must be >= 2");
+        if (!d || d->io != M3_BF16) return fail(M3_ERR_INVALID_ARG, "m3_selftest_segment_timeout: bf16 I/O only");
+        return scan_impl(M3_ALGO_TC_SEGMENTS(segments), d, x, B, C, dt, lam, theta, A, D, init, y, final_state,
+                         workspace, workspace_bytes, stream, false, nullptr, true);
     } catch (...) {
         return fail(M3_ERR_INVALID_ARG, "internal error");
     }

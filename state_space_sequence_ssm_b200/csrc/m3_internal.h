@@ -25,6 +25,7 @@ struct Problem {
     size_t ws_bytes;
     int segments;                 // tensor-core prefill: segments per sequence (0 = chosen by the library)
     size_t ws_cap;                // > 0: the library's choice of segments must fit this workspace
+    bool skip_summary;            // failure-path self-test: split sequences without their summary pass
     cudaStream_t stream;
 };
 
