@@ -1,6 +1,8 @@
 """Failure detection on the GPU without a fault: a bounded device wait that is
-made to give up must surface as M3_ERR_TIMEOUT through m3_stream_status, be
-cleared by that call, and leave the context usable."""
+made to give up -- in the self-test kernel, and in the split prefill's
+look-back on a segment flag that is never published -- must surface as
+M3_ERR_TIMEOUT through m3_stream_status, be cleared by that call, and leave
+the context usable."""
 import pytest
 import torch
 
