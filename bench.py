@@ -93,7 +93,8 @@ def run_case(args):
         for _ in range(args.case_launches):
             m3.scan_fwd(*(inp[k] for k in keys), None)
     else:
-        name = args.workload if args.workload.startswith("decode") else DECODE_WORKLOADS[0]
+        # a decode workload, or the long-context workload's own sequences
+        name = args.workload if args.workload.startswith(("decode", "long")) else DECODE_WORKLOADS[0]
         s = WORKLOADS[name]
         s = s.with_(batch=args.case_batch or s.batch)
         st = m3.State(*(t.cuda() for t in make_state(s)))

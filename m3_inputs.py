@@ -135,6 +135,40 @@ def make_bcnorm(shape: Shape, device="cpu", seed_offset: int = 3):
     return dict(wB=wB, wC=wC, bB=bB, bC=bC, eps=1e-6)
 
 
+def make_proj(shape: Shape, device="cpu", seed_offset: int = 4):
+    """Synthetic MIMO projection weights (fp32): wx [H, R, P], wB, wC [H, R, N]
+    ~ N(0, 1), so that each widened column keeps the scale of the SISO draw,
+    and wy [H, R, P] ~ N(0, 1) / sqrt(R), so that the sum over the R ranks
+    keeps the scale of one."""
+    H, R, P, N = shape.nheads, shape.rank, shape.headdim, shape.dstate
+    g = _gen(shape.seed + seed_offset, device)
+    f = dict(device=device, dtype=torch.float32, generator=g)
+    wx = torch.randn(H, R, P, **f)
+    wB = torch.randn(H, R, N, **f)
+    wC = torch.randn(H, R, N, **f)
+    wy = torch.randn(H, R, P, **f) / math.sqrt(R)
+    return dict(wx=wx, wB=wB, wC=wC, wy=wy)
+
+
+def make_prefill_proj(shape: Shape, device="cpu", **kw):
+    """Inputs of one prefill call with the MIMO projections: the draws of
+    make_prefill for this shape at rank 1, with x [Bt, T, H, P] and
+    B, C [Bt, T, H, N] (the rank axis dropped); the rest unchanged."""
+    d = make_prefill(shape.with_(rank=1), device=device, **kw)
+    for k in ("x", "B", "C"):
+        d[k] = d[k][:, :, :, 0].contiguous()
+    return d
+
+
+def make_steps_proj(shape: Shape, nsteps: int, device="cpu", **kw):
+    """Decode-step inputs with the MIMO projections: make_steps at rank 1 with
+    x [S, Bt, H, P] and B, C [S, Bt, H, N]."""
+    d = make_steps(shape.with_(rank=1), nsteps, device=device, **kw)
+    for k in ("x", "B", "C"):
+        d[k] = d[k][:, :, :, 0].contiguous()
+    return d
+
+
 def make_state(shape: Shape, device="cpu", seed_offset: int = 2, scale: float = 1.0):
     """A random (h, b_prev, x_prev) state in fp32, for tests that start from a
     nonzero state."""

@@ -134,6 +134,42 @@ def scan(x, B, C, dt, lam, theta, A, D, init: State | None = None, nthreads: int
     return y, State(hT, bpT, xpT)
 
 
+@dataclass
+class MimoProj:
+    """MIMO projections, as this build reads "Mamba-3, parte 1" (the
+    architecture paragraph: the MIMO projections widen B and C to the shape
+    the MIMO SSM needs) and "Знакомство с Mamba-3" (section 3: rank-R input
+    and output projections, B_t in R^{N x R}, x_t in R^{P x R}): per head and
+    rank, elementwise weights that widen the SISO-shaped x_t [P], B_t, C_t [N]
+    of a token-head to rank R, and project the rank-R output back to P."""
+    wx: np.ndarray  # [H, R, P]
+    wB: np.ndarray  # [H, R, N]
+    wC: np.ndarray  # [H, R, N]
+    wy: np.ndarray  # [H, R, P]
+
+
+def _widen(v, w):
+    """v [..., H, K] (SISO-shaped), w [H, R, K] -> [..., H, R, K]: column r is w[h, r] * v."""
+    return _f64(v)[..., :, None, :] * _f64(w)
+
+
+def scan_proj(x, B, C, dt, lam, theta, A, D, proj: MimoProj, init: State | None = None, nthreads: int = 0):
+    """Scan with the MIMO projections: x [Bt,T,H,P], B/C [Bt,T,H,N] are widened
+    to rank R (X[..., r, :] = wx[h, r] * x, likewise B and C), the rank-R scan
+    runs as `scan`, and y [Bt,T,H,P] = sum_r wy[h, r] * Y[..., r, :] (Y with its
+    D term).  The state keeps the rank-R form (b_prev, x_prev widened)."""
+    Y, st = scan(_widen(x, proj.wx), _widen(B, proj.wB), _widen(C, proj.wC), dt, lam, theta, A, D, init,
+                 nthreads=nthreads)
+    return (Y * _f64(proj.wy)).sum(axis=-2), st
+
+
+def step_proj(x, B, C, dt, lam, theta, A, D, proj: MimoProj, state: State):
+    """One decode step with the MIMO projections: x [Bt,H,P], B/C [Bt,H,N];
+    returns (y [Bt,H,P], new State)."""
+    Y, st = step(_widen(x, proj.wx), _widen(B, proj.wB), _widen(C, proj.wC), dt, lam, theta, A, D, state)
+    return (Y * _f64(proj.wy)).sum(axis=-2), st
+
+
 def step(x, B, C, dt, lam, theta, A, D, state: State, bcnorm: BCNorm | None = None):
     """One decode step for every (b,h).  x [Bt,H,R,P], B/C [Bt,H,R,N],
     dt/lam [Bt,H], theta [Bt,H,N/2], D [H], A [H] or [Bt,H] (per token).

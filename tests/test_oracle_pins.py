@@ -616,3 +616,97 @@ def test_bcnorm_eps_inside_the_root_with_both_options():
     d3["C"] = d["C"] / (np.sqrt(np.mean(d["C"] ** 2, axis=-1, keepdims=True)) + eps) * bn["wC"] + bn["bC"][None, None]
     y3, _ = run(d3, st)
     assert rel(y3, y1) > 1e-3
+
+
+# ---------------------------------------------------------------- MIMO projections
+def proj_case(T=29, H=2, P=5, N=8, R=3, seed=7):
+    from m3_inputs import make_prefill_proj, make_proj
+    s = Shape(1, T, H, P, N, R, "f32", seed)
+    d = {k: v.double().numpy() for k, v in make_prefill_proj(s).items()}
+    w = {k: v.double().numpy() for k, v in make_proj(s).items()}
+    return d, oracle.MimoProj(w["wx"], w["wB"], w["wC"], w["wy"])
+
+
+def run_proj(d, pr, st=None):
+    return oracle.scan_proj(d["x"], d["B"], d["C"], d["dt"], d["lam"], d["theta"], d["A"], d["D"], pr, st)
+
+
+def test_proj_is_a_sum_of_siso_runs():
+    """With the projections the rank-R write is still a sum of R outer
+    products on one state, so y equals sum_r wy_r * (sum_q SISO runs driven by
+    (wB_q b, wx_q x) and read out with wC_r c, plus D wx_r x) -- R^2 rank-1
+    runs of the plain scan, combined in numpy."""
+    d, pr = proj_case()
+    y, _ = run_proj(d, pr)
+    x, b, c = d["x"], d["B"], d["C"]
+    R = pr.wx.shape[1]
+    ref = np.zeros_like(y)
+    for r in range(R):
+        yr = pr.wx[None, None, :, r] * x * d["D"][None, None, :, None]
+        for q in range(R):
+            ys, _ = oracle.scan((pr.wx[None, None, :, q] * x)[:, :, :, None],
+                                (pr.wB[None, None, :, q] * b)[:, :, :, None],
+                                (pr.wC[None, None, :, r] * c)[:, :, :, None],
+                                d["dt"], d["lam"], d["theta"], d["A"], np.zeros_like(d["D"]))
+            yr = yr + ys[:, :, :, 0]
+        ref += pr.wy[None, None, :, r] * yr
+    assert rel(y, ref) < TOL
+
+
+def test_proj_with_unit_weights_is_r_times_siso():
+    """wx = wB = wC = 1 and wy = (1, 0, ..., 0): the R identical outer products
+    write R copies of the SISO update into the state, so y = R * (SISO scan
+    without its D term) + D x."""
+    d, pr = proj_case(R=4)
+    H, R, P = pr.wx.shape
+    N = pr.wB.shape[-1]
+    wy = np.zeros((H, R, P))
+    wy[:, 0] = 1.0
+    unit = oracle.MimoProj(np.ones((H, R, P)), np.ones((H, R, N)), np.ones((H, R, N)), wy)
+    y, st = run_proj(d, unit)
+    ys, ss = oracle.scan(d["x"][:, :, :, None], d["B"][:, :, :, None], d["C"][:, :, :, None], d["dt"],
+                         d["lam"], d["theta"], d["A"], np.zeros_like(d["D"]))
+    assert rel(y, R * ys[:, :, :, 0] + d["D"][None, None, :, None] * d["x"]) < TOL
+    assert rel(st.h, R * ss.h) < TOL
+
+
+def test_proj_rank_one_unit_weights_is_siso():
+    d, pr = proj_case(R=1)
+    H, R, P = pr.wx.shape
+    N = pr.wB.shape[-1]
+    unit = oracle.MimoProj(np.ones((H, 1, P)), np.ones((H, 1, N)), np.ones((H, 1, N)), np.ones((H, 1, P)))
+    y, _ = run_proj(d, unit)
+    ys, _ = oracle.scan(d["x"][:, :, :, None], d["B"][:, :, :, None], d["C"][:, :, :, None], d["dt"],
+                        d["lam"], d["theta"], d["A"], d["D"])
+    np.testing.assert_array_equal(y, ys[:, :, :, 0])
+
+
+def test_proj_output_is_linear_in_wy_and_state_ignores_it():
+    d, pr = proj_case()
+    y1, s1 = run_proj(d, pr)
+    pr2 = oracle.MimoProj(pr.wx, pr.wB, pr.wC, 2.5 * pr.wy - 0.5)
+    y2, s2 = run_proj(d, pr2)
+    pr0 = oracle.MimoProj(pr.wx, pr.wB, pr.wC, np.ones_like(pr.wy))
+    y0, _ = run_proj(d, pr0)
+    assert rel(y2, 2.5 * y1 - 0.5 * y0) < TOL
+    np.testing.assert_array_equal(s1.h, s2.h)
+
+
+def test_proj_prefill_then_decode_equals_full_scan():
+    """scan_proj over T1 tokens, then step_proj for the rest, equals one
+    scan_proj (the widened pending term crosses the boundary in the state)."""
+    d, pr = proj_case(T=21, R=2)
+    s = Shape(1, 21, 2, 5, 8, 2, "f32", 7)
+    h, bp, xp = (t.double().numpy() for t in make_state(s))
+    st0 = oracle.State(h, bp, xp)
+    yfull, sfull = run_proj(d, pr, st0)
+    T1 = 13
+    part = {k: (v[:, :T1] if v.ndim >= 3 else v) for k, v in d.items()}
+    y1, st = run_proj(part, pr, st0)
+    ys = [y1]
+    for t in range(T1, 21):
+        yt, st = oracle.step_proj(d["x"][:, t], d["B"][:, t], d["C"][:, t], d["dt"][:, t], d["lam"][:, t],
+                                  d["theta"][:, t], d["A"], d["D"], pr, st)
+        ys.append(yt[:, None])
+    np.testing.assert_allclose(np.concatenate(ys, axis=1), yfull, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(st.h, sfull.h, atol=1e-13, rtol=0)
