@@ -249,19 +249,23 @@ class ClockSampler:
                 "power_w_max": max(pw) if pw else None}
 
 
-def prefill_bytes(s, with_final=True, with_init=False, a_per_token=False, theta_per_head=False):
+def prefill_bytes(s, with_final=True, with_init=False, a_per_token=False, theta_per_head=False, proj=False):
     """Algorithmic HBM bytes of one prefill call: each input read once, y
     written once, the final state written once (init read once if given);
     a data-dependent A adds one fp32 per token-head, angle rates fixed per head
-    are read once per head instead of once per token-head."""
+    are read once per head instead of once per token-head; with the MIMO
+    projections x, B, C and y hold one row per token-head and the fp32
+    weights are read once."""
     io = 2 if s.io == "bf16" else 4
     th = s.batch * s.seqlen * s.nheads
     theta_tok = 0 if theta_per_head else s.dstate // 2
-    per_tok = io * (2 * s.rank * s.headdim + 2 * s.rank * s.dstate + 2 + theta_tok) + 4 * int(a_per_token)
+    rio = 1 if proj else s.rank
+    per_tok = io * (2 * rio * s.headdim + 2 * rio * s.dstate + 2 + theta_tok) + 4 * int(a_per_token)
+    th_w = 4 * s.nheads * s.rank * 2 * (s.headdim + s.dstate) if proj else 0
     state = 4 * s.batch * s.nheads * (s.dstate * s.headdim + s.rank * (s.dstate + s.headdim))
     a_bytes = 0 if a_per_token else 4 * s.nheads
     theta_bytes = io * s.nheads * (s.dstate // 2) if theta_per_head else 0
-    return th * per_tok + state * (int(with_final) + int(with_init)) + 4 * s.nheads + a_bytes + theta_bytes
+    return th * per_tok + state * (int(with_final) + int(with_init)) + 4 * s.nheads + a_bytes + theta_bytes + th_w
 
 
 def step_bytes(s):
@@ -667,7 +671,9 @@ def run_ours(args):
 
 VARIANTS = {"a_per_token": "data-dependent A_t (M3_FLAG_A_PER_TOKEN)",
             "theta_per_head": "angle rates fixed per head (M3_FLAG_THETA_PER_HEAD)",
-            "bcnorm": "fused BC-norm prologue (m3_scan_fwd_bcnorm)"}
+            "bcnorm": "fused BC-norm prologue (m3_scan_fwd_bcnorm)",
+            "mimo_proj": "fused MIMO projections (m3_scan_fwd_proj) on the MIMO workload's shape"}
+MIMO_WORKLOAD = "mimo_bf16_b8_t4096_h32_p64_n64_r4"
 
 
 def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_peak, peak_src, keys, stream):
@@ -679,35 +685,43 @@ def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_p
 
     from m3_inputs import make_bcnorm
 
-    s = replica_shape(args.workload, rank)
-    inp = make_prefill(s, device=dev, **({} if kind == "bcnorm" else {kind: True}))
-    bcn = None
+    from m3_inputs import make_prefill_proj, make_proj
+
+    workload = MIMO_WORKLOAD if kind == "mimo_proj" else args.workload
+    s = replica_shape(workload, rank)
+    bcn = proj = None
+    if kind == "mimo_proj":
+        inp = make_prefill_proj(s, device=dev)
+        w = make_proj(s, device=dev)
+        proj = m3.MimoProj(w["wx"], w["wB"], w["wC"], w["wy"])
+    else:
+        inp = make_prefill(s, device=dev, **({} if kind == "bcnorm" else {kind: True}))
     if kind == "bcnorm":
         p = make_bcnorm(s, device=dev)
         bcn = m3.BCNorm(p["wB"], p["wC"], p["bB"], p["bC"], p["eps"])
     y = torch.empty_like(inp["x"])
     fin = m3.empty_state(s.batch, s.nheads, s.dstate, s.headdim, s.rank, device=dev)
     for _ in range(args.warmup):
-        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream, bcnorm=bcn)
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream, bcnorm=bcn, proj=proj)
     K = args.steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(K):
-        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream, bcnorm=bcn)
+        m3.scan_fwd(*(inp[k] for k in keys), None, y=y, final=fin, stream=stream, bcnorm=bcn, proj=proj)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     m3.stream_status(stream)
     el = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-    ab = prefill_bytes(s, **({} if kind == "bcnorm" else {kind: True}))
+    ab = prefill_bytes(s, **({} if kind == "bcnorm" else {"proj" if kind == "mimo_proj" else kind: True}))
     if kind == "bcnorm":  # the norm weights and the biases, read once
         ab += 4 * (2 * s.dstate + 2 * s.nheads * s.rank * s.dstate)
     ach = ab / (el / K) / 1e9
     del inp, y, fin
     torch.cuda.empty_cache()
-    return {"variant": VARIANTS[kind], "workload": args.workload,
+    return {"variant": VARIANTS[kind], "workload": workload,
             "value": world * K * s.batch * s.seqlen / el, "unit": "tokens/s", "steps": K,
             "ms_per_step": 1e3 * el / K, "gpu_launches": K,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,

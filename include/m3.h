@@ -155,6 +155,46 @@ typedef enum m3_algo {
  * published. */
 #define M3_ALGO_TC_SEGMENTS(s) (M3_ALGO_TC | ((int)(s) << 8))
 
+/* MIMO projections, as read from "Mamba-3, parte 1" (architecture paragraph:
+ * the projections widen B and C to the shape the MIMO SSM needs; TileLang
+ * paragraph: the extra projections let the MIMO prefill save I/O through the
+ * memory hierarchy) and "Знакомство с Mamba-3", section 3 (rank-R input and
+ * output projections, B_t in R^{N x R}, x_t in R^{P x R}); the pages give no
+ * shapes, so this is the plainest form: per head h and rank r, elementwise
+ * fp32 weights widen the token-head's one row of x [P], B [N], C [N] to rank
+ * R -- X[.., r, p] = wx[h, r, p] x[p], likewise B with wB and C with wC --
+ * the rank-R scan runs on them, and the output row is y[p] = sum_r
+ * wy[h, r, p] Y[.., r, p] (Y including its D x term).  Layouts: wx, wy
+ * [H, R, P], wB, wC [H, R, N], fp32, 4-byte aligned, owned by the caller.
+ * The kernels widen on chip, so x, B, C and y cross HBM at one row per
+ * token-head. */
+typedef struct m3_mimo_proj {
+    const float *wx, *wB, *wC, *wy;
+} m3_mimo_proj;
+
+/* m3_scan_fwd_algo with the MIMO projections: x [B,T,H,P], B and C
+ * [B,T,H,N], y [B,T,H,P] (one row per token-head; dt, lam, theta, A, D as
+ * usual); d->rank is the rank R the projections widen to; the states (init,
+ * final_state) keep the rank-R layout, their pending term widened.  bf16
+ * I/O on the tensor-core prefill only (headdim 64, dstate 64 or 128, rank 1,
+ * 2 or 4; split sequences and the per-token A and per-head theta layouts
+ * included), M3_ERR_UNSUPPORTED otherwise and with algo M3_ALGO_SIMT; not
+ * combined with the BC-norm prologue.  The workspace is the same as for
+ * m3_scan_fwd_algo with these dims. */
+M3_API m3_status m3_scan_fwd_proj(int algo, const m3_dims *d, const m3_mimo_proj *proj, const void *x,
+                                  const void *B, const void *C, const void *dt, const void *lam,
+                                  const void *theta, const float *A, const float *D, const m3_state *init,
+                                  void *y, const m3_state *final_state, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
+/* m3_step with the MIMO projections: x [B,H,P], B and C [B,H,N], y [B,H,P];
+ * the state in the rank-R layout, updated in place (b_prev, x_prev widened).
+ * The register-tiled decode sizes only ((dstate, headdim) in {64, 128} x
+ * {64, 128} or (256, 64); rank 1, 2 or 4): M3_ERR_UNSUPPORTED otherwise. */
+M3_API m3_status m3_step_proj(const m3_dims *d, const m3_mimo_proj *proj, const void *x, const void *B,
+                              const void *C, const void *dt, const void *lam, const void *theta,
+                              const float *A, const float *D, const m3_state *state, void *y, void *stream);
+
 /* Bytes of device workspace m3_scan_fwd needs for these dims (0 = none; the
  * workspace pointer may then be NULL).  Host function; the answer depends on
  * the current CUDA device's SM count (it sets how sequences are split).  The
@@ -410,7 +450,8 @@ M3_API int m3_device_checks(void);
 
 /* ABI version of this header (major * 100 + minor): 101 adds m3_scan_plan_info,
  * 102 the fp32 tensor-core prefill (M3_KERNEL_TC32), 103 the bounds build
- * (m3_device_checks, M3_ERR_BOUNDS) and split sequences in two launches. */
+ * (m3_device_checks, M3_ERR_BOUNDS), split sequences in two launches and the
+ * MIMO projections (m3_scan_fwd_proj, m3_step_proj). */
 M3_API int m3_version(void);
 
 #ifdef __cplusplus

@@ -62,6 +62,24 @@ def _cbcn(b: BCNorm):
     return ctypes.byref(CBCNorm(b.wB.data_ptr(), b.wC.data_ptr(), b.bB.data_ptr(), b.bC.data_ptr(), float(b.eps)))
 
 
+class CMimoProj(ctypes.Structure):
+    _fields_ = [("wx", ctypes.c_void_p), ("wB", ctypes.c_void_p), ("wC", ctypes.c_void_p), ("wy", ctypes.c_void_p)]
+
+
+class MimoProj(NamedTuple):
+    """MIMO projection weights (device fp32 tensors): wx, wy [H, R, P] and
+    wB, wC [H, R, N]; with them x, B, C and y hold one row per token-head
+    (see m3_mimo_proj in include/m3.h)."""
+    wx: torch.Tensor
+    wB: torch.Tensor
+    wC: torch.Tensor
+    wy: torch.Tensor
+
+
+def _cproj(p: MimoProj):
+    return ctypes.byref(CMimoProj(p.wx.data_ptr(), p.wB.data_ptr(), p.wC.data_ptr(), p.wy.data_ptr()))
+
+
 class CPlanInfo(ctypes.Structure):
     _fields_ = [("workspace_bytes", ctypes.c_size_t), ("kernel", ctypes.c_int32), ("segments", ctypes.c_int32),
                 ("launches", ctypes.c_int32), ("reserved", ctypes.c_int32), ("ctas", ctypes.c_int64)]
@@ -108,6 +126,11 @@ def _load():
     lib.m3_scan_fwd_bcnorm.restype = ctypes.c_int
     lib.m3_step_bcnorm.argtypes = [dp, bp_] + [vp] * 8 + [sp, vp, vp]
     lib.m3_step_bcnorm.restype = ctypes.c_int
+    pp_ = ctypes.POINTER(CMimoProj)
+    lib.m3_scan_fwd_proj.argtypes = [ctypes.c_int, dp, pp_] + [vp] * 8 + [sp, vp, sp, vp, ctypes.c_size_t, vp]
+    lib.m3_scan_fwd_proj.restype = ctypes.c_int
+    lib.m3_step_proj.argtypes = [dp, pp_] + [vp] * 8 + [sp, vp, vp]
+    lib.m3_step_proj.restype = ctypes.c_int
     lib.m3_scan_fwd_static.argtypes = [ctypes.c_int, dp] + [vp] * 8 + [sp, vp, sp, vp]
     lib.m3_scan_fwd_static.restype = ctypes.c_int
     lib.m3_step.argtypes = [dp] + [vp] * 8 + [sp, vp, vp]
@@ -258,14 +281,22 @@ def scan_plan_info(dims: Dims, algo: int = ALGO_AUTO, flags: int = 0) -> PlanInf
 
 def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_state: bool = True,
              y=None, final: State | None = None, workspace=None, algo: int = ALGO_AUTO, stream=None,
-             bcnorm: BCNorm | None = None):
+             bcnorm: BCNorm | None = None, proj: MimoProj | None = None):
     """Prefill scan (with the BC-norm prologue when `bcnorm` is given).  x [Bt,T,H,R,P], B/C [Bt,T,H,R,N], dt/lam [Bt,T,H],
     theta [Bt,T,H,N/2] (or [H,N/2]: fixed per head) in one io dtype (fp32 or
     bf16); D [H] fp32; A [H] fp32, or [Bt,T,H] fp32 for a data-dependent A_t.
+    With the MIMO projections `proj`: x [Bt,T,H,P], B/C [Bt,T,H,N] and y
+    [Bt,T,H,P], widened to the rank of proj's weights on chip.
     Returns (y, final State or None)."""
     dev = _require_cuda(x, B, C, dt, lam, theta, A, D, y, workspace, *(init or ()), *(final or ()),
-                        *(bcnorm[:4] if bcnorm is not None else ()))
-    Bt, T, H, R, P = x.shape
+                        *(bcnorm[:4] if bcnorm is not None else ()), *(proj or ()))
+    if proj is not None:
+        if bcnorm is not None:
+            raise M3Error(M3_ERR_UNSUPPORTED, "the MIMO projections do not combine with the BC-norm prologue")
+        Bt, T, H, P = x.shape
+        R = proj.wx.shape[1]
+    else:
+        Bt, T, H, R, P = x.shape
     N = B.shape[-1]
     dims = make_dims(Bt, T, H, P, N, R, x.dtype, a_per_token=A.dim() == 3, theta_per_head=theta.dim() == 2)
     with torch.cuda.device(dev):
@@ -280,7 +311,9 @@ def scan_fwd(x, B, C, dt, lam, theta, A, D, init: State | None = None, *, want_s
         ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
         args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(init), _ptr(y), _cstate(final),
                 _ptr(workspace), ws_bytes, _stream(stream, dev))
-        if bcnorm is None:
+        if proj is not None:
+            _check(get_lib().m3_scan_fwd_proj(algo, ctypes.byref(dims), _cproj(proj), *args))
+        elif bcnorm is None:
             _check(get_lib().m3_scan_fwd_algo(algo, ctypes.byref(dims), *args))
         else:
             _check(get_lib().m3_scan_fwd_bcnorm(algo, ctypes.byref(dims), _cbcn(bcnorm), *args))
@@ -420,19 +453,28 @@ def stream_status(stream=None):
         _check(get_lib().m3_stream_status(_stream(stream, dev)))
 
 
-def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None, bcnorm: BCNorm | None = None):
+def step(x, B, C, dt, lam, theta, A, D, state: State, *, y=None, stream=None, bcnorm: BCNorm | None = None,
+         proj: MimoProj | None = None):
     """One decode step in place on `state`.  x [Bt,H,R,P], B/C [Bt,H,R,N],
     dt/lam [Bt,H], theta [Bt,H,N/2] (or [H,N/2]: fixed per head); A [H] fp32,
-    or [Bt,H] fp32 for a data-dependent A_t.  Returns y [Bt,H,R,P]."""
-    dev = _require_cuda(x, B, C, dt, lam, theta, A, D, y, *state, *(bcnorm[:4] if bcnorm is not None else ()))
-    Bt, H, R, P = x.shape
+    or [Bt,H] fp32 for a data-dependent A_t.  Returns y [Bt,H,R,P].  With the
+    MIMO projections `proj`: x [Bt,H,P], B/C [Bt,H,N], y [Bt,H,P]."""
+    dev = _require_cuda(x, B, C, dt, lam, theta, A, D, y, *state, *(bcnorm[:4] if bcnorm is not None else ()),
+                        *(proj or ()))
+    if proj is not None:
+        Bt, H, P = x.shape
+        R = proj.wx.shape[1]
+    else:
+        Bt, H, R, P = x.shape
     N = B.shape[-1]
     dims = make_dims(Bt, 1, H, P, N, R, x.dtype, a_per_token=A.dim() == 2, theta_per_head=theta.dim() == 2)
     with torch.cuda.device(dev):
         if y is None:
             y = torch.empty_like(x)
         args = (*map(_ptr, (x, B, C, dt, lam, theta, A, D)), _cstate(state), _ptr(y), _stream(stream, dev))
-        if bcnorm is None:
+        if proj is not None:
+            _check(get_lib().m3_step_proj(ctypes.byref(dims), _cproj(proj), *args))
+        elif bcnorm is None:
             _check(get_lib().m3_step(ctypes.byref(dims), *args))
         else:
             _check(get_lib().m3_step_bcnorm(ctypes.byref(dims), _cbcn(bcnorm), *args))

@@ -64,11 +64,13 @@ m3_status check_dims(const m3_dims *d, bool decode) {
 }
 
 // Shared validation of tensor pointers.  `tok` = number of token-heads.
+// proj: the MIMO projections' layout (x, B, C and y with one row per
+// token-head instead of R).
 m3_status check_tensors(const m3_dims *d, int64_t tok, const void *x, const void *B, const void *C,
                         const void *dt, const void *lam, const void *theta, const float *A,
-                        const float *D, const void *y, Range *ins, int *nin, Range *yr) {
+                        const float *D, const void *y, Range *ins, int *nin, Range *yr, bool proj = false) {
     const size_t es = d->io == M3_BF16 ? 2 : 4;
-    const int64_t R = d->rank, P = d->headdim, N = d->dstate;
+    const int64_t R = proj ? 1 : d->rank, P = d->headdim, N = d->dstate;
     if (tok > 0) {
         if (!x || !B || !C || !dt || !lam || !theta || !y)
             return fail(M3_ERR_INVALID_ARG, "x, B, C, dt, lam, theta and y are required");
@@ -154,6 +156,21 @@ m3_status check_bcnorm(const m3_dims *d, const m3_bcnorm *bcn, Range yr) {
     return M3_OK;
 }
 
+m3_status check_proj(const m3_dims *d, const m3_mimo_proj *pr, Range yr) {
+    if (!pr) return fail(M3_ERR_INVALID_ARG, "proj is NULL");
+    if (!pr->wx || !pr->wB || !pr->wC || !pr->wy)
+        return fail(M3_ERR_INVALID_ARG, "proj: wx, wB, wC and wy are all required");
+    if ((reinterpret_cast<uintptr_t>(pr->wx) | reinterpret_cast<uintptr_t>(pr->wB) |
+         reinterpret_cast<uintptr_t>(pr->wC) | reinterpret_cast<uintptr_t>(pr->wy)) % 4)
+        return fail(M3_ERR_INVALID_ARG, "proj arrays must be 4-byte aligned");
+    const int64_t hr = d->nheads * d->rank;
+    const Range rs[4] = {range(pr->wx, hr * d->headdim * 4), range(pr->wB, hr * d->dstate * 4),
+                         range(pr->wC, hr * d->dstate * 4), range(pr->wy, hr * d->headdim * 4)};
+    for (const Range &r : rs)
+        if (overlap(r, yr)) return fail(M3_ERR_INVALID_ARG, "y overlaps a proj array");
+    return M3_OK;
+}
+
 // The tensor-core kernel for p's I/O type (bf16: prefill_tc, fp32:
 // prefill_tc32) and whether it covers p.
 bool tc_supported(const m3::Problem &p, const char **why) {
@@ -163,7 +180,8 @@ bool tc_supported(const m3::Problem &p, const char **why) {
 m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
                     const void *lam, const void *theta, const float *A, const float *D, const m3_state *init,
                     void *y, const m3_state *fin, void *ws, size_t ws_bytes, void *stream,
-                    bool static_ws = false, const m3_bcnorm *bcn = nullptr, bool skip_summary = false) {
+                    bool static_ws = false, const m3_bcnorm *bcn = nullptr, bool skip_summary = false,
+                    const m3_mimo_proj *proj = nullptr) {
     m3_status s = check_dims(d, false);
     if (s != M3_OK) return s;
     const int segments = algo >> 8;
@@ -175,7 +193,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
     const int64_t tok = d->batch * d->seqlen * d->nheads;
     Range ins[8], yr;
     int nin = 0;
-    s = check_tensors(d, tok, x, B, C, dt, lam, theta, A, D, y, ins, &nin, &yr);
+    s = check_tensors(d, tok, x, B, C, dt, lam, theta, A, D, y, ins, &nin, &yr, proj != nullptr);
     if (s != M3_OK) return s;
     Range ir[3] = {}, fr[3] = {};
     if (init && (s = check_state(d, init, "init", ir)) != M3_OK) return s;
@@ -193,9 +211,16 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
         }
     }
     if (bcn && (s = check_bcnorm(d, bcn, yr)) != M3_OK) return s;
+    if (proj) {
+        if ((s = check_proj(d, proj, yr)) != M3_OK) return s;
+        if (bcn) return fail(M3_ERR_UNSUPPORTED, "the MIMO projections do not combine with the BC-norm prologue");
+        if (d->io != M3_BF16 || algo == M3_ALGO_SIMT)
+            return fail(M3_ERR_UNSUPPORTED, "the MIMO projections run on the bf16 tensor-core prefill only");
+    }
     if (d->batch == 0) return M3_OK;  // nothing to read or write, whichever kernel was asked for
     m3::Problem p = make_problem(d, x, B, C, dt, lam, theta, A, D, y, stream);
     if (bcn) { p.wB = bcn->wB; p.wC = bcn->wC; p.bB = bcn->bB; p.bC = bcn->bC; p.eps = bcn->eps; }
+    if (proj) { p.pwx = proj->wx; p.pwB = proj->wB; p.pwC = proj->wC; p.pwy = proj->wy; }
     if (init) { p.h0 = init->h; p.bp0 = init->b_prev; p.xp0 = init->x_prev; }
     if (fin) { p.hT = fin->h; p.bpT = fin->b_prev; p.xpT = fin->x_prev; }
     p.ws = ws;
@@ -207,7 +232,7 @@ m3_status scan_impl(int algo, const m3_dims *d, const void *x, const void *B, co
     const char *tc_why = nullptr;
     const bool tc_ok = tc_supported(p, &tc_why);
     bool use_tc = false;
-    if (algo == M3_ALGO_TC) {
+    if (algo == M3_ALGO_TC || proj) {
         if (!tc_ok) return fail(M3_ERR_UNSUPPORTED, "%s", tc_why ? tc_why : "tensor-core path unsupported");
         use_tc = true;
     } else if (algo == M3_ALGO_AUTO) {
@@ -369,6 +394,19 @@ m3_status m3_scan_fwd_bcnorm(int algo, const m3_dims *d, const m3_bcnorm *bcn, c
     }
 }
 
+m3_status m3_scan_fwd_proj(int algo, const m3_dims *d, const m3_mimo_proj *proj, const void *x, const void *B,
+                           const void *C, const void *dt, const void *lam, const void *theta, const float *A,
+                           const float *D, const m3_state *init, void *y, const m3_state *final_state,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    try {
+        if (!proj) return fail(M3_ERR_INVALID_ARG, "proj is NULL");
+        return scan_impl(algo, d, x, B, C, dt, lam, theta, A, D, init, y, final_state, workspace,
+                         workspace_bytes, stream, false, nullptr, false, proj);
+    } catch (...) {
+        return fail(M3_ERR_INVALID_ARG, "internal error");
+    }
+}
+
 m3_status m3_scan_fwd_static(int algo, const m3_dims *d, const void *x, const void *B, const void *C,
                              const void *dt, const void *lam, const void *theta, const float *A, const float *D,
                              const m3_state *init, void *y, const m3_state *final_state, void *stream) {
@@ -447,7 +485,14 @@ m3_status m3_stream_status(void *stream) {
 
 m3_status step_impl(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B, const void *C,
                     const void *dt, const void *lam, const void *theta, const float *A, const float *D,
-                    const m3_state *state, void *y, void *stream);
+                    const m3_state *state, void *y, void *stream, const m3_mimo_proj *proj = nullptr);
+
+m3_status m3_step_proj(const m3_dims *d, const m3_mimo_proj *proj, const void *x, const void *B, const void *C,
+                       const void *dt, const void *lam, const void *theta, const float *A, const float *D,
+                       const m3_state *state, void *y, void *stream) {
+    if (!proj) return fail(M3_ERR_INVALID_ARG, "proj is NULL");
+    return step_impl(d, nullptr, x, B, C, dt, lam, theta, A, D, state, y, stream, proj);
+}
 
 m3_status m3_step(const m3_dims *d, const void *x, const void *B, const void *C, const void *dt,
                   const void *lam, const void *theta, const float *A, const float *D, const m3_state *state,
@@ -464,14 +509,14 @@ m3_status m3_step_bcnorm(const m3_dims *d, const m3_bcnorm *bcn, const void *x, 
 
 m3_status step_impl(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const void *B, const void *C,
                     const void *dt, const void *lam, const void *theta, const float *A, const float *D,
-                    const m3_state *state, void *y, void *stream) {
+                    const m3_state *state, void *y, void *stream, const m3_mimo_proj *proj) {
     try {
         m3_status s = check_dims(d, true);
         if (s != M3_OK) return s;
         const int64_t tok = d->batch * d->nheads;
         Range ins[8], yr;
         int nin = 0;
-        s = check_tensors(d, tok, x, B, C, dt, lam, theta, A, D, y, ins, &nin, &yr);
+        s = check_tensors(d, tok, x, B, C, dt, lam, theta, A, D, y, ins, &nin, &yr, proj != nullptr);
         if (s != M3_OK) return s;
         if (!state) return fail(M3_ERR_INVALID_ARG, "state is required");
         Range sr[3];
@@ -482,8 +527,10 @@ m3_status step_impl(const m3_dims *d, const m3_bcnorm *bcn, const void *x, const
                 if (overlap(sr[i], ins[j])) return fail(M3_ERR_INVALID_ARG, "state overlaps an input tensor");
         }
         if (bcn && (s = check_bcnorm(d, bcn, yr)) != M3_OK) return s;
+        if (proj && (s = check_proj(d, proj, yr)) != M3_OK) return s;
         m3::Problem p = make_problem(d, x, B, C, dt, lam, theta, A, D, y, stream);
         if (bcn) { p.wB = bcn->wB; p.wC = bcn->wC; p.bB = bcn->bB; p.bC = bcn->bC; p.eps = bcn->eps; }
+        if (proj) { p.pwx = proj->wx; p.pwB = proj->wB; p.pwC = proj->wC; p.pwy = proj->wy; }
         p.T = 1;
         p.hT = state->h; p.bpT = state->b_prev; p.xpT = state->x_prev;
         const char *why = nullptr;

@@ -38,6 +38,7 @@ enum : unsigned {
     kSiteState = 0x405,    // the state h
     kSitePend = 0x406,     // b_prev, x_prev
     kSiteY = 0x407,        // output
+    kSiteProj = 0x408,     // MIMO projection weights
 };
 
 // Element i of a buffer of n elements (the bounds build checks i and reads 0
@@ -84,6 +85,9 @@ struct StepFeat {
     int th_head;  // theta is [H, N/2] (fixed per head)
     const float *wB, *wC, *bB, *bC;  // BC-norm prologue (wB == nullptr: off)
     float eps;
+    // MIMO projections (pwx == nullptr: off): x, B, C, y hold one row per
+    // slice; wx, wy [H, R, P] and wB, wC [H, R, N] widen them to rank R
+    const float *pwx, *pwB, *pwC, *pwy;
 };
 
 // Register-tiled kernel for the common sizes.  Each thread owns PT pairs x 4
@@ -138,15 +142,25 @@ step_kernel(const StepArgs<IO> a, const StepFeat f) {
     const float dtv = ldv(a.dt, bh, a.BH, kSiteScalars), lamv = ldv(a.lam, bh, a.BH, kSiteScalars);
     const float alpha = __expf(dtv * ldf(a.A, (GEN && f.a_tok) ? bh : h, (GEN && f.a_tok) ? a.BH : a.H, kSiteScalars));
     const float gam = lamv * dtv, betap = (1.f - lamv) * dtv;
-    // ---- stage the slice's small vectors
+    // ---- stage the slice's small vectors (with the MIMO projections: the
+    //      slice's one row of B, C and x, widened to its R rows)
+    const bool proj = GEN && f.pwx;
     for (int i = tid; i < R * N; i += NT) {
         (&sBp[0][0])[i] = ldf(a.bp, bh * R * N + i, nBN, kSitePend);
-        (&sB[0][0])[i] = ldv(a.B, bh * R * N + i, nBN, kSiteVec);
-        (&sC[0][0])[i] = ldv(a.C, bh * R * N + i, nBN, kSiteVec);
+        if (proj) {
+            const int64_t w = h * R * N + i, v = bh * N + i % N;
+            (&sB[0][0])[i] = ldf(f.pwB, w, a.H * R * N, kSiteProj) * ldv(a.B, v, a.BH * N, kSiteVec);
+            (&sC[0][0])[i] = ldf(f.pwC, w, a.H * R * N, kSiteProj) * ldv(a.C, v, a.BH * N, kSiteVec);
+        } else {
+            (&sB[0][0])[i] = ldv(a.B, bh * R * N + i, nBN, kSiteVec);
+            (&sC[0][0])[i] = ldv(a.C, bh * R * N + i, nBN, kSiteVec);
+        }
     }
     for (int i = tid; i < R * P; i += NT) {
         (&sXp[0][0])[i] = ldf(a.xp, bh * R * P + i, nBP, kSitePend);
-        (&sX[0][0])[i] = ldv(a.x, bh * R * P + i, nBP, kSiteVec);
+        (&sX[0][0])[i] = proj ? ldf(f.pwx, h * R * P + i, a.H * R * P, kSiteProj) *
+                                    ldv(a.x, bh * P + i % P, a.BH * P, kSiteVec)
+                              : ldv(a.x, bh * R * P + i, nBP, kSiteVec);
     }
     for (int k = tid; k < K2; k += NT) {
         float sn, cs;
@@ -235,14 +249,28 @@ step_kernel(const StepArgs<IO> a, const StepFeat f) {
     }
     __syncthreads();
     const float Dh = ldf(a.D, h, a.H, kSiteScalars);
-    for (int idx = tid; idx < R * P; idx += NT) {
-        const int r = idx / P, p = idx % P;
-        float s = 0.f;
+    if (proj) {  // y = sum over the R rows of wy_r times the row
+        for (int p = tid; p < P; p += NT) {
+            float acc = 0.f;
+            for (int r = 0; r < R; ++r) {
+                float s = 0.f;
 #pragma unroll
-        for (int w = 0; w < Cfg::WARPS; ++w) s += ypart[w][r][p];
-        const float xval = sX[r][p];
-        stv(a.y, (bh * R + r) * P + p, nBP, kSiteY, s + Dh * xval);
-        stv(a.xp, (bh * R + r) * P + p, nBP, kSitePend, xval);
+                for (int w = 0; w < Cfg::WARPS; ++w) s += ypart[w][r][p];
+                acc = fmaf(ldf(f.pwy, (h * R + r) * P + p, a.H * R * P, kSiteProj), s + Dh * sX[r][p], acc);
+            }
+            stv(a.y, bh * P + p, a.BH * P, kSiteY, acc);
+        }
+        for (int idx = tid; idx < R * P; idx += NT) stv(a.xp, bh * R * P + idx, nBP, kSitePend, (&sX[0][0])[idx]);
+    } else {
+        for (int idx = tid; idx < R * P; idx += NT) {
+            const int r = idx / P, p = idx % P;
+            float s = 0.f;
+#pragma unroll
+            for (int w = 0; w < Cfg::WARPS; ++w) s += ypart[w][r][p];
+            const float xval = sX[r][p];
+            stv(a.y, (bh * R + r) * P + p, nBP, kSiteY, s + Dh * xval);
+            stv(a.xp, (bh * R + r) * P + p, nBP, kSitePend, xval);
+        }
     }
     for (int i = tid; i < R * N; i += NT) stv(a.bp, bh * R * N + i, nBN, kSitePend, (&sB[0][0])[i]);
 }
@@ -585,7 +613,7 @@ cudaError_t dispatch_np(const StepArgs<IO> &a, const StepFeat &f, cudaStream_t s
     // rank 1: one CTA per slice (measured faster); rank >= 2: the persistent
     // streaming kernel (its heavier per-element work overlaps the next slice's load)
     // (BC-norm: the tiled kernel, which normalises its staged rows in place)
-    const bool tiled = R == 1 || f.wB;
+    const bool tiled = R == 1 || f.wB || f.pwx;
     if (a.N == 128 && a.P == 64)
         return tiled ? launch_tiled<128, 64, R, IO, GEN>(a, f, s) : launch_stream<128, 64, R, IO, GEN>(a, f, s);
     if (a.N == 64 && a.P == 64)
@@ -609,16 +637,18 @@ cudaError_t launch_typed(const Problem &p) {
     f.a_tok = p.a_tok;
     f.th_head = p.th_head;
     f.wB = p.wB; f.wC = p.wC; f.bB = p.bB; f.bC = p.bC; f.eps = p.eps;
+    f.pwx = p.pwx; f.pwB = p.pwB; f.pwC = p.pwC; f.pwy = p.pwy;
     a.h = p.hT; a.bp = p.bpT; a.xp = p.xpT;
     a.y = (IO *)p.y;
     if (a.BH == 0) return cudaSuccess;
     bool done = false;
     cudaError_t e = cudaSuccess;
-    const bool gen = f.a_tok || f.th_head || f.wB;  // any optional feature on
+    const bool gen = f.a_tok || f.th_head || f.wB || f.pwx;  // any optional feature on
     if (a.R == 1) e = gen ? dispatch_np<IO, 1, true>(a, f, p.stream, &done) : dispatch_np<IO, 1, false>(a, f, p.stream, &done);
     else if (a.R == 2) e = gen ? dispatch_np<IO, 2, true>(a, f, p.stream, &done) : dispatch_np<IO, 2, false>(a, f, p.stream, &done);
     else if (a.R == 4) e = gen ? dispatch_np<IO, 4, true>(a, f, p.stream, &done) : dispatch_np<IO, 4, false>(a, f, p.stream, &done);
     if (done) return e;
+    if (f.pwx) return cudaErrorNotSupported;  // the MIMO projections: the tiled sizes only
     const size_t smem = sizeof(float) * ((size_t)a.R * a.P + (f.wB ? 2 * (size_t)a.R * a.N : 0));
     step_generic_kernel<IO><<<(unsigned)a.BH, 256, smem, p.stream>>>(a, f);
     return cudaGetLastError();
@@ -626,8 +656,12 @@ cudaError_t launch_typed(const Problem &p) {
 
 }  // namespace
 
-cudaError_t launch_step(const Problem &p, const char **) {
-    return p.bf16 ? launch_typed<__nv_bfloat16>(p) : launch_typed<float>(p);
+cudaError_t launch_step(const Problem &p, const char **why) {
+    const cudaError_t e = p.bf16 ? launch_typed<__nv_bfloat16>(p) : launch_typed<float>(p);
+    if (e == cudaErrorNotSupported)
+        *why = "decode step with the MIMO projections: (dstate, headdim) in {(64|128, 64|128), (256, 64)} and "
+               "rank 1, 2 or 4 only";
+    return e;
 }
 
 cudaError_t read_decode_error(unsigned *code) {

@@ -16,6 +16,9 @@ struct Problem {
     bool th_head;                 // theta fixed per head ([H,N/2]) instead of per token-head
     const float *wB, *wC, *bB, *bC;  // BC-norm prologue (wB == nullptr: off)
     float eps;
+    // MIMO projections (pwx == nullptr: off): x, B, C, y hold one row per
+    // token-head; wx, wy [H, R, P] and wB, wC [H, R, N] widen them to rank R
+    const float *pwx, *pwB, *pwC, *pwy;
     const void *x, *B, *C, *dt, *lam, *theta;
     const float *A, *D;
     const float *h0, *bp0, *xp0;  // nullable (zero initial state)

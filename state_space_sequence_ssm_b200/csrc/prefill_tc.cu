@@ -116,9 +116,12 @@ struct Cfg {
     // kNX buffers of {cAl2, gam, ghat, colf}[Q] + {cos, sin}[K2] (read by the
     // state warpgroup a chunk later) + {wst, dts}[Q] + phis[NPART][K2] + wtot[16]
     static constexpr uint32_t SB = 4 * Q + 2 * K2;
-    // + the BC-norm biases of this head as bf16 pairs [2][R][K2] and the row
-    // scales of the chunk's B and C tiles [2][128]
-    static constexpr uint32_t SCAL_FLOATS = kNX * SB + 2 * Q + NPART * K2 + 16 + 2 * R * K2 + 2 * kRows;
+    // + the BC-norm biases of this head as bf16 pairs [2][R][K2] (with the
+    // MIMO projections: the B and C weights) and the row scales of the chunk's
+    // B and C tiles [2][128], + the MIMO projections' x weights as bf16 pairs
+    // [R][P/2] and y weights [R][P]
+    static constexpr uint32_t SCAL_FLOATS =
+        kNX * SB + 2 * Q + NPART * K2 + 16 + 2 * R * K2 + 2 * kRows + R * kP / 2 + R * kP;
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
     static constexpr uint32_t NBARS = 20;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
@@ -139,6 +142,9 @@ struct TcArgs {
     int th_head;         // theta fixed per head, [H, N/2]
     const float *wB, *wC, *bB, *bC;  // BC-norm prologue (BCN instantiations)
     float eps;
+    // MIMO projections (PROJ instantiations): x, B, C and y hold one row per
+    // token-head; wx, wy [H, R, P] and wB, wC [H, R, N] widen them to rank R
+    const float *pwx, *pwB, *pwC, *pwy;
     __nv_bfloat16 *y;
     float *hT, *bpT, *xpT;
     // Split sequences: ws_h [nseg][BH][N][P] fp32 holds in slot j + 1 the
@@ -348,12 +354,17 @@ enum : unsigned {
     kSiteInit = 0x108,     // initial state h0, b_prev, x_prev
     kSiteY = 0x109,        // output rows
     kSiteFinal = 0x10a,    // final state and the last token's B and x
+    kSiteProj = 0x10b,     // MIMO projection weights
 };
 
 // GEN = false: the plain method (A per head, theta per token), compiled
 // without the optional features' branches; GEN = true reads A_tok and th_head
-// from the arguments.  BCN: the BC-norm prologue (only with GEN).
-template <int N, int R, int MODE, bool GEN, bool BCN>
+// from the arguments.  BCN: the BC-norm prologue (only with GEN).  PROJ: the
+// MIMO projections (only with GEN, not with BCN): the tile loads bring one
+// row per token, the prologue widens B, C and x to the R rows of each token
+// in shared memory, and the epilogue sums each token's R output rows with
+// the y weights into one row.
+template <int N, int R, int MODE, bool GEN, bool BCN, bool PROJ = false>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmT,
@@ -379,6 +390,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     float *wtot = phis + NPART * K2;
     uint32_t *sbias = reinterpret_cast<uint32_t *>(wtot + 16);  // BC-norm biases [B, C][R][K2] (bf16 pairs)
     float *rsc = reinterpret_cast<float *>(sbias + 2 * R * C::K2);  // BC-norm row scales [B, C][128]
+    uint32_t *sxw = reinterpret_cast<uint32_t *>(rsc + 2 * kRows);  // projections: x weights [R][P/2] (bf16 pairs)
+    float *swy = reinterpret_cast<float *>(sxw + R * kP / 2);        // projections: y weights [R][P]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     Bars bb{bars, bars + 2, bars + 4, bars + 7, bars + 10, bars + 11, bars + 12, bars + 13, bars + 14, bars + 15,
             bars + 16, bars + 19};
@@ -468,7 +481,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (i >= 2 && !mbar_wait(&bb.empty_bc[s], ((i >> 1) - 1) & 1, abort_flag, err, kErrWaitMma)) break;
                 uint8_t *st = smem + C::OFF_BC + s * C::BCS_BYTES;
                 const int t0 = (cb + i) * Q;
-                mbar_arrive_expect_tx(&bb.full_bc[s], SUM ? C::BC_BYTES : C::BCS_BYTES);
+                // (with the projections a tile load brings one row per token)
+                mbar_arrive_expect_tx(&bb.full_bc[s], (SUM ? C::BC_BYTES : C::BCS_BYTES) / (PROJ ? R : 1));
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
                     tma_load_5d(st + kb * 16384, &tmB, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
@@ -490,7 +504,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const int s = i % kNX;
                 if (i >= kNX && !mbar_wait(&bb.empty_x[s], ((i / kNX) - 1) & 1, abort_flag, err, kErrWaitCompute))
                     break;
-                mbar_arrive_expect_tx(&bb.full_x[s], C::X_BYTES);
+                mbar_arrive_expect_tx(&bb.full_x[s], C::X_BYTES / (PROJ ? R : 1));
                 tma_load_5d(smem + C::OFF_X + s * C::X_BYTES, &tmX, &bb.full_x[s], 0, 0, (int)h, (cb + i) * Q,
                             (int)b);
                 issued = i + 1;
@@ -619,6 +633,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 sbias[i] = dchk::in(kSiteNorm, o, 2, H * R * N) ? pack_bf16(src[0], src[1]) : 0u;
             }
         }
+        if (PROJ) {  // the head's projection weights: B, C and x as bf16 pairs, y in fp32
+            for (int i = tid; i < 2 * R * K2; i += kPro) {
+                const int which = i / (R * K2), rk = i % (R * K2);
+                const int64_t o = (h * R + rk / K2) * N + 2 * (rk % K2);
+                const float *src = (which ? a.pwC : a.pwB) + o;
+                sbias[i] = dchk::in(kSiteProj, o, 2, H * R * N) ? pack_bf16(src[0], src[1]) : 0u;
+            }
+            for (int i = tid; i < R * kP / 2; i += kPro) {
+                const int64_t o = h * R * kP + 2 * i;
+                sxw[i] = dchk::in(kSiteProj, o, 2, H * R * kP) ? pack_bf16(a.pwx[o], a.pwx[o + 1]) : 0u;
+            }
+            for (int i = tid; i < R * kP; i += kPro)
+                swy[i] = dchk::in(kSiteProj, h * R * kP + i, 1, H * R * kP) ? a.pwy[h * R * kP + i] : 0.f;
+        }
         // angle rates fixed per head: the thread's 4 pairs, for the whole sequence
         float thh[4] = {0.f, 0.f, 0.f, 0.f};
         if (th_head) {
@@ -740,6 +768,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
                 const uint32_t kbo = (uint32_t)(g >> 3) * 16384u;
                 const uint32_t jchunk = (uint32_t)(g & 7);
+                // MIMO projections: the tiles hold one row per token (row i);
+                // for R > 1 every thread first takes its tokens' rows into
+                // registers, since the widened rows i R + r overwrite rows of
+                // other threads' tokens
+                constexpr bool kStage = PROJ && R > 1;
+                uint4 pb[kStage ? TPT : 1], pc[kStage ? TPT : 1];
+                if (kStage) {
+#pragma unroll
+                    for (int j = 0; j < TPT; ++j) {
+                        const uint32_t off = kbo + sw128((uint32_t)(part * TPT + j), jchunk);
+                        pb[j] = *reinterpret_cast<const uint4 *>(bst + off);
+                        if (!SUM) pc[j] = *reinterpret_cast<const uint4 *>(cst + off);
+                    }
+                    named_bar(kBarPro, kPro);
+                }
 #pragma unroll
                 for (int j0 = 0; j0 < TPT; j0 += TB) {
                     // all loads of the batch first (the stores below go to the same
@@ -750,6 +793,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         const int i = part * TPT + j0 + jj;
 #pragma unroll
                         for (int r = 0; r < R; ++r) {
+                            if (PROJ) {  // widen: this rank's weights times the token's row
+                                const uint4 src = kStage ? pb[j0 + jj]
+                                                         : *reinterpret_cast<const uint4 *>(
+                                                               bst + kbo + sw128((uint32_t)i, jchunk));
+                                const uint4 w = *reinterpret_cast<const uint4 *>(sbias + r * K2 + 4 * g);
+                                vb[jj][r] = make_uint4(mul_bf16x2(src.x, w.x), mul_bf16x2(src.y, w.y),
+                                                       mul_bf16x2(src.z, w.z), mul_bf16x2(src.w, w.w));
+                                if (!SUM) {
+                                    const uint4 srcc = kStage ? pc[j0 + jj]
+                                                              : *reinterpret_cast<const uint4 *>(
+                                                                    cst + kbo + sw128((uint32_t)i, jchunk));
+                                    const uint4 wc = *reinterpret_cast<const uint4 *>(sbias + (R + r) * K2 + 4 * g);
+                                    vc[jj][r] = make_uint4(mul_bf16x2(srcc.x, wc.x), mul_bf16x2(srcc.y, wc.y),
+                                                           mul_bf16x2(srcc.z, wc.z), mul_bf16x2(srcc.w, wc.w));
+                                }
+                                continue;
+                            }
                             const uint32_t off = kbo + sw128((uint32_t)(i * R + r), jchunk);
                             vb[jj][r] = *reinterpret_cast<const uint4 *>(bst + off);
                             if (!SUM) vc[jj][r] = *reinterpret_cast<const uint4 *>(cst + off);
@@ -833,8 +893,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const float wv = wst[row / R];
                 const uint32_t ww = pack_bf16(wv, wv);
                 uint4 v[4];
+                if (PROJ) {  // the x tile holds one row per token: widen it into rows i R + r
 #pragma unroll
-                for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4 *>(xst + sw128(row, j0 + j));
+                    for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4 *>(xst + sw128(row / R, j0 + j));
+                    if (R > 1) named_bar(kBarPro, kPro);  // every token's row read before any is overwritten
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(sxw + (row % R) * (kP / 2) + 4 * (j0 + j));
+                        v[j] = make_uint4(mul_bf16x2(v[j].x, w.x), mul_bf16x2(v[j].y, w.y), mul_bf16x2(v[j].z, w.z),
+                                          mul_bf16x2(v[j].w, w.w));
+                        *reinterpret_cast<uint4 *>(xst + sw128(row, j0 + j)) = v[j];
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4 *>(xst + sw128(row, j0 + j));
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     v[j].x = mul_bf16x2(v[j].x, ww);
@@ -1055,6 +1128,39 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     tmem_ld16(tl + kColYd + c0 + 16 * qq, yd);
                     tmem_ld16(tl + yo + c0 + 16 * qq, yv);
                     tmem_wait_ld();
+                    if (PROJ) {  // y of the token = sum over its R rows (R neighbouring lanes) of wy_r times the row
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const uint4 xv =
+                                *reinterpret_cast<const uint4 *>(xst + sw128(row, (c0 >> 3) + 2 * qq + q));
+                            const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+                            const float4 w0 = *reinterpret_cast<const float4 *>(swy + r * kP + c0 + 16 * qq + 8 * q);
+                            const float4 w1 =
+                                *reinterpret_cast<const float4 *>(swy + r * kP + c0 + 16 * qq + 8 * q + 4);
+                            const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 xf = unpack_bf16(xs[e]);
+                                const int p = 8 * q + 2 * e;
+                                yd[p] = w[2 * e] * fmaf(Dh, xf.x, fmaf(sc, yv[p], yd[p]));
+                                yd[p + 1] = w[2 * e + 1] * fmaf(Dh, xf.y, fmaf(sc, yv[p + 1], yd[p + 1]));
+                            }
+                        }
+#pragma unroll
+                        for (int off = 1; off < R; off <<= 1)
+#pragma unroll
+                            for (int p = 0; p < 16; ++p) yd[p] += __shfl_xor_sync(0xffffffffu, yd[p], off);
+                        if (r == 0 && t < T && dchk::in(kSiteY, tok(t) * kP + c0 + 16 * qq, 16, nTok * kP)) {
+                            __nv_bfloat16 *yrow = a.y + tok(t) * kP + c0 + 16 * qq;
+#pragma unroll
+                            for (int q = 0; q < 2; ++q)
+                                *reinterpret_cast<uint4 *>(yrow + 8 * q) =
+                                    make_uint4(pack_bf16(yd[8 * q], yd[8 * q + 1]), pack_bf16(yd[8 * q + 2], yd[8 * q + 3]),
+                                               pack_bf16(yd[8 * q + 4], yd[8 * q + 5]),
+                                               pack_bf16(yd[8 * q + 6], yd[8 * q + 7]));
+                        }
+                        continue;
+                    }
                     if (t < T && dchk::in(kSiteY, (tok(t) * R + r) * kP + c0 + 16 * qq, 16, nTok * R * kP)) {
                         __nv_bfloat16 *yrow = a.y + (tok(t) * R + r) * kP + c0 + 16 * qq;
 #pragma unroll
@@ -1126,13 +1232,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     for (int n = lane; n < N; n += 32)
                         a.bpT[(bh * R + wl) * N + n] = fmaf(bf(a.B, src + n) * sc, a.wB[n], a.bB[(h * R + wl) * N + n]);
                 }
+            } else if (PROJ) {  // the last token's B and x, widened to rank R
+                if (a.bpT && dchk::in(kSiteFinal, tok(T - 1) * N, N, nTok * N) &&
+                    dchk::in(kSiteFinal, bh * R * N, R * N, (int64_t)a.BH * R * N) &&
+                    dchk::in(kSiteProj, h * R * N, R * N, H * R * N))
+                    for (int i = lt; i < R * N; i += kSt)
+                        a.bpT[bh * R * N + i] = a.pwB[h * R * N + i] * bf(a.B, tok(T - 1) * N + i % N);
             } else if (a.bpT && dchk::in(kSiteFinal, tok(T - 1) * R * N, R * N, nTok * R * N) &&
                        dchk::in(kSiteFinal, bh * R * N, R * N, (int64_t)a.BH * R * N)) {
                 for (int i = lt; i < R * N; i += kSt) a.bpT[bh * R * N + i] = bf(a.B, tok(T - 1) * R * N + i);
             }
-            if (a.xpT && dchk::in(kSiteFinal, tok(T - 1) * R * kP, R * kP, nTok * R * kP) &&
-                dchk::in(kSiteFinal, bh * R * kP, R * kP, (int64_t)a.BH * R * kP))
+            if (PROJ) {
+                if (a.xpT && dchk::in(kSiteFinal, tok(T - 1) * kP, kP, nTok * kP) &&
+                    dchk::in(kSiteFinal, bh * R * kP, R * kP, (int64_t)a.BH * R * kP) &&
+                    dchk::in(kSiteProj, h * R * kP, R * kP, H * R * kP))
+                    for (int i = lt; i < R * kP; i += kSt)
+                        a.xpT[bh * R * kP + i] = a.pwx[h * R * kP + i] * bf(a.x, tok(T - 1) * kP + i % kP);
+            } else if (a.xpT && dchk::in(kSiteFinal, tok(T - 1) * R * kP, R * kP, nTok * R * kP) &&
+                       dchk::in(kSiteFinal, bh * R * kP, R * kP, (int64_t)a.BH * R * kP)) {
                 for (int i = lt; i < R * kP; i += kSt) a.xpT[bh * R * kP + i] = bf(a.x, tok(T - 1) * R * kP + i);
+            }
         }
     }
     __syncwarp();  // reconverge the single-lane roles before the block barrier
@@ -1197,11 +1316,11 @@ bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int
 
 // `dependent`: launched as a programmatic dependent of the previous kernel on
 // the stream (the main pass of a split sequence after its summary pass).
-template <int N, int R, int MODE, bool GEN, bool BCN>
+template <int N, int R, int MODE, bool GEN, bool BCN, bool PROJ>
 cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc, const CUtensorMap &mt,
                         const TcArgs &a, int64_t ctas, cudaStream_t stream, bool dependent = false) {
     using C = Cfg<N, R>;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, GEN, BCN>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, GEN, BCN, PROJ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
@@ -1214,18 +1333,20 @@ cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUte
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = dependent ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<N, R, MODE, GEN, BCN>, mx, mb, mc, mt, a);
+    e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<N, R, MODE, GEN, BCN, PROJ>, mx, mb, mc, mt, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-template <int N, int R, bool GEN, bool BCN>
+template <int N, int R, bool GEN, bool BCN, bool PROJ = false>
 cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     using C = Cfg<N, R>;
     CUtensorMap mx, mb, mc, mt;
-    // (theta fixed per head: a valid map over [H, N/2] that the kernel never loads from)
-    if (!make_map(&mx, p.x, kP, R, p.H, p.T, p.Bt, C::Q) || !make_map(&mb, p.B, N, R, p.H, p.T, p.Bt, C::Q) ||
-        !make_map(&mc, p.C, N, R, p.H, p.T, p.Bt, C::Q) ||
+    // (theta fixed per head: a valid map over [H, N/2] that the kernel never loads from;
+    // with the MIMO projections x, B, C have one row per token-head)
+    constexpr int RIO = PROJ ? 1 : R;
+    if (!make_map(&mx, p.x, kP, RIO, p.H, p.T, p.Bt, C::Q) || !make_map(&mb, p.B, N, RIO, p.H, p.T, p.Bt, C::Q) ||
+        !make_map(&mc, p.C, N, RIO, p.H, p.T, p.Bt, C::Q) ||
         !make_theta_map(&mt, p.theta, N / 2, p.H, p.th_head ? 1 : p.T, p.th_head ? 1 : p.Bt, p.th_head ? 1 : C::Q)) {
         *why = "tensor-core prefill: TMA descriptor encoding failed";
         return cudaErrorNotSupported;
@@ -1251,6 +1372,10 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     a.bB = p.bB;
     a.bC = p.bC;
     a.eps = p.eps;
+    a.pwx = p.pwx;
+    a.pwB = p.pwB;
+    a.pwC = p.pwC;
+    a.pwy = p.pwy;
     a.D = p.D;
     a.h0 = p.h0;
     a.bp0 = p.bp0;
@@ -1260,7 +1385,7 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
         a.hT = p.hT;
         a.bpT = p.bpT;
         a.xpT = p.xpT;
-        return launch_pass<N, R, kWhole, GEN, BCN>(mx, mb, mc, mt, a, BH, p.stream);
+        return launch_pass<N, R, kWhole, GEN, BCN, PROJ>(mx, mb, mc, mt, a, BH, p.stream);
     }
     // split sequences: the summary pass over segments 0 .. nseg-2 publishes
     // each segment's local end state and transition; the main pass over all
@@ -1274,14 +1399,15 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     // (the failure-path self-test leaves the summary pass out: its flags are
     // never published and the look-back waits give up)
     if (!p.skip_summary) {
-        e = launch_pass<N, R, kSummary, GEN, BCN>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
+        e = launch_pass<N, R, kSummary, GEN, BCN, PROJ>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
         if (e != cudaSuccess) return e;
     }
     a.y = (__nv_bfloat16 *)p.y;
     a.hT = p.hT;
     a.bpT = p.bpT;
     a.xpT = p.xpT;
-    return launch_pass<N, R, kSegment, GEN, BCN>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream, !p.skip_summary);
+    return launch_pass<N, R, kSegment, GEN, BCN, PROJ>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream,
+                                                       !p.skip_summary);
 }
 
 bool device_is_sm100() {
@@ -1380,7 +1506,17 @@ cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
         return cudaErrorNotSupported;
     }
     // plain instantiations unless an optional feature is on
-    const bool gen = p.a_tok || p.th_head || p.wB;
+    const bool gen = p.a_tok || p.th_head || p.wB || p.pwx;
+    if (p.pwx) {  // MIMO projections (never with the BC-norm prologue)
+        if (p.N == 128) {
+            if (p.R == 1) return launch_nr<128, 1, true, false, true>(p, plan, why);
+            if (p.R == 2) return launch_nr<128, 2, true, false, true>(p, plan, why);
+            return launch_nr<128, 4, true, false, true>(p, plan, why);
+        }
+        if (p.R == 1) return launch_nr<64, 1, true, false, true>(p, plan, why);
+        if (p.R == 2) return launch_nr<64, 2, true, false, true>(p, plan, why);
+        return launch_nr<64, 4, true, false, true>(p, plan, why);
+    }
     if (p.wB) {
         if (p.N == 128) {
             if (p.R == 1) return launch_nr<128, 1, true, true>(p, plan, why);
