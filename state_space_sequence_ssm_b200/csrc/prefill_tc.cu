@@ -360,7 +360,7 @@ enum : unsigned {
 // GEN = false: the plain method (A per head, theta per token), compiled
 // without the optional features' branches; GEN = true reads A_tok and th_head
 // from the arguments.  BCN: the BC-norm prologue (only with GEN).  PROJ: the
-// MIMO projections (only with GEN, not with BCN): the tile loads bring one
+// MIMO projections (not with BCN): the tile loads bring one
 // row per token, the prologue widens B, C and x to the R rows of each token
 // in shared memory, and the epilogue sums each token's R output rows with
 // the y weights into one row.
@@ -1146,18 +1146,38 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                                 yd[p + 1] = w[2 * e + 1] * fmaf(Dh, xf.y, fmaf(sc, yv[p + 1], yd[p + 1]));
                             }
                         }
+                        // reduce-scatter over the R lanes of the token: at each
+                        // halving step a lane keeps half of its columns and adds
+                        // the partner's copy of them; lane r ends with the sums
+                        // of 16 / R columns, at offset cofs
+                        int cofs = 0;
 #pragma unroll
-                        for (int off = 1; off < R; off <<= 1)
+                        for (int half = 8, bit = R / 2; bit >= 1; half >>= 1, bit >>= 1) {
+                            const bool up = (r & bit) != 0;
 #pragma unroll
-                            for (int p = 0; p < 16; ++p) yd[p] += __shfl_xor_sync(0xffffffffu, yd[p], off);
-                        if (r == 0 && t < T && dchk::in(kSiteY, tok(t) * kP + c0 + 16 * qq, 16, nTok * kP)) {
-                            __nv_bfloat16 *yrow = a.y + tok(t) * kP + c0 + 16 * qq;
+                            for (int k = 0; k < half; ++k) {
+                                const float mine = up ? yd[k + half] : yd[k];
+                                const float other = __shfl_xor_sync(0xffffffffu, up ? yd[k] : yd[k + half], bit);
+                                yd[k] = mine + other;
+                            }
+                            cofs += up ? half : 0;
+                        }
+                        constexpr int kOut = 16 / R;  // columns stored by each lane
+                        if (t < T && dchk::in(kSiteY, tok(t) * kP + c0 + 16 * qq + cofs, kOut, nTok * kP)) {
+                            __nv_bfloat16 *yp = a.y + tok(t) * kP + c0 + 16 * qq + cofs;
+                            if (kOut == 16) {
 #pragma unroll
-                            for (int q = 0; q < 2; ++q)
-                                *reinterpret_cast<uint4 *>(yrow + 8 * q) =
-                                    make_uint4(pack_bf16(yd[8 * q], yd[8 * q + 1]), pack_bf16(yd[8 * q + 2], yd[8 * q + 3]),
-                                               pack_bf16(yd[8 * q + 4], yd[8 * q + 5]),
-                                               pack_bf16(yd[8 * q + 6], yd[8 * q + 7]));
+                                for (int q = 0; q < 2; ++q)
+                                    *reinterpret_cast<uint4 *>(yp + 8 * q) = make_uint4(
+                                        pack_bf16(yd[8 * q], yd[8 * q + 1]), pack_bf16(yd[8 * q + 2], yd[8 * q + 3]),
+                                        pack_bf16(yd[8 * q + 4], yd[8 * q + 5]), pack_bf16(yd[8 * q + 6], yd[8 * q + 7]));
+                            } else if (kOut == 8) {
+                                *reinterpret_cast<uint4 *>(yp) =
+                                    make_uint4(pack_bf16(yd[0], yd[1]), pack_bf16(yd[2], yd[3]), pack_bf16(yd[4], yd[5]),
+                                               pack_bf16(yd[6], yd[7]));
+                            } else {
+                                *reinterpret_cast<uint2 *>(yp) = make_uint2(pack_bf16(yd[0], yd[1]), pack_bf16(yd[2], yd[3]));
+                            }
                         }
                         continue;
                     }
@@ -1507,15 +1527,21 @@ cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
     }
     // plain instantiations unless an optional feature is on
     const bool gen = p.a_tok || p.th_head || p.wB || p.pwx;
-    if (p.pwx) {  // MIMO projections (never with the BC-norm prologue)
+    if (p.pwx) {  // MIMO projections (never with the BC-norm prologue); plain unless A_t or theta per head
+        const bool g2 = p.a_tok || p.th_head;
         if (p.N == 128) {
-            if (p.R == 1) return launch_nr<128, 1, true, false, true>(p, plan, why);
-            if (p.R == 2) return launch_nr<128, 2, true, false, true>(p, plan, why);
-            return launch_nr<128, 4, true, false, true>(p, plan, why);
+            if (p.R == 1) return g2 ? launch_nr<128, 1, true, false, true>(p, plan, why)
+                                    : launch_nr<128, 1, false, false, true>(p, plan, why);
+            if (p.R == 2) return g2 ? launch_nr<128, 2, true, false, true>(p, plan, why)
+                                    : launch_nr<128, 2, false, false, true>(p, plan, why);
+            return g2 ? launch_nr<128, 4, true, false, true>(p, plan, why)
+                      : launch_nr<128, 4, false, false, true>(p, plan, why);
         }
-        if (p.R == 1) return launch_nr<64, 1, true, false, true>(p, plan, why);
-        if (p.R == 2) return launch_nr<64, 2, true, false, true>(p, plan, why);
-        return launch_nr<64, 4, true, false, true>(p, plan, why);
+        if (p.R == 1) return g2 ? launch_nr<64, 1, true, false, true>(p, plan, why)
+                                : launch_nr<64, 1, false, false, true>(p, plan, why);
+        if (p.R == 2) return g2 ? launch_nr<64, 2, true, false, true>(p, plan, why)
+                                : launch_nr<64, 2, false, false, true>(p, plan, why);
+        return g2 ? launch_nr<64, 4, true, false, true>(p, plan, why) : launch_nr<64, 4, false, false, true>(p, plan, why);
     }
     if (p.wB) {
         if (p.N == 128) {
