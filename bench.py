@@ -65,7 +65,7 @@ def parse():
                     help="skip the variant lines (per-token A, per-head theta, BC-norm) of the prefill workload")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads' lines (small fp32 scan, MIMO, decode, long context)")
-    ap.add_argument("--case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--case", choices=["prefill", "prefill_proj", "decode"], default=None,
                     help="profiling case: only run --case-launches launches of one kernel at --case-batch "
                          "(for ncu captures; prints no bench line)")
     ap.add_argument("--case-batch", type=int, default=None, help="batch of the profiling case")
@@ -86,12 +86,19 @@ def run_case(args):
     from m3_inputs import WORKLOADS, make_prefill, make_state, make_steps
 
     keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
-    if args.case == "prefill":
+    if args.case in ("prefill", "prefill_proj"):
         s = WORKLOADS[args.workload]
         s = s.with_(batch=args.case_batch or s.batch, seqlen=args.case_seqlen or s.seqlen)
-        inp = make_prefill(s, device="cuda")
+        proj = None
+        if args.case == "prefill_proj":  # the same shape with the fused MIMO projections
+            from m3_inputs import make_prefill_proj, make_proj
+            inp = make_prefill_proj(s, device="cuda")
+            w = make_proj(s, device="cuda")
+            proj = m3.MimoProj(w["wx"], w["wB"], w["wC"], w["wy"])
+        else:
+            inp = make_prefill(s, device="cuda")
         for _ in range(args.case_launches):
-            m3.scan_fwd(*(inp[k] for k in keys), None)
+            m3.scan_fwd(*(inp[k] for k in keys), None, proj=proj)
     else:
         # a decode workload, or the long-context workload's own sequences
         name = args.workload if args.workload.startswith(("decode", "long")) else DECODE_WORKLOADS[0]
@@ -725,7 +732,8 @@ def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_p
             "value": world * K * s.batch * s.seqlen / el, "unit": "tokens/s", "steps": K,
             "ms_per_step": 1e3 * el / K, "gpu_launches": K,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
-                         "traffic": None, "kernel": "prefill_tc_kernel", "algorithmic_bytes_per_launch": ab,
+                         "traffic": recorded_traffic("prefill_tc_kernel", f"{workload}+{kind}"),
+                         "kernel": "prefill_tc_kernel", "algorithmic_bytes_per_launch": ab,
                          "peak_source": peak_src}}
 
 
