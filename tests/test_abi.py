@@ -115,6 +115,27 @@ def test_unknown_algo(m3):
     assert call_scan(m3, dims(m3), algo=9) == 1
 
 
+def call_scan_proj(m3, d, proj, algo=0, y=None):
+    p = [ctypes.c_void_p(FAKE + i * 0x100000) for i in range(8)]
+    yv = ctypes.c_void_p(y if y is not None else FAKE + 9 * 0x100000)
+    return m3.lib.m3_scan_fwd_proj(algo, ctypes.byref(d), proj, *p, None, yv, None, None, 0, None)
+
+
+def test_proj_validation_on_the_host(m3):
+    """m3_scan_fwd_proj rejects a missing or incomplete weight set, misaligned
+    weights and y overlapping a weight array, and refuses fp32 I/O and the SIMT
+    algo, all before any launch (the tensors are fake addresses)."""
+    W = FAKE + 20 * 0x100000
+    ok = m3.CMimoProj(W, W + 0x10000, W + 0x20000, W + 0x30000)
+    d = dims(m3, P=64, N=64, R=2, io=1)
+    assert call_scan_proj(m3, d, None) == 1
+    assert call_scan_proj(m3, d, ctypes.byref(m3.CMimoProj(W, None, W + 0x20000, W + 0x30000))) == 1
+    assert call_scan_proj(m3, d, ctypes.byref(m3.CMimoProj(W + 2, W + 0x10000, W + 0x20000, W + 0x30000))) == 1
+    assert call_scan_proj(m3, d, ctypes.byref(ok), y=W + 0x30000) == 1  # y over wy
+    assert call_scan_proj(m3, dims(m3, P=64, N=64, R=2, io=0), ctypes.byref(ok)) == 2
+    assert call_scan_proj(m3, d, ctypes.byref(ok), algo=1) == 2
+
+
 def test_step_validation(m3):
     d = dims(m3)
     vp = [ctypes.c_void_p(FAKE + i * 0x100000) for i in range(8)]

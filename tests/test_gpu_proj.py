@@ -149,4 +149,21 @@ def test_proj_refusals():
     with pytest.raises(m3.M3Error) as e:
         m3.scan_fwd(*(inb[k] for k in KEYS), None, proj=prb)
     assert e.value.status == m3.M3_ERR_UNSUPPORTED
+    # decode: sizes outside the register-tiled kernel (dstate 32) are refused
+    small = Shape(1, 8, 2, 64, 32, 2, "bf16", 541)
+    prs, _ = weights(small)
+    st = m3.State(*(t.to(DEV) for t in make_state(small)))
+    steps = make_steps_proj(small, 1)
+    args = [steps[k][0].contiguous().to(DEV) for k in STEP_KEYS]
+    pre = make_prefill_proj(small)
+    with pytest.raises(m3.M3Error) as e:
+        m3.step(*args, pre["A"].to(DEV), pre["D"].to(DEV), st, proj=prs)
+    assert e.value.status == m3.M3_ERR_UNSUPPORTED
+    # BC-norm and the projections together are refused
+    from m3_inputs import make_bcnorm
+    b = make_bcnorm(s, device=DEV)
+    with pytest.raises(m3.M3Error) as e:
+        m3.scan_fwd(*(inp[k] for k in KEYS), None, proj=pr,
+                    bcnorm=m3.BCNorm(b["wB"], b["wC"], b["bB"], b["bC"], b["eps"]))
+    assert e.value.status == m3.M3_ERR_UNSUPPORTED
     m3.stream_status()
