@@ -117,3 +117,26 @@ def test_split_zero_batch_is_noop():
     y, fs = m3.scan_fwd(*(inp[k] for k in KEYS), None, algo=m3.ALGO_TC_SEGMENTS(3))
     m3.stream_status()
     assert y.numel() == 0 and fs.h.numel() == 0
+
+
+def test_split_calls_on_two_streams_at_once():
+    """Two split calls queued on two streams, each with its own workspace
+    (flags included), run at the same time: each equals the same call made
+    alone (the look-back only ever reads its own call's flags and summaries)."""
+    sa = Shape(1, 1500, 2, 64, 128, 1, "bf16", 161)
+    sb = Shape(2, 900, 1, 64, 64, 4, "bf16", 162)
+    ia, ib = to_dev(make_prefill(sa)), to_dev(make_prefill(sb))
+    alg = m3.ALGO_TC_SEGMENTS(4)
+    ya_ref, fa_ref = m3.scan_fwd(*(ia[k] for k in KEYS), None, algo=alg)
+    yb_ref, fb_ref = m3.scan_fwd(*(ib[k] for k in KEYS), None, algo=alg)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            ya, fa = m3.scan_fwd(*(ia[k] for k in KEYS), None, algo=alg, stream=s1)
+        with torch.cuda.stream(s2):
+            yb, fb = m3.scan_fwd(*(ib[k] for k in KEYS), None, algo=alg, stream=s2)
+        torch.cuda.synchronize()
+        m3.stream_status()
+        assert torch.equal(ya, ya_ref) and torch.equal(fa.h, fa_ref.h)
+        assert torch.equal(yb, yb_ref) and torch.equal(fb.h, fb_ref.h)
