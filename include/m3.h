@@ -189,8 +189,9 @@ M3_API m3_status m3_scan_fwd_proj(int algo, const m3_dims *d, const m3_mimo_proj
 
 /* m3_step with the MIMO projections: x [B,H,P], B and C [B,H,N], y [B,H,P];
  * the state in the rank-R layout, updated in place (b_prev, x_prev widened).
- * The register-tiled decode sizes only ((dstate, headdim) in {64, 128} x
- * {64, 128} or (256, 64); rank 1, 2 or 4): M3_ERR_UNSUPPORTED otherwise. */
+ * The register-tiled and streaming decode sizes only ((dstate, headdim) in
+ * {64, 128} x {64, 128} or (256, 64); rank 1, 2 or 4): M3_ERR_UNSUPPORTED
+ * otherwise. */
 M3_API m3_status m3_step_proj(const m3_dims *d, const m3_mimo_proj *proj, const void *x, const void *B,
                               const void *C, const void *dt, const void *lam, const void *theta,
                               const float *A, const float *D, const m3_state *state, void *y, void *stream);

@@ -414,6 +414,11 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
     // buffer extents in elements, for the bounds build's index checks
     const int64_t nSt = BH * N * P, nBN = BH * R * N, nBP = BH * R * P;
 
+    // MIMO projections: B, C and x hold one row per slice (the copies move
+    // 1/R of the bytes), widened with the head's weights when staged
+    const bool proj = GEN && f.pwx;
+    const int RIO = proj ? 1 : R;
+    const uint32_t cB = proj ? Cfg::B_B / R : Cfg::B_B, cX = proj ? Cfg::B_X / R : Cfg::B_X;
     // the slice's copies; the bounds build checks each source range and
     // copies from the buffer's start instead of outside it (so that the
     // expected bytes still arrive)
@@ -422,16 +427,18 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
         const int64_t th = ((GEN && f.th_head) ? bh % a.H : bh) * K2;
         const int64_t nth = ((GEN && f.th_head) ? a.H : BH) * K2;
         const bool ist = dchk::in(kSiteState, bh * N * P, N * P, nSt);
-        const bool ibn = dchk::in(kSitePend, bh * R * N, R * N, nBN) && dchk::in(kSiteVec, bh * R * N, R * N, nBN);
-        const bool ibp = dchk::in(kSitePend, bh * R * P, R * P, nBP) && dchk::in(kSiteVec, bh * R * P, R * P, nBP);
+        const bool ibn = dchk::in(kSitePend, bh * R * N, R * N, nBN) &&
+                         dchk::in(kSiteVec, bh * RIO * N, RIO * N, BH * RIO * N);
+        const bool ibp = dchk::in(kSitePend, bh * R * P, R * P, nBP) &&
+                         dchk::in(kSiteVec, bh * RIO * P, RIO * P, BH * RIO * P);
         const bool ith = dchk::in(kSiteTheta, th, K2, nth);
-        tc::mbar_arrive_expect_tx(&full[st], Cfg::TX);
+        tc::mbar_arrive_expect_tx(&full[st], Cfg::TX - 2 * (Cfg::B_B - cB) - (Cfg::B_X - cX));
         tc::bulk_g2s(s, a.h + (ist ? bh * N * P : 0), Cfg::B_H, &full[st]);
         tc::bulk_g2s(s + Cfg::O_BP, a.bp + (ibn ? bh * R * N : 0), Cfg::B_BP, &full[st]);
         tc::bulk_g2s(s + Cfg::O_XP, a.xp + (ibp ? bh * R * P : 0), Cfg::B_XP, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_B, a.B + (ibn ? bh * R * N : 0), Cfg::B_B, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_C, a.C + (ibn ? bh * R * N : 0), Cfg::B_B, &full[st]);
-        tc::bulk_g2s(s + Cfg::O_X, a.x + (ibp ? bh * R * P : 0), Cfg::B_X, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_B, a.B + (ibn ? bh * RIO * N : 0), cB, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_C, a.C + (ibn ? bh * RIO * N : 0), cB, &full[st]);
+        tc::bulk_g2s(s + Cfg::O_X, a.x + (ibp ? bh * RIO * P : 0), cX, &full[st]);
         tc::bulk_g2s(s + Cfg::O_TH, a.theta + (ith ? th : 0), Cfg::B_TH, &full[st]);
     };
     if (tid == 0) {
@@ -479,15 +486,29 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
         }
         for (int i = tid; i < R * N; i += NT) {
             vBp[i] = betap * sBp[i];
-            vB[i] = gam * sv(sB, i);
-            vC[i] = sv(sC, i);
+            if (proj) {
+                const int64_t w = (int64_t)h * R * N + i;
+                vB[i] = gam * ldf(f.pwB, w, a.H * R * N, kSiteProj) * sv(sB, i % N);
+                vC[i] = ldf(f.pwC, w, a.H * R * N, kSiteProj) * sv(sC, i % N);
+            } else {
+                vB[i] = gam * sv(sB, i);
+                vC[i] = sv(sC, i);
+            }
         }
         __syncthreads();
         float4 xp[R], xv[R], yacc[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             xp[r] = *reinterpret_cast<const float4 *>(sXp + r * P + p0);
-            xv[r] = sv4(sX, r * P + p0);
+            if (proj) {
+                const float4 x4 = sv4(sX, p0);
+                const int64_t w = ((int64_t)h * R + r) * P + p0;
+                const int64_t nw = a.H * R * P;
+                xv[r] = make_float4(ldf(f.pwx, w, nw, kSiteProj) * x4.x, ldf(f.pwx, w + 1, nw, kSiteProj) * x4.y,
+                                    ldf(f.pwx, w + 2, nw, kSiteProj) * x4.z, ldf(f.pwx, w + 3, nw, kSiteProj) * x4.w);
+            } else {
+                xv[r] = sv4(sX, r * P + p0);
+            }
             yacc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         float4 *hg = reinterpret_cast<float4 *>(a.h + bh * N * P);
@@ -550,15 +571,37 @@ step_stream_kernel(const StepArgs<IO> a, const StepFeat f) {
         }
         __syncthreads();
         const float Dh = ldf(a.D, h, a.H, kSiteScalars);
-        for (int idx = tid; idx < R * P; idx += NT) {
-            float sum = 0.f;
+        if (proj) {  // y = sum over the R rows of wy_r times the row; the pending rows widened
+            const int64_t nw = a.H * R * P;
+            for (int p = tid; p < P; p += NT) {
+                float acc = 0.f;
+                for (int r = 0; r < R; ++r) {
+                    float sum = 0.f;
 #pragma unroll
-            for (int w = 0; w < Cfg::WARPS; ++w) sum += ypart[w * R * P + idx];
-            const float xval = sv(sX, idx);
-            stv(a.y, bh * R * P + idx, nBP, kSiteY, sum + Dh * xval);
-            stv(a.xp, bh * R * P + idx, nBP, kSitePend, xval);
+                    for (int w = 0; w < Cfg::WARPS; ++w) sum += ypart[w * R * P + r * P + p];
+                    const int64_t wi = ((int64_t)h * R + r) * P + p;
+                    const float xval = ldf(f.pwx, wi, nw, kSiteProj) * sv(sX, p);
+                    acc = fmaf(ldf(f.pwy, wi, nw, kSiteProj), sum + Dh * xval, acc);
+                }
+                stv(a.y, bh * P + p, BH * P, kSiteY, acc);
+            }
+            for (int idx = tid; idx < R * P; idx += NT)
+                stv(a.xp, bh * R * P + idx, nBP, kSitePend,
+                    ldf(f.pwx, (int64_t)h * R * P + idx, nw, kSiteProj) * sv(sX, idx % P));
+            for (int i = tid; i < R * N; i += NT)
+                stv(a.bp, bh * R * N + i, nBN, kSitePend,
+                    ldf(f.pwB, (int64_t)h * R * N + i, a.H * R * N, kSiteProj) * sv(sB, i % N));
+        } else {
+            for (int idx = tid; idx < R * P; idx += NT) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < Cfg::WARPS; ++w) sum += ypart[w * R * P + idx];
+                const float xval = sv(sX, idx);
+                stv(a.y, bh * R * P + idx, nBP, kSiteY, sum + Dh * xval);
+                stv(a.xp, bh * R * P + idx, nBP, kSitePend, xval);
+            }
+            for (int i = tid; i < R * N; i += NT) stv(a.bp, bh * R * N + i, nBN, kSitePend, sv(sB, i));
         }
-        for (int i = tid; i < R * N; i += NT) stv(a.bp, bh * R * N + i, nBN, kSitePend, sv(sB, i));
         __syncthreads();  // every read of this stage is done: refill it
         if (tid == 0 && bh + 2 * step < BH) issue(bh + 2 * step, st);
     }
@@ -613,7 +656,7 @@ cudaError_t dispatch_np(const StepArgs<IO> &a, const StepFeat &f, cudaStream_t s
     // rank 1: one CTA per slice (measured faster); rank >= 2: the persistent
     // streaming kernel (its heavier per-element work overlaps the next slice's load)
     // (BC-norm: the tiled kernel, which normalises its staged rows in place)
-    const bool tiled = R == 1 || f.wB || f.pwx;
+    const bool tiled = R == 1 || f.wB;
     if (a.N == 128 && a.P == 64)
         return tiled ? launch_tiled<128, 64, R, IO, GEN>(a, f, s) : launch_stream<128, 64, R, IO, GEN>(a, f, s);
     if (a.N == 64 && a.P == 64)

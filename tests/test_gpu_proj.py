@@ -112,6 +112,31 @@ def test_proj_decode_continues_the_prefill(shape):
     assert max_rel_l2_state(host64(fs.h), ost.h) < TOL_BF16
 
 
+def test_proj_decode_many_slices_streaming():
+    """Rank 4 with more slices than the persistent streaming decode kernel has
+    CTAs (each CTA walks several slices through its two-stage copy ring), from
+    a random rank-4 state, two steps, against the oracle's step_proj."""
+    s = Shape(96, 1, 8, 64, 128, 4, "bf16", 525)
+    pr, opr = weights(s)
+    st = m3.State(*(t.to(DEV) for t in make_state(s)))
+    ost = oracle.State(*(host64(t) for t in st))
+    pre = make_prefill_proj(s)
+    A, D = pre["A"].to(DEV), pre["D"].to(DEV)
+    steps = make_steps_proj(s, 2)
+    worst = 0.0
+    for i in range(2):
+        args = [steps[k][i].contiguous().to(DEV) for k in STEP_KEYS]
+        yi = m3.step(*args, A, D, st, proj=pr).clone()
+        m3.stream_status()
+        yo, ost = oracle.step_proj(*(host64(a) for a in args), host64(A), host64(D), opr, ost)
+        worst = max(worst, rel_slices(host64(yi), yo))
+    record_margin("proj decode 768 slices r4 (streaming)", worst, TOL_BF16)
+    assert worst < TOL_BF16, f"decode rel-L2 {worst:.3e}"
+    assert max_rel_l2_state(host64(st.h), ost.h) < TOL_BF16
+    assert max_rel_l2_state(host64(st.b_prev), ost.b_prev) < 1e-6
+    assert max_rel_l2_state(host64(st.x_prev), ost.x_prev) < 1e-6
+
+
 def test_proj_full_size_sampled():
     """The MIMO workload's shape (batch 8, 4096 tokens, 32 heads, N 64, R 4)
     with the projections; the oracle recomputes two of its sequences' first
