@@ -90,7 +90,10 @@ constexpr int64_t kMaxSegments = 64, kMinSegChunks = 8;
 constexpr long long kFlagBudget = 2000000000LL;
 constexpr double kSumCost = 0.55, kCtaCost = 2.0;
 
-template <int N, int R>
+// SEP: the MIMO projections' token rows land in staging tiles of their own
+// (N = 64, R > 1, where shared memory has room) instead of in the first rows
+// of the rank-row tiles, so that widening them needs no barrier.
+template <int N, int R, bool SEP = false>
 struct Cfg {
     static constexpr int Q = kRows / R;      // tokens per chunk
     static constexpr int K2 = N / 2;         // state pairs
@@ -125,7 +128,13 @@ struct Cfg {
     static constexpr uint32_t OFF_BAR = OFF_SCAL + ((SCAL_FLOATS * 4 + 15) / 16) * 16;
     static constexpr uint32_t NBARS = 20;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
-    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024 alignment
+    // staging (SEP): 2 stages of {B, C} token-row tiles, then kNX x token-row tiles
+    static constexpr uint32_t STG_ROWS = SEP ? (uint32_t)Q * 128u : 0u;  // one 64-column block of token rows
+    static constexpr uint32_t STG_BC = KB * STG_ROWS;
+    static constexpr uint32_t OFF_STG = ((OFF_MISC + 16 + 1023) / 1024) * 1024;
+    static constexpr uint32_t OFF_STGX = OFF_STG + 4 * STG_BC;
+    static constexpr uint32_t SMEM_BYTES =
+        (SEP ? OFF_STGX + kNX * STG_ROWS : OFF_MISC + 16) + 1024;  // + slack for 1024 alignment
     static_assert(K2 % 4 == 0 && kPro % G4 == 0, "pair groups must tile the prologue threads");
     static_assert(Q % NPART == 0 && TPT % TB == 0, "tokens must split across the angle-pass parts");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -369,7 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmT,
                   const TcArgs a) {
-    using C = Cfg<N, R>;
+    constexpr bool kSep = PROJ && N == 64 && R > 1;  // the projections' token rows in staging tiles
+    using C = Cfg<N, R, kSep>;
     constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, G4 = C::G4, NPART = C::NPART, TPT = C::TPT, TB = C::TB;
     constexpr bool SUM = MODE == kSummary, SEGD = MODE != kWhole;
     const float *const A_tok = GEN ? a.A_tok : nullptr;  // A per token-head, or none
@@ -483,12 +493,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const int t0 = (cb + i) * Q;
                 // (with the projections a tile load brings one row per token)
                 mbar_arrive_expect_tx(&bb.full_bc[s], (SUM ? C::BC_BYTES : C::BCS_BYTES) / (PROJ ? R : 1));
+                uint8_t *sb = kSep ? smem + C::OFF_STG + s * 2 * C::STG_BC : st;
+                const uint32_t blk = kSep ? C::STG_ROWS : 16384u, ctile = kSep ? C::STG_BC : C::BC_BYTES;
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_5d(st + kb * 16384, &tmB, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
+                    tma_load_5d(sb + kb * blk, &tmB, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
                     if (!SUM)
-                        tma_load_5d(st + C::BC_BYTES + kb * 16384, &tmC, &bb.full_bc[s], kb * 64, 0, (int)h, t0,
-                                    (int)b);
+                        tma_load_5d(sb + ctile + kb * blk, &tmC, &bb.full_bc[s], kb * 64, 0, (int)h, t0, (int)b);
                 }
                 issued = i + 1;
             }
@@ -505,8 +516,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (i >= kNX && !mbar_wait(&bb.empty_x[s], ((i / kNX) - 1) & 1, abort_flag, err, kErrWaitCompute))
                     break;
                 mbar_arrive_expect_tx(&bb.full_x[s], C::X_BYTES / (PROJ ? R : 1));
-                tma_load_5d(smem + C::OFF_X + s * C::X_BYTES, &tmX, &bb.full_x[s], 0, 0, (int)h, (cb + i) * Q,
-                            (int)b);
+                tma_load_5d(kSep ? smem + C::OFF_STGX + s * C::STG_ROWS : smem + C::OFF_X + s * C::X_BYTES, &tmX,
+                            &bb.full_x[s], 0, 0, (int)h, (cb + i) * Q, (int)b);
                 issued = i + 1;
             }
             if (*abort_flag) {
@@ -772,7 +783,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 // for R > 1 every thread first takes its tokens' rows into
                 // registers, since the widened rows i R + r overwrite rows of
                 // other threads' tokens
-                constexpr bool kStage = PROJ && R > 1;
+                constexpr bool kStage = PROJ && R > 1 && !kSep;
+                // where the token rows are: the staging tiles (kSep) or the tiles' first rows
+                const uint8_t *bsrc = kSep ? smem + C::OFF_STG + s * 2 * C::STG_BC : bst;
+                const uint8_t *csrc = kSep ? bsrc + C::STG_BC : cst;
+                const uint32_t kbs = kSep ? (uint32_t)(g >> 3) * C::STG_ROWS : kbo;
                 uint4 pb[kStage ? TPT : 1], pc[kStage ? TPT : 1];
                 if (kStage) {
 #pragma unroll
@@ -796,14 +811,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                             if (PROJ) {  // widen: this rank's weights times the token's row
                                 const uint4 src = kStage ? pb[j0 + jj]
                                                          : *reinterpret_cast<const uint4 *>(
-                                                               bst + kbo + sw128((uint32_t)i, jchunk));
+                                                               bsrc + kbs + sw128((uint32_t)i, jchunk));
                                 const uint4 w = *reinterpret_cast<const uint4 *>(sbias + r * K2 + 4 * g);
                                 vb[jj][r] = make_uint4(mul_bf16x2(src.x, w.x), mul_bf16x2(src.y, w.y),
                                                        mul_bf16x2(src.z, w.z), mul_bf16x2(src.w, w.w));
                                 if (!SUM) {
                                     const uint4 srcc = kStage ? pc[j0 + jj]
                                                               : *reinterpret_cast<const uint4 *>(
-                                                                    cst + kbo + sw128((uint32_t)i, jchunk));
+                                                                    csrc + kbs + sw128((uint32_t)i, jchunk));
                                     const uint4 wc = *reinterpret_cast<const uint4 *>(sbias + (R + r) * K2 + 4 * g);
                                     vc[jj][r] = make_uint4(mul_bf16x2(srcc.x, wc.x), mul_bf16x2(srcc.y, wc.y),
                                                            mul_bf16x2(srcc.z, wc.z), mul_bf16x2(srcc.w, wc.w));
@@ -893,10 +908,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const float wv = wst[row / R];
                 const uint32_t ww = pack_bf16(wv, wv);
                 uint4 v[4];
-                if (PROJ) {  // the x tile holds one row per token: widen it into rows i R + r
+                if (PROJ) {  // one row per token (staging tile, or the x tile's first rows): widen into rows i R + r
+                    const uint8_t *xsrc = kSep ? smem + C::OFF_STGX + sx * C::STG_ROWS : xst;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4 *>(xst + sw128(row / R, j0 + j));
-                    if (R > 1) named_bar(kBarPro, kPro);  // every token's row read before any is overwritten
+                    for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4 *>(xsrc + sw128(row / R, j0 + j));
+                    if (R > 1 && !kSep) named_bar(kBarPro, kPro);  // every token's row read before any is overwritten
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(sxw + (row % R) * (kP / 2) + 4 * (j0 + j));
@@ -1339,7 +1355,7 @@ bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int
 template <int N, int R, int MODE, bool GEN, bool BCN, bool PROJ>
 cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc, const CUtensorMap &mt,
                         const TcArgs &a, int64_t ctas, cudaStream_t stream, bool dependent = false) {
-    using C = Cfg<N, R>;
+    using C = Cfg<N, R, (PROJ && N == 64 && R > 1)>;
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, GEN, BCN, PROJ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
