@@ -140,3 +140,19 @@ def test_split_calls_on_two_streams_at_once():
         m3.stream_status()
         assert torch.equal(ya, ya_ref) and torch.equal(fa.h, fa_ref.h)
         assert torch.equal(yb, yb_ref) and torch.equal(fb.h, fb_ref.h)
+
+
+@pytest.mark.parametrize("shape,segs", [
+    (Shape(1, 256 * 128, 1, 64, 128, 1, "bf16", 171), 256),   # one chunk per segment: 255 summaries scanned by the last
+    (Shape(1, 4096, 2, 64, 64, 4, "bf16", 172), 128),          # rank 4, 32-token chunks
+], ids=["n128r1s256", "n64r4s128"])
+def test_split_deep_lookback(shape, segs):
+    """Many one-chunk segments: the main pass of the last segment combines
+    every earlier segment's summary, and the summary grid runs in more than
+    one wave before the main grid has taken every SM."""
+    dims = m3.make_dims(shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.rank,
+                        shape.torch_io)
+    plan = m3.scan_plan(dims, m3.ALGO_TC_SEGMENTS(segs))
+    assert plan.segments == segs and plan.launches == 2
+    check_scan(shape, m3.ALGO_TC_SEGMENTS(segs), with_init=True)
+    m3.stream_status()
