@@ -220,9 +220,12 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 
 // BC-norm row scale 1 / sqrt(mean_n v^2 + eps) of row `row` of a 128B-swizzled
 // K-major tile of KB 64-column blocks (one thread per row).
+// The squares are formed by the mixed-precision multiply-add (bf16 operands,
+// fp32 addend and result: the bf16 product is exact in fp32), two running
+// sums for the two halves of each bf16 pair.
 template <int KB>
 __device__ __forceinline__ float bc_row_scale(const uint8_t *tile, uint32_t row, float inv_n, float eps) {
-    float ss = 0.f;
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
@@ -231,12 +234,13 @@ __device__ __forceinline__ float bc_row_scale(const uint8_t *tile, uint32_t row,
             const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 f = unpack_bf16(u[e]);
-                ss = fmaf(f.x, f.x, ss);
-                ss = fmaf(f.y, f.y, ss);
+                unsigned short lo, hi;
+                asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(u[e]));
+                asm("fma.rn.f32.bf16 %0, %1, %1, %0;" : "+f"(s0) : "h"(lo));
+                asm("fma.rn.f32.bf16 %0, %1, %1, %0;" : "+f"(s1) : "h"(hi));
             }
         }
-    return rsqrtf(fmaf(ss, inv_n, eps));
+    return rsqrtf(fmaf(s0 + s1, inv_n, eps));
 }
 
 // The BC-norm affine map of this thread's 4 pairs of one row: b * sc * w + bias
