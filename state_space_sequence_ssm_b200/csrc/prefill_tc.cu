@@ -370,14 +370,16 @@ enum : unsigned {
     kSiteProj = 0x10b,     // MIMO projection weights
 };
 
-// GEN = false: the plain method (A per head, theta per token), compiled
-// without the optional features' branches; GEN = true reads A_tok and th_head
-// from the arguments.  BCN: the BC-norm prologue (only with GEN).  PROJ: the
+// FEAT: which optional input layouts the instantiation reads from the
+// arguments -- bit 0: A per token-head (A_tok), bit 1: theta fixed per head
+// (th_head); 0 is the plain method, compiled without those branches, and
+// each layout alone has an instantiation of its own.  BCN: the BC-norm
+// prologue (with FEAT = 3).  PROJ: the
 // MIMO projections (not with BCN): the tile loads bring one
 // row per token, the prologue widens B, C and x to the R rows of each token
 // in shared memory, and the epilogue sums each token's R output rows with
 // the y weights into one row.
-template <int N, int R, int MODE, bool GEN, bool BCN, bool PROJ = false>
+template <int N, int R, int MODE, int FEAT, bool BCN, bool PROJ = false>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmT,
@@ -386,8 +388,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     using C = Cfg<N, R, kSep>;
     constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, G4 = C::G4, NPART = C::NPART, TPT = C::TPT, TB = C::TB;
     constexpr bool SUM = MODE == kSummary, SEGD = MODE != kWhole;
-    const float *const A_tok = GEN ? a.A_tok : nullptr;  // A per token-head, or none
-    const bool th_head = GEN && a.th_head;               // theta fixed per head
+    constexpr bool GEN = FEAT != 0;                               // some optional layout compiled in
+    const float *const A_tok = (FEAT & 1) ? a.A_tok : nullptr;  // A per token-head, or none
+    const bool th_head = (FEAT & 2) && a.th_head;               // theta fixed per head
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *scal = reinterpret_cast<float *>(smem + C::OFF_SCAL);
@@ -1356,11 +1359,11 @@ bool make_theta_map(CUtensorMap *m, const void *base, int64_t K2, int64_t H, int
 
 // `dependent`: launched as a programmatic dependent of the previous kernel on
 // the stream (the main pass of a split sequence after its summary pass).
-template <int N, int R, int MODE, bool GEN, bool BCN, bool PROJ>
+template <int N, int R, int MODE, int FEAT, bool BCN, bool PROJ>
 cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc, const CUtensorMap &mt,
                         const TcArgs &a, int64_t ctas, cudaStream_t stream, bool dependent = false) {
     using C = Cfg<N, R, (PROJ && N == 64 && R > 1)>;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, GEN, BCN, PROJ>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<N, R, MODE, FEAT, BCN, PROJ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
@@ -1373,12 +1376,12 @@ cudaError_t launch_pass(const CUtensorMap &mx, const CUtensorMap &mb, const CUte
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = dependent ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<N, R, MODE, GEN, BCN, PROJ>, mx, mb, mc, mt, a);
+    e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<N, R, MODE, FEAT, BCN, PROJ>, mx, mb, mc, mt, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-template <int N, int R, bool GEN, bool BCN, bool PROJ = false>
+template <int N, int R, int FEAT, bool BCN, bool PROJ = false>
 cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     using C = Cfg<N, R>;
     CUtensorMap mx, mb, mc, mt;
@@ -1425,7 +1428,7 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
         a.hT = p.hT;
         a.bpT = p.bpT;
         a.xpT = p.xpT;
-        return launch_pass<N, R, kWhole, GEN, BCN, PROJ>(mx, mb, mc, mt, a, BH, p.stream);
+        return launch_pass<N, R, kWhole, FEAT, BCN, PROJ>(mx, mb, mc, mt, a, BH, p.stream);
     }
     // split sequences: the summary pass over segments 0 .. nseg-2 publishes
     // each segment's local end state and transition; the main pass over all
@@ -1439,14 +1442,14 @@ cudaError_t launch_nr(const Problem &p, const TcPlan &plan, const char **why) {
     // (the failure-path self-test leaves the summary pass out: its flags are
     // never published and the look-back waits give up)
     if (!p.skip_summary) {
-        e = launch_pass<N, R, kSummary, GEN, BCN, PROJ>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
+        e = launch_pass<N, R, kSummary, FEAT, BCN, PROJ>(mx, mb, mc, mt, a, BH * (plan.nseg - 1), p.stream);
         if (e != cudaSuccess) return e;
     }
     a.y = (__nv_bfloat16 *)p.y;
     a.hT = p.hT;
     a.bpT = p.bpT;
     a.xpT = p.xpT;
-    return launch_pass<N, R, kSegment, GEN, BCN, PROJ>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream,
+    return launch_pass<N, R, kSegment, FEAT, BCN, PROJ>(mx, mb, mc, mt, a, BH * plan.nseg, p.stream,
                                                        !p.skip_summary);
 }
 
@@ -1539,58 +1542,37 @@ TcPlan prefill_tc_plan(const Problem &p) {
 
 size_t prefill_tc_workspace(const Problem &p) { return prefill_tc_plan(p).ws_bytes; }
 
+template <int FEAT, bool BCN, bool PROJ>
+cudaError_t dispatch_nr(const Problem &p, const TcPlan &plan, const char **why) {
+    if (p.N == 128) {
+        if (p.R == 1) return launch_nr<128, 1, FEAT, BCN, PROJ>(p, plan, why);
+        if (p.R == 2) return launch_nr<128, 2, FEAT, BCN, PROJ>(p, plan, why);
+        return launch_nr<128, 4, FEAT, BCN, PROJ>(p, plan, why);
+    }
+    if (p.R == 1) return launch_nr<64, 1, FEAT, BCN, PROJ>(p, plan, why);
+    if (p.R == 2) return launch_nr<64, 2, FEAT, BCN, PROJ>(p, plan, why);
+    return launch_nr<64, 4, FEAT, BCN, PROJ>(p, plan, why);
+}
+
 cudaError_t launch_prefill_tc(const Problem &p, const char **why) {
     const TcPlan plan = prefill_tc_plan(p);
     if (plan.nseg > 1 && (!p.ws || p.ws_bytes < plan.ws_bytes)) {
         *why = "tensor-core prefill: workspace too small for the split sequence";
         return cudaErrorNotSupported;
     }
-    // plain instantiations unless an optional feature is on
-    const bool gen = p.a_tok || p.th_head || p.wB || p.pwx;
+    // the instantiation for (N, R) with feature mask FEAT (bit 0 A per token,
+    // bit 1 theta per head), BC-norm and the MIMO projections
+    const int feat = (p.a_tok ? 1 : 0) | (p.th_head ? 2 : 0);
     if (p.pwx) {  // MIMO projections (never with the BC-norm prologue); plain unless A_t or theta per head
-        const bool g2 = p.a_tok || p.th_head;
-        if (p.N == 128) {
-            if (p.R == 1) return g2 ? launch_nr<128, 1, true, false, true>(p, plan, why)
-                                    : launch_nr<128, 1, false, false, true>(p, plan, why);
-            if (p.R == 2) return g2 ? launch_nr<128, 2, true, false, true>(p, plan, why)
-                                    : launch_nr<128, 2, false, false, true>(p, plan, why);
-            return g2 ? launch_nr<128, 4, true, false, true>(p, plan, why)
-                      : launch_nr<128, 4, false, false, true>(p, plan, why);
-        }
-        if (p.R == 1) return g2 ? launch_nr<64, 1, true, false, true>(p, plan, why)
-                                : launch_nr<64, 1, false, false, true>(p, plan, why);
-        if (p.R == 2) return g2 ? launch_nr<64, 2, true, false, true>(p, plan, why)
-                                : launch_nr<64, 2, false, false, true>(p, plan, why);
-        return g2 ? launch_nr<64, 4, true, false, true>(p, plan, why) : launch_nr<64, 4, false, false, true>(p, plan, why);
+        return feat ? dispatch_nr<3, false, true>(p, plan, why) : dispatch_nr<0, false, true>(p, plan, why);
     }
-    if (p.wB) {
-        if (p.N == 128) {
-            if (p.R == 1) return launch_nr<128, 1, true, true>(p, plan, why);
-            if (p.R == 2) return launch_nr<128, 2, true, true>(p, plan, why);
-            return launch_nr<128, 4, true, true>(p, plan, why);
-        }
-        if (p.R == 1) return launch_nr<64, 1, true, true>(p, plan, why);
-        if (p.R == 2) return launch_nr<64, 2, true, true>(p, plan, why);
-        return launch_nr<64, 4, true, true>(p, plan, why);
+    if (p.wB) return dispatch_nr<3, true, false>(p, plan, why);
+    switch (feat) {
+        case 1: return dispatch_nr<1, false, false>(p, plan, why);
+        case 2: return dispatch_nr<2, false, false>(p, plan, why);
+        case 3: return dispatch_nr<3, false, false>(p, plan, why);
+        default: return dispatch_nr<0, false, false>(p, plan, why);
     }
-    if (gen) {
-        if (p.N == 128) {
-            if (p.R == 1) return launch_nr<128, 1, true, false>(p, plan, why);
-            if (p.R == 2) return launch_nr<128, 2, true, false>(p, plan, why);
-            return launch_nr<128, 4, true, false>(p, plan, why);
-        }
-        if (p.R == 1) return launch_nr<64, 1, true, false>(p, plan, why);
-        if (p.R == 2) return launch_nr<64, 2, true, false>(p, plan, why);
-        return launch_nr<64, 4, true, false>(p, plan, why);
-    }
-    if (p.N == 128) {
-        if (p.R == 1) return launch_nr<128, 1, false, false>(p, plan, why);
-        if (p.R == 2) return launch_nr<128, 2, false, false>(p, plan, why);
-        return launch_nr<128, 4, false, false>(p, plan, why);
-    }
-    if (p.R == 1) return launch_nr<64, 1, false, false>(p, plan, why);
-    if (p.R == 2) return launch_nr<64, 2, false, false>(p, plan, why);
-    return launch_nr<64, 4, false, false>(p, plan, why);
 }
 
 // Failure-path self-test: one thread waits, with a bounded wait, on an
