@@ -1070,10 +1070,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             //      half 1 blocks 1 and 2 (balances the lower triangle).  The plain
             //      kernel takes it before the carried-state update, so that Yd runs
             //      under the update; for N = 64 it starts as soon as S is done (G
-            //      and Yo finish meanwhile; for N = 128 that measured slower).  The
-            //      optional features' instantiations measured 2 % slower with the
+            //      and Yo finish meanwhile; for N = 128 that measured slower).  So
+            //      does the per-head-theta instantiation (2 % faster that way); the
+            //      per-token-A, general and BC-norm ones measured slower with the
             //      mask first (register allocation) and take it after the update.
-            constexpr bool kMaskFirst = !GEN && !BCN && !SUM;
+            constexpr bool kMaskFirst = (FEAT == 0 || FEAT == 2) && !BCN && !SUM;
             constexpr bool kMaskOnS = kMaskFirst && N == 64;
             // scalars of chunk c (release/acquire through sc), its x tile, and
             // S(c) (mask on S alone) or S, G and Yo of chunk c
