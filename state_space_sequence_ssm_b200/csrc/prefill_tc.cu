@@ -185,6 +185,9 @@ __device__ __forceinline__ bool bar_any(bool pred) {
         : "memory");
     return r != 0;
 }
+// The same over one warp (no barrier between warps): a role whose warps signal
+// the MMA issuer one arrival each lets its warps drift apart within a chunk.
+__device__ __forceinline__ bool warp_any(bool pred) { return __any_sync(0xffffffffu, pred) != 0; }
 
 // bf16 copy of 32 fp32 values (columns 32*half ..) of state row n into the
 // 128B-swizzled MN-major operand tile (row n = K index of the readout MMA).
@@ -389,6 +392,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     constexpr int Q = C::Q, K2 = C::K2, KB = C::KB, G4 = C::G4, NPART = C::NPART, TPT = C::TPT, TB = C::TB;
     constexpr bool SUM = MODE == kSummary, SEGD = MODE != kWhole;
     constexpr bool GEN = FEAT != 0;                               // some optional layout compiled in
+    // The state warps signal the MMA issuer one arrival per warp (and agree on
+    // a failed wait within the warp), instead of a barrier of all 256 threads
+    // and one arrival, where that measured faster: the split passes.
+    constexpr bool kWarpSig = SEGD;
+    constexpr uint32_t kStArrivals = kWarpSig ? kSt / 32 : 1;
     const float *const A_tok = (FEAT & 1) ? a.A_tok : nullptr;  // A per token-head, or none
     const bool th_head = (FEAT & 2) && a.th_head;               // theta fixed per head
     extern __shared__ uint8_t smem_raw[];
@@ -442,13 +450,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         for (int i = 0; i < kNX; ++i) {
             mbar_init(&bb.full_x[i], 1);
-            mbar_init(&bb.empty_x[i], 1);
+            mbar_init(&bb.empty_x[i], kStArrivals);
             mbar_init(&bb.sc[i], 1);  // per-chunk scalars published to the state warpgroup
         }
         mbar_init(bb.ops, 1);
         mbar_init(bb.sg, 1);
-        mbar_init(bb.hrdy, 1);
-        mbar_init(bb.p, 1);
+        mbar_init(bb.hrdy, kStArrivals);
+        mbar_init(bb.p, kStArrivals);
         mbar_init(bb.yd, 1);
         mbar_init(bb.drain, 1);
         mbar_init(bb.sd, 1);
@@ -962,6 +970,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const uint32_t tl = tbase + ((uint32_t)(32 * wq) << 16);
         const int c0 = 32 * hf;            // first column of this thread's half
         float hreg[32];
+        // a failed wait anywhere in the role (or the warp); the role's (or the
+        // warp's) signal to the MMA issuer once all its threads are done
+        auto role_any = [&](bool pred) { return kWarpSig ? warp_any(pred) : bar_any<kBarState, kSt>(pred); };
+        auto role_done = [&]() {
+            if (kWarpSig) {
+                __syncwarp();
+                return lane == 0;
+            }
+            named_bar(kBarState, kSt);
+            return lt == 0;
+        };
         // Pending-inclusive state entering the segment.  The whole sequence and
         // segment 0 of either pass: the caller's h0 + beta'_0 b_prev x_prev^T
         // (pending write of token -1); later summary segments: zero (their
@@ -1051,8 +1070,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         float m_l2 = 0.f, m_cs = 1.f, m_sn = 0.f;
         fence_proxy_async_smem();
         named_bar(kBarState, kSt);
+        if (kWarpSig ? lane == 0 : lt == 0) mbar_arrive(bb.hrdy);
         if (lt == 0) {
-            mbar_arrive(bb.hrdy);
             // the caller's initial state is read (the last segment may now overwrite it)
             if (MODE == kSegment && seg == 0 && dchk::in(kSiteFlags, (int64_t)(a.nseg - 1) * BH + bh, 1, nSeg * BH))
                 flag_release(a.flags + (int64_t)(a.nseg - 1) * BH + bh, 1u);
@@ -1078,10 +1097,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             constexpr bool kMaskOnS = kMaskFirst && N == 64;
             // scalars of chunk c (release/acquire through sc), its x tile, and
             // S(c) (mask on S alone) or S, G and Yo of chunk c
-            if (bar_any<kBarState, kSt>(!mbar_wait(&bb.sc[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
-                                        !mbar_wait(&bb.full_x[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitTma) ||
-                                        !mbar_wait(kMaskOnS ? bb.sd : bb.sg, lc & 1, abort_flag, err,
-                                                   kErrWaitMma))) {
+            if (role_any(!mbar_wait(&bb.sc[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitCompute) ||
+                         !mbar_wait(&bb.full_x[sx], (lc / kNX) & 1, abort_flag, err, kErrWaitTma) ||
+                         !mbar_wait(kMaskOnS ? bb.sd : bb.sg, lc & 1, abort_flag, err, kErrWaitMma))) {
                 ok = false;
                 break;
             }
@@ -1089,12 +1107,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             auto decay_mask = [&]() {
                 mask_to_tmem<R, Q>(hf == 0 ? 0 : 1, hf == 0 ? 3 : 2, wq, lq, tl, cAl2, gam, ghat, colf);
                 tc_fence_before();
-                named_bar(kBarState, kSt);
-                if (lt == 0) mbar_arrive(bb.p);
+                if (role_done()) mbar_arrive(bb.p);
             };
             if (kMaskFirst) decay_mask();
             if (kMaskOnS) {  // G(c) and Yo(c), for the update below and the epilogue
-                if (bar_any<kBarState, kSt>(!mbar_wait(bb.sg, lc & 1, abort_flag, err, kErrWaitMma))) {
+                if (role_any(!mbar_wait(bb.sg, lc & 1, abort_flag, err, kErrWaitMma))) {
                     ok = false;
                     break;
                 }
@@ -1126,8 +1143,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(kBarState, kSt);
-            if (lt == 0) {
+            if (role_done()) {
                 mbar_arrive(bb.hrdy);
                 if (SUM) mbar_arrive(&bb.empty_x[sx]);  // x tile and scalars consumed
             }
@@ -1135,7 +1151,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (!kMaskFirst) decay_mask();
 
             // ---- F. epilogue: y = Yd + exp(cA_t) Yo + D x, this thread's 32 columns
-            if (bar_any<kBarState, kSt>(!mbar_wait(bb.yd, lc & 1, abort_flag, err, kErrWaitMma))) {
+            if (role_any(!mbar_wait(bb.yd, lc & 1, abort_flag, err, kErrWaitMma))) {
                 ok = false;
                 break;
             }
@@ -1227,9 +1243,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
             }
             tc_fence_before();
-            named_bar(kBarState, kSt);
-            if (lt == 0) mbar_arrive(&bb.empty_x[sx]);
+            if (role_done()) mbar_arrive(&bb.empty_x[sx]);
         }
+        // a warp that gave up left the loop on its own: agree before the barriers below
+        if (kWarpSig) ok = !bar_any<kBarState, kSt>(!ok);
         if (SUM) {
             // ---- summary: the segment's local end state (pending-inclusive) into
             //      slot seg + 1, its transition exp(cA) Rot(-Phi) per pair
