@@ -394,8 +394,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     constexpr bool GEN = FEAT != 0;                               // some optional layout compiled in
     // The state warps signal the MMA issuer one arrival per warp (and agree on
     // a failed wait within the warp), instead of a barrier of all 256 threads
-    // and one arrival, where that measured faster: the split passes.
-    constexpr bool kWarpSig = SEGD;
+    // and one arrival, where that measured faster: the split passes and the
+    // per-head-theta instantiation (the plain, per-token-A, BC-norm and
+    // projection ones measured the same or slower that way).
+    constexpr bool kWarpSig = SEGD || FEAT == 2;
     constexpr uint32_t kStArrivals = kWarpSig ? kSt / 32 : 1;
     const float *const A_tok = (FEAT & 1) ? a.A_tok : nullptr;  // A per token-head, or none
     const bool th_head = (FEAT & 2) && a.th_head;               // theta fixed per head
