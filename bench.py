@@ -65,9 +65,11 @@ def parse():
                     help="skip the variant lines (per-token A, per-head theta, BC-norm) of the prefill workload")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads' lines (small fp32 scan, MIMO, decode, long context)")
-    ap.add_argument("--case", choices=["prefill", "prefill_proj", "decode"], default=None,
+    ap.add_argument("--case", choices=["prefill", "prefill_proj", "prefill_a_per_token", "prefill_theta_per_head",
+                                       "prefill_bcnorm", "decode"], default=None,
                     help="profiling case: only run --case-launches launches of one kernel at --case-batch "
-                         "(for ncu captures; prints no bench line)")
+                         "(for ncu captures; prints no bench line); prefill_<variant> runs the workload "
+                         "with that variant's layout or prologue")
     ap.add_argument("--case-batch", type=int, default=None, help="batch of the profiling case")
     ap.add_argument("--case-seqlen", type=int, default=None, help="sequence length of the profiling case")
     ap.add_argument("--case-launches", type=int, default=3, help="launches of the profiling case")
@@ -86,19 +88,26 @@ def run_case(args):
     from m3_inputs import WORKLOADS, make_prefill, make_state, make_steps
 
     keys = ("x", "B", "C", "dt", "lam", "theta", "A", "D")
-    if args.case in ("prefill", "prefill_proj"):
+    if args.case.startswith("prefill"):
         s = WORKLOADS[args.workload]
         s = s.with_(batch=args.case_batch or s.batch, seqlen=args.case_seqlen or s.seqlen)
-        proj = None
-        if args.case == "prefill_proj":  # the same shape with the fused MIMO projections
+        kind = args.case[len("prefill_"):]
+        proj = bcn = None
+        if kind == "proj":  # the same shape with the fused MIMO projections
             from m3_inputs import make_prefill_proj, make_proj
             inp = make_prefill_proj(s, device="cuda")
             w = make_proj(s, device="cuda")
             proj = m3.MimoProj(w["wx"], w["wB"], w["wC"], w["wy"])
+        elif kind in ("a_per_token", "theta_per_head"):
+            inp = make_prefill(s, device="cuda", **{kind: True})
         else:
             inp = make_prefill(s, device="cuda")
+        if kind == "bcnorm":
+            from m3_inputs import make_bcnorm
+            p = make_bcnorm(s, device="cuda")
+            bcn = m3.BCNorm(p["wB"], p["wC"], p["bB"], p["bC"], p["eps"])
         for _ in range(args.case_launches):
-            m3.scan_fwd(*(inp[k] for k in keys), None, proj=proj)
+            m3.scan_fwd(*(inp[k] for k in keys), None, proj=proj, bcnorm=bcn)
     else:
         # a decode workload, or the long-context workload's own sequences
         name = args.workload if args.workload.startswith(("decode", "long")) else DECODE_WORKLOADS[0]
@@ -688,11 +697,7 @@ def run_variant(m3, kind, args, dev, rank, world, barrier, max_over_ranks, hbm_p
     with theta fixed per head ([H, N/2]), timed like the headline (CUDA events
     on the launching stream, K launches)."""
     import torch
-    from m3_inputs import WORKLOADS, make_prefill
-
-    from m3_inputs import make_bcnorm
-
-    from m3_inputs import make_prefill_proj, make_proj
+    from m3_inputs import make_bcnorm, make_prefill, make_prefill_proj, make_proj
 
     workload = MIMO_WORKLOAD if kind == "mimo_proj" else args.workload
     s = replica_shape(workload, rank)
